@@ -1,0 +1,478 @@
+"""Plain, slow, fp64 CPU oracle for one denoising step of block-wise discrete diffusion.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference arm of ``bench.py`` may import or run this module.
+It shares no code with the CUDA library and imports nothing from it; the only
+thing both sides take from a common place is the seeded synthetic inputs
+(``synth``), which carry none of the method's arithmetic.
+
+What it computes (the method as the pages describe it):
+
+* "DiffusionGemma Technical Report" (metalmedia.ai), Figure 4: a prompt is
+  encoded causally into a KV cache; a canvas is refined by a decoder with
+  bidirectional attention across the canvas and cross-attention to the cache;
+  the finished canvas goes back through the causal encoder and is appended.
+* Same page, explanatory visual, "Inference: block-wise diffusion decoding",
+  and "What they did": an entropy-bounded sampler with adaptive stopping
+  finishes a 256-token block in a number of steps.
+* Model card "diffusiongemma" (axforge.ai), "Mixture-of-Experts (MoE)
+  Efficiency": 8 active experts of 128; Table 1 of the report: vocabulary 262k.
+* The entropy-bounded (EB) rule itself is not printed on the pages; the oracle
+  follows the published EB sampler (Ben-Hamu et al., 2025, "Accelerated
+  Sampling from Masked Diffusion Models via Entropy Bounded Unmasking"):
+  commit masked positions in ascending entropy while the sum of the chosen
+  entropies minus their maximum stays within the bound gamma.
+
+Precision: every product and sum runs in fp64.  Where the workload stores an
+activation in bf16, the oracle rounds the fp64 value to the nearest bf16 at the
+same tensor (x, q, k, v, o, h, y, a, Y, the final normalised rows), so the
+oracle/GPU gap is accumulation-order error, not storage error.  fp32 workloads
+are not rounded at all.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional
+
+import numpy as np
+
+INT64_MAX = np.iinfo(np.int64).max
+EB_FRAC_BITS = 32  # fixed-point fraction bits of the EB entropy sums
+
+
+# --------------------------------------------------------------------------- number formats
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> value: the top half of an IEEE binary32."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), returned as fp64.
+
+    bf16 keeps 8 significant bits and binary32's exponent range: a normal value
+    m * 2**e with m in [0.5, 1) becomes rint(m * 2**8) * 2**(e - 8); values
+    below the smallest normal share the subnormal quantum 2**-133; values that
+    round past the largest finite bf16 become +-inf.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    e = np.maximum(e, -125)                     # subnormal range: fixed quantum 2**-133
+    q = np.ldexp(1.0, (e - 8))
+    r = np.rint(x / q) * q
+    bf16_max = (2.0 - 2.0 ** -7) * 2.0 ** 127
+    r = np.where(np.abs(r) > bf16_max, np.copysign(np.inf, x), r)
+    return np.where(np.isfinite(x), r, x)
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Decode OCP FP8 E4M3 codes: 1 sign, 4 exponent (bias 7), 3 mantissa bits.
+
+    Exponent field 0 is subnormal (m/8 * 2**-6); S.1111.111 is NaN; there is no
+    infinity, so the largest finite magnitude is 1.75 * 2**8 = 448.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    ex = (c >> 3) & 0xF
+    man = c & 0x7
+    val = np.where(ex == 0, man / 8.0 * 2.0 ** -6, (1.0 + man / 8.0) * np.exp2(ex - 7.0))
+    val = np.where((ex == 0xF) & (man == 0x7), np.nan, val)
+    return sign * val
+
+
+def decode_weight(arr: np.ndarray, kind: str, scale: Optional[np.ndarray] = None) -> np.ndarray:
+    """Stored weight -> fp64 value.  e4m3 rows are multiplied by their channel scale."""
+    if kind == "f32":
+        return np.asarray(arr, dtype=np.float64)
+    if kind == "bf16":
+        return bf16_bits_to_f64(arr)
+    if kind == "e4m3":
+        return e4m3_to_f64(arr) * np.asarray(scale, dtype=np.float64)[..., None]
+    raise ValueError(kind)
+
+
+def decode_act(arr: np.ndarray, kind: str) -> np.ndarray:
+    return bf16_bits_to_f64(arr) if kind == "bf16" else np.asarray(arr, dtype=np.float64)
+
+
+def storage_round(x: np.ndarray, act: str) -> np.ndarray:
+    return round_bf16(x) if act == "bf16" else np.asarray(x, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------- layer pieces
+
+def rmsnorm(x: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) over the last axis, unit gain."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+
+
+def gelu_tanh(x: np.ndarray) -> np.ndarray:
+    """0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half rotary embedding on the last axis.
+
+    Pairs (i, i + hd/2) rotate by angle pos * theta**(-2i/hd).  ``x`` is
+    [T, ..., hd] and ``pos`` is [T] (absolute positions).
+    """
+    hd = x.shape[-1]
+    half = hd // 2
+    inv = theta ** (-2.0 * np.arange(half, dtype=np.float64) / hd)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]
+    shape = (x.shape[0],) + (1,) * (x.ndim - 2) + (half,)
+    c = np.cos(ang).reshape(shape)
+    s = np.sin(ang).reshape(shape)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def attention(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+              k_new: np.ndarray, v_new: np.ndarray, causal: bool) -> np.ndarray:
+    """softmax(q K^T / sqrt(hd)) V for one canvas, GQA.
+
+    q [T, Hq, hd]; k_cache, v_cache [Hkv, P, hd] (the prompt/context rows);
+    k_new, v_new [T, Hkv, hd] (the canvas's own keys).  Query head h uses kv
+    head h // (Hq / Hkv).  Keys are the cache rows followed by the canvas rows.
+    ``causal`` False: every query sees every key (the decoder's bidirectional
+    canvas attention).  True: query i sees the whole cache and canvas keys
+    j <= i (the causal encoder used for the append).
+    Returns o [T, Hq, hd].
+    """
+    T, Hq, hd = q.shape
+    Hkv, P = k_cache.shape[0], k_cache.shape[1]
+    rep = Hq // Hkv
+    out = np.empty((T, Hq, hd))
+    mask = None
+    if causal:
+        mask = np.zeros((T, P + T), dtype=bool)
+        mask[:, P:] = np.triu(np.ones((T, T), dtype=bool), k=1)
+    for h in range(Hq):
+        g = h // rep
+        K = np.concatenate([k_cache[g], k_new[:, g]], axis=0)
+        V = np.concatenate([v_cache[g], v_new[:, g]], axis=0)
+        s = q[:, h] @ K.T / math.sqrt(hd)
+        if mask is not None:
+            s = np.where(mask, -np.inf, s)
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=1, keepdims=True)
+        out[:, h] = p @ V
+    return out
+
+
+def router_topk(y: np.ndarray, w_r: np.ndarray, top_k: int):
+    """Router: logits z = y W_r^T, p = softmax(z) over all experts, the top_k
+    largest p (lower expert index first among equals), renormalised to sum 1.
+
+    Returns (idx [T, k] int32, gates [T, k], z [T, E]).
+    """
+    z = y @ w_r.T
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    idx = np.argsort(-p, axis=1, kind="stable")[:, :top_k]
+    gp = np.take_along_axis(p, idx, axis=1)
+    return idx.astype(np.int32), gp / gp.sum(axis=1, keepdims=True), z
+
+
+def router_margin(z: np.ndarray, top_k: int) -> np.ndarray:
+    """Per token: gap between the k-th and (k+1)-th largest router logit (inf if k = E)."""
+    E = z.shape[1]
+    if top_k >= E:
+        return np.full(z.shape[0], np.inf)
+    s = -np.sort(-z, axis=1)
+    return s[:, top_k - 1] - s[:, top_k]
+
+
+def moe_ffn(y: np.ndarray, idx: np.ndarray, gates: np.ndarray, expert_w, residual: np.ndarray,
+            act: str) -> np.ndarray:
+    """Sparse expert FFN plus residual.
+
+    For token t and slot j with expert e = idx[t, j]:
+      [g; u] = y_t W_gu,e^T  (the first d_ff outputs are the gate, the next d_ff the up)
+      a      = gelu_tanh(g) * u                 (stored: rounded)
+      Y      = a W_d,e^T                        (stored: rounded)
+    out_t = residual_t + sum_j gates[t, j] Y_{t,j}          (stored: rounded)
+    ``expert_w(e)`` returns (W_gu,e [2F, d], W_d,e [d, F]) as fp64.
+    """
+    T, k = idx.shape
+    acc = np.array(residual, dtype=np.float64, copy=True)
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        w_gu, w_d = expert_w(int(e))
+        F = w_d.shape[1]
+        u = y[rows] @ w_gu.T
+        a = storage_round(gelu_tanh(u[:, :F]) * u[:, F:], act)
+        Y = storage_round(a @ w_d.T, act)
+        acc[rows] += gates[rows, slots][:, None] * Y
+    return storage_round(acc, act)
+
+
+def entropy_argmax(z: np.ndarray):
+    """Per row of logits z [R, V]: softmax entropy (natural log), greedy argmax
+    (lowest index among equal maxima) and the top-1 minus top-2 margin."""
+    z = np.asarray(z, dtype=np.float64)
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    p = e / e.sum(axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        plogp = np.where(p > 0, p * np.log(p), 0.0)
+    H = -plogp.sum(axis=1)
+    am = np.argmax(z, axis=1).astype(np.int32)
+    if z.shape[1] > 1:
+        part = -np.partition(-z, 1, axis=1)
+        margin = part[:, 0] - part[:, 1]
+    else:
+        margin = np.full(z.shape[0], np.inf)
+    return H, am, margin
+
+
+# --------------------------------------------------------------------------- EB sampler
+
+def eb_quantize(h: float) -> int:
+    """Fixed-point entropy: nearest integer to h * 2**32 (ties to even).
+
+    The argument is an fp32 value; its product with 2**32 is exact in fp64.
+    """
+    return int(np.rint(np.float64(h) * 2.0 ** EB_FRAC_BITS))
+
+
+def eb_quantize_bound(gamma: float) -> int:
+    """Fixed-point bound: floor(gamma * 2**32); +inf maps to the largest int64."""
+    if math.isinf(gamma):
+        return int(INT64_MAX)
+    v = math.floor(gamma * 2.0 ** EB_FRAC_BITS)
+    return int(min(v, INT64_MAX))
+
+
+def eb_select(H: np.ndarray, masked: np.ndarray, gamma: float, force_all: bool) -> np.ndarray:
+    """Positions of one canvas that the EB sampler commits this step.
+
+    Candidates are the masked positions.  They are ordered by entropy, ascending,
+    lower position first among equal entropies (negative rounding residue and
+    -0 count as 0).  With sorted entropies H_(1) <= H_(2) <= ..., the sampler
+    commits the first k, for the largest k >= 1 such that
+        sum_{i<=k} H_(i) - max_{i<=k} H_(i) = sum_{i<k} H_(i) <= gamma,
+    the sums taken in 32-fraction-bit fixed point.  ``force_all`` (the last
+    allowed step) commits every masked position.  Returns a bool array.
+    """
+    H = np.asarray(H, dtype=np.float32)
+    cand = np.nonzero(np.asarray(masked) != 0)[0]
+    sel = np.zeros(len(masked), dtype=bool)
+    if len(cand) == 0:
+        return sel
+    if not np.all(np.isfinite(H[cand])):
+        raise FloatingPointError("non-finite entropy at a masked position")
+    if not (gamma >= 0.0):
+        raise ValueError("the entropy bound must be >= 0")
+    hv = np.maximum(H[cand].astype(np.float64), 0.0)
+    order = sorted(range(len(cand)), key=lambda i: (hv[i], int(cand[i])))
+    if force_all:
+        sel[cand] = True
+        return sel
+    qg = eb_quantize_bound(gamma)
+    k = 1
+    prefix = 0
+    for j in range(1, len(order)):
+        prefix += eb_quantize(np.float32(hv[order[j - 1]]))
+        if prefix <= qg:
+            k = j + 1
+        else:
+            break
+    sel[cand[[order[i] for i in range(k)]]] = True
+    return sel
+
+
+# --------------------------------------------------------------------------- the model
+
+class OracleModel:
+    """Decoded view of a synthetic model (the numpy arrays from ``synth.to_numpy``).
+
+    Weights are decoded to fp64 on use so that large workloads fit in host RAM.
+    """
+
+    def __init__(self, cfg, arrays: dict):
+        self.cfg = cfg
+        self.a = arrays
+
+    def emb_rows(self, ids: np.ndarray) -> np.ndarray:
+        kind = "f32" if self.cfg.act == "f32" else "bf16"
+        return decode_weight(self.a["emb"][ids], kind)
+
+    def lm_head_chunks(self, chunk: int = 16384):
+        kind = "f32" if self.cfg.act == "f32" else "bf16"
+        V = self.cfg.vocab
+        for v0 in range(0, V, chunk):
+            v1 = min(V, v0 + chunk)
+            yield v0, decode_weight(self.a["emb"][v0:v1], kind)
+
+    def layer(self, l: int) -> dict:
+        return self.a["layers"][l]
+
+    def w(self, l: int, name: str) -> np.ndarray:
+        lay = self.layer(l)
+        sname = {"w_qkv": "s_qkv", "w_o": "s_o"}.get(name)
+        kind = self.cfg.w
+        if name == "w_router":
+            kind = "f32" if self.cfg.w == "f32" else "bf16"
+            return decode_weight(lay[name], kind)
+        return decode_weight(lay[name], kind, None if sname is None else lay.get(sname))
+
+    def expert(self, l: int, e: int):
+        lay = self.layer(l)
+        s_gu = None if lay.get("s_gate_up") is None else lay["s_gate_up"][e]
+        s_d = None if lay.get("s_down") is None else lay["s_down"][e]
+        return (decode_weight(lay["w_gate_up"][e], self.cfg.w, s_gu),
+                decode_weight(lay["w_down"][e], self.cfg.w, s_d))
+
+
+def layer_qkv(cfg, model: OracleModel, l: int, x: np.ndarray, pos: np.ndarray):
+    """Pre-norm and projection: a = RMSNorm(x); q, k, v = a W^T; RoPE on q and k."""
+    act = cfg.act
+    T = x.shape[0]
+    Hq, Hkv, hd = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    a = storage_round(rmsnorm(x, cfg.rms_eps), act)
+    qkv = a @ model.w(l, "w_qkv").T
+    q = qkv[:, :Hq * hd].reshape(T, Hq, hd)
+    k = qkv[:, Hq * hd:(Hq + Hkv) * hd].reshape(T, Hkv, hd)
+    v = qkv[:, (Hq + Hkv) * hd:].reshape(T, Hkv, hd)
+    q = storage_round(rope(q, pos, cfg.rope_theta), act)
+    k = storage_round(rope(k, pos, cfg.rope_theta), act)
+    v = storage_round(v, act)
+    return q, k, v
+
+
+def layer_rest(cfg, model: OracleModel, l: int, x, q, k, v, kc, vc, causal: bool, info=None):
+    """Attention, output projection with residual, and the MoE FFN with residual."""
+    act = cfg.act
+    T = x.shape[0]
+    o = storage_round(attention(q, kc, vc, k, v, causal), act).reshape(T, -1)
+    h = storage_round(x + o @ model.w(l, "w_o").T, act)
+    y = storage_round(rmsnorm(h, cfg.rms_eps), act)
+    idx, gates, z = router_topk(y, model.w(l, "w_router"), cfg.top_k)
+    if info is not None:
+        info.setdefault("router_margin", []).append(router_margin(z, cfg.top_k))
+        info.setdefault("router_idx", []).append(idx)
+    return moe_ffn(y, idx, gates, lambda e: model.expert(l, e), h, act)
+
+
+def lm_head_rows(cfg, model: OracleModel, x_rows: np.ndarray, keep_logits: bool = False):
+    """Final RMSNorm of the given rows, logits over [0, V), entropy and argmax."""
+    f = storage_round(rmsnorm(x_rows, cfg.rms_eps), cfg.act)
+    R = f.shape[0]
+    z = np.empty((R, cfg.vocab))
+    for v0, w in model.lm_head_chunks():
+        z[:, v0:v0 + w.shape[0]] = f @ w.T
+    H, am, margin = entropy_argmax(z)
+    return H, am, margin, (z if keep_logits else None)
+
+
+def canvas_forward(cfg, model: OracleModel, tokens: np.ndarray, masked: np.ndarray,
+                   kcache: np.ndarray, vcache: np.ndarray, cache_len: int, info=None):
+    """Decoder pass over one canvas.  Returns the final residual stream [C, d].
+
+    kcache, vcache: [L, Hkv, cap, hd] for this canvas (decoded values).
+    """
+    C = tokens.shape[0]
+    ids = np.where(masked != 0, cfg.mask_id, tokens)
+    x = model.emb_rows(ids)
+    pos = cache_len + np.arange(C)
+    for l in range(cfg.n_layers):
+        q, k, v = layer_qkv(cfg, model, l, x, pos)
+        x = layer_rest(cfg, model, l, x, q, k, v, kcache[l, :, :cache_len],
+                       vcache[l, :, :cache_len], False, info)
+    return x
+
+
+def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache: np.ndarray,
+                cache_len: np.ndarray, gamma: float, max_steps: int, keep_logits: bool = False):
+    """One denoising step for every canvas of the batch that is not done.
+
+    state: tokens int32 [B, C], masked uint8 [B, C], n_masked int32 [B],
+    done int32 [B], step int32 [B] (numpy; not modified).  kcache/vcache:
+    decoded [L, B, Hkv, cap, hd].
+    For each live canvas: decoder pass; for every masked position the entropy
+    (stored as fp32) and greedy argmax of its logits; EB selection (all masked
+    positions at step index max_steps - 1); commit selected positions to their
+    argmax; step += 1; done = no masked position left.
+    Returns (new_state, info) where info[b] holds H, argmax, margin, rows,
+    selected, router margins and (optionally) logits.
+    """
+    new = {k: np.array(v, copy=True) for k, v in state.items()}
+    infos: List[Optional[Dict]] = []
+    B = state["tokens"].shape[0]
+    for b in range(B):
+        if state["done"][b]:
+            infos.append(None)
+            continue
+        masked = state["masked"][b]
+        rows = np.nonzero(masked)[0]
+        info: Dict = {"rows": rows}
+        if len(rows) > 0:
+            x = canvas_forward(cfg, model, state["tokens"][b], masked, kcache[:, b], vcache[:, b],
+                               int(cache_len[b]), info)
+            H, am, margin, z = lm_head_rows(cfg, model, x[rows], keep_logits)
+            Hf = H.astype(np.float32)
+            full_H = np.zeros(cfg.canvas, dtype=np.float32)
+            full_H[rows] = Hf
+            force = state["step"][b] >= max_steps - 1
+            sel = eb_select(full_H, masked, gamma, force)
+            new["tokens"][b, sel] = am[np.searchsorted(rows, np.nonzero(sel)[0])]
+            new["masked"][b, sel] = 0
+            info.update(H=Hf, argmax=am, margin=margin, logits=z, selected=sel)
+        new["n_masked"][b] = int(new["masked"][b].sum())
+        new["step"][b] = state["step"][b] + 1
+        new["done"][b] = int(new["n_masked"][b] == 0)
+        infos.append(info)
+    return new, infos
+
+
+def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
+              cache_len: np.ndarray):
+    """Causal encoder pass over finished tokens; their K/V go to the cache.
+
+    tokens int32 [B, n]; kcache/vcache decoded [L, B, Hkv, cap, hd], updated in
+    place (rows [len, len+n) of every layer, values as stored).  The encoder
+    shares the decoder's weights; its attention sees the whole cache and the
+    new tokens causally.  Returns the new cache_len.
+    """
+    B, n = tokens.shape
+    new_len = np.array(cache_len, copy=True)
+    for b in range(B):
+        L0 = int(cache_len[b])
+        x = model.emb_rows(tokens[b])
+        pos = L0 + np.arange(n)
+        for l in range(cfg.n_layers):
+            q, k, v = layer_qkv(cfg, model, l, x, pos)
+            kc, vc = kcache[l, b, :, :L0], vcache[l, b, :, :L0]
+            if l + 1 < cfg.n_layers:
+                x = layer_rest(cfg, model, l, x, q, k, v, kc, vc, True)
+            kcache[l, b, :, L0:L0 + n] = k.transpose(1, 0, 2)
+            vcache[l, b, :, L0:L0 + n] = v.transpose(1, 0, 2)
+        new_len[b] = L0 + n
+    return new_len
+
+
+def generate(cfg, model: OracleModel, kcache, vcache, cache_len, n_canvases: int, gamma: float,
+             max_steps: int):
+    """Block-autoregressive loop: denoise a canvas from all-MASK until done, append it.
+
+    Returns (tokens [B, n_canvases, C], steps per canvas [B, n_canvases], cache_len).
+    """
+    B, C = cfg.batch, cfg.canvas
+    out = np.zeros((B, n_canvases, C), dtype=np.int32)
+    steps = np.zeros((B, n_canvases), dtype=np.int32)
+    for c in range(n_canvases):
+        st = {"tokens": np.full((B, C), cfg.mask_id, dtype=np.int32),
+              "masked": np.ones((B, C), dtype=np.uint8),
+              "n_masked": np.full(B, C, dtype=np.int32),
+              "done": np.zeros(B, dtype=np.int32), "step": np.zeros(B, dtype=np.int32)}
+        while not st["done"].all():
+            st, _ = canvas_step(cfg, model, st, kcache, vcache, cache_len, gamma, max_steps)
+        out[:, c] = st["tokens"]
+        steps[:, c] = st["step"]
+        cache_len = kv_append(cfg, model, st["tokens"], kcache, vcache, cache_len)
+    return out, steps, cache_len

@@ -1,0 +1,464 @@
+"""CPU pins of the oracle: each function is checked against something other
+than itself — a library routine for a special case, a closed form, an
+invariant, brute force on tiny inputs, or hand-worked values
+(tests/golden/).  These run without a GPU."""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import dg_oracle as O
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(1234)
+
+
+# ----------------------------------------------------------------- number formats
+
+def test_round_bf16_matches_torch_conversion():
+    x32 = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),   # subnormals
+        np.clip(rng.standard_normal(2000) * 3e38, -3.39e38, 3.39e38).astype(np.float32),  # near overflow
+        np.array([0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.3895313892515355e38], np.float32),
+    ])
+    ref = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.round_bf16(x32.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_round_bf16_halfway_ties_to_even():
+    assert O.round_bf16(np.array(1.0 + 2 ** -8)) == 1.0            # tie -> even (1.0)
+    assert O.round_bf16(np.array(1.0 + 3 * 2 ** -8)) == 1.0 + 2 ** -6
+    assert O.round_bf16(np.array(1.0 + 2 ** -8 + 2 ** -30)) == 1.0 + 2 ** -7
+
+
+def test_bf16_bits_roundtrip():
+    vals = np.array([0x3F80, 0xBF80, 0x0001, 0x7F7F, 0x4049], dtype=np.uint16)
+    got = O.bf16_bits_to_f64(vals)
+    ref = torch.from_numpy(vals.view(np.int16)).view(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(got, ref)
+    assert got[0] == 1.0 and got[1] == -1.0 and got[2] == 2.0 ** -133
+
+
+def test_e4m3_decode_all_codes_vs_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    got = O.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    # OCP FP8 spec values worked by hand
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+    assert got[0x38] == 1.0 and got[0xB8] == -1.0
+
+
+# ----------------------------------------------------------------- layer pieces
+
+def test_rmsnorm_unit_rms_scale_invariance_and_torch():
+    x = rng.standard_normal((7, 96))
+    y = O.rmsnorm(x, 0.0)
+    np.testing.assert_allclose(np.sqrt((y * y).mean(-1)), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(O.rmsnorm(5.0 * x, 0.0), y, rtol=1e-13)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (96,), eps=1e-6).numpy()
+    np.testing.assert_allclose(O.rmsnorm(x, 1e-6), ref, rtol=1e-12)
+
+
+def test_gelu_tanh_vs_torch_and_limits():
+    x = np.linspace(-8, 8, 1001)
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    np.testing.assert_allclose(O.gelu_tanh(x), ref, rtol=1e-12, atol=1e-15)
+    assert O.gelu_tanh(np.array(0.0)) == 0.0
+    assert abs(O.gelu_tanh(np.array(30.0)) - 30.0) < 1e-12
+
+
+def test_rope_matches_complex_rotation_and_relative_position():
+    T, H, hd, theta = 5, 3, 16, 10000.0
+    x = rng.standard_normal((T, H, hd))
+    pos = np.array([0, 1, 7, 4096, 131071])
+    got = O.rope(x, pos, theta)
+    half = hd // 2
+    zc = x[..., :half] + 1j * x[..., half:]
+    freqs = np.array([theta ** (-(2 * i) / hd) for i in range(half)])
+    rot = zc * np.exp(1j * pos[:, None, None] * freqs[None, None, :])
+    np.testing.assert_allclose(got[..., :half], rot.real, atol=1e-12)
+    np.testing.assert_allclose(got[..., half:], rot.imag, atol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(got, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+    q, k = rng.standard_normal((1, 1, hd)), rng.standard_normal((1, 1, hd))
+    d1 = (O.rope(q, np.array([10]), theta) * O.rope(k, np.array([3]), theta)).sum()
+    d2 = (O.rope(q, np.array([107]), theta) * O.rope(k, np.array([100]), theta)).sum()
+    assert abs(d1 - d2) < 1e-10
+
+
+def _brute_attention(q, kc, vc, kn, vn, causal):
+    T, Hq, hd = q.shape
+    Hkv, P, _ = kc.shape
+    out = np.zeros_like(q)
+    for i in range(T):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            keys, vals = [], []
+            for j in range(P):
+                keys.append(kc[g, j]); vals.append(vc[g, j])
+            for j in range(T):
+                if causal and j > i:
+                    continue
+                keys.append(kn[j, g]); vals.append(vn[j, g])
+            s = [sum(q[i, h, d] * kk[d] for d in range(hd)) / math.sqrt(hd) for kk in keys]
+            m = max(s)
+            w = [math.exp(v - m) for v in s]
+            tot = sum(w)
+            for d in range(hd):
+                out[i, h, d] = sum(w[n] * vals[n][d] for n in range(len(w))) / tot
+    return out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_brute_force(causal):
+    T, Hq, Hkv, hd, P = 4, 4, 2, 8, 3
+    q = rng.standard_normal((T, Hq, hd))
+    kc, vc = rng.standard_normal((Hkv, P, hd)), rng.standard_normal((Hkv, P, hd))
+    kn, vn = rng.standard_normal((T, Hkv, hd)), rng.standard_normal((T, Hkv, hd))
+    got = O.attention(q, kc, vc, kn, vn, causal)
+    np.testing.assert_allclose(got, _brute_attention(q, kc, vc, kn, vn, causal), atol=1e-12)
+
+
+def test_attention_vs_torch_sdpa_gqa():
+    T, Hq, Hkv, hd, P = 6, 4, 2, 16, 9
+    q = rng.standard_normal((T, Hq, hd))
+    kc, vc = rng.standard_normal((Hkv, P, hd)), rng.standard_normal((Hkv, P, hd))
+    kn, vn = rng.standard_normal((T, Hkv, hd)), rng.standard_normal((T, Hkv, hd))
+    K = np.concatenate([kc, kn.transpose(1, 0, 2)], axis=1)
+    V = np.concatenate([vc, vn.transpose(1, 0, 2)], axis=1)
+    Kr = np.repeat(K, Hq // Hkv, axis=0)
+    Vr = np.repeat(V, Hq // Hkv, axis=0)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q.transpose(1, 0, 2)), torch.from_numpy(Kr), torch.from_numpy(Vr)).numpy()
+    np.testing.assert_allclose(O.attention(q, kc, vc, kn, vn, False), ref.transpose(1, 0, 2), atol=1e-12)
+
+
+def test_attention_special_cases():
+    hd = 8
+    q = rng.standard_normal((1, 1, hd))
+    v = rng.standard_normal((1, 1, hd))
+    k = rng.standard_normal((1, 1, hd))
+    empty = np.zeros((1, 0, hd))
+    # single key returns its value
+    np.testing.assert_allclose(O.attention(q, empty, empty, k, v, False)[0, 0], v[0, 0], atol=1e-14)
+    # all-equal keys return the mean of the values
+    kc = np.repeat(k[0][:, None, :], 5, axis=1)          # [1, 5, hd]
+    vc = rng.standard_normal((1, 5, hd))
+    got = O.attention(q, kc, vc, k, v, False)[0, 0]
+    np.testing.assert_allclose(got, np.concatenate([vc[0], v[0]]).mean(0), atol=1e-13)
+    # duplicating every key/value leaves the output unchanged
+    q2 = rng.standard_normal((3, 2, hd))
+    kc2, vc2 = rng.standard_normal((1, 4, hd)), rng.standard_normal((1, 4, hd))
+    kn2, vn2 = rng.standard_normal((3, 1, hd)), rng.standard_normal((3, 1, hd))
+    a = O.attention(q2, kc2, vc2, kn2, vn2, False)
+    b = O.attention(q2, np.concatenate([kc2, kc2, kn2.transpose(1, 0, 2)], 1),
+                    np.concatenate([vc2, vc2, vn2.transpose(1, 0, 2)], 1), kn2, vn2, False)
+    np.testing.assert_allclose(a, b, atol=1e-13)
+
+
+def test_router_uniform_ties_and_brute_force():
+    T, d, E = 5, 12, 8
+    y = rng.standard_normal((T, d))
+    idx, g, z = O.router_topk(y, np.zeros((E, d)), E)
+    np.testing.assert_allclose(g, 1.0 / E)
+    assert (idx == np.arange(E)).all()                    # all tied: lower index first
+    idx, g, z = O.router_topk(y, np.zeros((E, d)), 3)
+    assert (idx == np.arange(3)).all()
+    w = rng.standard_normal((E, d))
+    idx, g, z = O.router_topk(y, w, 3)
+    np.testing.assert_allclose(g.sum(1), 1.0, rtol=1e-14)
+    for t in range(T):
+        logits = [float(np.dot(y[t], w[e])) for e in range(E)]
+        best = sorted(range(E), key=lambda e: (-logits[e], e))[:3]
+        assert list(idx[t]) == best
+        ex = [math.exp(logits[e]) for e in best]
+        np.testing.assert_allclose(g[t], np.array(ex) / sum(ex), rtol=1e-12)
+
+
+def _experts(E, F, d):
+    return [(rng.standard_normal((2 * F, d)) * 0.3, rng.standard_normal((d, F)) * 0.3) for _ in range(E)]
+
+
+def test_moe_k_equals_E_uniform_gates_is_dense_mean():
+    T, d, F, E = 6, 10, 7, 4
+    y = rng.standard_normal((T, d))
+    res = rng.standard_normal((T, d))
+    ws = _experts(E, F, d)
+    idx, g, _ = O.router_topk(y, np.zeros((E, d)), E)
+    got = O.moe_ffn(y, idx, g, lambda e: ws[e], res, "f32")
+    dense = np.zeros((T, d))
+    for wgu, wd in ws:
+        u = y @ wgu.T
+        dense += (O.gelu_tanh(u[:, :F]) * u[:, F:]) @ wd.T
+    np.testing.assert_allclose(got, res + dense / E, atol=1e-12)
+
+
+def test_moe_single_expert_is_plain_gated_ffn():
+    T, d, F = 5, 9, 6
+    y = rng.standard_normal((T, d))
+    res = rng.standard_normal((T, d))
+    wgu, wd = _experts(1, F, d)[0]
+    idx, g, _ = O.router_topk(y, rng.standard_normal((1, d)), 1)
+    got = O.moe_ffn(y, idx, g, lambda e: (wgu, wd), res, "f32")
+    for t in range(T):
+        gate = [sum(y[t, c] * wgu[f, c] for c in range(d)) for f in range(F)]
+        up = [sum(y[t, c] * wgu[F + f, c] for c in range(d)) for f in range(F)]
+        act = [0.5 * gv * (1 + math.tanh(math.sqrt(2 / math.pi) * (gv + 0.044715 * gv ** 3))) * uv
+               for gv, uv in zip(gate, up)]
+        for c in range(d):
+            want = res[t, c] + sum(act[f] * wd[c, f] for f in range(F))
+            assert abs(got[t, c] - want) < 1e-12
+
+
+def test_moe_token_permutation_equivariance():
+    T, d, F, E = 8, 10, 6, 5
+    y = rng.standard_normal((T, d))
+    res = rng.standard_normal((T, d))
+    ws = _experts(E, F, d)
+    wr = rng.standard_normal((E, d))
+    idx, g, _ = O.router_topk(y, wr, 2)
+    a = O.moe_ffn(y, idx, g, lambda e: ws[e], res, "f32")
+    p = rng.permutation(T)
+    idx2, g2, _ = O.router_topk(y[p], wr, 2)
+    b = O.moe_ffn(y[p], idx2, g2, lambda e: ws[e], res[p], "f32")
+    np.testing.assert_allclose(b, a[p], atol=1e-13)
+
+
+def test_entropy_closed_forms():
+    V = 512
+    H, am, _ = O.entropy_argmax(np.zeros((1, V)))
+    assert abs(H[0] - math.log(V)) < 1e-12 and am[0] == 0
+    z = np.zeros((1, V)); z[0, 17] = 100.0
+    H, am, _ = O.entropy_argmax(z)
+    eps = math.exp(-100.0)
+    p1 = 1.0 / (1.0 + (V - 1) * eps)
+    pr = eps * p1
+    want = -(p1 * math.log(p1) + (V - 1) * pr * math.log(pr))
+    assert abs(H[0] - want) < 1e-40 + 1e-9 * want and am[0] == 17
+    z = np.full((1, V), -200.0); z[0, 300] = 50.0; z[0, 42] = 50.0
+    H, am, margin = O.entropy_argmax(z)
+    assert abs(H[0] - math.log(2.0)) < 1e-12 and am[0] == 42 and margin[0] == 0.0
+
+
+def test_entropy_random_rows_vs_scipy():
+    from scipy.stats import entropy as sp_entropy
+    from scipy.special import softmax
+    z = rng.standard_normal((4, 3000)) * 3.0
+    H, am, margin = O.entropy_argmax(z)
+    for r in range(4):
+        assert abs(H[r] - sp_entropy(softmax(z[r]))) < 1e-10
+        assert am[r] == int(np.argmax(z[r]))
+        s = np.sort(z[r])
+        assert margin[r] == s[-1] - s[-2]
+
+
+# ----------------------------------------------------------------- EB sampler
+
+def _golden_eb():
+    cases = []
+    with open(os.path.join(GOLDEN, "eb_cases.txt")) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            g, h, m, sel = [p.strip() for p in line.split("|")]
+            cases.append((float(g), np.array([float(v) for v in h.split(",")], np.float32),
+                          np.array([int(v) for v in m.split(",")], np.uint8),
+                          [int(v) for v in sel.split(",")] if sel else []))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_eb())
+def test_eb_hand_worked(case):
+    gamma, H, masked, want = case
+    sel = O.eb_select(H, masked, gamma, False)
+    assert sorted(np.nonzero(sel)[0].tolist()) == want
+
+
+def test_eb_bound_zero_commits_lowest_single():
+    for _ in range(50):
+        n = 32
+        H = rng.uniform(0.01, 12.0, n).astype(np.float32)
+        masked = (rng.uniform(size=n) < 0.7).astype(np.uint8)
+        if masked.sum() == 0:
+            continue
+        sel = O.eb_select(H, masked, 0.0, False)
+        cand = np.nonzero(masked)[0]
+        best = cand[np.lexsort((cand, H[cand]))[0]]
+        assert sel.sum() == 1 and sel[best]
+
+
+def test_eb_infinite_bound_and_force_commit_all():
+    H = rng.uniform(0, 12, 40).astype(np.float32)
+    masked = (rng.uniform(size=40) < 0.5).astype(np.uint8)
+    assert (O.eb_select(H, masked, math.inf, False) == (masked != 0)).all()
+    assert (O.eb_select(H, masked, 0.0, True) == (masked != 0)).all()
+
+
+def test_eb_brute_force_prefix_enumeration():
+    for _ in range(200):
+        n = int(rng.integers(1, 7))
+        H = rng.choice(np.array([0.0, 0.25, 0.5, 0.75, 1.0, 1.5], np.float32), n)
+        masked = (rng.uniform(size=n) < 0.8).astype(np.uint8)
+        gamma = float(rng.choice([0.0, 0.3, 0.5, 1.0, 2.0]))
+        cand = [i for i in range(n) if masked[i]]
+        if not cand:
+            continue
+        order = sorted(cand, key=lambda i: (float(H[i]), i))
+        best = 1
+        for k in range(1, len(order) + 1):          # every prefix of the sorted candidates
+            chosen = [float(H[i]) for i in order[:k]]
+            if sum(chosen) - max(chosen) <= gamma:
+                best = max(best, k)
+        sel = O.eb_select(H, masked, gamma, False)
+        assert sorted(np.nonzero(sel)[0].tolist()) == sorted(order[:best])
+
+
+def test_eb_permutation_invariance():
+    n = 64
+    H = rng.choice(np.array([0.1, 0.2, 0.3, 5.0], np.float32), n)   # many ties
+    masked = np.ones(n, np.uint8)
+    sel = O.eb_select(H, masked, 0.65, False)
+    p = rng.permutation(n)
+    sel_p = O.eb_select(H[p], masked[p], 0.65, False)
+    # the committed multiset of entropies is the same; only tie-broken identities may move
+    assert sorted(H[sel].tolist()) == sorted(H[p][sel_p].tolist())
+
+
+def test_eb_rejects_non_finite():
+    with pytest.raises(FloatingPointError):
+        O.eb_select(np.array([0.1, np.nan], np.float32), np.array([1, 1], np.uint8), 1.0, False)
+
+
+# ----------------------------------------------------------------- whole-step invariants (tiny workload)
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = synth.get_config("tiny")
+    m = synth.make_model(cfg, "cpu")
+    arr = {"emb": synth.to_numpy(m["emb"]),
+           "layers": [{k: synth.to_numpy(v) for k, v in lay.items()} for lay in m["layers"]]}
+    kv = synth.make_prompt_kv(cfg, "cpu")
+    return cfg, O.OracleModel(cfg, arr), kv
+
+
+def _state(cfg):
+    st = synth.make_canvas_state(cfg, "all_mask")
+    return {k: synth.to_numpy(v) for k, v in st.items()}
+
+
+def test_tiny_generate_one_commit_per_step(tiny):
+    cfg, model, kv = tiny
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    st = _state(cfg)
+    seen = 0
+    for s in range(cfg.canvas):
+        st2, info = O.canvas_step(cfg, model, st, kc, vc, cl, cfg.gamma, cfg.max_steps)
+        H = info[0]["H"]
+        # random-init logits are nearly uniform: entropy ~ ln V >> gamma -> exactly one commit
+        assert np.all(H > 0.9 * math.log(cfg.vocab))
+        assert st["n_masked"][0] - st2["n_masked"][0] == 1
+        lowest = info[0]["rows"][np.lexsort((info[0]["rows"], H))[0]]
+        assert st2["masked"][0, lowest] == 0 and st2["tokens"][0, lowest] != cfg.mask_id
+        st = st2
+        seen += 1
+        if st["done"][0]:
+            break
+    assert seen == cfg.canvas and st["done"][0] == 1 and st["step"][0] == cfg.canvas
+    assert (st["tokens"][0] < cfg.vocab).all()
+
+
+def test_tiny_zero_lm_head_gives_ln_v_and_index_order(tiny):
+    cfg, model, kv = tiny
+    arr = dict(model.a)
+    emb = arr["emb"].copy()
+    emb[:cfg.vocab] = 0.0                                  # every logit 0: uniform softmax
+    m0 = O.OracleModel(cfg, dict(arr, emb=emb))
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    st = _state(cfg)
+    st2, info = O.canvas_step(cfg, m0, st, kc, vc, synth.to_numpy(kv["cache_len"]), 0.0, 16)
+    np.testing.assert_allclose(info[0]["H"], math.log(cfg.vocab), rtol=1e-6)
+    assert (info[0]["argmax"] == 0).all()
+    assert st2["masked"][0, 0] == 0 and st2["masked"][0, 1:].all() and st2["tokens"][0, 0] == 0
+
+
+def test_tiny_infinite_bound_and_step_cap(tiny):
+    cfg, model, kv = tiny
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    st2, _ = O.canvas_step(cfg, model, _state(cfg), kc, vc, cl, math.inf, 16)
+    assert st2["done"][0] == 1 and st2["n_masked"][0] == 0
+    st = _state(cfg)
+    st["step"][:] = 15
+    st2, _ = O.canvas_step(cfg, model, st, kc, vc, cl, 0.0, 16)   # last allowed step
+    assert st2["done"][0] == 1
+
+
+def test_tiny_kv_append_single_layer_is_direct_projection(tiny):
+    cfg, model, kv = tiny
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    toks = rng.integers(0, cfg.vocab, (1, cfg.canvas)).astype(np.int32)
+    new_len = O.kv_append(cfg, model, toks, kc, vc, cl)
+    assert new_len[0] == cl[0] + cfg.canvas
+    # one layer: the appended K/V are the projections of the normed embeddings, rotated
+    x = model.emb_rows(toks[0])
+    a = O.rmsnorm(x, cfg.rms_eps)
+    w = model.w(0, "w_qkv")
+    Hq, Hkv, hd = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    kraw = (a @ w[Hq * hd:(Hq + Hkv) * hd].T).reshape(cfg.canvas, Hkv, hd)
+    vraw = (a @ w[(Hq + Hkv) * hd:].T).reshape(cfg.canvas, Hkv, hd)
+    pos = cl[0] + np.arange(cfg.canvas)
+    np.testing.assert_allclose(kc[0, 0, :, cl[0]:new_len[0]],
+                               O.rope(kraw, pos, cfg.rope_theta).transpose(1, 0, 2), atol=1e-12)
+    np.testing.assert_allclose(vc[0, 0, :, cl[0]:new_len[0]], vraw.transpose(1, 0, 2), atol=1e-12)
+    # rows outside the appended range are untouched
+    assert (kc[0, 0, :, new_len[0]:] == 0).all()
+
+
+def test_tiny_full_generate_two_canvases(tiny):
+    cfg, model, kv = tiny
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    toks, steps, new_len = O.generate(cfg, model, kc, vc, cl, cfg.n_canvases, cfg.gamma, cfg.max_steps)
+    assert (steps == cfg.canvas).all()            # one commit per step at gamma 0.1
+    assert new_len[0] == cfg.prompt_len + cfg.n_canvases * cfg.canvas
+    assert (toks < cfg.vocab).all()
+
+
+def test_tiny_layer_residual_wiring(tiny):
+    """Zero output projection and zero expert down-projections: the layer is the
+    identity on its residual stream; zero output projection alone: the layer no
+    longer depends on the prompt cache."""
+    cfg, model, kv = tiny
+    lay = dict(model.a["layers"][0])
+    lay_zero = dict(lay, w_o=np.zeros_like(lay["w_o"]), w_down=np.zeros_like(lay["w_down"]))
+    m0 = O.OracleModel(cfg, dict(model.a, layers=[lay_zero]))
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)[:, 0]
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)[:, 0]
+    toks = rng.integers(0, cfg.vocab, cfg.canvas).astype(np.int32)
+    masked = np.zeros(cfg.canvas, np.uint8)
+    x = O.canvas_forward(cfg, m0, toks, masked, kc, vc, cfg.prompt_len)
+    np.testing.assert_array_equal(x, model.emb_rows(toks))
+    m1 = O.OracleModel(cfg, dict(model.a, layers=[dict(lay, w_o=np.zeros_like(lay["w_o"]))]))
+    xa = O.canvas_forward(cfg, m1, toks, masked, kc, vc, cfg.prompt_len)
+    xb = O.canvas_forward(cfg, m1, toks, masked, kc * 3.0 + 1.0, vc * -2.0, cfg.prompt_len)
+    np.testing.assert_array_equal(xa, xb)
+    assert not np.array_equal(xa, model.emb_rows(toks))
+    xc = O.canvas_forward(cfg, model, toks, masked, kc * 3.0 + 1.0, vc * -2.0, cfg.prompt_len)
+    assert np.abs(xc - O.canvas_forward(cfg, model, toks, masked, kc, vc, cfg.prompt_len)).max() > 1e-6
