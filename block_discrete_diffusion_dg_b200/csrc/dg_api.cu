@@ -1,0 +1,511 @@
+// C ABI of the canvas-step library: argument checks, the scratch layout, and the chaining of the
+// kernels into the operations declared in include/dg.h.  Nothing here allocates device memory or
+// synchronises; every launch goes to the caller's stream.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+
+static std::atomic<unsigned long long> g_launches{0};
+static thread_local char g_err[256] = "no error";
+
+// Per-thread launch timeline for dg_profile_*: one event recorded before every launch.
+struct Profile {
+  std::vector<cudaEvent_t> ev;
+  std::vector<const char *> name;
+  int n = 0;
+  bool on = false;
+};
+static thread_local Profile g_prof;
+
+void note_launch(cudaStream_t s, const char *name) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (g_prof.on && g_prof.n < (int)g_prof.ev.size()) {
+    cudaEventRecord(g_prof.ev[g_prof.n], s);
+    g_prof.name[g_prof.n] = name;
+    ++g_prof.n;
+  }
+}
+
+int check_launch(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return DG_OK;
+  snprintf(g_err, sizeof(g_err), "%s: %s", what, cudaGetErrorString(e));
+  return DG_ERR_CUDA;
+}
+
+namespace {
+
+constexpr int TILE_M = 64;  // rows per grouped-GEMM tile
+
+inline size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
+inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
+
+enum Buf {
+  B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
+  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_LIVE, B_ROWS, B_NROWS, B_FIN, B_LOGITS, B_ENT, B_AM,
+  B_ATTN, B_COUNT
+};
+
+struct Layout {
+  size_t off[B_COUNT];
+  size_t total;
+  int max_tiles;
+};
+
+Layout make_layout(const dg_config &c, int batch, int n, int cap) {
+  const size_t T = (size_t)batch * n, a = esz(c.act_dtype);
+  const size_t d = c.d_model, hd = c.head_dim, k = c.top_k, F = c.d_ff;
+  const size_t qkvw = (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * hd;
+  const size_t TK = T * k;
+  Layout L;
+  L.max_tiles = (int)((TK + TILE_M - 1) / TILE_M) + c.n_experts;
+  size_t sz[B_COUNT];
+  sz[B_X] = T * d * a;
+  sz[B_A] = T * d * a;
+  sz[B_QKV] = T * qkvw * 4;
+  sz[B_CS] = T * hd * 4;
+  sz[B_Q] = T * c.n_q_heads * hd * a;
+  sz[B_KN] = T * c.n_kv_heads * hd * a;
+  sz[B_VN] = T * c.n_kv_heads * hd * a;
+  sz[B_O] = T * c.n_q_heads * hd * a;
+  sz[B_H] = T * d * a;
+  sz[B_Y] = T * d * a;
+  sz[B_IDX] = TK * 4;
+  sz[B_W] = TK * 4;
+  sz[B_OFF] = (size_t)(c.n_experts + 1) * 4;
+  sz[B_PERM] = TK * 4;
+  sz[B_INV] = TK * 4;
+  sz[B_TILES] = (size_t)L.max_tiles * sizeof(GroupTile);
+  sz[B_NTILES] = 4;
+  sz[B_U] = TK * 2 * F * 4;
+  sz[B_ACT] = TK * F * a;
+  sz[B_YE] = TK * d * a;
+  sz[B_LIVE] = T;
+  sz[B_ROWS] = T * 4;
+  sz[B_NROWS] = 4;
+  sz[B_FIN] = T * d * a;
+  sz[B_LOGITS] = T * (size_t)c.vocab * 4;
+  sz[B_ENT] = T * 4;
+  sz[B_AM] = T * 4;
+  sz[B_ATTN] = attention_ws_bytes(batch, n, c.n_q_heads, c.head_dim, cap);
+  size_t o = 0;
+  for (int i = 0; i < B_COUNT; ++i) {
+    L.off[i] = o;
+    o += align_up(sz[i]);
+  }
+  L.total = o;
+  return L;
+}
+
+struct Ws {
+  char *base;
+  const Layout *L;
+  template <typename P> P *at(Buf b) const { return reinterpret_cast<P *>(base + L->off[b]); }
+};
+
+bool cfg_ok(const dg_config *c) {
+  if (!c) return false;
+  if (c->d_model <= 0 || c->d_model % 8 || c->n_q_heads <= 0 || c->n_kv_heads <= 0) return false;
+  if (c->n_q_heads % c->n_kv_heads) return false;
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->n_experts <= 0 || c->n_experts > 256 || c->top_k <= 0 || c->top_k > c->n_experts ||
+      c->top_k > 32)
+    return false;
+  if (c->d_ff <= 0 || c->d_ff % 8 || c->vocab < 2 || c->canvas <= 0 || c->canvas > 1024)
+    return false;
+  if (c->n_layers <= 0) return false;
+  if (!(c->rope_theta > 0.0) || !(c->rms_eps >= 0.0)) return false;
+  if (c->act_dtype == DG_F32) return c->w_dtype == DG_F32;
+  if (c->act_dtype == DG_BF16) return c->w_dtype == DG_BF16 || c->w_dtype == DG_E4M3;
+  return false;
+}
+
+bool lw_ok(const dg_config *c, const dg_layer_weights *w) {
+  if (!w || !w->w_qkv || !w->w_o || !w->w_router || !w->w_gate_up || !w->w_down) return false;
+  if (c->w_dtype == DG_E4M3 && (!w->s_qkv || !w->s_o || !w->s_gate_up || !w->s_down))
+    return false;
+  return true;
+}
+
+int router_type(const dg_config *c) { return c->w_dtype == DG_F32 ? DG_F32 : DG_BF16; }
+const float *scale_or_null(const dg_config *c, const float *s) {
+  return c->w_dtype == DG_E4M3 ? s : nullptr;
+}
+
+#define DG_TRY(x)                 \
+  do {                            \
+    const int rc__ = (x);         \
+    if (rc__ != DG_OK) return rc__; \
+  } while (0)
+
+// ---- one layer's pieces, shared by the step and the append --------------------------------
+
+int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T, cudaStream_t s) {
+  GemmDesc g{};
+  g.act = c.act_dtype; g.w = c.w_dtype;
+  g.A = ws.at<void>(B_A); g.lda = c.d_model;
+  g.B = w.w_qkv; g.ldb = c.d_model; g.strideB = 0;
+  g.bscale = scale_or_null(&c, w.s_qkv);
+  g.M = T; g.N = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim; g.K = c.d_model;
+  g.name = "gemm_qkv";
+  return launch_gemm_simt(g, EPI_F32, ws.at<void>(B_QKV), g.N, nullptr, s);
+}
+
+// o -> h = x + o W_o^T -> y = RMSNorm(h) -> router -> permute -> experts -> x
+int attn_out_and_moe(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
+                     const uint8_t *token_live, cudaStream_t s) {
+  const int d = c.d_model, hq = c.n_q_heads * c.head_dim;
+  GemmDesc g{};
+  g.act = c.act_dtype; g.w = c.w_dtype;
+  g.A = ws.at<void>(B_O); g.lda = hq;
+  g.B = w.w_o; g.ldb = hq;
+  g.bscale = scale_or_null(&c, w.s_o);
+  g.M = T; g.N = d; g.K = hq;
+  g.name = "gemm_o_resid";
+  DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
+  DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
+                        ws.at<void>(B_Y), s));
+  DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
+                       ws.at<void>(B_Y), w.w_router, token_live, ws.at<int32_t>(B_IDX),
+                       ws.at<float>(B_W), s));
+  DG_TRY(launch_permute(T, c.top_k, c.n_experts, ws.at<int32_t>(B_IDX), ws.at<int32_t>(B_OFF),
+                        ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV), s));
+  return DG_OK;
+}
+
+int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
+                const void *y, const int32_t *topk_idx, const float *topk_w,
+                const int32_t *expert_off, const int32_t *perm, const int32_t *inv_perm,
+                const void *residual, void *out, cudaStream_t s) {
+  const int d = c.d_model, F = c.d_ff, E = c.n_experts, k = c.top_k;
+  const int TK = T * k;
+  DG_TRY(launch_build_tiles(E, expert_off, TILE_M, ws.at<GroupTile>(B_TILES),
+                            ws.at<int32_t>(B_NTILES), ws.L->max_tiles, s));
+  GemmDesc g1{};
+  g1.act = c.act_dtype; g1.w = c.w_dtype;
+  g1.A = y; g1.lda = d; g1.a_rowmap = perm; g1.a_rowdiv = k;
+  g1.B = w.w_gate_up; g1.ldb = d; g1.strideB = (long long)2 * F * d;
+  g1.bscale = scale_or_null(&c, w.s_gate_up);
+  g1.M = TK; g1.N = 2 * F; g1.K = d;
+  g1.tiles = ws.at<GroupTile>(B_TILES); g1.n_tiles = ws.at<int32_t>(B_NTILES);
+  g1.group_off = expert_off; g1.max_tiles = ws.L->max_tiles;
+  g1.name = "moe_gemm_gate_up";
+  DG_TRY(launch_gemm_simt(g1, EPI_F32, ws.at<void>(B_U), 2 * F, nullptr, s));
+  DG_TRY(launch_gate(c.act_dtype, TK, F, ws.at<float>(B_U), expert_off, E, ws.at<void>(B_ACT), s));
+  GemmDesc g2{};
+  g2.act = c.act_dtype; g2.w = c.w_dtype;
+  g2.A = ws.at<void>(B_ACT); g2.lda = F;
+  g2.B = w.w_down; g2.ldb = F; g2.strideB = (long long)d * F;
+  g2.bscale = scale_or_null(&c, w.s_down);
+  g2.M = TK; g2.N = d; g2.K = F;
+  g2.tiles = g1.tiles; g2.n_tiles = g1.n_tiles; g2.group_off = expert_off;
+  g2.max_tiles = ws.L->max_tiles;
+  g2.name = "moe_gemm_down";
+  DG_TRY(launch_gemm_simt(g2, EPI_ACT, ws.at<void>(B_YE), d, nullptr, s));
+  return launch_combine(c.act_dtype, T, d, k, topk_idx, topk_w, inv_perm, ws.at<void>(B_YE),
+                        residual, out, s);
+}
+
+// Final RMSNorm of rows row_idx[r] (r < *n_rows) of h, LM head, entropy/argmax at source rows.
+int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_rows_dev,
+               const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
+               int32_t *argmax, float *logits_out, int scatter_logits, int32_t *st,
+               cudaStream_t s) {
+  DG_TRY(launch_rmsnorm(c.act_dtype, h, row_idx, n_rows_dev, max_rows, c.d_model, c.rms_eps,
+                        ws.at<void>(B_FIN), s));
+  float *logits = (logits_out && !scatter_logits) ? logits_out : ws.at<float>(B_LOGITS);
+  GemmDesc g{};
+  g.act = c.act_dtype; g.w = c.act_dtype;
+  g.A = ws.at<void>(B_FIN); g.lda = c.d_model;
+  g.B = w_lm; g.ldb = c.d_model;
+  g.M = max_rows; g.M_dev = n_rows_dev; g.N = c.vocab; g.K = c.d_model;
+  g.name = "lm_head_logits";
+  DG_TRY(launch_gemm_simt(g, EPI_F32, logits, c.vocab, nullptr, s));
+  DG_TRY(launch_entropy_rows(logits, c.vocab, max_rows, n_rows_dev, row_idx, entropy, argmax, st,
+                             s));
+  if (logits_out && scatter_logits)
+    DG_TRY(launch_scatter_rows(logits, c.vocab, max_rows, n_rows_dev, row_idx, logits_out, s));
+  return DG_OK;
+}
+
+long long quant_gamma(double gamma) {
+  if (std::isinf(gamma)) return INT64_MAX;
+  const double v = std::floor(gamma * 4294967296.0);
+  if (v >= 9.2233720368547758e18) return INT64_MAX;
+  return (long long)v;
+}
+
+int check_ws(const dg_config *c, int batch, int n, int cap, const void *ws, size_t ws_bytes,
+             Layout *L) {
+  *L = make_layout(*c, batch, n, cap);
+  if (!ws) return DG_ERR_INVALID_ARG;
+  if (((uintptr_t)ws) & 255) return DG_ERR_INVALID_ARG;
+  if (ws_bytes < L->total) return DG_ERR_WORKSPACE;
+  return DG_OK;
+}
+
+}  // namespace
+}  // namespace dg
+
+using namespace dg;
+
+extern "C" {
+
+size_t dg_workspace_size(const dg_config *cfg, int batch, int n_tokens, int cache_cap) {
+  if (!cfg_ok(cfg) || batch <= 0 || n_tokens <= 0 || cache_cap < 0) return 0;
+  return make_layout(*cfg, batch, n_tokens, cache_cap).total;
+}
+
+int dg_read_status(const int32_t *dev_status, void *stream) {
+  if (!dev_status) return DG_ERR_INVALID_ARG;
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, dev_status, 4, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    snprintf(g_err, sizeof(g_err), "dg_read_status: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return h;
+}
+
+int dg_clear_status(int32_t *dev_status, void *stream) {
+  if (!dev_status) return DG_ERR_INVALID_ARG;
+  const cudaError_t e = cudaMemsetAsync(dev_status, 0, 4, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    snprintf(g_err, sizeof(g_err), "dg_clear_status: %s", cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+const char *dg_last_cuda_error(void) { return g_err; }
+
+uint64_t dg_launch_count(void) { return g_launches.load(); }
+
+int dg_profile_begin(int max_records) {
+  if (max_records <= 0) return DG_ERR_INVALID_ARG;
+  while ((int)g_prof.ev.size() < max_records) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return check_launch("dg_profile_begin");
+    g_prof.ev.push_back(e);
+    g_prof.name.push_back(nullptr);
+  }
+  g_prof.n = 0;
+  g_prof.on = true;
+  return DG_OK;
+}
+
+int dg_profile_mark(void *stream) {
+  if (!g_prof.on) return DG_ERR_INVALID_ARG;
+  note_launch((cudaStream_t)stream, "(mark)");
+  g_launches.fetch_sub(1, std::memory_order_relaxed);  // a mark is not a kernel
+  return DG_OK;
+}
+
+int dg_profile_end(float *ms, int max_out, int *n_out) {
+  if (!g_prof.on) return DG_ERR_INVALID_ARG;
+  g_prof.on = false;
+  const int n = g_prof.n;
+  if (n > 0 && cudaEventSynchronize(g_prof.ev[n - 1]) != cudaSuccess)
+    return check_launch("dg_profile_end");
+  int k = 0;
+  for (int i = 0; i + 1 < n && k < max_out; ++i, ++k) {
+    float t = 0.f;
+    cudaEventElapsedTime(&t, g_prof.ev[i], g_prof.ev[i + 1]);
+    if (ms) ms[k] = t;
+  }
+  if (n_out) *n_out = k;
+  return DG_OK;
+}
+
+const char *dg_profile_name(int i) {
+  if (i < 0 || i >= g_prof.n || !g_prof.name[i]) return "";
+  return g_prof.name[i];
+}
+
+int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
+                   const void *k_cache, const void *v_cache, const int32_t *cache_len,
+                   int cache_cap, const void *k_new, const void *v_new, int causal,
+                   const int32_t *done, void *out, void *ws, size_t ws_bytes,
+                   int32_t *dev_status, void *stream) {
+  (void)dev_status;
+  if (!cfg_ok(cfg) || batch <= 0 || n_tokens <= 0 || cache_cap < 0) return DG_ERR_INVALID_ARG;
+  if (!q || !cache_len || !k_new || !v_new || !out) return DG_ERR_INVALID_ARG;
+  if (cache_cap > 0 && (!k_cache || !v_cache)) return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
+  return launch_attention(cfg->act_dtype, batch, n_tokens, cfg->n_q_heads, cfg->n_kv_heads,
+                          cfg->head_dim, q, k_cache, v_cache, cache_len, cache_cap, k_new, v_new,
+                          causal ? 1 : 0, done, out, (char *)ws + L.off[B_ATTN],
+                          (cudaStream_t)stream);
+}
+
+int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *w_router,
+                 const uint8_t *token_live, int32_t *topk_idx, float *topk_w,
+                 int32_t *expert_off, int32_t *perm, int32_t *inv_perm, void *ws,
+                 size_t ws_bytes, int32_t *dev_status, void *stream) {
+  (void)dev_status;
+  if (!cfg_ok(cfg) || n_tokens <= 0) return DG_ERR_INVALID_ARG;
+  if (!y || !w_router || !topk_idx || !topk_w || !expert_off || !perm || !inv_perm)
+    return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, 1, n_tokens, 0, ws, ws_bytes, &L));
+  const cudaStream_t s = (cudaStream_t)stream;
+  DG_TRY(launch_router(cfg->act_dtype, router_type(cfg), n_tokens, cfg->d_model, cfg->n_experts,
+                       cfg->top_k, y, w_router, token_live, topk_idx, topk_w, s));
+  return launch_permute(n_tokens, cfg->top_k, cfg->n_experts, topk_idx, expert_off, perm,
+                        inv_perm, s);
+}
+
+int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t *topk_idx,
+               const float *topk_w, const int32_t *expert_off, const int32_t *perm,
+               const int32_t *inv_perm, const dg_layer_weights *lw, const void *residual,
+               void *out, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  (void)dev_status;
+  if (!cfg_ok(cfg) || n_tokens <= 0 || !lw_ok(cfg, lw)) return DG_ERR_INVALID_ARG;
+  if (!y || !topk_idx || !topk_w || !expert_off || !perm || !inv_perm || !residual || !out)
+    return DG_ERR_INVALID_ARG;
+  if (out == y) return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, 1, n_tokens, 0, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  return moe_experts(*cfg, *lw, w, n_tokens, y, topk_idx, topk_w, expert_off, perm, inv_perm,
+                     residual, out, (cudaStream_t)stream);
+}
+
+int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_dev,
+                      const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
+                      int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
+                      int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg) || n_rows <= 0 || !h || !w_lm || !entropy || !argmax)
+    return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, 1, n_rows, 0, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  return lm_entropy(*cfg, w, n_rows, n_rows_dev, h, row_idx, w_lm, entropy, argmax, logits_dbg,
+                    0, dev_status, (cudaStream_t)stream);
+}
+
+int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
+                 double gamma, int max_steps, int32_t *tokens, uint8_t *masked,
+                 uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
+                 int32_t *dev_status, void *stream) {
+  if (batch <= 0 || canvas <= 0 || canvas > 1024 || max_steps <= 0) return DG_ERR_INVALID_ARG;
+  if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
+  if (!entropy || !argmax || !tokens || !masked || !n_masked || !done || !step)
+    return DG_ERR_INVALID_ARG;
+  return launch_eb_select(batch, canvas, entropy, argmax, quant_gamma(gamma), max_steps, tokens,
+                          masked, selected, n_masked, done, step, dev_status,
+                          (cudaStream_t)stream);
+}
+
+int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
+                 int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
+                 void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || n_tokens <= 0)
+    return DG_ERR_INVALID_ARG;
+  if (!tokens || !k_cache || !v_cache || !cache_len || cache_cap <= 0) return DG_ERR_INVALID_ARG;
+  if (n_tokens > cache_cap) return DG_ERR_CAPACITY;
+  for (int l = 0; l < cfg->n_layers; ++l)
+    if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  const dg_config &c = *cfg;
+  const cudaStream_t s = (cudaStream_t)stream;
+  const int T = batch * n_tokens, d = c.d_model;
+  const size_t layer_elems = (size_t)batch * c.n_kv_heads * cache_cap * c.head_dim;
+  const size_t ae = esz(c.act_dtype);
+  DG_TRY(launch_embed_norm(c.act_dtype, tokens, nullptr, model->emb, T, d, c.vocab, c.rms_eps,
+                           w.at<void>(B_X), w.at<void>(B_A), dev_status, s));
+  DG_TRY(launch_rope_table(batch, n_tokens, c.head_dim, c.rope_theta, cache_len,
+                           w.at<float>(B_CS), s));
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights &lw = model->layers[l];
+    char *kc = (char *)k_cache + l * layer_elems * ae;
+    char *vc = (char *)v_cache + l * layer_elems * ae;
+    if (l > 0)
+      DG_TRY(launch_rmsnorm(c.act_dtype, w.at<void>(B_X), nullptr, nullptr, T, d, c.rms_eps,
+                            w.at<void>(B_A), s));
+    DG_TRY(qkv_proj(c, lw, w, T, s));
+    DG_TRY(launch_qkv_split(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                            w.at<float>(B_QKV), w.at<float>(B_CS), w.at<void>(B_Q),
+                            w.at<void>(B_KN), w.at<void>(B_VN), kc, vc, cache_len, cache_cap,
+                            dev_status, s));
+    if (l + 1 == c.n_layers) break;
+    DG_TRY(launch_attention(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                            w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
+                            w.at<void>(B_VN), 1, nullptr, w.at<void>(B_O),
+                            w.at<void>(B_ATTN), s));
+    DG_TRY(attn_out_and_moe(c, lw, w, T, nullptr, s));
+    DG_TRY(moe_experts(c, lw, w, T, w.at<void>(B_Y), w.at<int32_t>(B_IDX), w.at<float>(B_W),
+                       w.at<int32_t>(B_OFF), w.at<int32_t>(B_PERM), w.at<int32_t>(B_INV),
+                       w.at<void>(B_H), w.at<void>(B_X), s));
+  }
+  return launch_add_cache_len(batch, n_tokens, cache_cap, cache_len, s);
+}
+
+int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
+                   uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
+                   int max_steps, double gamma, const void *k_cache, const void *v_cache,
+                   const int32_t *cache_len, int cache_cap, float *entropy_out,
+                   int32_t *argmax_out, float *logits_dbg, void *ws, size_t ws_bytes,
+                   int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
+    return DG_ERR_INVALID_ARG;
+  if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
+  if (cache_cap < 0 || (cache_cap > 0 && (!k_cache || !v_cache))) return DG_ERR_INVALID_ARG;
+  if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
+  for (int l = 0; l < cfg->n_layers; ++l)
+    if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
+  const dg_config &c = *cfg;
+  const int C = c.canvas, T = batch * C, d = c.d_model;
+  Layout L;
+  DG_TRY(check_ws(cfg, batch, C, cache_cap, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  const cudaStream_t s = (cudaStream_t)stream;
+  const size_t layer_elems = (size_t)batch * c.n_kv_heads * cache_cap * c.head_dim;
+  const size_t ae = esz(c.act_dtype);
+  uint8_t *live = w.at<uint8_t>(B_LIVE);
+  int32_t *rows = w.at<int32_t>(B_ROWS), *n_rows = w.at<int32_t>(B_NROWS);
+
+  DG_TRY(launch_compact_rows(batch, C, masked, done, rows, n_rows, live, s));
+  DG_TRY(launch_embed_norm(c.act_dtype, tokens, masked, model->emb, T, d, c.vocab, c.rms_eps,
+                           w.at<void>(B_X), w.at<void>(B_A), dev_status, s));
+  DG_TRY(launch_rope_table(batch, C, c.head_dim, c.rope_theta, cache_len, w.at<float>(B_CS), s));
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights &lw = model->layers[l];
+    const char *kc = (const char *)k_cache + l * layer_elems * ae;
+    const char *vc = (const char *)v_cache + l * layer_elems * ae;
+    if (l > 0)
+      DG_TRY(launch_rmsnorm(c.act_dtype, w.at<void>(B_X), nullptr, nullptr, T, d, c.rms_eps,
+                            w.at<void>(B_A), s));
+    DG_TRY(qkv_proj(c, lw, w, T, s));
+    DG_TRY(launch_qkv_split(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                            w.at<float>(B_QKV), w.at<float>(B_CS), w.at<void>(B_Q),
+                            w.at<void>(B_KN), w.at<void>(B_VN), nullptr, nullptr, cache_len,
+                            cache_cap, dev_status, s));
+    DG_TRY(launch_attention(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                            w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
+                            w.at<void>(B_VN), 0, done, w.at<void>(B_O), w.at<void>(B_ATTN), s));
+    DG_TRY(attn_out_and_moe(c, lw, w, T, live, s));
+    DG_TRY(moe_experts(c, lw, w, T, w.at<void>(B_Y), w.at<int32_t>(B_IDX), w.at<float>(B_W),
+                       w.at<int32_t>(B_OFF), w.at<int32_t>(B_PERM), w.at<int32_t>(B_INV),
+                       w.at<void>(B_H), w.at<void>(B_X), s));
+  }
+  float *ent = entropy_out ? entropy_out : w.at<float>(B_ENT);
+  int32_t *am = argmax_out ? argmax_out : w.at<int32_t>(B_AM);
+  DG_TRY(lm_entropy(c, w, T, n_rows, w.at<void>(B_X), rows, model->emb, ent, am, logits_dbg, 1,
+                    dev_status, s));
+  return launch_eb_select(batch, C, ent, am, quant_gamma(gamma), max_steps, tokens, masked,
+                          nullptr, n_masked, done, step, dev_status, s);
+}
+
+}  // extern "C"

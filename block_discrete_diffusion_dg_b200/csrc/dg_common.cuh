@@ -1,0 +1,67 @@
+// Shared device helpers of the canvas-step library: element types, the device status word,
+// warp/block reductions and the launch bookkeeping used by every kernel file.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/dg.h"
+
+namespace dg {
+
+using bf16 = __nv_bfloat16;
+using fp8 = __nv_fp8_e4m3;
+
+// ---- element conversion -------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f(fp8 v) { return float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// Round an fp32 value to the storage type and back (what a store/load round trip yields).
+template <typename T> __device__ __forceinline__ float round_to(float v) { return to_f(from_f<T>(v)); }
+
+// ---- device status word ------------------------------------------------------------------
+// First error wins; later errors leave the word alone.
+__device__ __forceinline__ void set_status(int32_t *st, int code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+// ---- reductions ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum in a fixed order (deterministic); `red` needs blockDim.x/32 floats.
+__device__ __forceinline__ float block_sum(float v, float *red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+}  // namespace dg
+
+// ---- host-side launch bookkeeping (defined in dg_api.cu) ----------------------------------
+namespace dg {
+// Counts a kernel launch on stream `s` (and, while profiling is on in this thread, records a
+// timing event on `s` before the launch, labelled `name`).
+void note_launch(cudaStream_t s, const char *name);
+int check_launch(const char *what);      // DG_OK or DG_ERR_CUDA (records the message)
+}  // namespace dg

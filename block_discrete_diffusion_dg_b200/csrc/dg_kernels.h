@@ -1,0 +1,101 @@
+// Internal launchers of the canvas-step library (host functions, one per kernel family).
+// Each returns DG_OK or DG_ERR_CUDA and never synchronises.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dg.h"
+
+namespace dg {
+
+// A tile of a grouped GEMM: rows [m0, m0 + tile) of group `g` (MoE expert).
+struct GroupTile { int32_t g, m0; };
+
+// ---- rows: embedding, RMSNorm, compaction (k_rows.cu) -----------------------------------
+int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, const void *emb,
+                      int rows, int d, int vocab, double eps, void *x_out, void *a_out,
+                      int32_t *st, cudaStream_t s);
+int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
+                   int max_rows, int d, double eps, void *out, cudaStream_t s);
+// live[b*C+i] = !done[b] && (masked == NULL || masked[b*C+i]); row_idx = positions with live
+// set, in order; *n_rows = their count; token_live[t] = !done[b] (may be NULL).
+int launch_compact_rows(int batch, int canvas, const uint8_t *masked, const int32_t *done,
+                        int32_t *row_idx, int32_t *n_rows, uint8_t *token_live, cudaStream_t s);
+
+// ---- GEMM on CUDA cores (k_gemm_simt.cu) --------------------------------------------------
+// C[m][n] = sum_k A[arow(m)][k] * B[g][n][k] (* bscale[g][n]); fp32 accumulation in k order.
+struct GemmDesc {
+  int act, w;                  // element types of A and B (DG_F32 / DG_BF16 / DG_E4M3)
+  const void *A; int lda;
+  const void *B; int ldb; long long strideB;   // group stride of B in elements
+  const float *bscale;         // [groups][N] or NULL
+  int M, N, K;                 // M: rows (max rows if M_dev set)
+  const int32_t *M_dev;        // device row count (<= M) or NULL
+  const int32_t *a_rowmap;     // A row of output row m = a_rowmap[m] / a_rowdiv, or NULL
+  int a_rowdiv;
+  const GroupTile *tiles;      // grouped mode: tile list, count at *n_tiles, max_tiles
+  const int32_t *n_tiles;
+  const int32_t *group_off;    // grouped mode: row offsets [groups + 1]
+  int max_tiles;
+  const char *name;            // label for launch accounting / profiling
+};
+enum EpiKind { EPI_F32 = 0, EPI_ACT = 1, EPI_RESID = 2 };
+// EPI_F32: out fp32 [M][ldo]; EPI_ACT: out act type; EPI_RESID: out = act(acc + res[m][n]).
+int launch_gemm_simt(const GemmDesc &g, int epi, void *out, int ldo, const void *res,
+                     cudaStream_t s);
+
+// ---- RoPE and head split (k_rope.cu) -----------------------------------------------------
+// Positions cache_len[b] + i; cos/sin of angle pos * theta^(-2j/hd) in fp64, stored fp32.
+int launch_rope_table(int batch, int n, int hd, double theta, const int32_t *cache_len,
+                      float *cs, cudaStream_t s);
+// qkv fp32 [B*n][(Hq+2Hkv)hd] -> q [B*n][Hq][hd], k_new/v_new [B][Hkv][n][hd] (act type, RoPE
+// on q and k).  If k_cache != NULL also writes k/v to cache rows cache_len[b] + i (< cap).
+int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const float *qkv,
+                     const float *cs, void *q, void *k_new, void *v_new, void *k_cache,
+                     void *v_cache, const int32_t *cache_len, int cap, int32_t *st,
+                     cudaStream_t s);
+int launch_add_cache_len(int batch, int n, int cap, int32_t *cache_len, cudaStream_t s);
+
+// ---- attention (k_attn.cu) ----------------------------------------------------------------
+int launch_attention(int act, int batch, int n, int Hq, int Hkv, int hd, const void *q,
+                     const void *k_cache, const void *v_cache, const int32_t *cache_len,
+                     int cap, const void *k_new, const void *v_new, int causal,
+                     const int32_t *done, void *out, void *ws, cudaStream_t s);
+size_t attention_ws_bytes(int batch, int n, int Hq, int hd, int cap);
+
+// ---- MoE (k_moe.cu) ---------------------------------------------------------------------------
+int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *y,
+                  const void *w_router, const uint8_t *token_live, int32_t *topk_idx,
+                  float *topk_w, cudaStream_t s);
+// Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
+int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
+                   int32_t *perm, int32_t *inv_perm, cudaStream_t s);
+// Grouped-GEMM tile list from expert_off: tiles of tile_m rows, count at *n_tiles.
+int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *tiles,
+                       int32_t *n_tiles, int max_tiles, cudaStream_t s);
+// Scatter rows: dst[row_idx[r]][:] = src[r][:] for r < *n_rows.
+int launch_scatter_rows(const float *src, int width, int max_rows, const int32_t *n_rows,
+                        const int32_t *row_idx, float *dst, cudaStream_t s);
+// a = act(gelu_tanh(u[:, :F]) * u[:, F:]) for rows < expert_off[E].
+int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *expert_off, int E,
+                void *a, cudaStream_t s);
+// out_t = act(res_t + sum_j w[t][j] Y[inv_perm[t k + j]]).
+int launch_combine(int act, int T, int d, int k, const int32_t *topk_idx, const float *topk_w,
+                   const int32_t *inv_perm, const void *Y, const void *res, void *out,
+                   cudaStream_t s);
+
+// ---- entropy / argmax (k_entropy.cu) -----------------------------------------------------------
+// From materialised fp32 logits [rows][V]: per row r < *n_rows: H and argmax stored at
+// out index row_idx ? row_idx[r] : r.
+int launch_entropy_rows(const float *logits, int V, int max_rows, const int32_t *n_rows,
+                        const int32_t *row_idx, float *entropy, int32_t *argmax, int32_t *st,
+                        cudaStream_t s);
+
+// ---- EB select (k_eb.cu) -------------------------------------------------------------------
+int launch_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
+                     long long q_gamma, int max_steps, int32_t *tokens, uint8_t *masked,
+                     uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
+                     int32_t *st, cudaStream_t s);
+
+}  // namespace dg

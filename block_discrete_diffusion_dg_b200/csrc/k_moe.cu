@@ -1,0 +1,259 @@
+// Mixture-of-experts routing and the element-wise parts of the expert FFN.
+// Model card "diffusiongemma", "Mixture-of-Experts (MoE) Efficiency": 8 of 128 experts active per
+// token; "DiffusionGemma Technical Report", Table 1: 8 / 128 experts.
+//
+// Router: z = y W_r^T in fp32 (fixed k order), p = softmax(z) over all E; the k largest p with the
+// lower expert index first among equal values; gates renormalised to sum 1 — computed as a softmax
+// over the selected logits, which is the same quantity.
+// Permutation: assignments (t, j) grouped by expert, stable in flat order t k + j; expert_off is the
+// exclusive prefix of the per-expert counts; the grouped GEMMs read a tile list built here.
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+
+namespace {
+
+constexpr int ROUTER_TPB = 4;  // tokens per router block
+
+template <typename T, typename WT>
+__global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__ y,
+                              const WT *__restrict__ wr, const uint8_t *__restrict__ token_live,
+                              int32_t *topk_idx, float *topk_w) {
+  extern __shared__ float sm[];
+  float *ys = sm;                        // [TPB][d]
+  float *zs = sm + ROUTER_TPB * d;       // [TPB][E]
+  const int t0 = blockIdx.x * ROUTER_TPB;
+  for (int e = threadIdx.x; e < ROUTER_TPB * d; e += blockDim.x) {
+    const int tt = e / d, c = e % d;
+    ys[e] = (t0 + tt < T_) ? to_f(y[(size_t)(t0 + tt) * d + c]) : 0.f;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const WT *w = wr + (size_t)e * d;
+    float acc[ROUTER_TPB];
+#pragma unroll
+    for (int tt = 0; tt < ROUTER_TPB; ++tt) acc[tt] = 0.f;
+    for (int c = 0; c < d; ++c) {
+      const float wv = to_f(w[c]);
+#pragma unroll
+      for (int tt = 0; tt < ROUTER_TPB; ++tt) acc[tt] = fmaf(ys[tt * d + c], wv, acc[tt]);
+    }
+#pragma unroll
+    for (int tt = 0; tt < ROUTER_TPB; ++tt) zs[tt * E + e] = acc[tt];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int tt = warp; tt < ROUTER_TPB; tt += blockDim.x >> 5) {
+    const int t = t0 + tt;
+    if (t >= T_) continue;
+    const bool live = token_live == nullptr || token_live[t] != 0;
+    const float *z = zs + tt * E;
+    float zsel0 = 0.f, denom = 0.f;
+    // selected set as a bitmask over the lane's experts e = lane + 32 i (E <= 256)
+    unsigned taken = 0u;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int i = 0, e = lane; e < E; ++i, e += 32) {
+        if (taken & (1u << i)) continue;
+        const float v = z[e];
+        if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (j == 0) zsel0 = bv;
+      const float p = expf(bv - zsel0);
+      denom += p;
+      if (lane == 0) {
+        topk_idx[(size_t)t * k + j] = live ? bi : -1;
+        topk_w[(size_t)t * k + j] = p;  // normalised below
+      }
+    }
+    __syncwarp();
+    if (lane < k) topk_w[(size_t)t * k + lane] = live ? topk_w[(size_t)t * k + lane] / denom : 0.f;
+  }
+}
+
+// Single block of 1024 threads; E <= 256.
+__global__ void __launch_bounds__(1024) permute_kernel(int n_assign, int E,
+                                                       const int32_t *__restrict__ topk_idx,
+                                                       int32_t *expert_off, int32_t *perm,
+                                                       int32_t *inv_perm) {
+  __shared__ int cnt[256], off[257], running[256];
+  __shared__ int wc[32][256];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) { cnt[e] = 0; running[e] = 0; }
+  __syncthreads();
+  for (int a = tid; a < n_assign; a += blockDim.x) {
+    const int e = topk_idx[a];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) { off[e] = acc; acc += cnt[e]; }
+    off[E] = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) expert_off[e] = off[e];
+  for (int c0 = 0; c0 < n_assign; c0 += blockDim.x) {
+    for (int i = tid; i < 32 * E; i += blockDim.x) wc[i / E][i % E] = 0;
+    __syncthreads();
+    const int a = c0 + tid;
+    int e = -1;
+    if (a < n_assign) {
+      e = topk_idx[a];
+      if (e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank == 0) wc[w][e] = __popc(peers);
+    __syncthreads();
+    if (e >= 0) {
+      int before = 0;
+      for (int ww = 0; ww < w; ++ww) before += wc[ww][e];
+      const int pos = off[e] + running[e] + before + rank;
+      perm[pos] = a;
+      inv_perm[a] = pos;
+    } else if (a < n_assign) {
+      inv_perm[a] = -1;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int t = 0;
+      for (int ww = 0; ww < 32; ++ww) t += wc[ww][ee];
+      running[ee] += t;
+    }
+    __syncthreads();
+  }
+}
+
+// Tile list of the grouped expert GEMMs: for each expert with rows, tiles of tile_m rows.
+__global__ void build_tiles_kernel(int E, const int32_t *__restrict__ expert_off, int tile_m,
+                                   GroupTile *tiles, int32_t *n_tiles, int max_tiles) {
+  __shared__ int toff[257];
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      toff[e] = acc;
+      acc += (expert_off[e + 1] - expert_off[e] + tile_m - 1) / tile_m;
+    }
+    toff[E] = acc;
+    *n_tiles = min(acc, max_tiles);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int nt = toff[e + 1] - toff[e];
+    for (int i = 0; i < nt; ++i) {
+      const int slot = toff[e] + i;
+      if (slot < max_tiles) tiles[slot] = GroupTile{e, i * tile_m};
+    }
+  }
+}
+
+template <typename T>
+__global__ void gate_kernel(int F, const float *__restrict__ u, const int32_t *__restrict__ expert_off,
+                            int E, T *a) {
+  const int p = blockIdx.x;
+  if (p >= expert_off[E]) return;
+  const float *ur = u + (size_t)p * 2 * F;
+  T *ar = a + (size_t)p * F;
+  for (int f = threadIdx.x; f < F; f += blockDim.x) {
+    const float g = ur[f], up = ur[F + f];
+    const float gl = 0.5f * g * (1.0f + tanhf(0.7978845608028654f * (g + 0.044715f * g * g * g)));
+    ar[f] = from_f<T>(gl * up);
+  }
+}
+
+template <typename T>
+__global__ void combine_kernel(int d, int k, const int32_t *__restrict__ topk_idx,
+                               const float *__restrict__ topk_w, const int32_t *__restrict__ inv_perm,
+                               const T *__restrict__ Y, const T *__restrict__ res, T *out) {
+  const int t = blockIdx.x;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float acc = to_f(res[(size_t)t * d + c]);
+    for (int j = 0; j < k; ++j) {
+      const int a = t * k + j;
+      if (topk_idx[a] < 0) continue;
+      acc = fmaf(topk_w[a], to_f(Y[(size_t)inv_perm[a] * d + c]), acc);
+    }
+    out[(size_t)t * d + c] = from_f<T>(acc);
+  }
+}
+
+}  // namespace
+
+int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void *y,
+                  const void *w_router, const uint8_t *token_live, int32_t *topk_idx,
+                  float *topk_w, cudaStream_t s) {
+  if (T_ <= 0) return DG_OK;
+  const int threads = E < 32 ? 32 : (E > 256 ? 256 : ((E + 31) / 32) * 32);
+  const size_t smem = sizeof(float) * ROUTER_TPB * (size_t)(d + E);
+  const int grid = (T_ + ROUTER_TPB - 1) / ROUTER_TPB;
+  if (act == DG_F32 && wr_type == DG_F32) {
+    auto kf = router_kernel<float, float>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    note_launch(s, "router");
+    kf<<<grid, threads, smem, s>>>(T_, d, E, k, (const float *)y, (const float *)w_router,
+                                   token_live, topk_idx, topk_w);
+  } else if (act == DG_BF16 && wr_type == DG_BF16) {
+    auto kb = router_kernel<bf16, bf16>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    note_launch(s, "router");
+    kb<<<grid, threads, smem, s>>>(T_, d, E, k, (const bf16 *)y, (const bf16 *)w_router,
+                                   token_live, topk_idx, topk_w);
+  } else {
+    return DG_ERR_UNSUPPORTED;
+  }
+  return check_launch("router");
+}
+
+int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
+                   int32_t *perm, int32_t *inv_perm, cudaStream_t s) {
+  if (E > 256) return DG_ERR_UNSUPPORTED;
+  note_launch(s, "permute");
+  permute_kernel<<<1, 1024, 0, s>>>(T_ * k, E, topk_idx, expert_off, perm, inv_perm);
+  return check_launch("permute");
+}
+
+int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *tiles,
+                       int32_t *n_tiles, int max_tiles, cudaStream_t s) {
+  if (E > 256) return DG_ERR_UNSUPPORTED;
+  note_launch(s, "build_tiles");
+  build_tiles_kernel<<<1, 256, 0, s>>>(E, expert_off, tile_m, tiles, n_tiles, max_tiles);
+  return check_launch("build_tiles");
+}
+
+int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *expert_off, int E,
+                void *a, cudaStream_t s) {
+  if (rows_max <= 0) return DG_OK;
+  note_launch(s, "gate");
+  if (act == DG_F32)
+    gate_kernel<float><<<rows_max, 128, 0, s>>>(F, u, expert_off, E, (float *)a);
+  else
+    gate_kernel<bf16><<<rows_max, 128, 0, s>>>(F, u, expert_off, E, (bf16 *)a);
+  return check_launch("gate");
+}
+
+int launch_combine(int act, int T_, int d, int k, const int32_t *topk_idx, const float *topk_w,
+                   const int32_t *inv_perm, const void *Y, const void *res, void *out,
+                   cudaStream_t s) {
+  if (T_ <= 0) return DG_OK;
+  note_launch(s, "combine");
+  if (act == DG_F32)
+    combine_kernel<float><<<T_, 256, 0, s>>>(d, k, topk_idx, topk_w, inv_perm, (const float *)Y,
+                                             (const float *)res, (float *)out);
+  else
+    combine_kernel<bf16><<<T_, 256, 0, s>>>(d, k, topk_idx, topk_w, inv_perm, (const bf16 *)Y,
+                                            (const bf16 *)res, (bf16 *)out);
+  return check_launch("combine");
+}
+
+}  // namespace dg

@@ -1,0 +1,137 @@
+// Row kernels: embedding gather + pre-norm, RMSNorm (optionally over a gathered row list), and
+// the compaction of the positions that need logits this step.
+//
+// RMSNorm(x) = x / sqrt(mean(x^2) + eps), unit gain, computed in fp32 with a fixed-order
+// reduction and rounded once to the activation type (the pre-norm of every layer and the
+// final norm before the LM head; the pages' model is the Gemma 4 transformer,
+// "DiffusionGemma Technical Report", What they did).
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+
+template <typename T>
+__global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t *__restrict__ tokens,
+                                                         const uint8_t *__restrict__ masked,
+                                                         const T *__restrict__ emb, int d,
+                                                         int vocab, float eps, T *x_out, T *a_out,
+                                                         int32_t *st) {
+  __shared__ float red[8];
+  const int row = blockIdx.x;
+  int id = (masked && masked[row]) ? vocab : tokens[row];
+  if (id < 0 || id > vocab) {  // out-of-range id: report, embed as MASK
+    if (threadIdx.x == 0) set_status(st, DG_ERR_INVALID_ARG);
+    id = vocab;
+  }
+  const T *src = emb + (size_t)id * d;
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float v = to_f(src[j]);
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  T *xo = x_out + (size_t)row * d;
+  T *ao = a_out + (size_t)row * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    T v = src[j];
+    xo[j] = v;
+    ao[j] = from_f<T>(to_f(v) * inv);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T *__restrict__ in,
+                                                      const int32_t *__restrict__ row_idx,
+                                                      const int32_t *__restrict__ n_rows_dev,
+                                                      int d, float eps, T *out) {
+  __shared__ float red[8];
+  const int r = blockIdx.x;
+  if (n_rows_dev && r >= *n_rows_dev) return;
+  const int src_row = row_idx ? row_idx[r] : r;
+  const T *src = in + (size_t)src_row * d;
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float v = to_f(src[j]);
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  T *o = out + (size_t)r * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f<T>(to_f(src[j]) * inv);
+}
+
+// One block of 1024 threads scans all B*C positions in chunks (B*C <= 65536).
+__global__ void __launch_bounds__(1024) compact_rows_kernel(int batch, int canvas,
+                                                            const uint8_t *__restrict__ masked,
+                                                            const int32_t *__restrict__ done,
+                                                            int32_t *row_idx, int32_t *n_rows,
+                                                            uint8_t *token_live) {
+  __shared__ int warp_tot[32];
+  __shared__ int base;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  const int total = batch * canvas;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int c0 = 0; c0 < total; c0 += blockDim.x) {
+    const int p = c0 + threadIdx.x;
+    int live = 0;
+    if (p < total) {
+      const int b = p / canvas;
+      const int alive = done ? (done[b] == 0) : 1;
+      if (token_live) token_live[p] = (uint8_t)alive;
+      live = alive && (masked == nullptr || masked[p] != 0);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, live);
+    if (lane == 0) warp_tot[w] = __popc(bal);
+    __syncthreads();
+    int before = 0;
+    for (int i = 0; i < w; ++i) before += warp_tot[i];
+    const int pos = base + before + __popc(bal & ((1u << lane) - 1u));
+    if (live) row_idx[pos] = p;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int i = 0; i < 32; ++i) t += warp_tot[i];
+      base += t;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *n_rows = base;
+}
+
+int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, const void *emb,
+                      int rows, int d, int vocab, double eps, void *x_out, void *a_out,
+                      int32_t *st, cudaStream_t s) {
+  if (rows <= 0) return DG_OK;
+  note_launch(s, "embed_norm");
+  if (act == DG_F32)
+    embed_norm_kernel<float><<<rows, 256, 0, s>>>(tokens, masked, (const float *)emb, d, vocab,
+                                                  (float)eps, (float *)x_out, (float *)a_out, st);
+  else
+    embed_norm_kernel<bf16><<<rows, 256, 0, s>>>(tokens, masked, (const bf16 *)emb, d, vocab,
+                                                 (float)eps, (bf16 *)x_out, (bf16 *)a_out, st);
+  return check_launch("embed_norm");
+}
+
+int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
+                   int max_rows, int d, double eps, void *out, cudaStream_t s) {
+  if (max_rows <= 0) return DG_OK;
+  note_launch(s, "rmsnorm");
+  if (act == DG_F32)
+    rmsnorm_kernel<float><<<max_rows, 256, 0, s>>>((const float *)in, row_idx, n_rows_dev, d,
+                                                   (float)eps, (float *)out);
+  else
+    rmsnorm_kernel<bf16><<<max_rows, 256, 0, s>>>((const bf16 *)in, row_idx, n_rows_dev, d,
+                                                  (float)eps, (bf16 *)out);
+  return check_launch("rmsnorm");
+}
+
+int launch_compact_rows(int batch, int canvas, const uint8_t *masked, const int32_t *done,
+                        int32_t *row_idx, int32_t *n_rows, uint8_t *token_live, cudaStream_t s) {
+  note_launch(s, "compact_rows");
+  compact_rows_kernel<<<1, 1024, 0, s>>>(batch, canvas, masked, done, row_idx, n_rows, token_live);
+  return check_launch("compact_rows");
+}
+
+}  // namespace dg

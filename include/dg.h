@@ -1,0 +1,231 @@
+/*
+ * dg.h — C ABI of the canvas-step library (block-wise discrete diffusion, sm_100a).
+ *
+ * One denoising step of block-wise discrete-diffusion decoding, as the pages describe it:
+ *   "DiffusionGemma Technical Report" (metalmedia.ai), Figure 4: a prompt is encoded
+ *   causally into a KV cache; the decoder refines a canvas with bidirectional attention over
+ *   the canvas and cross-attention to the cache; the finished canvas is re-encoded causally and
+ *   appended to the cache.  Same page, explanatory visual ("Inference: block-wise diffusion
+ *   decoding"): an entropy-bounded sampler with adaptive stopping finishes a 256-token block in
+ *   a few steps.  Model card "diffusiongemma" (axforge.ai), "Model Overview" and
+ *   "Mixture-of-Experts (MoE) Efficiency": encoder-decoder, 8 of 128 experts active.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library never allocates,
+ *     frees or keeps them.  Structs (dg_config, dg_model, dg_layer_weights) are HOST memory
+ *     read during the call only.
+ *   - Scratch memory is a caller-provided device buffer `ws` of at least the size that
+ *     dg_workspace_size() returns for the same (cfg, batch, n_tokens, cache_cap); 256-byte
+ *     aligned.  Contents need not be initialised and are clobbered.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*) and does not
+ *     synchronise.  The return value reports host-detectable problems (bad arguments, launch
+ *     failure) before or at launch; nothing is launched when an argument is rejected.
+ *   - Problems only the device can see (a non-finite entropy, a token id out of range, a full
+ *     KV cache) are recorded in the caller's device word `dev_status` (int32, first error
+ *     wins) and the affected work is skipped; read it with dg_read_status().  `dev_status`
+ *     may be NULL, in which case such problems are not reported.
+ *   - Layouts are row-major with the LAST index contiguous.  B = batch (independent canvases),
+ *     C = cfg->canvas, d = cfg->d_model, Hq/Hkv = query/kv heads, hd = head_dim, E = experts,
+ *     k = top_k, F = d_ff, V = vocab.  Activation element type = cfg->act_dtype (F32 or BF16);
+ *     layer-weight element type = cfg->w_dtype (F32, BF16, or E4M3 with one fp32 scale per
+ *     output channel).  The K/V cache of one layer is [B][Hkv][cache_cap][hd], the full cache
+ *     [L][B][Hkv][cache_cap][hd], both in the activation type.
+ *   - Functions are stateless and may be called from several host threads on different streams.
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------------- */
+enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,  /* bad pointer, size, or combination of arguments               */
+  DG_ERR_UNSUPPORTED = 2,  /* a shape or dtype combination this build has no kernel for     */
+  DG_ERR_CAPACITY = 3,     /* KV-cache rows would exceed cache_cap (device-detected)        */
+  DG_ERR_CUDA = 4,         /* a CUDA call or launch failed; see dg_last_cuda_error()         */
+  DG_ERR_NUMERIC = 5,      /* a non-finite logit or entropy was seen (device-detected)       */
+  DG_ERR_TIMEOUT = 6,      /* a bounded device-side wait expired (device-detected)           */
+  DG_ERR_WORKSPACE = 7     /* ws_bytes smaller than dg_workspace_size()                      */
+};
+
+enum { DG_F32 = 0, DG_BF16 = 1, DG_E4M3 = 2 };
+
+/* Model shape.  The MASK token id is `vocab` (one extra embedding row); the LM head covers
+ * ids [0, vocab), so argmax never returns MASK.  rope_theta: rotary base; rms_eps: RMSNorm eps. */
+typedef struct dg_config {
+  int32_t d_model, n_q_heads, n_kv_heads, head_dim;
+  int32_t n_experts, top_k, d_ff;
+  int32_t vocab, canvas, n_layers;
+  double rope_theta, rms_eps;
+  int32_t act_dtype; /* DG_F32 or DG_BF16 */
+  int32_t w_dtype;   /* DG_F32 (with act F32), DG_BF16 or DG_E4M3 (with act BF16) */
+} dg_config;
+
+/* One layer's weights (device pointers).  Every matrix is [out][in], `in` contiguous.
+ *   w_qkv     [(Hq + 2 Hkv) hd][d]   rows: q heads, then k heads, then v heads
+ *   w_o       [d][Hq hd]
+ *   w_router  [E][d]                 BF16 (F32 when w_dtype is F32), never E4M3
+ *   w_gate_up [E][2F][d]             rows [0,F) gate, [F,2F) up
+ *   w_down    [E][d][F]
+ * s_* : fp32 per-output-channel scales, required for E4M3 and ignored otherwise. */
+typedef struct dg_layer_weights {
+  const void *w_qkv;     const float *s_qkv;
+  const void *w_o;       const float *s_o;
+  const void *w_router;
+  const void *w_gate_up; const float *s_gate_up;
+  const void *w_down;    const float *s_down;
+} dg_layer_weights;
+
+/* A whole model: `layers` is a HOST array of n_layers structs; `emb` the tied embedding /
+ * LM head [V + 1][d] in the activation type (row V = MASK; rows [0,V) = LM head). */
+typedef struct dg_model {
+  const dg_layer_weights *layers;
+  const void *emb;
+} dg_model;
+
+/* ---- sizes and status ------------------------------------------------------------------ */
+
+/* Bytes of scratch the calls below need for `batch` canvases of `n_tokens` tokens each and a
+ * cache of `cache_cap` rows per (layer, batch, kv head).  0 on an invalid config. */
+size_t dg_workspace_size(const dg_config *cfg, int batch, int n_tokens, int cache_cap);
+
+/* Synchronises `stream`, copies *dev_status to the host and returns it (DG_ERR_CUDA if the
+ * copy fails).  Does not clear it; dg_clear_status() zeroes it asynchronously. */
+int dg_read_status(const int32_t *dev_status, void *stream);
+int dg_clear_status(int32_t *dev_status, void *stream);
+
+/* Last CUDA error string seen by this thread's calls (static storage, never NULL). */
+const char *dg_last_cuda_error(void);
+
+/* Number of kernels this process has launched through the library (monotone counter). */
+uint64_t dg_launch_count(void);
+
+/* Profiling aid (host side, per calling thread): after dg_profile_begin(max_records) every
+ * kernel launch of the library first records a CUDA timing event on its stream (up to
+ * max_records).  dg_profile_mark(stream) records a closing event labelled "(mark)".
+ * dg_profile_end synchronises on the last event, writes ms[i] = time from record i to record
+ * i + 1 (i < *n_out <= max_out) and stops recording; dg_profile_name(i) is record i's kernel
+ * name ("" when out of range).  Events are created once and reused; no device memory is
+ * allocated.  Not for use inside CUDA graph capture. */
+int dg_profile_begin(int max_records);
+int dg_profile_mark(void *stream);
+int dg_profile_end(float *ms, int max_out, int *n_out);
+const char *dg_profile_name(int i);
+
+/* ---- the hot-path operations ------------------------------------------------------------ */
+
+/* Canvas attention, "DiffusionGemma Technical Report", Figure 4 (bidirectional attention
+ * across the canvas, cross-attention to the KV cache) and the model card's "Model Overview".
+ * For canvas b, query token i, query head h (kv head g = h / (Hq/Hkv)):
+ *   o = softmax(q K^T / sqrt(hd)) V over keys = cache rows [0, cache_len[b]) followed by the
+ *   n_tokens new rows; causal = 0: every new key visible (decoder); causal = 1: new key j
+ *   visible iff j <= i (causal encoder, used by the append).  Cache rows are all visible.
+ *   q      [B][n_tokens][Hq][hd]        k_cache, v_cache [B][Hkv][cache_cap][hd] (one layer)
+ *   k_new, v_new [B][Hkv][n_tokens][hd] out [B][n_tokens][Hq][hd]
+ *   cache_len: device int32[B], each <= cache_cap.  done: device int32[B] or NULL; canvases
+ *   with done[b] != 0 are skipped (their `out` rows are left as they were). */
+int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
+                   const void *k_cache, const void *v_cache, const int32_t *cache_len,
+                   int cache_cap, const void *k_new, const void *v_new, int causal,
+                   const int32_t *done, void *out, void *ws, size_t ws_bytes,
+                   int32_t *dev_status, void *stream);
+
+/* Router top-k and token permutation, model card "diffusiongemma", "Mixture-of-Experts (MoE)
+ * Efficiency" (8 active of 128) and "DiffusionGemma Technical Report", Table 1.
+ * z = y W_r^T (fp32), p = softmax(z) over all E, the k largest p (lower expert index first on
+ * equal values), renormalised to sum 1.  Then assignments (t, j) are grouped by expert,
+ * stable in (t, j) order:
+ *   y [T][d]; topk_idx int32 [T][k]; topk_w fp32 [T][k]; expert_off int32 [E + 1]
+ *   (exclusive prefix of per-expert counts); perm int32 [T k]: perm[p] = t k + j of the
+ *   assignment at permuted position p; inv_perm int32 [T k]: the inverse.
+ *   token_live: device uint8 [T] or NULL; a token with token_live[t] == 0 gets no experts
+ *   (topk_idx = -1, weight 0) and no assignments. */
+int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *w_router,
+                 const uint8_t *token_live, int32_t *topk_idx, float *topk_w,
+                 int32_t *expert_off, int32_t *perm, int32_t *inv_perm, void *ws,
+                 size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* Expert FFN with combine and residual (same passages).  For assignment (t, j) with expert e:
+ *   [g; u] = y_t W_gu,e^T ; a = gelu_tanh(g) * u (stored in the activation type) ;
+ *   Y = a W_d,e^T (stored in the activation type) ;
+ *   out_t = residual_t + sum_j topk_w[t][j] Y_(t,j), summed in fp32 in slot order j = 0..k-1.
+ * Routing arrays as produced by dg_moe_route.  y, residual, out [T][d] (out may not alias y;
+ * it may alias residual). */
+int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t *topk_idx,
+               const float *topk_w, const int32_t *expert_off, const int32_t *perm,
+               const int32_t *inv_perm, const dg_layer_weights *lw, const void *residual,
+               void *out, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* Final RMSNorm, LM head and fused softmax entropy / greedy argmax, per masked position
+ * ("DiffusionGemma Technical Report", explanatory visual: the entropy-bounded sampler consumes
+ * per-position confidence; Table 1: vocabulary 262k; model card, Benchmark Results: EB sampler).
+ * For r < n_rows (or < *n_rows_dev when that pointer is non-NULL), with source row
+ * s = row_idx ? row_idx[r] : r:
+ *   f = RMSNorm(h_s) (stored in the activation type);  z = f W_lm^T over ids [0, V) (fp32);
+ *   entropy[s] = -sum_v p_v ln p_v with p = softmax(z);  argmax[s] = first index of max z.
+ *   h [*][d]; w_lm = the embedding [V + 1][d] (rows [0, V) used); entropy fp32, argmax int32
+ *   indexed by source row; logits_dbg fp32 [n_rows][V] or NULL (written when non-NULL).
+ * A non-finite logit sets DG_ERR_NUMERIC. */
+int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_dev,
+                      const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
+                      int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
+                      int32_t *dev_status, void *stream);
+
+/* Entropy-bounded selection and commit (model card "diffusiongemma", Benchmark Results: the
+ * EB sampler; "DiffusionGemma Technical Report", What they did: adaptive stopping).  The
+ * pages name the sampler but print no formula; the rule is the published EB sampler
+ * (Ben-Hamu et al., 2025): for each canvas b with done[b] == 0, order its masked positions by
+ * entropy ascending (negative values and -0 as 0; lower position first on ties) and commit the
+ * first k for the largest k >= 1 with  sum_{i<k} Q(H_(i)) <= Q(gamma), where
+ * Q(H) = nearest integer to H * 2^32 (ties to even) and Q(gamma) = floor(gamma * 2^32)
+ * (+inf: no bound).  When step[b] >= max_steps - 1 every masked position is committed.
+ * Commit: tokens[b][i] = argmax[b][i], masked[b][i] = 0, selected[b][i] = 1.  Then
+ * n_masked[b] -= k, step[b] += 1, done[b] = (n_masked[b] == 0).
+ *   entropy fp32 [B][C] and argmax int32 [B][C] are read at masked positions only;
+ *   tokens int32, masked uint8, selected uint8 (or NULL) [B][C]; n_masked, done, step int32 [B].
+ * canvas <= 1024, gamma >= 0.  A non-finite entropy at a masked position sets DG_ERR_NUMERIC
+ * and leaves that canvas unchanged. */
+int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
+                 double gamma, int max_steps, int32_t *tokens, uint8_t *masked,
+                 uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
+                 int32_t *dev_status, void *stream);
+
+/* Encode & append ("DiffusionGemma Technical Report", Figure 4, stage 3; model card,
+ * "Model Overview"): run the causal encoder (the decoder's weights, causal within the new
+ * tokens, full visibility of the cache) over tokens [B][n_tokens] (device int32, ids in
+ * [0, V]) at positions cache_len[b] + i, write every layer's K/V (after RoPE) into cache rows
+ * [cache_len[b], cache_len[b] + n_tokens), then cache_len[b] += n_tokens.  Also used to
+ * prefill a prompt in chunks.  k_cache, v_cache: [L][B][Hkv][cache_cap][hd].  A canvas whose
+ * rows would pass cache_cap is left unchanged and sets DG_ERR_CAPACITY. */
+int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
+                 int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
+                 void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* One denoising step of every live canvas ("DiffusionGemma Technical Report", Figure 4,
+ * stage 2 and the explanatory visual): embed the canvas (masked positions as MASK = V), run
+ * the n_layers decoder layers (pre-norm RMSNorm; GQA attention with RoPE at absolute positions
+ * cache_len[b] + i over the cache plus the canvas, bidirectional; output projection + residual;
+ * RMSNorm; top-k MoE FFN + residual), then for the masked positions the final RMSNorm, LM head
+ * entropy / argmax and the EB select-and-commit of dg_eb_select.  Canvases with done[b] != 0
+ * are left unchanged.  State arrays as in dg_eb_select.  k_cache, v_cache
+ * [L][B][Hkv][cache_cap][hd] are read only (the canvas's own K/V live in `ws`).
+ * entropy_out fp32 [B][C], argmax_out int32 [B][C] (or NULL): written at the positions that
+ * were masked when the step began.  logits_dbg (or NULL): fp32 [B C][V], row b C + i written for
+ * each such position (debug and parity only; costs a full logits write). */
+int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
+                   uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
+                   int max_steps, double gamma, const void *k_cache, const void *v_cache,
+                   const int32_t *cache_len, int cache_cap, float *entropy_out,
+                   int32_t *argmax_out, float *logits_dbg, void *ws, size_t ws_bytes,
+                   int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H */

@@ -196,11 +196,14 @@ def moe_ffn(y: np.ndarray, idx: np.ndarray, gates: np.ndarray, expert_w, residua
       a      = gelu_tanh(g) * u                 (stored: rounded)
       Y      = a W_d,e^T                        (stored: rounded)
     out_t = residual_t + sum_j gates[t, j] Y_{t,j}          (stored: rounded)
-    ``expert_w(e)`` returns (W_gu,e [2F, d], W_d,e [d, F]) as fp64.
+    ``expert_w(e)`` returns (W_gu,e [2F, d], W_d,e [d, F]) as fp64.  A slot whose expert id is
+    negative has no expert and contributes nothing.
     """
     T, k = idx.shape
     acc = np.array(residual, dtype=np.float64, copy=True)
     for e in np.unique(idx):
+        if e < 0:
+            continue
         rows, slots = np.nonzero(idx == e)
         w_gu, w_d = expert_w(int(e))
         F = w_d.shape[1]

@@ -462,3 +462,17 @@ def test_tiny_layer_residual_wiring(tiny):
     assert not np.array_equal(xa, model.emb_rows(toks))
     xc = O.canvas_forward(cfg, model, toks, masked, kc * 3.0 + 1.0, vc * -2.0, cfg.prompt_len)
     assert np.abs(xc - O.canvas_forward(cfg, model, toks, masked, kc, vc, cfg.prompt_len)).max() > 1e-6
+
+
+def test_moe_negative_expert_slot_contributes_nothing():
+    T, d, F, E = 6, 8, 5, 4
+    y = rng.standard_normal((T, d))
+    res = rng.standard_normal((T, d))
+    ws = _experts(E, F, d)
+    idx, g, _ = O.router_topk(y, rng.standard_normal((E, d)), 2)
+    full = O.moe_ffn(y, idx, g, lambda e: ws[e], res, "f32")
+    idx1 = idx.copy(); idx1[:, 1] = -1
+    part = O.moe_ffn(y, idx1, g, lambda e: ws[e], res, "f32")
+    only0 = O.moe_ffn(y, idx[:, :1], g[:, :1], lambda e: ws[e], res, "f32")
+    np.testing.assert_allclose(part, only0, atol=1e-13)
+    assert not np.allclose(part, full)
