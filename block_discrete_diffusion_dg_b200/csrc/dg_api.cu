@@ -49,8 +49,8 @@ inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
-  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_LIVE, B_ROWS, B_NROWS, B_FIN, B_LOGITS, B_ENT, B_AM,
-  B_ATTN, B_COUNT
+  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_LIVE, B_ROWS, B_NROWS, B_FIN, B_LOGITS, B_PART,
+  B_ENT, B_AM, B_ATTN, B_COUNT
 };
 
 struct Layout {
@@ -67,14 +67,15 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   Layout L;
   L.max_tiles = (int)((TK + TILE_M - 1) / TILE_M) + c.n_experts;
   size_t sz[B_COUNT];
+  const size_t T128 = (T + 127) / 128 * 128;  // tensor-core A operands read whole 128-row tiles
   sz[B_X] = T * d * a;
-  sz[B_A] = T * d * a;
+  sz[B_A] = T128 * d * a;
   sz[B_QKV] = T * qkvw * 4;
   sz[B_CS] = T * hd * 4;
   sz[B_Q] = T * c.n_q_heads * hd * a;
   sz[B_KN] = T * c.n_kv_heads * hd * a;
   sz[B_VN] = T * c.n_kv_heads * hd * a;
-  sz[B_O] = T * c.n_q_heads * hd * a;
+  sz[B_O] = T128 * c.n_q_heads * hd * a;
   sz[B_H] = T * d * a;
   sz[B_Y] = T * d * a;
   sz[B_IDX] = TK * 4;
@@ -87,14 +88,18 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_U] = TK * 2 * F * 4;
   sz[B_ACT] = TK * F * a;
   sz[B_YE] = TK * d * a;
+  sz[B_XP] = TK * d * a;
   sz[B_LIVE] = T;
   sz[B_ROWS] = T * 4;
   sz[B_NROWS] = 4;
-  sz[B_FIN] = T * d * a;
-  sz[B_LOGITS] = T * (size_t)c.vocab * 4;
+  const bool tc_lm = lmhead_tc_supported(c.act_dtype, c.d_model);
+  sz[B_FIN] = T128 * d * a;
+  sz[B_LOGITS] = tc_lm ? 0 : T * (size_t)c.vocab * 4;
+  sz[B_PART] = tc_lm ? lmhead_tc_ws_bytes((int)T, c.vocab) : 0;
   sz[B_ENT] = T * 4;
   sz[B_AM] = T * 4;
-  sz[B_ATTN] = attention_ws_bytes(batch, n, c.n_q_heads, c.head_dim, cap);
+  sz[B_ATTN] = attention_ws_bytes(c.act_dtype, batch, n, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                                  cap);
   size_t o = 0;
   for (int i = 0; i < B_COUNT; ++i) {
     L.off[i] = o;
@@ -155,6 +160,9 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
   g.bscale = scale_or_null(&c, w.s_qkv);
   g.M = T; g.N = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim; g.K = c.d_model;
   g.name = "gemm_qkv";
+  if (gemm_tc_supported(c.act_dtype, c.w_dtype, c.d_model))
+    return launch_gemm_tc_dense(ws.at<void>(B_A), T, w.w_qkv, g.N, c.d_model, ws.at<float>(B_QKV),
+                                nullptr, nullptr, g.N, "gemm_qkv_tc", nullptr, s);
   return launch_gemm_simt(g, EPI_F32, ws.at<void>(B_QKV), g.N, nullptr, s);
 }
 
@@ -169,7 +177,11 @@ int attn_out_and_moe(const dg_config &c, const dg_layer_weights &w, const Ws &ws
   g.bscale = scale_or_null(&c, w.s_o);
   g.M = T; g.N = d; g.K = hq;
   g.name = "gemm_o_resid";
-  DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
+  if (gemm_tc_supported(c.act_dtype, c.w_dtype, hq))
+    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, w.w_o, d, hq, nullptr, ws.at<void>(B_H),
+                                ws.at<void>(B_X), d, "gemm_o_resid_tc", nullptr, s));
+  else
+    DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
   DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
                         ws.at<void>(B_Y), s));
   DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
@@ -188,6 +200,20 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
   const int TK = T * k;
   DG_TRY(launch_build_tiles(E, expert_off, TILE_M, ws.at<GroupTile>(B_TILES),
                             ws.at<int32_t>(B_NTILES), ws.L->max_tiles, s));
+  if (gemm_tc_supported(c.act_dtype, c.w_dtype, d) && F % 64 == 0 && d % 128 == 0 &&
+      experts_tc_tile_tokens() == TILE_M) {
+    DG_TRY(launch_gather_rows(TK, d, k, perm, expert_off, E, y, ws.at<void>(B_XP), s));
+    DG_TRY(launch_gemm_tc_experts(1, w.w_gate_up, E, 2 * F, F, ws.at<void>(B_XP), TK, d,
+                                  ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
+                                  ws.L->max_tiles, expert_off, ws.at<void>(B_ACT), F,
+                                  "moe_gate_up_tc", nullptr, s));
+    DG_TRY(launch_gemm_tc_experts(0, w.w_down, E, d, F, ws.at<void>(B_ACT), TK, F,
+                                  ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
+                                  ws.L->max_tiles, expert_off, ws.at<void>(B_YE), d,
+                                  "moe_down_tc", nullptr, s));
+    return launch_combine(c.act_dtype, T, d, k, topk_idx, topk_w, inv_perm, ws.at<void>(B_YE),
+                          residual, out, s);
+  }
   GemmDesc g1{};
   g1.act = c.act_dtype; g1.w = c.w_dtype;
   g1.A = y; g1.lda = d; g1.a_rowmap = perm; g1.a_rowdiv = k;
@@ -220,6 +246,10 @@ int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_
                cudaStream_t s) {
   DG_TRY(launch_rmsnorm(c.act_dtype, h, row_idx, n_rows_dev, max_rows, c.d_model, c.rms_eps,
                         ws.at<void>(B_FIN), s));
+  if (lmhead_tc_supported(c.act_dtype, c.d_model))
+    return launch_lmhead_tc(ws.at<void>(B_FIN), max_rows, n_rows_dev, w_lm, c.vocab, c.d_model,
+                            row_idx, entropy, argmax, logits_out,
+                            scatter_logits ? row_idx : nullptr, ws.at<void>(B_PART), st, s);
   float *logits = (logits_out && !scatter_logits) ? logits_out : ws.at<float>(B_LOGITS);
   GemmDesc g{};
   g.act = c.act_dtype; g.w = c.act_dtype;

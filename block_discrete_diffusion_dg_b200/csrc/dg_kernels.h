@@ -62,7 +62,14 @@ int launch_attention(int act, int batch, int n, int Hq, int Hkv, int hd, const v
                      const void *k_cache, const void *v_cache, const int32_t *cache_len,
                      int cap, const void *k_new, const void *v_new, int causal,
                      const int32_t *done, void *out, void *ws, cudaStream_t s);
-size_t attention_ws_bytes(int batch, int n, int Hq, int hd, int cap);
+size_t attention_ws_bytes(int act, int batch, int n, int Hq, int Hkv, int hd, int cap);
+// bf16 tensor-core path (k_attn_tc.cu): split-KV flash attention + merge.
+bool attention_tc_supported(int act, int Hq, int Hkv, int hd);
+size_t attention_tc_ws_bytes(int batch, int n, int Hq, int hd, int cap);
+int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q,
+                        const void *k_cache, const void *v_cache, const int32_t *cache_len, int cap,
+                        const void *k_new, const void *v_new, int causal, const int32_t *done,
+                        void *out, void *ws, cudaStream_t s);
 
 // ---- MoE (k_moe.cu) ---------------------------------------------------------------------------
 int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *y,
@@ -77,6 +84,9 @@ int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *
 // Scatter rows: dst[row_idx[r]][:] = src[r][:] for r < *n_rows.
 int launch_scatter_rows(const float *src, int width, int max_rows, const int32_t *n_rows,
                         const int32_t *row_idx, float *dst, cudaStream_t s);
+// X[p] = y[perm[p] / k] for p < expert_off[E]; bf16 rows of d elements (d % 8 == 0).
+int launch_gather_rows(int rows_max, int d, int k, const int32_t *perm, const int32_t *expert_off,
+                       int E, const void *y, void *X, cudaStream_t s);
 // a = act(gelu_tanh(u[:, :F]) * u[:, F:]) for rows < expert_off[E].
 int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *expert_off, int E,
                 void *a, cudaStream_t s);
@@ -91,6 +101,30 @@ int launch_combine(int act, int T, int d, int k, const int32_t *topk_idx, const 
 int launch_entropy_rows(const float *logits, int V, int max_rows, const int32_t *n_rows,
                         const int32_t *row_idx, float *entropy, int32_t *argmax, int32_t *st,
                         cudaStream_t s);
+
+// ---- LM head on tensor cores with fused entropy (k_lmhead_tc.cu) ----------------------------
+// F: normalised rows [roundup(max_rows, 128)][K] bf16 (rows >= *n_rows_dev ignored); w_lm [V][K].
+// Entropy/argmax of row r stored at row_idx ? row_idx[r] : r.  logits (debug, may be null):
+// row r written at logits_rows ? logits_rows[r] : r.  ws: lmhead_tc_ws_bytes(max_rows, V).
+bool lmhead_tc_supported(int act, int d);
+size_t lmhead_tc_ws_bytes(int max_rows, int V);
+int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,
+                     int V, int K, const int32_t *row_idx, float *entropy, int32_t *argmax,
+                     float *logits, const int32_t *logits_rows, void *ws, int32_t *st,
+                     cudaStream_t s);
+
+// ---- tensor-core GEMMs (k_gemm_tc.cu) -----------------------------------------------------------
+bool gemm_tc_supported(int act, int w, int K);
+// out[M][N] (+ res) = A[M][K] W[N][K]^T; A must have room for roundup(M, 128) rows.
+int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out_f32,
+                         void *out_bf16, const void *res, int ldo, const char *name, int32_t *st,
+                         cudaStream_t s);
+// Swap-AB expert GEMM over token tiles of experts_tc_tile_tokens() rows.
+int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
+                           int n_assign_max, int K, const GroupTile *tiles,
+                           const int32_t *n_tiles_dev, int max_tiles, const int32_t *expert_off,
+                           void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s);
+int experts_tc_tile_tokens();
 
 // ---- EB select (k_eb.cu) -------------------------------------------------------------------
 int launch_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,

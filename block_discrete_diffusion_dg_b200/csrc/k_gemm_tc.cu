@@ -1,0 +1,391 @@
+// Tensor-core GEMMs of the layer: the dense projections (QKV, output projection + residual) and
+// the grouped expert GEMMs of the MoE FFN (model card "diffusiongemma", Mixture-of-Experts
+// bullet: 8 of 128 experts per token).
+//
+// D[128 x n] = A[128 x K] * B[n x K]^T on tcgen05 (kind::f16, bf16 operands, fp32 accumulator in
+// TMEM), K-major operands staged by TMA with the 128-byte swizzle.  Persistent and
+// warp-specialised like the LM-head kernel: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+// warps 2-5 epilogue over a double-buffered accumulator.
+//
+// Dense:  A = activation rows (M = tokens), B = weight rows (N = output channels).
+// Experts (swap-AB): A = expert weight rows (M = 128 output channels), B = the tokens routed to
+// the expert (N = their count rounded up to 16, at most BN_MAX per unit), so the weights stream
+// through the tensor cores once at the small per-expert token counts of batch 1.  For the
+// gate/up GEMM the 128 A rows are 64 gate rows and the matching 64 up rows, and the epilogue
+// forms a = gelu_tanh(gate) * up; the down GEMM stores Y.
+// Waits are bounded (tc::WAIT_LIMIT_CYCLES) and record DG_ERR_TIMEOUT on expiry.
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace dg {
+
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128, BK = 64;
+constexpr int NUM_THREADS = 192;
+
+enum Kind { K_DENSE_F32 = 0, K_DENSE_RESID = 1, K_MOE_GATE = 2, K_MOE_DOWN = 3 };
+
+struct Params {
+  int kind, K;
+  // dense: M rows (tokens), N columns (channels), tile width bn
+  int M, N, m_tiles, bn;
+  float *out_f32;
+  bf16 *out_bf16;
+  const bf16 *res;
+  int ldo;
+  // experts: token tiles (expert, first token) and per-expert row offsets
+  const GroupTile *tiles;
+  const int32_t *n_tiles_dev;
+  const int32_t *expert_off;
+  int w_rows;       // weight rows per expert (2F for gate/up, d for down)
+  int F;            // expert FFN width (gate/up half)
+  int ld_out;       // row stride of the expert output (F for a, d for Y)
+  bf16 *out;        // a [assignments][F] or Y [assignments][d]
+  int32_t *status;
+};
+
+struct Unit {
+  int a_row0, a_row1;  // A box rows (a_row1 < 0: one 128-row box)
+  int b_row0, n_mma;   // first B row, MMA N (multiple of 16)
+  int n_valid;         // valid columns
+  int row0, col0;      // dense: first token row / first channel; experts: first channel, pos0
+};
+
+__device__ __forceinline__ int n_units(const Params &p) {
+  if (p.kind <= K_DENSE_RESID) return p.m_tiles * ((p.N + p.bn - 1) / p.bn);
+  return *p.n_tiles_dev * p.m_tiles;
+}
+
+template <int BN_MAX>
+__device__ __forceinline__ Unit decode(const Params &p, int u) {
+  Unit x;
+  const int mt = u % p.m_tiles, t = u / p.m_tiles;
+  if (p.kind <= K_DENSE_RESID) {
+    x.a_row0 = mt * BM;
+    x.a_row1 = -1;
+    x.b_row0 = t * p.bn;
+    x.n_valid = min(p.bn, p.N - x.b_row0);
+    x.n_mma = (x.n_valid + 15) & ~15;
+    x.row0 = mt * BM;
+    x.col0 = x.b_row0;
+  } else {
+    const GroupTile g = p.tiles[t];
+    const int off = p.expert_off[g.g];
+    const int cnt = p.expert_off[g.g + 1] - off;
+    x.n_valid = min(BN_MAX, cnt - g.m0);
+    x.n_mma = (x.n_valid + 15) & ~15;
+    x.b_row0 = off + g.m0;
+    x.col0 = off + g.m0;  // first output row (assignment position)
+    if (p.kind == K_MOE_GATE) {
+      x.a_row0 = g.g * p.w_rows + mt * 64;
+      x.a_row1 = g.g * p.w_rows + p.F + mt * 64;
+      x.row0 = mt * 64;  // first gate channel
+    } else {
+      x.a_row0 = g.g * p.w_rows + mt * BM;
+      x.a_row1 = -1;
+      x.row0 = mt * BM;  // first output channel
+    }
+  }
+  return x;
+}
+
+__device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
+  set_status(st, DG_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN_MAX, int STAGES>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN_MAX * BK * 2;
+  static constexpr uint32_t TMEM_COLS = 2 * BN_MAX < 32 ? 32 : 2 * BN_MAX;
+  static constexpr int XCH_BYTES = 64 * 33 * 4;  // gate/up exchange: 64 rows x 32 columns
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + XCH_BYTES + 256;
+};
+
+template <int BN_MAX, int STAGES, int B_BOX>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   Params p) {
+  using C = Cfg<BN_MAX, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * C::A_BYTES;
+  float *xch = reinterpret_cast<float *>(sB + STAGES * C::B_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(xch) + C::XCH_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = n_units(p);
+  if ((int)blockIdx.x >= units) return;
+  const int kblocks = p.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int armed[STAGES];
+      uint32_t armed_ph[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const Unit x = decode<BN_MAX>(p, u);
+        const int nb = (x.n_mma + B_BOX - 1) / B_BOX;
+        const uint32_t bytes = C::A_BYTES + (uint32_t)nb * B_BOX * BK * 2;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
+          mbar_expect_tx(&full[stage], bytes);
+          uint8_t *a = sA + stage * C::A_BYTES;
+          if (x.a_row1 < 0) {
+            tma_load_2d(a, &tmA, &full[stage], kb * BK, x.a_row0);
+          } else {
+            tma_load_2d(a, &tmA, &full[stage], kb * BK, x.a_row0);
+            tma_load_2d(a + 64 * BK * 2, &tmA, &full[stage], kb * BK, x.a_row1);
+          }
+          uint8_t *b = sB + stage * C::B_BYTES;
+          for (int i = 0; i < nb; ++i)
+            tma_load_2d(b + i * B_BOX * BK * 2, &tmB, &full[stage], kb * BK, x.b_row0 + i * B_BOX);
+          armed[stage] = 1;
+          armed_ph[stage] = ph;
+          if (++stage == STAGES) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s]) (void)mbar_wait(&full[s], armed_ph[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      int last_stage = -1;
+      uint32_t last_ph = 0;
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const Unit x = decode<BN_MAX>(p, u);
+        const uint32_t idesc = idesc_bf16(BM, x.n_mma);
+        if (!mbar_wait(&tempty[acc], aph ^ 1)) { fail(p.status, abort_flag); break; }
+        fence_after();
+        const uint32_t d = tmem + acc * BN_MAX;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], ph)) { fail(p.status, abort_flag); ok = false; break; }
+          fence_after();
+          const uint64_t ad = sdesc_sw128(sA + stage * C::A_BYTES);
+          const uint64_t bd = sdesc_sw128(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          commit(&empty[stage]);
+          last_stage = stage;
+          last_ph = ph;
+          if (++stage == STAGES) { stage = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      if (*abort_flag && last_stage >= 0) (void)mbar_wait(&empty[last_stage], last_ph);
+    }
+  } else {
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      if (*abort_flag) break;
+      const Unit x = decode<BN_MAX>(p, u);
+      if (!mbar_wait(&tfull[acc], aph)) { fail(p.status, abort_flag); break; }
+      fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const int r = q * 32 + lane;  // accumulator row of this thread
+#pragma unroll 1
+      for (int c = 0; c * 32 < x.n_valid; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tbase + c * 32, v);
+        tmem_ld_wait(v);
+        const int nv = min(32, x.n_valid - c * 32);
+        if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
+          const int row = x.row0 + r;
+          if (row < p.M) {
+            const int col = x.col0 + c * 32;
+            if (p.kind == K_DENSE_F32) {
+              float *o = p.out_f32 + (size_t)row * p.ldo + col;
+              if (nv == 32) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                  *reinterpret_cast<float4 *>(o + j) =
+                      make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                  __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) o[j] = __uint_as_float(v[j]);
+              }
+            } else {
+              const bf16 *rs = p.res + (size_t)row * p.ldo + col;
+              bf16 *o = p.out_bf16 + (size_t)row * p.ldo + col;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nv)
+                  o[j] = __float2bfloat16_rn(__uint_as_float(v[j]) + __bfloat162float(rs[j]));
+            }
+          }
+        } else if (p.kind == K_MOE_DOWN) {
+          const int ch = x.row0 + r;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nv)
+              p.out[(size_t)(x.col0 + c * 32 + j) * p.ld_out + ch] =
+                  __float2bfloat16_rn(__uint_as_float(v[j]));
+        } else {  // K_MOE_GATE: rows 0-63 gate, 64-127 up of the same channels
+          if (q >= 2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xch[((q - 2) * 32 + lane) * 33 + j] = __uint_as_float(v[j]);
+          }
+          epi_bar();
+          if (q < 2) {
+            const int ch = x.row0 + r;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j >= nv) continue;
+              const float g = __uint_as_float(v[j]);
+              const float up = xch[(q * 32 + lane) * 33 + j];
+              const float gl =
+                  0.5f * g * (1.0f + tanhf(0.7978845608028654f * (g + 0.044715f * g * g * g)));
+              p.out[(size_t)(x.col0 + c * 32 + j) * p.ld_out + ch] = __float2bfloat16_rn(gl * up);
+            }
+          }
+          epi_bar();
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN_MAX, int STAGES, int B_BOX>
+int launch(const CUtensorMap &tmA, const CUtensorMap &tmB, const Params &p, int units_max,
+           const char *name, cudaStream_t s) {
+  using C = Cfg<BN_MAX, STAGES>;
+  auto k = gemm_tc_kernel<BN_MAX, STAGES, B_BOX>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  const int grid = units_max < num_sms() ? units_max : num_sms();
+  if (grid <= 0) return DG_OK;
+  note_launch(s, name);
+  k<<<grid, NUM_THREADS, C::SMEM, s>>>(tmA, tmB, p);
+  return check_launch(name);
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int act, int w, int K) {
+  return act == DG_BF16 && w == DG_BF16 && K % BK == 0 && K >= BK;
+}
+
+// Dense: out[M][N] (+ res) = A[M][K] * W[N][K]^T.  out_f32 xor out_bf16 (with res).
+int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out_f32,
+                         void *out_bf16, const void *res, int ldo, const char *name,
+                         int32_t *st, cudaStream_t s) {
+  constexpr int BN = 64;
+  const int M_alloc = (M + BM - 1) / BM * BM;  // A has room for whole tiles (caller's layout)
+  CUtensorMap ta, tb;
+  int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M_alloc, (uint64_t)K * 2, BK,
+                        BM);
+  if (rc != DG_OK) return rc;
+  rc = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, N, (uint64_t)K * 2, BK, BN);
+  if (rc != DG_OK) return rc;
+  Params p{};
+  p.kind = out_f32 ? K_DENSE_F32 : K_DENSE_RESID;
+  p.K = K;
+  p.M = M;
+  p.N = N;
+  p.m_tiles = M_alloc / BM;
+  p.bn = BN;
+  p.out_f32 = out_f32;
+  p.out_bf16 = reinterpret_cast<bf16 *>(out_bf16);
+  p.res = reinterpret_cast<const bf16 *>(res);
+  p.ldo = ldo;
+  p.status = st;
+  const int units = p.m_tiles * ((N + BN - 1) / BN);
+  return launch<BN, 8, BN>(ta, tb, p, units, name, s);
+}
+
+// Experts (swap-AB).  gate_up: W [E][2F][K], X = the routed rows [assignments][K] (permuted order)
+// -> a [assignments][F].  down: W [E][d][F], X = a -> Y [assignments][d].
+int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
+                           int n_assign_max, int K, const GroupTile *tiles,
+                           const int32_t *n_tiles_dev, int max_tiles, const int32_t *expert_off,
+                           void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s) {
+  constexpr int BN_MAX = 64, B_BOX = 32;
+  CUtensorMap ta, tb;
+  int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, (uint64_t)E * w_rows,
+                        (uint64_t)K * 2, BK, gate_up ? 64 : BM);
+  if (rc != DG_OK) return rc;
+  rc = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, n_assign_max, (uint64_t)K * 2,
+                    BK, B_BOX);
+  if (rc != DG_OK) return rc;
+  Params p{};
+  p.kind = gate_up ? K_MOE_GATE : K_MOE_DOWN;
+  p.K = K;
+  p.tiles = tiles;
+  p.n_tiles_dev = n_tiles_dev;
+  p.expert_off = expert_off;
+  p.w_rows = w_rows;
+  p.F = F;
+  p.m_tiles = gate_up ? F / 64 : w_rows / BM;
+  p.ld_out = ld_out;
+  p.out = reinterpret_cast<bf16 *>(out);
+  p.status = st;
+  return launch<BN_MAX, 8, B_BOX>(ta, tb, p, max_tiles * p.m_tiles, name, s);
+}
+
+int experts_tc_tile_tokens() { return 64; }
+
+}  // namespace dg

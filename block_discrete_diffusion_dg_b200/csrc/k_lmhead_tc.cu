@@ -1,0 +1,322 @@
+// LM head with fused softmax entropy and greedy argmax on the 5th-generation tensor cores.
+// "DiffusionGemma Technical Report", explanatory visual and What they did: the entropy-bounded
+// sampler ranks canvas positions by the entropy of their predictive distribution; Table 1:
+// vocabulary 262k.  The logits z = f W_lm^T of the masked rows are never stored (except for
+// debugging); each (row, vocabulary tile) leaves a partial softmax state that a second kernel
+// merges exactly.
+//
+// Persistent, warp-specialised kernel, one CTA per SM:
+//   warp 0      TMA producer: A = 128 normalised rows x 64 k, B = 256 vocabulary rows x 64 k,
+//               4-stage ring in shared memory (48 KB per stage, 128-byte swizzle);
+//   warp 1      allocates 512 TMEM columns and issues tcgen05.mma (M 128, N 256, K 16) into one
+//               of two 256-column fp32 accumulators, so the epilogue of one tile overlaps the
+//               MMAs of the next;
+//   warps 2-5   epilogue: each thread owns one row and reads its 256 logits from TMEM in chunks
+//               of 32, keeping m = max, s = sum e^(z-m), u = sum e^(z-m)(z-m) and the first
+//               argmax (see entropy_state.cuh).
+// Work units are (row tile, vocabulary tile) with the row tile varying fastest, so the CTAs
+// working on the same vocabulary tile run together and share it through L2.
+// Every wait is bounded (tc::WAIT_LIMIT_CYCLES); on expiry the kernel records DG_ERR_TIMEOUT,
+// drains what it issued, frees TMEM and returns.
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+#include "entropy_state.cuh"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace dg {
+
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256;
+
+struct Params {
+  const int32_t *n_rows_dev;
+  int max_rows, V, K, n_vtiles;
+  float4 *part;             // [max_rows][n_vtiles]: (m, s, u, max value)
+  int32_t *part_am;         // [max_rows][n_vtiles]: first argmax in the tile
+  float *logits;            // debug: [*][V] or null
+  const int32_t *logits_rows;  // debug: output row of row r (null: r)
+  int32_t *status;
+};
+
+__device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
+  set_status(st, DG_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * A_BYTES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sB + STAGES * B_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n_rows = p.max_rows;
+  if (p.n_rows_dev) n_rows = min(*p.n_rows_dev, p.max_rows);
+  const int m_tiles = (n_rows + BM - 1) / BM;
+  const int units = m_tiles * p.n_vtiles;
+  if ((int)blockIdx.x >= units) return;  // uniform across the block
+  const int kblocks = p.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int armed[STAGES];
+      uint32_t armed_ph[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const int mt = u % m_tiles, nt = u / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
+          mbar_expect_tx(&full[stage], A_BYTES + B_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, &full[stage], kb * BK, mt * BM);
+          tma_load_2d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, nt * BN);
+          armed[stage] = 1;
+          armed_ph[stage] = ph;
+          if (++stage == STAGES) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) {  // let every issued copy land before the CTA's shared memory goes away
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s]) (void)mbar_wait(&full[s], armed_ph[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(BM, BN);
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      int last_stage = -1;
+      uint32_t last_ph = 0;
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], aph ^ 1)) { fail(p.status, abort_flag); break; }
+        fence_after();
+        const uint32_t d = tmem + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], ph)) { fail(p.status, abort_flag); ok = false; break; }
+          fence_after();
+          const uint64_t ad = sdesc_sw128(sA + stage * A_BYTES);
+          const uint64_t bd = sdesc_sw128(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          commit(&empty[stage]);
+          last_stage = stage;
+          last_ph = ph;
+          if (++stage == STAGES) { stage = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      if (*abort_flag && last_stage >= 0)  // the MMAs issued so far finish before TMEM is freed
+        (void)mbar_wait(&empty[last_stage], last_ph);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      if (*abort_flag) break;
+      const int mt = u % m_tiles, nt = u / m_tiles;
+      if (!mbar_wait(&tfull[acc], aph)) { fail(p.status, abort_flag); break; }
+      fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const bool row_ok = row < n_rows;
+      float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
+      int am = 0x7fffffff;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float *lrow = nullptr;
+      if (p.logits && row_ok)
+        lrow = p.logits + (size_t)(p.logits_rows ? p.logits_rows[row] : row) * p.V;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nt * BN + c * 32;
+        if (col0 >= p.V) break;  // uniform in the warp
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_ld_wait(r);
+        const int nvalid = min(32, p.V - col0);
+        float cm = -INFINITY;
+        int ci = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float v = __uint_as_float(r[j]);
+          if (j < nvalid && v > cm) { cm = v; ci = j; }
+        }
+        if (cm > av) { av = cm; am = col0 + ci; }
+        const float mn = fmaxf(m, cm);
+        float cs = 0.f, cu = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j < nvalid) {
+            const float t = __uint_as_float(r[j]) - mn;
+            const float e = __expf(t);
+            cs += e;
+            cu = fmaf(e, t, cu);
+          }
+        }
+        if (s > 0.f) {
+          const float sc = __expf(m - mn);
+          uu = sc * fmaf(s, m - mn, uu);
+          s *= sc;
+        }
+        s += cs;
+        uu += cu;
+        m = mn;
+        if (lrow) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid) lrow[col0 + j] = __uint_as_float(r[j]);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (row_ok) {
+        const size_t o = (size_t)row * p.n_vtiles + nt;
+        p.part[o] = make_float4(m, s, uu, av);
+        p.part_am[o] = am;
+      }
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Merge the partial states of one row over all vocabulary tiles (fixed order) and store the
+// entropy and argmax at the row's source index.
+__global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restrict__ part,
+                                                         const int32_t *__restrict__ part_am,
+                                                         int n_vtiles,
+                                                         const int32_t *__restrict__ n_rows_dev,
+                                                         const int32_t *__restrict__ row_idx,
+                                                         float *entropy, int32_t *argmax,
+                                                         int32_t *st) {
+  const int r = blockIdx.x;
+  if (n_rows_dev && r >= *n_rows_dev) return;
+  EntState es;
+  es.init();
+  for (int t = threadIdx.x; t < n_vtiles; t += blockDim.x) {
+    const float4 v = part[(size_t)r * n_vtiles + t];
+    EntState o;
+    o.m = v.x; o.s = v.y; o.u = v.z; o.av = v.w;
+    o.am = part_am[(size_t)r * n_vtiles + t];
+    es.merge(o);
+  }
+  __shared__ EntState red[8];
+  es = es.warp_reduce();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = es;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    EntState t = red[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) t.merge(red[i]);
+    const float H = t.entropy();
+    if (!isfinite(H)) set_status(st, DG_ERR_NUMERIC);
+    const int out = row_idx ? row_idx[r] : r;
+    entropy[out] = H;
+    argmax[out] = t.am;
+  }
+}
+
+}  // namespace
+
+size_t lmhead_tc_ws_bytes(int max_rows, int V) {
+  const size_t nvt = (size_t)(V + BN - 1) / BN;
+  return (size_t)max_rows * nvt * (sizeof(float4) + sizeof(int32_t)) + 256;
+}
+
+bool lmhead_tc_supported(int act, int d) { return act == DG_BF16 && d % BK == 0 && d >= BK; }
+
+int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,
+                     int V, int K, const int32_t *row_idx, float *entropy, int32_t *argmax,
+                     float *logits, const int32_t *logits_rows, void *ws, int32_t *st,
+                     cudaStream_t s) {
+  if (max_rows <= 0) return DG_OK;
+  const int n_vtiles = (V + BN - 1) / BN;
+  CUtensorMap tmA, tmB;
+  // F has room for whole 128-row tiles (rows past max_rows are never stored)
+  const int rows_alloc = (max_rows + BM - 1) / BM * BM;
+  int rc = make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, F, (uint64_t)K,
+                        (uint64_t)rows_alloc, (uint64_t)K * 2, BK, BM);
+  if (rc != DG_OK) return rc;
+  rc = make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_lm, (uint64_t)K, (uint64_t)V,
+                    (uint64_t)K * 2, BK, BN);
+  if (rc != DG_OK) return rc;
+  Params p;
+  p.n_rows_dev = n_rows_dev;
+  p.max_rows = max_rows;
+  p.V = V;
+  p.K = K;
+  p.n_vtiles = n_vtiles;
+  p.part = reinterpret_cast<float4 *>(ws);
+  p.part_am = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(ws) +
+                                          (size_t)max_rows * n_vtiles * sizeof(float4));
+  p.logits = logits;
+  p.logits_rows = logits_rows;
+  p.status = st;
+  cudaFuncSetAttribute(lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)SMEM_BYTES);
+  const int units_max = ((max_rows + BM - 1) / BM) * n_vtiles;
+  const int grid = units_max < num_sms() ? units_max : num_sms();
+  note_launch(s, "lm_head_tc");
+  lmhead_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tmA, tmB, p);
+  rc = check_launch("lm_head_tc");
+  if (rc != DG_OK) return rc;
+  note_launch(s, "lm_combine");
+  lm_combine_kernel<<<max_rows, 256, 0, s>>>(p.part, p.part_am, n_vtiles, n_rows_dev, row_idx,
+                                             entropy, argmax, st);
+  return check_launch("lm_combine");
+}
+
+}  // namespace dg

@@ -158,6 +158,17 @@ __global__ void build_tiles_kernel(int E, const int32_t *__restrict__ expert_off
   }
 }
 
+// X[p] = y[perm[p] / k] for the routed assignments p < expert_off[E] (bf16 rows, 16-byte copies).
+__global__ void gather_rows_kernel(int d, int k, const int32_t *__restrict__ perm,
+                                   const int32_t *__restrict__ expert_off, int E,
+                                   const uint4 *__restrict__ y, uint4 *X) {
+  const int p = blockIdx.x;
+  if (p >= expert_off[E]) return;
+  const int t = perm[p] / k;
+  const int n16 = d / 8;
+  for (int i = threadIdx.x; i < n16; i += blockDim.x) X[(size_t)p * n16 + i] = y[(size_t)t * n16 + i];
+}
+
 template <typename T>
 __global__ void gate_kernel(int F, const float *__restrict__ u, const int32_t *__restrict__ expert_off,
                             int E, T *a) {
@@ -229,6 +240,14 @@ int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *
   note_launch(s, "build_tiles");
   build_tiles_kernel<<<1, 256, 0, s>>>(E, expert_off, tile_m, tiles, n_tiles, max_tiles);
   return check_launch("build_tiles");
+}
+
+int launch_gather_rows(int rows_max, int d, int k, const int32_t *perm, const int32_t *expert_off,
+                       int E, const void *y, void *X, cudaStream_t s) {
+  if (rows_max <= 0) return DG_OK;
+  note_launch(s, "gather_rows");
+  gather_rows_kernel<<<rows_max, 128, 0, s>>>(d, k, perm, expert_off, E, (const uint4 *)y, (uint4 *)X);
+  return check_launch("gather_rows");
 }
 
 int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *expert_off, int E,
