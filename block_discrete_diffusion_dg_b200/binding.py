@@ -72,6 +72,7 @@ _SIGS = {
     "dg_moe_ffn": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _PLW, _VP, _VP, _VP, _SZ, _VP,
                           _VP]),
     "dg_logits_entropy": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "dg_logits_entropy_static": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dg_eb_select": (_I32, [_I32, _I32, _VP, _VP, ctypes.c_double, _I32, _VP, _VP, _VP, _VP, _VP,
                             _VP, _VP, _VP]),
     "dg_kv_append": (_I32, [_PCFG, _PMODEL, _I32, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _SZ, _VP,
@@ -225,6 +226,15 @@ def dg_logits_entropy(cfg, n_rows, n_rows_dev, h, row_idx, w_lm, entropy, argmax
     _check(lib().dg_logits_entropy(ctypes.byref(cfg), n_rows, _p(n_rows_dev), _p(h), _p(row_idx),
                                    _p(w_lm), _p(entropy), _p(argmax), _p(logits_dbg), w, wb,
                                    _p(dev_status), _stream(stream)), "dg_logits_entropy")
+
+
+def dg_logits_entropy_static(cfg, n_rows, n_rows_dev, h, row_idx, w_lm, entropy, argmax,
+                             dev_status=None, stream=None):
+    """dg_logits_entropy without a scratch argument (its scratch is a fixed array in the library)."""
+    _check(lib().dg_logits_entropy_static(ctypes.byref(cfg), n_rows, _p(n_rows_dev), _p(h),
+                                          _p(row_idx), _p(w_lm), _p(entropy), _p(argmax),
+                                          _p(dev_status), _stream(stream)),
+           "dg_logits_entropy_static")
 
 
 def dg_eb_select(batch, canvas, entropy, argmax, gamma, max_steps, tokens, masked, selected,

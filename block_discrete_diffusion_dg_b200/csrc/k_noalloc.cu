@@ -1,0 +1,82 @@
+// dg_logits_entropy_static: the final-norm + LM-head + entropy/argmax operation of
+// dg_logits_entropy, for callers that cannot hand the library a scratch buffer.
+//
+// Who needs it: code that runs where device allocation is not available to it — for example a
+// serving engine that reserves all device memory for its own pools at start-up (a later
+// cudaMalloc fails or fragments the pool), or a plugin whose host application owns every device
+// allocation and only lends it the model's tensors.  Such a caller still owns its inputs and
+// outputs; the scratch this operation needs lives in a fixed array in the library's device image.
+//
+// The array is a file-scope __device__ object of DG_STATIC_SCRATCH_BYTES bytes; every GPU that
+// loads the library holds it until the process exits.  Its device address is looked up once per
+// device (cudaGetSymbolAddress with that device current) on the first call made on that device.
+#include <mutex>
+
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+namespace {
+
+constexpr int MAX_ROWS = 256;       // rows per call
+constexpr int MAX_D = 2048;         // d_model
+constexpr int MAX_VOCAB = 262144;   // vocabulary
+constexpr size_t NORM_BYTES = (size_t)MAX_ROWS * MAX_D * 2;   // normalised rows (bf16)
+
+__device__ __align__(256) uint8_t g_static_scratch[DG_STATIC_SCRATCH_BYTES];
+
+constexpr int MAX_DEVICES = 64;
+std::mutex g_mu;
+void *g_scratch_addr[MAX_DEVICES] = {};
+
+// Device address of the array on the current device (looked up on first use).
+int scratch_address(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("dg_logits_entropy_static");
+  if (dev < 0 || dev >= MAX_DEVICES) return DG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_addr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();
+      return DG_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return DG_OK;
+}
+
+}  // namespace
+}  // namespace dg
+
+using namespace dg;
+
+extern "C" int dg_logits_entropy_static(const dg_config *cfg, int n_rows,
+                                        const int32_t *n_rows_dev, const void *h,
+                                        const int32_t *row_idx, const void *w_lm,
+                                        float *entropy, int32_t *argmax, int32_t *dev_status,
+                                        void *stream) {
+  if (!cfg || n_rows <= 0 || !h || !w_lm || !entropy || !argmax) return DG_ERR_INVALID_ARG;
+  if (cfg->d_model <= 0 || cfg->vocab < 2) return DG_ERR_INVALID_ARG;
+  if (!lmhead_tc_supported(cfg->act_dtype, cfg->d_model)) return DG_ERR_UNSUPPORTED;
+  // requests larger than the fixed array: rejected, nothing launched
+  if (n_rows > MAX_ROWS || cfg->d_model > MAX_D || cfg->vocab > MAX_VOCAB)
+    return DG_ERR_WORKSPACE;
+  const int rows128 = (n_rows + 127) / 128 * 128;
+  if ((size_t)rows128 * cfg->d_model * 2 > NORM_BYTES ||
+      NORM_BYTES + lmhead_tc_ws_bytes(n_rows, cfg->vocab) > (size_t)DG_STATIC_SCRATCH_BYTES)
+    return DG_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != DG_OK) return rc;
+  char *norm_rows = static_cast<char *>(scratch);
+  char *partials = norm_rows + NORM_BYTES;
+  const cudaStream_t s = (cudaStream_t)stream;
+  const int r1 = launch_rmsnorm(cfg->act_dtype, h, row_idx, n_rows_dev, n_rows, cfg->d_model,
+                                cfg->rms_eps, norm_rows, s);
+  if (r1 != DG_OK) return r1;
+  return launch_lmhead_tc(norm_rows, n_rows, n_rows_dev, w_lm, cfg->vocab, cfg->d_model, row_idx,
+                          entropy, argmax, nullptr, nullptr, partials, dev_status, s);
+}

@@ -225,6 +225,27 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                    int32_t *argmax_out, float *logits_dbg, void *ws, size_t ws_bytes,
                    int32_t *dev_status, void *stream);
 
+/* ---- fixed-scratch entry point ---------------------------------------------------------- */
+
+/* dg_logits_entropy for callers that cannot provide device scratch memory.  The pages have no
+ * counterpart: this is a library-integration variant, not a step of the method.  Some callers
+ * cannot allocate device memory at all — an engine that has reserved the whole device for its
+ * own pools, or a plugin whose host owns every allocation — so this call takes no `ws` and keeps
+ * its scratch in a fixed array of DG_STATIC_SCRATCH_BYTES inside the library's device image,
+ * which every GPU that loads the library holds until the process exits.  It allocates nothing.
+ *   Same arguments and results as dg_logits_entropy, without logits_dbg and ws.
+ *   Limits: bf16 activations (DG_ERR_UNSUPPORTED otherwise), n_rows <= 256, d_model <= 2048,
+ *   vocab <= 262144; larger requests return DG_ERR_WORKSPACE and launch nothing.
+ *   The first call on a device looks up the array's device address with that device current
+ *   (cudaGetSymbolAddress); make that first call before any stream capture on the device.
+ *   All calls share the one array and it keeps the last call's contents (nothing in it has to
+ *   start at zero): calls whose work overlaps on the GPU — on different streams, or from
+ *   different threads — race on it and must be serialised by the caller. */
+#define DG_STATIC_SCRATCH_BYTES (6u * 1024u * 1024u + 4096u)
+int dg_logits_entropy_static(const dg_config *cfg, int n_rows, const int32_t *n_rows_dev,
+                             const void *h, const int32_t *row_idx, const void *w_lm,
+                             float *entropy, int32_t *argmax, int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
