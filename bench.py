@@ -44,7 +44,7 @@ def load_peaks():
 
 # ------------------------------------------------------------------------------ accounting
 
-def step_bytes(cfg, experts_touched: int) -> dict:
+def step_bytes(cfg, experts_touched: float) -> dict:
     """Algorithmic HBM bytes of one step: every weight byte the step must read once, the
     prompt K/V, and the canvas rows (activations are small and are not counted)."""
     wb = 1 if cfg.w == "e4m3" else (4 if cfg.w == "f32" else 2)
@@ -248,6 +248,12 @@ def workload_desc(cfg) -> str:
             f"half-committed canvases")
 
 
+# DRAM traffic per launch of the dominant kernel from one ncu capture of the same kernel build
+# (profiles/tc_kernels_canvas_step_layer.md); set to None when the kernel changes.
+NCU_TRAFFIC = {"lm_head_tc": {"bytes": 1076431000 + 6052352,
+                              "source": "profiles/tc_kernels_canvas_step_layer.md"}}
+
+
 def run_dg(args, world, rank, local):
     import synth
     from block_discrete_diffusion_dg_b200 import binding as B
@@ -263,19 +269,27 @@ def run_dg(args, world, rank, local):
     init = [{k: v.to(dev) for k, v in synth.make_canvas_state(cfg, s).items()}
             for s in ("all_mask", "half")]
     st = {k: v.clone() for k, v in init[0].items()}
-    stream = torch.cuda.current_stream()
+    load = torch.zeros((cfg.n_layers, cfg.n_experts), dtype=torch.int32, device=dev)
 
-    def one_step(i):
+    def one_step(i, stream=None, expert_load=None):
         src = init[i % 2]
         for k in st:
             st[k].copy_(src[k], non_blocking=True)
         B.dg_canvas_step(dgcfg, dgm, cfg.batch, st["tokens"], st["masked"], st["n_masked"],
                          st["done"], st["step"], cfg.max_steps, cfg.gamma, kv["k"], kv["v"],
-                         kv["cache_len"], cap, None, None, None, ws, status, stream)
+                         kv["cache_len"], cap, None, None, None, ws, status, stream,
+                         expert_load=expert_load)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world > 1:
+            t = torch.tensor([x], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            return float(t.item())
+        return x
 
     for i in range(args.warmup):
         one_step(i)
@@ -283,49 +297,89 @@ def run_dg(args, world, rank, local):
     rc = B.dg_read_status(status)
     if rc != B.DG_OK:
         raise RuntimeError(f"device status {B.STATUS_NAMES.get(rc, rc)} during warm-up")
-    committed_per_step = []
-    for i in range(2):   # commits per step of each state (for output tok/s)
-        one_step(i)
-        torch.cuda.synchronize()
-        committed_per_step.append(int(init[i % 2]["n_masked"].sum() - st["n_masked"].sum()))
 
+    # per state: tokens committed by one step, experts the step routes to, kernels it launches
+    committed, touched, per_step_launches = [], [], 0
+    for i in range(2):
+        n0 = B.dg_launch_count()
+        one_step(i, expert_load=load)
+        torch.cuda.synchronize()
+        per_step_launches = B.dg_launch_count() - n0
+        committed.append(int(init[i]["n_masked"].sum() - st["n_masked"].sum()))
+        touched.append(float((load > 0).sum(dim=1).float().mean().item()))
+
+    # ---- timed region: K steps replayed from CUDA graphs (one graph per canvas state) ----
+    graphs = []
+    if not args.no_graph:
+        try:
+            for i in range(2):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    one_step(i)
+                graphs.append(g)
+            for g in graphs:
+                g.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture not possible: time the direct launches instead
+            print(f"graph capture failed ({e}); timing direct launches", file=sys.stderr)
+            graphs = []
+    stream = torch.cuda.current_stream()
     uuid = None
     try:
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
     clocks = ClockSampler(uuid)
-    # ---- timed region: K steps, per-launch events recorded by the library ----
-    n_rec = args.steps * 64 + 16
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
-    l0 = B.dg_launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    B.dg_profile_begin(n_rec)
     ev0.record(stream)
     for i in range(args.steps):
-        one_step(args.warmup + i)
-        B.dg_profile_mark(stream)
+        if graphs:
+            graphs[i % 2].replay()
+        else:
+            one_step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
-    prof = B.dg_profile_end(n_rec)
-    launches = B.dg_launch_count() - l0
     barrier()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
     rc = B.dg_read_status(status)
     if rc != B.DG_OK:
         raise RuntimeError(f"device status {B.STATUS_NAMES.get(rc, rc)} in the timed region")
     ms_step = ms / args.steps
     steps_s = world * args.steps / (ms / 1e3)
+    launches = per_step_launches * args.steps
 
-    # ---- per-kernel breakdown and the dominant kernel's roofline ----
+    # ---- profile pass: the same steps with a CUDA event before every kernel, captured into one
+    # graph (external event-record nodes) and replayed, so launch gaps are not counted ----
+    kp = max(4, min(args.steps, 20))
+    n_rec = kp * 64 + 16
+    torch.cuda.synchronize()
+    B.dg_profile_begin(n_rec)
+    prof_mode = "graph"
+    try:
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gp):
+            cs = torch.cuda.current_stream()
+            for i in range(kp):
+                one_step(i)
+                B.dg_profile_mark(cs)
+        gp.replay()
+        torch.cuda.synchronize()
+        prof = B.dg_profile_end(n_rec)
+        del gp
+    except Exception as e:
+        print(f"profile graph failed ({e}); profiling direct launches", file=sys.stderr)
+        prof_mode = "direct"
+        B.dg_profile_begin(n_rec)
+        for i in range(kp):
+            one_step(i, stream)
+            B.dg_profile_mark(stream)
+        B.dg_profile_mark(stream)
+        prof = B.dg_profile_end(n_rec)
     per = {}
     for name, t in prof:
         if name == "(mark)":
@@ -338,20 +392,24 @@ def run_dg(args, world, rank, local):
                      "ms_per_launch": round(v[0] / v[1], 5), "share": round(v[0] / tot, 4)}
                  for k, v in sorted(per.items(), key=lambda kv_: -kv_[1][0])}
     peaks, peak_src = load_peaks()
-    experts_touched = cfg.n_experts
-    sb = step_bytes(cfg, experts_touched)
+    t_avg = float(np.mean(touched))
+    sb = step_bytes(cfg, t_avg)
     dom = next(iter(breakdown))
-    dom_bytes = {"lm_head_logits": sb["lm_head"], "moe_gemm_gate_up": sb["expert_gate_up"],
-                 "moe_gemm_down": sb["expert_down"], "lm_head_entropy": sb["lm_head"]}.get(dom)
+    dom_bytes = {"lm_head_tc": sb["lm_head"] + cfg.batch * cfg.canvas * cfg.d_model * 2,
+                 "moe_gate_up_tc": sb["expert_gate_up"], "moe_down_tc": sb["expert_down"]}.get(dom)
     roof = None
     if dom_bytes:
         dur = breakdown[dom]["ms_per_launch"] / 1e3
         ach = dom_bytes / dur / 1e9
         peak = peaks["hbm_gbs"]
+        tr = NCU_TRAFFIC.get(dom)
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(ach / peak, 4), "traffic": None,
-                "algorithmic_bytes_per_launch": dom_bytes,
-                "peak_source": f"{peak_src} (burst copy)"}
+                "unit": "GB/s", "frac": round(ach / peak, 4),
+                "traffic": tr["bytes"] if tr else None,
+                "algorithmic_bytes_per_launch": int(dom_bytes),
+                "peak_source": f"{peak_src} (burst copy, of measured)",
+                "timing": f"CUDA events before each launch, {kp}-step profile pass ({prof_mode})",
+                "traffic_source": tr["source"] if tr else None}
     masked_avg = 0.5 * (cfg.canvas + cfg.canvas // 2) * cfg.batch
     t_bytes = sb["total"] / (peaks["hbm_gbs"] * 1e9)
     t_flops = step_flops(cfg, masked_avg) / (peaks["bf16_tflops_sustained"] * 1e12)
@@ -359,12 +417,14 @@ def run_dg(args, world, rank, local):
                  "roofline_us": round(1e6 * max(t_bytes, t_flops), 1),
                  "measured_us": round(1e3 * ms_step, 1),
                  "frac": round(1e6 * max(t_bytes, t_flops) / (1e3 * ms_step), 4),
-                 "algorithmic_bytes": sb["total"], "algorithmic_flops": step_flops(cfg, masked_avg),
+                 "algorithmic_bytes": int(sb["total"]),
+                 "algorithmic_flops": step_flops(cfg, masked_avg),
+                 "experts_touched_per_state": touched,
                  "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, "
-                          f"{peaks['bf16_tflops_sustained']} TF/s sustained"}
+                          f"{peaks['bf16_tflops_sustained']} TF/s sustained (of measured)"}
 
     # ---- end to end through the C ABI with host buffers ----
-    pin = [{k: v.cpu().pin_memory() for k, v in s.items()} for s in init]
+    pin = [{k: v.cpu().pin_memory() for k, v in s_.items()} for s_ in init]
     out_h = {k: torch.empty_like(pin[0][k]).pin_memory() for k in ("tokens", "masked", "done")}
     h2d = sum(t.numel() * t.element_size() for t in pin[0].values())
     d2h = sum(t.numel() * t.element_size() for t in out_h.values())
@@ -382,13 +442,10 @@ def run_dg(args, world, rank, local):
         for k in out_h:
             out_h[k].copy_(st[k], non_blocking=True)
         stream.synchronize()       # the caller reads the committed tokens and the done flag
-    e_s = time.perf_counter() - e0
-    if world > 1:
-        t = torch.tensor([e_s], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e_s = float(t.item())
+    e_s = max_over_ranks(time.perf_counter() - e0)
     e2e = {"value": world * e_steps / e_s, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h}
+           "d2h_bytes_per_step": d2h,
+           "note": "direct calls (no graph), host state copied in and result read back every step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -405,19 +462,19 @@ def run_dg(args, world, rank, local):
                          f"canvas, experts e < E/{args.ref_frac} and an LM-head vocab slice of "
                          f"V/{args.ref_frac}, both scaled by {args.ref_frac}"}
 
-    tok_s = steps_s * float(np.mean(committed_per_step)) / cfg.batch
+    tok_s = steps_s * float(np.mean(committed)) / cfg.batch
     line = {"metric": METRIC, "value": round(steps_s, 3), "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random-init weights, N(0,1) prompt K/V)",
             "config": {"workload": workload_desc(cfg), "batch": cfg.batch, "canvas": cfg.canvas,
                        "prompt_kv": cfg.prompt_len, "parallelism": f"replicas x{world}",
+                       "cuda_graph": bool(graphs),
                        "l2": "inputs larger than L2 (>2 GB of weights per step); no flush"},
-            "output_tok_s": round(tok_s, 2),
-            "tokens_committed_per_step": committed_per_step,
+            "output_tok_s": round(tok_s, 2), "tokens_committed_per_step": committed,
             "step_roofline": step_roof, "roofline": roof, "kernels": breakdown,
-            "gpu_launches": int(launches), "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
-            "impl": "dg"}
+            "gpu_launches": int(launches), "launches_per_step": int(per_step_launches),
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clk, "impl": "dg"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -431,6 +488,7 @@ def main():
     ap.add_argument("--workload", default="layer")
     ap.add_argument("--ref-frac", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time direct launches")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

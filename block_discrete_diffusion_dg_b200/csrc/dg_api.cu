@@ -27,7 +27,13 @@ static thread_local Profile g_prof;
 void note_launch(cudaStream_t s, const char *name) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (g_prof.on && g_prof.n < (int)g_prof.ev.size()) {
-    cudaEventRecord(g_prof.ev[g_prof.n], s);
+    // inside stream capture the record becomes a graph node whose timestamp is taken at replay
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+      cudaEventRecordWithFlags(g_prof.ev[g_prof.n], s, cudaEventRecordExternal);
+    else
+      cudaEventRecord(g_prof.ev[g_prof.n], s);
     g_prof.name[g_prof.n] = name;
     ++g_prof.n;
   }
@@ -49,7 +55,7 @@ inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
-  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_LIVE, B_ROWS, B_NROWS, B_FIN, B_LOGITS, B_PART,
+  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_LIVE, B_ROWS, B_NROWS, B_FIN, B_LOGITS, B_PART,
   B_ENT, B_AM, B_ATTN, B_COUNT
 };
 
@@ -68,7 +74,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   L.max_tiles = (int)((TK + TILE_M - 1) / TILE_M) + c.n_experts;
   size_t sz[B_COUNT];
   const size_t T128 = (T + 127) / 128 * 128;  // tensor-core A operands read whole 128-row tiles
-  sz[B_X] = T * d * a;
+  sz[B_X] = T * d * 4;  // residual stream: fp32
   sz[B_A] = T128 * d * a;
   sz[B_QKV] = T * qkvw * 4;
   sz[B_CS] = T * hd * 4;
@@ -76,8 +82,9 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_KN] = T * c.n_kv_heads * hd * a;
   sz[B_VN] = T * c.n_kv_heads * hd * a;
   sz[B_O] = T128 * c.n_q_heads * hd * a;
-  sz[B_H] = T * d * a;
-  sz[B_Y] = T * d * a;
+  sz[B_H] = T * d * 4;
+  sz[B_Y] = T128 * d * a;
+  sz[B_Z] = T * (size_t)c.n_experts * 4;
   sz[B_IDX] = TK * 4;
   sz[B_W] = TK * 4;
   sz[B_OFF] = (size_t)(c.n_experts + 1) * 4;
@@ -87,7 +94,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_NTILES] = 4;
   sz[B_U] = TK * 2 * F * 4;
   sz[B_ACT] = TK * F * a;
-  sz[B_YE] = TK * d * a;
+  sz[B_YE] = TK * d * 4;  // expert outputs: fp32
   sz[B_XP] = TK * d * a;
   sz[B_LIVE] = T;
   sz[B_ROWS] = T * 4;
@@ -162,7 +169,7 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
   g.name = "gemm_qkv";
   if (gemm_tc_supported(c.act_dtype, c.w_dtype, c.d_model))
     return launch_gemm_tc_dense(ws.at<void>(B_A), T, w.w_qkv, g.N, c.d_model, ws.at<float>(B_QKV),
-                                nullptr, nullptr, g.N, "gemm_qkv_tc", nullptr, s);
+                                nullptr, g.N, "gemm_qkv_tc", nullptr, s);
   return launch_gemm_simt(g, EPI_F32, ws.at<void>(B_QKV), g.N, nullptr, s);
 }
 
@@ -178,15 +185,22 @@ int attn_out_and_moe(const dg_config &c, const dg_layer_weights &w, const Ws &ws
   g.M = T; g.N = d; g.K = hq;
   g.name = "gemm_o_resid";
   if (gemm_tc_supported(c.act_dtype, c.w_dtype, hq))
-    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, w.w_o, d, hq, nullptr, ws.at<void>(B_H),
-                                ws.at<void>(B_X), d, "gemm_o_resid_tc", nullptr, s));
+    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, w.w_o, d, hq, ws.at<float>(B_H),
+                                ws.at<float>(B_X), d, "gemm_o_resid_tc", nullptr, s));
   else
     DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
   DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
                         ws.at<void>(B_Y), s));
-  DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
-                       ws.at<void>(B_Y), w.w_router, token_live, ws.at<int32_t>(B_IDX),
-                       ws.at<float>(B_W), s));
+  if (gemm_tc_supported(c.act_dtype, router_type(&c), d) && c.n_experts % 16 == 0) {
+    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_Y), T, w.w_router, c.n_experts, d, ws.at<float>(B_Z),
+                                nullptr, c.n_experts, "router_logits_tc", nullptr, s));
+    DG_TRY(launch_router_topk(T, c.n_experts, c.top_k, ws.at<float>(B_Z), token_live,
+                              ws.at<int32_t>(B_IDX), ws.at<float>(B_W), s));
+  } else {
+    DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
+                         ws.at<void>(B_Y), w.w_router, token_live, ws.at<int32_t>(B_IDX),
+                         ws.at<float>(B_W), s));
+  }
   DG_TRY(launch_permute(T, c.top_k, c.n_experts, ws.at<int32_t>(B_IDX), ws.at<int32_t>(B_OFF),
                         ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV), s));
   return DG_OK;
@@ -195,11 +209,11 @@ int attn_out_and_moe(const dg_config &c, const dg_layer_weights &w, const Ws &ws
 int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
                 const void *y, const int32_t *topk_idx, const float *topk_w,
                 const int32_t *expert_off, const int32_t *perm, const int32_t *inv_perm,
-                const void *residual, void *out, cudaStream_t s) {
+                const void *residual, void *out, cudaStream_t s, int32_t *load_out = nullptr) {
   const int d = c.d_model, F = c.d_ff, E = c.n_experts, k = c.top_k;
   const int TK = T * k;
   DG_TRY(launch_build_tiles(E, expert_off, TILE_M, ws.at<GroupTile>(B_TILES),
-                            ws.at<int32_t>(B_NTILES), ws.L->max_tiles, s));
+                            ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s));
   if (gemm_tc_supported(c.act_dtype, c.w_dtype, d) && F % 64 == 0 && d % 128 == 0 &&
       experts_tc_tile_tokens() == TILE_M) {
     DG_TRY(launch_gather_rows(TK, d, k, perm, expert_off, E, y, ws.at<void>(B_XP), s));
@@ -234,7 +248,7 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
   g2.tiles = g1.tiles; g2.n_tiles = g1.n_tiles; g2.group_off = expert_off;
   g2.max_tiles = ws.L->max_tiles;
   g2.name = "moe_gemm_down";
-  DG_TRY(launch_gemm_simt(g2, EPI_ACT, ws.at<void>(B_YE), d, nullptr, s));
+  DG_TRY(launch_gemm_simt(g2, EPI_F32, ws.at<void>(B_YE), d, nullptr, s));
   return launch_combine(c.act_dtype, T, d, k, topk_idx, topk_w, inv_perm, ws.at<void>(B_YE),
                         residual, out, s);
 }
@@ -388,8 +402,21 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
   Layout L;
   DG_TRY(check_ws(cfg, 1, n_tokens, 0, ws, ws_bytes, &L));
   const cudaStream_t s = (cudaStream_t)stream;
-  DG_TRY(launch_router(cfg->act_dtype, router_type(cfg), n_tokens, cfg->d_model, cfg->n_experts,
-                       cfg->top_k, y, w_router, token_live, topk_idx, topk_w, s));
+  Ws w{(char *)ws, &L};
+  const int d = cfg->d_model, E = cfg->n_experts;
+  if (gemm_tc_supported(cfg->act_dtype, router_type(cfg), d) && E % 16 == 0) {
+    // the tensor-core router reads whole 128-row tiles: stage y into the padded scratch rows
+    const cudaError_t e = cudaMemcpyAsync(w.at<void>(B_Y), y, (size_t)n_tokens * d * esz(cfg->act_dtype),
+                                          cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return check_launch("dg_moe_route copy");
+    DG_TRY(launch_gemm_tc_dense(w.at<void>(B_Y), n_tokens, w_router, E, d, w.at<float>(B_Z), nullptr,
+                                E, "router_logits_tc", nullptr, s));
+    DG_TRY(launch_router_topk(n_tokens, E, cfg->top_k, w.at<float>(B_Z), token_live, topk_idx,
+                              topk_w, s));
+  } else {
+    DG_TRY(launch_router(cfg->act_dtype, router_type(cfg), n_tokens, d, E, cfg->top_k, y,
+                         w_router, token_live, topk_idx, topk_w, s));
+  }
   return launch_permute(n_tokens, cfg->top_k, cfg->n_experts, topk_idx, expert_off, perm,
                         inv_perm, s);
 }
@@ -486,8 +513,8 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                    uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
                    int max_steps, double gamma, const void *k_cache, const void *v_cache,
                    const int32_t *cache_len, int cache_cap, float *entropy_out,
-                   int32_t *argmax_out, float *logits_dbg, void *ws, size_t ws_bytes,
-                   int32_t *dev_status, void *stream) {
+                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load, void *ws,
+                   size_t ws_bytes, int32_t *dev_status, void *stream) {
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
@@ -528,7 +555,8 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
     DG_TRY(attn_out_and_moe(c, lw, w, T, live, s));
     DG_TRY(moe_experts(c, lw, w, T, w.at<void>(B_Y), w.at<int32_t>(B_IDX), w.at<float>(B_W),
                        w.at<int32_t>(B_OFF), w.at<int32_t>(B_PERM), w.at<int32_t>(B_INV),
-                       w.at<void>(B_H), w.at<void>(B_X), s));
+                       w.at<void>(B_H), w.at<void>(B_X), s,
+                       expert_load ? expert_load + (size_t)l * c.n_experts : nullptr));
   }
   float *ent = entropy_out ? entropy_out : w.at<float>(B_ENT);
   int32_t *am = argmax_out ? argmax_out : w.at<int32_t>(B_AM);

@@ -13,9 +13,11 @@ namespace dg {
 struct GroupTile { int32_t g, m0; };
 
 // ---- rows: embedding, RMSNorm, compaction (k_rows.cu) -----------------------------------
+// x_out: fp32 residual stream rows; a_out: RMSNorm(x) in the activation type.
 int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, const void *emb,
                       int rows, int d, int vocab, double eps, void *x_out, void *a_out,
                       int32_t *st, cudaStream_t s);
+// in: fp32 rows (residual stream); out: activation type.
 int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
                    int max_rows, int d, double eps, void *out, cudaStream_t s);
 // live[b*C+i] = !done[b] && (masked == NULL || masked[b*C+i]); row_idx = positions with live
@@ -41,7 +43,7 @@ struct GemmDesc {
   const char *name;            // label for launch accounting / profiling
 };
 enum EpiKind { EPI_F32 = 0, EPI_ACT = 1, EPI_RESID = 2 };
-// EPI_F32: out fp32 [M][ldo]; EPI_ACT: out act type; EPI_RESID: out = act(acc + res[m][n]).
+// EPI_F32: out fp32 [M][ldo]; EPI_ACT: out act type; EPI_RESID: out = acc + res[m][n] (fp32).
 int launch_gemm_simt(const GemmDesc &g, int epi, void *out, int ldo, const void *res,
                      cudaStream_t s);
 
@@ -75,12 +77,16 @@ int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q
 int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *y,
                   const void *w_router, const uint8_t *token_live, int32_t *topk_idx,
                   float *topk_w, cudaStream_t s);
+// Top-k + gates from fp32 router logits z [T][E] (E <= 256, k <= 32), one warp per token.
+int launch_router_topk(int T, int E, int k, const float *z, const uint8_t *token_live,
+                       int32_t *topk_idx, float *topk_w, cudaStream_t s);
 // Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
 int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s);
-// Grouped-GEMM tile list from expert_off: tiles of tile_m rows, count at *n_tiles.
+// Grouped-GEMM tile list from expert_off: tiles of tile_m rows, count at *n_tiles; the
+// per-expert counts also go to load_out [E] when it is non-null.
 int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *tiles,
-                       int32_t *n_tiles, int max_tiles, cudaStream_t s);
+                       int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s);
 // Scatter rows: dst[row_idx[r]][:] = src[r][:] for r < *n_rows.
 int launch_scatter_rows(const float *src, int width, int max_rows, const int32_t *n_rows,
                         const int32_t *row_idx, float *dst, cudaStream_t s);
@@ -90,7 +96,7 @@ int launch_gather_rows(int rows_max, int d, int k, const int32_t *perm, const in
 // a = act(gelu_tanh(u[:, :F]) * u[:, F:]) for rows < expert_off[E].
 int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *expert_off, int E,
                 void *a, cudaStream_t s);
-// out_t = act(res_t + sum_j w[t][j] Y[inv_perm[t k + j]]).
+// out_t = res_t + sum_j w[t][j] Y[inv_perm[t k + j]]; res, Y and out fp32.
 int launch_combine(int act, int T, int d, int k, const int32_t *topk_idx, const float *topk_w,
                    const int32_t *inv_perm, const void *Y, const void *res, void *out,
                    cudaStream_t s);
@@ -115,10 +121,9 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
 
 // ---- tensor-core GEMMs (k_gemm_tc.cu) -----------------------------------------------------------
 bool gemm_tc_supported(int act, int w, int K);
-// out[M][N] (+ res) = A[M][K] W[N][K]^T; A must have room for roundup(M, 128) rows.
-int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out_f32,
-                         void *out_bf16, const void *res, int ldo, const char *name, int32_t *st,
-                         cudaStream_t s);
+// out[M][N] = A[M][K] W[N][K]^T (+ res[M][N]) in fp32; A has room for roundup(M, 128) rows.
+int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
+                         const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s);
 // Swap-AB expert GEMM over token tiles of experts_tc_tile_tokens() rows.
 int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
                            int n_assign_max, int K, const GroupTile *tiles,

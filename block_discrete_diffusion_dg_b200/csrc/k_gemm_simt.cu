@@ -120,8 +120,8 @@ int run(const GemmDesc &d, int epi, void *out, int ldo, const void *res, cudaStr
   else if (epi == EPI_ACT)
     gemm_simt_kernel<AT, WT, AT, EPI_ACT><<<grid, 256, 0, s>>>(a, (AT *)out, ldo, nullptr);
   else
-    gemm_simt_kernel<AT, WT, AT, EPI_RESID><<<grid, 256, 0, s>>>(a, (AT *)out, ldo,
-                                                                 (const AT *)res);
+    gemm_simt_kernel<AT, WT, float, EPI_RESID><<<grid, 256, 0, s>>>(a, (float *)out, ldo,
+                                                                    (const float *)res);
   return check_launch("gemm_simt");
 }
 

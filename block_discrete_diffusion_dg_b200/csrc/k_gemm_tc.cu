@@ -34,9 +34,8 @@ struct Params {
   int kind, K;
   // dense: M rows (tokens), N columns (channels), tile width bn
   int M, N, m_tiles, bn;
-  float *out_f32;
-  bf16 *out_bf16;
-  const bf16 *res;
+  float *out_f32;        // dense output (fp32)
+  const float *res;      // dense residual (fp32) or null
   int ldo;
   // experts: token tiles (expert, first token) and per-expert row offsets
   const GroupTile *tiles;
@@ -45,7 +44,7 @@ struct Params {
   int w_rows;       // weight rows per expert (2F for gate/up, d for down)
   int F;            // expert FFN width (gate/up half)
   int ld_out;       // row stride of the expert output (F for a, d for Y)
-  bf16 *out;        // a [assignments][F] or Y [assignments][d]
+  void *out;        // gate/up: a [assignments][F] (bf16); down: Y [assignments][d] (fp32)
   int32_t *status;
 };
 
@@ -260,21 +259,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   if (j < nv) o[j] = __uint_as_float(v[j]);
               }
             } else {
-              const bf16 *rs = p.res + (size_t)row * p.ldo + col;
-              bf16 *o = p.out_bf16 + (size_t)row * p.ldo + col;
+              const float *rs = p.res + (size_t)row * p.ldo + col;
+              float *o = p.out_f32 + (size_t)row * p.ldo + col;
+              if (nv == 32) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nv)
-                  o[j] = __float2bfloat16_rn(__uint_as_float(v[j]) + __bfloat162float(rs[j]));
+                for (int j = 0; j < 32; j += 4) {
+                  const float4 rr = *reinterpret_cast<const float4 *>(rs + j);
+                  *reinterpret_cast<float4 *>(o + j) =
+                      make_float4(__uint_as_float(v[j]) + rr.x, __uint_as_float(v[j + 1]) + rr.y,
+                                  __uint_as_float(v[j + 2]) + rr.z, __uint_as_float(v[j + 3]) + rr.w);
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) o[j] = __uint_as_float(v[j]) + rs[j];
+              }
             }
           }
         } else if (p.kind == K_MOE_DOWN) {
           const int ch = x.row0 + r;
+          float *Y = reinterpret_cast<float *>(p.out);
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < nv)
-              p.out[(size_t)(x.col0 + c * 32 + j) * p.ld_out + ch] =
-                  __float2bfloat16_rn(__uint_as_float(v[j]));
+            if (j < nv) Y[(size_t)(x.col0 + c * 32 + j) * p.ld_out + ch] = __uint_as_float(v[j]);
         } else {  // K_MOE_GATE: rows 0-63 gate, 64-127 up of the same channels
           if (q >= 2) {
 #pragma unroll
@@ -290,7 +297,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const float up = xch[(q * 32 + lane) * 33 + j];
               const float gl =
                   0.5f * g * (1.0f + tanhf(0.7978845608028654f * (g + 0.044715f * g * g * g)));
-              p.out[(size_t)(x.col0 + c * 32 + j) * p.ld_out + ch] = __float2bfloat16_rn(gl * up);
+              reinterpret_cast<bf16 *>(p.out)[(size_t)(x.col0 + c * 32 + j) * p.ld_out + ch] =
+                  __float2bfloat16_rn(gl * up);
             }
           }
           epi_bar();
@@ -329,10 +337,9 @@ bool gemm_tc_supported(int act, int w, int K) {
   return act == DG_BF16 && w == DG_BF16 && K % BK == 0 && K >= BK;
 }
 
-// Dense: out[M][N] (+ res) = A[M][K] * W[N][K]^T.  out_f32 xor out_bf16 (with res).
-int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out_f32,
-                         void *out_bf16, const void *res, int ldo, const char *name,
-                         int32_t *st, cudaStream_t s) {
+// Dense: out[M][N] = A[M][K] * W[N][K]^T (+ res[M][N]), fp32 output.
+int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
+                         const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s) {
   constexpr int BN = 64;
   const int M_alloc = (M + BM - 1) / BM * BM;  // A has room for whole tiles (caller's layout)
   CUtensorMap ta, tb;
@@ -342,15 +349,14 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
   rc = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, N, (uint64_t)K * 2, BK, BN);
   if (rc != DG_OK) return rc;
   Params p{};
-  p.kind = out_f32 ? K_DENSE_F32 : K_DENSE_RESID;
+  p.kind = res ? K_DENSE_RESID : K_DENSE_F32;
   p.K = K;
   p.M = M;
   p.N = N;
   p.m_tiles = M_alloc / BM;
   p.bn = BN;
-  p.out_f32 = out_f32;
-  p.out_bf16 = reinterpret_cast<bf16 *>(out_bf16);
-  p.res = reinterpret_cast<const bf16 *>(res);
+  p.out_f32 = out;
+  p.res = res;
   p.ldo = ldo;
   p.status = st;
   const int units = p.m_tiles * ((N + BN - 1) / BN);
@@ -358,7 +364,7 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
 }
 
 // Experts (swap-AB).  gate_up: W [E][2F][K], X = the routed rows [assignments][K] (permuted order)
-// -> a [assignments][F].  down: W [E][d][F], X = a -> Y [assignments][d].
+// -> a [assignments][F] (bf16).  down: W [E][d][F], X = a -> Y [assignments][d] (fp32).
 int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
                            int n_assign_max, int K, const GroupTile *tiles,
                            const int32_t *n_tiles_dev, int max_tiles, const int32_t *expert_off,
@@ -381,9 +387,10 @@ int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F,
   p.F = F;
   p.m_tiles = gate_up ? F / 64 : w_rows / BM;
   p.ld_out = ld_out;
-  p.out = reinterpret_cast<bf16 *>(out);
+  p.out = out;
   p.status = st;
-  return launch<BN_MAX, 8, B_BOX>(ta, tb, p, max_tiles * p.m_tiles, name, s);
+  // 9 stages of 16 KB weights + 8 KB tokens: ~216 KB in flight per SM for the weight stream
+  return launch<BN_MAX, 9, B_BOX>(ta, tb, p, max_tiles * p.m_tiles, name, s);
 }
 
 int experts_tc_tile_tokens() { return 64; }

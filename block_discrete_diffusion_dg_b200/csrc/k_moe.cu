@@ -80,6 +80,51 @@ __global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__
   }
 }
 
+// Top-k and gates from router logits z [T][E] (fp32), one warp per token: the k largest logits
+// (lower expert index first on equal values), gates = softmax over the selected logits.
+__global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict__ z,
+                                   const uint8_t *__restrict__ token_live, int32_t *topk_idx,
+                                   float *topk_w) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T_) return;
+  const bool live = token_live == nullptr || token_live[t] != 0;
+  const float *zr = z + (size_t)t * E;
+  float zv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) zv[i] = (lane + 32 * i < E) ? zr[lane + 32 * i] : -INFINITY;
+  unsigned taken = 0u;
+  float z0 = 0.f, denom = 0.f, mine = 0.f;
+  int my_idx = -1;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !(taken & (1u << i)) && (zv[i] > bv || (zv[i] == bv && e < bi))) {
+        bv = zv[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (j == 0) z0 = bv;
+    const float p = expf(bv - z0);
+    denom += p;
+    if (lane == j) { mine = p; my_idx = bi; }
+  }
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = live ? my_idx : -1;
+    topk_w[(size_t)t * k + lane] = live ? mine / denom : 0.f;
+  }
+}
+
 // Single block of 1024 threads; E <= 256.
 __global__ void __launch_bounds__(1024) permute_kernel(int n_assign, int E,
                                                        const int32_t *__restrict__ topk_idx,
@@ -135,10 +180,14 @@ __global__ void __launch_bounds__(1024) permute_kernel(int n_assign, int E,
 }
 
 // Tile list of the grouped expert GEMMs: for each expert with rows, tiles of tile_m rows.
+// Optionally also stores the per-expert assignment counts (expert load) in load_out [E].
 __global__ void build_tiles_kernel(int E, const int32_t *__restrict__ expert_off, int tile_m,
-                                   GroupTile *tiles, int32_t *n_tiles, int max_tiles) {
+                                   GroupTile *tiles, int32_t *n_tiles, int max_tiles,
+                                   int32_t *load_out) {
   __shared__ int toff[257];
   const int tid = threadIdx.x;
+  if (load_out)
+    for (int e = tid; e < E; e += blockDim.x) load_out[e] = expert_off[e + 1] - expert_off[e];
   if (tid == 0) {
     int acc = 0;
     for (int e = 0; e < E; ++e) {
@@ -183,19 +232,21 @@ __global__ void gate_kernel(int F, const float *__restrict__ u, const int32_t *_
   }
 }
 
-template <typename T>
+// out_t = res_t + sum_j w[t][j] Y[inv_perm[t k + j]] in fp32, slot order j = 0..k-1 (the
+// residual stream and the expert outputs are fp32).
 __global__ void combine_kernel(int d, int k, const int32_t *__restrict__ topk_idx,
                                const float *__restrict__ topk_w, const int32_t *__restrict__ inv_perm,
-                               const T *__restrict__ Y, const T *__restrict__ res, T *out) {
+                               const float *__restrict__ Y, const float *__restrict__ res,
+                               float *out) {
   const int t = blockIdx.x;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float acc = to_f(res[(size_t)t * d + c]);
+    float acc = res[(size_t)t * d + c];
     for (int j = 0; j < k; ++j) {
       const int a = t * k + j;
       if (topk_idx[a] < 0) continue;
-      acc = fmaf(topk_w[a], to_f(Y[(size_t)inv_perm[a] * d + c]), acc);
+      acc = fmaf(topk_w[a], Y[(size_t)inv_perm[a] * d + c], acc);
     }
-    out[(size_t)t * d + c] = from_f<T>(acc);
+    out[(size_t)t * d + c] = acc;
   }
 }
 
@@ -226,6 +277,15 @@ int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void 
   return check_launch("router");
 }
 
+int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *token_live,
+                       int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+  if (T_ <= 0) return DG_OK;
+  if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
+  note_launch(s, "router_topk");
+  router_topk_kernel<<<(T_ + 7) / 8, 256, 0, s>>>(T_, E, k, z, token_live, topk_idx, topk_w);
+  return check_launch("router_topk");
+}
+
 int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s) {
   if (E > 256) return DG_ERR_UNSUPPORTED;
@@ -235,10 +295,10 @@ int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *exper
 }
 
 int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *tiles,
-                       int32_t *n_tiles, int max_tiles, cudaStream_t s) {
+                       int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s) {
   if (E > 256) return DG_ERR_UNSUPPORTED;
   note_launch(s, "build_tiles");
-  build_tiles_kernel<<<1, 256, 0, s>>>(E, expert_off, tile_m, tiles, n_tiles, max_tiles);
+  build_tiles_kernel<<<1, 256, 0, s>>>(E, expert_off, tile_m, tiles, n_tiles, max_tiles, load_out);
   return check_launch("build_tiles");
 }
 
@@ -265,13 +325,10 @@ int launch_combine(int act, int T_, int d, int k, const int32_t *topk_idx, const
                    const int32_t *inv_perm, const void *Y, const void *res, void *out,
                    cudaStream_t s) {
   if (T_ <= 0) return DG_OK;
+  (void)act;
   note_launch(s, "combine");
-  if (act == DG_F32)
-    combine_kernel<float><<<T_, 256, 0, s>>>(d, k, topk_idx, topk_w, inv_perm, (const float *)Y,
-                                             (const float *)res, (float *)out);
-  else
-    combine_kernel<bf16><<<T_, 256, 0, s>>>(d, k, topk_idx, topk_w, inv_perm, (const bf16 *)Y,
-                                            (const bf16 *)res, (bf16 *)out);
+  combine_kernel<<<T_, 256, 0, s>>>(d, k, topk_idx, topk_w, inv_perm, (const float *)Y,
+                                    (const float *)res, (float *)out);
   return check_launch("combine");
 }
 

@@ -1,6 +1,8 @@
 // Row kernels: embedding gather + pre-norm, RMSNorm (optionally over a gathered row list), and
 // the compaction of the positions that need logits this step.
 //
+// The residual stream (embedding rows, layer outputs) is fp32; RMSNorm reads it and writes the
+// normalised rows in the activation type, the input of the next matrix product.
 // RMSNorm(x) = x / sqrt(mean(x^2) + eps), unit gain, computed in fp32 with a fixed-order
 // reduction and rounded once to the activation type (the pre-norm of every layer and the
 // final norm before the LM head; the pages' model is the Gemma 4 transformer,
@@ -14,8 +16,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t *__restrict__ tokens,
                                                          const uint8_t *__restrict__ masked,
                                                          const T *__restrict__ emb, int d,
-                                                         int vocab, float eps, T *x_out, T *a_out,
-                                                         int32_t *st) {
+                                                         int vocab, float eps, float *x_out,
+                                                         T *a_out, int32_t *st) {
   __shared__ float red[8];
   const int row = blockIdx.x;
   int id = (masked && masked[row]) ? vocab : tokens[row];
@@ -31,17 +33,17 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t *__restri
   }
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
-  T *xo = x_out + (size_t)row * d;
+  float *xo = x_out + (size_t)row * d;
   T *ao = a_out + (size_t)row * d;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    T v = src[j];
+    const float v = to_f(src[j]);
     xo[j] = v;
-    ao[j] = from_f<T>(to_f(v) * inv);
+    ao[j] = from_f<T>(v * inv);
   }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const T *__restrict__ in,
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float *__restrict__ in,
                                                       const int32_t *__restrict__ row_idx,
                                                       const int32_t *__restrict__ n_rows_dev,
                                                       int d, float eps, T *out) {
@@ -49,16 +51,16 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T *__restrict__ in,
   const int r = blockIdx.x;
   if (n_rows_dev && r >= *n_rows_dev) return;
   const int src_row = row_idx ? row_idx[r] : r;
-  const T *src = in + (size_t)src_row * d;
+  const float *src = in + (size_t)src_row * d;
   float ss = 0.f;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float v = to_f(src[j]);
+    const float v = src[j];
     ss += v * v;
   }
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
   T *o = out + (size_t)r * d;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f<T>(to_f(src[j]) * inv);
+  for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f<T>(src[j] * inv);
 }
 
 // One block of 1024 threads scans all B*C positions in chunks (B*C <= 65536).
@@ -110,7 +112,7 @@ int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, con
                                                   (float)eps, (float *)x_out, (float *)a_out, st);
   else
     embed_norm_kernel<bf16><<<rows, 256, 0, s>>>(tokens, masked, (const bf16 *)emb, d, vocab,
-                                                 (float)eps, (bf16 *)x_out, (bf16 *)a_out, st);
+                                                 (float)eps, (float *)x_out, (bf16 *)a_out, st);
   return check_launch("embed_norm");
 }
 
@@ -122,7 +124,7 @@ int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_
     rmsnorm_kernel<float><<<max_rows, 256, 0, s>>>((const float *)in, row_idx, n_rows_dev, d,
                                                    (float)eps, (float *)out);
   else
-    rmsnorm_kernel<bf16><<<max_rows, 256, 0, s>>>((const bf16 *)in, row_idx, n_rows_dev, d,
+    rmsnorm_kernel<bf16><<<max_rows, 256, 0, s>>>((const float *)in, row_idx, n_rows_dev, d,
                                                   (float)eps, (bf16 *)out);
   return check_launch("rmsnorm");
 }

@@ -30,6 +30,10 @@
  *     layer-weight element type = cfg->w_dtype (F32, BF16, or E4M3 with one fp32 scale per
  *     output channel).  The K/V cache of one layer is [B][Hkv][cache_cap][hd], the full cache
  *     [L][B][Hkv][cache_cap][hd], both in the activation type.
+ *   - The residual stream (embedding rows, the hidden rows after the attention block and after
+ *     the expert FFN) is fp32 for every activation type; the tensors that feed a matrix product
+ *     or the attention (normalised rows, q, k, v, attention output, expert activations) are in
+ *     the activation type.
  *   - Functions are stateless and may be called from several host threads on different streams.
  */
 #ifndef DG_H
@@ -112,7 +116,8 @@ uint64_t dg_launch_count(void);
  * dg_profile_end synchronises on the last event, writes ms[i] = time from record i to record
  * i + 1 (i < *n_out <= max_out) and stops recording; dg_profile_name(i) is record i's kernel
  * name ("" when out of range).  Events are created once and reused; no device memory is
- * allocated.  Not for use inside CUDA graph capture. */
+ * allocated.  Under stream capture the records become external event-record nodes, so the
+ * times are those of the graph's replay (call dg_profile_end after the replay). */
 int dg_profile_begin(int max_records);
 int dg_profile_mark(void *stream);
 int dg_profile_end(float *ms, int max_out, int *n_out);
@@ -153,10 +158,10 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
 
 /* Expert FFN with combine and residual (same passages).  For assignment (t, j) with expert e:
  *   [g; u] = y_t W_gu,e^T ; a = gelu_tanh(g) * u (stored in the activation type) ;
- *   Y = a W_d,e^T (stored in the activation type) ;
+ *   Y = a W_d,e^T (fp32) ;
  *   out_t = residual_t + sum_j topk_w[t][j] Y_(t,j), summed in fp32 in slot order j = 0..k-1.
- * Routing arrays as produced by dg_moe_route.  y, residual, out [T][d] (out may not alias y;
- * it may alias residual). */
+ * Routing arrays as produced by dg_moe_route.  y [T][d] in the activation type; residual and
+ * out [T][d] fp32 (out may not alias y; it may alias residual). */
 int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t *topk_idx,
                const float *topk_w, const int32_t *expert_off, const int32_t *perm,
                const int32_t *inv_perm, const dg_layer_weights *lw, const void *residual,
@@ -169,7 +174,8 @@ int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t 
  * s = row_idx ? row_idx[r] : r:
  *   f = RMSNorm(h_s) (stored in the activation type);  z = f W_lm^T over ids [0, V) (fp32);
  *   entropy[s] = -sum_v p_v ln p_v with p = softmax(z);  argmax[s] = first index of max z.
- *   h [*][d]; w_lm = the embedding [V + 1][d] (rows [0, V) used); entropy fp32, argmax int32
+ *   h [*][d] fp32 (residual stream); w_lm = the embedding [V + 1][d] in the activation type
+ *   (rows [0, V) used); entropy fp32, argmax int32
  *   indexed by source row; logits_dbg fp32 [n_rows][V] or NULL (written when non-NULL).
  * A non-finite logit sets DG_ERR_NUMERIC. */
 int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_dev,
@@ -217,13 +223,15 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
  * [L][B][Hkv][cache_cap][hd] are read only (the canvas's own K/V live in `ws`).
  * entropy_out fp32 [B][C], argmax_out int32 [B][C] (or NULL): written at the positions that
  * were masked when the step began.  logits_dbg (or NULL): fp32 [B C][V], row b C + i written for
- * each such position (debug and parity only; costs a full logits write). */
+ * each such position (debug and parity only; costs a full logits write).  expert_load (or
+ * NULL): int32 [n_layers][E], the number of (token, slot) assignments each expert received in
+ * each layer this step (for load monitoring and byte accounting). */
 int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
                    uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
                    int max_steps, double gamma, const void *k_cache, const void *v_cache,
                    const int32_t *cache_len, int cache_cap, float *entropy_out,
-                   int32_t *argmax_out, float *logits_dbg, void *ws, size_t ws_bytes,
-                   int32_t *dev_status, void *stream);
+                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load, void *ws,
+                   size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* ---- fixed-scratch entry point ---------------------------------------------------------- */
 

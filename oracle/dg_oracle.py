@@ -23,11 +23,15 @@ What it computes (the method as the pages describe it):
   commit masked positions in ascending entropy while the sum of the chosen
   entropies minus their maximum stays within the bound gamma.
 
-Precision: every product and sum runs in fp64.  Where the workload stores an
-activation in bf16, the oracle rounds the fp64 value to the nearest bf16 at the
-same tensor (x, q, k, v, o, h, y, a, Y, the final normalised rows), so the
-oracle/GPU gap is accumulation-order error, not storage error.  fp32 workloads
-are not rounded at all.
+Precision: every product and sum runs in fp64.  The pages fix no storage
+precision for intermediates; the reading taken is that the tensors that feed a
+bf16 matrix product or the attention are stored in the workload's activation type
+(the normalised rows a, y and f, the attention inputs and output q, k, v, o, and
+the expert activation a), while the residual stream (embedding, h, layer
+outputs) and the expert outputs Y are kept in fp32.  Where the activation type
+is bf16 the oracle rounds the fp64 value to the nearest bf16 at exactly those
+tensors and leaves the others unrounded, so the oracle/GPU gap is
+accumulation-order error, not storage error.  fp32 workloads are not rounded.
 """
 from __future__ import annotations
 
@@ -193,9 +197,9 @@ def moe_ffn(y: np.ndarray, idx: np.ndarray, gates: np.ndarray, expert_w, residua
 
     For token t and slot j with expert e = idx[t, j]:
       [g; u] = y_t W_gu,e^T  (the first d_ff outputs are the gate, the next d_ff the up)
-      a      = gelu_tanh(g) * u                 (stored: rounded)
-      Y      = a W_d,e^T                        (stored: rounded)
-    out_t = residual_t + sum_j gates[t, j] Y_{t,j}          (stored: rounded)
+      a      = gelu_tanh(g) * u                 (stored in the activation type: rounded)
+      Y      = a W_d,e^T                        (fp32 on the device: unrounded)
+    out_t = residual_t + sum_j gates[t, j] Y_{t,j}          (residual stream: unrounded)
     ``expert_w(e)`` returns (W_gu,e [2F, d], W_d,e [d, F]) as fp64.  A slot whose expert id is
     negative has no expert and contributes nothing.
     """
@@ -209,9 +213,9 @@ def moe_ffn(y: np.ndarray, idx: np.ndarray, gates: np.ndarray, expert_w, residua
         F = w_d.shape[1]
         u = y[rows] @ w_gu.T
         a = storage_round(gelu_tanh(u[:, :F]) * u[:, F:], act)
-        Y = storage_round(a @ w_d.T, act)
+        Y = a @ w_d.T
         acc[rows] += gates[rows, slots][:, None] * Y
-    return storage_round(acc, act)
+    return acc
 
 
 def entropy_argmax(z: np.ndarray):
@@ -349,11 +353,13 @@ def layer_qkv(cfg, model: OracleModel, l: int, x: np.ndarray, pos: np.ndarray):
 
 
 def layer_rest(cfg, model: OracleModel, l: int, x, q, k, v, kc, vc, causal: bool, info=None):
-    """Attention, output projection with residual, and the MoE FFN with residual."""
+    """Attention, output projection with residual, and the MoE FFN with residual.
+
+    x and the returned layer output are the residual stream (unrounded)."""
     act = cfg.act
     T = x.shape[0]
     o = storage_round(attention(q, kc, vc, k, v, causal), act).reshape(T, -1)
-    h = storage_round(x + o @ model.w(l, "w_o").T, act)
+    h = x + o @ model.w(l, "w_o").T
     y = storage_round(rmsnorm(h, cfg.rms_eps), act)
     idx, gates, z = router_topk(y, model.w(l, "w_router"), cfg.top_k)
     if info is not None:

@@ -23,7 +23,7 @@ ENT_RTOL = 1e-3
 def _case(cfg, emb, n_all, n_rows, seed):
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
-    h = (torch.randn((n_all, cfg.d_model), generator=g) * 0.07).to(torch.bfloat16).cuda()
+    h = (torch.randn((n_all, cfg.d_model), generator=g) * 0.07).cuda()   # fp32 hidden rows
     rows = torch.sort(torch.randperm(n_all, generator=g)[:n_rows]).values.to(torch.int32).cuda()
     dgc = B.make_config(cfg)
     e_ref = torch.full((n_all,), -1.0, device="cuda")
