@@ -75,10 +75,10 @@ _SIGS = {
     "dg_logits_entropy_static": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dg_eb_select": (_I32, [_I32, _I32, _VP, _VP, ctypes.c_double, _I32, _VP, _VP, _VP, _VP, _VP,
                             _VP, _VP, _VP]),
-    "dg_kv_append": (_I32, [_PCFG, _PMODEL, _I32, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _SZ, _VP,
-                            _VP]),
+    "dg_kv_append": (_I32, [_PCFG, _PMODEL, _I32, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _SZ,
+                            _VP, _VP]),
     "dg_canvas_step": (_I32, [_PCFG, _PMODEL, _I32, _VP, _VP, _VP, _VP, _VP, _I32, ctypes.c_double,
-                              _VP, _VP, _VP, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+                              _VP, _VP, _VP, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
 }
 
 
@@ -245,22 +245,24 @@ def dg_eb_select(batch, canvas, entropy, argmax, gamma, max_steps, tokens, maske
 
 
 def dg_kv_append(cfg, model: Model, batch, tokens, n_tokens, k_cache, v_cache, cache_len, cache_cap,
-                 ws, dev_status=None, stream=None):
+                 ws, dev_status=None, stream=None, forced_topk=None):
     w, wb = _ws(ws)
     _check(lib().dg_kv_append(ctypes.byref(cfg), ctypes.byref(model.struct), batch, _p(tokens),
-                              n_tokens, _p(k_cache), _p(v_cache), _p(cache_len), cache_cap, w, wb,
-                              _p(dev_status), _stream(stream)), "dg_kv_append")
+                              n_tokens, _p(k_cache), _p(v_cache), _p(cache_len), cache_cap,
+                              _p(forced_topk), w, wb, _p(dev_status), _stream(stream)),
+           "dg_kv_append")
 
 
 def dg_canvas_step(cfg, model: Model, batch, tokens, masked, n_masked, done, step, max_steps, gamma,
                    k_cache, v_cache, cache_len, cache_cap, entropy_out, argmax_out, logits_dbg, ws,
-                   dev_status=None, stream=None, expert_load=None):
+                   dev_status=None, stream=None, expert_load=None, forced_topk=None):
     w, wb = _ws(ws)
     _check(lib().dg_canvas_step(ctypes.byref(cfg), ctypes.byref(model.struct), batch, _p(tokens),
                                 _p(masked), _p(n_masked), _p(done), _p(step), max_steps,
                                 float(gamma), _p(k_cache), _p(v_cache), _p(cache_len), cache_cap,
                                 _p(entropy_out), _p(argmax_out), _p(logits_dbg), _p(expert_load),
-                                w, wb, _p(dev_status), _stream(stream)), "dg_canvas_step")
+                                _p(forced_topk), w, wb, _p(dev_status), _stream(stream)),
+           "dg_canvas_step")
 
 
 def exported_symbols() -> Sequence[str]:

@@ -48,14 +48,19 @@ int check_launch(const char *what) {
 
 namespace {
 
-constexpr int TILE_M = 64;  // rows per grouped-GEMM tile
+// Rows per grouped-GEMM tile: the tensor-core expert GEMM's token tile, or the CUDA-core GEMM's
+// 64-row tile; the scratch tile list is sized for the smaller of the two.
+constexpr int SIMT_TILE_M = 64;
+inline int min_tile_m() {
+  return experts_tc_tile_tokens() < SIMT_TILE_M ? experts_tc_tile_tokens() : SIMT_TILE_M;
+}
 
 inline size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
 inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
-  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_LIVE, B_ROWS, B_NROWS, B_FIN, B_LOGITS, B_PART,
+  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_LIVE, B_ROWS, B_NROWS, B_SLOT, B_FIN, B_LOGITS, B_PART,
   B_ENT, B_AM, B_ATTN, B_COUNT
 };
 
@@ -71,7 +76,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   const size_t qkvw = (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * hd;
   const size_t TK = T * k;
   Layout L;
-  L.max_tiles = (int)((TK + TILE_M - 1) / TILE_M) + c.n_experts;
+  L.max_tiles = (int)((TK + min_tile_m() - 1) / min_tile_m()) + c.n_experts;
   size_t sz[B_COUNT];
   const size_t T128 = (T + 127) / 128 * 128;  // tensor-core A operands read whole 128-row tiles
   sz[B_X] = T * d * 4;  // residual stream: fp32
@@ -99,6 +104,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_LIVE] = T;
   sz[B_ROWS] = T * 4;
   sz[B_NROWS] = 4;
+  sz[B_SLOT] = T * 4;
   const bool tc_lm = lmhead_tc_supported(c.act_dtype, c.d_model);
   sz[B_FIN] = T128 * d * a;
   sz[B_LOGITS] = tc_lm ? 0 : T * (size_t)c.vocab * 4;
@@ -173,9 +179,19 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
   return launch_gemm_simt(g, EPI_F32, ws.at<void>(B_QKV), g.N, nullptr, s);
 }
 
-// o -> h = x + o W_o^T -> y = RMSNorm(h) -> router -> permute -> experts -> x
-int attn_out_and_moe(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
-                     const uint8_t *token_live, cudaStream_t s) {
+bool experts_tc(const dg_config &c) {
+  return gemm_tc_supported(c.act_dtype, c.w_dtype, c.d_model) && c.d_ff % 64 == 0 &&
+         c.d_model % 128 == 0;
+}
+bool router_tc(const dg_config &c) {
+  return gemm_tc_supported(c.act_dtype, router_type(&c), c.d_model) && c.n_experts % 16 == 0;
+}
+
+// o -> h = x + o W_o^T -> y = RMSNorm(h) -> router top-k -> stable permutation (+ tile list for the
+// tensor-core experts, built here when the router runs on tensor cores: *tiles_ready).
+int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
+                       const uint8_t *token_live, int32_t *load_out, bool *tiles_ready,
+                       cudaStream_t s, const int32_t *forced = nullptr) {
   const int d = c.d_model, hq = c.n_q_heads * c.head_dim;
   GemmDesc g{};
   g.act = c.act_dtype; g.w = c.w_dtype;
@@ -191,31 +207,43 @@ int attn_out_and_moe(const dg_config &c, const dg_layer_weights &w, const Ws &ws
     DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
   DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
                         ws.at<void>(B_Y), s));
-  if (gemm_tc_supported(c.act_dtype, router_type(&c), d) && c.n_experts % 16 == 0) {
+  *tiles_ready = false;
+  if (router_tc(c)) {
     DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_Y), T, w.w_router, c.n_experts, d, ws.at<float>(B_Z),
                                 nullptr, c.n_experts, "router_logits_tc", nullptr, s));
-    DG_TRY(launch_router_topk(T, c.n_experts, c.top_k, ws.at<float>(B_Z), token_live,
-                              ws.at<int32_t>(B_IDX), ws.at<float>(B_W), s));
-  } else {
-    DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
-                         ws.at<void>(B_Y), w.w_router, token_live, ws.at<int32_t>(B_IDX),
-                         ws.at<float>(B_W), s));
+    const bool tc = experts_tc(c);
+    DG_TRY(launch_route(T, c.n_experts, c.top_k, ws.at<float>(B_Z), token_live,
+                        ws.at<int32_t>(B_IDX), ws.at<float>(B_W), ws.at<int32_t>(B_OFF),
+                        ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV),
+                        tc ? experts_tc_tile_tokens() : SIMT_TILE_M, ws.at<GroupTile>(B_TILES),
+                        ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s, forced));
+    *tiles_ready = true;
+    return DG_OK;
   }
-  DG_TRY(launch_permute(T, c.top_k, c.n_experts, ws.at<int32_t>(B_IDX), ws.at<int32_t>(B_OFF),
-                        ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV), s));
-  return DG_OK;
+  if (forced) return DG_ERR_UNSUPPORTED;  // forced routing needs the tensor-core router
+  DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
+                       ws.at<void>(B_Y), w.w_router, token_live, ws.at<int32_t>(B_IDX),
+                       ws.at<float>(B_W), s));
+  return launch_permute(T, c.top_k, c.n_experts, ws.at<int32_t>(B_IDX), ws.at<int32_t>(B_OFF),
+                        ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV), s);
 }
 
+// The expert FFN, then combine + residual into `out`; the combine also writes RMSNorm(out) to
+// a_out (next layer's input) and/or to f_out rows slot[t] (final-norm rows), when given.
 int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
                 const void *y, const int32_t *topk_idx, const float *topk_w,
                 const int32_t *expert_off, const int32_t *perm, const int32_t *inv_perm,
-                const void *residual, void *out, cudaStream_t s, int32_t *load_out = nullptr) {
+                const void *residual, void *out, cudaStream_t s, bool tiles_ready = false,
+                int32_t *load_out = nullptr, void *a_out = nullptr,
+                const int32_t *slot = nullptr, void *f_out = nullptr) {
   const int d = c.d_model, F = c.d_ff, E = c.n_experts, k = c.top_k;
   const int TK = T * k;
-  DG_TRY(launch_build_tiles(E, expert_off, TILE_M, ws.at<GroupTile>(B_TILES),
-                            ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s));
-  if (gemm_tc_supported(c.act_dtype, c.w_dtype, d) && F % 64 == 0 && d % 128 == 0 &&
-      experts_tc_tile_tokens() == TILE_M) {
+  const bool tc = experts_tc(c);
+  if (!tiles_ready)
+    DG_TRY(launch_build_tiles(E, expert_off, tc ? experts_tc_tile_tokens() : SIMT_TILE_M,
+                              ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
+                              ws.L->max_tiles, load_out, s));
+  if (tc) {
     DG_TRY(launch_gather_rows(TK, d, k, perm, expert_off, E, y, ws.at<void>(B_XP), s));
     DG_TRY(launch_gemm_tc_experts(1, w.w_gate_up, E, 2 * F, F, ws.at<void>(B_XP), TK, d,
                                   ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
@@ -225,41 +253,42 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
                                   ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
                                   ws.L->max_tiles, expert_off, ws.at<void>(B_YE), d,
                                   "moe_down_tc", nullptr, s));
-    return launch_combine(c.act_dtype, T, d, k, topk_idx, topk_w, inv_perm, ws.at<void>(B_YE),
-                          residual, out, s);
+  } else {
+    GemmDesc g1{};
+    g1.act = c.act_dtype; g1.w = c.w_dtype;
+    g1.A = y; g1.lda = d; g1.a_rowmap = perm; g1.a_rowdiv = k;
+    g1.B = w.w_gate_up; g1.ldb = d; g1.strideB = (long long)2 * F * d;
+    g1.bscale = scale_or_null(&c, w.s_gate_up);
+    g1.M = TK; g1.N = 2 * F; g1.K = d;
+    g1.tiles = ws.at<GroupTile>(B_TILES); g1.n_tiles = ws.at<int32_t>(B_NTILES);
+    g1.group_off = expert_off; g1.max_tiles = ws.L->max_tiles;
+    g1.name = "moe_gemm_gate_up";
+    DG_TRY(launch_gemm_simt(g1, EPI_F32, ws.at<void>(B_U), 2 * F, nullptr, s));
+    DG_TRY(launch_gate(c.act_dtype, TK, F, ws.at<float>(B_U), expert_off, E, ws.at<void>(B_ACT), s));
+    GemmDesc g2{};
+    g2.act = c.act_dtype; g2.w = c.w_dtype;
+    g2.A = ws.at<void>(B_ACT); g2.lda = F;
+    g2.B = w.w_down; g2.ldb = F; g2.strideB = (long long)d * F;
+    g2.bscale = scale_or_null(&c, w.s_down);
+    g2.M = TK; g2.N = d; g2.K = F;
+    g2.tiles = g1.tiles; g2.n_tiles = g1.n_tiles; g2.group_off = expert_off;
+    g2.max_tiles = ws.L->max_tiles;
+    g2.name = "moe_gemm_down";
+    DG_TRY(launch_gemm_simt(g2, EPI_F32, ws.at<void>(B_YE), d, nullptr, s));
   }
-  GemmDesc g1{};
-  g1.act = c.act_dtype; g1.w = c.w_dtype;
-  g1.A = y; g1.lda = d; g1.a_rowmap = perm; g1.a_rowdiv = k;
-  g1.B = w.w_gate_up; g1.ldb = d; g1.strideB = (long long)2 * F * d;
-  g1.bscale = scale_or_null(&c, w.s_gate_up);
-  g1.M = TK; g1.N = 2 * F; g1.K = d;
-  g1.tiles = ws.at<GroupTile>(B_TILES); g1.n_tiles = ws.at<int32_t>(B_NTILES);
-  g1.group_off = expert_off; g1.max_tiles = ws.L->max_tiles;
-  g1.name = "moe_gemm_gate_up";
-  DG_TRY(launch_gemm_simt(g1, EPI_F32, ws.at<void>(B_U), 2 * F, nullptr, s));
-  DG_TRY(launch_gate(c.act_dtype, TK, F, ws.at<float>(B_U), expert_off, E, ws.at<void>(B_ACT), s));
-  GemmDesc g2{};
-  g2.act = c.act_dtype; g2.w = c.w_dtype;
-  g2.A = ws.at<void>(B_ACT); g2.lda = F;
-  g2.B = w.w_down; g2.ldb = F; g2.strideB = (long long)d * F;
-  g2.bscale = scale_or_null(&c, w.s_down);
-  g2.M = TK; g2.N = d; g2.K = F;
-  g2.tiles = g1.tiles; g2.n_tiles = g1.n_tiles; g2.group_off = expert_off;
-  g2.max_tiles = ws.L->max_tiles;
-  g2.name = "moe_gemm_down";
-  DG_TRY(launch_gemm_simt(g2, EPI_F32, ws.at<void>(B_YE), d, nullptr, s));
-  return launch_combine(c.act_dtype, T, d, k, topk_idx, topk_w, inv_perm, ws.at<void>(B_YE),
-                        residual, out, s);
+  return launch_combine_norm(c.act_dtype, T, d, k, c.rms_eps, topk_idx, topk_w, inv_perm,
+                             ws.at<void>(B_YE), residual, out, a_out, slot, f_out, s);
 }
 
 // Final RMSNorm of rows row_idx[r] (r < *n_rows) of h, LM head, entropy/argmax at source rows.
+// (h == nullptr: the normalised rows are already in the B_FIN scratch rows.)
 int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_rows_dev,
                const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
                int32_t *argmax, float *logits_out, int scatter_logits, int32_t *st,
                cudaStream_t s) {
-  DG_TRY(launch_rmsnorm(c.act_dtype, h, row_idx, n_rows_dev, max_rows, c.d_model, c.rms_eps,
-                        ws.at<void>(B_FIN), s));
+  if (h)
+    DG_TRY(launch_rmsnorm(c.act_dtype, h, row_idx, n_rows_dev, max_rows, c.d_model, c.rms_eps,
+                          ws.at<void>(B_FIN), s));
   if (lmhead_tc_supported(c.act_dtype, c.d_model))
     return launch_lmhead_tc(ws.at<void>(B_FIN), max_rows, n_rows_dev, w_lm, c.vocab, c.d_model,
                             row_idx, entropy, argmax, logits_out,
@@ -465,7 +494,8 @@ int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *arg
 
 int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
                  int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
-                 void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+                 const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+                 void *stream) {
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || n_tokens <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !k_cache || !v_cache || !cache_len || cache_cap <= 0) return DG_ERR_INVALID_ARG;
@@ -480,17 +510,14 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
   const int T = batch * n_tokens, d = c.d_model;
   const size_t layer_elems = (size_t)batch * c.n_kv_heads * cache_cap * c.head_dim;
   const size_t ae = esz(c.act_dtype);
-  DG_TRY(launch_embed_norm(c.act_dtype, tokens, nullptr, model->emb, T, d, c.vocab, c.rms_eps,
-                           w.at<void>(B_X), w.at<void>(B_A), dev_status, s));
-  DG_TRY(launch_rope_table(batch, n_tokens, c.head_dim, c.rope_theta, cache_len,
-                           w.at<float>(B_CS), s));
+  DG_TRY(launch_prologue(c.act_dtype, tokens, nullptr, model->emb, T, d, c.vocab, c.rms_eps,
+                         w.at<void>(B_X), w.at<void>(B_A), dev_status, batch, n_tokens, c.head_dim,
+                         c.rope_theta, cache_len, w.at<float>(B_CS), nullptr, nullptr, nullptr,
+                         nullptr, nullptr, s));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights &lw = model->layers[l];
     char *kc = (char *)k_cache + l * layer_elems * ae;
     char *vc = (char *)v_cache + l * layer_elems * ae;
-    if (l > 0)
-      DG_TRY(launch_rmsnorm(c.act_dtype, w.at<void>(B_X), nullptr, nullptr, T, d, c.rms_eps,
-                            w.at<void>(B_A), s));
     DG_TRY(qkv_proj(c, lw, w, T, s));
     DG_TRY(launch_qkv_split(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
                             w.at<float>(B_QKV), w.at<float>(B_CS), w.at<void>(B_Q),
@@ -501,10 +528,14 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
                             w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
                             w.at<void>(B_VN), 1, nullptr, w.at<void>(B_O),
                             w.at<void>(B_ATTN), s));
-    DG_TRY(attn_out_and_moe(c, lw, w, T, nullptr, s));
+    bool tiles_ready = false;
+    DG_TRY(attn_out_and_route(c, lw, w, T, nullptr, nullptr, &tiles_ready, s,
+                              forced_topk ? forced_topk + (size_t)l * T * c.top_k : nullptr));
+    // the combine also forms the next layer's normalised input
     DG_TRY(moe_experts(c, lw, w, T, w.at<void>(B_Y), w.at<int32_t>(B_IDX), w.at<float>(B_W),
                        w.at<int32_t>(B_OFF), w.at<int32_t>(B_PERM), w.at<int32_t>(B_INV),
-                       w.at<void>(B_H), w.at<void>(B_X), s));
+                       w.at<void>(B_H), w.at<void>(B_X), s, tiles_ready, nullptr,
+                       w.at<void>(B_A)));
   }
   return launch_add_cache_len(batch, n_tokens, cache_cap, cache_len, s);
 }
@@ -513,8 +544,9 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                    uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
                    int max_steps, double gamma, const void *k_cache, const void *v_cache,
                    const int32_t *cache_len, int cache_cap, float *entropy_out,
-                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load, void *ws,
-                   size_t ws_bytes, int32_t *dev_status, void *stream) {
+                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load,
+                   const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+                   void *stream) {
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
@@ -533,17 +565,15 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
   uint8_t *live = w.at<uint8_t>(B_LIVE);
   int32_t *rows = w.at<int32_t>(B_ROWS), *n_rows = w.at<int32_t>(B_NROWS);
 
-  DG_TRY(launch_compact_rows(batch, C, masked, done, rows, n_rows, live, s));
-  DG_TRY(launch_embed_norm(c.act_dtype, tokens, masked, model->emb, T, d, c.vocab, c.rms_eps,
-                           w.at<void>(B_X), w.at<void>(B_A), dev_status, s));
-  DG_TRY(launch_rope_table(batch, C, c.head_dim, c.rope_theta, cache_len, w.at<float>(B_CS), s));
+  int32_t *slot = w.at<int32_t>(B_SLOT);
+  DG_TRY(launch_prologue(c.act_dtype, tokens, masked, model->emb, T, d, c.vocab, c.rms_eps,
+                         w.at<void>(B_X), w.at<void>(B_A), dev_status, batch, C, c.head_dim,
+                         c.rope_theta, cache_len, w.at<float>(B_CS), done, rows, n_rows, slot, live,
+                         s));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights &lw = model->layers[l];
     const char *kc = (const char *)k_cache + l * layer_elems * ae;
     const char *vc = (const char *)v_cache + l * layer_elems * ae;
-    if (l > 0)
-      DG_TRY(launch_rmsnorm(c.act_dtype, w.at<void>(B_X), nullptr, nullptr, T, d, c.rms_eps,
-                            w.at<void>(B_A), s));
     DG_TRY(qkv_proj(c, lw, w, T, s));
     DG_TRY(launch_qkv_split(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,
                             w.at<float>(B_QKV), w.at<float>(B_CS), w.at<void>(B_Q),
@@ -552,15 +582,22 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
     DG_TRY(launch_attention(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,
                             w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
                             w.at<void>(B_VN), 0, done, w.at<void>(B_O), w.at<void>(B_ATTN), s));
-    DG_TRY(attn_out_and_moe(c, lw, w, T, live, s));
+    int32_t *load_l = expert_load ? expert_load + (size_t)l * c.n_experts : nullptr;
+    bool tiles_ready = false;
+    DG_TRY(attn_out_and_route(c, lw, w, T, live, load_l, &tiles_ready, s,
+                              forced_topk ? forced_topk + (size_t)l * T * c.top_k : nullptr));
+    // the combine also forms the next layer's normalised input, or after the last layer the
+    // final-norm rows of the masked positions (the LM head's input)
+    const bool last = l + 1 == c.n_layers;
     DG_TRY(moe_experts(c, lw, w, T, w.at<void>(B_Y), w.at<int32_t>(B_IDX), w.at<float>(B_W),
                        w.at<int32_t>(B_OFF), w.at<int32_t>(B_PERM), w.at<int32_t>(B_INV),
-                       w.at<void>(B_H), w.at<void>(B_X), s,
-                       expert_load ? expert_load + (size_t)l * c.n_experts : nullptr));
+                       w.at<void>(B_H), w.at<void>(B_X), s, tiles_ready, load_l,
+                       last ? nullptr : w.at<void>(B_A), last ? slot : nullptr,
+                       last ? w.at<void>(B_FIN) : nullptr));
   }
   float *ent = entropy_out ? entropy_out : w.at<float>(B_ENT);
   int32_t *am = argmax_out ? argmax_out : w.at<int32_t>(B_AM);
-  DG_TRY(lm_entropy(c, w, T, n_rows, w.at<void>(B_X), rows, model->emb, ent, am, logits_dbg, 1,
+  DG_TRY(lm_entropy(c, w, T, n_rows, nullptr, rows, model->emb, ent, am, logits_dbg, 1,
                     dev_status, s));
   return launch_eb_select(batch, C, ent, am, quant_gamma(gamma), max_steps, tokens, masked,
                           nullptr, n_masked, done, step, dev_status, s);

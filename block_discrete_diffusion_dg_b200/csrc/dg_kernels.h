@@ -17,6 +17,13 @@ struct GroupTile { int32_t g, m0; };
 int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, const void *emb,
                       int rows, int d, int vocab, double eps, void *x_out, void *a_out,
                       int32_t *st, cudaStream_t s);
+// Embedding + pre-norm of `rows` rows, the RoPE table, and (row_idx non-null) the compaction of
+// the rows needing logits (row_idx, *n_rows, slot [rows]: index in row_idx or -1, token_live).
+int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const void *emb, int rows,
+                    int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
+                    int n, int hd, double theta, const int32_t *cache_len, float *cs,
+                    const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
+                    uint8_t *token_live, cudaStream_t s);
 // in: fp32 rows (residual stream); out: activation type.
 int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
                    int max_rows, int d, double eps, void *out, cudaStream_t s);
@@ -67,7 +74,7 @@ int launch_attention(int act, int batch, int n, int Hq, int Hkv, int hd, const v
 size_t attention_ws_bytes(int act, int batch, int n, int Hq, int Hkv, int hd, int cap);
 // bf16 tensor-core path (k_attn_tc.cu): split-KV flash attention + merge.
 bool attention_tc_supported(int act, int Hq, int Hkv, int hd);
-size_t attention_tc_ws_bytes(int batch, int n, int Hq, int hd, int cap);
+size_t attention_tc_ws_bytes(int batch, int n, int Hq, int Hkv, int hd, int cap);
 int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q,
                         const void *k_cache, const void *v_cache, const int32_t *cache_len, int cap,
                         const void *k_new, const void *v_new, int causal, const int32_t *done,
@@ -79,7 +86,14 @@ int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *
                   float *topk_w, cudaStream_t s);
 // Top-k + gates from fp32 router logits z [T][E] (E <= 256, k <= 32), one warp per token.
 int launch_router_topk(int T, int E, int k, const float *z, const uint8_t *token_live,
-                       int32_t *topk_idx, float *topk_w, cudaStream_t s);
+                       int32_t *topk_idx, float *topk_w, cudaStream_t s,
+                       const int32_t *forced = nullptr);
+// Top-k + gates (router_topk, many blocks), then the stable permutation and the tile list in one
+// block (permute_tiles).
+int launch_route(int T, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
+                 float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
+                 GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
+                 cudaStream_t s, const int32_t *forced = nullptr);
 // Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
 int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s);
@@ -96,6 +110,13 @@ int launch_gather_rows(int rows_max, int d, int k, const int32_t *perm, const in
 // a = act(gelu_tanh(u[:, :F]) * u[:, F:]) for rows < expert_off[E].
 int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *expert_off, int E,
                 void *a, cudaStream_t s);
+// Combine and the following RMSNorm: out (fp32 residual stream) as launch_combine; then
+// RMSNorm(out_t) in the activation type to a_out[t] (if non-null) and to f_out[slot[t]] (if
+// slot non-null and slot[t] >= 0).
+int launch_combine_norm(int act, int T, int d, int k, double eps, const int32_t *topk_idx,
+                        const float *topk_w, const int32_t *inv_perm, const void *Y,
+                        const void *res, void *out, void *a_out, const int32_t *slot, void *f_out,
+                        cudaStream_t s);
 // out_t = res_t + sum_j w[t][j] Y[inv_perm[t k + j]]; res, Y and out fp32.
 int launch_combine(int act, int T, int d, int k, const int32_t *topk_idx, const float *topk_w,
                    const int32_t *inv_perm, const void *Y, const void *res, void *out,

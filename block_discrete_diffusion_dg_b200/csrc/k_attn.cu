@@ -156,8 +156,9 @@ int run(int hd, dim3 grid, cudaStream_t s, int n, int Hq, int Hkv, const void *q
 }  // namespace
 
 size_t attention_ws_bytes(int act, int batch, int n, int Hq, int Hkv, int hd, int cap) {
-  return attention_tc_supported(act, Hq, Hkv, hd) ? attention_tc_ws_bytes(batch, n, Hq, hd, cap)
-                                                  : 0;
+  return attention_tc_supported(act, Hq, Hkv, hd)
+             ? attention_tc_ws_bytes(batch, n, Hq, Hkv, hd, cap)
+             : 0;
 }
 
 int launch_attention(int act, int batch, int n, int Hq, int Hkv, int hd, const void *q,

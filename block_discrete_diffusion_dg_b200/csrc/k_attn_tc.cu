@@ -3,13 +3,13 @@
 // canvas and to the cached context (cross-attention to the KV cache); the causal encoder of the
 // append attends causally within the new tokens.  Model card "diffusiongemma", Model Overview.
 //
-// One CTA = 64 query rows that share one kv head: the rep = Hq / Hkv query heads of that kv head
-// times 64 / rep consecutive canvas positions, so every K/V tile is read once per GQA group.
+// One CTA = 128 query rows that share one kv head: the rep = Hq / Hkv query heads of that kv head
+// times 128 / rep consecutive canvas positions, so every K/V tile is read once per GQA group.
 // Keys are split into chunks (split-KV) so that short and 131k-key contexts both fill the GPU;
 // each split leaves an unnormalised partial (O, running max m, sum l) that lm-style merging
 // combines exactly:  m = max m_s, l = sum l_s 2^(m_s - m), O = sum O_s 2^(m_s - m) / l.
 // Scores are kept in the log2 domain: t = q.k / sqrt(hd) * log2(e).
-// 4 warps x 16 rows; K/V tiles of 64 keys double-buffered with cp.async (zero-filled past the end)
+// 8 warps x 16 rows; K/V tiles of 64 keys double-buffered with cp.async (zero-filled past the end)
 // in XOR-swizzled shared memory read by ldmatrix.
 // Precision: S = Q K^T takes the stored bf16 q and k exactly.  The second product takes P and V
 // in fp16: P in [0, 1] keeps 11 significant bits instead of bf16's 8 (the rounding of P is the
@@ -18,15 +18,15 @@
 // Each thread converts the V chunks it loaded, in place, once they have landed.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
+#include "tc_host.h"
 
 namespace dg {
 
 namespace {
 
-constexpr int ROWS = 64;     // query rows per CTA
+constexpr int ROWS = 128;    // query rows per CTA
 constexpr int KT = 64;       // keys per tile
-constexpr int NTHR = 128;    // 4 warps
-constexpr int MIN_KEYS_PER_SPLIT = 512;
+constexpr int NTHR = 256;    // 8 warps x 16 rows
 constexpr int MAX_SPLITS = 64;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -311,36 +311,49 @@ __global__ void __launch_bounds__(NTHR) attn_tc_kernel(AttnArgs a) {
   }
 }
 
-// One block per (batch, head, position): merge the splits in order.
+// One warp per (batch, head, position): merge the splits in order; lanes cover head_dim with
+// float4 loads.
 template <int HD>
 __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float *__restrict__ part_o,
                                   const float2 *__restrict__ part_ml,
                                   const int32_t *__restrict__ done, bf16 *out) {
-  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= B * Hq * n) return;
+  const int i = w % n, h = (w / n) % Hq, b = w / (n * Hq);
   if (done && done[b]) return;
   float m = -INFINITY;
-  for (int s = 0; s < splits; ++s)
-    m = fmaxf(m, part_ml[(((size_t)s * B + b) * Hq + h) * n + i].x);
+  for (int s = 0; s < splits; ++s) m = fmaxf(m, part_ml[(((size_t)s * B + b) * Hq + h) * n + i].x);
   const float base = m == -INFINITY ? 0.f : m;
   float l = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < splits; ++s) {
-    const float2 ml = part_ml[(((size_t)s * B + b) * Hq + h) * n + i];
-    l += ml.y * exp2f(ml.x - base);
+    const size_t r = (((size_t)s * B + b) * Hq + h) * n + i;
+    const float2 ml = part_ml[r];
+    const float c = exp2f(ml.x - base);
+    l += ml.y * c;
+    if (lane * 4 < HD) {
+      const float4 v = reinterpret_cast<const float4 *>(part_o + r * HD)[lane];
+      acc.x += v.x * c; acc.y += v.y * c; acc.z += v.z * c; acc.w += v.w * c;
+    }
   }
   const float il = l > 0.f ? 1.f / l : 0.f;
-  for (int c = threadIdx.x; c < HD; c += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const size_t r = (((size_t)s * B + b) * Hq + h) * n + i;
-      acc += part_o[r * HD + c] * exp2f(part_ml[r].x - base);
-    }
-    out[(((size_t)b * n + i) * Hq + h) * HD + c] = __float2bfloat16_rn(acc * il);
+  if (lane * 4 < HD) {
+    bf16 *o = out + (((size_t)b * n + i) * Hq + h) * HD + lane * 4;
+    *reinterpret_cast<__nv_bfloat162 *>(o) = __floats2bfloat162_rn(acc.x * il, acc.y * il);
+    *reinterpret_cast<__nv_bfloat162 *>(o + 2) = __floats2bfloat162_rn(acc.z * il, acc.w * il);
   }
 }
 
-void plan(int n, int cap, int *splits, int *chunk) {
+// Split-KV plan: as many key splits as fill one wave of CTAs (one CTA per SM at this kernel's
+// register use), at least one tile of keys per split, at most MAX_SPLITS.
+void plan(int batch, int n, int Hq, int Hkv, int cap, int *splits, int *chunk) {
   const int keys = cap + n;
-  int s = (keys + MIN_KEYS_PER_SPLIT - 1) / MIN_KEYS_PER_SPLIT;
+  const int qpc = ROWS / (Hq / Hkv);
+  const int base = ((n + qpc - 1) / qpc) * Hkv * batch;
+  int s = num_sms() / (base > 0 ? base : 1);
+  const int max_by_keys = (keys + KT - 1) / KT;
+  if (s > max_by_keys) s = max_by_keys;
   if (s > MAX_SPLITS) s = MAX_SPLITS;
   if (s < 1) s = 1;
   int c = (keys + s - 1) / s;
@@ -356,9 +369,9 @@ bool attention_tc_supported(int act, int Hq, int Hkv, int hd) {
   return act == DG_BF16 && (hd == 64 || hd == 128) && rep >= 1 && rep <= 64 && (ROWS % rep) == 0;
 }
 
-size_t attention_tc_ws_bytes(int batch, int n, int Hq, int hd, int cap) {
+size_t attention_tc_ws_bytes(int batch, int n, int Hq, int Hkv, int hd, int cap) {
   int s, c;
-  plan(n, cap, &s, &c);
+  plan(batch, n, Hq, Hkv, cap, &s, &c);
   if (s == 1) return 0;
   const size_t rows = (size_t)s * batch * Hq * n;
   return rows * hd * 4 + 256 + rows * sizeof(float2);
@@ -381,7 +394,7 @@ int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q
   a.Hkv = Hkv;
   a.cap = cap;
   a.causal = causal;
-  plan(n, cap, &a.splits, &a.chunk);
+  plan(batch, n, Hq, Hkv, cap, &a.splits, &a.chunk);
   a.out = (bf16 *)out;
   const size_t rows = (size_t)a.splits * batch * Hq * n;
   a.part_o = (float *)ws;
@@ -402,13 +415,14 @@ int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q
   int rc = check_launch("attn_tc");
   if (rc != DG_OK || a.splits == 1) return rc;
   note_launch(s, "attn_merge");
-  dim3 mg(n, Hq, batch);
+  const int warps = batch * Hq * n;
+  const int mgrid = (warps + 7) / 8;
   if (hd == 128)
-    attn_merge_kernel<128><<<mg, 128, 0, s>>>(a.splits, batch, Hq, n, a.part_o, a.part_ml, done,
-                                              (bf16 *)out);
+    attn_merge_kernel<128><<<mgrid, 256, 0, s>>>(a.splits, batch, Hq, n, a.part_o, a.part_ml,
+                                                 done, (bf16 *)out);
   else
-    attn_merge_kernel<64><<<mg, 64, 0, s>>>(a.splits, batch, Hq, n, a.part_o, a.part_ml, done,
-                                            (bf16 *)out);
+    attn_merge_kernel<64><<<mgrid, 256, 0, s>>>(a.splits, batch, Hq, n, a.part_o, a.part_ml, done,
+                                                (bf16 *)out);
   return check_launch("attn_merge");
 }
 

@@ -104,7 +104,9 @@ template <int BN_MAX, int STAGES>
 struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN_MAX * BK * 2;
-  static constexpr uint32_t TMEM_COLS = 2 * BN_MAX < 32 ? 32 : 2 * BN_MAX;
+  // accumulators are read in chunks of 32 columns, so each buffer spans at least 32
+  static constexpr int ACC_STRIDE = BN_MAX < 32 ? 32 : BN_MAX;
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
   static constexpr int XCH_BYTES = 64 * 33 * 4;  // gate/up exchange: 64 rows x 32 columns
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + XCH_BYTES + 256;
 };
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t idesc = idesc_bf16(BM, x.n_mma);
         if (!mbar_wait(&tempty[acc], aph ^ 1)) { fail(p.status, abort_flag); break; }
         fence_after();
-        const uint32_t d = tmem + acc * BN_MAX;
+        const uint32_t d = tmem + acc * C::ACC_STRIDE;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full[stage], ph)) { fail(p.status, abort_flag); ok = false; break; }
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Unit x = decode<BN_MAX>(p, u);
       if (!mbar_wait(&tfull[acc], aph)) { fail(p.status, abort_flag); break; }
       fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE);
       const int r = q * 32 + lane;  // accumulator row of this thread
 #pragma unroll 1
       for (int c = 0; c * 32 < x.n_valid; ++c) {
@@ -320,11 +322,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int BN_MAX, int STAGES, int B_BOX>
 int launch(const CUtensorMap &tmA, const CUtensorMap &tmB, const Params &p, int units_max,
-           const char *name, cudaStream_t s) {
+           const char *name, cudaStream_t s, int ctas_per_sm = 1) {
   using C = Cfg<BN_MAX, STAGES>;
   auto k = gemm_tc_kernel<BN_MAX, STAGES, B_BOX>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  const int grid = units_max < num_sms() ? units_max : num_sms();
+  const int slots = num_sms() * ctas_per_sm;
+  const int grid = units_max < slots ? units_max : slots;
   if (grid <= 0) return DG_OK;
   note_launch(s, name);
   k<<<grid, NUM_THREADS, C::SMEM, s>>>(tmA, tmB, p);
@@ -337,10 +340,12 @@ bool gemm_tc_supported(int act, int w, int K) {
   return act == DG_BF16 && w == DG_BF16 && K % BK == 0 && K >= BK;
 }
 
-// Dense: out[M][N] = A[M][K] * W[N][K]^T (+ res[M][N]), fp32 output.
+// Dense: out[M][N] = A[M][K] * W[N][K]^T (+ res[M][N]), fp32 output.  At batch 1 these are
+// latency-bound weight streams (M = 256 tokens), so the channel tiles are narrow (32, or 16 for
+// N <= 256) to spread each weight matrix over enough CTAs.
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
                          const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s) {
-  constexpr int BN = 64;
+  const int BN = N <= 256 ? 16 : 64;
   const int M_alloc = (M + BM - 1) / BM * BM;  // A has room for whole tiles (caller's layout)
   CUtensorMap ta, tb;
   int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M_alloc, (uint64_t)K * 2, BK,
@@ -360,16 +365,29 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
   p.ldo = ldo;
   p.status = st;
   const int units = p.m_tiles * ((N + BN - 1) / BN);
-  return launch<BN, 8, BN>(ta, tb, p, units, name, s);
+  if (BN == 16) return launch<16, 10, 16>(ta, tb, p, units, name, s);
+  return launch<64, 8, 64>(ta, tb, p, units, name, s);
 }
 
 // Experts (swap-AB).  gate_up: W [E][2F][K], X = the routed rows [assignments][K] (permuted order)
 // -> a [assignments][F] (bf16).  down: W [E][d][F], X = a -> Y [assignments][d] (fp32).
+// Token tile of the expert GEMMs and the depth of their shared-memory ring (weights stream through
+// STAGES x 16 KB; the routed tokens take BN_MAX x 128 bytes per stage).
+#ifndef DG_MOE_BN
+#define DG_MOE_BN 64
+#endif
+#ifndef DG_MOE_STAGES
+#define DG_MOE_STAGES 4
+#endif
+#ifndef DG_MOE_CTAS_PER_SM
+#define DG_MOE_CTAS_PER_SM 2
+#endif
+
 int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
                            int n_assign_max, int K, const GroupTile *tiles,
                            const int32_t *n_tiles_dev, int max_tiles, const int32_t *expert_off,
                            void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s) {
-  constexpr int BN_MAX = 64, B_BOX = 32;
+  constexpr int BN_MAX = DG_MOE_BN, B_BOX = 32;
   CUtensorMap ta, tb;
   int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, (uint64_t)E * w_rows,
                         (uint64_t)K * 2, BK, gate_up ? 64 : BM);
@@ -389,10 +407,10 @@ int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F,
   p.ld_out = ld_out;
   p.out = out;
   p.status = st;
-  // 9 stages of 16 KB weights + 8 KB tokens: ~216 KB in flight per SM for the weight stream
-  return launch<BN_MAX, 9, B_BOX>(ta, tb, p, max_tiles * p.m_tiles, name, s);
+  return launch<BN_MAX, DG_MOE_STAGES, B_BOX>(ta, tb, p, max_tiles * p.m_tiles, name, s,
+                                              DG_MOE_CTAS_PER_SM);
 }
 
-int experts_tc_tile_tokens() { return 64; }
+int experts_tc_tile_tokens() { return DG_MOE_BN; }
 
 }  // namespace dg

@@ -82,14 +82,32 @@ __global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__
 
 // Top-k and gates from router logits z [T][E] (fp32), one warp per token: the k largest logits
 // (lower expert index first on equal values), gates = softmax over the selected logits.
+// With `forced` non-null the k experts of token t are forced[t][0..k-1] (in that order) instead of
+// the k largest logits; the gates are still the softmax over the selected logits.
 __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict__ z,
-                                   const uint8_t *__restrict__ token_live, int32_t *topk_idx,
+                                   const uint8_t *__restrict__ token_live,
+                                   const int32_t *__restrict__ forced, int32_t *topk_idx,
                                    float *topk_w) {
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T_) return;
   const bool live = token_live == nullptr || token_live[t] != 0;
   const float *zr = z + (size_t)t * E;
+  if (forced) {
+    const int e = lane < k ? forced[(size_t)t * k + lane] : -1;
+    const bool ok = e >= 0 && e < E;
+    const float ze = ok ? zr[e] : -INFINITY;
+    const float z0 = __shfl_sync(0xffffffffu, ze, 0);
+    const float p = (lane < k && ok) ? expf(ze - z0) : 0.f;
+    float denom = p;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = (live && ok) ? e : -1;
+      topk_w[(size_t)t * k + lane] = (live && ok) ? p / denom : 0.f;
+    }
+    return;
+  }
   float zv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) zv[i] = (lane + 32 * i < E) ? zr[lane + 32 * i] : -INFINITY;
@@ -122,6 +140,80 @@ __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict
   if (lane < k) {
     topk_idx[(size_t)t * k + lane] = live ? my_idx : -1;
     topk_w[(size_t)t * k + lane] = live ? mine / denom : 0.f;
+  }
+}
+
+// Permutation and tile list in one block of 1024 threads (T k <= 65536, E <= 256): from the top-k
+// expert ids (router_topk_kernel's output) the per-expert counts, expert_off, the stable grouping
+// of the assignments by expert (as permute_kernel) and the grouped-GEMM tile list (as
+// build_tiles_kernel), with the per-expert counts in load_out when it is non-null.
+__global__ void __launch_bounds__(1024) permute_tiles_kernel(int n_assign, int E,
+                                                             const int32_t *__restrict__ topk_idx,
+                                                             int32_t *expert_off, int32_t *perm,
+                                                             int32_t *inv_perm, int tile_m,
+                                                             GroupTile *tiles, int32_t *n_tiles,
+                                                             int max_tiles, int32_t *load_out) {
+  __shared__ int cnt[256], off[257], running[256], toff[257];
+  __shared__ int wc[32][256];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) { cnt[e] = 0; running[e] = 0; }
+  __syncthreads();
+  for (int a = tid; a < n_assign; a += blockDim.x) {
+    const int e = topk_idx[a];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, tacc = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e] = acc;
+      toff[e] = tacc;
+      acc += cnt[e];
+      tacc += (cnt[e] + tile_m - 1) / tile_m;
+    }
+    off[E] = acc;
+    toff[E] = tacc;
+    *n_tiles = min(tacc, max_tiles);
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) expert_off[e] = off[e];
+  for (int e = tid; e < E; e += blockDim.x) {
+    if (load_out) load_out[e] = cnt[e];
+    const int nt = toff[e + 1] - toff[e];
+    for (int i = 0; i < nt; ++i) {
+      const int slot = toff[e] + i;
+      if (slot < max_tiles) tiles[slot] = GroupTile{e, i * tile_m};
+    }
+  }
+  for (int c0 = 0; c0 < n_assign; c0 += blockDim.x) {
+    for (int i = tid; i < 32 * E; i += blockDim.x) wc[i / E][i % E] = 0;
+    __syncthreads();
+    const int a = c0 + tid;
+    int e = -1;
+    if (a < n_assign) {
+      e = topk_idx[a];
+      if (e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank == 0) wc[w][e] = __popc(peers);
+    __syncthreads();
+    if (e >= 0) {
+      int before = 0;
+      for (int ww = 0; ww < w; ++ww) before += wc[ww][e];
+      const int pos = off[e] + running[e] + before + rank;
+      perm[pos] = a;
+      inv_perm[a] = pos;
+    } else if (a < n_assign) {
+      inv_perm[a] = -1;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int t = 0;
+      for (int ww = 0; ww < 32; ++ww) t += wc[ww][ee];
+      running[ee] += t;
+    }
+    __syncthreads();
   }
 }
 
@@ -250,7 +342,76 @@ __global__ void combine_kernel(int d, int k, const int32_t *__restrict__ topk_id
   }
 }
 
+// Combine + the next RMSNorm, one block per token: x_t = res_t + sum_j w[t][j] Y[inv_perm[t k + j]]
+// (fp32, slot order), stored; then RMSNorm(x_t) rounded to the activation type, stored in a_out
+// (the next layer's QKV input) and/or in f_out row slot[t] (the final-norm rows of the masked
+// positions that the LM head reads).  d <= 256 * 16.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_norm_kernel(int d, int k, float eps,
+                                                           const int32_t *__restrict__ topk_idx,
+                                                           const float *__restrict__ topk_w,
+                                                           const int32_t *__restrict__ inv_perm,
+                                                           const float *__restrict__ Y,
+                                                           const float *__restrict__ res, float *out,
+                                                           T *a_out, const int32_t *__restrict__ slot,
+                                                           T *f_out) {
+  __shared__ float red[8];
+  __shared__ int idx[32];
+  __shared__ float wt[32];
+  const int t = blockIdx.x;
+  float xv[16];
+  float ss = 0.f;
+  if (threadIdx.x < k) {
+    idx[threadIdx.x] = topk_idx[t * k + threadIdx.x] >= 0 ? inv_perm[t * k + threadIdx.x] : -1;
+    wt[threadIdx.x] = topk_w[t * k + threadIdx.x];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int c = threadIdx.x + u * 256;
+    if (c < d) {
+      float acc = res[(size_t)t * d + c];
+      for (int j = 0; j < k; ++j)
+        if (idx[j] >= 0) acc = fmaf(wt[j], Y[(size_t)idx[j] * d + c], acc);
+      out[(size_t)t * d + c] = acc;
+      xv[u] = acc;
+      ss += acc * acc;
+    }
+  }
+  const int sl = slot ? slot[t] : -1;
+  if (!a_out && sl < 0) return;  // uniform in the block
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int c = threadIdx.x + u * 256;
+    if (c < d) {
+      const T v = from_f<T>(xv[u] * inv);
+      if (a_out) a_out[(size_t)t * d + c] = v;
+      if (sl >= 0) f_out[(size_t)sl * d + c] = v;
+    }
+  }
+}
+
 }  // namespace
+
+int launch_combine_norm(int act, int T_, int d, int k, double eps, const int32_t *topk_idx,
+                        const float *topk_w, const int32_t *inv_perm, const void *Y,
+                        const void *res, void *out, void *a_out, const int32_t *slot, void *f_out,
+                        cudaStream_t s) {
+  if (T_ <= 0) return DG_OK;
+  if (d > 256 * 16 || k > 32) return DG_ERR_UNSUPPORTED;
+  note_launch(s, "combine_norm");
+  if (act == DG_F32)
+    combine_norm_kernel<float><<<T_, 256, 0, s>>>(d, k, (float)eps, topk_idx, topk_w, inv_perm,
+                                                  (const float *)Y, (const float *)res, (float *)out,
+                                                  (float *)a_out, slot, (float *)f_out);
+  else
+    combine_norm_kernel<bf16><<<T_, 256, 0, s>>>(d, k, (float)eps, topk_idx, topk_w, inv_perm,
+                                                 (const float *)Y, (const float *)res, (float *)out,
+                                                 (bf16 *)a_out, slot, (bf16 *)f_out);
+  return check_launch("combine_norm");
+}
 
 int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void *y,
                   const void *w_router, const uint8_t *token_live, int32_t *topk_idx,
@@ -278,12 +439,27 @@ int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void 
 }
 
 int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *token_live,
-                       int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+                       int32_t *topk_idx, float *topk_w, cudaStream_t s, const int32_t *forced) {
   if (T_ <= 0) return DG_OK;
   if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
   note_launch(s, "router_topk");
-  router_topk_kernel<<<(T_ + 7) / 8, 256, 0, s>>>(T_, E, k, z, token_live, topk_idx, topk_w);
+  router_topk_kernel<<<(T_ + 7) / 8, 256, 0, s>>>(T_, E, k, z, token_live, forced, topk_idx,
+                                                  topk_w);
   return check_launch("router_topk");
+}
+
+int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
+                 float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
+                 GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
+                 cudaStream_t s, const int32_t *forced) {
+  if (T_ <= 0) return DG_OK;
+  if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
+  const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced);
+  if (rc != DG_OK) return rc;
+  note_launch(s, "permute_tiles");
+  permute_tiles_kernel<<<1, 1024, 0, s>>>(T_ * k, E, topk_idx, expert_off, perm, inv_perm, tile_m,
+                                          tiles, n_tiles, max_tiles, load_out);
+  return check_launch("permute_tiles");
 }
 
 int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *expert_off,

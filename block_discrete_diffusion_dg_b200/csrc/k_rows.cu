@@ -102,6 +102,112 @@ __global__ void __launch_bounds__(1024) compact_rows_kernel(int batch, int canva
   if (threadIdx.x == 0) *n_rows = base;
 }
 
+// Step prologue in one launch: blocks [0, rows) embed + pre-norm one row each (as
+// embed_norm_kernel); the next rope_blocks blocks fill the RoPE table (as rope_table_kernel);
+// with compaction requested, the last block lists the rows that need logits (as
+// compact_rows_kernel, 256 threads) and the slot of each row in that list (-1 if none).
+template <typename T>
+__global__ void __launch_bounds__(256) prologue_kernel(
+    const int32_t *__restrict__ tokens, const uint8_t *__restrict__ masked, const T *__restrict__ emb,
+    int rows, int d, int vocab, float eps, float *x_out, T *a_out, int32_t *st, int rope_blocks,
+    int n, int hd, double theta, const int32_t *__restrict__ cache_len, float *cs, int batch,
+    int canvas, const int32_t *__restrict__ done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
+    uint8_t *token_live) {
+  __shared__ float red[8];
+  __shared__ int warp_tot[8];
+  __shared__ int base;
+  const int bid = blockIdx.x;
+  if (bid < rows) {  // embedding + pre-norm
+    const int row = bid;
+    int id = (masked && masked[row]) ? vocab : tokens[row];
+    if (id < 0 || id > vocab) {
+      if (threadIdx.x == 0) set_status(st, DG_ERR_INVALID_ARG);
+      id = vocab;
+    }
+    const T *src = emb + (size_t)id * d;
+    float ss = 0.f;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+      const float v = to_f(src[j]);
+      ss += v * v;
+    }
+    ss = block_sum(ss, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+      const float v = to_f(src[j]);
+      x_out[(size_t)row * d + j] = v;
+      a_out[(size_t)row * d + j] = from_f<T>(v * inv);
+    }
+    return;
+  }
+  if (bid < rows + rope_blocks) {  // RoPE table: cos/sin of (cache_len[b] + i) * theta^(-2j/hd)
+    const int half = hd / 2;
+    const int e = (bid - rows) * blockDim.x + threadIdx.x;
+    if (e >= batch * n * half) return;
+    const int b = e / (n * half), r = e % (n * half);
+    const int i = r / half, j = r % half;
+    const double inv = pow(theta, -2.0 * (double)j / (double)hd);
+    const double ang = ((cache_len ? (double)cache_len[b] : 0.0) + (double)i) * inv;
+    double sn, c;
+    sincos(ang, &sn, &c);
+    float *o = cs + ((size_t)(b * n + i) * hd + 2 * j);
+    o[0] = (float)c;
+    o[1] = (float)sn;
+    return;
+  }
+  // compaction of the rows that need logits
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  const int total = batch * canvas;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int c0 = 0; c0 < total; c0 += blockDim.x) {
+    const int p = c0 + threadIdx.x;
+    int live = 0;
+    if (p < total) {
+      const int alive = done ? (done[p / canvas] == 0) : 1;
+      if (token_live) token_live[p] = (uint8_t)alive;
+      live = alive && (masked == nullptr || masked[p] != 0);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, live);
+    if (lane == 0) warp_tot[w] = __popc(bal);
+    __syncthreads();
+    int before = 0;
+    for (int i = 0; i < w; ++i) before += warp_tot[i];
+    const int pos = base + before + __popc(bal & ((1u << lane) - 1u));
+    if (live) row_idx[pos] = p;
+    if (p < total && slot) slot[p] = live ? pos : -1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int i = 0; i < nw; ++i) t += warp_tot[i];
+      base += t;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *n_rows = base;
+}
+
+int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const void *emb, int rows,
+                    int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
+                    int n, int hd, double theta, const int32_t *cache_len, float *cs,
+                    const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
+                    uint8_t *token_live, cudaStream_t s) {
+  if (rows <= 0) return DG_OK;
+  const int rope_blocks = (batch * n * (hd / 2) + 255) / 256;
+  const int grid = rows + rope_blocks + (row_idx ? 1 : 0);
+  note_launch(s, "prologue");
+  if (act == DG_F32)
+    prologue_kernel<float><<<grid, 256, 0, s>>>(
+        tokens, masked, (const float *)emb, rows, d, vocab, (float)eps, (float *)x_out,
+        (float *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
+        n_rows, slot, token_live);
+  else
+    prologue_kernel<bf16><<<grid, 256, 0, s>>>(
+        tokens, masked, (const bf16 *)emb, rows, d, vocab, (float)eps, (float *)x_out,
+        (bf16 *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
+        n_rows, slot, token_live);
+  return check_launch("prologue");
+}
+
 int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, const void *emb,
                       int rows, int d, int vocab, double eps, void *x_out, void *a_out,
                       int32_t *st, cudaStream_t s) {

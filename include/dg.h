@@ -96,7 +96,8 @@ typedef struct dg_model {
 /* ---- sizes and status ------------------------------------------------------------------ */
 
 /* Bytes of scratch the calls below need for `batch` canvases of `n_tokens` tokens each and a
- * cache of `cache_cap` rows per (layer, batch, kv head).  0 on an invalid config. */
+ * cache of `cache_cap` rows per (layer, batch, kv head), on the current device (the attention's
+ * key-split plan depends on its SM count).  0 on an invalid config. */
 size_t dg_workspace_size(const dg_config *cfg, int batch, int n_tokens, int cache_cap);
 
 /* Synchronises `stream`, copies *dev_status to the host and returns it (DG_ERR_CUDA if the
@@ -208,10 +209,13 @@ int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *arg
  * [0, V]) at positions cache_len[b] + i, write every layer's K/V (after RoPE) into cache rows
  * [cache_len[b], cache_len[b] + n_tokens), then cache_len[b] += n_tokens.  Also used to
  * prefill a prompt in chunks.  k_cache, v_cache: [L][B][Hkv][cache_cap][hd].  A canvas whose
- * rows would pass cache_cap is left unchanged and sets DG_ERR_CAPACITY. */
+ * rows would pass cache_cap is left unchanged and sets DG_ERR_CAPACITY.  forced_topk: NULL, or
+ * int32 [n_layers][B n_tokens][k] expert ids used instead of each layer's router top-k (see
+ * dg_canvas_step). */
 int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
                  int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
-                 void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+                 const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+                 void *stream);
 
 /* One denoising step of every live canvas ("DiffusionGemma Technical Report", Figure 4,
  * stage 2 and the explanatory visual): embed the canvas (masked positions as MASK = V), run
@@ -225,13 +229,19 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
  * were masked when the step began.  logits_dbg (or NULL): fp32 [B C][V], row b C + i written for
  * each such position (debug and parity only; costs a full logits write).  expert_load (or
  * NULL): int32 [n_layers][E], the number of (token, slot) assignments each expert received in
- * each layer this step (for load monitoring and byte accounting). */
+ * each layer this step (for load monitoring and byte accounting).  forced_topk (or NULL):
+ * int32 [n_layers][B C][k] expert ids that replace each layer's router top-k choice (the gates
+ * are still the softmax of this step's router logits over the given experts).  It lets a caller
+ * reproduce another computation's expert choices exactly — e.g. to compare a deep stack with a
+ * reference, where bf16 rounding legitimately flips near-tied routing decisions; bf16 models
+ * with a tensor-core router only (DG_ERR_UNSUPPORTED otherwise). */
 int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
                    uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
                    int max_steps, double gamma, const void *k_cache, const void *v_cache,
                    const int32_t *cache_len, int cache_cap, float *entropy_out,
-                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load, void *ws,
-                   size_t ws_bytes, int32_t *dev_status, void *stream);
+                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load,
+                   const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+                   void *stream);
 
 /* ---- fixed-scratch entry point ---------------------------------------------------------- */
 

@@ -440,13 +440,14 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
 
 
 def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
-              cache_len: np.ndarray):
+              cache_len: np.ndarray, info=None):
     """Causal encoder pass over finished tokens; their K/V go to the cache.
 
     tokens int32 [B, n]; kcache/vcache decoded [L, B, Hkv, cap, hd], updated in
     place (rows [len, len+n) of every layer, values as stored).  The encoder
     shares the decoder's weights; its attention sees the whole cache and the
-    new tokens causally.  Returns the new cache_len.
+    new tokens causally.  Returns the new cache_len.  With ``info`` (a dict) given, the expert
+    choices of each routed layer are collected in info["router_idx"][l] as [B, n, k].
     """
     B, n = tokens.shape
     new_len = np.array(cache_len, copy=True)
@@ -458,7 +459,12 @@ def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, v
             q, k, v = layer_qkv(cfg, model, l, x, pos)
             kc, vc = kcache[l, b, :, :L0], vcache[l, b, :, :L0]
             if l + 1 < cfg.n_layers:
-                x = layer_rest(cfg, model, l, x, q, k, v, kc, vc, True)
+                li = {} if info is not None else None
+                x = layer_rest(cfg, model, l, x, q, k, v, kc, vc, True, li)
+                if info is not None:
+                    ri = info.setdefault("router_idx", [np.zeros((B, n, cfg.top_k), np.int32)
+                                                        for _ in range(cfg.n_layers)])
+                    ri[l][b] = li["router_idx"][0]
             kcache[l, b, :, L0:L0 + n] = k.transpose(1, 0, 2)
             vcache[l, b, :, L0:L0 + n] = v.transpose(1, 0, 2)
         new_len[b] = L0 + n

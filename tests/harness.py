@@ -49,7 +49,7 @@ class Workload:
     def oracle(self) -> O.OracleModel:
         return oracle_model(self.cfg, self.model)
 
-    def step(self, state=None, gamma=None, max_steps=None, logits=False):
+    def step(self, state=None, gamma=None, max_steps=None, logits=False, forced=None):
         """One dg_canvas_step on a copy of `state`; returns (new_state, entropy, argmax, logits)."""
         cfg = self.cfg
         st = {k: v.clone() for k, v in (state or self.state).items()}
@@ -60,7 +60,8 @@ class Workload:
         B.dg_canvas_step(self.dgcfg, self.dgmodel, B_, st["tokens"], st["masked"], st["n_masked"],
                          st["done"], st["step"], cfg.max_steps if max_steps is None else max_steps,
                          cfg.gamma if gamma is None else gamma, self.kv["k"], self.kv["v"],
-                         self.kv["cache_len"], self.cap, ent, am, lg, self.ws, self.status)
+                         self.kv["cache_len"], self.cap, ent, am, lg, self.ws, self.status,
+                         forced_topk=forced)
         torch.cuda.synchronize()
         return st, ent, am, lg
 

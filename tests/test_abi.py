@@ -72,7 +72,7 @@ def test_host_side_argument_rejection_launches_nothing():
         == B.DG_ERR_INVALID_ARG
     # model with a null layer pointer
     assert L.dg_canvas_step(ctypes.byref(cfg), None, 1, 8, 8, 8, 8, 8, 16, 0.1, 8, 8, 8, 64, None,
-                            None, None, None, 256, 1 << 30, None, None) == B.DG_ERR_INVALID_ARG
+                            None, None, None, None, 256, 1 << 30, None, None) == B.DG_ERR_INVALID_ARG
     assert L.dg_launch_count() == n0
 
 

@@ -1,0 +1,228 @@
+"""GPU parity at the full sizes of the long-context, batched-FP8 and 30-layer workloads.
+
+* long context: the one-layer model with 131072 prompt K/V tokens, half-committed canvas; the
+  oracle runs the whole step (fp64 attention over 131328 keys).
+* batch of 32: 32 canvases x 256 through the one-layer model with e4m3 expert/attention weights
+  (one fp32 scale per output channel), 1024 prompt tokens each; the oracle runs two sampled
+  canvases (the others are marked done on its side; canvases are independent).
+* 30-layer stack: a full-width step of a 4-layer stack on synthetic prompt K/V against the oracle;
+  prefill -> denoise -> append against the oracle at full width and 2 layers; and the 30-layer
+  generate loop of the workload (prompt 2048 prefilled in 256-token chunks, 4 canvases, at most 32
+  steps each) checked by its invariants.
+  Through several layers two valid bf16 computations route a growing share of tokens to
+  different experts (a near tie flips, and that token's later state, hence its later choices,
+  differ by O(1): about 10% of the tokens by the 4th layer).  The multi-layer comparisons
+  therefore hand the device the oracle's expert choices (forced_topk; the gates are still the
+  device's own) and then hold every row to the float bars, the logit bar widened with depth
+  (logit_tol) by the measured growth of bf16 rounding noise.
+Bars as in test_gpu_full: logits 2e-2 max-abs and entropies 1e-3 relative on rows without a
+router near tie, argmax bit-exact against the device's own logits, EB bit-exact on the oracle's
+entropies."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import dg_oracle as O
+from block_discrete_diffusion_dg_b200 import binding as B
+from harness import Workload, np_state, torch_state, decode_cache
+
+pytestmark = pytest.mark.gpu
+
+LOGIT_TOL = 2e-2
+ENT_RTOL = 1e-3
+ROUTER_TIE = 1e-2
+
+
+def logit_tol(n_layers: int) -> float:
+    """The 2e-2 bf16 bar for one layer, widened for a stack by the growth of bf16 rounding noise
+    with depth.  Two valid bf16 computations of a full-width stack that share their routing
+    differ in the logits by std 0.0022 / 0.0027 / 0.0033 and max 0.021 / 0.025 / 0.031 (over
+    8.4M logits) at 1 / 2 / 4 layers; the bar grows by log2(L) / 3 per unit."""
+    return LOGIT_TOL * (1.0 + np.log2(max(n_layers, 1)) / 3.0)
+
+
+def kv_close(g, o, n_layers):
+    """K/V rows after layer 0 carry the same depth noise: each element within 2^-5 of its
+    row's RMS (the noise is ~0.3% of it), the median error within 2^-9 of it."""
+    scale = np.sqrt(np.mean(o * o, axis=-1, keepdims=True)) + 1e-30
+    rel = np.abs(g - o) / scale
+    return rel.max() <= 2.0 ** -5 and np.median(rel) <= 2.0 ** -9, (rel.max(), np.median(rel))
+
+
+def _forced(cfg, infos):
+    """The oracle's expert choices of a step as the device's forced-routing table
+    [n_layers][B C][k] (canvases the oracle skipped: zeros; the device skips them too)."""
+    f = np.zeros((cfg.n_layers, cfg.batch * cfg.canvas, cfg.top_k), np.int32)
+    for b, inf in enumerate(infos):
+        if inf is None or "router_idx" not in inf:
+            continue
+        for l, idx in enumerate(inf["router_idx"]):
+            f[l, b * cfg.canvas:(b + 1) * cfg.canvas] = idx
+    return torch.from_numpy(f).cuda()
+
+
+def _check_step(wl, st_np, canvases=None, min_ok=0.6, force=False):
+    """One device step against the oracle on the canvases listed (default: all).  With force,
+    the device takes the oracle's expert choices (deep stacks: see test module docstring) and
+    every row is held to the float bars."""
+    cfg = wl.cfg
+    om = wl.oracle() if not hasattr(wl, "_om") else wl._om
+    wl._om = om
+    kc, vc = decode_cache(cfg, wl.kv["k"]), decode_cache(cfg, wl.kv["v"])
+    cl = synth.to_numpy(wl.kv["cache_len"])
+    o_st = {k: np.array(v, copy=True) for k, v in st_np.items()}
+    if canvases is not None:
+        skip = np.ones(cfg.batch, bool)
+        skip[list(canvases)] = False
+        o_st["done"][skip] = 1
+    new_np, infos = O.canvas_step(cfg, om, o_st, kc, vc, cl, cfg.gamma, cfg.max_steps,
+                                  keep_logits=True)
+    g_st, ent, am, lg = wl.step(torch_state(st_np), logits=True,
+                                forced=_forced(cfg, infos) if force else None)
+    wl.check_status()
+    ent, am = ent.cpu().numpy(), am.cpu().numpy()
+    n_rows = 0
+    for b, inf in enumerate(infos):
+        if inf is None:
+            continue
+        rows = inf["rows"]
+        lgb = lg[b * cfg.canvas:(b + 1) * cfg.canvas].cpu().numpy()[rows]
+        assert (am[b, rows] == np.argmax(lgb, axis=1)).all()
+        rmarg = np.min(np.stack(inf["router_margin"]), axis=0)[rows]
+        ok = np.ones(len(rows), bool) if force else rmarg > ROUTER_TIE
+        assert ok.sum() >= min_ok * len(rows), ok.sum()
+        assert np.abs(lgb[ok] - inf["logits"][ok]).max() <= logit_tol(cfg.n_layers)
+        np.testing.assert_allclose(ent[b, rows][ok], inf["H"][ok], rtol=ENT_RTOL)
+        safe = ok & (inf["margin"] > 2 * LOGIT_TOL)
+        assert (am[b, rows][safe] == inf["argmax"][safe]).all()
+        # EB on the oracle's entropies, this canvas alone
+        e_in = np.zeros((1, cfg.canvas), np.float32)
+        a_in = np.zeros((1, cfg.canvas), np.int32)
+        e_in[0, rows] = inf["H"]
+        a_in[0, rows] = inf["argmax"]
+        one = {k: torch.from_numpy(np.ascontiguousarray(v[b:b + 1])).cuda() for k, v in st_np.items()}
+        B.dg_eb_select(1, cfg.canvas, torch.from_numpy(e_in).cuda(), torch.from_numpy(a_in).cuda(),
+                       cfg.gamma, cfg.max_steps, one["tokens"], one["masked"], None,
+                       one["n_masked"], one["done"], one["step"])
+        for k in ("tokens", "masked", "n_masked", "done", "step"):
+            assert (one[k].cpu().numpy()[0] == new_np[k][b]).all(), k
+        n_rows += len(rows)
+    # canvases the device skipped are unchanged
+    if canvases is None:
+        assert n_rows > 0
+    return g_st
+
+
+def test_longctx_step_full_size():
+    cfg = synth.get_config("longctx")
+    wl = Workload(cfg, gen_device="cuda")
+    _check_step(wl, np_state(synth.make_canvas_state(cfg, "half")))
+
+
+def test_batch32_fp8_step_sampled_canvases():
+    cfg = synth.get_config("batch32")
+    wl = Workload(cfg, gen_device="cuda")
+    st = np_state(synth.make_canvas_state(cfg, "all_mask"))
+    g_st = _check_step(wl, st, canvases=(0, 17))
+    # every canvas advanced by one step and committed exactly one token (entropies ~ ln V >> gamma)
+    assert (g_st["step"].cpu().numpy() == 1).all()
+    assert (g_st["n_masked"].cpu().numpy() == cfg.canvas - 1).all()
+
+
+def test_stack_step_full_width_four_layers():
+    cfg = synth.get_config("stack30", n_layers=4, prefill_ids=False, prompt_len=1024)
+    wl = Workload(cfg, gen_device="cuda")
+    _check_step(wl, np_state(synth.make_canvas_state(cfg, "half")), force=True)
+
+
+def test_stack_prefill_denoise_append_two_layers():
+    """Prefill 512 prompt ids in two 256-token chunks, two lockstep denoising steps of a canvas,
+    then its append: caches and step outputs against the oracle (full width, 2 layers)."""
+    cfg = synth.get_config("stack30", n_layers=2, prompt_len=512, n_canvases=1)
+    wl = Workload(cfg, gen_device="cuda")
+    om = wl.oracle()
+    ids = wl.kv["prompt_ids"]
+    k_dev, v_dev, len_dev = wl.kv["k"], wl.kv["v"], wl.kv["cache_len"]
+    ok = np.zeros(decode_cache(cfg, k_dev).shape)
+    ov = np.zeros_like(ok)
+    ln = np.zeros(1, np.int32)
+    for c0 in range(0, cfg.prompt_len, 256):
+        chunk = ids[:, c0:c0 + 256].contiguous()
+        info = {}
+        ln = O.kv_append(cfg, om, chunk.cpu().numpy(), ok, ov, ln, info)
+        forced = torch.from_numpy(np.stack([r.reshape(-1, cfg.top_k) for r in info["router_idx"]])).cuda()
+        B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, chunk, 256, k_dev, v_dev, len_dev, wl.cap, wl.ws,
+                       wl.status, forced_topk=forced)
+    torch.cuda.synchronize()
+    wl.check_status()
+    assert int(len_dev.item()) == ln[0] == cfg.prompt_len
+    gk = decode_cache(cfg, k_dev)[:, :, :, :cfg.prompt_len, :]   # [L][B][Hkv][rows][hd]
+    good, stat = kv_close(gk, ok[:, :, :, :cfg.prompt_len, :], cfg.n_layers)
+    assert good, stat
+    # two denoising steps from the oracle's state on the oracle-prefilled cache
+    wl.kv["k"] = torch.from_numpy(ok).to(torch.bfloat16).cuda()
+    wl.kv["v"] = torch.from_numpy(ov).to(torch.bfloat16).cuda()
+    wl.kv["cache_len"] = torch.from_numpy(ln).cuda()
+    st = np_state(synth.make_canvas_state(cfg, "all_mask"))
+    for _ in range(2):
+        _check_step(wl, st, force=True)
+        kc, vc = decode_cache(cfg, wl.kv["k"]), decode_cache(cfg, wl.kv["v"])
+        st, _ = O.canvas_step(cfg, om, st, kc, vc, ln, cfg.gamma, cfg.max_steps)
+    # append a committed canvas
+    toks = torch.randint(0, cfg.vocab, (1, cfg.canvas), dtype=torch.int32).cuda()
+    info = {}
+    ln2 = O.kv_append(cfg, om, toks.cpu().numpy(), ok, ov, ln, info)
+    forced = torch.from_numpy(np.stack([r.reshape(-1, cfg.top_k) for r in info["router_idx"]])).cuda()
+    B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, toks, cfg.canvas, wl.kv["k"], wl.kv["v"],
+                   wl.kv["cache_len"], wl.cap, wl.ws, wl.status, forced_topk=forced)
+    torch.cuda.synchronize()
+    wl.check_status()
+    assert int(wl.kv["cache_len"].item()) == ln2[0]
+    gk = decode_cache(cfg, wl.kv["k"])[:, :, :, ln[0]:ln2[0], :]
+    assert gk.shape[3] == cfg.canvas
+    good, stat = kv_close(gk, ok[:, :, :, ln[0]:ln2[0], :], cfg.n_layers)
+    assert good, stat
+
+
+def test_stack30_generate_invariants():
+    """The full 30-layer workload: prefill, 4 canvases of at most 32 steps, appends."""
+    cfg = synth.get_config("stack30")
+    wl = Workload(cfg, gen_device="cuda")
+    ids = wl.kv["prompt_ids"]
+    k_dev, v_dev, len_dev = wl.kv["k"], wl.kv["v"], wl.kv["cache_len"]
+    for c0 in range(0, cfg.prompt_len, 256):
+        B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, ids[:, c0:c0 + 256].contiguous(), 256, k_dev,
+                       v_dev, len_dev, wl.cap, wl.ws, wl.status)
+    out = []
+    for c in range(cfg.n_canvases):
+        st = {k: v.cuda() for k, v in synth.make_canvas_state(cfg, "all_mask").items()}
+        steps = 0
+        while not int(st["done"].item()):
+            B.dg_canvas_step(wl.dgcfg, wl.dgmodel, 1, st["tokens"], st["masked"], st["n_masked"],
+                             st["done"], st["step"], cfg.max_steps, cfg.gamma, k_dev, v_dev,
+                             len_dev, wl.cap, None, None, None, wl.ws, wl.status)
+            steps += 1
+            assert steps <= cfg.max_steps
+        # the canvas always finishes within the step cap (the last allowed step commits the rest)
+        assert int(st["step"].item()) == steps <= cfg.max_steps and int(st["n_masked"].item()) == 0
+        toks = st["tokens"].cpu().numpy()
+        assert (toks >= 0).all() and (toks < cfg.vocab).all()
+        out.append(toks)
+        B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, st["tokens"], cfg.canvas, k_dev, v_dev, len_dev,
+                       wl.cap, wl.ws, wl.status)
+    torch.cuda.synchronize()
+    wl.check_status()
+    assert int(len_dev.item()) == cfg.prompt_len + cfg.n_canvases * cfg.canvas == wl.cap
+    assert torch.isfinite(k_dev.float()).all() and torch.isfinite(v_dev.float()).all()
+    # a second canvas step from the same state reproduces the first bit for bit
+    st0 = {k: v.cuda() for k, v in synth.make_canvas_state(cfg, "half").items()}
+    ents = []
+    for _ in range(2):
+        st = {k: v.clone() for k, v in st0.items()}
+        ent = torch.zeros((1, cfg.canvas), device="cuda")
+        B.dg_canvas_step(wl.dgcfg, wl.dgmodel, 1, st["tokens"], st["masked"], st["n_masked"],
+                         st["done"], st["step"], cfg.max_steps, cfg.gamma, k_dev, v_dev, len_dev,
+                         wl.cap, ent, None, None, wl.ws, wl.status)
+        ents.append(ent.cpu())
+    assert torch.equal(ents[0], ents[1])
