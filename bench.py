@@ -45,17 +45,19 @@ def load_peaks():
 # ------------------------------------------------------------------------------ accounting
 
 def step_bytes(cfg, experts_touched: float) -> dict:
-    """Algorithmic HBM bytes of one step: every weight byte the step must read once, the
-    prompt K/V, and the canvas rows (activations are small and are not counted)."""
+    """Algorithmic HBM bytes of one step: every weight byte the step must read once (for the
+    experts: the experts the step routes tokens to, summed over layers), the prompt K/V, and the
+    canvas rows (activations are small and are not counted)."""
+    L = cfg.n_layers
     wb = 1 if cfg.w == "e4m3" else (4 if cfg.w == "f32" else 2)
     ab = 4 if cfg.act == "f32" else 2
     d, hd = cfg.d_model, cfg.head_dim
-    qkv = cfg.qkv_rows * d * wb
-    wo = d * cfg.n_q_heads * hd * wb
-    router = cfg.n_experts * d * (4 if cfg.w == "f32" else 2)
+    qkv = L * cfg.qkv_rows * d * wb
+    wo = L * d * cfg.n_q_heads * hd * wb
+    router = L * cfg.n_experts * d * (4 if cfg.w == "f32" else 2)
     expert = (2 * cfg.d_ff * d + d * cfg.d_ff) * wb
     lm = cfg.vocab * d * ab
-    kv = cfg.batch * cfg.prompt_len * cfg.n_kv_heads * hd * 2 * ab
+    kv = L * cfg.batch * cfg.prompt_len * cfg.n_kv_heads * hd * 2 * ab
     emb_rows = cfg.batch * cfg.canvas * d * ab
     return {"qkv": qkv, "o": wo, "router": router, "experts": experts_touched * expert,
             "expert_gate_up": experts_touched * 2 * cfg.d_ff * d * wb,
@@ -64,16 +66,22 @@ def step_bytes(cfg, experts_touched: float) -> dict:
             "total": qkv + wo + router + experts_touched * expert + lm + kv + emb_rows}
 
 
-def step_flops(cfg, masked_rows: int) -> float:
+def step_flops(cfg, masked_rows: float) -> dict:
     T = cfg.batch * cfg.canvas
+    L = cfg.n_layers
     d, hd = cfg.d_model, cfg.head_dim
-    qkv = 2 * T * d * cfg.qkv_rows
-    o = 2 * T * cfg.n_q_heads * hd * d
-    attn = 4 * cfg.batch * cfg.n_q_heads * cfg.canvas * (cfg.prompt_len + cfg.canvas) * hd
-    router = 2 * T * d * cfg.n_experts
-    moe = 2 * T * cfg.top_k * (2 * cfg.d_ff * d + d * cfg.d_ff)
+    qkv = L * 2 * T * d * cfg.qkv_rows
+    o = L * 2 * T * cfg.n_q_heads * hd * d
+    attn = L * 4 * cfg.batch * cfg.n_q_heads * cfg.canvas * (cfg.prompt_len + cfg.canvas) * hd
+    router = L * 2 * T * d * cfg.n_experts
+    moe = L * 2 * T * cfg.top_k * (2 * cfg.d_ff * d + d * cfg.d_ff)
     lm = 2 * masked_rows * d * cfg.vocab
-    return float(qkv + o + attn + router + moe + lm)
+    return {"lm_head": float(lm), "attention": float(attn), "experts": float(moe),
+            "total": float(qkv + o + attn + router + moe + lm)}
+
+
+STATES = {"layer": ("all_mask", "half"), "longctx": ("half",), "batch32": ("all_mask",),
+          "tiny": ("all_mask",)}
 
 
 # ------------------------------------------------------------------------------ clocks
@@ -241,11 +249,77 @@ def run_reference(args, world, rank):
 
 
 def workload_desc(cfg) -> str:
+    states = " / ".join(STATES.get(cfg.name, ("all_mask",)))
     return (f"{cfg.name}: {cfg.n_layers} decoder layer(s) {cfg.act}/{cfg.w}, d_model {cfg.d_model}, "
             f"{cfg.n_q_heads}q/{cfg.n_kv_heads}kv x {cfg.head_dim}, {cfg.n_experts} experts top-"
             f"{cfg.top_k} ff {cfg.d_ff}, vocab {cfg.vocab}, canvas {cfg.canvas}, prompt KV "
-            f"{cfg.prompt_len}, gamma {cfg.gamma}, batch {cfg.batch}; steps alternate all-MASK / "
-            f"half-committed canvases")
+            f"{cfg.prompt_len}, gamma {cfg.gamma}, batch {cfg.batch}; canvas states: {states}")
+
+
+def run_generate(args, world, rank):
+    """Block-autoregressive generation of the 30-layer workload: the prompt (2048 ids) is
+    prefilled through the append in 256-token chunks (not timed), then n_canvases canvases are
+    denoised from all-MASK until done (the host reads each step's done flag) and appended.
+    Timed: the denoising steps and the appends (the pages' TPS excludes prefill)."""
+    import synth
+    from block_discrete_diffusion_dg_b200 import binding as B
+    B.lib()
+    cfg = synth.get_config(args.workload)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    model = synth.make_model(cfg, dev)
+    kv = synth.make_prompt_kv(cfg, dev)
+    cap = kv["k"].shape[3]
+    dgcfg, dgm = B.make_config(cfg), B.Model(model)
+    ws = B.alloc_workspace(dgcfg, cfg.batch, cfg.canvas, cap)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ids = kv["prompt_ids"]
+    for c0 in range(0, cfg.prompt_len, 256):
+        B.dg_kv_append(dgcfg, dgm, cfg.batch, ids[:, c0:c0 + 256].contiguous(), 256, kv["k"],
+                       kv["v"], kv["cache_len"], cap, ws, status)
+    k0, v0, l0 = kv["k"].clone(), kv["v"].clone(), kv["cache_len"].clone()
+    stream = torch.cuda.current_stream()
+
+    def generate():
+        kv["k"].copy_(k0); kv["v"].copy_(v0); kv["cache_len"].copy_(l0)
+        steps = 0
+        for _ in range(cfg.n_canvases):
+            st = {k: v.to(dev) for k, v in synth.make_canvas_state(cfg, "all_mask").items()}
+            while True:
+                B.dg_canvas_step(dgcfg, dgm, cfg.batch, st["tokens"], st["masked"], st["n_masked"],
+                                 st["done"], st["step"], cfg.max_steps, cfg.gamma, kv["k"], kv["v"],
+                                 kv["cache_len"], cap, None, None, None, ws, status, stream)
+                steps += 1
+                if int(st["done"].item()):
+                    break
+            B.dg_kv_append(dgcfg, dgm, cfg.batch, st["tokens"], cfg.canvas, kv["k"], kv["v"],
+                           kv["cache_len"], cap, ws, status, stream)
+        return steps
+
+    generate()                              # warm-up
+    torch.cuda.synchronize()
+    n0 = B.dg_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    steps = generate()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if B.dg_read_status(status) != B.DG_OK:
+        raise RuntimeError("device status set during generation")
+    launches = B.dg_launch_count() - n0
+    ms = e0.elapsed_time(e1)
+    toks = cfg.n_canvases * cfg.canvas * cfg.batch
+    peaks, peak_src = load_peaks()
+    line = {"metric": METRIC, "value": round(steps / (ms / 1e3), 3), "unit": "steps/s",
+            "n_gpus": world, "steps": steps, "warmup": 1, "ms_per_step": round(ms / steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random-init weights, random prompt ids)",
+            "config": {"workload": workload_desc(cfg) + f"; generate {cfg.n_canvases} canvases, "
+                       f"at most {cfg.max_steps} steps each, prefill not timed",
+                       "batch": cfg.batch, "mode": "generate"},
+            "output_tok_s": round(toks / (ms / 1e3), 2), "gpu_launches": int(launches),
+            "impl": "dg", "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 # DRAM traffic per launch of the dominant kernel from one ncu capture of the same kernel build
@@ -266,13 +340,14 @@ def run_dg(args, world, rank, local):
     dgcfg, dgm = B.make_config(cfg), B.Model(model)
     ws = B.alloc_workspace(dgcfg, cfg.batch, cfg.canvas, cap)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    init = [{k: v.to(dev) for k, v in synth.make_canvas_state(cfg, s).items()}
-            for s in ("all_mask", "half")]
+    states = STATES.get(cfg.name, ("all_mask",))
+    init = [{k: v.to(dev) for k, v in synth.make_canvas_state(cfg, s_).items()} for s_ in states]
+    ns = len(init)
     st = {k: v.clone() for k, v in init[0].items()}
     load = torch.zeros((cfg.n_layers, cfg.n_experts), dtype=torch.int32, device=dev)
 
     def one_step(i, stream=None, expert_load=None):
-        src = init[i % 2]
+        src = init[i % ns]
         for k in st:
             st[k].copy_(src[k], non_blocking=True)
         B.dg_canvas_step(dgcfg, dgm, cfg.batch, st["tokens"], st["masked"], st["n_masked"],
@@ -299,20 +374,21 @@ def run_dg(args, world, rank, local):
         raise RuntimeError(f"device status {B.STATUS_NAMES.get(rc, rc)} during warm-up")
 
     # per state: tokens committed by one step, experts the step routes to, kernels it launches
-    committed, touched, per_step_launches = [], [], 0
-    for i in range(2):
+    committed, touched, masked_rows, per_step_launches = [], [], [], 0
+    for i in range(ns):
         n0 = B.dg_launch_count()
         one_step(i, expert_load=load)
         torch.cuda.synchronize()
         per_step_launches = B.dg_launch_count() - n0
         committed.append(int(init[i]["n_masked"].sum() - st["n_masked"].sum()))
-        touched.append(float((load > 0).sum(dim=1).float().mean().item()))
+        touched.append(float((load > 0).sum().item()))      # (layer, expert) pairs with tokens
+        masked_rows.append(float(init[i]["n_masked"].sum().item()))
 
     # ---- timed region: K steps replayed from CUDA graphs (one graph per canvas state) ----
     graphs = []
     if not args.no_graph:
         try:
-            for i in range(2):
+            for i in range(ns):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
                     one_step(i)
@@ -338,7 +414,7 @@ def run_dg(args, world, rank, local):
     ev0.record(stream)
     for i in range(args.steps):
         if graphs:
-            graphs[i % 2].replay()
+            graphs[i % ns].replay()
         else:
             one_step(i)
     ev1.record(stream)
@@ -393,32 +469,45 @@ def run_dg(args, world, rank, local):
                  for k, v in sorted(per.items(), key=lambda kv_: -kv_[1][0])}
     peaks, peak_src = load_peaks()
     t_avg = float(np.mean(touched))
+    m_avg = float(np.mean(masked_rows))
     sb = step_bytes(cfg, t_avg)
+    sf = step_flops(cfg, m_avg)
     dom = next(iter(breakdown))
-    dom_bytes = {"lm_head_tc": sb["lm_head"] + cfg.batch * cfg.canvas * cfg.d_model * 2,
-                 "moe_gate_up_tc": sb["expert_gate_up"], "moe_down_tc": sb["expert_down"]}.get(dom)
+    ab = 4 if cfg.act == "f32" else 2
+    lm_bytes = sb["lm_head"] + m_avg * cfg.d_model * ab
+    dur = breakdown[dom]["ms_per_launch"] / 1e3
     roof = None
-    if dom_bytes:
-        dur = breakdown[dom]["ms_per_launch"] / 1e3
-        ach = dom_bytes / dur / 1e9
-        peak = peaks["hbm_gbs"]
-        tr = NCU_TRAFFIC.get(dom)
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(ach / peak, 4),
-                "traffic": tr["bytes"] if tr else None,
-                "algorithmic_bytes_per_launch": int(dom_bytes),
-                "peak_source": f"{peak_src} (burst copy, of measured)",
-                "timing": f"CUDA events before each launch, {kp}-step profile pass ({prof_mode})",
-                "traffic_source": tr["source"] if tr else None}
-    masked_avg = 0.5 * (cfg.canvas + cfg.canvas // 2) * cfg.batch
+    if dom == "lm_head_tc" and sf["lm_head"] / (peaks["bf16_tflops_sustained"] * 1e12) > \
+            lm_bytes / (peaks["hbm_gbs"] * 1e9):
+        ach = sf["lm_head"] / dur / 1e12     # the batched LM head is a tensor-bound contraction
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 1),
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
+                "traffic": None, "algorithmic_flops_per_launch": sf["lm_head"],
+                "peak_source": f"{peak_src} (cuBLAS bf16, sustained, of measured)"}
+    else:
+        dom_bytes = {"lm_head_tc": lm_bytes, "moe_gate_up_tc": sb["expert_gate_up"],
+                     "moe_down_tc": sb["expert_down"]}.get(dom)
+        if dom_bytes:
+            ach = dom_bytes / dur / 1e9
+            peak = peaks["hbm_gbs"]
+            tr = NCU_TRAFFIC.get(dom) if cfg.name == "layer" else None
+            roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
+                    "unit": "GB/s", "frac": round(ach / peak, 4),
+                    "traffic": tr["bytes"] if tr else None,
+                    "algorithmic_bytes_per_launch": int(dom_bytes),
+                    "peak_source": f"{peak_src} (burst copy, of measured)",
+                    "traffic_source": tr["source"] if tr else None}
+    if roof:
+        roof["timing"] = f"CUDA events before each launch, {kp}-step profile pass ({prof_mode})"
     t_bytes = sb["total"] / (peaks["hbm_gbs"] * 1e9)
-    t_flops = step_flops(cfg, masked_avg) / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_flops = sf["total"] / (peaks["bf16_tflops_sustained"] * 1e12)
     step_roof = {"bound": "hbm" if t_bytes >= t_flops else "tensor",
                  "roofline_us": round(1e6 * max(t_bytes, t_flops), 1),
                  "measured_us": round(1e3 * ms_step, 1),
                  "frac": round(1e6 * max(t_bytes, t_flops) / (1e3 * ms_step), 4),
                  "algorithmic_bytes": int(sb["total"]),
-                 "algorithmic_flops": step_flops(cfg, masked_avg),
+                 "algorithmic_flops": sf["total"],
                  "experts_touched_per_state": touched,
                  "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, "
                           f"{peaks['bf16_tflops_sustained']} TF/s sustained (of measured)"}
@@ -433,7 +522,7 @@ def run_dg(args, world, rank, local):
     torch.cuda.synchronize()
     e0 = time.perf_counter()
     for i in range(e_steps):
-        src = pin[i % 2]
+        src = pin[i % ns]
         for k in st:
             st[k].copy_(src[k], non_blocking=True)
         B.dg_canvas_step(dgcfg, dgm, cfg.batch, st["tokens"], st["masked"], st["n_masked"],
@@ -455,8 +544,8 @@ def run_dg(args, world, rank, local):
         vc = O.decode_act(synth.to_numpy(kv["v"]), cfg.act)
         cl = synth.to_numpy(kv["cache_len"])
         ts = [oracle_sample_step(cfg, om, {k: synth.to_numpy(v) for k, v in init[i].items()},
-                                 kc, vc, cl, args.ref_frac) for i in range(2)]
-        tstep = float(np.mean(ts))
+                                 kc, vc, cl, args.ref_frac) for i in range(ns)]
+        tstep = float(np.mean(ts)) * cfg.batch      # the sample runs one canvas
         cpu = {"value": 1.0 / tstep, "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"one all-MASK and one half-committed step; attention part over the whole "
                          f"canvas, experts e < E/{args.ref_frac} and an LM-head vocab slice of "
@@ -496,6 +585,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.workload == "stack30":
+            run_generate(args, world, rank)
         else:
             run_dg(args, world, rank, local)
     finally:

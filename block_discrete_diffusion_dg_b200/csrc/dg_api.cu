@@ -60,7 +60,7 @@ inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
-  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_LIVE, B_ROWS, B_NROWS, B_SLOT, B_FIN, B_LOGITS, B_PART,
+  B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_WDQ, B_LIVE, B_ROWS, B_NROWS, B_SLOT, B_FIN, B_LOGITS, B_PART,
   B_ENT, B_AM, B_ATTN, B_COUNT
 };
 
@@ -101,6 +101,12 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_ACT] = TK * F * a;
   sz[B_YE] = TK * d * 4;  // expert outputs: fp32
   sz[B_XP] = TK * d * a;
+  // e4m3 weights on the tensor-core path: bf16 copies of one layer's matrices (the expert
+  // matrices are the largest; QKV and the output projection reuse the front of the region)
+  sz[B_WDQ] = c.w_dtype == DG_E4M3
+                  ? ((size_t)c.n_experts * 3 * F * d +
+                     (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * hd * d) * 2
+                  : 0;
   sz[B_LIVE] = T;
   sz[B_ROWS] = T * 4;
   sz[B_NROWS] = 4;
@@ -165,6 +171,17 @@ const float *scale_or_null(const dg_config *c, const float *s) {
 
 // ---- one layer's pieces, shared by the step and the append --------------------------------
 
+// The weights the tensor-core GEMMs read: bf16 weights as given; e4m3 weights dequantised into the
+// B_WDQ scratch at element offset `off` (the per-channel scales are applied in the epilogues).
+const void *tc_weight(const dg_config &c, const Ws &ws, const void *w, size_t n, size_t off,
+                      cudaStream_t s, int *rc) {
+  *rc = DG_OK;
+  if (c.w_dtype != DG_E4M3) return w;
+  bf16 *dst = ws.at<bf16>(B_WDQ) + off;
+  *rc = launch_dequant_e4m3(w, n, dst, s);
+  return dst;
+}
+
 int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T, cudaStream_t s) {
   GemmDesc g{};
   g.act = c.act_dtype; g.w = c.w_dtype;
@@ -173,9 +190,13 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
   g.bscale = scale_or_null(&c, w.s_qkv);
   g.M = T; g.N = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim; g.K = c.d_model;
   g.name = "gemm_qkv";
-  if (gemm_tc_supported(c.act_dtype, c.w_dtype, c.d_model))
-    return launch_gemm_tc_dense(ws.at<void>(B_A), T, w.w_qkv, g.N, c.d_model, ws.at<float>(B_QKV),
-                                nullptr, g.N, "gemm_qkv_tc", nullptr, s);
+  if (gemm_tc_supported(c.act_dtype, c.w_dtype, c.d_model)) {
+    int rc;
+    const void *wq = tc_weight(c, ws, w.w_qkv, (size_t)g.N * c.d_model, 0, s, &rc);
+    if (rc != DG_OK) return rc;
+    return launch_gemm_tc_dense(ws.at<void>(B_A), T, wq, g.N, c.d_model, ws.at<float>(B_QKV),
+                                nullptr, g.N, "gemm_qkv_tc", nullptr, s, g.bscale);
+  }
   return launch_gemm_simt(g, EPI_F32, ws.at<void>(B_QKV), g.N, nullptr, s);
 }
 
@@ -200,10 +221,13 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
   g.bscale = scale_or_null(&c, w.s_o);
   g.M = T; g.N = d; g.K = hq;
   g.name = "gemm_o_resid";
-  if (gemm_tc_supported(c.act_dtype, c.w_dtype, hq))
-    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, w.w_o, d, hq, ws.at<float>(B_H),
-                                ws.at<float>(B_X), d, "gemm_o_resid_tc", nullptr, s));
-  else
+  if (gemm_tc_supported(c.act_dtype, c.w_dtype, hq)) {
+    int rc;
+    const void *wo = tc_weight(c, ws, w.w_o, (size_t)d * hq, 0, s, &rc);
+    if (rc != DG_OK) return rc;
+    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, wo, d, hq, ws.at<float>(B_H),
+                                ws.at<float>(B_X), d, "gemm_o_resid_tc", nullptr, s, g.bscale));
+  } else
     DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
   DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
                         ws.at<void>(B_Y), s));
@@ -244,15 +268,22 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
                               ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
                               ws.L->max_tiles, load_out, s));
   if (tc) {
+    int rc;
+    const size_t n_gu = (size_t)E * 2 * F * d, n_dn = (size_t)E * d * F;
+    const void *wgu = tc_weight(c, ws, w.w_gate_up, n_gu, 0, s, &rc);
+    if (rc != DG_OK) return rc;
+    const void *wdn = tc_weight(c, ws, w.w_down, n_dn, n_gu, s, &rc);
+    if (rc != DG_OK) return rc;
+    const bool e4 = c.w_dtype == DG_E4M3;
     DG_TRY(launch_gather_rows(TK, d, k, perm, expert_off, E, y, ws.at<void>(B_XP), s));
-    DG_TRY(launch_gemm_tc_experts(1, w.w_gate_up, E, 2 * F, F, ws.at<void>(B_XP), TK, d,
+    DG_TRY(launch_gemm_tc_experts(1, wgu, E, 2 * F, F, ws.at<void>(B_XP), TK, d,
                                   ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
                                   ws.L->max_tiles, expert_off, ws.at<void>(B_ACT), F,
-                                  "moe_gate_up_tc", nullptr, s));
-    DG_TRY(launch_gemm_tc_experts(0, w.w_down, E, d, F, ws.at<void>(B_ACT), TK, F,
+                                  "moe_gate_up_tc", nullptr, s, e4 ? w.s_gate_up : nullptr));
+    DG_TRY(launch_gemm_tc_experts(0, wdn, E, d, F, ws.at<void>(B_ACT), TK, F,
                                   ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
                                   ws.L->max_tiles, expert_off, ws.at<void>(B_YE), d,
-                                  "moe_down_tc", nullptr, s));
+                                  "moe_down_tc", nullptr, s, e4 ? w.s_down : nullptr));
   } else {
     GemmDesc g1{};
     g1.act = c.act_dtype; g1.w = c.w_dtype;

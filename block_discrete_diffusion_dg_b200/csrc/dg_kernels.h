@@ -24,6 +24,8 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
                     int n, int hd, double theta, const int32_t *cache_len, float *cs,
                     const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
                     uint8_t *token_live, cudaStream_t s);
+// e4m3 codes [n] -> bf16 [n] (n % 16 == 0), exact.
+int launch_dequant_e4m3(const void *src, size_t n, void *dst, cudaStream_t s);
 // in: fp32 rows (residual stream); out: activation type.
 int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
                    int max_rows, int d, double eps, void *out, cudaStream_t s);
@@ -143,13 +145,16 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
 // ---- tensor-core GEMMs (k_gemm_tc.cu) -----------------------------------------------------------
 bool gemm_tc_supported(int act, int w, int K);
 // out[M][N] = A[M][K] W[N][K]^T (+ res[M][N]) in fp32; A has room for roundup(M, 128) rows.
+// scale (or null): per output channel (W row), multiplies the fp32 accumulator.
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
-                         const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s);
+                         const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s,
+                         const float *scale = nullptr);
 // Swap-AB expert GEMM over token tiles of experts_tc_tile_tokens() rows.
 int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
                            int n_assign_max, int K, const GroupTile *tiles,
                            const int32_t *n_tiles_dev, int max_tiles, const int32_t *expert_off,
-                           void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s);
+                           void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s,
+                           const float *scale = nullptr);
 int experts_tc_tile_tokens();
 
 // ---- EB select (k_eb.cu) -------------------------------------------------------------------

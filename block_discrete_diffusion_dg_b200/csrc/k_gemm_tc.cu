@@ -45,6 +45,7 @@ struct Params {
   int F;            // expert FFN width (gate/up half)
   int ld_out;       // row stride of the expert output (F for a, d for Y)
   void *out;        // gate/up: a [assignments][F] (bf16); down: Y [assignments][d] (fp32)
+  const float *scale;  // per output channel (dense: [N]; experts: [E][w_rows]) or null
   int32_t *status;
 };
 
@@ -243,6 +244,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tbase + c * 32, v);
         tmem_ld_wait(v);
         const int nv = min(32, x.n_valid - c * 32);
+        if (p.scale) {  // e4m3 weights: the fp32 accumulator times the output channel's scale
+          if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
+            const float *sc = p.scale + x.col0 + c * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nv) v[j] = __float_as_uint(__uint_as_float(v[j]) * sc[j]);
+          } else {
+            const GroupTile g = p.tiles[u / p.m_tiles];
+            const int arow = (p.kind == K_MOE_GATE)
+                                 ? (q < 2 ? x.row0 + r : p.F + x.row0 + (r - 64))
+                                 : x.row0 + r;
+            const float sc = p.scale[(size_t)g.g * p.w_rows + arow];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * sc);
+          }
+        }
         if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
           const int row = x.row0 + r;
           if (row < p.M) {
@@ -336,15 +353,18 @@ int launch(const CUtensorMap &tmA, const CUtensorMap &tmB, const Params &p, int 
 
 }  // namespace
 
+// bf16 activations with bf16 weights, or with e4m3 weights that the caller dequantises to bf16
+// first (the scales are applied in the epilogue).
 bool gemm_tc_supported(int act, int w, int K) {
-  return act == DG_BF16 && w == DG_BF16 && K % BK == 0 && K >= BK;
+  return act == DG_BF16 && (w == DG_BF16 || w == DG_E4M3) && K % BK == 0 && K >= BK;
 }
 
 // Dense: out[M][N] = A[M][K] * W[N][K]^T (+ res[M][N]), fp32 output.  At batch 1 these are
 // latency-bound weight streams (M = 256 tokens), so the channel tiles are narrow (32, or 16 for
 // N <= 256) to spread each weight matrix over enough CTAs.
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
-                         const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s) {
+                         const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s,
+                         const float *scale) {
   const int BN = N <= 256 ? 16 : 64;
   const int M_alloc = (M + BM - 1) / BM * BM;  // A has room for whole tiles (caller's layout)
   CUtensorMap ta, tb;
@@ -362,6 +382,7 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
   p.bn = BN;
   p.out_f32 = out;
   p.res = res;
+  p.scale = scale;
   p.ldo = ldo;
   p.status = st;
   const int units = p.m_tiles * ((N + BN - 1) / BN);
@@ -386,7 +407,8 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
 int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F, const void *X,
                            int n_assign_max, int K, const GroupTile *tiles,
                            const int32_t *n_tiles_dev, int max_tiles, const int32_t *expert_off,
-                           void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s) {
+                           void *out, int ld_out, const char *name, int32_t *st, cudaStream_t s,
+                           const float *scale) {
   constexpr int BN_MAX = DG_MOE_BN, B_BOX = 32;
   CUtensorMap ta, tb;
   int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, (uint64_t)E * w_rows,
@@ -406,6 +428,7 @@ int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F,
   p.m_tiles = gate_up ? F / 64 : w_rows / BM;
   p.ld_out = ld_out;
   p.out = out;
+  p.scale = scale;
   p.status = st;
   return launch<BN_MAX, DG_MOE_STAGES, B_BOX>(ta, tb, p, max_tiles * p.m_tiles, name, s,
                                               DG_MOE_CTAS_PER_SM);

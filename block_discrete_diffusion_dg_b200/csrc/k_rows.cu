@@ -186,6 +186,37 @@ __global__ void __launch_bounds__(256) prologue_kernel(
   if (threadIdx.x == 0) *n_rows = base;
 }
 
+// e4m3 -> bf16, exact (every e4m3 value is a bf16 value); 16 codes per thread step.  The
+// per-output-channel scales stay separate and are applied to the fp32 accumulators.
+__global__ void dequant_e4m3_kernel(const uint4 *__restrict__ src, size_t n16, uint4 *dst) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 v = src[i];
+    const uint8_t *c = reinterpret_cast<const uint8_t *>(&v);
+    uint4 o[2];
+    bf16 *ob = reinterpret_cast<bf16 *>(o);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      fp8 f;
+      f.__x = c[j];
+      ob[j] = __float2bfloat16_rn(float(f));
+    }
+    dst[2 * i] = o[0];
+    dst[2 * i + 1] = o[1];
+  }
+}
+
+int launch_dequant_e4m3(const void *src, size_t n, void *dst, cudaStream_t s) {
+  if (n == 0) return DG_OK;
+  if (n % 16) return DG_ERR_UNSUPPORTED;
+  const size_t n16 = n / 16;
+  size_t blocks = (n16 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  note_launch(s, "dequant_e4m3");
+  dequant_e4m3_kernel<<<(unsigned)blocks, 256, 0, s>>>((const uint4 *)src, n16, (uint4 *)dst);
+  return check_launch("dequant_e4m3");
+}
+
 int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const void *emb, int rows,
                     int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
                     int n, int hd, double theta, const int32_t *cache_len, float *cs,
