@@ -215,6 +215,30 @@ def dist_setup(args):
     return world, rank, local
 
 
+def barrier(world: int) -> None:
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (a device tensor under NCCL, a host one under gloo)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(units_per_rank: float, ms_local: float, world: int) -> tuple:
+    """Whole-job rate of `world` replicas that each processed `units_per_rank` units: all ranks'
+    units / the slowest rank's device time.  Returns (units per second, max ms)."""
+    ms = max_over_ranks(ms_local, world)
+    return world * units_per_rank / (ms / 1e3), ms
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: timed on the host cores, rank 0 only."""
     import synth
@@ -295,28 +319,41 @@ def run_generate(args, world, rank):
                            kv["cache_len"], cap, ws, status, stream)
         return steps
 
-    generate()                              # warm-up
+    for _ in range(args.warmup):
+        generate()
     torch.cuda.synchronize()
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    barrier(world)
+    clocks.start()
+    time.sleep(0.3)
     n0 = B.dg_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     steps = generate()
     e1.record(stream)
     torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
     if B.dg_read_status(status) != B.DG_OK:
         raise RuntimeError("device status set during generation")
     launches = B.dg_launch_count() - n0
-    ms = e0.elapsed_time(e1)
+    rate, ms = replica_rate(steps, e0.elapsed_time(e1), world)
     toks = cfg.n_canvases * cfg.canvas * cfg.batch
     peaks, peak_src = load_peaks()
-    line = {"metric": METRIC, "value": round(steps / (ms / 1e3), 3), "unit": "steps/s",
-            "n_gpus": world, "steps": steps, "warmup": 1, "ms_per_step": round(ms / steps, 4),
+    line = {"metric": METRIC, "value": round(rate, 3), "unit": "steps/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / steps, 4), "clocks": clk,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random-init weights, random prompt ids)",
             "config": {"workload": workload_desc(cfg) + f"; generate {cfg.n_canvases} canvases, "
                        f"at most {cfg.max_steps} steps each, prefill not timed",
                        "batch": cfg.batch, "mode": "generate"},
-            "output_tok_s": round(toks / (ms / 1e3), 2), "gpu_launches": int(launches),
+            "output_tok_s": round(world * toks / (ms / 1e3), 2), "gpu_launches": int(launches),
             "impl": "dg", "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -354,17 +391,6 @@ def run_dg(args, world, rank, local):
                          st["done"], st["step"], cfg.max_steps, cfg.gamma, kv["k"], kv["v"],
                          kv["cache_len"], cap, None, None, None, ws, status, stream,
                          expert_load=expert_load)
-
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world > 1:
-            t = torch.tensor([x], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            return float(t.item())
-        return x
 
     for i in range(args.warmup):
         one_step(i)
@@ -406,7 +432,7 @@ def run_dg(args, world, rank, local):
     except Exception:
         pass
     clocks = ClockSampler(uuid)
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
@@ -419,14 +445,13 @@ def run_dg(args, world, rank, local):
             one_step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     clk = clocks.stop()
-    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    steps_s, ms = replica_rate(args.steps, ev0.elapsed_time(ev1), world)
     rc = B.dg_read_status(status)
     if rc != B.DG_OK:
         raise RuntimeError(f"device status {B.STATUS_NAMES.get(rc, rc)} in the timed region")
     ms_step = ms / args.steps
-    steps_s = world * args.steps / (ms / 1e3)
     launches = per_step_launches * args.steps
 
     # ---- profile pass: the same steps with a CUDA event before every kernel, captured into one
@@ -518,9 +543,10 @@ def run_dg(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in pin[0].values())
     d2h = sum(t.numel() * t.element_size() for t in out_h.values())
     e_steps = max(4, args.steps // 2)
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
-    e0 = time.perf_counter()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
     for i in range(e_steps):
         src = pin[i % ns]
         for k in st:
@@ -531,10 +557,13 @@ def run_dg(args, world, rank, local):
         for k in out_h:
             out_h[k].copy_(st[k], non_blocking=True)
         stream.synchronize()       # the caller reads the committed tokens and the done flag
-    e_s = max_over_ranks(time.perf_counter() - e0)
-    e2e = {"value": world * e_steps / e_s, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e_rate, _ = replica_rate(e_steps, x0.elapsed_time(x1), world)
+    e2e = {"value": round(e_rate, 3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h,
-           "note": "direct calls (no graph), host state copied in and result read back every step"}
+           "note": "direct calls (no graph), host state copied in from pinned memory and the "
+                   "result read back every step; CUDA events around the loop"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -551,7 +580,7 @@ def run_dg(args, world, rank, local):
                          f"canvas, experts e < E/{args.ref_frac} and an LM-head vocab slice of "
                          f"V/{args.ref_frac}, both scaled by {args.ref_frac}"}
 
-    tok_s = steps_s * float(np.mean(committed)) / cfg.batch
+    tok_s = steps_s * float(np.mean(committed))     # tokens committed over all canvases
     line = {"metric": METRIC, "value": round(steps_s, 3), "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",

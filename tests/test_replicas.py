@@ -1,0 +1,84 @@
+"""The benchmark's multi-rank host logic on CPU: world-size-2 gloo process groups.
+
+Every workload is independent per canvas, so several GPUs run replicas with no collective on the
+data path.  What crosses ranks is only the timing: a barrier around the timed region, the max of
+the per-rank device times, and the whole-job rate (all ranks' units / the slowest rank's time).
+These tests run that logic in two gloo ranks, and run the benchmark's reference arm under
+torchrun with two ranks (rank 0 alone prints its line; rank 1 exits 0 without work)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, ms_by_rank, units, out):
+    import torch.distributed as dist
+    from datetime import timedelta
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import bench
+        bench.barrier(world)
+        m = bench.max_over_ranks(ms_by_rank[rank], world)
+        rate, ms = bench.replica_rate(units, ms_by_rank[rank], world)
+        out.put((rank, m, rate, ms))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replica_rate_is_all_units_over_slowest_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world, port = 2, _free_port()
+    ms_by_rank = [12.5, 20.0]          # rank 1 is the slow one
+    units = 40                         # steps each rank ran
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, ms_by_rank, units, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, m, rate, ms in res:
+        assert m == 20.0 and ms == 20.0
+        assert rate == pytest.approx(world * units / 0.020)
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.0, 1) == 3.0
+    rate, ms = bench.replica_rate(10, 5.0, 1)
+    assert ms == 5.0 and rate == pytest.approx(2000.0)
+
+
+def test_reference_arm_under_torchrun_two_ranks(tmp_path):
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+           "--gpus", "2", "--steps", "2", "--warmup", "3"]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    r = subprocess.run(cmd, cwd=str(tmp_path), env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1                   # rank 0 only
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 2
+    assert d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
