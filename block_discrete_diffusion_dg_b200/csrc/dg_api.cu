@@ -439,7 +439,6 @@ int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
                    int cache_cap, const void *k_new, const void *v_new, int causal,
                    const int32_t *done, void *out, void *ws, size_t ws_bytes,
                    int32_t *dev_status, void *stream) {
-  (void)dev_status;
   if (!cfg_ok(cfg) || batch <= 0 || n_tokens <= 0 || cache_cap < 0) return DG_ERR_INVALID_ARG;
   if (!q || !cache_len || !k_new || !v_new || !out) return DG_ERR_INVALID_ARG;
   if (cache_cap > 0 && (!k_cache || !v_cache)) return DG_ERR_INVALID_ARG;
@@ -447,7 +446,7 @@ int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
   DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
   return launch_attention(cfg->act_dtype, batch, n_tokens, cfg->n_q_heads, cfg->n_kv_heads,
                           cfg->head_dim, q, k_cache, v_cache, cache_len, cache_cap, k_new, v_new,
-                          causal ? 1 : 0, done, out, (char *)ws + L.off[B_ATTN],
+                          causal ? 1 : 0, done, out, (char *)ws + L.off[B_ATTN], dev_status,
                           (cudaStream_t)stream);
 }
 
@@ -558,7 +557,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
     DG_TRY(launch_attention(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
                             w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
                             w.at<void>(B_VN), 1, nullptr, w.at<void>(B_O),
-                            w.at<void>(B_ATTN), s));
+                            w.at<void>(B_ATTN), dev_status, s));
     bool tiles_ready = false;
     DG_TRY(attn_out_and_route(c, lw, w, T, nullptr, nullptr, &tiles_ready, s,
                               forced_topk ? forced_topk + (size_t)l * T * c.top_k : nullptr));
@@ -612,7 +611,8 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                             cache_cap, dev_status, s));
     DG_TRY(launch_attention(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,
                             w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
-                            w.at<void>(B_VN), 0, done, w.at<void>(B_O), w.at<void>(B_ATTN), s));
+                            w.at<void>(B_VN), 0, done, w.at<void>(B_O), w.at<void>(B_ATTN),
+                            dev_status, s));
     int32_t *load_l = expert_load ? expert_load + (size_t)l * c.n_experts : nullptr;
     bool tiles_ready = false;
     DG_TRY(attn_out_and_route(c, lw, w, T, live, load_l, &tiles_ready, s,

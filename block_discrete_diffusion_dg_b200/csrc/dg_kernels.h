@@ -72,15 +72,16 @@ int launch_add_cache_len(int batch, int n, int cap, int32_t *cache_len, cudaStre
 int launch_attention(int act, int batch, int n, int Hq, int Hkv, int hd, const void *q,
                      const void *k_cache, const void *v_cache, const int32_t *cache_len,
                      int cap, const void *k_new, const void *v_new, int causal,
-                     const int32_t *done, void *out, void *ws, cudaStream_t s);
+                     const int32_t *done, void *out, void *ws, int32_t *st, cudaStream_t s);
 size_t attention_ws_bytes(int act, int batch, int n, int Hq, int Hkv, int hd, int cap);
-// bf16 tensor-core path (k_attn_tc.cu): split-KV flash attention + merge.
+// bf16 tensor-core path (k_attn_tc.cu): split-KV flash attention (tcgen05 for head_dim 128,
+// mma.sync otherwise) + merge.  st: device status word (bounded-wait timeouts), may be NULL.
 bool attention_tc_supported(int act, int Hq, int Hkv, int hd);
 size_t attention_tc_ws_bytes(int batch, int n, int Hq, int Hkv, int hd, int cap);
 int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q,
                         const void *k_cache, const void *v_cache, const int32_t *cache_len, int cap,
                         const void *k_new, const void *v_new, int causal, const int32_t *done,
-                        void *out, void *ws, cudaStream_t s);
+                        void *out, void *ws, int32_t *st, cudaStream_t s);
 
 // ---- MoE (k_moe.cu) ---------------------------------------------------------------------------
 int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *y,

@@ -164,11 +164,11 @@ size_t attention_ws_bytes(int act, int batch, int n, int Hq, int Hkv, int hd, in
 int launch_attention(int act, int batch, int n, int Hq, int Hkv, int hd, const void *q,
                      const void *k_cache, const void *v_cache, const int32_t *cache_len, int cap,
                      const void *k_new, const void *v_new, int causal, const int32_t *done,
-                     void *out, void *ws, cudaStream_t s) {
+                     void *out, void *ws, int32_t *st, cudaStream_t s) {
   if (n <= 0 || batch <= 0) return DG_OK;
   if (attention_tc_supported(act, Hq, Hkv, hd))
     return launch_attention_tc(batch, n, Hq, Hkv, hd, q, k_cache, v_cache, cache_len, cap, k_new,
-                               v_new, causal, done, out, ws, s);
+                               v_new, causal, done, out, ws, st, s);
   dim3 grid((n + QB - 1) / QB, Hq, batch);
   if (act == DG_F32)
     return run<float>(hd, grid, s, n, Hq, Hkv, q, k_cache, v_cache, cache_len, cap, k_new, v_new,

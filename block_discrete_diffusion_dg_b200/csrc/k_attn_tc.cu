@@ -18,6 +18,7 @@
 // Each thread converts the V chunks it loaded, in place, once they have landed.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
+#include "tc_common.cuh"
 #include "tc_host.h"
 
 namespace dg {
@@ -345,6 +346,402 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
   }
 }
 
+// ================================================================================================
+// tcgen05 path (head_dim 128).  One CTA = the same 128 query rows as above x one key split, with
+// both products on the 5th-generation tensor cores and the accumulators in tensor memory:
+//   S_i = Q K_i^T   (M 128 rows, N 128 keys, K 128 = head_dim; bf16 operands from shared memory)
+//   O  += P_i V_i   (M 128 rows, N 128 = head_dim, K 128 keys; P fp16 from tensor memory, V fp16
+//                    in shared memory, read MN-major)
+// Warp roles (256 threads):
+//   warp 0     TMA: the Q tile once, then K and V tiles of 128 keys into 3-stage rings;
+//   warp 1     owns the 512 TMEM columns (S0, S1, O, P0, P1) and issues the MMAs:
+//              S_0, S_1, then per tile PV_i followed by S_(i+2) into the S buffer just released;
+//   warps 2-3  convert each landed V tile from bf16 to fp16 in place and zero the rows past the
+//              last valid key (so masked keys contribute exactly 0 * 0);
+//   warps 4-7  softmax, one query row per thread (= TMEM lane): read S_i, mask, running max in the
+//              log2 domain, P_i = 2^(t - m) written back to TMEM as fp16 pairs, row sum in fp32.
+// The running maximum is applied lazily: O is rescaled (read, scaled, written back in TMEM) only
+// when a row's maximum grows by more than 2^8, so between rescales P can reach 256 (exact in
+// fp16's range; the final O / l is unchanged because O and l always share the same base).
+// Every wait is bounded; on expiry the kernel records DG_ERR_TIMEOUT, lets issued copies and
+// MMAs finish, frees TMEM and returns.
+constexpr int T5_HD = 128, T5_KT = 128, T5_KS = 3, T5_VS = 3, T5_THR = 256;
+constexpr int T5_HALF = 128 * 128;       // one box: 128 rows x 64 bf16 (128-byte rows) = 16 KB
+constexpr int T5_TILE = 2 * T5_HALF;     // 128 rows x 128 head dims = 32 KB
+constexpr uint32_t T5_COL_S = 0, T5_COL_O = 256, T5_COL_P = 384, T5_TMEM_COLS = 512;
+constexpr float T5_RESCALE = 8.f;        // log2 of the largest P between rescales
+constexpr size_t T5_SMEM = 1024 + (size_t)T5_TILE * (1 + T5_KS + T5_VS) + 256;
+constexpr unsigned FULL = 0xffffffffu;
+
+struct T5Args {
+  const int32_t *cache_len, *done;
+  int n, Hq, Hkv, cap, causal, splits, chunk_tiles;
+  bf16 *out;          // splits == 1
+  float *part_o;      // [splits][B][Hq][n][HD]
+  float2 *part_ml;    // [splits][B][Hq][n]
+  int32_t *status;
+};
+
+__device__ __forceinline__ void t5_fail(int32_t *st, volatile int *abort_flag) {
+  set_status(st, DG_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+
+__global__ void __launch_bounds__(T5_THR, 1)
+    attn_tc5_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmKc,
+                    const __grid_constant__ CUtensorMap tmVc,
+                    const __grid_constant__ CUtensorMap tmKn,
+                    const __grid_constant__ CUtensorMap tmVn, T5Args a) {
+  using namespace tc;
+  extern __shared__ uint8_t t5_smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)t5_smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sQ = smem;
+  uint8_t *sK = sQ + T5_TILE;
+  uint8_t *sV = sK + T5_KS * T5_TILE;
+  uint64_t *q_full = reinterpret_cast<uint64_t *>(sV + T5_VS * T5_TILE);
+  uint64_t *k_full = q_full + 1, *k_empty = k_full + T5_KS;
+  uint64_t *v_full = k_empty + T5_KS, *v_ready = v_full + T5_VS, *v_empty = v_ready + T5_VS;
+  uint64_t *s_full = v_empty + T5_VS, *p_full = s_full + 2, *pv_done = p_full + 2;
+  uint64_t *mma_fin = pv_done + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_fin + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int split = blockIdx.z % a.splits, b = blockIdx.z / a.splits;
+  if (a.done && a.done[b]) return;  // uniform across the block
+  const int g = blockIdx.y, rep = a.Hq / a.Hkv, qpc = ROWS / rep, i0 = blockIdx.x * qpc;
+  const int len = min(max(a.cache_len[b], 0), a.cap);
+  const int tcache = (len + T5_KT - 1) / T5_KT;
+  int tiles = tcache + (a.n + T5_KT - 1) / T5_KT;
+  if (a.causal) tiles = tcache + (min(a.n, i0 + qpc) - 1) / T5_KT + 1;  // later canvas keys unseen
+  const int t_begin = split * a.chunk_tiles;
+  const int N = max(0, min(tiles, t_begin + a.chunk_tiles) - t_begin);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slab_c = (b * a.Hkv + g) * a.cap, slab_n = (b * a.Hkv + g) * a.n;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < T5_KS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < T5_VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_ready[s], 2);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&pv_done[x], 1);
+    }
+    mbar_init(mma_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmKc);
+    tma_prefetch_desc(&tmVc);
+    tma_prefetch_desc(&tmKn);
+    tma_prefetch_desc(&tmVn);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, T5_TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // tile i of this split: cache rows [j0, j0 + 128) or canvas rows; `valid` keys in it
+  auto tile_src = [&](int i, bool &cache, int &row, int &j0, int &valid) {
+    const int t = t_begin + i;
+    cache = t < tcache;
+    j0 = cache ? t * T5_KT : (t - tcache) * T5_KT;
+    row = (cache ? slab_c : slab_n) + j0;
+    valid = min(T5_KT, (cache ? len : a.n) - j0);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t armed_k = 0, armed_v = 0;  // tiles whose copies were issued
+      bool ok = true;
+      mbar_expect_tx(q_full, T5_TILE);
+      for (int hl = 0; hl < rep; ++hl)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_2d(sQ + hf * T5_HALF + hl * qpc * 128, &tmQ, q_full,
+                      (g * rep + hl) * T5_HD + hf * 64, b * a.n + i0);
+      for (int i = 0; i < N && ok && !*abort_flag; ++i) {
+        bool cache;
+        int row, j0, valid;
+        tile_src(i, cache, row, j0, valid);
+        const int ks = i % T5_KS, vs = i % T5_VS;
+        if (!mbar_wait(&k_empty[ks], ((i / T5_KS) & 1) ^ 1)) { ok = false; break; }
+        mbar_expect_tx(&k_full[ks], T5_TILE);
+        const CUtensorMap *tk = cache ? &tmKc : &tmKn;
+        tma_load_2d(sK + ks * T5_TILE, tk, &k_full[ks], 0, row);
+        tma_load_2d(sK + ks * T5_TILE + T5_HALF, tk, &k_full[ks], 64, row);
+        armed_k = i + 1;
+        if (!mbar_wait(&v_empty[vs], ((i / T5_VS) & 1) ^ 1)) { ok = false; break; }
+        mbar_expect_tx(&v_full[vs], T5_TILE);
+        const CUtensorMap *tv = cache ? &tmVc : &tmVn;
+        tma_load_2d(sV + vs * T5_TILE, tv, &v_full[vs], 0, row);
+        tma_load_2d(sV + vs * T5_TILE + T5_HALF, tv, &v_full[vs], 64, row);
+        armed_v = i + 1;
+      }
+      if (!ok) t5_fail(a.status, abort_flag);
+      // the copies in flight land before the CTA's shared memory can go away
+      (void)mbar_wait(q_full, 0);
+      for (uint32_t i = armed_k > T5_KS ? armed_k - T5_KS : 0; i < armed_k; ++i)
+        (void)mbar_wait(&k_full[i % T5_KS], (i / T5_KS) & 1);
+      for (uint32_t i = armed_v > T5_VS ? armed_v - T5_VS : 0; i < armed_v; ++i)
+        (void)mbar_wait(&v_full[i % T5_VS], (i / T5_VS) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(ROWS, T5_KT);
+      const uint32_t id_p = idesc_f16_bmn(ROWS, T5_HD);
+      bool ok = mbar_wait(q_full, 0);
+      fence_after();
+      auto issue_s = [&](int i) -> bool {
+        const int ks = i % T5_KS;
+        if (!mbar_wait(&k_full[ks], (i / T5_KS) & 1)) return false;
+        fence_after();
+        const uint32_t d = tmem + T5_COL_S + (uint32_t)(i & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < T5_HD / 16; ++kk) {
+          const int hf = kk >> 2, k4 = kk & 3;
+          const uint64_t ad = sdesc_sw128(sQ + hf * T5_HALF) + 2 * k4;
+          const uint64_t bd = sdesc_sw128(sK + ks * T5_TILE + hf * T5_HALF) + 2 * k4;
+          mma_bf16(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
+        }
+        commit(&k_empty[ks]);
+        commit(&s_full[i & 1]);
+        return true;
+      };
+      if (ok && N > 0) ok = issue_s(0);
+      if (ok && N > 1) ok = issue_s(1);
+      for (int i = 0; ok && i < N && !*abort_flag; ++i) {
+        const int vs = i % T5_VS;
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1) ||
+            !mbar_wait(&v_ready[vs], (i / T5_VS) & 1)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t pa = tmem + T5_COL_P + (uint32_t)(i & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < T5_KT / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128_mn(sV + vs * T5_TILE + kk * 16 * 128, T5_HALF);
+          mma_f16_ts(tmem + T5_COL_O, pa + kk * 8, bd, id_p, (i | kk) != 0 ? 1u : 0u);
+        }
+        commit(&v_empty[vs]);
+        commit(&pv_done[i & 1]);
+        if (i + 2 < N) ok = issue_s(i + 2);
+      }
+      if (!ok) t5_fail(a.status, abort_flag);
+      commit(mma_fin);  // every MMA issued above has completed when this phase does
+      (void)mbar_wait(mma_fin, 0);
+    }
+  } else if (warp < 4) {
+    const int ct = threadIdx.x - 64;  // 0..63
+    for (int i = 0; i < N; ++i) {
+      if (__any_sync(FULL, *abort_flag != 0)) break;
+      const int vs = i % T5_VS;
+      if (!__all_sync(FULL, mbar_wait(&v_full[vs], (i / T5_VS) & 1))) {
+        t5_fail(a.status, abort_flag);
+        break;
+      }
+      bool cache;
+      int row, j0, valid;
+      tile_src(i, cache, row, j0, valid);
+      uint8_t *base = sV + vs * T5_TILE;
+      // 16-byte chunk c sits in key row (c mod 1024) / 8 of its half (the swizzle only permutes
+      // chunks within a row), so the conversion is in place and per chunk
+      for (int c = ct; c < T5_TILE / 16; c += 64) {
+        uint4 *pc = reinterpret_cast<uint4 *>(base + c * 16);
+        if (((c & 1023) >> 3) < valid) bf16x8_to_f16x8(pc);
+        else *pc = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v_ready[vs]);
+    }
+  } else {
+    const int q4 = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = q4 * 32 + lane;            // query row of the tile
+    const int hl = r / qpc, pos = i0 + r % qpc, h = g * rep + hl;
+    const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
+    const float sl2 = 1.4426950408889634f / sqrtf((float)T5_HD);
+    float m_use = -INFINITY, l = 0.f;
+    bool ok = true;
+    // Control flow stays warp-uniform (votes on every exit and on the rescale decision): the TMEM
+    // loads and stores below are .sync.aligned and need all 32 lanes.
+    for (int i = 0; i < N; ++i) {
+      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+      if (!__all_sync(FULL, mbar_wait(&s_full[i & 1], (i >> 1) & 1))) {
+        t5_fail(a.status, abort_flag);
+        ok = false;
+        break;
+      }
+      fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lrow + T5_COL_S + (uint32_t)(i & 1) * 128 + c * 32, sr[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+      bool cache;
+      int row, j0, valid;
+      tile_src(i, cache, row, j0, valid);
+      int lim = valid;
+      if (a.causal && !cache) lim = min(lim, pos - j0 + 1);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float t = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) * sl2 : -INFINITY;
+          sr[c][j] = __float_as_uint(t);
+          mx = fmaxf(mx, t);
+        }
+      const float m_new = fmaxf(m_use, mx);
+      // a row whose maximum grew by more than 2^8 needs O rescaled; the whole warp then rescales
+      // (factor 1 where nothing changed; a row with nothing accumulated yet only takes m_new)
+      if (__any_sync(FULL, m_use != -INFINITY && m_new > m_use + T5_RESCALE)) {
+        const float f = m_use == -INFINITY ? 1.f : exp2f(m_use - m_new);
+        if (i >= 1 && !__all_sync(FULL, mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) {
+          t5_fail(a.status, abort_flag);
+          ok = false;
+          break;
+        }
+        fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lrow + T5_COL_O + c * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+          tmem_st32(tmem + lrow + T5_COL_O + c * 32, o);
+        }
+        tmem_st_wait();
+        l *= f;
+        m_use = m_new;
+      } else if (m_use == -INFINITY) {
+        m_use = m_new;  // nothing accumulated yet (O is exactly 0 or not yet written)
+      }
+      const float base = m_use == -INFINITY ? 0.f : m_use;
+      uint32_t pk[2][32];
+      float ps = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float p0 = exp2f(__uint_as_float(sr[c][j]) - base);
+          const float p1 = exp2f(__uint_as_float(sr[c][j + 1]) - base);
+          ps += p0 + p1;
+          pk[c >> 1][(c & 1) * 16 + j / 2] = pack_f16(p0, p1);
+        }
+      l += ps;
+      // P buffer (i & 1) was last read by PV_(i-2)
+      if (i >= 2 && !__all_sync(FULL, mbar_wait(&pv_done[i & 1], ((i - 2) >> 1) & 1))) {
+        t5_fail(a.status, abort_flag);
+        ok = false;
+        break;
+      }
+      fence_after();
+      tmem_st32(tmem + lrow + T5_COL_P + (uint32_t)(i & 1) * 64, pk[0]);
+      tmem_st32(tmem + lrow + T5_COL_P + (uint32_t)(i & 1) * 64 + 32, pk[1]);
+      tmem_st_wait();
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+    }
+    if (ok && N > 0) {
+      if (!__all_sync(FULL, mbar_wait(&pv_done[(N - 1) & 1], ((N - 1) >> 1) & 1))) {
+        t5_fail(a.status, abort_flag);
+        ok = false;
+      }
+      fence_after();
+    }
+    const bool row_ok = pos < a.n;  // guards the stores only; every lane reads TMEM
+    if (ok) {
+      if (a.splits == 1) {
+        const float il = l > 0.f ? 1.f / l : 0.f;
+        bf16 *dst = a.out + (((size_t)b * a.n + min(pos, a.n - 1)) * a.Hq + h) * T5_HD;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lrow + T5_COL_O + c * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 v;
+            uint32_t *w = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 t = __floats2bfloat162_rn(__uint_as_float(o[j + 2 * e]) * il,
+                                                             __uint_as_float(o[j + 2 * e + 1]) * il);
+              w[e] = *reinterpret_cast<const uint32_t *>(&t);
+            }
+            if (row_ok) *reinterpret_cast<uint4 *>(dst + c * 32 + j) = v;
+          }
+        }
+      } else {
+        const int B = gridDim.z / a.splits;
+        const size_t pr = (((size_t)split * B + b) * a.Hq + h) * a.n + min(pos, a.n - 1);
+        float *dst = a.part_o + pr * T5_HD;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          if (N > 0) {
+            tmem_ld32(tmem + lrow + T5_COL_O + c * 32, o);
+            tmem_ld_wait(o);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<uint4 *>(dst + c * 32 + j) =
+                  make_uint4(o[j], o[j + 1], o[j + 2], o[j + 3]);
+          }
+        }
+        if (row_ok) a.part_ml[pr] = make_float2(m_use, l);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, T5_TMEM_COLS);
+  }
+}
+
+// Split plan of the tcgen05 path: tiles of 128 keys; as many splits as fill one wave.
+void plan5(int batch, int n, int Hq, int Hkv, int cap, int *splits, int *chunk_tiles) {
+  const int tiles = (cap + T5_KT - 1) / T5_KT + (n + T5_KT - 1) / T5_KT;
+  const int qpc = ROWS / (Hq / Hkv);
+  const int base = ((n + qpc - 1) / qpc) * Hkv * batch;
+  int s = num_sms() / (base > 0 ? base : 1);
+  if (s > tiles) s = tiles;
+  if (s > MAX_SPLITS) s = MAX_SPLITS;
+  if (s < 1) s = 1;
+  const int c = (tiles + s - 1) / s;
+  *chunk_tiles = c;
+  *splits = (tiles + c - 1) / c;
+}
+
+bool use_tc5(int batch, int n, int Hq, int Hkv, int hd, int cap) {
+  const int rep = Hq / Hkv;
+  return hd == T5_HD && rep <= 16 && (size_t)batch * Hkv * (size_t)(cap > n ? cap : n) < (1u << 31) &&
+         (size_t)batch * n < (1u << 31);
+}
+
 // Split-KV plan: as many key splits as fill one wave of CTAs (one CTA per SM at this kernel's
 // register use), at least one tile of keys per split, at most MAX_SPLITS.
 void plan(int batch, int n, int Hq, int Hkv, int cap, int *splits, int *chunk) {
@@ -371,16 +768,75 @@ bool attention_tc_supported(int act, int Hq, int Hkv, int hd) {
 
 size_t attention_tc_ws_bytes(int batch, int n, int Hq, int Hkv, int hd, int cap) {
   int s, c;
-  plan(batch, n, Hq, Hkv, cap, &s, &c);
+  if (use_tc5(batch, n, Hq, Hkv, hd, cap)) plan5(batch, n, Hq, Hkv, cap, &s, &c);
+  else plan(batch, n, Hq, Hkv, cap, &s, &c);
   if (s == 1) return 0;
   const size_t rows = (size_t)s * batch * Hq * n;
   return rows * hd * 4 + 256 + rows * sizeof(float2);
 }
 
+namespace {
+
+int launch_tc5(int batch, int n, int Hq, int Hkv, const void *q, const void *k_cache,
+               const void *v_cache, const int32_t *cache_len, int cap, const void *k_new,
+               const void *v_new, int causal, const int32_t *done, void *out, void *ws,
+               int32_t *st, cudaStream_t s) {
+  T5Args a;
+  a.cache_len = cache_len;
+  a.done = done;
+  a.n = n;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.cap = cap;
+  a.causal = causal;
+  a.status = st;
+  plan5(batch, n, Hq, Hkv, cap, &a.splits, &a.chunk_tiles);
+  a.out = (bf16 *)out;
+  const size_t rows = (size_t)a.splits * batch * Hq * n;
+  a.part_o = (float *)ws;
+  a.part_ml = (float2 *)((char *)ws + ((rows * T5_HD * 4 + 255) & ~(size_t)255));
+  const int qpc = ROWS / (Hq / Hkv);
+  CUtensorMap tq, tkc, tvc, tkn, tvn;
+  const CUtensorMapDataType bt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  int rc = make_tmap_2d(&tq, bt, 2, q, (uint64_t)Hq * T5_HD, (uint64_t)batch * n,
+                        (uint64_t)Hq * T5_HD * 2, 64, qpc);
+  if (rc == DG_OK)
+    rc = make_tmap_2d(&tkn, bt, 2, k_new, T5_HD, (uint64_t)batch * Hkv * n, T5_HD * 2, 64, T5_KT);
+  if (rc == DG_OK)
+    rc = make_tmap_2d(&tvn, bt, 2, v_new, T5_HD, (uint64_t)batch * Hkv * n, T5_HD * 2, 64, T5_KT);
+  if (rc == DG_OK && cap > 0 && k_cache && v_cache) {
+    rc = make_tmap_2d(&tkc, bt, 2, k_cache, T5_HD, (uint64_t)batch * Hkv * cap, T5_HD * 2, 64,
+                      T5_KT);
+    if (rc == DG_OK)
+      rc = make_tmap_2d(&tvc, bt, 2, v_cache, T5_HD, (uint64_t)batch * Hkv * cap, T5_HD * 2, 64,
+                        T5_KT);
+  } else {
+    tkc = tkn;  // no cache rows: never read
+    tvc = tvn;
+  }
+  if (rc != DG_OK) return rc;
+  dim3 grid((n + qpc - 1) / qpc, Hkv, batch * a.splits);
+  note_launch(s, "attn_tc");
+  cudaFuncSetAttribute(attn_tc5_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T5_SMEM);
+  attn_tc5_kernel<<<grid, T5_THR, T5_SMEM, s>>>(tq, tkc, tvc, tkn, tvn, a);
+  rc = check_launch("attn_tc");
+  if (rc != DG_OK || a.splits == 1) return rc;
+  note_launch(s, "attn_merge");
+  const int warps = batch * Hq * n;
+  attn_merge_kernel<128><<<(warps + 7) / 8, 256, 0, s>>>(a.splits, batch, Hq, n, a.part_o,
+                                                          a.part_ml, done, (bf16 *)out);
+  return check_launch("attn_merge");
+}
+
+}  // namespace
+
 int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q,
                         const void *k_cache, const void *v_cache, const int32_t *cache_len, int cap,
                         const void *k_new, const void *v_new, int causal, const int32_t *done,
-                        void *out, void *ws, cudaStream_t s) {
+                        void *out, void *ws, int32_t *st, cudaStream_t s) {
+  if (use_tc5(batch, n, Hq, Hkv, hd, cap))
+    return launch_tc5(batch, n, Hq, Hkv, q, k_cache, v_cache, cache_len, cap, k_new, v_new, causal,
+                      done, out, ws, st, s);
   AttnArgs a;
   a.q = (const bf16 *)q;
   a.kc = (const bf16 *)k_cache;

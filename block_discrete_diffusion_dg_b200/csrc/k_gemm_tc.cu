@@ -232,9 +232,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t aph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      if (*abort_flag) break;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
       const Unit x = decode<BN_MAX>(p, u);
-      if (!mbar_wait(&tfull[acc], aph)) { fail(p.status, abort_flag); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph))) {
+        fail(p.status, abort_flag);
+        break;
+      }
       fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE);
       const int r = q * 32 + lane;  // accumulator row of this thread

@@ -162,9 +162,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t aph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      if (*abort_flag) break;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
       const int mt = u % m_tiles, nt = u / m_tiles;
-      if (!mbar_wait(&tfull[acc], aph)) { fail(p.status, abort_flag); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph))) {
+        fail(p.status, abort_flag);
+        break;
+      }
       fence_after();
       const int row = mt * BM + q * 32 + lane;
       const bool row_ok = row < n_rows;

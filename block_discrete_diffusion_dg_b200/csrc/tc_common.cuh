@@ -135,6 +135,43 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
                : "memory");
 }
 
+// 32 lanes x 32 consecutive 32-bit columns from registers: thread i of the warp writes lane
+// (base lane + i).  tmem_st_wait() makes the stores complete before a later fence / arrive.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+      "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+      "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: the A operand (M rows = TMEM lanes, 16-bit elements packed two
+// per 32-bit column, K-major) is read from tensor memory.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy reads (the
+// tensor cores, TMA) that are synchronised through an mbarrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major bf16 tile stored as rows of 128 bytes with the
 // 128-byte swizzle (8-row atoms of 1024 bytes; the tile base is 1024-byte aligned).
 // Fields: start address >> 4 (bits 0-13), leading-dimension offset (unused for this layout, 1),
@@ -148,6 +185,25 @@ __device__ __forceinline__ uint64_t sdesc_sw128(const void *tile) {
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// Descriptor of an MN-major 16-bit operand with the 128-byte swizzle: rows of 128 bytes hold 64
+// consecutive MN elements, consecutive rows are consecutive K; 8-row atoms of 1024 bytes follow
+// each other along K (stride offset 1024), and the next 64 MN elements start `mn_block_bytes`
+// further on (leading offset).  The base is 1024-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(const void *tile, uint32_t mn_block_bytes) {
+  const uint32_t a = smem_u32(tile);
+  uint64_t d = (uint64_t)((a & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// kind::f16 with fp16 A and B, fp32 D, A K-major, B MN-major (bit 16), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) {
+  return (1u << 4) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, both K-major, shape M x N.
