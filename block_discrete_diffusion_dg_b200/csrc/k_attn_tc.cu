@@ -72,6 +72,12 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// 2^x by the hardware approximation (PTX ex2.approx.ftz: relative error ~2^-22, -inf -> +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   const __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
@@ -352,25 +358,29 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
 //   S_i = Q K_i^T   (M 128 rows, N 128 keys, K 128 = head_dim; bf16 operands from shared memory)
 //   O  += P_i V_i   (M 128 rows, N 128 = head_dim, K 128 keys; P fp16 from tensor memory, V fp16
 //                    in shared memory, read MN-major)
-// Warp roles (256 threads):
+// Warp roles (384 threads):
 //   warp 0     TMA: the Q tile once, then K and V tiles of 128 keys into 3-stage rings;
 //   warp 1     owns the 512 TMEM columns (S0, S1, O, P0, P1) and issues the MMAs:
 //              S_0, S_1, then per tile PV_i followed by S_(i+2) into the S buffer just released;
 //   warps 2-3  convert each landed V tile from bf16 to fp16 in place and zero the rows past the
 //              last valid key (so masked keys contribute exactly 0 * 0);
-//   warps 4-7  softmax, one query row per thread (= TMEM lane): read S_i, mask, running max in the
-//              log2 domain, P_i = 2^(t - m) written back to TMEM as fp16 pairs, row sum in fp32.
+//   warps 4-11 softmax, two warps per query row block of 32 (one TMEM lane quarter), each on half
+//              of the columns: read S_i, mask, running max in the log2 domain (the pair exchanges
+//              partial maxima), P_i = 2^(t - m) written back to TMEM as fp16 pairs, row sums fp32.
 // The running maximum is applied lazily: O is rescaled (read, scaled, written back in TMEM) only
 // when a row's maximum grows by more than 2^8, so between rescales P can reach 256 (exact in
 // fp16's range; the final O / l is unchanged because O and l always share the same base).
 // Every wait is bounded; on expiry the kernel records DG_ERR_TIMEOUT, lets issued copies and
 // MMAs finish, frees TMEM and returns.
-constexpr int T5_HD = 128, T5_KT = 128, T5_KS = 3, T5_VS = 3, T5_THR = 256;
+constexpr int T5_HD = 128, T5_KT = 128, T5_KS = 3, T5_VS = 2, T5_THR = 384;
 constexpr int T5_HALF = 128 * 128;       // one box: 128 rows x 64 bf16 (128-byte rows) = 16 KB
 constexpr int T5_TILE = 2 * T5_HALF;     // 128 rows x 128 head dims = 32 KB
 constexpr uint32_t T5_COL_S = 0, T5_COL_O = 256, T5_COL_P = 384, T5_TMEM_COLS = 512;
 constexpr float T5_RESCALE = 8.f;        // log2 of the largest P between rescales
-constexpr size_t T5_SMEM = 1024 + (size_t)T5_TILE * (1 + T5_KS + T5_VS) + 256;
+// exchange area of the softmax warp pairs: partial maxima [2 tiles][2 halves][128 rows], warp
+// flags [2][2][4], partial row sums [2][128]
+constexpr int T5_XCH = 2 * 2 * 128 * 4 + 2 * 2 * 4 * 4 + 2 * 128 * 4;
+constexpr size_t T5_SMEM = 1024 + (size_t)T5_TILE * (1 + T5_KS + T5_VS) + 512 + T5_XCH;
 constexpr unsigned FULL = 0xffffffffu;
 
 struct T5Args {
@@ -404,8 +414,13 @@ __global__ void __launch_bounds__(T5_THR, 1)
   uint64_t *v_full = k_empty + T5_KS, *v_ready = v_full + T5_VS, *v_empty = v_ready + T5_VS;
   uint64_t *s_full = v_empty + T5_VS, *p_full = s_full + 2, *pv_done = p_full + 2;
   uint64_t *mma_fin = pv_done + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_fin + 1);
+  uint64_t *xbar = mma_fin + 1;   // [4 lane quarters][2 tile parities]: softmax pair exchange
+  uint64_t *xfin = xbar + 8;      // [4]: final row-sum exchange
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xfin + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *x_max = reinterpret_cast<float *>(smem + T5_TILE * (1 + T5_KS + T5_VS) + 512);
+  int *x_good = reinterpret_cast<int *>(x_max + 2 * 2 * 128);
+  float *x_sum = reinterpret_cast<float *>(x_good + 2 * 2 * 4);
 
   const int split = blockIdx.z % a.splits, b = blockIdx.z / a.splits;
   if (a.done && a.done[b]) return;  // uniform across the block
@@ -432,10 +447,12 @@ __global__ void __launch_bounds__(T5_THR, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 4);
+      mbar_init(&p_full[x], 8);
       mbar_init(&pv_done[x], 1);
     }
     mbar_init(mma_fin, 1);
+    for (int x = 0; x < 8; ++x) mbar_init(&xbar[x], 64);
+    for (int x = 0; x < 4; ++x) mbar_init(&xfin[x], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -570,47 +587,66 @@ __global__ void __launch_bounds__(T5_THR, 1)
       if (lane == 0) mbar_arrive(&v_ready[vs]);
     }
   } else {
-    const int q4 = warp & 3;                 // TMEM lane quarter of this warp
+    // Softmax: 8 warps, two per TMEM lane quarter; warp (q4, half) owns rows q4*32 + lane and the
+    // columns [64 half, 64 half + 64) of S and O (P: [32 half, 32 half + 32)).  The two warps of a
+    // quarter combine their partial row maxima through shared memory once per tile (an mbarrier
+    // exchange, bounded like every other wait), so both apply the same running maximum; each
+    // keeps the row sum over its own columns and the two are added at the end.
+    // Control flow stays warp-uniform (votes on every exit and on the rescale decision): the TMEM
+    // loads and stores are .sync.aligned and need all 32 lanes.
+    const int q4 = warp & 3, half = (warp - 4) >> 2;
     const int r = q4 * 32 + lane;            // query row of the tile
     const int hl = r / qpc, pos = i0 + r % qpc, h = g * rep + hl;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
+    const uint32_t cS = T5_COL_S + half * 64, cO = T5_COL_O + half * 64, cP = T5_COL_P + half * 32;
     const float sl2 = 1.4426950408889634f / sqrtf((float)T5_HD);
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    // Control flow stays warp-uniform (votes on every exit and on the rescale decision): the TMEM
-    // loads and stores below are .sync.aligned and need all 32 lanes.
     for (int i = 0; i < N; ++i) {
-      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-      if (!__all_sync(FULL, mbar_wait(&s_full[i & 1], (i >> 1) & 1))) {
-        t5_fail(a.status, abort_flag);
-        ok = false;
-        break;
-      }
-      fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lrow + T5_COL_S + (uint32_t)(i & 1) * 128 + c * 32, sr[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+      const int par = i & 1;
+      bool good = !__any_sync(FULL, *abort_flag != 0);
+      if (good) good = __all_sync(FULL, mbar_wait(&s_full[par], (i >> 1) & 1));
+      uint32_t sr[2][32];
+      float mx = -INFINITY;
       bool cache;
       int row, j0, valid;
       tile_src(i, cache, row, j0, valid);
-      int lim = valid;
-      if (a.causal && !cache) lim = min(lim, pos - j0 + 1);
-      float mx = -INFINITY;
+      if (good) {
+        fence_after();
+        tmem_ld32(tmem + lrow + cS + (uint32_t)par * 128, sr[0]);
+        tmem_ld32(tmem + lrow + cS + (uint32_t)par * 128 + 32, sr[1]);
+        tmem_ld_wait(sr[0]);
+        tmem_ld_wait(sr[1]);
+        int lim = valid - half * 64;
+        if (a.causal && !cache) lim = min(lim, pos - j0 + 1 - half * 64);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float t = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) * sl2 : -INFINITY;
-          sr[c][j] = __float_as_uint(t);
-          mx = fmaxf(mx, t);
-        }
-      const float m_new = fmaxf(m_use, mx);
-      // a row whose maximum grew by more than 2^8 needs O rescaled; the whole warp then rescales
-      // (factor 1 where nothing changed; a row with nothing accumulated yet only takes m_new)
+          for (int j = 0; j < 32; ++j) {
+            const float v = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
+            sr[c][j] = __float_as_uint(v);
+            m4[j & 3] = fmaxf(m4[j & 3], v);
+          }
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      }
+      // exchange the partial maxima with the other warp of this quarter
+      x_max[(par * 2 + half) * 128 + r] = mx;
+      if (lane == 0) x_good[(par * 2 + half) * 4 + q4] = good ? 1 : 0;
+      mbar_arrive(&xbar[q4 * 2 + par]);
+      const bool xok = __all_sync(FULL, mbar_wait(&xbar[q4 * 2 + par], (i >> 1) & 1));
+      const bool pgood = x_good[(par * 2 + (half ^ 1)) * 4 + q4] != 0;
+      if (!(good && xok && pgood)) {
+        if (!(good && xok)) t5_fail(a.status, abort_flag);
+        ok = false;
+        break;
+      }
+      const float mt = fmaxf(mx, x_max[(par * 2 + (half ^ 1)) * 128 + r]) * sl2;
+      const float m_new = fmaxf(m_use, mt);
+      // a row whose maximum grew by more than 2^8 needs O rescaled; the whole warp (and its
+      // partner, which sees the same values) then rescales, factor 1 where nothing changed
       if (__any_sync(FULL, m_use != -INFINITY && m_new > m_use + T5_RESCALE)) {
-        const float f = m_use == -INFINITY ? 1.f : exp2f(m_use - m_new);
+        const float f = m_use == -INFINITY ? 1.f : ex2_approx(m_use - m_new);
         if (i >= 1 && !__all_sync(FULL, mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) {
           t5_fail(a.status, abort_flag);
           ok = false;
@@ -618,13 +654,13 @@ __global__ void __launch_bounds__(T5_THR, 1)
         }
         fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lrow + T5_COL_O + c * 32, o);
+          tmem_ld32(tmem + lrow + cO + c * 32, o);
           tmem_ld_wait(o);
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-          tmem_st32(tmem + lrow + T5_COL_O + c * 32, o);
+          tmem_st32(tmem + lrow + cO + c * 32, o);
         }
         tmem_st_wait();
         l *= f;
@@ -632,32 +668,31 @@ __global__ void __launch_bounds__(T5_THR, 1)
       } else if (m_use == -INFINITY) {
         m_use = m_new;  // nothing accumulated yet (O is exactly 0 or not yet written)
       }
-      const float base = m_use == -INFINITY ? 0.f : m_use;
-      uint32_t pk[2][32];
-      float ps = 0.f;
+      const float nb = m_use == -INFINITY ? 0.f : -m_use;
+      uint32_t pk[32];
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float p0 = exp2f(__uint_as_float(sr[c][j]) - base);
-          const float p1 = exp2f(__uint_as_float(sr[c][j + 1]) - base);
-          ps += p0 + p1;
-          pk[c >> 1][(c & 1) * 16 + j / 2] = pack_f16(p0, p1);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), sl2, nb));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), sl2, nb));
+          s4[(j >> 1) & 3] += p0 + p1;
+          pk[c * 16 + j / 2] = pack_f16(p0, p1);
         }
-      l += ps;
+      l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
       // P buffer (i & 1) was last read by PV_(i-2)
-      if (i >= 2 && !__all_sync(FULL, mbar_wait(&pv_done[i & 1], ((i - 2) >> 1) & 1))) {
+      if (i >= 2 && !__all_sync(FULL, mbar_wait(&pv_done[par], ((i - 2) >> 1) & 1))) {
         t5_fail(a.status, abort_flag);
         ok = false;
         break;
       }
       fence_after();
-      tmem_st32(tmem + lrow + T5_COL_P + (uint32_t)(i & 1) * 64, pk[0]);
-      tmem_st32(tmem + lrow + T5_COL_P + (uint32_t)(i & 1) * 64 + 32, pk[1]);
+      tmem_st32(tmem + lrow + cP + (uint32_t)par * 64, pk);
       tmem_st_wait();
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[i & 1]);
+      if (lane == 0) mbar_arrive(&p_full[par]);
     }
     if (ok && N > 0) {
       if (!__all_sync(FULL, mbar_wait(&pv_done[(N - 1) & 1], ((N - 1) >> 1) & 1))) {
@@ -666,15 +701,23 @@ __global__ void __launch_bounds__(T5_THR, 1)
       }
       fence_after();
     }
+    // the row sum over both halves
+    x_sum[half * 128 + r] = l;
+    mbar_arrive(&xfin[q4]);
+    if (!__all_sync(FULL, mbar_wait(&xfin[q4], 0))) {
+      if (ok) t5_fail(a.status, abort_flag);
+      ok = false;
+    }
+    const float lt = l + x_sum[(half ^ 1) * 128 + r];
     const bool row_ok = pos < a.n;  // guards the stores only; every lane reads TMEM
     if (ok) {
       if (a.splits == 1) {
-        const float il = l > 0.f ? 1.f / l : 0.f;
-        bf16 *dst = a.out + (((size_t)b * a.n + min(pos, a.n - 1)) * a.Hq + h) * T5_HD;
+        const float il = lt > 0.f ? 1.f / lt : 0.f;
+        bf16 *dst = a.out + (((size_t)b * a.n + min(pos, a.n - 1)) * a.Hq + h) * T5_HD + half * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lrow + T5_COL_O + c * 32, o);
+          tmem_ld32(tmem + lrow + cO + c * 32, o);
           tmem_ld_wait(o);
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
@@ -692,12 +735,12 @@ __global__ void __launch_bounds__(T5_THR, 1)
       } else {
         const int B = gridDim.z / a.splits;
         const size_t pr = (((size_t)split * B + b) * a.Hq + h) * a.n + min(pos, a.n - 1);
-        float *dst = a.part_o + pr * T5_HD;
+        float *dst = a.part_o + pr * T5_HD + half * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
           if (N > 0) {
-            tmem_ld32(tmem + lrow + T5_COL_O + c * 32, o);
+            tmem_ld32(tmem + lrow + cO + c * 32, o);
             tmem_ld_wait(o);
           } else {
 #pragma unroll
@@ -710,7 +753,7 @@ __global__ void __launch_bounds__(T5_THR, 1)
                   make_uint4(o[j], o[j + 1], o[j + 2], o[j + 3]);
           }
         }
-        if (row_ok) a.part_ml[pr] = make_float2(m_use, l);
+        if (row_ok && half == 0) a.part_ml[pr] = make_float2(m_use, lt);
       }
     }
   }
