@@ -1,21 +1,24 @@
-// Canvas attention on tensor cores (bf16 mma.sync m16n8k16, fp32 accumulation) with split-KV.
+// Canvas attention on tensor cores with split-KV: a tcgen05 kernel for head_dim 128 (below) and an
+// mma.sync m16n8k16 kernel for head_dim 64.
 // "DiffusionGemma Technical Report", Figure 4: the decoder attends bidirectionally across the
 // canvas and to the cached context (cross-attention to the KV cache); the causal encoder of the
 // append attends causally within the new tokens.  Model card "diffusiongemma", Model Overview.
 //
-// One CTA = 128 query rows that share one kv head: the rep = Hq / Hkv query heads of that kv head
+// A tile of 128 query rows shares one kv head: the rep = Hq / Hkv query heads of that kv head
 // times 128 / rep consecutive canvas positions, so every K/V tile is read once per GQA group.
 // Keys are split into chunks (split-KV) so that short and 131k-key contexts both fill the GPU;
 // each split leaves an unnormalised partial (O, running max m, sum l) that lm-style merging
 // combines exactly:  m = max m_s, l = sum l_s 2^(m_s - m), O = sum O_s 2^(m_s - m) / l.
 // Scores are kept in the log2 domain: t = q.k / sqrt(hd) * log2(e).
-// 8 warps x 16 rows; K/V tiles of 64 keys double-buffered with cp.async (zero-filled past the end)
-// in XOR-swizzled shared memory read by ldmatrix.
-// Precision: S = Q K^T takes the stored bf16 q and k exactly.  The second product takes P and V
-// in fp16: P in [0, 1] keeps 11 significant bits instead of bf16's 8 (the rounding of P is the
-// one rounding of this kernel the stored tensors do not have), and every bf16 value of V is
-// exact in fp16 for |v| < 65504 (below fp16's normal range the absolute error stays < 3e-8).
-// Each thread converts the V chunks it loaded, in place, once they have landed.
+// Precision: S = Q K^T takes the stored bf16 q and k exactly (fp32 accumulation).  The second
+// product takes V in fp16 (every bf16 value of V is exact in fp16 for |v| < 65504; below fp16's
+// normal range the absolute error stays < 3e-8) and P:
+//   tcgen05 kernel: P = P_hi + P_lo, two fp16 parts (~22 significant bits), so P adds no
+//                   rounding visible at bf16 storage of the output;
+//   mma.sync kernel: P in fp16 (11 significant bits).
+// The mma.sync kernel: 8 warps x 16 rows; K/V tiles of 64 keys double-buffered with cp.async
+// (zero-filled past the end) in XOR-swizzled shared memory read by ldmatrix; each thread converts
+// the V chunks it loaded, in place, once they have landed.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 #include "tc_common.cuh"
@@ -353,34 +356,38 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
 }
 
 // ================================================================================================
-// tcgen05 path (head_dim 128).  One CTA = the same 128 query rows as above x one key split, with
-// both products on the 5th-generation tensor cores and the accumulators in tensor memory:
-//   S_i = Q K_i^T   (M 128 rows, N 128 keys, K 128 = head_dim; bf16 operands from shared memory)
-//   O  += P_i V_i   (M 128 rows, N 128 = head_dim, K 128 keys; P fp16 from tensor memory, V fp16
-//                    in shared memory, read MN-major)
+// tcgen05 path (head_dim 128).  One CTA = two tiles of 128 query rows (A and B: the rep query
+// heads of one kv head times 2 x 128/rep consecutive canvas positions) x one key split, with both
+// products on the 5th-generation tensor cores and the accumulators in tensor memory:
+//   S_X = Q_X K_i^T  (M 128 rows, N 128 keys, K 128 = head_dim; bf16 operands from shared memory)
+//   O_X += P_X V_i   (M 128 rows, N 128 = head_dim, K 128 keys, twice: P_hi and P_lo fp16 from
+//                     tensor memory, V fp16 in shared memory, read MN-major)
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).  P_X is written
+// over S_X as two fp16 parts, P = P_hi + P_lo (hi pairs in columns [0,64), lo pairs in [64,128)),
+// and O_X += P_hi V + P_lo V, so P reaches the product with ~22 significant bits; S_X of the next
+// key tile is issued only once P_X V of this one has completed.  The tensor cores run PV_A(i), S_A(i+1), PV_B(i), S_B(i+1):
+// while one softmax warpgroup works on its tile, the MMAs of the other proceed.
 // Warp roles (384 threads):
-//   warp 0     TMA: the Q tile once, then K and V tiles of 128 keys into 3-stage rings;
-//   warp 1     owns the 512 TMEM columns (S0, S1, O, P0, P1) and issues the MMAs:
-//              S_0, S_1, then per tile PV_i followed by S_(i+2) into the S buffer just released;
+//   warp 0     TMA: both Q tiles once, then K and V tiles of 128 keys (3- and 2-stage rings);
+//   warp 1     owns the TMEM columns and issues the MMAs;
 //   warps 2-3  convert each landed V tile from bf16 to fp16 in place and zero the rows past the
 //              last valid key (so masked keys contribute exactly 0 * 0);
-//   warps 4-11 softmax, two warps per query row block of 32 (one TMEM lane quarter), each on half
-//              of the columns: read S_i, mask, running max in the log2 domain (the pair exchanges
-//              partial maxima), P_i = 2^(t - m) written back to TMEM as fp16 pairs, row sums fp32.
+//   warps 4-7  softmax of tile A, warps 8-11 of tile B: one query row per thread (= TMEM lane);
+//              read S, mask, running max in the log2 domain, P = 2^(t - m) written back to TMEM
+//              as fp16 hi and lo pairs, row sum in fp32.
 // The running maximum is applied lazily: O is rescaled (read, scaled, written back in TMEM) only
 // when a row's maximum grows by more than 2^8, so between rescales P can reach 256 (exact in
 // fp16's range; the final O / l is unchanged because O and l always share the same base).
+// Control flow of the softmax warps is warp-uniform (votes on every exit and on the rescale
+// decision): TMEM loads and stores are .sync.aligned and need all 32 lanes.
 // Every wait is bounded; on expiry the kernel records DG_ERR_TIMEOUT, lets issued copies and
 // MMAs finish, frees TMEM and returns.
 constexpr int T5_HD = 128, T5_KT = 128, T5_KS = 3, T5_VS = 2, T5_THR = 384;
 constexpr int T5_HALF = 128 * 128;       // one box: 128 rows x 64 bf16 (128-byte rows) = 16 KB
 constexpr int T5_TILE = 2 * T5_HALF;     // 128 rows x 128 head dims = 32 KB
-constexpr uint32_t T5_COL_S = 0, T5_COL_O = 256, T5_COL_P = 384, T5_TMEM_COLS = 512;
+constexpr uint32_t T5_COL_S = 0, T5_COL_O = 256, T5_TMEM_COLS = 512;
 constexpr float T5_RESCALE = 8.f;        // log2 of the largest P between rescales
-// exchange area of the softmax warp pairs: partial maxima [2 tiles][2 halves][128 rows], warp
-// flags [2][2][4], partial row sums [2][128]
-constexpr int T5_XCH = 2 * 2 * 128 * 4 + 2 * 2 * 4 * 4 + 2 * 128 * 4;
-constexpr size_t T5_SMEM = 1024 + (size_t)T5_TILE * (1 + T5_KS + T5_VS) + 512 + T5_XCH;
+constexpr size_t T5_SMEM = 1024 + (size_t)T5_TILE * (2 + T5_KS + T5_VS) + 512;
 constexpr unsigned FULL = 0xffffffffu;
 
 struct T5Args {
@@ -406,29 +413,24 @@ __global__ void __launch_bounds__(T5_THR, 1)
   using namespace tc;
   extern __shared__ uint8_t t5_smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)t5_smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sQ = smem;
-  uint8_t *sK = sQ + T5_TILE;
+  uint8_t *sQ = smem;                       // [2 tiles][TILE]
+  uint8_t *sK = sQ + 2 * T5_TILE;
   uint8_t *sV = sK + T5_KS * T5_TILE;
   uint64_t *q_full = reinterpret_cast<uint64_t *>(sV + T5_VS * T5_TILE);
   uint64_t *k_full = q_full + 1, *k_empty = k_full + T5_KS;
   uint64_t *v_full = k_empty + T5_KS, *v_ready = v_full + T5_VS, *v_empty = v_ready + T5_VS;
-  uint64_t *s_full = v_empty + T5_VS, *p_full = s_full + 2, *pv_done = p_full + 2;
+  uint64_t *s_full = v_empty + T5_VS, *p_full = s_full + 2, *pv_done = p_full + 2;  // [tile]
   uint64_t *mma_fin = pv_done + 2;
-  uint64_t *xbar = mma_fin + 1;   // [4 lane quarters][2 tile parities]: softmax pair exchange
-  uint64_t *xfin = xbar + 8;      // [4]: final row-sum exchange
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xfin + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_fin + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  float *x_max = reinterpret_cast<float *>(smem + T5_TILE * (1 + T5_KS + T5_VS) + 512);
-  int *x_good = reinterpret_cast<int *>(x_max + 2 * 2 * 128);
-  float *x_sum = reinterpret_cast<float *>(x_good + 2 * 2 * 4);
 
   const int split = blockIdx.z % a.splits, b = blockIdx.z / a.splits;
   if (a.done && a.done[b]) return;  // uniform across the block
-  const int g = blockIdx.y, rep = a.Hq / a.Hkv, qpc = ROWS / rep, i0 = blockIdx.x * qpc;
+  const int g = blockIdx.y, rep = a.Hq / a.Hkv, qpc = ROWS / rep, i0 = blockIdx.x * 2 * qpc;
   const int len = min(max(a.cache_len[b], 0), a.cap);
   const int tcache = (len + T5_KT - 1) / T5_KT;
   int tiles = tcache + (a.n + T5_KT - 1) / T5_KT;
-  if (a.causal) tiles = tcache + (min(a.n, i0 + qpc) - 1) / T5_KT + 1;  // later canvas keys unseen
+  if (a.causal) tiles = tcache + (min(a.n, i0 + 2 * qpc) - 1) / T5_KT + 1;  // later keys unseen
   const int t_begin = split * a.chunk_tiles;
   const int N = max(0, min(tiles, t_begin + a.chunk_tiles) - t_begin);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -447,12 +449,10 @@ __global__ void __launch_bounds__(T5_THR, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 8);
+      mbar_init(&p_full[x], 4);
       mbar_init(&pv_done[x], 1);
     }
     mbar_init(mma_fin, 1);
-    for (int x = 0; x < 8; ++x) mbar_init(&xbar[x], 64);
-    for (int x = 0; x < 4; ++x) mbar_init(&xfin[x], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(T5_THR, 1)
   fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // tile i of this split: cache rows [j0, j0 + 128) or canvas rows; `valid` keys in it
+  // key tile i of this split: cache rows [j0, j0 + 128) or canvas rows; `valid` keys in it
   auto tile_src = [&](int i, bool &cache, int &row, int &j0, int &valid) {
     const int t = t_begin + i;
     cache = t < tcache;
@@ -485,11 +485,12 @@ __global__ void __launch_bounds__(T5_THR, 1)
     if (lane == 0) {
       uint32_t armed_k = 0, armed_v = 0;  // tiles whose copies were issued
       bool ok = true;
-      mbar_expect_tx(q_full, T5_TILE);
-      for (int hl = 0; hl < rep; ++hl)
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_2d(sQ + hf * T5_HALF + hl * qpc * 128, &tmQ, q_full,
-                      (g * rep + hl) * T5_HD + hf * 64, b * a.n + i0);
+      mbar_expect_tx(q_full, 2 * T5_TILE);
+      for (int x = 0; x < 2; ++x)
+        for (int hl = 0; hl < rep; ++hl)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(sQ + x * T5_TILE + hf * T5_HALF + hl * qpc * 128, &tmQ, q_full,
+                        (g * rep + hl) * T5_HD + hf * 64, b * a.n + i0 + x * qpc);
       for (int i = 0; i < N && ok && !*abort_flag; ++i) {
         bool cache;
         int row, j0, valid;
@@ -522,41 +523,68 @@ __global__ void __launch_bounds__(T5_THR, 1)
       const uint32_t id_p = idesc_f16_bmn(ROWS, T5_HD);
       bool ok = mbar_wait(q_full, 0);
       fence_after();
-      auto issue_s = [&](int i) -> bool {
+      auto issue_s = [&](int x, int i) {   // S_x(i) = Q_x K_i^T into S_x
         const int ks = i % T5_KS;
-        if (!mbar_wait(&k_full[ks], (i / T5_KS) & 1)) return false;
-        fence_after();
-        const uint32_t d = tmem + T5_COL_S + (uint32_t)(i & 1) * 128;
+        const uint32_t d = tmem + T5_COL_S + (uint32_t)x * 128;
 #pragma unroll
         for (int kk = 0; kk < T5_HD / 16; ++kk) {
           const int hf = kk >> 2, k4 = kk & 3;
-          const uint64_t ad = sdesc_sw128(sQ + hf * T5_HALF) + 2 * k4;
+          const uint64_t ad = sdesc_sw128(sQ + x * T5_TILE + hf * T5_HALF) + 2 * k4;
           const uint64_t bd = sdesc_sw128(sK + ks * T5_TILE + hf * T5_HALF) + 2 * k4;
           mma_bf16(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
         }
-        commit(&k_empty[ks]);
-        commit(&s_full[i & 1]);
-        return true;
+        commit(&s_full[x]);
       };
-      if (ok && N > 0) ok = issue_s(0);
-      if (ok && N > 1) ok = issue_s(1);
+      auto issue_pv = [&](int x, int i) {  // O_x += P_x V_i
+        const int vs = i % T5_VS;
+        const uint32_t pa = tmem + T5_COL_S + (uint32_t)x * 128;
+        const uint32_t d = tmem + T5_COL_O + (uint32_t)x * 128;
+#pragma unroll
+        for (int kk = 0; kk < T5_KT / 16; ++kk) {  // P = P_hi + P_lo, both against the same V
+          const uint64_t bd = sdesc_sw128_mn(sV + vs * T5_TILE + kk * 16 * 128, T5_HALF);
+          mma_f16_ts(d, pa + kk * 8, bd, id_p, (i | kk) != 0 ? 1u : 0u);
+          mma_f16_ts(d, pa + 64 + kk * 8, bd, id_p, 1u);
+        }
+        commit(&pv_done[x]);
+      };
+      if (ok && N > 0) {
+        ok = mbar_wait(&k_full[0], 0);
+        if (ok) {
+          fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          commit(&k_empty[0]);
+        }
+      }
       for (int i = 0; ok && i < N && !*abort_flag; ++i) {
         const int vs = i % T5_VS;
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1) ||
-            !mbar_wait(&v_ready[vs], (i / T5_VS) & 1)) {
+        const uint32_t ph = i & 1;
+        if (!mbar_wait(&v_ready[vs], (i / T5_VS) & 1) || !mbar_wait(&p_full[0], ph)) {
           ok = false;
           break;
         }
         fence_after();
-        const uint32_t pa = tmem + T5_COL_P + (uint32_t)(i & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < T5_KT / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128_mn(sV + vs * T5_TILE + kk * 16 * 128, T5_HALF);
-          mma_f16_ts(tmem + T5_COL_O, pa + kk * 8, bd, id_p, (i | kk) != 0 ? 1u : 0u);
+        issue_pv(0, i);
+        const bool more = i + 1 < N;
+        if (more) {  // S_A(i+1) overwrites P_A(i): wait for PV_A(i) to complete
+          if (!mbar_wait(&k_full[(i + 1) % T5_KS], ((i + 1) / T5_KS) & 1) ||
+              !mbar_wait(&pv_done[0], ph)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          issue_s(0, i + 1);
         }
+        if (!mbar_wait(&p_full[1], ph)) { ok = false; break; }
+        fence_after();
+        issue_pv(1, i);
         commit(&v_empty[vs]);
-        commit(&pv_done[i & 1]);
-        if (i + 2 < N) ok = issue_s(i + 2);
+        if (more) {
+          if (!mbar_wait(&pv_done[1], ph)) { ok = false; break; }
+          fence_after();
+          issue_s(1, i + 1);
+          commit(&k_empty[(i + 1) % T5_KS]);
+        }
       }
       if (!ok) t5_fail(a.status, abort_flag);
       commit(mma_fin);  // every MMA issued above has completed when this phase does
@@ -577,6 +605,7 @@ __global__ void __launch_bounds__(T5_THR, 1)
       uint8_t *base = sV + vs * T5_TILE;
       // 16-byte chunk c sits in key row (c mod 1024) / 8 of its half (the swizzle only permutes
       // chunks within a row), so the conversion is in place and per chunk
+#pragma unroll 4
       for (int c = ct; c < T5_TILE / 16; c += 64) {
         uint4 *pc = reinterpret_cast<uint4 *>(base + c * 16);
         if (((c & 1023) >> 3) < valid) bf16x8_to_f16x8(pc);
@@ -587,74 +616,76 @@ __global__ void __launch_bounds__(T5_THR, 1)
       if (lane == 0) mbar_arrive(&v_ready[vs]);
     }
   } else {
-    // Softmax: 8 warps, two per TMEM lane quarter; warp (q4, half) owns rows q4*32 + lane and the
-    // columns [64 half, 64 half + 64) of S and O (P: [32 half, 32 half + 32)).  The two warps of a
-    // quarter combine their partial row maxima through shared memory once per tile (an mbarrier
-    // exchange, bounded like every other wait), so both apply the same running maximum; each
-    // keeps the row sum over its own columns and the two are added at the end.
-    // Control flow stays warp-uniform (votes on every exit and on the rescale decision): the TMEM
-    // loads and stores are .sync.aligned and need all 32 lanes.
-    const int q4 = warp & 3, half = (warp - 4) >> 2;
-    const int r = q4 * 32 + lane;            // query row of the tile
-    const int hl = r / qpc, pos = i0 + r % qpc, h = g * rep + hl;
+    const int x = (warp - 4) >> 2;          // query tile (A or B) of this warpgroup
+    const int q4 = warp & 3;                // TMEM lane quarter of this warp
+    const int r = q4 * 32 + lane;           // query row of the tile
+    const int hl = r / qpc, pos = i0 + x * qpc + r % qpc, h = g * rep + hl;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
-    const uint32_t cS = T5_COL_S + half * 64, cO = T5_COL_O + half * 64, cP = T5_COL_P + half * 32;
+    const uint32_t cS = T5_COL_S + (uint32_t)x * 128, cO = T5_COL_O + (uint32_t)x * 128;
     const float sl2 = 1.4426950408889634f / sqrtf((float)T5_HD);
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < N; ++i) {
-      const int par = i & 1;
-      bool good = !__any_sync(FULL, *abort_flag != 0);
-      if (good) good = __all_sync(FULL, mbar_wait(&s_full[par], (i >> 1) & 1));
-      uint32_t sr[2][32];
-      float mx = -INFINITY;
-      bool cache;
-      int row, j0, valid;
-      tile_src(i, cache, row, j0, valid);
-      if (good) {
-        fence_after();
-        tmem_ld32(tmem + lrow + cS + (uint32_t)par * 128, sr[0]);
-        tmem_ld32(tmem + lrow + cS + (uint32_t)par * 128 + 32, sr[1]);
-        tmem_ld_wait(sr[0]);
-        tmem_ld_wait(sr[1]);
-        int lim = valid - half * 64;
-        if (a.causal && !cache) lim = min(lim, pos - j0 + 1 - half * 64);
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float v = (c * 32 + j < lim) ? __uint_as_float(sr[c][j]) : -INFINITY;
-            sr[c][j] = __float_as_uint(v);
-            m4[j & 3] = fmaxf(m4[j & 3], v);
-          }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      }
-      // exchange the partial maxima with the other warp of this quarter
-      x_max[(par * 2 + half) * 128 + r] = mx;
-      if (lane == 0) x_good[(par * 2 + half) * 4 + q4] = good ? 1 : 0;
-      mbar_arrive(&xbar[q4 * 2 + par]);
-      const bool xok = __all_sync(FULL, mbar_wait(&xbar[q4 * 2 + par], (i >> 1) & 1));
-      const bool pgood = x_good[(par * 2 + (half ^ 1)) * 4 + q4] != 0;
-      if (!(good && xok && pgood)) {
-        if (!(good && xok)) t5_fail(a.status, abort_flag);
+      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+      if (!__all_sync(FULL, mbar_wait(&s_full[x], i & 1))) {
+        t5_fail(a.status, abort_flag);
         ok = false;
         break;
       }
-      const float mt = fmaxf(mx, x_max[(par * 2 + (half ^ 1)) * 128 + r]) * sl2;
+      fence_after();
+      bool cache;
+      int row, j0, valid;
+      tile_src(i, cache, row, j0, valid);
+      int lim = valid;
+      if (a.causal && !cache) lim = min(lim, pos - j0 + 1);
+      const bool partial = __any_sync(FULL, lim < T5_KT);   // a partial or causal tile: mask
+      auto mask = [&](uint32_t (&v)[32], int c) {
+        if (partial) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j >= lim) v[j] = __float_as_uint(-INFINITY);
+        }
+      };
+      float m8[8];
+      auto fold_max = [&](const uint32_t (&v)[32], bool first) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          m8[j & 7] = (first && j < 8) ? __uint_as_float(v[j]) : fmaxf(m8[j & 7], __uint_as_float(v[j]));
+      };
+      // S chunks (32 columns each) 1 and 3 for the maximum, then 0 and 2, kept in registers
+      uint32_t sa[32], sb[32];
+      tmem_ld32(tmem + lrow + cS + 32, sa);
+      tmem_ld32(tmem + lrow + cS + 96, sb);
+      tmem_ld_wait(sa);
+      tmem_ld_wait(sb);
+      mask(sa, 1);
+      mask(sb, 3);
+      fold_max(sa, true);
+      fold_max(sb, false);
+      tmem_ld32(tmem + lrow + cS + 0, sa);
+      tmem_ld32(tmem + lrow + cS + 64, sb);
+      tmem_ld_wait(sa);
+      tmem_ld_wait(sb);
+      mask(sa, 0);
+      mask(sb, 2);
+      fold_max(sa, false);
+      fold_max(sb, false);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
       const float m_new = fmaxf(m_use, mt);
-      // a row whose maximum grew by more than 2^8 needs O rescaled; the whole warp (and its
-      // partner, which sees the same values) then rescales, factor 1 where nothing changed
+      // a row whose maximum grew by more than 2^8 needs O rescaled; the whole warp then rescales
+      // (factor 1 where nothing changed; a row with nothing accumulated yet only takes m_new)
       if (__any_sync(FULL, m_use != -INFINITY && m_new > m_use + T5_RESCALE)) {
         const float f = m_use == -INFINITY ? 1.f : ex2_approx(m_use - m_new);
-        if (i >= 1 && !__all_sync(FULL, mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) {
+        // O must include PV(i-1) before scaling
+        if (i >= 1 && !__all_sync(FULL, mbar_wait(&pv_done[x], (i - 1) & 1))) {
           t5_fail(a.status, abort_flag);
           ok = false;
           break;
         }
         fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tmem + lrow + cO + c * 32, o);
           tmem_ld_wait(o);
@@ -669,53 +700,57 @@ __global__ void __launch_bounds__(T5_THR, 1)
         m_use = m_new;  // nothing accumulated yet (O is exactly 0 or not yet written)
       }
       const float nb = m_use == -INFINITY ? 0.f : -m_use;
-      uint32_t pk[32];
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
+      // P of the 32 keys of S chunk c, split into two fp16 parts (P = hi + lo to ~22 bits):
+      // hi pairs go to columns [16c, 16c + 16) of S, lo pairs to [64 + 16c, 64 + 16c + 16).
+      // Chunk c's columns are overwritten by the P of chunks 2c and 2c + 1 (hi) and of chunks
+      // 2c - 4 and 2c - 3 (lo), so the order below reads every chunk before it is covered.
+      auto emit = [&](const uint32_t (&v)[32], int c) {
+        uint32_t ph[16], pl[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), sl2, nb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), sl2, nb));
+          const float p0 = ex2_approx(fmaf(__uint_as_float(v[j]), sl2, nb));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), sl2, nb));
           s4[(j >> 1) & 3] += p0 + p1;
-          pk[c * 16 + j / 2] = pack_f16(p0, p1);
+          const __half2 hi = __floats2half2_rn(p0, p1);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __floats2half2_rn(p0 - hf.x, p1 - hf.y);
+          ph[j >> 1] = *reinterpret_cast<const uint32_t *>(&hi);
+          pl[j >> 1] = *reinterpret_cast<const uint32_t *>(&lo);
         }
+        tmem_st16(tmem + lrow + cS + c * 16, ph);
+        tmem_st16(tmem + lrow + cS + 64 + c * 16, pl);
+      };
+      emit(sa, 0);                            // writes over S chunks 0 (held) and 2 (held in sb)
+      tmem_ld32(tmem + lrow + cS + 32, sa);   // S chunk 1 again (untouched so far)
+      tmem_ld_wait(sa);
+      mask(sa, 1);
+      emit(sa, 1);                            // over S chunks 0 and 2 (both consumed or held)
+      tmem_ld32(tmem + lrow + cS + 96, sa);   // S chunk 3 again (untouched so far)
+      tmem_ld_wait(sa);
+      mask(sa, 3);
+      emit(sb, 2);                            // over S chunks 1 (consumed) and 3 (held in sa)
+      emit(sa, 3);
       l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      // P buffer (i & 1) was last read by PV_(i-2)
-      if (i >= 2 && !__all_sync(FULL, mbar_wait(&pv_done[par], ((i - 2) >> 1) & 1))) {
-        t5_fail(a.status, abort_flag);
-        ok = false;
-        break;
-      }
-      fence_after();
-      tmem_st32(tmem + lrow + cP + (uint32_t)par * 64, pk);
       tmem_st_wait();
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[par]);
+      if (lane == 0) mbar_arrive(&p_full[x]);
     }
     if (ok && N > 0) {
-      if (!__all_sync(FULL, mbar_wait(&pv_done[(N - 1) & 1], ((N - 1) >> 1) & 1))) {
+      if (!__all_sync(FULL, mbar_wait(&pv_done[x], (N - 1) & 1))) {
         t5_fail(a.status, abort_flag);
         ok = false;
       }
       fence_after();
     }
-    // the row sum over both halves
-    x_sum[half * 128 + r] = l;
-    mbar_arrive(&xfin[q4]);
-    if (!__all_sync(FULL, mbar_wait(&xfin[q4], 0))) {
-      if (ok) t5_fail(a.status, abort_flag);
-      ok = false;
-    }
-    const float lt = l + x_sum[(half ^ 1) * 128 + r];
     const bool row_ok = pos < a.n;  // guards the stores only; every lane reads TMEM
     if (ok) {
       if (a.splits == 1) {
-        const float il = lt > 0.f ? 1.f / lt : 0.f;
-        bf16 *dst = a.out + (((size_t)b * a.n + min(pos, a.n - 1)) * a.Hq + h) * T5_HD + half * 64;
+        const float il = l > 0.f ? 1.f / l : 0.f;
+        bf16 *dst = a.out + (((size_t)b * a.n + min(pos, a.n - 1)) * a.Hq + h) * T5_HD;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tmem + lrow + cO + c * 32, o);
           tmem_ld_wait(o);
@@ -735,9 +770,9 @@ __global__ void __launch_bounds__(T5_THR, 1)
       } else {
         const int B = gridDim.z / a.splits;
         const size_t pr = (((size_t)split * B + b) * a.Hq + h) * a.n + min(pos, a.n - 1);
-        float *dst = a.part_o + pr * T5_HD + half * 64;
+        float *dst = a.part_o + pr * T5_HD;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           if (N > 0) {
             tmem_ld32(tmem + lrow + cO + c * 32, o);
@@ -753,7 +788,7 @@ __global__ void __launch_bounds__(T5_THR, 1)
                   make_uint4(o[j], o[j + 1], o[j + 2], o[j + 3]);
           }
         }
-        if (row_ok && half == 0) a.part_ml[pr] = make_float2(m_use, lt);
+        if (row_ok) a.part_ml[pr] = make_float2(m_use, l);
       }
     }
   }
@@ -768,8 +803,8 @@ __global__ void __launch_bounds__(T5_THR, 1)
 // Split plan of the tcgen05 path: tiles of 128 keys; as many splits as fill one wave.
 void plan5(int batch, int n, int Hq, int Hkv, int cap, int *splits, int *chunk_tiles) {
   const int tiles = (cap + T5_KT - 1) / T5_KT + (n + T5_KT - 1) / T5_KT;
-  const int qpc = ROWS / (Hq / Hkv);
-  const int base = ((n + qpc - 1) / qpc) * Hkv * batch;
+  const int qpc2 = 2 * (ROWS / (Hq / Hkv));
+  const int base = ((n + qpc2 - 1) / qpc2) * Hkv * batch;
   int s = num_sms() / (base > 0 ? base : 1);
   if (s > tiles) s = tiles;
   if (s > MAX_SPLITS) s = MAX_SPLITS;
@@ -858,7 +893,7 @@ int launch_tc5(int batch, int n, int Hq, int Hkv, const void *q, const void *k_c
     tvc = tvn;
   }
   if (rc != DG_OK) return rc;
-  dim3 grid((n + qpc - 1) / qpc, Hkv, batch * a.splits);
+  dim3 grid((n + 2 * qpc - 1) / (2 * qpc), Hkv, batch * a.splits);
   note_launch(s, "attn_tc");
   cudaFuncSetAttribute(attn_tc5_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T5_SMEM);
   attn_tc5_kernel<<<grid, T5_THR, T5_SMEM, s>>>(tq, tkc, tvc, tkn, tvn, a);
