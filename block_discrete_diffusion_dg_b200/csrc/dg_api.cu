@@ -61,7 +61,7 @@ inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
   B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_WDQ, B_LIVE, B_ROWS, B_NROWS, B_SLOT, B_FIN, B_LOGITS, B_PART,
-  B_ENT, B_AM, B_ATTN, B_COUNT
+  B_ENT, B_AM, B_ATTN, B_HP, B_COUNT
 };
 
 struct Layout {
@@ -69,6 +69,23 @@ struct Layout {
   size_t total;
   int max_tiles;
 };
+
+// K slices of the split-K projections for T tokens (1: the projection runs unsplit).
+int router_type(const dg_config *c);
+int qkv_parts(const dg_config &c, int T) {
+  const int N = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim, K = c.d_model;
+  return split_supported(c.act_dtype, c.w_dtype, T, N, K) ? split_k_slices(N, K) : 1;
+}
+int o_parts(const dg_config &c, int T) {
+  const int N = c.d_model, K = c.n_q_heads * c.head_dim;
+  return split_supported(c.act_dtype, c.w_dtype, T, N, K) ? split_k_slices(N, K) : 1;
+}
+int router_parts(const dg_config &c, int T) {
+  // few channel tiles: cap the slices, or the partials outweigh the router's weights
+  return split_supported(c.act_dtype, router_type(&c), T, c.n_experts, c.d_model)
+             ? split_k_slices(c.n_experts, c.d_model, 8)
+             : 1;
+}
 
 Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   const size_t T = (size_t)batch * n, a = esz(c.act_dtype);
@@ -81,7 +98,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   const size_t T128 = (T + 127) / 128 * 128;  // tensor-core A operands read whole 128-row tiles
   sz[B_X] = T * d * 4;  // residual stream: fp32
   sz[B_A] = T128 * d * a;
-  sz[B_QKV] = T * qkvw * 4;
+  sz[B_QKV] = T * qkvw * 4 * qkv_parts(c, (int)T);
   sz[B_CS] = T * hd * 4;
   sz[B_Q] = T * c.n_q_heads * hd * a;
   sz[B_KN] = T * c.n_kv_heads * hd * a;
@@ -89,7 +106,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_O] = T128 * c.n_q_heads * hd * a;
   sz[B_H] = T * d * 4;
   sz[B_Y] = T128 * d * a;
-  sz[B_Z] = T * (size_t)c.n_experts * 4;
+  sz[B_Z] = T * (size_t)c.n_experts * 4 * router_parts(c, (int)T);
   sz[B_IDX] = TK * 4;
   sz[B_W] = TK * 4;
   sz[B_OFF] = (size_t)(c.n_experts + 1) * 4;
@@ -117,6 +134,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_PART] = tc_lm ? lmhead_tc_ws_bytes((int)T, c.vocab) : 0;
   sz[B_ENT] = T * 4;
   sz[B_AM] = T * 4;
+  { const int op = o_parts(c, (int)T); sz[B_HP] = op > 1 ? T * d * 4 * op : 0; }
   sz[B_ATTN] = attention_ws_bytes(c.act_dtype, batch, n, c.n_q_heads, c.n_kv_heads, c.head_dim,
                                   cap);
   size_t o = 0;
@@ -194,6 +212,10 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
     int rc;
     const void *wq = tc_weight(c, ws, w.w_qkv, (size_t)g.N * c.d_model, 0, s, &rc);
     if (rc != DG_OK) return rc;
+    const int parts = qkv_parts(c, T);
+    if (parts > 1)
+      return launch_gemm_tc_split(wq, g.N, ws.at<void>(B_A), T, (T + 127) / 128 * 128, c.d_model,
+                                  parts, ws.at<float>(B_QKV), "gemm_qkv_tc", nullptr, s, g.bscale);
     return launch_gemm_tc_dense(ws.at<void>(B_A), T, wq, g.N, c.d_model, ws.at<float>(B_QKV),
                                 nullptr, g.N, "gemm_qkv_tc", nullptr, s, g.bscale);
   }
@@ -221,26 +243,44 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
   g.bscale = scale_or_null(&c, w.s_o);
   g.M = T; g.N = d; g.K = hq;
   g.name = "gemm_o_resid";
-  if (gemm_tc_supported(c.act_dtype, c.w_dtype, hq)) {
+  const int T128 = (T + 127) / 128 * 128;
+  const int op = o_parts(c, T);
+  if (op > 1) {  // split-K partials; the residual add happens in resid_norm
     int rc;
     const void *wo = tc_weight(c, ws, w.w_o, (size_t)d * hq, 0, s, &rc);
     if (rc != DG_OK) return rc;
-    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, wo, d, hq, ws.at<float>(B_H),
-                                ws.at<float>(B_X), d, "gemm_o_resid_tc", nullptr, s, g.bscale));
-  } else
-    DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
-  DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
-                        ws.at<void>(B_Y), s));
+    DG_TRY(launch_gemm_tc_split(wo, d, ws.at<void>(B_O), T, T128, hq, op, ws.at<float>(B_HP),
+                                "gemm_o_resid_tc", nullptr, s, g.bscale));
+    DG_TRY(launch_resid_norm(c.act_dtype, ws.at<float>(B_HP), op, ws.at<float>(B_X), T, d,
+                             c.rms_eps, ws.at<float>(B_H), ws.at<void>(B_Y), s));
+  } else {
+    if (gemm_tc_supported(c.act_dtype, c.w_dtype, hq)) {
+      int rc;
+      const void *wo = tc_weight(c, ws, w.w_o, (size_t)d * hq, 0, s, &rc);
+      if (rc != DG_OK) return rc;
+      DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, wo, d, hq, ws.at<float>(B_H),
+                                  ws.at<float>(B_X), d, "gemm_o_resid_tc", nullptr, s, g.bscale));
+    } else
+      DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
+    DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
+                          ws.at<void>(B_Y), s));
+  }
   *tiles_ready = false;
   if (router_tc(c)) {
-    DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_Y), T, w.w_router, c.n_experts, d, ws.at<float>(B_Z),
-                                nullptr, c.n_experts, "router_logits_tc", nullptr, s));
+    const int rp = router_parts(c, T);
+    if (rp > 1)
+      DG_TRY(launch_gemm_tc_split(w.w_router, c.n_experts, ws.at<void>(B_Y), T, T128, d, rp,
+                                  ws.at<float>(B_Z), "router_logits_tc", nullptr, s, nullptr));
+    else
+      DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_Y), T, w.w_router, c.n_experts, d,
+                                  ws.at<float>(B_Z), nullptr, c.n_experts, "router_logits_tc",
+                                  nullptr, s));
     const bool tc = experts_tc(c);
     DG_TRY(launch_route(T, c.n_experts, c.top_k, ws.at<float>(B_Z), token_live,
                         ws.at<int32_t>(B_IDX), ws.at<float>(B_W), ws.at<int32_t>(B_OFF),
                         ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV),
                         tc ? experts_tc_tile_tokens() : SIMT_TILE_M, ws.at<GroupTile>(B_TILES),
-                        ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s, forced));
+                        ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s, forced, rp));
     *tiles_ready = true;
     return DG_OK;
   }
@@ -550,7 +590,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
     char *vc = (char *)v_cache + l * layer_elems * ae;
     DG_TRY(qkv_proj(c, lw, w, T, s));
     DG_TRY(launch_qkv_split(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
-                            w.at<float>(B_QKV), w.at<float>(B_CS), w.at<void>(B_Q),
+                            w.at<float>(B_QKV), qkv_parts(c, T), w.at<float>(B_CS), w.at<void>(B_Q),
                             w.at<void>(B_KN), w.at<void>(B_VN), kc, vc, cache_len, cache_cap,
                             dev_status, s));
     if (l + 1 == c.n_layers) break;
@@ -606,7 +646,7 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
     const char *vc = (const char *)v_cache + l * layer_elems * ae;
     DG_TRY(qkv_proj(c, lw, w, T, s));
     DG_TRY(launch_qkv_split(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,
-                            w.at<float>(B_QKV), w.at<float>(B_CS), w.at<void>(B_Q),
+                            w.at<float>(B_QKV), qkv_parts(c, T), w.at<float>(B_CS), w.at<void>(B_Q),
                             w.at<void>(B_KN), w.at<void>(B_VN), nullptr, nullptr, cache_len,
                             cache_cap, dev_status, s));
     DG_TRY(launch_attention(c.act_dtype, batch, C, c.n_q_heads, c.n_kv_heads, c.head_dim,

@@ -57,6 +57,26 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
   return t;
 }
 
+// acc[j] = p[e_j] + p[stride + e_j] + ... + p[(n - 1) stride + e_j] for the 8 elements
+// e_j = e0 + j * step (those < count; the others get 0), added in slice order (deterministic).  The
+// slice loop is outermost so the 8 loads of a slice are in flight together.
+__device__ __forceinline__ void sum_parts8(const float *__restrict__ p, int n, size_t stride,
+                                           int e0, int step, int count, float (&acc)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = e0 + j * step;
+    acc[j] = e < count ? p[e] : 0.f;
+  }
+  for (int s = 1; s < n; ++s) {
+    const float *q = p + (size_t)s * stride;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + j * step;
+      if (e < count) acc[j] += q[e];
+    }
+  }
+}
+
 }  // namespace dg
 
 // ---- host-side launch bookkeeping (defined in dg_api.cu) ----------------------------------
@@ -65,4 +85,5 @@ namespace dg {
 // timing event on `s` before the launch, labelled `name`).
 void note_launch(cudaStream_t s, const char *name);
 int check_launch(const char *what);      // DG_OK or DG_ERR_CUDA (records the message)
+
 }  // namespace dg

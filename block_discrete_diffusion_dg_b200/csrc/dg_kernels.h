@@ -27,6 +27,9 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
 // e4m3 codes [n] -> bf16 [n] (n % 16 == 0), exact.
 int launch_dequant_e4m3(const void *src, size_t n, void *dst, cudaStream_t s);
 // in: fp32 rows (residual stream); out: activation type.
+// h_out = res + sum of n_parts fp32 partials [n_parts][rows][d]; out = RMSNorm(h_out).
+int launch_resid_norm(int act, const float *part, int n_parts, const float *res, int rows, int d,
+                      double eps, float *h_out, void *out, cudaStream_t s);
 int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
                    int max_rows, int d, double eps, void *out, cudaStream_t s);
 // live[b*C+i] = !done[b] && (masked == NULL || masked[b*C+i]); row_idx = positions with live
@@ -63,8 +66,8 @@ int launch_rope_table(int batch, int n, int hd, double theta, const int32_t *cac
 // qkv fp32 [B*n][(Hq+2Hkv)hd] -> q [B*n][Hq][hd], k_new/v_new [B][Hkv][n][hd] (act type, RoPE
 // on q and k).  If k_cache != NULL also writes k/v to cache rows cache_len[b] + i (< cap).
 int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const float *qkv,
-                     const float *cs, void *q, void *k_new, void *v_new, void *k_cache,
-                     void *v_cache, const int32_t *cache_len, int cap, int32_t *st,
+                     int n_parts, const float *cs, void *q, void *k_new, void *v_new,
+                     void *k_cache, void *v_cache, const int32_t *cache_len, int cap, int32_t *st,
                      cudaStream_t s);
 int launch_add_cache_len(int batch, int n, int cap, int32_t *cache_len, cudaStream_t s);
 
@@ -90,13 +93,15 @@ int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *
 // Top-k + gates from fp32 router logits z [T][E] (E <= 256, k <= 32), one warp per token.
 int launch_router_topk(int T, int E, int k, const float *z, const uint8_t *token_live,
                        int32_t *topk_idx, float *topk_w, cudaStream_t s,
-                       const int32_t *forced = nullptr);
+                       const int32_t *forced = nullptr,
+                       int n_parts = 1);
 // Top-k + gates (router_topk, many blocks), then the stable permutation and the tile list in one
 // block (permute_tiles).
 int launch_route(int T, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
-                 cudaStream_t s, const int32_t *forced = nullptr);
+                 cudaStream_t s, const int32_t *forced = nullptr,
+                 int n_parts = 1);
 // Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
 int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s);
@@ -145,6 +150,12 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
 
 // ---- tensor-core GEMMs (k_gemm_tc.cu) -----------------------------------------------------------
 bool gemm_tc_supported(int act, int w, int K);
+// Swap-AB split-K projection for at most 256 tokens: part[s][t][n] (fp32) over K slices s.
+bool split_supported(int act, int w, int T, int N, int K);
+int split_k_slices(int N, int K, int max_slices = 16);
+int launch_gemm_tc_split(const void *W, int N, const void *X, int T, int T_alloc, int K,
+                         int k_split, float *part, const char *name, int32_t *st, cudaStream_t s,
+                         const float *scale);
 // out[M][N] = A[M][K] W[N][K]^T (+ res[M][N]) in fp32; A has room for roundup(M, 128) rows.
 // scale (or null): per output channel (W row), multiplies the fp32 accumulator.
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,

@@ -8,6 +8,11 @@
 // warps 2-5 epilogue over a double-buffered accumulator.
 //
 // Dense:  A = activation rows (M = tokens), B = weight rows (N = output channels).
+// Split (swap-AB, split-K; at most 256 tokens): A = 128 weight rows (output channels), B = all
+// the token rows; a unit is (channel tile, K slice) and leaves an fp32 partial
+// part[slice][token][channel] that the consumer sums over the slices in order.  Each unit runs
+// K / slices of the reduction, so ~128 CTAs stream the weights in a few k-steps each, and the
+// activation rows are read once per channel tile instead of once per 64 channels.
 // Experts (swap-AB): A = expert weight rows (M = 128 output channels), B = the tokens routed to
 // the expert (N = their count rounded up to 16, at most BN_MAX per unit), so the weights stream
 // through the tensor cores once at the small per-expert token counts of batch 1.  For the
@@ -28,12 +33,13 @@ using namespace tc;
 constexpr int BM = 128, BK = 64;
 constexpr int NUM_THREADS = 192;
 
-enum Kind { K_DENSE_F32 = 0, K_DENSE_RESID = 1, K_MOE_GATE = 2, K_MOE_DOWN = 3 };
+enum Kind { K_DENSE_F32 = 0, K_DENSE_RESID = 1, K_MOE_GATE = 2, K_MOE_DOWN = 3, K_SPLIT = 4 };
 
 struct Params {
   int kind, K;
   // dense: M rows (tokens), N columns (channels), tile width bn
-  int M, N, m_tiles, bn;
+  // split: M tokens, N channels, m_tiles = N / 128 channel tiles, k_split K slices
+  int M, N, m_tiles, bn, k_split;
   float *out_f32;        // dense output (fp32)
   const float *res;      // dense residual (fp32) or null
   int ldo;
@@ -46,6 +52,8 @@ struct Params {
   int ld_out;       // row stride of the expert output (F for a, d for Y)
   void *out;        // gate/up: a [assignments][F] (bf16); down: Y [assignments][d] (fp32)
   const float *scale;  // per output channel (dense: [N]; experts: [E][w_rows]) or null
+  int smem_epi;        // split with one unit per CTA: stage the tile in the (then idle) pipeline
+                       // buffers and write it with one TMA store through tmC
   int32_t *status;
 };
 
@@ -58,6 +66,7 @@ struct Unit {
 
 __device__ __forceinline__ int n_units(const Params &p) {
   if (p.kind <= K_DENSE_RESID) return p.m_tiles * ((p.N + p.bn - 1) / p.bn);
+  if (p.kind == K_SPLIT) return p.m_tiles * p.k_split;
   return *p.n_tiles_dev * p.m_tiles;
 }
 
@@ -65,7 +74,15 @@ template <int BN_MAX>
 __device__ __forceinline__ Unit decode(const Params &p, int u) {
   Unit x;
   const int mt = u % p.m_tiles, t = u / p.m_tiles;
-  if (p.kind <= K_DENSE_RESID) {
+  if (p.kind == K_SPLIT) {
+    x.a_row0 = mt * BM;
+    x.a_row1 = -1;
+    x.b_row0 = 0;
+    x.n_valid = p.M;
+    x.n_mma = (p.M + 15) & ~15;
+    x.row0 = mt * BM;  // first channel
+    x.col0 = t;        // K slice
+  } else if (p.kind <= K_DENSE_RESID) {
     x.a_row0 = mt * BM;
     x.a_row1 = -1;
     x.b_row0 = t * p.bn;
@@ -115,7 +132,7 @@ struct Cfg {
 template <int BN_MAX, int STAGES, int B_BOX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   Params p) {
+                   const __grid_constant__ CUtensorMap tmC, Params p) {
   using C = Cfg<BN_MAX, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -149,6 +166,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (p.smem_epi) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -171,7 +189,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const Unit x = decode<BN_MAX>(p, u);
         const int nb = (x.n_mma + B_BOX - 1) / B_BOX;
         const uint32_t bytes = C::A_BYTES + (uint32_t)nb * B_BOX * BK * 2;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kpb = p.kind == K_SPLIT ? kblocks / p.k_split : kblocks;
+        const int kb0 = p.kind == K_SPLIT ? x.col0 * kpb : 0;
+        for (int kb = kb0; kb < kb0 + kpb; ++kb) {
           if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
           mbar_expect_tx(&full[stage], bytes);
           uint8_t *a = sA + stage * C::A_BYTES;
@@ -207,14 +227,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_after();
         const uint32_t d = tmem + acc * C::ACC_STRIDE;
         bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kpb = p.kind == K_SPLIT ? kblocks / p.k_split : kblocks;
+        const int kb0 = p.kind == K_SPLIT ? x.col0 * kpb : 0;
+        for (int kb = kb0; kb < kb0 + kpb; ++kb) {
           if (!mbar_wait(&full[stage], ph)) { fail(p.status, abort_flag); ok = false; break; }
           fence_after();
           const uint64_t ad = sdesc_sw128(sA + stage * C::A_BYTES);
           const uint64_t bd = sdesc_sw128(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           commit(&empty[stage]);
           last_stage = stage;
           last_ph = ph;
@@ -248,7 +270,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld_wait(v);
         const int nv = min(32, x.n_valid - c * 32);
         if (p.scale) {  // e4m3 weights: the fp32 accumulator times the output channel's scale
-          if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
+          if (p.kind == K_SPLIT) {
+            const float sc = p.scale[x.row0 + r];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * sc);
+          } else if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
             const float *sc = p.scale + x.col0 + c * 32;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -263,7 +289,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * sc);
           }
         }
-        if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
+        if (p.kind == K_SPLIT && p.smem_epi) {
+          // staged as [token][128 channels] over the pipeline buffers (all MMAs of the CTA's only
+          // unit have completed, so nothing reads or fills them any more)
+          float *stg = reinterpret_cast<float *>(sA);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[(c * 32 + j) * BM + r] = __uint_as_float(v[j]);
+        } else if (p.kind == K_SPLIT) {
+          // part[slice][token][channel]: for each token the 32 lanes store 32 consecutive channels
+          const int ch = x.row0 + r;
+          float *o = p.out_f32 + ((size_t)x.col0 * p.M + c * 32) * p.ldo + ch;
+          if (ch < p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nv) o[(size_t)j * p.ldo] = __uint_as_float(v[j]);
+          }
+        } else if (p.kind == K_DENSE_F32 || p.kind == K_DENSE_RESID) {
           const int row = x.row0 + r;
           if (row < p.M) {
             const int col = x.col0 + c * 32;
@@ -326,6 +367,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           epi_bar();
         }
       }
+      if (p.kind == K_SPLIT && p.smem_epi) {  // one TMA store of the [tokens][128] fp32 tile
+        fence_proxy_async_smem();
+        epi_bar();
+        if (warp == 2 && lane == 0) {
+          tma_store_3d(&tmC, sA, x.row0, 0, x.col0);
+          bulk_commit();
+          bulk_wait_all();
+        }
+      }
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -342,7 +392,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int BN_MAX, int STAGES, int B_BOX>
 int launch(const CUtensorMap &tmA, const CUtensorMap &tmB, const Params &p, int units_max,
-           const char *name, cudaStream_t s, int ctas_per_sm = 1) {
+           const char *name, cudaStream_t s, int ctas_per_sm = 1,
+           const CUtensorMap *tmC = nullptr) {
   using C = Cfg<BN_MAX, STAGES>;
   auto k = gemm_tc_kernel<BN_MAX, STAGES, B_BOX>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
@@ -350,7 +401,7 @@ int launch(const CUtensorMap &tmA, const CUtensorMap &tmB, const Params &p, int 
   const int grid = units_max < slots ? units_max : slots;
   if (grid <= 0) return DG_OK;
   note_launch(s, name);
-  k<<<grid, NUM_THREADS, C::SMEM, s>>>(tmA, tmB, p);
+  k<<<grid, NUM_THREADS, C::SMEM, s>>>(tmA, tmB, tmC ? *tmC : tmA, p);
   return check_launch(name);
 }
 
@@ -391,6 +442,58 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
   const int units = p.m_tiles * ((N + BN - 1) / BN);
   if (BN == 16) return launch<16, 10, 16>(ta, tb, p, units, name, s);
   return launch<64, 8, 64>(ta, tb, p, units, name, s);
+}
+
+// Split: part[s][t][n] = sum over k in slice s of W[n][k] X[t][k] (times scale[n] when given), for
+// t < T <= 256, n < N (N a multiple of 128), slices s < k_split (K a multiple of 64 k_split).  X is
+// the activation buffer [T_alloc][K] with T_alloc >= T rows allocated.
+int split_k_slices(int N, int K, int max_slices) {
+  const int m_tiles = N / BM, kblocks = K / BK;
+  int s = num_sms() / (m_tiles > 0 ? m_tiles : 1);
+  if (s > max_slices) s = max_slices;
+  if (s < 1) s = 1;
+  if (s > kblocks) s = kblocks;
+  while (kblocks % s) --s;
+  return s;
+}
+
+bool split_supported(int act, int w, int T, int N, int K) {
+  return gemm_tc_supported(act, w, K) && T > 0 && T <= 256 && N % BM == 0;
+}
+
+int launch_gemm_tc_split(const void *W, int N, const void *X, int T, int T_alloc, int K,
+                         int k_split, float *part, const char *name, int32_t *st, cudaStream_t s,
+                         const float *scale) {
+  if (T <= 0 || T > 256 || N % BM || K % (BK * k_split)) return DG_ERR_UNSUPPORTED;
+  const int bn = T <= 128 ? 128 : 256;
+  CUtensorMap ta, tb;
+  int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, N, (uint64_t)K * 2, BK, BM);
+  if (rc != DG_OK) return rc;
+  rc = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, T_alloc, (uint64_t)K * 2, BK,
+                    bn);
+  if (rc != DG_OK) return rc;
+  Params p{};
+  p.kind = K_SPLIT;
+  p.K = K;
+  p.M = T;
+  p.N = N;
+  p.m_tiles = N / BM;
+  p.k_split = k_split;
+  p.out_f32 = part;
+  p.ldo = N;
+  p.scale = scale;
+  p.status = st;
+  const int units = p.m_tiles * k_split;
+  // one unit per CTA: the epilogue stages the tile in shared memory and stores it with TMA
+  CUtensorMap tc_out;
+  p.smem_epi = 0;
+  if (units <= num_sms()) {
+    rc = make_tmap_3d_f32(&tc_out, part, N, T, k_split, BM, bn, 1);
+    if (rc != DG_OK) return rc;
+    p.smem_epi = 1;
+  }
+  if (bn == 128) return launch<128, 6, 128>(ta, tb, p, units, name, s, 1, &tc_out);
+  return launch<256, 4, 256>(ta, tb, p, units, name, s, 1, &tc_out);
 }
 
 // Experts (swap-AB).  gate_up: W [E][2F][K], X = the routed rows [assignments][K] (permuted order)

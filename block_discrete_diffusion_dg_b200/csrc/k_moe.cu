@@ -84,7 +84,9 @@ __global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__
 // (lower expert index first on equal values), gates = softmax over the selected logits.
 // With `forced` non-null the k experts of token t are forced[t][0..k-1] (in that order) instead of
 // the k largest logits; the gates are still the softmax over the selected logits.
-__global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict__ z,
+// z may hold n_parts fp32 partial sums [n_parts][T][E] (split-K router logits), added in order.
+
+__global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict__ z, int n_parts,
                                    const uint8_t *__restrict__ token_live,
                                    const int32_t *__restrict__ forced, int32_t *topk_idx,
                                    float *topk_w) {
@@ -93,10 +95,15 @@ __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict
   if (t >= T_) return;
   const bool live = token_live == nullptr || token_live[t] != 0;
   const float *zr = z + (size_t)t * E;
+  const size_t zs = (size_t)T_ * E;
   if (forced) {
     const int e = lane < k ? forced[(size_t)t * k + lane] : -1;
     const bool ok = e >= 0 && e < E;
-    const float ze = ok ? zr[e] : -INFINITY;
+    float ze = -INFINITY;
+    if (ok) {
+      ze = zr[e];
+      for (int s = 1; s < n_parts; ++s) ze += zr[s * zs + e];
+    }
     const float z0 = __shfl_sync(0xffffffffu, ze, 0);
     const float p = (lane < k && ok) ? expf(ze - z0) : 0.f;
     float denom = p;
@@ -110,7 +117,11 @@ __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict
   }
   float zv[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) zv[i] = (lane + 32 * i < E) ? zr[lane + 32 * i] : -INFINITY;
+  for (int i = 0; i < 8; ++i) zv[i] = 0.f;
+  sum_parts8(zr, n_parts, zs, lane, 32, E, zv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (lane + 32 * i >= E) zv[i] = -INFINITY;
   unsigned taken = 0u;
   float z0 = 0.f, denom = 0.f, mine = 0.f;
   int my_idx = -1;
@@ -439,22 +450,23 @@ int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void 
 }
 
 int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *token_live,
-                       int32_t *topk_idx, float *topk_w, cudaStream_t s, const int32_t *forced) {
+                       int32_t *topk_idx, float *topk_w, cudaStream_t s, const int32_t *forced,
+                       int n_parts) {
   if (T_ <= 0) return DG_OK;
   if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
   note_launch(s, "router_topk");
-  router_topk_kernel<<<(T_ + 7) / 8, 256, 0, s>>>(T_, E, k, z, token_live, forced, topk_idx,
-                                                  topk_w);
+  router_topk_kernel<<<(T_ + 7) / 8, 256, 0, s>>>(T_, E, k, z, n_parts, token_live, forced,
+                                                  topk_idx, topk_w);
   return check_launch("router_topk");
 }
 
 int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
-                 cudaStream_t s, const int32_t *forced) {
+                 cudaStream_t s, const int32_t *forced, int n_parts) {
   if (T_ <= 0) return DG_OK;
   if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
-  const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced);
+  const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced, n_parts);
   if (rc != DG_OK) return rc;
   note_launch(s, "permute_tiles");
   permute_tiles_kernel<<<1, 1024, 0, s>>>(T_ * k, E, topk_idx, expert_off, perm, inv_perm, tile_m,

@@ -29,16 +29,27 @@ __global__ void rope_table_kernel(int n, int hd, double theta, const int32_t *__
   }
 }
 
+// qkv holds n_parts fp32 partial sums [n_parts][B n][width] (split-K projection), added here in
+// slice order; the summed row is staged in shared memory.
 template <typename T>
 __global__ void qkv_split_kernel(int n, int Hq, int Hkv, int hd, const float *__restrict__ qkv,
-                                 const float *__restrict__ cs, T *q, T *k_new, T *v_new, T *k_cache,
-                                 T *v_cache, const int32_t *__restrict__ cache_len, int cap,
-                                 int32_t *st) {
+                                 int n_parts, size_t part_stride, const float *__restrict__ cs,
+                                 T *q, T *k_new, T *v_new, T *k_cache, T *v_cache,
+                                 const int32_t *__restrict__ cache_len, int cap, int32_t *st) {
+  extern __shared__ float qkv_row[];
   const int row = blockIdx.x;  // b*n + i
   const int b = row / n, i = row % n;
   const int half = hd / 2;
   const int width = (Hq + 2 * Hkv) * hd;
-  const float *src = qkv + (size_t)row * width;
+  for (int e0 = threadIdx.x; e0 < width; e0 += 8 * blockDim.x) {
+    float acc[8];
+    sum_parts8(qkv + (size_t)row * width, n_parts, part_stride, e0, blockDim.x, width, acc);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (e0 + j * (int)blockDim.x < width) qkv_row[e0 + j * blockDim.x] = acc[j];
+  }
+  __syncthreads();
+  const float *src = qkv_row;
   const float *c = cs + (size_t)row * hd;
   int crow = -1;
   if (k_cache) {
@@ -89,20 +100,24 @@ int launch_rope_table(int batch, int n, int hd, double theta, const int32_t *cac
 }
 
 int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const float *qkv,
-                     const float *cs, void *q, void *k_new, void *v_new, void *k_cache,
-                     void *v_cache, const int32_t *cache_len, int cap, int32_t *st,
+                     int n_parts, const float *cs, void *q, void *k_new, void *v_new,
+                     void *k_cache, void *v_cache, const int32_t *cache_len, int cap, int32_t *st,
                      cudaStream_t s) {
   note_launch(s, "qkv_split");
+  const int width = (Hq + 2 * Hkv) * hd;
+  const size_t smem = (size_t)width * sizeof(float);
+  const size_t stride = (size_t)batch * n * width;
+  if (smem > 48 * 1024) return DG_ERR_UNSUPPORTED;
   if (act == DG_F32)
-    qkv_split_kernel<float><<<batch * n, 256, 0, s>>>(n, Hq, Hkv, hd, qkv, cs, (float *)q,
-                                                      (float *)k_new, (float *)v_new,
-                                                      (float *)k_cache, (float *)v_cache,
-                                                      cache_len, cap, st);
+    qkv_split_kernel<float><<<batch * n, 256, smem, s>>>(n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
+                                                         (float *)q, (float *)k_new,
+                                                         (float *)v_new, (float *)k_cache,
+                                                         (float *)v_cache, cache_len, cap, st);
   else
-    qkv_split_kernel<bf16><<<batch * n, 256, 0, s>>>(n, Hq, Hkv, hd, qkv, cs, (bf16 *)q,
-                                                     (bf16 *)k_new, (bf16 *)v_new,
-                                                     (bf16 *)k_cache, (bf16 *)v_cache, cache_len,
-                                                     cap, st);
+    qkv_split_kernel<bf16><<<batch * n, 256, smem, s>>>(n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
+                                                        (bf16 *)q, (bf16 *)k_new, (bf16 *)v_new,
+                                                        (bf16 *)k_cache, (bf16 *)v_cache,
+                                                        cache_len, cap, st);
   return check_launch("qkv_split");
 }
 

@@ -63,6 +63,38 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float *__restrict__ 
   for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f<T>(src[j] * inv);
 }
 
+// h = res + sum of n_parts fp32 partials [n_parts][rows][d] (split-K output projection, added in
+// slice order), written to h_out; out = RMSNorm(h) in the activation type.  One block per row,
+// the row staged in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) resid_norm_kernel(const float *__restrict__ part,
+                                                         int n_parts, size_t part_stride,
+                                                         const float *__restrict__ res, int d,
+                                                         float eps, float *h_out, T *out) {
+  extern __shared__ float hrow[];
+  __shared__ float red[8];
+  const int r = blockIdx.x;
+  float ss = 0.f;
+  for (int j0 = threadIdx.x; j0 < d; j0 += 8 * blockDim.x) {
+    float acc[8];
+    sum_parts8(part + (size_t)r * d, n_parts, part_stride, j0, blockDim.x, d, acc);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = j0 + q * blockDim.x;
+      if (j < d) {
+        const float v = res[(size_t)r * d + j] + acc[q];
+        hrow[j] = v;
+        h_out[(size_t)r * d + j] = v;
+        ss += v * v;
+      }
+    }
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  T *o = out + (size_t)r * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f<T>(hrow[j] * inv);
+}
+
 // One block of 1024 threads scans all B*C positions in chunks (B*C <= 65536).
 __global__ void __launch_bounds__(1024) compact_rows_kernel(int batch, int canvas,
                                                             const uint8_t *__restrict__ masked,
@@ -264,6 +296,22 @@ int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_
     rmsnorm_kernel<bf16><<<max_rows, 256, 0, s>>>((const float *)in, row_idx, n_rows_dev, d,
                                                   (float)eps, (bf16 *)out);
   return check_launch("rmsnorm");
+}
+
+int launch_resid_norm(int act, const float *part, int n_parts, const float *res, int rows, int d,
+                      double eps, float *h_out, void *out, cudaStream_t s) {
+  if (rows <= 0) return DG_OK;
+  const size_t smem = (size_t)d * sizeof(float);
+  if (smem > 48 * 1024) return DG_ERR_UNSUPPORTED;
+  note_launch(s, "resid_norm");
+  const size_t stride = (size_t)rows * d;
+  if (act == DG_F32)
+    resid_norm_kernel<float><<<rows, 256, smem, s>>>(part, n_parts, stride, res, d, (float)eps,
+                                                     h_out, (float *)out);
+  else
+    resid_norm_kernel<bf16><<<rows, 256, smem, s>>>(part, n_parts, stride, res, d, (float)eps,
+                                                    h_out, (bf16 *)out);
+  return check_launch("resid_norm");
 }
 
 int launch_compact_rows(int batch, int canvas, const uint8_t *masked, const int32_t *done,
