@@ -2,6 +2,8 @@
 // warp/block reductions and the launch bookkeeping used by every kernel file.
 #pragma once
 
+#include <utility>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -77,6 +79,15 @@ __device__ __forceinline__ void sum_parts8(const float *__restrict__ p, int n, s
   }
 }
 
+// Programmatic dependent launch.  Every kernel of the library starts with pdl_wait() (nothing is
+// read before the preceding kernel of the stream has completed and its writes are visible) and
+// pdl_trigger() (the next kernel may be scheduled now, so its launch and block setup overlap this
+// kernel's work instead of following it).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace dg
 
 // ---- host-side launch bookkeeping (defined in dg_api.cu) ----------------------------------
@@ -86,4 +97,22 @@ namespace dg {
 void note_launch(cudaStream_t s, const char *name);
 int check_launch(const char *what);      // DG_OK or DG_ERR_CUDA (records the message)
 
+
+// Launches `k` with programmatic stream serialisation allowed (see pdl_wait); errors surface
+// through check_launch() like a <<<>>> launch.
+template <typename... P, typename... A>
+inline void launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       A &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, k, static_cast<P>(args)...);
+}
 }  // namespace dg

@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(int n, int Hq, int Hkv,
                                                        int cap, const T *__restrict__ kn,
                                                        const T *__restrict__ vn, int causal,
                                                        const int32_t *__restrict__ done, T *out) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int KB = (HD >= 128) ? 32 : 64;  // keys per tile (static smem stays < 48 KB)
   constexpr int G = NT / HD;                  // query groups
   constexpr int QPT = QB / G;                 // queries per thread
@@ -140,7 +142,7 @@ int run(int hd, dim3 grid, cudaStream_t s, int n, int Hq, int Hkv, const void *q
   note_launch(s, "attn_simt");
 #define DG_ATTN_CASE(HDV)                                                                    \
   case HDV:                                                                                  \
-    attn_simt_kernel<T, HDV><<<grid, NT, 0, s>>>(n, Hq, Hkv, (const T *)q, (const T *)kc,    \
+    launch_pdl(attn_simt_kernel<T, HDV>, grid, NT, 0, s, n, Hq, Hkv, (const T *)q, (const T *)kc, \
                                                  (const T *)vc, len, cap, (const T *)kn,     \
                                                  (const T *)vn, causal, done, (T *)out);     \
     break;

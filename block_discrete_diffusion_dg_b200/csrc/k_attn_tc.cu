@@ -121,6 +121,8 @@ constexpr size_t attn_smem_bytes() {
 
 template <int HD>
 __global__ void __launch_bounds__(NTHR) attn_tc_kernel(AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t attn_smem[];
   bf16 *sQ = reinterpret_cast<bf16 *>(attn_smem);
   bf16 *sKb = sQ + ROWS * HD;           // [2][KT * HD]
@@ -327,6 +329,8 @@ template <int HD>
 __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float *__restrict__ part_o,
                                   const float2 *__restrict__ part_ml,
                                   const int32_t *__restrict__ done, bf16 *out) {
+  pdl_wait();
+  pdl_trigger();
   const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= B * Hq * n) return;
@@ -410,6 +414,8 @@ __global__ void __launch_bounds__(T5_THR, 1)
                     const __grid_constant__ CUtensorMap tmVc,
                     const __grid_constant__ CUtensorMap tmKn,
                     const __grid_constant__ CUtensorMap tmVn, T5Args a) {
+  pdl_wait();
+  pdl_trigger();
   using namespace tc;
   extern __shared__ uint8_t t5_smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)t5_smem_raw + 1023) & ~(uintptr_t)1023);
@@ -896,12 +902,12 @@ int launch_tc5(int batch, int n, int Hq, int Hkv, const void *q, const void *k_c
   dim3 grid((n + 2 * qpc - 1) / (2 * qpc), Hkv, batch * a.splits);
   note_launch(s, "attn_tc");
   cudaFuncSetAttribute(attn_tc5_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T5_SMEM);
-  attn_tc5_kernel<<<grid, T5_THR, T5_SMEM, s>>>(tq, tkc, tvc, tkn, tvn, a);
+  launch_pdl(attn_tc5_kernel, grid, T5_THR, T5_SMEM, s, tq, tkc, tvc, tkn, tvn, a);
   rc = check_launch("attn_tc");
   if (rc != DG_OK || a.splits == 1) return rc;
   note_launch(s, "attn_merge");
   const int warps = batch * Hq * n;
-  attn_merge_kernel<128><<<(warps + 7) / 8, 256, 0, s>>>(a.splits, batch, Hq, n, a.part_o,
+  launch_pdl(attn_merge_kernel<128>, (warps + 7) / 8, 256, 0, s, a.splits, batch, Hq, n, a.part_o,
                                                           a.part_ml, done, (bf16 *)out);
   return check_launch("attn_merge");
 }
@@ -940,11 +946,11 @@ int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q
   if (hd == 128) {
     cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)attn_smem_bytes<128>());
-    attn_tc_kernel<128><<<grid, NTHR, attn_smem_bytes<128>(), s>>>(a);
+    launch_pdl(attn_tc_kernel<128>, grid, NTHR, attn_smem_bytes<128>(), s, a);
   } else {
     cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)attn_smem_bytes<64>());
-    attn_tc_kernel<64><<<grid, NTHR, attn_smem_bytes<64>(), s>>>(a);
+    launch_pdl(attn_tc_kernel<64>, grid, NTHR, attn_smem_bytes<64>(), s, a);
   }
   int rc = check_launch("attn_tc");
   if (rc != DG_OK || a.splits == 1) return rc;
@@ -952,11 +958,11 @@ int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q
   const int warps = batch * Hq * n;
   const int mgrid = (warps + 7) / 8;
   if (hd == 128)
-    attn_merge_kernel<128><<<mgrid, 256, 0, s>>>(a.splits, batch, Hq, n, a.part_o, a.part_ml,
-                                                 done, (bf16 *)out);
+    launch_pdl(attn_merge_kernel<128>, mgrid, 256, 0, s, a.splits, batch, Hq, n, a.part_o,
+               a.part_ml, done, (bf16 *)out);
   else
-    attn_merge_kernel<64><<<mgrid, 256, 0, s>>>(a.splits, batch, Hq, n, a.part_o, a.part_ml, done,
-                                                (bf16 *)out);
+    launch_pdl(attn_merge_kernel<64>, mgrid, 256, 0, s, a.splits, batch, Hq, n, a.part_o,
+               a.part_ml, done, (bf16 *)out);
   return check_launch("attn_merge");
 }
 

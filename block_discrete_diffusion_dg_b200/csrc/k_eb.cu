@@ -8,10 +8,13 @@
 // per step.  With entropies sorted, that is: commit rank r iff r == 0 or sum_{i<r} H_(i) <= gamma.
 //
 // Bit-exactness: keys are (fp32 bits of max(H, 0), position) — order-preserving for H >= 0 and
-// lower position first on ties — sorted by a block bitonic sort; sums run in int64 fixed point
-// with 32 fraction bits (Q(H) = nearest integer to H * 2^32, exact in fp64), so the prefix
-// test is exact and independent of summation order.  At step index >= max_steps - 1 every
-// masked position is committed (the canvas always finishes within max_steps).
+// lower position first on ties, so all keys are distinct; sums run in int64 fixed point with 32
+// fraction bits (Q(H) = nearest integer to H * 2^32, exact in fp64), so the prefix test is exact
+// and independent of summation order.  The sum over the ranks before r in sorted order is the
+// sum of Q over the keys smaller than the rank-r key, which each thread forms directly by one pass
+// over the keys in shared memory (every thread reads the same key at a time: a broadcast), so no
+// sort is needed.  At step index >= max_steps - 1 every masked position is committed (the canvas
+// always finishes within max_steps).
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -24,80 +27,60 @@ __global__ void __launch_bounds__(1024) eb_kernel(int C, const float *__restrict
                                                   int max_steps, int32_t *tokens, uint8_t *masked,
                                                   uint8_t *selected, int32_t *n_masked,
                                                   int32_t *done, int32_t *step, int32_t *st) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ unsigned long long keys[1024];
-  __shared__ long long scan[1024];
+  __shared__ long long qv[1024];
   __shared__ int bad, n_valid, n_commit;
   const int b = blockIdx.x, tid = threadIdx.x;
   if (done[b]) return;
-  int N = 1;
-  while (N < C) N <<= 1;
   if (tid == 0) { bad = 0; n_valid = 0; n_commit = 0; }
   __syncthreads();
   const size_t base = (size_t)b * C;
-  if (tid < N) {
-    unsigned long long key = ~0ull;
-    if (tid < C && masked[base + tid]) {
-      float h = H[base + tid];
-      if (!isfinite(h)) atomicOr(&bad, 1);
-      h = (h > 0.f) ? h : 0.f;  // negative rounding residue and -0 count as +0
-      key = ((unsigned long long)__float_as_uint(h) << 32) | (unsigned)tid;
-      atomicAdd(&n_valid, 1);
-    }
+  unsigned long long key = ~0ull;
+  long long q = 0;
+  const bool mine = tid < C && masked[base + tid];
+  if (mine) {
+    float h = H[base + tid];
+    if (!isfinite(h)) atomicOr(&bad, 1);
+    h = (h > 0.f) ? h : 0.f;  // negative rounding residue and -0 count as +0
+    key = ((unsigned long long)__float_as_uint(h) << 32) | (unsigned)tid;
+    q = __double2ll_rn((double)h * 4294967296.0);
+    atomicAdd(&n_valid, 1);
+  }
+  if (tid < C) {
     keys[tid] = key;
+    qv[tid] = q;
   }
   __syncthreads();
   if (bad) {
     if (tid == 0) set_status(st, DG_ERR_NUMERIC);
     return;
   }
-  // bitonic sort, ascending
-  for (int kk = 2; kk <= N; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      if (tid < N) {
-        const int ixj = tid ^ j;
-        if (ixj > tid) {
-          const unsigned long long a = keys[tid], c = keys[ixj];
-          const bool up = (tid & kk) == 0;
-          if ((a > c) == up) { keys[tid] = c; keys[ixj] = a; }
+  if (tid < C) {
+    bool commit = false;
+    if (mine) {
+      int rank = 0;
+      long long excl = 0;  // sum of Q over the smaller keys = the exclusive prefix in sorted order
+      for (int j = 0; j < C; ++j) {
+        const unsigned long long kj = keys[j];
+        if (kj < key) {
+          ++rank;
+          excl += qv[j];
         }
       }
-      __syncthreads();
+      commit = step[b] >= max_steps - 1 || rank == 0 || excl <= qg;
+      if (commit) {
+        tokens[base + tid] = am[base + tid];
+        masked[base + tid] = 0;
+        atomicAdd(&n_commit, 1);
+      }
     }
-  }
-  const int nv = n_valid;
-  long long q = 0;
-  unsigned long long key = ~0ull;
-  if (tid < nv) {
-    key = keys[tid];
-    const float h = __uint_as_float((unsigned)(key >> 32));
-    q = __double2ll_rn((double)h * 4294967296.0);
-  }
-  if (tid < N) scan[tid] = q;
-  __syncthreads();
-  // inclusive Hillis-Steele scan over ranks
-  for (int o = 1; o < N; o <<= 1) {
-    long long v = 0;
-    if (tid < N && tid >= o) v = scan[tid - o];
-    __syncthreads();
-    if (tid < N) scan[tid] += v;
-    __syncthreads();
-  }
-  if (tid < C) selected ? (void)(selected[base + tid] = 0) : (void)0;
-  __syncthreads();
-  if (tid < nv) {
-    const long long excl = scan[tid] - q;
-    const bool force = step[b] >= max_steps - 1;
-    if (force || tid == 0 || excl <= qg) {
-      const int pos = (int)(key & 0xffffffffu);
-      tokens[base + pos] = am[base + pos];
-      masked[base + pos] = 0;
-      if (selected) selected[base + pos] = 1;
-      atomicAdd(&n_commit, 1);
-    }
+    if (selected) selected[base + tid] = commit ? 1 : 0;
   }
   __syncthreads();
   if (tid == 0) {
-    const int left = nv - n_commit;
+    const int left = n_valid - n_commit;
     n_masked[b] = left;
     step[b] = step[b] + 1;
     done[b] = (left == 0);
@@ -114,7 +97,7 @@ int launch_eb_select(int batch, int canvas, const float *entropy, const int32_t 
   int N = 32;
   while (N < canvas) N <<= 1;
   note_launch(s, "eb_select");
-  eb_kernel<<<batch, N, 0, s>>>(canvas, entropy, argmax, q_gamma, max_steps, tokens, masked,
+  launch_pdl(eb_kernel, batch, N, 0, s, canvas, entropy, argmax, q_gamma, max_steps, tokens, masked,
                                 selected, n_masked, done, step, st);
   return check_launch("eb_select");
 }

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) entropy_rows_kernel(const float *__restri
                                                            const int32_t *__restrict__ row_idx,
                                                            float *entropy, int32_t *argmax,
                                                            int32_t *st) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   if (n_rows && r >= *n_rows) return;
   const float *z = logits + (size_t)r * V;
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(256) entropy_rows_kernel(const float *__restri
 __global__ void scatter_rows_kernel(const float *__restrict__ src, int width,
                                     const int32_t *__restrict__ n_rows,
                                     const int32_t *__restrict__ row_idx, float *dst) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.y;
   if (n_rows && r >= *n_rows) return;
   const float *sr = src + (size_t)r * width;
@@ -72,7 +76,7 @@ int launch_scatter_rows(const float *src, int width, int max_rows, const int32_t
   if (max_rows <= 0) return DG_OK;
   note_launch(s, "scatter_rows");
   dim3 grid((width + 1023) / 1024 < 64 ? (width + 1023) / 1024 : 64, max_rows);
-  scatter_rows_kernel<<<grid, 256, 0, s>>>(src, width, n_rows, row_idx, dst);
+  launch_pdl(scatter_rows_kernel, grid, 256, 0, s, src, width, n_rows, row_idx, dst);
   return check_launch("scatter_rows");
 }
 
@@ -81,7 +85,7 @@ int launch_entropy_rows(const float *logits, int V, int max_rows, const int32_t 
                         cudaStream_t s) {
   if (max_rows <= 0) return DG_OK;
   note_launch(s, "entropy_rows");
-  entropy_rows_kernel<<<max_rows, 256, 0, s>>>(logits, V, n_rows, row_idx, entropy, argmax, st);
+  launch_pdl(entropy_rows_kernel, max_rows, 256, 0, s, logits, V, n_rows, row_idx, entropy, argmax, st);
   return check_launch("entropy_rows");
 }
 

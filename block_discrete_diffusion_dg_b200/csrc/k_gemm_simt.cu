@@ -29,6 +29,8 @@ struct Args {
 template <typename AT, typename WT, typename OT, int EPI>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(Args<AT, WT> g, OT *out, int ldo,
                                                         const OT *res) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN + 4];
   const int n0 = blockIdx.y * BN;
@@ -116,11 +118,11 @@ int run(const GemmDesc &d, int epi, void *out, int ldo, const void *res, cudaStr
   if (gx <= 0) return DG_OK;
   note_launch(s, d.name ? d.name : "gemm_simt");
   if (epi == EPI_F32)
-    gemm_simt_kernel<AT, WT, float, EPI_F32><<<grid, 256, 0, s>>>(a, (float *)out, ldo, nullptr);
+    launch_pdl(gemm_simt_kernel<AT, WT, float, EPI_F32>, grid, 256, 0, s, a, (float *)out, ldo, nullptr);
   else if (epi == EPI_ACT)
-    gemm_simt_kernel<AT, WT, AT, EPI_ACT><<<grid, 256, 0, s>>>(a, (AT *)out, ldo, nullptr);
+    launch_pdl(gemm_simt_kernel<AT, WT, AT, EPI_ACT>, grid, 256, 0, s, a, (AT *)out, ldo, nullptr);
   else
-    gemm_simt_kernel<AT, WT, float, EPI_RESID><<<grid, 256, 0, s>>>(a, (float *)out, ldo,
+    launch_pdl(gemm_simt_kernel<AT, WT, float, EPI_RESID>, grid, 256, 0, s, a, (float *)out, ldo,
                                                                     (const float *)res);
   return check_launch("gemm_simt");
 }

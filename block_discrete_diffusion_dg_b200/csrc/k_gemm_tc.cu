@@ -133,6 +133,8 @@ template <int BN_MAX, int STAGES, int B_BOX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, Params p) {
+  pdl_wait();
+  pdl_trigger();
   using C = Cfg<BN_MAX, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -401,7 +403,7 @@ int launch(const CUtensorMap &tmA, const CUtensorMap &tmB, const Params &p, int 
   const int grid = units_max < slots ? units_max : slots;
   if (grid <= 0) return DG_OK;
   note_launch(s, name);
-  k<<<grid, NUM_THREADS, C::SMEM, s>>>(tmA, tmB, tmC ? *tmC : tmA, p);
+  launch_pdl(k, grid, NUM_THREADS, C::SMEM, s, tmA, tmB, tmC ? *tmC : tmA, p);
   return check_launch(name);
 }
 

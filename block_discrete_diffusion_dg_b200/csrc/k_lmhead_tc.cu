@@ -55,6 +55,8 @@ __device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, Params p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sA = smem;
@@ -246,6 +248,8 @@ __global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restric
                                                          const int32_t *__restrict__ row_idx,
                                                          float *entropy, int32_t *argmax,
                                                          int32_t *st) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   if (n_rows_dev && r >= *n_rows_dev) return;
   EntState es;
@@ -313,11 +317,11 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
   const int units_max = ((max_rows + BM - 1) / BM) * n_vtiles;
   const int grid = units_max < num_sms() ? units_max : num_sms();
   note_launch(s, "lm_head_tc");
-  lmhead_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(tmA, tmB, p);
+  launch_pdl(lmhead_tc_kernel, grid, NUM_THREADS, SMEM_BYTES, s, tmA, tmB, p);
   rc = check_launch("lm_head_tc");
   if (rc != DG_OK) return rc;
   note_launch(s, "lm_combine");
-  lm_combine_kernel<<<max_rows, 256, 0, s>>>(p.part, p.part_am, n_vtiles, n_rows_dev, row_idx,
+  launch_pdl(lm_combine_kernel, max_rows, 256, 0, s, p.part, p.part_am, n_vtiles, n_rows_dev, row_idx,
                                              entropy, argmax, st);
   return check_launch("lm_combine");
 }

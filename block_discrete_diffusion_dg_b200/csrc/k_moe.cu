@@ -20,6 +20,8 @@ template <typename T, typename WT>
 __global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__ y,
                               const WT *__restrict__ wr, const uint8_t *__restrict__ token_live,
                               int32_t *topk_idx, float *topk_w) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float sm[];
   float *ys = sm;                        // [TPB][d]
   float *zs = sm + ROUTER_TPB * d;       // [TPB][E]
@@ -90,6 +92,8 @@ __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict
                                    const uint8_t *__restrict__ token_live,
                                    const int32_t *__restrict__ forced, int32_t *topk_idx,
                                    float *topk_w) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T_) return;
@@ -164,6 +168,8 @@ __global__ void __launch_bounds__(1024) permute_tiles_kernel(int n_assign, int E
                                                              int32_t *inv_perm, int tile_m,
                                                              GroupTile *tiles, int32_t *n_tiles,
                                                              int max_tiles, int32_t *load_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int cnt[256], off[257], running[256], toff[257];
   __shared__ int wc[32][256];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -228,11 +234,139 @@ __global__ void __launch_bounds__(1024) permute_tiles_kernel(int n_assign, int E
   }
 }
 
+// permute_tiles_kernel for at most 2048 assignments in one pass (one block of 1024 threads, two
+// assignments per thread: a0 = 64 w + lane and a1 = a0 + 32 for warp w).  Counting sort: the rank
+// of an assignment among the same-expert ones of its warp half comes from __match_any_sync, the
+// warp leaders write a per-(expert, warp) histogram, and one block-wide exclusive scan of that
+// histogram in expert-major order gives every expert's offset and every warp's first position
+// within it, so the grouping is stable in assignment order.  Same outputs as
+// permute_tiles_kernel.
+__global__ void __launch_bounds__(1024) permute_tiles_small_kernel(
+    int n_assign, int E, const int32_t *__restrict__ topk_idx, int32_t *expert_off, int32_t *perm,
+    int32_t *inv_perm, int tile_m, GroupTile *tiles, int32_t *n_tiles, int max_tiles,
+    int32_t *load_out) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int hist[256 * 32];  // [expert][warp], then its exclusive scan
+  __shared__ int wtot[32], s_total;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int H = 32 * E;
+  for (int i = tid; i < H; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int a0 = w * 64 + lane, a1 = a0 + 32;
+  int e0 = a0 < n_assign ? topk_idx[a0] : -1;
+  int e1 = a1 < n_assign ? topk_idx[a1] : -1;
+  if (e0 >= E) e0 = -1;
+  if (e1 >= E) e1 = -1;
+  const unsigned lt = (1u << lane) - 1u;
+  const unsigned m0 = __match_any_sync(0xffffffffu, e0), m1 = __match_any_sync(0xffffffffu, e1);
+  const int r0 = __popc(m0 & lt), r1 = __popc(m1 & lt);
+  if (e0 >= 0 && r0 == 0) hist[e0 * 32 + w] = __popc(m0);
+  __syncwarp();
+  const int base1 = e1 >= 0 ? hist[e1 * 32 + w] : 0;  // e1's count in the warp's first half
+  __syncwarp();
+  if (e1 >= 0 && r1 == 0) hist[e1 * 32 + w] = base1 + __popc(m1);
+  __syncthreads();
+  // exclusive scan of hist[0, H): thread t owns the run [t P, t P + P)
+  const int P = (H + blockDim.x - 1) / blockDim.x;
+  int run = 0;
+  for (int j = 0; j < P; ++j) {
+    const int i = tid * P + j;
+    if (i < H) run += hist[i];
+  }
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wtot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int v = wtot[lane];
+    int iv = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, iv, o);
+      if (lane >= o) iv += u;
+    }
+    wtot[lane] = iv - v;  // exclusive over warps
+    if (lane == 31) s_total = iv;
+  }
+  __syncthreads();
+  int acc = wtot[w] + incl - run;  // exclusive prefix of this thread's run
+  for (int j = 0; j < P; ++j) {
+    const int i = tid * P + j;
+    if (i < H) {
+      const int v = hist[i];
+      hist[i] = acc;
+      acc += v;
+    }
+  }
+  __syncthreads();
+  if (e0 >= 0) {
+    const int pos = hist[e0 * 32 + w] + r0;
+    perm[pos] = a0;
+    inv_perm[a0] = pos;
+  } else if (a0 < n_assign) {
+    inv_perm[a0] = -1;
+  }
+  if (e1 >= 0) {
+    const int pos = hist[e1 * 32 + w] + base1 + r1;
+    perm[pos] = a1;
+    inv_perm[a1] = pos;
+  } else if (a1 < n_assign) {
+    inv_perm[a1] = -1;
+  }
+  // expert offsets (hist[32 e] = the first position of expert e), counts and the tile list:
+  // warp 0, eight experts per lane (E <= 256)
+  if (w == 0) {
+    int cnt[8], nt[8], tsum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      cnt[j] = 0;
+      nt[j] = 0;
+      if (e < E) {
+        const int hi = e + 1 < E ? hist[(e + 1) * 32] : s_total;
+        cnt[j] = hi - hist[e * 32];
+        nt[j] = (cnt[j] + tile_m - 1) / tile_m;
+        tsum += nt[j];
+      }
+    }
+    int tinc = tsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, tinc, o);
+      if (lane >= o) tinc += v;
+    }
+    int tbase = tinc - tsum;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e >= E) continue;
+      expert_off[e] = hist[e * 32];
+      if (load_out) load_out[e] = cnt[j];
+      for (int i = 0; i < nt[j]; ++i) {
+        const int slot = tbase + i;
+        if (slot < max_tiles) tiles[slot] = GroupTile{e, i * tile_m};
+      }
+      tbase += nt[j];
+    }
+    if (lane == 31) {
+      expert_off[E] = s_total;
+      *n_tiles = min(tinc, max_tiles);
+    }
+  }
+}
+
 // Single block of 1024 threads; E <= 256.
 __global__ void __launch_bounds__(1024) permute_kernel(int n_assign, int E,
                                                        const int32_t *__restrict__ topk_idx,
                                                        int32_t *expert_off, int32_t *perm,
                                                        int32_t *inv_perm) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int cnt[256], off[257], running[256];
   __shared__ int wc[32][256];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -287,6 +421,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(int n_assign, int E,
 __global__ void build_tiles_kernel(int E, const int32_t *__restrict__ expert_off, int tile_m,
                                    GroupTile *tiles, int32_t *n_tiles, int max_tiles,
                                    int32_t *load_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int toff[257];
   const int tid = threadIdx.x;
   if (load_out)
@@ -314,6 +450,8 @@ __global__ void build_tiles_kernel(int E, const int32_t *__restrict__ expert_off
 __global__ void gather_rows_kernel(int d, int k, const int32_t *__restrict__ perm,
                                    const int32_t *__restrict__ expert_off, int E,
                                    const uint4 *__restrict__ y, uint4 *X) {
+  pdl_wait();
+  pdl_trigger();
   const int p = blockIdx.x;
   if (p >= expert_off[E]) return;
   const int t = perm[p] / k;
@@ -324,6 +462,8 @@ __global__ void gather_rows_kernel(int d, int k, const int32_t *__restrict__ per
 template <typename T>
 __global__ void gate_kernel(int F, const float *__restrict__ u, const int32_t *__restrict__ expert_off,
                             int E, T *a) {
+  pdl_wait();
+  pdl_trigger();
   const int p = blockIdx.x;
   if (p >= expert_off[E]) return;
   const float *ur = u + (size_t)p * 2 * F;
@@ -341,6 +481,8 @@ __global__ void combine_kernel(int d, int k, const int32_t *__restrict__ topk_id
                                const float *__restrict__ topk_w, const int32_t *__restrict__ inv_perm,
                                const float *__restrict__ Y, const float *__restrict__ res,
                                float *out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float acc = res[(size_t)t * d + c];
@@ -366,6 +508,8 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(int d, int k, float e
                                                            const float *__restrict__ res, float *out,
                                                            T *a_out, const int32_t *__restrict__ slot,
                                                            T *f_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   __shared__ int idx[32];
   __shared__ float wt[32];
@@ -382,8 +526,19 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(int d, int k, float e
     const int c = threadIdx.x + u * 256;
     if (c < d) {
       float acc = res[(size_t)t * d + c];
-      for (int j = 0; j < k; ++j)
-        if (idx[j] >= 0) acc = fmaf(wt[j], Y[(size_t)idx[j] * d + c], acc);
+      for (int j0 = 0; j0 < k; j0 += 8) {  // eight expert rows in flight, added in slot order
+        float yv[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = j0 + jj;
+          yv[jj] = (j < k && idx[j] >= 0) ? Y[(size_t)idx[j] * d + c] : 0.f;
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && idx[j] >= 0) acc = fmaf(wt[j], yv[jj], acc);
+        }
+      }
       out[(size_t)t * d + c] = acc;
       xv[u] = acc;
       ss += acc * acc;
@@ -414,11 +569,11 @@ int launch_combine_norm(int act, int T_, int d, int k, double eps, const int32_t
   if (d > 256 * 16 || k > 32) return DG_ERR_UNSUPPORTED;
   note_launch(s, "combine_norm");
   if (act == DG_F32)
-    combine_norm_kernel<float><<<T_, 256, 0, s>>>(d, k, (float)eps, topk_idx, topk_w, inv_perm,
+    launch_pdl(combine_norm_kernel<float>, T_, 256, 0, s, d, k, (float)eps, topk_idx, topk_w, inv_perm,
                                                   (const float *)Y, (const float *)res, (float *)out,
                                                   (float *)a_out, slot, (float *)f_out);
   else
-    combine_norm_kernel<bf16><<<T_, 256, 0, s>>>(d, k, (float)eps, topk_idx, topk_w, inv_perm,
+    launch_pdl(combine_norm_kernel<bf16>, T_, 256, 0, s, d, k, (float)eps, topk_idx, topk_w, inv_perm,
                                                  (const float *)Y, (const float *)res, (float *)out,
                                                  (bf16 *)a_out, slot, (bf16 *)f_out);
   return check_launch("combine_norm");
@@ -435,13 +590,13 @@ int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void 
     auto kf = router_kernel<float, float>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     note_launch(s, "router");
-    kf<<<grid, threads, smem, s>>>(T_, d, E, k, (const float *)y, (const float *)w_router,
+    launch_pdl(kf, grid, threads, smem, s, T_, d, E, k, (const float *)y, (const float *)w_router,
                                    token_live, topk_idx, topk_w);
   } else if (act == DG_BF16 && wr_type == DG_BF16) {
     auto kb = router_kernel<bf16, bf16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     note_launch(s, "router");
-    kb<<<grid, threads, smem, s>>>(T_, d, E, k, (const bf16 *)y, (const bf16 *)w_router,
+    launch_pdl(kb, grid, threads, smem, s, T_, d, E, k, (const bf16 *)y, (const bf16 *)w_router,
                                    token_live, topk_idx, topk_w);
   } else {
     return DG_ERR_UNSUPPORTED;
@@ -455,7 +610,7 @@ int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *toke
   if (T_ <= 0) return DG_OK;
   if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
   note_launch(s, "router_topk");
-  router_topk_kernel<<<(T_ + 7) / 8, 256, 0, s>>>(T_, E, k, z, n_parts, token_live, forced,
+  launch_pdl(router_topk_kernel, (T_ + 7) / 8, 256, 0, s, T_, E, k, z, n_parts, token_live, forced,
                                                   topk_idx, topk_w);
   return check_launch("router_topk");
 }
@@ -469,8 +624,12 @@ int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live
   const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced, n_parts);
   if (rc != DG_OK) return rc;
   note_launch(s, "permute_tiles");
-  permute_tiles_kernel<<<1, 1024, 0, s>>>(T_ * k, E, topk_idx, expert_off, perm, inv_perm, tile_m,
-                                          tiles, n_tiles, max_tiles, load_out);
+  if (T_ * k <= 2048)
+    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, T_ * k, E, topk_idx, expert_off, perm,
+               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
+  else
+    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, T_ * k, E, topk_idx, expert_off, perm,
+               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
   return check_launch("permute_tiles");
 }
 
@@ -478,7 +637,7 @@ int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *exper
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s) {
   if (E > 256) return DG_ERR_UNSUPPORTED;
   note_launch(s, "permute");
-  permute_kernel<<<1, 1024, 0, s>>>(T_ * k, E, topk_idx, expert_off, perm, inv_perm);
+  launch_pdl(permute_kernel, 1, 1024, 0, s, T_ * k, E, topk_idx, expert_off, perm, inv_perm);
   return check_launch("permute");
 }
 
@@ -486,7 +645,7 @@ int launch_build_tiles(int E, const int32_t *expert_off, int tile_m, GroupTile *
                        int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s) {
   if (E > 256) return DG_ERR_UNSUPPORTED;
   note_launch(s, "build_tiles");
-  build_tiles_kernel<<<1, 256, 0, s>>>(E, expert_off, tile_m, tiles, n_tiles, max_tiles, load_out);
+  launch_pdl(build_tiles_kernel, 1, 256, 0, s, E, expert_off, tile_m, tiles, n_tiles, max_tiles, load_out);
   return check_launch("build_tiles");
 }
 
@@ -494,7 +653,7 @@ int launch_gather_rows(int rows_max, int d, int k, const int32_t *perm, const in
                        int E, const void *y, void *X, cudaStream_t s) {
   if (rows_max <= 0) return DG_OK;
   note_launch(s, "gather_rows");
-  gather_rows_kernel<<<rows_max, 128, 0, s>>>(d, k, perm, expert_off, E, (const uint4 *)y, (uint4 *)X);
+  launch_pdl(gather_rows_kernel, rows_max, 128, 0, s, d, k, perm, expert_off, E, (const uint4 *)y, (uint4 *)X);
   return check_launch("gather_rows");
 }
 
@@ -503,9 +662,9 @@ int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *exp
   if (rows_max <= 0) return DG_OK;
   note_launch(s, "gate");
   if (act == DG_F32)
-    gate_kernel<float><<<rows_max, 128, 0, s>>>(F, u, expert_off, E, (float *)a);
+    launch_pdl(gate_kernel<float>, rows_max, 128, 0, s, F, u, expert_off, E, (float *)a);
   else
-    gate_kernel<bf16><<<rows_max, 128, 0, s>>>(F, u, expert_off, E, (bf16 *)a);
+    launch_pdl(gate_kernel<bf16>, rows_max, 128, 0, s, F, u, expert_off, E, (bf16 *)a);
   return check_launch("gate");
 }
 
@@ -515,7 +674,7 @@ int launch_combine(int act, int T_, int d, int k, const int32_t *topk_idx, const
   if (T_ <= 0) return DG_OK;
   (void)act;
   note_launch(s, "combine");
-  combine_kernel<<<T_, 256, 0, s>>>(d, k, topk_idx, topk_w, inv_perm, (const float *)Y,
+  launch_pdl(combine_kernel, T_, 256, 0, s, d, k, topk_idx, topk_w, inv_perm, (const float *)Y,
                                     (const float *)res, (float *)out);
   return check_launch("combine");
 }

@@ -13,6 +13,8 @@ namespace dg {
 // cs[(b*n + i)*hd + 2j] = cos, [.. + 2j + 1] = sin
 __global__ void rope_table_kernel(int n, int hd, double theta, const int32_t *__restrict__ cache_len,
                                   float *cs) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const int half = hd / 2;
   const int total = n * half;
@@ -36,6 +38,8 @@ __global__ void qkv_split_kernel(int n, int Hq, int Hkv, int hd, const float *__
                                  int n_parts, size_t part_stride, const float *__restrict__ cs,
                                  T *q, T *k_new, T *v_new, T *k_cache, T *v_cache,
                                  const int32_t *__restrict__ cache_len, int cap, int32_t *st) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float qkv_row[];
   const int row = blockIdx.x;  // b*n + i
   const int b = row / n, i = row % n;
@@ -86,6 +90,8 @@ __global__ void qkv_split_kernel(int n, int Hq, int Hkv, int hd, const float *__
 }
 
 __global__ void add_cache_len_kernel(int batch, int n, int cap, int32_t *cache_len) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < batch && cache_len[b] + n <= cap) cache_len[b] += n;
 }
@@ -95,7 +101,7 @@ int launch_rope_table(int batch, int n, int hd, double theta, const int32_t *cac
   note_launch(s, "rope_table");
   const int total = n * (hd / 2);
   dim3 grid((total + 255) / 256, batch);
-  rope_table_kernel<<<grid, 256, 0, s>>>(n, hd, theta, cache_len, cs);
+  launch_pdl(rope_table_kernel, grid, 256, 0, s, n, hd, theta, cache_len, cs);
   return check_launch("rope_table");
 }
 
@@ -109,12 +115,12 @@ int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const f
   const size_t stride = (size_t)batch * n * width;
   if (smem > 48 * 1024) return DG_ERR_UNSUPPORTED;
   if (act == DG_F32)
-    qkv_split_kernel<float><<<batch * n, 256, smem, s>>>(n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
+    launch_pdl(qkv_split_kernel<float>, batch * n, 256, smem, s, n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
                                                          (float *)q, (float *)k_new,
                                                          (float *)v_new, (float *)k_cache,
                                                          (float *)v_cache, cache_len, cap, st);
   else
-    qkv_split_kernel<bf16><<<batch * n, 256, smem, s>>>(n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
+    launch_pdl(qkv_split_kernel<bf16>, batch * n, 256, smem, s, n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
                                                         (bf16 *)q, (bf16 *)k_new, (bf16 *)v_new,
                                                         (bf16 *)k_cache, (bf16 *)v_cache,
                                                         cache_len, cap, st);
@@ -123,7 +129,7 @@ int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const f
 
 int launch_add_cache_len(int batch, int n, int cap, int32_t *cache_len, cudaStream_t s) {
   note_launch(s, "add_cache_len");
-  add_cache_len_kernel<<<(batch + 127) / 128, 128, 0, s>>>(batch, n, cap, cache_len);
+  launch_pdl(add_cache_len_kernel, (batch + 127) / 128, 128, 0, s, batch, n, cap, cache_len);
   return check_launch("add_cache_len");
 }
 

@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t *__restri
                                                          const T *__restrict__ emb, int d,
                                                          int vocab, float eps, float *x_out,
                                                          T *a_out, int32_t *st) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   const int row = blockIdx.x;
   int id = (masked && masked[row]) ? vocab : tokens[row];
@@ -47,6 +49,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float *__restrict__ 
                                                       const int32_t *__restrict__ row_idx,
                                                       const int32_t *__restrict__ n_rows_dev,
                                                       int d, float eps, T *out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   const int r = blockIdx.x;
   if (n_rows_dev && r >= *n_rows_dev) return;
@@ -71,6 +75,8 @@ __global__ void __launch_bounds__(256) resid_norm_kernel(const float *__restrict
                                                          int n_parts, size_t part_stride,
                                                          const float *__restrict__ res, int d,
                                                          float eps, float *h_out, T *out) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float hrow[];
   __shared__ float red[8];
   const int r = blockIdx.x;
@@ -101,6 +107,8 @@ __global__ void __launch_bounds__(1024) compact_rows_kernel(int batch, int canva
                                                             const int32_t *__restrict__ done,
                                                             int32_t *row_idx, int32_t *n_rows,
                                                             uint8_t *token_live) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int warp_tot[32];
   __shared__ int base;
   if (threadIdx.x == 0) base = 0;
@@ -145,6 +153,8 @@ __global__ void __launch_bounds__(256) prologue_kernel(
     int n, int hd, double theta, const int32_t *__restrict__ cache_len, float *cs, int batch,
     int canvas, const int32_t *__restrict__ done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
     uint8_t *token_live) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   __shared__ int warp_tot[8];
   __shared__ int base;
@@ -221,6 +231,8 @@ __global__ void __launch_bounds__(256) prologue_kernel(
 // e4m3 -> bf16, exact (every e4m3 value is a bf16 value); 16 codes per thread step.  The
 // per-output-channel scales stay separate and are applied to the fp32 accumulators.
 __global__ void dequant_e4m3_kernel(const uint4 *__restrict__ src, size_t n16, uint4 *dst) {
+  pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16;
        i += (size_t)gridDim.x * blockDim.x) {
     const uint4 v = src[i];
@@ -245,7 +257,7 @@ int launch_dequant_e4m3(const void *src, size_t n, void *dst, cudaStream_t s) {
   size_t blocks = (n16 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   note_launch(s, "dequant_e4m3");
-  dequant_e4m3_kernel<<<(unsigned)blocks, 256, 0, s>>>((const uint4 *)src, n16, (uint4 *)dst);
+  launch_pdl(dequant_e4m3_kernel, (unsigned)blocks, 256, 0, s, (const uint4 *)src, n16, (uint4 *)dst);
   return check_launch("dequant_e4m3");
 }
 
@@ -259,13 +271,11 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
   const int grid = rows + rope_blocks + (row_idx ? 1 : 0);
   note_launch(s, "prologue");
   if (act == DG_F32)
-    prologue_kernel<float><<<grid, 256, 0, s>>>(
-        tokens, masked, (const float *)emb, rows, d, vocab, (float)eps, (float *)x_out,
+    launch_pdl(prologue_kernel<float>, grid, 256, 0, s, tokens, masked, (const float *)emb, rows, d, vocab, (float)eps, (float *)x_out,
         (float *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
         n_rows, slot, token_live);
   else
-    prologue_kernel<bf16><<<grid, 256, 0, s>>>(
-        tokens, masked, (const bf16 *)emb, rows, d, vocab, (float)eps, (float *)x_out,
+    launch_pdl(prologue_kernel<bf16>, grid, 256, 0, s, tokens, masked, (const bf16 *)emb, rows, d, vocab, (float)eps, (float *)x_out,
         (bf16 *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
         n_rows, slot, token_live);
   return check_launch("prologue");
@@ -277,10 +287,10 @@ int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, con
   if (rows <= 0) return DG_OK;
   note_launch(s, "embed_norm");
   if (act == DG_F32)
-    embed_norm_kernel<float><<<rows, 256, 0, s>>>(tokens, masked, (const float *)emb, d, vocab,
+    launch_pdl(embed_norm_kernel<float>, rows, 256, 0, s, tokens, masked, (const float *)emb, d, vocab,
                                                   (float)eps, (float *)x_out, (float *)a_out, st);
   else
-    embed_norm_kernel<bf16><<<rows, 256, 0, s>>>(tokens, masked, (const bf16 *)emb, d, vocab,
+    launch_pdl(embed_norm_kernel<bf16>, rows, 256, 0, s, tokens, masked, (const bf16 *)emb, d, vocab,
                                                  (float)eps, (float *)x_out, (bf16 *)a_out, st);
   return check_launch("embed_norm");
 }
@@ -290,10 +300,10 @@ int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_
   if (max_rows <= 0) return DG_OK;
   note_launch(s, "rmsnorm");
   if (act == DG_F32)
-    rmsnorm_kernel<float><<<max_rows, 256, 0, s>>>((const float *)in, row_idx, n_rows_dev, d,
+    launch_pdl(rmsnorm_kernel<float>, max_rows, 256, 0, s, (const float *)in, row_idx, n_rows_dev, d,
                                                    (float)eps, (float *)out);
   else
-    rmsnorm_kernel<bf16><<<max_rows, 256, 0, s>>>((const float *)in, row_idx, n_rows_dev, d,
+    launch_pdl(rmsnorm_kernel<bf16>, max_rows, 256, 0, s, (const float *)in, row_idx, n_rows_dev, d,
                                                   (float)eps, (bf16 *)out);
   return check_launch("rmsnorm");
 }
@@ -306,10 +316,10 @@ int launch_resid_norm(int act, const float *part, int n_parts, const float *res,
   note_launch(s, "resid_norm");
   const size_t stride = (size_t)rows * d;
   if (act == DG_F32)
-    resid_norm_kernel<float><<<rows, 256, smem, s>>>(part, n_parts, stride, res, d, (float)eps,
+    launch_pdl(resid_norm_kernel<float>, rows, 256, smem, s, part, n_parts, stride, res, d, (float)eps,
                                                      h_out, (float *)out);
   else
-    resid_norm_kernel<bf16><<<rows, 256, smem, s>>>(part, n_parts, stride, res, d, (float)eps,
+    launch_pdl(resid_norm_kernel<bf16>, rows, 256, smem, s, part, n_parts, stride, res, d, (float)eps,
                                                     h_out, (bf16 *)out);
   return check_launch("resid_norm");
 }
@@ -317,7 +327,7 @@ int launch_resid_norm(int act, const float *part, int n_parts, const float *res,
 int launch_compact_rows(int batch, int canvas, const uint8_t *masked, const int32_t *done,
                         int32_t *row_idx, int32_t *n_rows, uint8_t *token_live, cudaStream_t s) {
   note_launch(s, "compact_rows");
-  compact_rows_kernel<<<1, 1024, 0, s>>>(batch, canvas, masked, done, row_idx, n_rows, token_live);
+  launch_pdl(compact_rows_kernel, 1, 1024, 0, s, batch, canvas, masked, done, row_idx, n_rows, token_live);
   return check_launch("compact_rows");
 }
 
