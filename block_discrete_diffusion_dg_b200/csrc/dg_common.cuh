@@ -59,6 +59,43 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
   return t;
 }
 
+// p[0] + p[stride] + ... + p[(n - 1) stride], component-wise, added in slice order
+// (deterministic); the loads of up to eight slices are issued before their adds.
+__device__ __forceinline__ float4 sum_parts4(const float4 *__restrict__ p, int n, size_t stride) {
+  float4 acc = p[0];
+  for (int s0 = 1; s0 < n; s0 += 8) {
+    float4 t[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (s0 + j < n) t[j] = p[(size_t)(s0 + j) * stride];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (s0 + j < n) {
+        acc.x += t[j].x;
+        acc.y += t[j].y;
+        acc.z += t[j].z;
+        acc.w += t[j].w;
+      }
+  }
+  return acc;
+}
+
+// Four consecutive values to `dst` in the activation type (one 16- or 8-byte store).
+template <typename T>
+__device__ __forceinline__ void store4(T *dst, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float *dst, float a, float b, float c, float d) {
+  *reinterpret_cast<float4 *>(dst) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16 *dst, float a, float b, float c, float d) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 v;
+  v.x = *reinterpret_cast<const uint32_t *>(&lo);
+  v.y = *reinterpret_cast<const uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = v;
+}
+
 // acc[j] = p[e_j] + p[stride + e_j] + ... + p[(n - 1) stride + e_j] for the 8 elements
 // e_j = e0 + j * step (those < count; the others get 0), added in slice order (deterministic).  The
 // slice loop is outermost so the 8 loads of a slice are in flight together.

@@ -336,19 +336,39 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
   if (w >= B * Hq * n) return;
   const int i = w % n, h = (w / n) % Hq, b = w / (n * Hq);
   if (done && done[b]) return;
+  // the (m, l) of up to eight splits and their O slices are loaded together, then combined in
+  // split order
+  const size_t sstride = (size_t)B * Hq * n, r0 = ((size_t)b * Hq + h) * n + i;
   float m = -INFINITY;
-  for (int s = 0; s < splits; ++s) m = fmaxf(m, part_ml[(((size_t)s * B + b) * Hq + h) * n + i].x);
+  for (int s0 = 0; s0 < splits; s0 += 8) {
+    float mv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mv[j] = s0 + j < splits ? part_ml[(s0 + j) * sstride + r0].x : -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, mv[j]);
+  }
   const float base = m == -INFINITY ? 0.f : m;
   float l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < splits; ++s) {
-    const size_t r = (((size_t)s * B + b) * Hq + h) * n + i;
-    const float2 ml = part_ml[r];
-    const float c = exp2f(ml.x - base);
-    l += ml.y * c;
-    if (lane * 4 < HD) {
-      const float4 v = reinterpret_cast<const float4 *>(part_o + r * HD)[lane];
-      acc.x += v.x * c; acc.y += v.y * c; acc.z += v.z * c; acc.w += v.w * c;
+  for (int s0 = 0; s0 < splits; s0 += 8) {
+    float2 ml[8];
+    float4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (s0 + j < splits) {
+        const size_t r = (s0 + j) * sstride + r0;
+        ml[j] = part_ml[r];
+        if (lane * 4 < HD) v[j] = reinterpret_cast<const float4 *>(part_o + r * HD)[lane];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (s0 + j >= splits) continue;
+      const float c = exp2f(ml[j].x - base);
+      l += ml[j].y * c;
+      if (lane * 4 < HD) {
+        acc.x += v[j].x * c; acc.y += v[j].y * c; acc.z += v[j].z * c; acc.w += v[j].w * c;
+      }
     }
   }
   const float il = l > 0.f ? 1.f / l : 0.f;

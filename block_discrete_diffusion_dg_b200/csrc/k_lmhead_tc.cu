@@ -254,12 +254,25 @@ __global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restric
   if (n_rows_dev && r >= *n_rows_dev) return;
   EntState es;
   es.init();
-  for (int t = threadIdx.x; t < n_vtiles; t += blockDim.x) {
-    const float4 v = part[(size_t)r * n_vtiles + t];
-    EntState o;
-    o.m = v.x; o.s = v.y; o.u = v.z; o.av = v.w;
-    o.am = part_am[(size_t)r * n_vtiles + t];
-    es.merge(o);
+  for (int t0 = threadIdx.x; t0 < n_vtiles; t0 += 4 * blockDim.x) {  // four tiles in flight
+    float4 v[4];
+    int a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + j * blockDim.x;
+      if (t < n_vtiles) {
+        v[j] = part[(size_t)r * n_vtiles + t];
+        a[j] = part_am[(size_t)r * n_vtiles + t];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (t0 + j * (int)blockDim.x >= n_vtiles) continue;
+      EntState o;
+      o.m = v[j].x; o.s = v[j].y; o.u = v[j].z; o.av = v[j].w;
+      o.am = a[j];
+      es.merge(o);
+    }
   }
   __shared__ EntState red[8];
   es = es.warp_reduce();

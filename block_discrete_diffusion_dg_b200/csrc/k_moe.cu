@@ -559,6 +559,60 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(int d, int k, float e
   }
 }
 
+// combine_norm_kernel with one float4 per thread (blockDim = d / 4 <= 1024); same arithmetic in
+// the same order, with the eight expert rows of a thread loaded ahead of the FMAs.
+template <typename T>
+__global__ void __launch_bounds__(1024) combine_norm4_kernel(
+    int d4, int k, float eps, const int32_t *__restrict__ topk_idx,
+    const float *__restrict__ topk_w, const int32_t *__restrict__ inv_perm,
+    const float4 *__restrict__ Y, const float4 *__restrict__ res, float4 *out, T *a_out,
+    const int32_t *__restrict__ slot, T *f_out) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float red[32];
+  __shared__ int idx[32];
+  __shared__ float wt[32];
+  const int t = blockIdx.x, c = threadIdx.x;
+  if (threadIdx.x < k) {
+    idx[threadIdx.x] = topk_idx[t * k + threadIdx.x] >= 0 ? inv_perm[t * k + threadIdx.x] : -1;
+    wt[threadIdx.x] = topk_w[t * k + threadIdx.x];
+  }
+  __syncthreads();
+  float4 acc = res[(size_t)t * d4 + c];
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    float4 yv[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = j0 + jj;
+      if (j < k && idx[j] >= 0) yv[jj] = Y[(size_t)idx[j] * d4 + c];
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = j0 + jj;
+      if (j < k && idx[j] >= 0) {
+        const float w = wt[j];
+        acc.x = fmaf(w, yv[jj].x, acc.x);
+        acc.y = fmaf(w, yv[jj].y, acc.y);
+        acc.z = fmaf(w, yv[jj].z, acc.z);
+        acc.w = fmaf(w, yv[jj].w, acc.w);
+      }
+    }
+  }
+  out[(size_t)t * d4 + c] = acc;
+  const int sl = slot ? slot[t] : -1;
+  if (!a_out && sl < 0) return;  // uniform in the block
+  float ss = acc.x * acc.x;
+  ss += acc.y * acc.y;
+  ss += acc.z * acc.z;
+  ss += acc.w * acc.w;
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)(4 * d4) + eps);
+  if (a_out) store4<T>(a_out + ((size_t)t * d4 + c) * 4, acc.x * inv, acc.y * inv, acc.z * inv,
+                       acc.w * inv);
+  if (sl >= 0) store4<T>(f_out + ((size_t)sl * d4 + c) * 4, acc.x * inv, acc.y * inv, acc.z * inv,
+                         acc.w * inv);
+}
+
 }  // namespace
 
 int launch_combine_norm(int act, int T_, int d, int k, double eps, const int32_t *topk_idx,
@@ -568,6 +622,17 @@ int launch_combine_norm(int act, int T_, int d, int k, double eps, const int32_t
   if (T_ <= 0) return DG_OK;
   if (d > 256 * 16 || k > 32) return DG_ERR_UNSUPPORTED;
   note_launch(s, "combine_norm");
+  if (d % 4 == 0 && d / 4 <= 1024 && d / 4 >= 32) {
+    if (act == DG_F32)
+      launch_pdl(combine_norm4_kernel<float>, T_, d / 4, 0, s, d / 4, k, (float)eps, topk_idx,
+                 topk_w, inv_perm, (const float4 *)Y, (const float4 *)res, (float4 *)out,
+                 (float *)a_out, slot, (float *)f_out);
+    else
+      launch_pdl(combine_norm4_kernel<bf16>, T_, d / 4, 0, s, d / 4, k, (float)eps, topk_idx,
+                 topk_w, inv_perm, (const float4 *)Y, (const float4 *)res, (float4 *)out,
+                 (bf16 *)a_out, slot, (bf16 *)f_out);
+    return check_launch("combine_norm");
+  }
   if (act == DG_F32)
     launch_pdl(combine_norm_kernel<float>, T_, 256, 0, s, d, k, (float)eps, topk_idx, topk_w, inv_perm,
                                                   (const float *)Y, (const float *)res, (float *)out,

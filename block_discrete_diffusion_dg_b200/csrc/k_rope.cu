@@ -89,6 +89,60 @@ __global__ void qkv_split_kernel(int n, int Hq, int Hkv, int hd, const float *__
   }
 }
 
+// qkv_split_kernel with one float4 per thread (blockDim = width / 4 <= 1024): the summed row is
+// staged in shared memory, then each thread rotates and stores its four consecutive values.
+template <typename T>
+__global__ void __launch_bounds__(1024) qkv_split4_kernel(
+    int n, int Hq, int Hkv, int hd, const float4 *__restrict__ qkv, int n_parts,
+    size_t part_stride4, const float *__restrict__ cs, T *q, T *k_new, T *v_new, T *k_cache,
+    T *v_cache, const int32_t *__restrict__ cache_len, int cap, int32_t *st) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ float4 qkv_row4[];
+  const int row = blockIdx.x;  // b*n + i
+  const int b = row / n, i = row % n;
+  const int half = hd / 2;
+  const int width4 = (Hq + 2 * Hkv) * hd / 4;
+  const int t = threadIdx.x;
+  qkv_row4[t] = sum_parts4(qkv + (size_t)row * width4 + t, n_parts, part_stride4);
+  int crow = -1;
+  if (k_cache) {
+    if (cache_len[b] + n > cap) {
+      if (t == 0) set_status(st, DG_ERR_CAPACITY);
+    } else {
+      crow = cache_len[b] + i;
+    }
+  }
+  __syncthreads();
+  const float *src = reinterpret_cast<const float *>(qkv_row4);
+  const float *c = cs + (size_t)row * hd;
+  const int e0 = 4 * t, head = e0 / hd, dd0 = e0 % hd;
+  float v[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int dd = dd0 + u;
+    v[u] = src[e0 + u];
+    if (head < Hq + Hkv) {  // rotate q and k
+      const int j = dd % half;
+      const float co = c[2 * j], si = c[2 * j + 1];
+      const float x1 = src[head * hd + j], x2 = src[head * hd + j + half];
+      v[u] = (dd < half) ? (x1 * co - x2 * si) : (x2 * co + x1 * si);
+    }
+  }
+  if (head < Hq) {
+    store4<T>(q + (size_t)row * Hq * hd + e0, v[0], v[1], v[2], v[3]);
+  } else {
+    const bool is_k = head < Hq + Hkv;
+    const int g = is_k ? head - Hq : head - Hq - Hkv;
+    T *dst = is_k ? k_new : v_new;
+    store4<T>(dst + (((size_t)b * Hkv + g) * n + i) * hd + dd0, v[0], v[1], v[2], v[3]);
+    if (crow >= 0) {
+      T *cd = is_k ? k_cache : v_cache;
+      store4<T>(cd + (((size_t)b * Hkv + g) * cap + crow) * hd + dd0, v[0], v[1], v[2], v[3]);
+    }
+  }
+}
+
 __global__ void add_cache_len_kernel(int batch, int n, int cap, int32_t *cache_len) {
   pdl_wait();
   pdl_trigger();
@@ -114,6 +168,17 @@ int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const f
   const size_t smem = (size_t)width * sizeof(float);
   const size_t stride = (size_t)batch * n * width;
   if (smem > 48 * 1024) return DG_ERR_UNSUPPORTED;
+  if (width % 4 == 0 && width / 4 <= 1024 && width / 4 >= 32 && hd % 4 == 0) {
+    if (act == DG_F32)
+      launch_pdl(qkv_split4_kernel<float>, batch * n, width / 4, smem, s, n, Hq, Hkv, hd,
+                 (const float4 *)qkv, n_parts, stride / 4, cs, (float *)q, (float *)k_new,
+                 (float *)v_new, (float *)k_cache, (float *)v_cache, cache_len, cap, st);
+    else
+      launch_pdl(qkv_split4_kernel<bf16>, batch * n, width / 4, smem, s, n, Hq, Hkv, hd,
+                 (const float4 *)qkv, n_parts, stride / 4, cs, (bf16 *)q, (bf16 *)k_new,
+                 (bf16 *)v_new, (bf16 *)k_cache, (bf16 *)v_cache, cache_len, cap, st);
+    return check_launch("qkv_split");
+  }
   if (act == DG_F32)
     launch_pdl(qkv_split_kernel<float>, batch * n, 256, smem, s, n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
                                                          (float *)q, (float *)k_new,

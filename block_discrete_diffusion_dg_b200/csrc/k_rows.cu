@@ -101,6 +101,31 @@ __global__ void __launch_bounds__(256) resid_norm_kernel(const float *__restrict
   for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f<T>(hrow[j] * inv);
 }
 
+// resid_norm_kernel with one float4 per thread (blockDim = d / 4 <= 1024): the slices of a thread's
+// four elements are loaded together, then summed in slice order as above.
+template <typename T>
+__global__ void __launch_bounds__(1024) resid_norm4_kernel(const float4 *__restrict__ part,
+                                                          int n_parts, size_t stride4,
+                                                          const float4 *__restrict__ res, int d4,
+                                                          float eps, float4 *h_out, T *out) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float red[32];
+  const int r = blockIdx.x, j = threadIdx.x;
+  const size_t o = (size_t)r * d4 + j;
+  const float4 a = sum_parts4(part + o, n_parts, stride4);
+  const float4 x = res[o];
+  const float4 h = make_float4(x.x + a.x, x.y + a.y, x.z + a.z, x.w + a.w);
+  h_out[o] = h;
+  float ss = h.x * h.x;
+  ss += h.y * h.y;
+  ss += h.z * h.z;
+  ss += h.w * h.w;
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)(4 * d4) + eps);
+  store4<T>(out + o * 4, h.x * inv, h.y * inv, h.z * inv, h.w * inv);
+}
+
 // One block of 1024 threads scans all B*C positions in chunks (B*C <= 65536).
 __global__ void __launch_bounds__(1024) compact_rows_kernel(int batch, int canvas,
                                                             const uint8_t *__restrict__ masked,
@@ -167,6 +192,44 @@ __global__ void __launch_bounds__(256) prologue_kernel(
       id = vocab;
     }
     const T *src = emb + (size_t)id * d;
+    if (sizeof(T) == 2 && d % 8 == 0 && d / 8 <= 4 * (int)blockDim.x) {
+      // bf16 rows: eight values per 16-byte load, one pass (the row stays in registers)
+      uint4 raw[4];
+      float ss = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j8 = threadIdx.x + u * blockDim.x;
+        if (j8 < d / 8) raw[u] = reinterpret_cast<const uint4 *>(src)[j8];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (threadIdx.x + u * (int)blockDim.x >= d / 8) continue;
+        const bf16 *h = reinterpret_cast<const bf16 *>(&raw[u]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float v = __bfloat162float(h[e]);
+          ss += v * v;
+        }
+      }
+      ss = block_sum(ss, red);
+      const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j8 = threadIdx.x + u * blockDim.x;
+        if (j8 >= d / 8) continue;
+        const bf16 *h = reinterpret_cast<const bf16 *>(&raw[u]);
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __bfloat162float(h[e]);
+        float4 *xo = reinterpret_cast<float4 *>(x_out + (size_t)row * d + 8 * j8);
+        xo[0] = make_float4(f[0], f[1], f[2], f[3]);
+        xo[1] = make_float4(f[4], f[5], f[6], f[7]);
+        store4<T>(a_out + (size_t)row * d + 8 * j8, f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv);
+        store4<T>(a_out + (size_t)row * d + 8 * j8 + 4, f[4] * inv, f[5] * inv, f[6] * inv,
+                  f[7] * inv);
+      }
+      return;
+    }
     float ss = 0.f;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
       const float v = to_f(src[j]);
@@ -315,6 +378,16 @@ int launch_resid_norm(int act, const float *part, int n_parts, const float *res,
   if (smem > 48 * 1024) return DG_ERR_UNSUPPORTED;
   note_launch(s, "resid_norm");
   const size_t stride = (size_t)rows * d;
+  if (d % 4 == 0 && d / 4 <= 1024 && d / 4 >= 32) {
+    if (act == DG_F32)
+      launch_pdl(resid_norm4_kernel<float>, rows, d / 4, 0, s, (const float4 *)part, n_parts,
+                 stride / 4, (const float4 *)res, d / 4, (float)eps, (float4 *)h_out,
+                 (float *)out);
+    else
+      launch_pdl(resid_norm4_kernel<bf16>, rows, d / 4, 0, s, (const float4 *)part, n_parts,
+                 stride / 4, (const float4 *)res, d / 4, (float)eps, (float4 *)h_out, (bf16 *)out);
+    return check_launch("resid_norm");
+  }
   if (act == DG_F32)
     launch_pdl(resid_norm_kernel<float>, rows, 256, smem, s, part, n_parts, stride, res, d, (float)eps,
                                                      h_out, (float *)out);
