@@ -361,7 +361,9 @@ def run_generate(args, world, rank):
 
 # DRAM traffic per launch of the dominant kernel from one ncu capture of the same kernel build
 # (profiles/tc_kernels_canvas_step_layer.md); set to None when the kernel changes.
-NCU_TRAFFIC = {"lm_head_tc": {"bytes": 1076431000 + 6052352,
+# DRAM bytes (read + write) per LM-head launch from one ncu capture of this workload: the mean of
+# the all-MASK (1075.189 MB + 8.956 MB) and half-committed (1076.852 MB + 5.998 MB) launches.
+NCU_TRAFFIC = {"lm_head_tc": {"bytes": (1075189000 + 8956160 + 1076852000 + 5998080) // 2,
                               "source": "profiles/tc_kernels_canvas_step_layer.md"}}
 
 
