@@ -152,4 +152,25 @@ inline void launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cuda
   cfg.numAttrs = 1;
   (void)cudaLaunchKernelEx(&cfg, k, static_cast<P>(args)...);
 }
+
+// launch_pdl for a kernel run as clusters of `cluster_x` CTAs along x.
+template <typename... P, typename... A>
+inline void launch_pdl_cluster(void (*k)(P...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t s, int cluster_x, A &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = cluster_x;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  (void)cudaLaunchKernelEx(&cfg, k, static_cast<P>(args)...);
+}
 }  // namespace dg

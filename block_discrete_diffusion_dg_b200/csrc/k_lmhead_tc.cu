@@ -44,6 +44,7 @@ struct Params {
   int32_t *part_am;         // [max_rows][n_vtiles]: first argmax in the tile
   float *logits;            // debug: [*][V] or null
   const int32_t *logits_rows;  // debug: output row of row r (null: r)
+  int only_one_tile;        // the single-CTA kernel leaves more than 128 rows to the pair kernel
   int32_t *status;
 };
 
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int m_tiles = (n_rows + BM - 1) / BM;
   const int units = m_tiles * p.n_vtiles;
   if ((int)blockIdx.x >= units) return;  // uniform across the block
+  if (p.only_one_tile && m_tiles > 1) return;  // the pair kernel handles these rows
   const int kblocks = p.K / BK;
 
   if (threadIdx.x == 0) {
@@ -239,6 +241,223 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// The same LM head on CTA pairs (clusters of 2) with the 2-SM MMA form, for more than 128 rows.
+// A unit is (256 rows, 256 vocabulary rows): CTA r of the pair holds rows 128 r .. 128 r + 127
+// and vocabulary rows 128 r .. 128 r + 127 of the unit, so each SM streams half the weight tile
+// and its stage is 32 KB (6 stages in the same 192 KB); the tensor cores of both SMs compute
+// the 256 x 256 product, each into its own TMEM (its 128 rows, all 256 vocabulary columns).
+//   warp 0 of both CTAs: TMA into its own shared memory, completion counted on the leading
+//     CTA's full barrier (the leader arms it with both CTAs' bytes);
+//   warp 1 of the leading CTA: the 2-SM MMAs; commits arrive on the stage-empty and
+//     accumulator-full barriers of both CTAs;
+//   warps 2-5 of both CTAs: the entropy epilogue of its own rows, then an arrival on the
+//     leading CTA's accumulator-empty barrier (8 arrivals per use).
+// Every wait is bounded.  On expiry a CTA records DG_ERR_TIMEOUT and unwinds; its peer then
+// times out on the barrier the aborted CTA no longer feeds.  Both reach the final cluster
+// barrier, so neither frees TMEM or leaves while the other may still use its shared memory.
+// The copies a producer issued before a stall land within microseconds, long before the ~2 s
+// limit ends the wait.
+constexpr int P_STAGES = 6;
+constexpr int PA_BYTES = BM * BK * 2;        // this CTA's 128 rows x 64 k
+constexpr int PB_BYTES = (BN / 2) * BK * 2;  // this CTA's 128 of the unit's 256 vocabulary rows
+constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * (PA_BYTES + PB_BYTES) + 256;
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, Params p) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + P_STAGES * PA_BYTES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sB + P_STAGES * PB_BYTES);
+  uint64_t *empty = full + P_STAGES;
+  uint64_t *tfull = empty + P_STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  int n_rows = p.max_rows;
+  if (p.n_rows_dev) n_rows = min(*p.n_rows_dev, p.max_rows);
+  const int m_pairs = (n_rows + 2 * BM - 1) / (2 * BM);
+  const int units = m_pairs * p.n_vtiles;
+  if (pair >= units || n_rows <= BM) return;  // uniform across the pair; <= 128 rows: 1-CTA kernel
+  const int kblocks = p.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  fence_before();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t full_lead = mapa_shared(smem_u32(&full[0]), 0);
+  const uint32_t tempty_lead = mapa_shared(smem_u32(&tempty[0]), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int armed[P_STAGES];
+      uint32_t armed_ph[P_STAGES];
+#pragma unroll
+      for (int s = 0; s < P_STAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      for (int u = pair; u < units && !*abort_flag; u += npairs) {
+        const int mp = u % m_pairs, nt = u / m_pairs;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * (PA_BYTES + PB_BYTES));
+          const uint32_t fb = full_lead + 8u * stage;
+          tma_load_2d_pair(sA + stage * PA_BYTES, &tmA, fb, kb * BK, mp * 2 * BM + rank * BM);
+          tma_load_2d_pair(sB + stage * PB_BYTES, &tmB, fb, kb * BK, nt * BN + rank * (BN / 2));
+          armed[stage] = 1;
+          armed_ph[stage] = ph;
+          if (++stage == P_STAGES) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag && rank == 0) {  // the leader's full barriers count both CTAs' copies
+        for (int s = 0; s < P_STAGES; ++s)
+          if (armed[s]) (void)mbar_wait(&full[s], armed_ph[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16(2 * BM, BN);
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      int last_stage = -1;
+      uint32_t last_ph = 0;
+      for (int u = pair; u < units && !*abort_flag; u += npairs) {
+        if (!mbar_wait(&tempty[acc], aph ^ 1)) { fail(p.status, abort_flag); break; }
+        fence_after();
+        const uint32_t d = tmem + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], ph)) { fail(p.status, abort_flag); ok = false; break; }
+          fence_after();
+          const uint64_t ad = sdesc_sw128(sA + stage * PA_BYTES);
+          const uint64_t bd = sdesc_sw128(sB + stage * PB_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          commit_pair(&empty[stage]);
+          last_stage = stage;
+          last_ph = ph;
+          if (++stage == P_STAGES) { stage = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        commit_pair(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      if (*abort_flag && last_stage >= 0)  // the MMAs issued so far finish before TMEM is freed
+        (void)mbar_wait(&empty[last_stage], last_ph);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = pair; u < units; u += npairs) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
+      const int mp = u % m_pairs, nt = u / m_pairs;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph))) {
+        fail(p.status, abort_flag);
+        break;
+      }
+      fence_after();
+      const int row = mp * 2 * BM + (int)rank * BM + q * 32 + lane;
+      const bool row_ok = row < n_rows;
+      float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
+      int am = 0x7fffffff;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float *lrow = nullptr;
+      if (p.logits && row_ok)
+        lrow = p.logits + (size_t)(p.logits_rows ? p.logits_rows[row] : row) * p.V;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nt * BN + c * 32;
+        if (col0 >= p.V) break;  // uniform in the warp
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_ld_wait(r);
+        const int nvalid = min(32, p.V - col0);
+        float cm = -INFINITY;
+        int ci = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float v = __uint_as_float(r[j]);
+          if (j < nvalid && v > cm) { cm = v; ci = j; }
+        }
+        if (cm > av) { av = cm; am = col0 + ci; }
+        const float mn = fmaxf(m, cm);
+        float cs = 0.f, cu = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j < nvalid) {
+            const float t = __uint_as_float(r[j]) - mn;
+            const float e = __expf(t);
+            cs += e;
+            cu = fmaf(e, t, cu);
+          }
+        }
+        if (s > 0.f) {
+          const float sc = __expf(m - mn);
+          uu = sc * fmaf(s, m - mn, uu);
+          s *= sc;
+        }
+        s += cs;
+        uu += cu;
+        m = mn;
+        if (lrow) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid) lrow[col0 + j] = __uint_as_float(r[j]);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_cluster(tempty_lead + 8u * acc);
+      }
+      if (row_ok) {
+        const size_t o = (size_t)row * p.n_vtiles + nt;
+        p.part[o] = make_float4(m, s, uu, av);
+        p.part_am[o] = am;
+      }
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  }
+  fence_before();
+  cluster_sync();  // no CTA frees TMEM or exits while its peer may still use its shared memory
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 // Merge the partial states of one row over all vocabulary tiles (fixed order) and store the
 // entropy and argmax at the row's source index.
 __global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restrict__ part,
@@ -325,12 +544,35 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
   p.logits = logits;
   p.logits_rows = logits_rows;
   p.status = st;
+  // The number of rows is known on the device only.  Up to 128 rows the single-CTA kernel runs;
+  // beyond, CTA pairs with the 2-SM MMA (each SM streams half of every weight tile).  When both
+  // are possible both are launched and the one that does not apply returns at once.
+  p.only_one_tile = max_rows > BM;
+  if (max_rows > BM) {
+    CUtensorMap tmB2;
+    rc = make_tmap_2d(&tmB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_lm, (uint64_t)K, (uint64_t)V,
+                      (uint64_t)K * 2, BK, BN / 2);  // each CTA loads 128 of the 256 rows
+    if (rc != DG_OK) return rc;
+    cudaFuncSetAttribute(lmhead_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)P_SMEM_BYTES);
+    const int pairs_max = ((max_rows + 2 * BM - 1) / (2 * BM)) * n_vtiles;
+    const int pairs = pairs_max < num_sms() / 2 ? pairs_max : num_sms() / 2;
+    note_launch(s, "lm_head_tc2");
+    launch_pdl_cluster(lmhead_tc2_kernel, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, tmA, tmB2,
+                       p);
+    rc = check_launch("lm_head_tc2");
+    if (rc != DG_OK) return rc;
+  }
   cudaFuncSetAttribute(lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)SMEM_BYTES);
-  const int units_max = ((max_rows + BM - 1) / BM) * n_vtiles;
-  const int grid = units_max < num_sms() ? units_max : num_sms();
-  note_launch(s, "lm_head_tc");
-  launch_pdl(lmhead_tc_kernel, grid, NUM_THREADS, SMEM_BYTES, s, tmA, tmB, p);
+  {
+    const int units_max = n_vtiles;  // one row tile: the single-CTA kernel's only case here
+    const int units_all = ((max_rows + BM - 1) / BM) * n_vtiles;
+    const int um = p.only_one_tile ? units_max : units_all;
+    const int grid = um < num_sms() ? um : num_sms();
+    note_launch(s, "lm_head_tc");
+    launch_pdl(lmhead_tc_kernel, grid, NUM_THREADS, SMEM_BYTES, s, tmA, tmB, p);
+  }
   rc = check_launch("lm_head_tc");
   if (rc != DG_OK) return rc;
   note_launch(s, "lm_combine");
