@@ -53,6 +53,79 @@ __device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
   *abort_flag = 1;
 }
 
+// Online update of one row's softmax state with 32 consecutive logits r (columns col0 ..
+// col0 + nvalid - 1 valid): m = running max, s = sum e^(z - m), u = sum e^(z - m)(z - m), and
+// av / am = the maximum and the first column holding it.  A full chunk takes the branch-free
+// path: tree maximum, first argmax from the bit mask of the columns equal to it, and four
+// partial sums, so the exponentials of different columns overlap (a per-column test inside the
+// unrolled loop made every column its own dependent block, and the epilogue took ~14 us per
+// 256-column tile instead of ~5).  A ragged chunk (the end of the vocabulary) tests each column.
+__device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, int col0, float &m,
+                                          float &s, float &u, float &av, int &am) {
+  float cm, cs, cu;
+  float mn;
+  if (nvalid == 32) {
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    float t[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+      for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+    cm = t[0];
+    if (cm > av) {
+      uint32_t bits = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) bits |= (v[j] == cm) ? (1u << j) : 0u;
+      av = cm;
+      am = col0 + __ffs(bits) - 1;
+    }
+    mn = fmaxf(m, cm);
+    float ps[4] = {0.f, 0.f, 0.f, 0.f}, pu[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float d = v[j] - mn;
+      const float e = __expf(d);
+      ps[j & 3] += e;
+      pu[j & 3] = fmaf(e, d, pu[j & 3]);
+    }
+    cs = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+    cu = (pu[0] + pu[1]) + (pu[2] + pu[3]);
+  } else {
+    cm = -INFINITY;
+    int ci = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float v = __uint_as_float(r[j]);
+      if (j < nvalid && v > cm) { cm = v; ci = j; }
+    }
+    if (cm > av) { av = cm; am = col0 + ci; }
+    mn = fmaxf(m, cm);
+    cs = 0.f;
+    cu = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j < nvalid) {
+        const float d = __uint_as_float(r[j]) - mn;
+        const float e = __expf(d);
+        cs += e;
+        cu = fmaf(e, d, cu);
+      }
+    }
+  }
+  if (s > 0.f) {
+    const float sc = __expf(m - mn);
+    u = sc * fmaf(s, m - mn, u);
+    s *= sc;
+  }
+  s += cs;
+  u += cu;
+  m = mn;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, Params p) {
@@ -189,33 +262,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tbase + c * 32, r);
         tmem_ld_wait(r);
         const int nvalid = min(32, p.V - col0);
-        float cm = -INFINITY;
-        int ci = 0;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float v = __uint_as_float(r[j]);
-          if (j < nvalid && v > cm) { cm = v; ci = j; }
-        }
-        if (cm > av) { av = cm; am = col0 + ci; }
-        const float mn = fmaxf(m, cm);
-        float cs = 0.f, cu = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < nvalid) {
-            const float t = __uint_as_float(r[j]) - mn;
-            const float e = __expf(t);
-            cs += e;
-            cu = fmaf(e, t, cu);
-          }
-        }
-        if (s > 0.f) {
-          const float sc = __expf(m - mn);
-          uu = sc * fmaf(s, m - mn, uu);
-          s *= sc;
-        }
-        s += cs;
-        uu += cu;
-        m = mn;
+        ent_chunk(r, nvalid, col0, m, s, uu, av, am);
         if (lrow) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -244,7 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // The same LM head on CTA pairs (clusters of 2) with the 2-SM MMA form, for more than 128 rows.
 // A unit is (256 rows, 256 vocabulary rows): CTA r of the pair holds rows 128 r .. 128 r + 127
 // and vocabulary rows 128 r .. 128 r + 127 of the unit, so each SM streams half the weight tile
-// and its stage is 32 KB (6 stages in the same 192 KB); the tensor cores of both SMs compute
+// and its stage is 32 KB (7 stages, 224 KB); the tensor cores of both SMs compute
 // the 256 x 256 product, each into its own TMEM (its 128 rows, all 256 vocabulary columns).
 //   warp 0 of both CTAs: TMA into its own shared memory, completion counted on the leading
 //     CTA's full barrier (the leader arms it with both CTAs' bytes);
@@ -257,10 +304,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // barrier, so neither frees TMEM or leaves while the other may still use its shared memory.
 // The copies a producer issued before a stall land within microseconds, long before the ~2 s
 // limit ends the wait.
-constexpr int P_STAGES = 6;
+constexpr int P_STAGES = 7;  // 7 x 32 KB + barriers: within the 227 KB of one CTA
 constexpr int PA_BYTES = BM * BK * 2;        // this CTA's 128 rows x 64 k
 constexpr int PB_BYTES = (BN / 2) * BK * 2;  // this CTA's 128 of the unit's 256 vocabulary rows
 constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * (PA_BYTES + PB_BYTES) + 256;
+static_assert(P_SMEM_BYTES <= 232448, "more shared memory than one CTA may have");
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -402,33 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tbase + c * 32, r);
         tmem_ld_wait(r);
         const int nvalid = min(32, p.V - col0);
-        float cm = -INFINITY;
-        int ci = 0;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float v = __uint_as_float(r[j]);
-          if (j < nvalid && v > cm) { cm = v; ci = j; }
-        }
-        if (cm > av) { av = cm; am = col0 + ci; }
-        const float mn = fmaxf(m, cm);
-        float cs = 0.f, cu = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < nvalid) {
-            const float t = __uint_as_float(r[j]) - mn;
-            const float e = __expf(t);
-            cs += e;
-            cu = fmaf(e, t, cu);
-          }
-        }
-        if (s > 0.f) {
-          const float sc = __expf(m - mn);
-          uu = sc * fmaf(s, m - mn, uu);
-          s *= sc;
-        }
-        s += cs;
-        uu += cu;
-        m = mn;
+        ent_chunk(r, nvalid, col0, m, s, uu, av, am);
         if (lrow) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)

@@ -7,6 +7,7 @@ bf16 activations within a few bf16 units in the last place of the oracle's value
 rounds once; intermediates that land on the other side of a rounding boundary add at most one
 unit each).  Integer outputs (expert ids, permutations, argmax, EB selections) bit-exact, except
 where the oracle's own decision is a near tie, which is excluded and counted."""
+import dataclasses
 import math
 
 import numpy as np
@@ -221,6 +222,45 @@ def test_logits_entropy_parity(cfg, gen):
     others = np.setdiff1d(np.arange(R_all), rows)
     assert (ent[others] == -1.0).all() and (am[others] == -1).all()
 
+
+
+@pytest.mark.parametrize("R,n_dev,vocab", [(1, None, 0), (128, None, 0), (129, None, 0),
+                                           (200, 77, 0), (256, None, 0), (300, None, 0),
+                                           (300, 129, 0), (513, 400, 0), (100, None, 3700),
+                                           (200, None, 3700), (256, 250, 3700), (300, None, 3700)])
+def test_logits_entropy_row_counts(cfg, R, n_dev, vocab):
+    """Row counts around the 128-row tile and the 256-row CTA-pair tile, with ragged tails (pair
+    tiles whose second CTA holds no live row) and a device-side count below the host maximum: up
+    to 128 live rows the single-CTA kernel does the work, beyond it the CTA-pair kernel, and the
+    one that does not apply must leave every output alone.  Vocabulary 3700 ends in a ragged
+    256-wide tile (116 valid columns), which takes the per-column path of the epilogue."""
+    c = dataclasses.replace(cfg, vocab=vocab) if vocab else cfg
+    g = torch.Generator(device="cpu")
+    g.manual_seed(1000 + R + (n_dev or 0))
+    model = synth.make_model(c, "cpu", seed=23)
+    R_all = R + 37
+    live = R if n_dev is None else n_dev
+    h = torch.randn((R_all, c.d_model), generator=g) * 0.07
+    rows = torch.randperm(R_all, generator=g).numpy()[:R].astype(np.int32)   # unsorted gather
+    dgc = B.make_config(c)
+    ent = torch.full((R_all,), -1.0, device="cuda")
+    am = torch.full((R_all,), -1, dtype=torch.int32, device="cuda")
+    lg = torch.zeros((R, c.vocab), device="cuda")
+    nd = None if n_dev is None else torch.tensor([n_dev], dtype=torch.int32, device="cuda")
+    B.dg_logits_entropy(dgc, R, nd, h.cuda(), torch.from_numpy(rows).cuda(), model["emb"].cuda(),
+                        ent, am, lg, B.alloc_workspace(dgc, 1, R, 0))
+    torch.cuda.synchronize()
+    om = oracle_model(c, model)
+    src = rows[:live]
+    H, oam, margin, z = O.lm_head_rows(c, om, h.double().numpy()[src], keep_logits=True)
+    lg, ent, am = lg.cpu().numpy()[:live], ent.cpu().numpy(), am.cpu().numpy()
+    assert np.abs(lg - z).max() <= LOGIT_TOL
+    np.testing.assert_allclose(ent[src], H, rtol=ENT_RTOL)
+    assert (am[src] == np.argmax(lg, axis=1)).all()
+    safe = margin > 2 * LOGIT_TOL
+    assert (am[src][safe] == oam[safe]).all()
+    others = np.setdiff1d(np.arange(R_all), src)
+    assert (ent[others] == -1.0).all() and (am[others] == -1).all()
 
 def _step_compare(wl, st_np, check_eb=True):
     """One dg_canvas_step vs the oracle from the same state; returns the oracle's new state."""
