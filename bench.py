@@ -362,8 +362,8 @@ def run_generate(args, world, rank):
 # DRAM traffic per launch of the dominant kernel from one ncu capture of the same kernel build
 # (profiles/tc_kernels_canvas_step_layer.md); set to None when the kernel changes.
 # DRAM bytes (read + write) per LM-head launch from one ncu capture of this workload: the mean of
-# the all-MASK (1075.189 MB + 8.956 MB) and half-committed (1076.852 MB + 5.998 MB) launches.
-NCU_TRAFFIC = {"lm_head_tc": {"bytes": (1075189000 + 8956160 + 1076852000 + 5998080) // 2,
+# the all-MASK (1075.327 MB + 8.534 MB) and half-committed (1076.766 MB + 5.687 MB) launches.
+NCU_TRAFFIC = {"lm_head_tc": {"bytes": (1075327000 + 8534016 + 1076766000 + 5686528) // 2,
                               "source": "profiles/tc_kernels_canvas_step_layer.md"}}
 
 
