@@ -32,6 +32,12 @@ outputs) and the expert outputs Y are kept in fp32.  Where the activation type
 is bf16 the oracle rounds the fp64 value to the nearest bf16 at exactly those
 tensors and leaves the others unrounded, so the oracle/GPU gap is
 accumulation-order error, not storage error.  fp32 workloads are not rounded.
+
+Weights are decoded exactly from their storage: bf16, FP8 E4M3 times a per-channel scale, or
+(for the tied embedding / LM head of the NVFP4 workload) NVFP4, FP4 E2M1 codes times an E4M3
+scale per 16 elements times one tensor scale; the model card names an NVFP4 build of the
+checkpoint but the pages do not define the format, so the oracle follows NVIDIA's published
+definition of it (see nvfp4_rows).
 """
 from __future__ import annotations
 
@@ -83,6 +89,44 @@ def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
     val = np.where(ex == 0, man / 8.0 * 2.0 ** -6, (1.0 + man / 8.0) * np.exp2(ex - 7.0))
     val = np.where((ex == 0xF) & (man == 0x7), np.nan, val)
     return sign * val
+
+
+def e2m1_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Decode FP4 E2M1 codes (the low 4 bits): 1 sign, 2 exponent (bias 1), 1 mantissa bit.
+
+    Exponent field 0 is subnormal (m/2); otherwise (1 + m/2) * 2**(e - 1).  No infinities or
+    NaNs, so the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4 and 6.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    ex = (c >> 1) & 0x3
+    man = c & 0x1
+    val = np.where(ex == 0, man / 2.0, (1.0 + man / 2.0) * np.exp2(ex - 1.0))
+    return sign * val
+
+
+def nvfp4_rows(codes: np.ndarray, scales: np.ndarray, tensor_scale: float,
+               rows: np.ndarray) -> np.ndarray:
+    """Decode rows of an NVFP4 matrix stored in k-blocks of 64 elements.
+
+    NVFP4 (NVIDIA's 4-bit floating-point format; the model card names an NVFP4 build of the
+    checkpoint): element = e2m1(code) * e4m3(block scale) * tensor_scale, one E4M3 scale per 16
+    consecutive elements of a row.  Storage: codes [K/64][R][32] bytes, element kb*64 + 2i of
+    row r in the low nibble of codes[kb, r, i] and element kb*64 + 2i + 1 in its high nibble;
+    scales [K/64][R][4], scales[kb, r, j] for elements kb*64 + 16j .. kb*64 + 16j + 15.
+    Returns fp64 [len(rows)][K].
+    """
+    rows = np.asarray(rows)
+    nk = codes.shape[0]
+    c = codes[:, rows, :]                                   # [nk][n][32]
+    lo = e2m1_to_f64(c & 0xF)
+    hi = e2m1_to_f64(c >> 4)
+    vals = np.empty(c.shape[:2] + (64,))
+    vals[..., 0::2] = lo
+    vals[..., 1::2] = hi
+    sc = e4m3_to_f64(scales[:, rows, :])                    # [nk][n][4]
+    vals = vals * np.repeat(sc, 16, axis=-1) * float(tensor_scale)
+    return vals.transpose(1, 0, 2).reshape(len(rows), nk * 64)
 
 
 def decode_weight(arr: np.ndarray, kind: str, scale: Optional[np.ndarray] = None) -> np.ndarray:
@@ -305,7 +349,12 @@ class OracleModel:
         self.cfg = cfg
         self.a = arrays
 
+    def _nvfp4(self) -> bool:
+        return getattr(self.cfg, "emb", "") == "nvfp4"
+
     def emb_rows(self, ids: np.ndarray) -> np.ndarray:
+        if self._nvfp4():
+            return nvfp4_rows(self.a["emb"], self.a["emb_scale"], self.a["emb_scale_global"], ids)
         kind = "f32" if self.cfg.act == "f32" else "bf16"
         return decode_weight(self.a["emb"][ids], kind)
 
@@ -314,7 +363,11 @@ class OracleModel:
         V = self.cfg.vocab
         for v0 in range(0, V, chunk):
             v1 = min(V, v0 + chunk)
-            yield v0, decode_weight(self.a["emb"][v0:v1], kind)
+            if self._nvfp4():
+                yield v0, nvfp4_rows(self.a["emb"], self.a["emb_scale"],
+                                     self.a["emb_scale_global"], np.arange(v0, v1))
+            else:
+                yield v0, decode_weight(self.a["emb"][v0:v1], kind)
 
     def layer(self, l: int) -> dict:
         return self.a["layers"][l]

@@ -61,6 +61,7 @@ class Cfg:
     rms_eps: float = 1e-6
     state: str = "all_mask"  # initial canvas state: "all_mask" or "half"
     prefill_ids: bool = False  # prompt given as token ids (prefilled by the append path)
+    emb: str = ""            # tied embedding / LM head storage: "" = the activation type, or "nvfp4"
 
     @property
     def mask_id(self) -> int:
@@ -87,7 +88,16 @@ CONFIGS: Dict[str, Cfg] = {
     "batch32": Cfg("batch32", 2048, 16, 8, 128, 128, 8, 768, 262144, 256, 1, "bf16",
                    "e4m3", 32, 1024, 1.0, 256, 1, 4,
                    router_std=1.0 / float(np.sqrt(2048.0))),
+    # the layer workload with the tied embedding / LM head stored in NVFP4
+    "layer_nvfp4": Cfg("layer_nvfp4", 2048, 16, 8, 128, 128, 8, 768, 262144, 256, 1, "bf16",
+                       "bf16", 1, 4096, 1.0, 256, 1, 5, emb="nvfp4"),
 }
+
+# NVFP4 storage of the embedding (see make_nvfp4_emb): k-blocks of 64 elements, 16-element
+# scale blocks, rows padded to a multiple of NVFP4_ROW_PAD
+NVFP4_KB = 64
+NVFP4_BLOCK = 16
+NVFP4_ROW_PAD = 256
 
 
 def get_config(name: str, **overrides) -> Cfg:
@@ -129,6 +139,33 @@ def _store_weight(w32: torch.Tensor, kind: str):
     return w32.to(_dtype(kind)), None
 
 
+def nvfp4_rows_padded(n_rows: int) -> int:
+    return (n_rows + NVFP4_ROW_PAD - 1) // NVFP4_ROW_PAD * NVFP4_ROW_PAD
+
+
+def make_nvfp4_emb(g, n_rows: int, d: int, std: float, device):
+    """Draw an embedding [n_rows, d] directly in NVFP4 storage (no rounding of drawn values).
+
+    Returns (codes, scales, tensor_scale):
+      codes  uint8 [d/64][Rp][32]: k-block kb, row r; byte i holds element kb*64 + 2i in its low
+             nibble and element kb*64 + 2i + 1 in its high nibble (FP4 E2M1 codes);
+      scales uint8 [d/64][Rp][4]: the FP8 E4M3 scale of elements kb*64 + 16j .. + 15 of row r;
+      tensor_scale: one fp32 value; element = e2m1(code) * e4m3(scale) * tensor_scale.
+    Rp = n_rows rounded up to 256; rows [n_rows, Rp) are zero.  Codes are uniform over all 16
+    values and scales uniform over the E4M3 codes 0x30..0x3F (0.5 .. 1.875), whose RMS products
+    are 3.391; the tensor scale brings the element RMS to std.
+    """
+    Rp = nvfp4_rows_padded(n_rows)
+    nk = d // NVFP4_KB
+    codes = torch.randint(0, 256, (nk, Rp, NVFP4_KB // 2), generator=g, device=device,
+                          dtype=torch.int32).to(torch.uint8)
+    scales = torch.randint(0x30, 0x40, (nk, Rp, NVFP4_KB // NVFP4_BLOCK), generator=g,
+                           device=device, dtype=torch.int32).to(torch.uint8)
+    codes[:, n_rows:] = 0
+    scales[:, n_rows:] = 0
+    return codes.contiguous(), scales.contiguous(), float(std / 3.391)
+
+
 def make_model(cfg: Cfg, device="cpu", seed: Optional[int] = None) -> dict:
     """Draw the tied embedding / LM head and every layer's weights.
 
@@ -141,8 +178,12 @@ def make_model(cfg: Cfg, device="cpu", seed: Optional[int] = None) -> dict:
     g.manual_seed(seed)
     d, std = cfg.d_model, cfg.weight_std
     emb_kind = "f32" if cfg.act == "f32" else "bf16"
-    model = {"emb": _normal(g, (cfg.vocab + 1, d), std, device).to(_dtype(emb_kind)),
-             "layers": []}
+    if cfg.emb == "nvfp4":
+        codes, scales, ts = make_nvfp4_emb(g, cfg.vocab + 1, d, std, device)
+        model = {"emb": codes, "emb_scale": scales, "emb_scale_global": ts, "layers": []}
+    else:
+        model = {"emb": _normal(g, (cfg.vocab + 1, d), std, device).to(_dtype(emb_kind)),
+                 "layers": []}
     for _ in range(cfg.n_layers):
         lay = {}
         lay["w_qkv"], lay["s_qkv"] = _store_weight(_normal(g, (cfg.qkv_rows, d), std, device), cfg.w)

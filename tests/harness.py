@@ -13,6 +13,9 @@ from block_discrete_diffusion_dg_b200 import binding as B
 def oracle_model(cfg, model) -> O.OracleModel:
     arr = {"emb": synth.to_numpy(model["emb"]),
            "layers": [{k: synth.to_numpy(v) for k, v in lay.items()} for lay in model["layers"]]}
+    if "emb_scale" in model:
+        arr["emb_scale"] = synth.to_numpy(model["emb_scale"])
+        arr["emb_scale_global"] = float(model["emb_scale_global"])
     return O.OracleModel(cfg, arr)
 
 

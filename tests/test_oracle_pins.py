@@ -58,6 +58,78 @@ def test_e4m3_decode_all_codes_vs_torch():
     assert got[0x38] == 1.0 and got[0xB8] == -1.0
 
 
+def test_e2m1_decode_all_codes_vs_ml_dtypes():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    codes = np.arange(16, dtype=np.uint8)
+    got = O.e2m1_to_f64(codes)
+    ref = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    np.testing.assert_array_equal(got, ref)
+    # OCP MX FP4 E2M1 values worked by hand: 0b0111 = 6, 0b0001 = 0.5 (subnormal), 0b1010 = -1
+    assert got[0x7] == 6.0 and got[0x1] == 0.5 and got[0xA] == -1.0 and got[0x8] == 0.0
+    # only the low nibble is a code
+    assert np.array_equal(O.e2m1_to_f64(codes | 0xF0), got)
+
+
+def test_nvfp4_rows_hand_built_layout():
+    """Four nonzero elements placed by hand: nibble order, k-block and 16-element scale block."""
+    d, R = 128, 3
+    codes = np.zeros((d // 64, R, 32), np.uint8)
+    scales = np.full((d // 64, R, 4), 0x38, np.uint8)      # 1.0 everywhere
+    codes[1, 2, 5] = 0x4A     # row 2, elements 64+10 (low nibble 0xA = -1), 64+11 (0x4 = 2)
+    scales[1, 2, 0] = 0x40    # row 2, elements 64..79: scale 2
+    codes[0, 0, 31] = 0x17    # row 0, elements 62 (0x7 = 6), 63 (0x1 = 0.5)
+    scales[0, 0, 3] = 0x30    # row 0, elements 48..63: scale 0.5
+    got = O.nvfp4_rows(codes, scales, 0.25, np.arange(R))
+    want = np.zeros((R, d))
+    want[2, 74], want[2, 75] = -1.0 * 2.0 * 0.25, 2.0 * 2.0 * 0.25
+    want[0, 62], want[0, 63] = 6.0 * 0.5 * 0.25, 0.5 * 0.5 * 0.25
+    np.testing.assert_array_equal(got, want)
+    # row selection and order
+    np.testing.assert_array_equal(O.nvfp4_rows(codes, scales, 0.25, np.array([2, 0])),
+                                  want[[2, 0]])
+
+
+def test_nvfp4_rows_random_vs_library_decoders():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    g = np.random.default_rng(7)
+    d, R = 256, 5
+    codes = g.integers(0, 256, (d // 64, R, 32), dtype=np.uint8)
+    scales = g.integers(0, 0x7F, (d // 64, R, 4), dtype=np.uint8)   # every finite positive E4M3
+    got = O.nvfp4_rows(codes, scales, 0.37, np.arange(R))
+    nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(d // 64, R, 64)
+    el = nib.astype(np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    sc = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    want = (el * np.repeat(sc, 16, axis=-1) * 0.37).transpose(1, 0, 2).reshape(R, d)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_nvfp4_model_matches_bf16_model_with_the_same_values():
+    """With a power-of-two tensor scale every NVFP4 element is exactly a bf16 value, so the
+    oracle's NVFP4 embedding / LM head must reproduce the bf16 model holding those values."""
+    c16 = synth.reduced("layer", vocab=300, d_model=256)
+    c4 = synth.reduced("layer", vocab=300, d_model=256, emb="nvfp4")
+    gen = torch.Generator()
+    gen.manual_seed(3)
+    codes, scales, _ = synth.make_nvfp4_emb(gen, c4.vocab + 1, c4.d_model, 0.02, "cpu")
+    codes, scales = codes.numpy(), scales.numpy()
+    assert codes.shape == (4, 512, 32) and scales.shape == (4, 512, 4)
+    assert not codes[:, 301:].any() and not scales[:, 301:].any()
+    ts = 2.0 ** -7
+    dense = O.nvfp4_rows(codes, scales, ts, np.arange(c4.vocab + 1))
+    assert np.array_equal(O.round_bf16(dense), dense)
+    bits = torch.from_numpy(dense.astype(np.float32)).to(torch.bfloat16).view(torch.int16)
+    m16 = O.OracleModel(c16, {"emb": bits.numpy().view(np.uint16), "layers": []})
+    m4 = O.OracleModel(c4, {"emb": codes, "emb_scale": scales, "emb_scale_global": ts,
+                            "layers": []})
+    ids = np.array([0, 7, 299, 300])
+    np.testing.assert_array_equal(m4.emb_rows(ids), m16.emb_rows(ids))
+    x = rng.standard_normal((6, c4.d_model))
+    a = O.lm_head_rows(c16, m16, x, keep_logits=True)
+    b = O.lm_head_rows(c4, m4, x, keep_logits=True)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
 # ----------------------------------------------------------------- layer pieces
 
 def test_rmsnorm_unit_rms_scale_invariance_and_torch():
