@@ -56,9 +56,11 @@ def step_bytes(cfg, experts_touched: float) -> dict:
     wo = L * d * cfg.n_q_heads * hd * wb
     router = L * cfg.n_experts * d * (4 if cfg.w == "f32" else 2)
     expert = (2 * cfg.d_ff * d + d * cfg.d_ff) * wb
-    lm = cfg.vocab * d * ab
+    # the tied embedding / LM head: NVFP4 is half a byte per element plus one E4M3 scale per 16
+    eb = 9.0 / 16.0 if getattr(cfg, "emb", "") == "nvfp4" else ab
+    lm = cfg.vocab * d * eb
     kv = L * cfg.batch * cfg.prompt_len * cfg.n_kv_heads * hd * 2 * ab
-    emb_rows = cfg.batch * cfg.canvas * d * ab
+    emb_rows = cfg.batch * cfg.canvas * d * eb
     return {"qkv": qkv, "o": wo, "router": router, "experts": experts_touched * expert,
             "expert_gate_up": experts_touched * 2 * cfg.d_ff * d * wb,
             "expert_down": experts_touched * d * cfg.d_ff * wb, "lm_head": lm, "kv": kv,
@@ -81,7 +83,7 @@ def step_flops(cfg, masked_rows: float) -> dict:
 
 
 STATES = {"layer": ("all_mask", "half"), "longctx": ("half",), "batch32": ("all_mask",),
-          "tiny": ("all_mask",)}
+          "tiny": ("all_mask",), "layer_nvfp4": ("all_mask", "half")}
 
 
 # ------------------------------------------------------------------------------ clocks
@@ -170,8 +172,7 @@ def oracle_sample_step(cfg, om, state_np, kc, vc, cache_len, frac_den: int = 16)
     rows = np.nonzero(state_np["masked"][0])[0]
     f = O.storage_round(O.rmsnorm(h[rows], cfg.rms_eps), cfg.act)
     vs = cfg.vocab // frac_den
-    kind = "f32" if cfg.act == "f32" else "bf16"
-    w = O.decode_weight(om.a["emb"][:vs], kind)
+    _, w = next(om.lm_head_chunks(vs))      # vocabulary rows [0, vs), decoded
     O.entropy_argmax(f @ w.T)
     t3 = time.perf_counter()
     return (t1 - t0) + frac_den * ((t2 - t1) + (t3 - t2))
@@ -194,6 +195,9 @@ def host_model(cfg, model):
     from oracle import dg_oracle as O
     arr = {"emb": synth.to_numpy(model["emb"]),
            "layers": [{k: synth.to_numpy(v) for k, v in l.items()} for l in model["layers"]]}
+    if "emb_scale" in model:
+        arr["emb_scale"] = synth.to_numpy(model["emb_scale"])
+        arr["emb_scale_global"] = float(model["emb_scale_global"])
     return O.OracleModel(cfg, arr)
 
 
@@ -274,7 +278,8 @@ def run_reference(args, world, rank):
 
 def workload_desc(cfg) -> str:
     states = " / ".join(STATES.get(cfg.name, ("all_mask",)))
-    return (f"{cfg.name}: {cfg.n_layers} decoder layer(s) {cfg.act}/{cfg.w}, d_model {cfg.d_model}, "
+    lm = ", embedding / LM head NVFP4" if getattr(cfg, "emb", "") == "nvfp4" else ""
+    return (f"{cfg.name}: {cfg.n_layers} decoder layer(s) {cfg.act}/{cfg.w}{lm}, d_model {cfg.d_model}, "
             f"{cfg.n_q_heads}q/{cfg.n_kv_heads}kv x {cfg.head_dim}, {cfg.n_experts} experts top-"
             f"{cfg.top_k} ff {cfg.d_ff}, vocab {cfg.vocab}, canvas {cfg.canvas}, prompt KV "
             f"{cfg.prompt_len}, gamma {cfg.gamma}, batch {cfg.batch}; canvas states: {states}")
@@ -514,7 +519,8 @@ def run_dg(args, world, rank, local):
                 "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "traffic": None,
                 "algorithmic_flops_per_launch": sf["attention"] / cfg.n_layers,
                 "peak_source": f"{peak_src} (cuBLAS bf16, sustained, of measured)"}
-    elif dom == "lm_head_tc" and sf["lm_head"] / (peaks["bf16_tflops_sustained"] * 1e12) > \
+    elif dom in ("lm_head_tc", "lm_head_q4") and \
+            sf["lm_head"] / (peaks["bf16_tflops_sustained"] * 1e12) > \
             lm_bytes / (peaks["hbm_gbs"] * 1e9):
         ach = sf["lm_head"] / dur / 1e12     # the batched LM head is a tensor-bound contraction
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 1),
@@ -523,7 +529,8 @@ def run_dg(args, world, rank, local):
                 "traffic": None, "algorithmic_flops_per_launch": sf["lm_head"],
                 "peak_source": f"{peak_src} (cuBLAS bf16, sustained, of measured)"}
     else:
-        dom_bytes = {"lm_head_tc": lm_bytes, "moe_gate_up_tc": sb["expert_gate_up"],
+        dom_bytes = {"lm_head_tc": lm_bytes, "lm_head_q4": lm_bytes,
+                     "moe_gate_up_tc": sb["expert_gate_up"],
                      "moe_down_tc": sb["expert_down"]}.get(dom)
         if dom_bytes:
             ach = dom_bytes / dur / 1e9

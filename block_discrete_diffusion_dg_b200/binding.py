@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED, DG_ERR_CAPACITY, DG_ERR_CUDA, \
     DG_ERR_NUMERIC, DG_ERR_TIMEOUT, DG_ERR_WORKSPACE = range(8)
-DG_F32, DG_BF16, DG_E4M3 = 0, 1, 2
+DG_F32, DG_BF16, DG_E4M3, DG_NVFP4 = 0, 1, 2, 3
 STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_UNSUPPORTED", 3: "DG_ERR_CAPACITY",
                 4: "DG_ERR_CUDA", 5: "DG_ERR_NUMERIC", 6: "DG_ERR_TIMEOUT", 7: "DG_ERR_WORKSPACE"}
 
@@ -37,7 +37,8 @@ class DgConfig(ctypes.Structure):
                 ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("d_ff", ctypes.c_int32),
                 ("vocab", ctypes.c_int32), ("canvas", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("rope_theta", ctypes.c_double), ("rms_eps", ctypes.c_double),
-                ("act_dtype", ctypes.c_int32), ("w_dtype", ctypes.c_int32)]
+                ("act_dtype", ctypes.c_int32), ("w_dtype", ctypes.c_int32),
+                ("emb_dtype", ctypes.c_int32)]
 
 
 class DgLayerWeights(ctypes.Structure):
@@ -49,7 +50,8 @@ class DgLayerWeights(ctypes.Structure):
 
 
 class DgModel(ctypes.Structure):
-    _fields_ = [("layers", ctypes.POINTER(DgLayerWeights)), ("emb", ctypes.c_void_p)]
+    _fields_ = [("layers", ctypes.POINTER(DgLayerWeights)), ("emb", ctypes.c_void_p),
+                ("emb_scale", ctypes.c_void_p), ("emb_scale_global", ctypes.c_float)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -73,6 +75,8 @@ _SIGS = {
                           _VP]),
     "dg_logits_entropy": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "dg_logits_entropy_static": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "dg_logits_entropy_nvfp4": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, ctypes.c_float, _VP,
+                                       _VP, _VP, _VP, _SZ, _VP, _VP]),
     "dg_eb_select": (_I32, [_I32, _I32, _VP, _VP, ctypes.c_double, _I32, _VP, _VP, _VP, _VP, _VP,
                             _VP, _VP, _VP]),
     "dg_kv_append": (_I32, [_PCFG, _PMODEL, _I32, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _SZ,
@@ -121,10 +125,11 @@ def _check(rc: int, what: str):
 
 def make_config(c) -> DgConfig:
     """dg_config from a workload description (``synth.Cfg`` or any object with the fields)."""
+    act = DG_F32 if c.act == "f32" else DG_BF16
+    emb = DG_NVFP4 if getattr(c, "emb", "") == "nvfp4" else act
     return DgConfig(c.d_model, c.n_q_heads, c.n_kv_heads, c.head_dim, c.n_experts, c.top_k, c.d_ff,
-                    c.vocab, c.canvas, c.n_layers, float(c.rope_theta), float(c.rms_eps),
-                    DG_F32 if c.act == "f32" else DG_BF16,
-                    {"f32": DG_F32, "bf16": DG_BF16, "e4m3": DG_E4M3}[c.w])
+                    c.vocab, c.canvas, c.n_layers, float(c.rope_theta), float(c.rms_eps), act,
+                    {"f32": DG_F32, "bf16": DG_BF16, "e4m3": DG_E4M3}[c.w], emb)
 
 
 def make_layer(lay: dict) -> DgLayerWeights:
@@ -140,8 +145,10 @@ class Model:
         self.tensors = model
         n = len(model["layers"])
         self.layer_array = (DgLayerWeights * n)(*[make_layer(l) for l in model["layers"]])
+        sc = model.get("emb_scale")
         self.struct = DgModel(ctypes.cast(self.layer_array, ctypes.POINTER(DgLayerWeights)),
-                              _p(model["emb"]))
+                              _p(model["emb"]), _p(sc) if sc is not None else None,
+                              float(model.get("emb_scale_global", 1.0)))
 
     def layer(self, l: int) -> DgLayerWeights:
         return self.layer_array[l]
@@ -235,6 +242,16 @@ def dg_logits_entropy_static(cfg, n_rows, n_rows_dev, h, row_idx, w_lm, entropy,
                                           _p(row_idx), _p(w_lm), _p(entropy), _p(argmax),
                                           _p(dev_status), _stream(stream)),
            "dg_logits_entropy_static")
+
+
+def dg_logits_entropy_nvfp4(cfg, n_rows, n_rows_dev, h, row_idx, w_codes, w_scale, w_scale_global,
+                            entropy, argmax, logits_dbg, ws, dev_status=None, stream=None):
+    w, wb = _ws(ws)
+    _check(lib().dg_logits_entropy_nvfp4(ctypes.byref(cfg), n_rows, _p(n_rows_dev), _p(h),
+                                         _p(row_idx), _p(w_codes), _p(w_scale),
+                                         float(w_scale_global), _p(entropy), _p(argmax),
+                                         _p(logits_dbg), w, wb, _p(dev_status), _stream(stream)),
+           "dg_logits_entropy_nvfp4")
 
 
 def dg_eb_select(batch, canvas, entropy, argmax, gamma, max_steps, tokens, masked, selected,

@@ -164,9 +164,29 @@ bool cfg_ok(const dg_config *c) {
     return false;
   if (c->n_layers <= 0) return false;
   if (!(c->rope_theta > 0.0) || !(c->rms_eps >= 0.0)) return false;
-  if (c->act_dtype == DG_F32) return c->w_dtype == DG_F32;
-  if (c->act_dtype == DG_BF16) return c->w_dtype == DG_BF16 || c->w_dtype == DG_E4M3;
-  return false;
+  if (c->act_dtype == DG_F32) return c->w_dtype == DG_F32 && c->emb_dtype == DG_F32;
+  if (c->act_dtype != DG_BF16 || (c->w_dtype != DG_BF16 && c->w_dtype != DG_E4M3)) return false;
+  if (c->emb_dtype == DG_NVFP4) return c->d_model % 256 == 0 && c->d_model <= 4096;
+  return c->emb_dtype == DG_BF16;
+}
+
+// The tied embedding / LM head as the calls take it.
+struct LmWeights {
+  const void *w;             // bf16 / fp32 rows, or NVFP4 codes
+  const uint8_t *scale;      // NVFP4 block scales (null otherwise)
+  float g;                   // NVFP4 tensor scale
+};
+
+LmWeights lm_weights(const dg_config &c, const dg_model *m) {
+  if (c.emb_dtype == DG_NVFP4) return LmWeights{m->emb, m->emb_scale, m->emb_scale_global};
+  return LmWeights{m->emb, nullptr, 1.0f};
+}
+
+bool lm_weights_ok(const dg_config &c, const LmWeights &lw) {
+  if (!lw.w) return false;
+  if (c.emb_dtype != DG_NVFP4) return true;
+  return lw.scale && std::isfinite(lw.g) && lw.g > 0.f && !((uintptr_t)lw.w & 15) &&
+         !((uintptr_t)lw.scale & 15);
 }
 
 bool lw_ok(const dg_config *c, const dg_layer_weights *w) {
@@ -348,18 +368,25 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
     DG_TRY(launch_gemm_simt(g2, EPI_F32, ws.at<void>(B_YE), d, nullptr, s));
   }
   return launch_combine_norm(c.act_dtype, T, d, k, c.rms_eps, topk_idx, topk_w, inv_perm,
-                             ws.at<void>(B_YE), residual, out, a_out, slot, f_out, s);
+                             ws.at<void>(B_YE), residual, out, a_out, slot, f_out, s,
+                             f_out && c.emb_dtype == DG_NVFP4);
 }
 
 // Final RMSNorm of rows row_idx[r] (r < *n_rows) of h, LM head, entropy/argmax at source rows.
 // (h == nullptr: the normalised rows are already in the B_FIN scratch rows.)
 int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_rows_dev,
-               const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
+               const void *h, const int32_t *row_idx, const LmWeights &lw, float *entropy,
                int32_t *argmax, float *logits_out, int scatter_logits, int32_t *st,
                cudaStream_t s) {
-  if (h)
+  const void *w_lm = lw.w;
+  if (h)  // an NVFP4 LM head multiplies fp16 rows
     DG_TRY(launch_rmsnorm(c.act_dtype, h, row_idx, n_rows_dev, max_rows, c.d_model, c.rms_eps,
-                          ws.at<void>(B_FIN), s));
+                          ws.at<void>(B_FIN), s, c.emb_dtype == DG_NVFP4));
+  if (c.emb_dtype == DG_NVFP4)
+    return launch_lmhead_q4(ws.at<void>(B_FIN), max_rows, n_rows_dev,
+                            static_cast<const uint8_t *>(lw.w), lw.scale, lw.g, c.vocab,
+                            c.d_model, row_idx, entropy, argmax, logits_out,
+                            scatter_logits ? row_idx : nullptr, ws.at<void>(B_PART), st, s);
   if (lmhead_tc_supported(c.act_dtype, c.d_model))
     return launch_lmhead_tc(ws.at<void>(B_FIN), max_rows, n_rows_dev, w_lm, c.vocab, c.d_model,
                             row_idx, entropy, argmax, logits_out,
@@ -540,13 +567,30 @@ int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_de
                       const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
                       int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
                       int32_t *dev_status, void *stream) {
-  if (!cfg_ok(cfg) || n_rows <= 0 || !h || !w_lm || !entropy || !argmax)
+  if (!cfg_ok(cfg) || cfg->emb_dtype == DG_NVFP4 || n_rows <= 0 || !h || !w_lm || !entropy ||
+      !argmax)
     return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, 1, n_rows, 0, ws, ws_bytes, &L));
   Ws w{(char *)ws, &L};
-  return lm_entropy(*cfg, w, n_rows, n_rows_dev, h, row_idx, w_lm, entropy, argmax, logits_dbg,
-                    0, dev_status, (cudaStream_t)stream);
+  return lm_entropy(*cfg, w, n_rows, n_rows_dev, h, row_idx, LmWeights{w_lm, nullptr, 1.0f},
+                    entropy, argmax, logits_dbg, 0, dev_status, (cudaStream_t)stream);
+}
+
+int dg_logits_entropy_nvfp4(const dg_config *cfg, int n_rows, const int32_t *n_rows_dev,
+                            const void *h, const int32_t *row_idx, const uint8_t *w_codes,
+                            const uint8_t *w_scale, float w_scale_global, float *entropy,
+                            int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
+                            int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg) || cfg->emb_dtype != DG_NVFP4 || n_rows <= 0 || !h || !entropy || !argmax)
+    return DG_ERR_INVALID_ARG;
+  const LmWeights lw{w_codes, w_scale, w_scale_global};
+  if (!lm_weights_ok(*cfg, lw)) return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, 1, n_rows, 0, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  return lm_entropy(*cfg, w, n_rows, n_rows_dev, h, row_idx, lw, entropy, argmax, logits_dbg, 0,
+                    dev_status, (cudaStream_t)stream);
 }
 
 int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
@@ -572,6 +616,8 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
   if (n_tokens > cache_cap) return DG_ERR_CAPACITY;
   for (int l = 0; l < cfg->n_layers; ++l)
     if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
+  const LmWeights emb = lm_weights(*cfg, model);
+  if (!lm_weights_ok(*cfg, emb)) return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
   Ws w{(char *)ws, &L};
@@ -583,7 +629,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
   DG_TRY(launch_prologue(c.act_dtype, tokens, nullptr, model->emb, T, d, c.vocab, c.rms_eps,
                          w.at<void>(B_X), w.at<void>(B_A), dev_status, batch, n_tokens, c.head_dim,
                          c.rope_theta, cache_len, w.at<float>(B_CS), nullptr, nullptr, nullptr,
-                         nullptr, nullptr, s));
+                         nullptr, nullptr, s, emb.scale, emb.g));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights &lw = model->layers[l];
     char *kc = (char *)k_cache + l * layer_elems * ae;
@@ -624,6 +670,8 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
   if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
   for (int l = 0; l < cfg->n_layers; ++l)
     if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
+  const LmWeights emb = lm_weights(*cfg, model);
+  if (!lm_weights_ok(*cfg, emb)) return DG_ERR_INVALID_ARG;
   const dg_config &c = *cfg;
   const int C = c.canvas, T = batch * C, d = c.d_model;
   Layout L;
@@ -639,7 +687,7 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
   DG_TRY(launch_prologue(c.act_dtype, tokens, masked, model->emb, T, d, c.vocab, c.rms_eps,
                          w.at<void>(B_X), w.at<void>(B_A), dev_status, batch, C, c.head_dim,
                          c.rope_theta, cache_len, w.at<float>(B_CS), done, rows, n_rows, slot, live,
-                         s));
+                         s, emb.scale, emb.g));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights &lw = model->layers[l];
     const char *kc = (const char *)k_cache + l * layer_elems * ae;
@@ -668,8 +716,8 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
   }
   float *ent = entropy_out ? entropy_out : w.at<float>(B_ENT);
   int32_t *am = argmax_out ? argmax_out : w.at<int32_t>(B_AM);
-  DG_TRY(lm_entropy(c, w, T, n_rows, nullptr, rows, model->emb, ent, am, logits_dbg, 1,
-                    dev_status, s));
+  DG_TRY(lm_entropy(c, w, T, n_rows, nullptr, rows, emb, ent, am, logits_dbg, 1, dev_status,
+                    s));
   return launch_eb_select(batch, C, ent, am, quant_gamma(gamma), max_steps, tokens, masked,
                           nullptr, n_masked, done, step, dev_status, s);
 }

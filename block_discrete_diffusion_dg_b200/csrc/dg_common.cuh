@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
+#include <cuda_fp4.h>
 #include <stdint.h>
 
 #include "../../include/dg.h"
@@ -25,9 +26,22 @@ __device__ __forceinline__ float to_f(fp8 v) { return float(v); }
 template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ __half from_f<__half>(float v) { return __float2half_rn(v); }
 
 // Round an fp32 value to the storage type and back (what a store/load round trip yields).
 template <typename T> __device__ __forceinline__ float round_to(float v) { return to_f(from_f<T>(v)); }
+
+// NVFP4 elements: two FP4 E2M1 codes of a byte (low nibble first) times their FP8 E4M3 block
+// scale, as fp16 (exact: the products have at most 5 significant bits and lie in [2^-10, 2688]).
+__device__ __forceinline__ __half2 nvfp4_pair_f16(uint32_t byte, __half2 scale2) {
+  const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(byte & 0xFFu), __NV_E2M1);
+  return __hmul2(*reinterpret_cast<const __half2 *>(&r), scale2);
+}
+__device__ __forceinline__ __half2 e4m3_scale_f16x2(uint32_t code) {
+  const __half_raw r = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)(code & 0xFFu), __NV_E4M3);
+  const __half h = *reinterpret_cast<const __half *>(&r);
+  return __halves2half2(h, h);
+}
 
 // ---- device status word ------------------------------------------------------------------
 // First error wins; later errors leave the word alone.
@@ -90,6 +104,14 @@ __device__ __forceinline__ void store4<float>(float *dst, float a, float b, floa
 template <>
 __device__ __forceinline__ void store4<bf16>(bf16 *dst, float a, float b, float c, float d) {
   const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 v;
+  v.x = *reinterpret_cast<const uint32_t *>(&lo);
+  v.y = *reinterpret_cast<const uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__half>(__half *dst, float a, float b, float c, float d) {
+  const __half2 lo = __floats2half2_rn(a, b), hi = __floats2half2_rn(c, d);
   uint2 v;
   v.x = *reinterpret_cast<const uint32_t *>(&lo);
   v.y = *reinterpret_cast<const uint32_t *>(&hi);

@@ -23,15 +23,19 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
                     int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
                     int n, int hd, double theta, const int32_t *cache_len, float *cs,
                     const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
-                    uint8_t *token_live, cudaStream_t s);
+                    uint8_t *token_live, cudaStream_t s, const uint8_t *emb_scale = nullptr,
+                    float emb_g = 1.0f);
+// Rows of an NVFP4 matrix of `rows` rows as stored (padded to a multiple of 256).
+inline int nvfp4_rows_pad(int rows) { return (rows + 255) / 256 * 256; }
 // e4m3 codes [n] -> bf16 [n] (n % 16 == 0), exact.
 int launch_dequant_e4m3(const void *src, size_t n, void *dst, cudaStream_t s);
 // in: fp32 rows (residual stream); out: activation type.
 // h_out = res + sum of n_parts fp32 partials [n_parts][rows][d]; out = RMSNorm(h_out).
 int launch_resid_norm(int act, const float *part, int n_parts, const float *res, int rows, int d,
                       double eps, float *h_out, void *out, cudaStream_t s);
+// f16_out: out in fp16 instead (the rows an NVFP4 LM head multiplies).
 int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
-                   int max_rows, int d, double eps, void *out, cudaStream_t s);
+                   int max_rows, int d, double eps, void *out, cudaStream_t s, int f16_out = 0);
 // live[b*C+i] = !done[b] && (masked == NULL || masked[b*C+i]); row_idx = positions with live
 // set, in order; *n_rows = their count; token_live[t] = !done[b] (may be NULL).
 int launch_compact_rows(int batch, int canvas, const uint8_t *masked, const int32_t *done,
@@ -120,11 +124,11 @@ int launch_gate(int act, int rows_max, int F, const float *u, const int32_t *exp
                 void *a, cudaStream_t s);
 // Combine and the following RMSNorm: out (fp32 residual stream) as launch_combine; then
 // RMSNorm(out_t) in the activation type to a_out[t] (if non-null) and to f_out[slot[t]] (if
-// slot non-null and slot[t] >= 0).
+// slot non-null and slot[t] >= 0; in fp16 when f_out_f16, with bf16 activations).
 int launch_combine_norm(int act, int T, int d, int k, double eps, const int32_t *topk_idx,
                         const float *topk_w, const int32_t *inv_perm, const void *Y,
                         const void *res, void *out, void *a_out, const int32_t *slot, void *f_out,
-                        cudaStream_t s);
+                        cudaStream_t s, int f_out_f16 = 0);
 // out_t = res_t + sum_j w[t][j] Y[inv_perm[t k + j]]; res, Y and out fp32.
 int launch_combine(int act, int T, int d, int k, const int32_t *topk_idx, const float *topk_w,
                    const int32_t *inv_perm, const void *Y, const void *res, void *out,
@@ -142,6 +146,13 @@ int launch_entropy_rows(const float *logits, int V, int max_rows, const int32_t 
 // Entropy/argmax of row r stored at row_idx ? row_idx[r] : r.  logits (debug, may be null):
 // row r written at logits_rows ? logits_rows[r] : r.  ws: lmhead_tc_ws_bytes(max_rows, V).
 bool lmhead_tc_supported(int act, int d);
+// The same with the weights in NVFP4 (codes and scales in the k-block-major layout of dg.h, rows
+// padded to nvfp4_rows_pad(V + 1)) and F in fp16; logits = gscale * (F (e2m1 * e4m3)^T).
+// K % 256 == 0.
+int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, const uint8_t *codes,
+                     const uint8_t *scales, float gscale, int V, int K, const int32_t *row_idx,
+                     float *entropy, int32_t *argmax, float *logits, const int32_t *logits_rows,
+                     void *ws, int32_t *st, cudaStream_t s);
 size_t lmhead_tc_ws_bytes(int max_rows, int V);
 int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,
                      int V, int K, const int32_t *row_idx, float *entropy, int32_t *argmax,

@@ -46,6 +46,10 @@ struct Params {
   const int32_t *logits_rows;  // debug: output row of row r (null: r)
   int only_one_tile;        // the single-CTA kernel leaves more than 128 rows to the pair kernel
   int32_t *status;
+  // NVFP4 weights (lmhead_q4_kernel): k-block-major codes and scales, rows padded to rows_pad
+  const uint8_t *q_codes, *q_scales;
+  int rows_pad;
+  float gscale;
 };
 
 __device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
@@ -60,14 +64,16 @@ __device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
 // partial sums, so the exponentials of different columns overlap (a per-column test inside the
 // unrolled loop made every column its own dependent block, and the epilogue took ~14 us per
 // 256-column tile instead of ~5).  A ragged chunk (the end of the vocabulary) tests each column.
+// SCALED: the logits are the accumulator values times gs (the NVFP4 tensor scale).
+template <bool SCALED = false>
 __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, int col0, float &m,
-                                          float &s, float &u, float &av, int &am) {
+                                          float &s, float &u, float &av, int &am, float gs = 1.f) {
   float cm, cs, cu;
   float mn;
   if (nvalid == 32) {
     float v[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    for (int j = 0; j < 32; ++j) v[j] = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
     float t[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
@@ -99,7 +105,7 @@ __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, i
     int ci = 0;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const float v = __uint_as_float(r[j]);
+      const float v = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
       if (j < nvalid && v > cm) { cm = v; ci = j; }
     }
     if (cm > av) { av = cm; am = col0 + ci; }
@@ -109,7 +115,7 @@ __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, i
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       if (j < nvalid) {
-        const float d = __uint_as_float(r[j]) - mn;
+        const float d = (SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j])) - mn;
         const float e = __expf(d);
         cs += e;
         cu = fmaf(e, d, cu);
@@ -480,6 +486,253 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// The LM head with NVFP4 weights, one CTA per SM, for any number of rows (units (row tile,
+// vocabulary tile), the row tile varying fastest).  The weight tile of a k-block arrives as 8 KB
+// of FP4 codes and 1 KB of E4M3 block scales (two 1-D bulk copies from the k-block-major
+// layout); converter warps expand it in shared memory into the fp16 tile the MMA reads, in the
+// 128-byte-swizzled K-major layout TMA would have written: one hardware e2m1x2 -> f16x2
+// conversion and one f16x2 multiply by the block scale per pair of weights (e2m1 * e4m3 is exact
+// in fp16).  The MMA is kind::f16 with fp16 operands, so the normalised rows come in fp16 too;
+// the tensor scale is applied to the fp32 logits in the epilogue.  (A bf16 tile would need two
+// more conversions per pair, and those run at a quarter of the FP32 rate: the converters, not
+// the tensor cores, then set the pace.)
+//   warp 0      producer: A (128 fp16 normalised rows x 64 k, TMA) and the codes and scales of
+//               256 vocabulary rows x 64 k, 4-stage ring;
+//   warp 1      TMEM owner and MMA issuer (M 128, N 256, K 16), two 256-column accumulators;
+//   warps 2-5   entropy epilogue (as lmhead_tc_kernel, logits times the tensor scale);
+//   warps 6-13  converters: thread i expands vocabulary row i of the tile into a 3-stage ring of
+//               fp16 tiles, then fences its stores for the tensor cores' (async) proxy.
+// A raw stage is free once the MMAs that read its A tile have completed and every converter
+// warp has read its codes (1 + 8 arrivals).  Every wait is bounded.
+constexpr int Q_RSTAGES = 4, Q_CSTAGES = 3, Q_CONV_WARPS = 8;
+constexpr int Q_A_BYTES = BM * BK * 2;   // 16 KB normalised rows (fp16)
+constexpr int Q_C_BYTES = BN * BK / 2;   // 8 KB FP4 codes
+constexpr int Q_S_BYTES = BN * BK / 16;  // 1 KB E4M3 scales
+constexpr int Q_B_BYTES = BN * BK * 2;   // 32 KB expanded fp16 tile
+constexpr int Q_THREADS = 192 + 32 * Q_CONV_WARPS;
+constexpr size_t Q_SMEM = 1024 + (size_t)Q_CSTAGES * Q_B_BYTES +
+                          (size_t)Q_RSTAGES * (Q_A_BYTES + Q_C_BYTES + Q_S_BYTES) + 256;
+static_assert(Q_SMEM <= 232448, "more shared memory than one CTA may have");
+static_assert(Q_CONV_WARPS * 32 == BN, "one converter thread per vocabulary row of a tile");
+
+__global__ void __launch_bounds__(Q_THREADS, 1)
+    lmhead_q4_kernel(const __grid_constant__ CUtensorMap tmA, Params p) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sB = smem;                               // [Q_CSTAGES][32 KB], 1024-aligned
+  uint8_t *sA = sB + Q_CSTAGES * Q_B_BYTES;         // [Q_RSTAGES][16 KB], 1024-aligned
+  uint8_t *sQ = sA + Q_RSTAGES * Q_A_BYTES;         // [Q_RSTAGES][8 KB]
+  uint8_t *sS = sQ + Q_RSTAGES * Q_C_BYTES;         // [Q_RSTAGES][1 KB]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sS + Q_RSTAGES * Q_S_BYTES);
+  uint64_t *empty = full + Q_RSTAGES;
+  uint64_t *cfull = empty + Q_RSTAGES;
+  uint64_t *cempty = cfull + Q_CSTAGES;
+  uint64_t *tfull = cempty + Q_CSTAGES;
+  uint64_t *tempty = tfull + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n_rows = p.max_rows;
+  if (p.n_rows_dev) n_rows = min(*p.n_rows_dev, p.max_rows);
+  const int m_tiles = (n_rows + BM - 1) / BM;
+  const int units = m_tiles * p.n_vtiles;
+  if ((int)blockIdx.x >= units) return;  // uniform across the block
+  const int kblocks = p.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Q_RSTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + Q_CONV_WARPS);
+    }
+    for (int c = 0; c < Q_CSTAGES; ++c) {
+      mbar_init(&cfull[c], Q_CONV_WARPS);
+      mbar_init(&cempty[c], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int armed[Q_RSTAGES];
+      uint32_t armed_ph[Q_RSTAGES];
+#pragma unroll
+      for (int s = 0; s < Q_RSTAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const int mt = u % m_tiles, nt = u / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
+          mbar_expect_tx(&full[stage], Q_A_BYTES + Q_C_BYTES + Q_S_BYTES);
+          tma_load_2d(sA + stage * Q_A_BYTES, &tmA, &full[stage], kb * BK, mt * BM);
+          const size_t slab = (size_t)kb * p.rows_pad + (size_t)nt * BN;
+          bulk_load(sQ + stage * Q_C_BYTES, p.q_codes + slab * (BK / 2), Q_C_BYTES, &full[stage]);
+          bulk_load(sS + stage * Q_S_BYTES, p.q_scales + slab * (BK / 16), Q_S_BYTES,
+                    &full[stage]);
+          armed[stage] = 1;
+          armed_ph[stage] = ph;
+          if (++stage == Q_RSTAGES) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) {  // let every issued copy land before the CTA's shared memory goes away
+        for (int s = 0; s < Q_RSTAGES; ++s)
+          if (armed[s]) (void)mbar_wait(&full[s], armed_ph[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(BM, BN);
+      int stage = 0, cst = 0, acc = 0;
+      uint32_t ph = 0, cph = 0, aph = 0;
+      int last_stage = -1;
+      uint32_t last_ph = 0;
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], aph ^ 1)) { fail(p.status, abort_flag); break; }
+        fence_after();
+        const uint32_t d = tmem + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], ph) || !mbar_wait(&cfull[cst], cph)) {
+            fail(p.status, abort_flag);
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint64_t ad = sdesc_sw128(sA + stage * Q_A_BYTES);
+          const uint64_t bd = sdesc_sw128(sB + cst * Q_B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          commit(&empty[stage]);
+          commit(&cempty[cst]);
+          last_stage = stage;
+          last_ph = ph;
+          if (++stage == Q_RSTAGES) { stage = 0; ph ^= 1; }
+          if (++cst == Q_CSTAGES) { cst = 0; cph ^= 1; }
+        }
+        if (!ok) break;
+        commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      if (*abort_flag && last_stage >= 0)  // the MMAs issued so far finish before TMEM is freed
+        (void)mbar_wait(&empty[last_stage], last_ph);
+    }
+  } else if (warp < 6) {
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
+      const int mt = u % m_tiles, nt = u / m_tiles;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph))) {
+        fail(p.status, abort_flag);
+        break;
+      }
+      fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const bool row_ok = row < n_rows;
+      float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
+      int am = 0x7fffffff;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float *lrow = nullptr;
+      if (p.logits && row_ok)
+        lrow = p.logits + (size_t)(p.logits_rows ? p.logits_rows[row] : row) * p.V;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nt * BN + c * 32;
+        if (col0 >= p.V) break;  // uniform in the warp
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_ld_wait(r);
+        const int nvalid = min(32, p.V - col0);
+        ent_chunk<true>(r, nvalid, col0, m, s, uu, av, am, p.gscale);
+        if (lrow) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid) lrow[col0 + j] = __uint_as_float(r[j]) * p.gscale;
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (row_ok) {
+        const size_t o = (size_t)row * p.n_vtiles + nt;
+        p.part[o] = make_float4(m, s, uu, av);
+        p.part_am[o] = am;
+      }
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  } else {
+    // converter: thread i of warps 6-13 owns vocabulary row i of the tile.  Codes word w (8
+    // codes, columns 8w .. 8w + 7 of the k-block) becomes 16-byte chunk w of the row's 128 bytes,
+    // stored at chunk position w ^ (row % 8) (the 128-byte swizzle).
+    const int row = (warp - 6) * 32 + lane;
+    int stage = 0, cst = 0;
+    uint32_t ph = 0, cph = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
+      bool ok = true;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], ph)) ||
+            !__all_sync(0xffffffffu, mbar_wait(&cempty[cst], cph ^ 1))) {
+          fail(p.status, abort_flag);
+          ok = false;
+          break;
+        }
+        const uint4 *src = reinterpret_cast<const uint4 *>(sQ + stage * Q_C_BYTES + row * 32);
+        const uint4 q0 = src[0], q1 = src[1];
+        const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sS + stage * Q_S_BYTES + row * 4);
+        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        uint8_t *dst = sB + cst * Q_B_BYTES + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const __half2 sc = e4m3_scale_f16x2(sc4 >> (8 * (c >> 1)));
+          uint32_t o[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const __half2 v = nvfp4_pair_f16(w[c] >> (8 * b), sc);
+            o[b] = *reinterpret_cast<const uint32_t *>(&v);
+          }
+          *reinterpret_cast<uint4 *>(dst + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();  // the tensor cores read these stores through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&cfull[cst]);
+          mbar_arrive(&empty[stage]);
+        }
+        if (++stage == Q_RSTAGES) { stage = 0; ph ^= 1; }
+        if (++cst == Q_CSTAGES) { cst = 0; cph ^= 1; }
+      }
+      if (!ok) break;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 // Merge the partial states of one row over all vocabulary tiles (fixed order) and store the
 // entropy and argmax at the row's source index.
 __global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restrict__ part,
@@ -531,6 +784,47 @@ __global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restric
 }
 
 }  // namespace
+
+int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, const uint8_t *codes,
+                     const uint8_t *scales, float gscale, int V, int K, const int32_t *row_idx,
+                     float *entropy, int32_t *argmax, float *logits, const int32_t *logits_rows,
+                     void *ws, int32_t *st, cudaStream_t s) {
+  if (max_rows <= 0) return DG_OK;
+  if (K % 256 != 0 || ((uintptr_t)codes & 15) || ((uintptr_t)scales & 15)) return DG_ERR_UNSUPPORTED;
+  const int n_vtiles = (V + BN - 1) / BN;
+  CUtensorMap tmA;
+  const int rows_alloc = (max_rows + BM - 1) / BM * BM;
+  int rc = make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, F, (uint64_t)K,
+                        (uint64_t)rows_alloc, (uint64_t)K * 2, BK, BM);
+  if (rc != DG_OK) return rc;
+  Params p{};
+  p.n_rows_dev = n_rows_dev;
+  p.max_rows = max_rows;
+  p.V = V;
+  p.K = K;
+  p.n_vtiles = n_vtiles;
+  p.part = reinterpret_cast<float4 *>(ws);
+  p.part_am = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(ws) +
+                                          (size_t)max_rows * n_vtiles * sizeof(float4));
+  p.logits = logits;
+  p.logits_rows = logits_rows;
+  p.status = st;
+  p.q_codes = codes;
+  p.q_scales = scales;
+  p.rows_pad = nvfp4_rows_pad(V + 1);
+  p.gscale = gscale;
+  cudaFuncSetAttribute(lmhead_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Q_SMEM);
+  const int units_all = ((max_rows + BM - 1) / BM) * n_vtiles;
+  const int grid = units_all < num_sms() ? units_all : num_sms();
+  note_launch(s, "lm_head_q4");
+  launch_pdl(lmhead_q4_kernel, grid, Q_THREADS, Q_SMEM, s, tmA, p);
+  rc = check_launch("lm_head_q4");
+  if (rc != DG_OK) return rc;
+  note_launch(s, "lm_combine");
+  launch_pdl(lm_combine_kernel, max_rows, 256, 0, s, p.part, p.part_am, n_vtiles, n_rows_dev,
+             row_idx, entropy, argmax, st);
+  return check_launch("lm_combine");
+}
 
 size_t lmhead_tc_ws_bytes(int max_rows, int V) {
   const size_t nvt = (size_t)(V + BN - 1) / BN;

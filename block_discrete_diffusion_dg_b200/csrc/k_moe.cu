@@ -561,12 +561,12 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(int d, int k, float e
 
 // combine_norm_kernel with one float4 per thread (blockDim = d / 4 <= 1024); same arithmetic in
 // the same order, with the eight expert rows of a thread loaded ahead of the FMAs.
-template <typename T>
+template <typename T, typename TF = T>
 __global__ void __launch_bounds__(1024) combine_norm4_kernel(
     int d4, int k, float eps, const int32_t *__restrict__ topk_idx,
     const float *__restrict__ topk_w, const int32_t *__restrict__ inv_perm,
     const float4 *__restrict__ Y, const float4 *__restrict__ res, float4 *out, T *a_out,
-    const int32_t *__restrict__ slot, T *f_out) {
+    const int32_t *__restrict__ slot, TF *f_out) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red[32];
@@ -609,8 +609,8 @@ __global__ void __launch_bounds__(1024) combine_norm4_kernel(
   const float inv = 1.0f / sqrtf(ss / (float)(4 * d4) + eps);
   if (a_out) store4<T>(a_out + ((size_t)t * d4 + c) * 4, acc.x * inv, acc.y * inv, acc.z * inv,
                        acc.w * inv);
-  if (sl >= 0) store4<T>(f_out + ((size_t)sl * d4 + c) * 4, acc.x * inv, acc.y * inv, acc.z * inv,
-                         acc.w * inv);
+  if (sl >= 0) store4<TF>(f_out + ((size_t)sl * d4 + c) * 4, acc.x * inv, acc.y * inv, acc.z * inv,
+                          acc.w * inv);
 }
 
 }  // namespace
@@ -618,12 +618,18 @@ __global__ void __launch_bounds__(1024) combine_norm4_kernel(
 int launch_combine_norm(int act, int T_, int d, int k, double eps, const int32_t *topk_idx,
                         const float *topk_w, const int32_t *inv_perm, const void *Y,
                         const void *res, void *out, void *a_out, const int32_t *slot, void *f_out,
-                        cudaStream_t s) {
+                        cudaStream_t s, int f_out_f16) {
   if (T_ <= 0) return DG_OK;
   if (d > 256 * 16 || k > 32) return DG_ERR_UNSUPPORTED;
+  const bool vec4 = d % 4 == 0 && d / 4 <= 1024 && d / 4 >= 32;
+  if (f_out_f16 && (act != DG_BF16 || !vec4)) return DG_ERR_UNSUPPORTED;
   note_launch(s, "combine_norm");
-  if (d % 4 == 0 && d / 4 <= 1024 && d / 4 >= 32) {
-    if (act == DG_F32)
+  if (vec4) {
+    if (f_out_f16)
+      launch_pdl(combine_norm4_kernel<bf16, __half>, T_, d / 4, 0, s, d / 4, k, (float)eps,
+                 topk_idx, topk_w, inv_perm, (const float4 *)Y, (const float4 *)res,
+                 (float4 *)out, (bf16 *)a_out, slot, (__half *)f_out);
+    else if (act == DG_F32)
       launch_pdl(combine_norm4_kernel<float>, T_, d / 4, 0, s, d / 4, k, (float)eps, topk_idx,
                  topk_w, inv_perm, (const float4 *)Y, (const float4 *)res, (float4 *)out,
                  (float *)a_out, slot, (float *)f_out);

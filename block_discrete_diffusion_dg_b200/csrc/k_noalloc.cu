@@ -61,6 +61,7 @@ extern "C" int dg_logits_entropy_static(const dg_config *cfg, int n_rows,
   if (!cfg || n_rows <= 0 || !h || !w_lm || !entropy || !argmax) return DG_ERR_INVALID_ARG;
   if (cfg->d_model <= 0 || cfg->vocab < 2) return DG_ERR_INVALID_ARG;
   if (!lmhead_tc_supported(cfg->act_dtype, cfg->d_model)) return DG_ERR_UNSUPPORTED;
+  if (cfg->emb_dtype != cfg->act_dtype) return DG_ERR_UNSUPPORTED;  // NVFP4: not here
   // requests larger than the fixed array: rejected, nothing launched
   if (n_rows > MAX_ROWS || cfg->d_model > MAX_D || cfg->vocab > MAX_VOCAB)
     return DG_ERR_WORKSPACE;

@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(256) prologue_kernel(
     int rows, int d, int vocab, float eps, float *x_out, T *a_out, int32_t *st, int rope_blocks,
     int n, int hd, double theta, const int32_t *__restrict__ cache_len, float *cs, int batch,
     int canvas, const int32_t *__restrict__ done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
-    uint8_t *token_live) {
+    uint8_t *token_live, const uint8_t *__restrict__ emb_q, const uint8_t *__restrict__ emb_s,
+    float emb_g, int emb_rows_pad) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red[8];
@@ -190,6 +191,43 @@ __global__ void __launch_bounds__(256) prologue_kernel(
     if (id < 0 || id > vocab) {
       if (threadIdx.x == 0) set_status(st, DG_ERR_INVALID_ARG);
       id = vocab;
+    }
+    if (emb_q) {
+      // NVFP4 rows (d % 256 == 0, d <= 8192): thread t decodes groups of 8 columns j8 = t + 256 u;
+      // group j8 lies in k-block j8 / 8 at byte (j8 % 8) * 4 and shares scale (j8 % 8) / 2.
+      // e2m1 * e4m3 is exact in fp16; the tensor scale is one fp32 rounding.
+      float f[4][8];
+      float ss = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j8 = threadIdx.x + u * blockDim.x;
+        if (j8 >= d / 8) continue;
+        const size_t slab = (size_t)(j8 >> 3) * emb_rows_pad + id;
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(emb_q + slab * 32 + (j8 & 7) * 4);
+        const __half2 sc = e4m3_scale_f16x2(emb_s[slab * 4 + ((j8 & 7) >> 1)]);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float2 v = __half22float2(nvfp4_pair_f16(w >> (8 * b), sc));
+          f[u][2 * b] = v.x * emb_g;
+          f[u][2 * b + 1] = v.y * emb_g;
+          ss += f[u][2 * b] * f[u][2 * b] + f[u][2 * b + 1] * f[u][2 * b + 1];
+        }
+      }
+      ss = block_sum(ss, red);
+      const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j8 = threadIdx.x + u * blockDim.x;
+        if (j8 >= d / 8) continue;
+        float4 *xo = reinterpret_cast<float4 *>(x_out + (size_t)row * d + 8 * j8);
+        xo[0] = make_float4(f[u][0], f[u][1], f[u][2], f[u][3]);
+        xo[1] = make_float4(f[u][4], f[u][5], f[u][6], f[u][7]);
+        store4<T>(a_out + (size_t)row * d + 8 * j8, f[u][0] * inv, f[u][1] * inv, f[u][2] * inv,
+                  f[u][3] * inv);
+        store4<T>(a_out + (size_t)row * d + 8 * j8 + 4, f[u][4] * inv, f[u][5] * inv,
+                  f[u][6] * inv, f[u][7] * inv);
+      }
+      return;
     }
     const T *src = emb + (size_t)id * d;
     if (sizeof(T) == 2 && d % 8 == 0 && d / 8 <= 4 * (int)blockDim.x) {
@@ -328,19 +366,22 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
                     int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
                     int n, int hd, double theta, const int32_t *cache_len, float *cs,
                     const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
-                    uint8_t *token_live, cudaStream_t s) {
+                    uint8_t *token_live, cudaStream_t s, const uint8_t *emb_scale, float emb_g) {
   if (rows <= 0) return DG_OK;
+  const uint8_t *emb_q = emb_scale ? static_cast<const uint8_t *>(emb) : nullptr;
+  const int rows_pad = nvfp4_rows_pad(vocab + 1);
+  if (emb_q && (act != DG_BF16 || d % 256 != 0 || d > 8192)) return DG_ERR_UNSUPPORTED;
   const int rope_blocks = (batch * n * (hd / 2) + 255) / 256;
   const int grid = rows + rope_blocks + (row_idx ? 1 : 0);
   note_launch(s, "prologue");
   if (act == DG_F32)
     launch_pdl(prologue_kernel<float>, grid, 256, 0, s, tokens, masked, (const float *)emb, rows, d, vocab, (float)eps, (float *)x_out,
         (float *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
-        n_rows, slot, token_live);
+        n_rows, slot, token_live, emb_q, emb_scale, emb_g, rows_pad);
   else
     launch_pdl(prologue_kernel<bf16>, grid, 256, 0, s, tokens, masked, (const bf16 *)emb, rows, d, vocab, (float)eps, (float *)x_out,
         (bf16 *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
-        n_rows, slot, token_live);
+        n_rows, slot, token_live, emb_q, emb_scale, emb_g, rows_pad);
   return check_launch("prologue");
 }
 
@@ -359,10 +400,13 @@ int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, con
 }
 
 int launch_rmsnorm(int act, const void *in, const int32_t *row_idx, const int32_t *n_rows_dev,
-                   int max_rows, int d, double eps, void *out, cudaStream_t s) {
+                   int max_rows, int d, double eps, void *out, cudaStream_t s, int f16_out) {
   if (max_rows <= 0) return DG_OK;
   note_launch(s, "rmsnorm");
-  if (act == DG_F32)
+  if (f16_out)
+    launch_pdl(rmsnorm_kernel<__half>, max_rows, 256, 0, s, (const float *)in, row_idx, n_rows_dev,
+               d, (float)eps, (__half *)out);
+  else if (act == DG_F32)
     launch_pdl(rmsnorm_kernel<float>, max_rows, 256, 0, s, (const float *)in, row_idx, n_rows_dev, d,
                                                    (float)eps, (float *)out);
   else

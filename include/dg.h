@@ -58,7 +58,16 @@ enum {
   DG_ERR_WORKSPACE = 7     /* ws_bytes smaller than dg_workspace_size()                      */
 };
 
-enum { DG_F32 = 0, DG_BF16 = 1, DG_E4M3 = 2 };
+enum { DG_F32 = 0, DG_BF16 = 1, DG_E4M3 = 2, DG_NVFP4 = 3 };
+
+/* NVFP4 storage (the tied embedding / LM head only; the model card names an NVFP4 build of the
+ * checkpoint, and the format is NVIDIA's: FP4 E2M1 elements, one FP8 E4M3 scale per 16
+ * consecutive elements of a row, one fp32 tensor scale g; element = e2m1 * e4m3 * g).  For a
+ * matrix of R rows and K columns (K a multiple of 256), Rp = R rounded up to a multiple of 256:
+ *   codes  uint8 [K/64][Rp][32]: byte i of (k-block kb, row r) holds column kb*64 + 2i in its
+ *          low nibble and column kb*64 + 2i + 1 in its high nibble;
+ *   scales uint8 [K/64][Rp][4]:  scale j of (kb, r) covers columns kb*64 + 16j .. + 15.
+ * Rows [R, Rp) are padding (read, never used).  Both arrays 16-byte aligned. */
 
 /* Model shape.  The MASK token id is `vocab` (one extra embedding row); the LM head covers
  * ids [0, vocab), so argmax never returns MASK.  rope_theta: rotary base; rms_eps: RMSNorm eps. */
@@ -69,6 +78,8 @@ typedef struct dg_config {
   double rope_theta, rms_eps;
   int32_t act_dtype; /* DG_F32 or DG_BF16 */
   int32_t w_dtype;   /* DG_F32 (with act F32), DG_BF16 or DG_E4M3 (with act BF16) */
+  int32_t emb_dtype; /* the tied embedding / LM head: act_dtype, or DG_NVFP4 (with act BF16,
+                        d_model a multiple of 256, at most 4096) */
 } dg_config;
 
 /* One layer's weights (device pointers).  Every matrix is [out][in], `in` contiguous.
@@ -87,10 +98,15 @@ typedef struct dg_layer_weights {
 } dg_layer_weights;
 
 /* A whole model: `layers` is a HOST array of n_layers structs; `emb` the tied embedding /
- * LM head [V + 1][d] in the activation type (row V = MASK; rows [0,V) = LM head). */
+ * LM head [V + 1][d] in the activation type (row V = MASK; rows [0,V) = LM head).  With
+ * emb_dtype DG_NVFP4, `emb` holds the NVFP4 codes of that [V + 1][d] matrix, emb_scale its
+ * block scales and emb_scale_global its tensor scale (layout above); otherwise both are
+ * ignored. */
 typedef struct dg_model {
   const dg_layer_weights *layers;
   const void *emb;
+  const uint8_t *emb_scale;
+  float emb_scale_global;
 } dg_model;
 
 /* ---- sizes and status ------------------------------------------------------------------ */
@@ -184,6 +200,18 @@ int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_de
                       int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
                       int32_t *dev_status, void *stream);
 
+/* dg_logits_entropy with the LM head in NVFP4 (cfg->emb_dtype DG_NVFP4): w_codes, w_scale and
+ * w_scale_global hold the [V + 1][d] embedding in the NVFP4 layout above; the logits are
+ * z = f (e2m1 * e4m3)^T, accumulated in fp32 from the normalised rows f stored in fp16 and the
+ * exact fp16 products e2m1 * e4m3, then times w_scale_global.  (The same holds for the final
+ * RMSNorm rows of dg_canvas_step with an NVFP4 model.)  Other arguments, outputs and errors as
+ * dg_logits_entropy; DG_ERR_INVALID_ARG if cfg->emb_dtype is not DG_NVFP4. */
+int dg_logits_entropy_nvfp4(const dg_config *cfg, int n_rows, const int32_t *n_rows_dev,
+                            const void *h, const int32_t *row_idx, const uint8_t *w_codes,
+                            const uint8_t *w_scale, float w_scale_global, float *entropy,
+                            int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
+                            int32_t *dev_status, void *stream);
+
 /* Entropy-bounded selection and commit (model card "diffusiongemma", Benchmark Results: the
  * EB sampler; "DiffusionGemma Technical Report", What they did: adaptive stopping).  The
  * pages name the sampler but print no formula; the rule is the published EB sampler
@@ -252,7 +280,8 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
  * its scratch in a fixed array of DG_STATIC_SCRATCH_BYTES inside the library's device image,
  * which every GPU that loads the library holds until the process exits.  It allocates nothing.
  *   Same arguments and results as dg_logits_entropy, without logits_dbg and ws.
- *   Limits: bf16 activations (DG_ERR_UNSUPPORTED otherwise), n_rows <= 256, d_model <= 2048,
+ *   Limits: bf16 activations and a bf16 LM head (DG_ERR_UNSUPPORTED otherwise; NVFP4 takes
+ *   dg_logits_entropy_nvfp4), n_rows <= 256, d_model <= 2048,
  *   vocab <= 262144; larger requests return DG_ERR_WORKSPACE and launch nothing.
  *   The first call on a device looks up the array's device address with that device current
  *   (cudaGetSymbolAddress); make that first call before any stream capture on the device.

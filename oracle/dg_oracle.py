@@ -76,6 +76,11 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return np.where(np.isfinite(x), r, x)
 
 
+def round_f16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest IEEE binary16 value (ties to even), returned as fp64."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
 def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
     """Decode OCP FP8 E4M3 codes: 1 sign, 4 exponent (bias 7), 3 mantissa bits.
 
@@ -422,8 +427,15 @@ def layer_rest(cfg, model: OracleModel, l: int, x, q, k, v, kc, vc, causal: bool
 
 
 def lm_head_rows(cfg, model: OracleModel, x_rows: np.ndarray, keep_logits: bool = False):
-    """Final RMSNorm of the given rows, logits over [0, V), entropy and argmax."""
-    f = storage_round(rmsnorm(x_rows, cfg.rms_eps), cfg.act)
+    """Final RMSNorm of the given rows, logits over [0, V), entropy and argmax.
+
+    The normalised rows are stored in the activation type, except in front of an NVFP4 LM head:
+    its dequantised weights (e2m1 times an E4M3 scale, exact in fp16) meet the rows in an fp16
+    product, so the rows are stored in fp16 (the reading taken for the NVFP4 workload)."""
+    if getattr(cfg, "emb", "") == "nvfp4":
+        f = round_f16(rmsnorm(x_rows, cfg.rms_eps))
+    else:
+        f = storage_round(rmsnorm(x_rows, cfg.rms_eps), cfg.act)
     R = f.shape[0]
     z = np.empty((R, cfg.vocab))
     for v0, w in model.lm_head_chunks():

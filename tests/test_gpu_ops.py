@@ -262,6 +262,64 @@ def test_logits_entropy_row_counts(cfg, R, n_dev, vocab):
     others = np.setdiff1d(np.arange(R_all), src)
     assert (ent[others] == -1.0).all() and (am[others] == -1).all()
 
+
+@pytest.mark.parametrize("R,n_dev,vocab", [(1, None, 0), (128, None, 0), (129, None, 0),
+                                           (300, 129, 0), (513, 400, 0), (100, None, 3700),
+                                           (256, 250, 3700)])
+def test_logits_entropy_nvfp4_row_counts(R, n_dev, vocab):
+    """The LM head with NVFP4 weights (codes expanded to bf16 in shared memory, tensor scale in
+    the epilogue) against the oracle's exact decode, over row counts that span several 128-row
+    tiles with ragged tails, a device-side count below the host maximum, and a vocabulary that
+    ends in a ragged tile."""
+    c = synth.reduced("layer_nvfp4")
+    if vocab:
+        c = dataclasses.replace(c, vocab=vocab)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(2000 + R + (n_dev or 0))
+    model = synth.make_model(c, "cpu", seed=29)
+    R_all = R + 37
+    live = R if n_dev is None else n_dev
+    h = torch.randn((R_all, c.d_model), generator=g) * 0.07
+    rows = torch.randperm(R_all, generator=g).numpy()[:R].astype(np.int32)
+    dgc = B.make_config(c)
+    ent = torch.full((R_all,), -1.0, device="cuda")
+    am = torch.full((R_all,), -1, dtype=torch.int32, device="cuda")
+    lg = torch.zeros((R, c.vocab), device="cuda")
+    nd = None if n_dev is None else torch.tensor([n_dev], dtype=torch.int32, device="cuda")
+    B.dg_logits_entropy_nvfp4(dgc, R, nd, h.cuda(), torch.from_numpy(rows).cuda(),
+                              model["emb"].cuda(), model["emb_scale"].cuda(),
+                              model["emb_scale_global"], ent, am, lg,
+                              B.alloc_workspace(dgc, 1, R, 0))
+    torch.cuda.synchronize()
+    om = oracle_model(c, model)
+    src = rows[:live]
+    H, oam, margin, z = O.lm_head_rows(c, om, h.double().numpy()[src], keep_logits=True)
+    lg, ent, am = lg.cpu().numpy()[:live], ent.cpu().numpy(), am.cpu().numpy()
+    assert np.abs(lg - z).max() <= LOGIT_TOL
+    np.testing.assert_allclose(ent[src], H, rtol=ENT_RTOL)
+    assert (am[src] == np.argmax(lg, axis=1)).all()
+    safe = margin > 2 * LOGIT_TOL
+    assert (am[src][safe] == oam[safe]).all()
+    others = np.setdiff1d(np.arange(R_all), src)
+    assert (ent[others] == -1.0).all() and (am[others] == -1).all()
+
+
+def test_logits_entropy_nvfp4_argument_checks():
+    c = synth.reduced("layer_nvfp4")
+    dgc = B.make_config(c)
+    model = synth.make_model(c, "cpu", seed=29)
+    codes, scales = model["emb"].cuda(), model["emb_scale"].cuda()
+    h = torch.zeros((4, c.d_model), device="cuda")
+    ent = torch.zeros(4, device="cuda")
+    am = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ws = B.alloc_workspace(dgc, 1, 4, 0)
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        with pytest.raises(B.DgError):
+            B.dg_logits_entropy_nvfp4(dgc, 4, None, h, None, codes, scales, bad, ent, am, None, ws)
+    with pytest.raises(B.DgError):   # the bf16 entry point refuses an NVFP4 config
+        B.dg_logits_entropy(dgc, 4, None, h, None, codes, ent, am, None, ws)
+
+
 def _step_compare(wl, st_np, check_eb=True):
     """One dg_canvas_step vs the oracle from the same state; returns the oracle's new state."""
     cfg = wl.cfg
@@ -304,9 +362,13 @@ def _step_compare(wl, st_np, check_eb=True):
     return new_np, n_tie
 
 
-@pytest.mark.parametrize("name,batch", [("layer", 1), ("batch32", 2)])
+@pytest.mark.parametrize("name,batch", [("layer", 1), ("batch32", 2), ("layer_nvfp4", 1)])
 def test_step_parity_reduced(name, batch):
-    cfg = synth.reduced(name, batch=batch)
+    # the NVFP4 case draws its router with std 1/sqrt(d) (as the batch-32 workload does): with
+    # 0.02 its all-MASK rows put 68 of 192 router decisions within the near-tie margin, which
+    # leaves too few rows to compare (39 for the bf16 layer, 28 with this router)
+    over = {"router_std": 1.0 / 16.0} if name == "layer_nvfp4" else {}
+    cfg = synth.reduced(name, batch=batch, **over)
     wl = Workload(cfg, gen_device="cpu", state_kind="all_mask")
     st = np_state(wl.state)
     total_tie = 0
@@ -320,8 +382,9 @@ def test_step_parity_reduced(name, batch):
     assert total_tie < 0.3 * 3 * cfg.canvas * batch
 
 
-def test_kv_append_parity_two_layers():
-    cfg = synth.reduced("stack30", n_layers=2, prompt_len=64, n_canvases=2)
+@pytest.mark.parametrize("emb", ["", "nvfp4"])
+def test_kv_append_parity_two_layers(emb):
+    cfg = synth.reduced("stack30", n_layers=2, prompt_len=64, n_canvases=2, emb=emb)
     wl = Workload(cfg, gen_device="cpu")
     kc = torch.zeros_like(wl.kv["k"]); vc = torch.zeros_like(wl.kv["v"])
     # prefill 64 random prompt ids first, then append one canvas of 64

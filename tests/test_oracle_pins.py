@@ -70,6 +70,20 @@ def test_e2m1_decode_all_codes_vs_ml_dtypes():
     assert np.array_equal(O.e2m1_to_f64(codes | 0xF0), got)
 
 
+def test_round_f16_matches_struct_half_and_ties():
+    """Against Python's IEEE binary16 packing of a double (struct 'e'), which rounds once; torch
+    converts float64 through binary32 and can round twice near halfway points."""
+    import struct
+    x = rng.standard_normal(20000) * np.exp2(rng.integers(-20, 12, 20000))
+    ref = np.array([struct.unpack("e", struct.pack("e", float(v)))[0] for v in x])
+    np.testing.assert_array_equal(O.round_f16(x), ref)
+    # halfway between 1 and 1 + 2**-10 rounds to the even 1; 65520 (halfway past the largest
+    # finite 65504) overflows to inf; 2**-25 (half the smallest subnormal) rounds to 0
+    assert O.round_f16(np.array([1 + 2.0 ** -11]))[0] == 1.0
+    assert np.isinf(O.round_f16(np.array([65520.0]))[0])
+    assert O.round_f16(np.array([2.0 ** -25]))[0] == 0.0
+
+
 def test_nvfp4_rows_hand_built_layout():
     """Four nonzero elements placed by hand: nibble order, k-block and 16-element scale block."""
     d, R = 128, 3
@@ -123,11 +137,17 @@ def test_nvfp4_model_matches_bf16_model_with_the_same_values():
                             "layers": []})
     ids = np.array([0, 7, 299, 300])
     np.testing.assert_array_equal(m4.emb_rows(ids), m16.emb_rows(ids))
+    for (v0, w16), (v1, w4) in zip(m16.lm_head_chunks(128), m4.lm_head_chunks(128)):
+        assert v0 == v1
+        np.testing.assert_array_equal(w4, w16)
+    # the NVFP4 LM head stores its normalised rows in fp16 (the bf16 one in bf16)
     x = rng.standard_normal((6, c4.d_model))
-    a = O.lm_head_rows(c16, m16, x, keep_logits=True)
-    b = O.lm_head_rows(c4, m4, x, keep_logits=True)
-    for u, v in zip(a, b):
-        np.testing.assert_array_equal(u, v)
+    f = O.round_f16(O.rmsnorm(x, c4.rms_eps))
+    H, am, _, z = O.lm_head_rows(c4, m4, x, keep_logits=True)
+    np.testing.assert_array_equal(z, f @ dense[:c4.vocab].T)
+    H2, am2, _ = O.entropy_argmax(z)
+    np.testing.assert_array_equal(H, H2)
+    np.testing.assert_array_equal(am, am2)
 
 
 # ----------------------------------------------------------------- layer pieces
