@@ -494,24 +494,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // conversion and one f16x2 multiply by the block scale per pair of weights (e2m1 * e4m3 is exact
 // in fp16).  The MMA is kind::f16 with fp16 operands, so the normalised rows come in fp16 too;
 // the tensor scale is applied to the fp32 logits in the epilogue.  (A bf16 tile would need two
-// more conversions per pair, and those run at a quarter of the FP32 rate: the converters, not
-// the tensor cores, then set the pace.)
-//   warp 0      producer: A (128 fp16 normalised rows x 64 k, TMA) and the codes and scales of
-//               256 vocabulary rows x 64 k, 4-stage ring;
+// more conversions per pair, and those run at a quarter of the FP32 rate.)
+// Three rings.  A k-block carries only 9 KB of weight bytes from DRAM, so the codes and scales
+// get a deep ring of their own (12 stages, 108 KB in flight per SM, about what the bf16 kernel
+// keeps in flight), filled by one producer warp; the normalised rows (L2-resident) get a short
+// TMA ring filled by another; the expanded tiles a 2-stage ring between converters and MMA.
+// With one ring for all three, a stage's 9 KB could not be refilled before its MMA completed,
+// and four stages kept ~36 KB in flight: the loop ran at DRAM latency / 4 per k-block.
+//   warp 0      producer of the codes and scales ring;
 //   warp 1      TMEM owner and MMA issuer (M 128, N 256, K 16), two 256-column accumulators;
 //   warps 2-5   entropy epilogue (as lmhead_tc_kernel, logits times the tensor scale);
-//   warps 6-13  converters: thread i expands vocabulary row i of the tile into a 3-stage ring of
-//               fp16 tiles, then fences its stores for the tensor cores' (async) proxy.
-// A raw stage is free once the MMAs that read its A tile have completed and every converter
-// warp has read its codes (1 + 8 arrivals).  Every wait is bounded.
-constexpr int Q_RSTAGES = 4, Q_CSTAGES = 3, Q_CONV_WARPS = 8;
+//   warps 6-13  converters: thread i expands vocabulary row i of the tile, then fences its stores
+//               for the tensor cores' (async) proxy;
+//   warp 14     producer of the normalised-rows ring (TMA).
+// Every wait is bounded.
+constexpr int Q_QSTAGES = 12, Q_ASTAGES = 3, Q_CSTAGES = 2, Q_CONV_WARPS = 8;
 constexpr int Q_A_BYTES = BM * BK * 2;   // 16 KB normalised rows (fp16)
 constexpr int Q_C_BYTES = BN * BK / 2;   // 8 KB FP4 codes
 constexpr int Q_S_BYTES = BN * BK / 16;  // 1 KB E4M3 scales
+constexpr int Q_R_BYTES = Q_C_BYTES + Q_S_BYTES;
 constexpr int Q_B_BYTES = BN * BK * 2;   // 32 KB expanded fp16 tile
-constexpr int Q_THREADS = 192 + 32 * Q_CONV_WARPS;
-constexpr size_t Q_SMEM = 1024 + (size_t)Q_CSTAGES * Q_B_BYTES +
-                          (size_t)Q_RSTAGES * (Q_A_BYTES + Q_C_BYTES + Q_S_BYTES) + 256;
+constexpr int Q_THREADS = 32 * (6 + Q_CONV_WARPS + 1);
+constexpr int Q_APROD_WARP = 6 + Q_CONV_WARPS;
+constexpr size_t Q_SMEM = 1024 + (size_t)Q_CSTAGES * Q_B_BYTES + (size_t)Q_ASTAGES * Q_A_BYTES +
+                          (size_t)Q_QSTAGES * Q_R_BYTES + 512;
 static_assert(Q_SMEM <= 232448, "more shared memory than one CTA may have");
 static_assert(Q_CONV_WARPS * 32 == BN, "one converter thread per vocabulary row of a tile");
 
@@ -522,12 +528,13 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sB = smem;                               // [Q_CSTAGES][32 KB], 1024-aligned
-  uint8_t *sA = sB + Q_CSTAGES * Q_B_BYTES;         // [Q_RSTAGES][16 KB], 1024-aligned
-  uint8_t *sQ = sA + Q_RSTAGES * Q_A_BYTES;         // [Q_RSTAGES][8 KB]
-  uint8_t *sS = sQ + Q_RSTAGES * Q_C_BYTES;         // [Q_RSTAGES][1 KB]
-  uint64_t *full = reinterpret_cast<uint64_t *>(sS + Q_RSTAGES * Q_S_BYTES);
-  uint64_t *empty = full + Q_RSTAGES;
-  uint64_t *cfull = empty + Q_RSTAGES;
+  uint8_t *sA = sB + Q_CSTAGES * Q_B_BYTES;         // [Q_ASTAGES][16 KB], 1024-aligned
+  uint8_t *sR = sA + Q_ASTAGES * Q_A_BYTES;         // [Q_QSTAGES][8 KB codes + 1 KB scales]
+  uint64_t *qfull = reinterpret_cast<uint64_t *>(sR + Q_QSTAGES * Q_R_BYTES);
+  uint64_t *qempty = qfull + Q_QSTAGES;
+  uint64_t *afull = qempty + Q_QSTAGES;
+  uint64_t *aempty = afull + Q_ASTAGES;
+  uint64_t *cfull = aempty + Q_ASTAGES;
   uint64_t *cempty = cfull + Q_CSTAGES;
   uint64_t *tfull = cempty + Q_CSTAGES;
   uint64_t *tempty = tfull + 2;
@@ -543,9 +550,13 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   const int kblocks = p.K / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < Q_RSTAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + Q_CONV_WARPS);
+    for (int s = 0; s < Q_QSTAGES; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], Q_CONV_WARPS);
+    }
+    for (int s = 0; s < Q_ASTAGES; ++s) {
+      mbar_init(&afull[s], 1);
+      mbar_init(&aempty[s], 1);
     }
     for (int c = 0; c < Q_CSTAGES; ++c) {
       mbar_init(&cfull[c], Q_CONV_WARPS);
@@ -558,7 +569,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == Q_APROD_WARP && lane == 0) tma_prefetch_desc(&tmA);
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
@@ -569,71 +580,94 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == 0) {  // codes and scales
       int stage = 0;
       uint32_t ph = 0;
-      int armed[Q_RSTAGES];
-      uint32_t armed_ph[Q_RSTAGES];
+      int armed[Q_QSTAGES];
+      uint32_t armed_ph[Q_QSTAGES];
 #pragma unroll
-      for (int s = 0; s < Q_RSTAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      for (int s = 0; s < Q_QSTAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        const int mt = u % m_tiles, nt = u / m_tiles;
+        const int nt = u / m_tiles;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
-          mbar_expect_tx(&full[stage], Q_A_BYTES + Q_C_BYTES + Q_S_BYTES);
-          tma_load_2d(sA + stage * Q_A_BYTES, &tmA, &full[stage], kb * BK, mt * BM);
+          if (!mbar_wait(&qempty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
+          mbar_expect_tx(&qfull[stage], Q_R_BYTES);
           const size_t slab = (size_t)kb * p.rows_pad + (size_t)nt * BN;
-          bulk_load(sQ + stage * Q_C_BYTES, p.q_codes + slab * (BK / 2), Q_C_BYTES, &full[stage]);
-          bulk_load(sS + stage * Q_S_BYTES, p.q_scales + slab * (BK / 16), Q_S_BYTES,
-                    &full[stage]);
+          uint8_t *dst = sR + stage * Q_R_BYTES;
+          bulk_load(dst, p.q_codes + slab * (BK / 2), Q_C_BYTES, &qfull[stage]);
+          bulk_load(dst + Q_C_BYTES, p.q_scales + slab * (BK / 16), Q_S_BYTES, &qfull[stage]);
           armed[stage] = 1;
           armed_ph[stage] = ph;
-          if (++stage == Q_RSTAGES) { stage = 0; ph ^= 1; }
+          if (++stage == Q_QSTAGES) { stage = 0; ph ^= 1; }
         }
       }
       if (*abort_flag) {  // let every issued copy land before the CTA's shared memory goes away
-        for (int s = 0; s < Q_RSTAGES; ++s)
-          if (armed[s]) (void)mbar_wait(&full[s], armed_ph[s]);
+        for (int s = 0; s < Q_QSTAGES; ++s)
+          if (armed[s]) (void)mbar_wait(&qfull[s], armed_ph[s]);
+      }
+    }
+  } else if (warp == Q_APROD_WARP) {
+    if (lane == 0) {  // normalised rows
+      int stage = 0;
+      uint32_t ph = 0;
+      int armed[Q_ASTAGES];
+      uint32_t armed_ph[Q_ASTAGES];
+#pragma unroll
+      for (int s = 0; s < Q_ASTAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const int mt = u % m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&aempty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
+          mbar_expect_tx(&afull[stage], Q_A_BYTES);
+          tma_load_2d(sA + stage * Q_A_BYTES, &tmA, &afull[stage], kb * BK, mt * BM);
+          armed[stage] = 1;
+          armed_ph[stage] = ph;
+          if (++stage == Q_ASTAGES) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < Q_ASTAGES; ++s)
+          if (armed[s]) (void)mbar_wait(&afull[s], armed_ph[s]);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(BM, BN);
-      int stage = 0, cst = 0, acc = 0;
-      uint32_t ph = 0, cph = 0, aph = 0;
-      int last_stage = -1;
-      uint32_t last_ph = 0;
+      int ast = 0, cst = 0, acc = 0;
+      uint32_t aph = 0, cph = 0, tph = 0;
+      int last_ast = -1;
+      uint32_t last_aph = 0;
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], aph ^ 1)) { fail(p.status, abort_flag); break; }
+        if (!mbar_wait(&tempty[acc], tph ^ 1)) { fail(p.status, abort_flag); break; }
         fence_after();
         const uint32_t d = tmem + acc * BN;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], ph) || !mbar_wait(&cfull[cst], cph)) {
+          if (!mbar_wait(&afull[ast], aph) || !mbar_wait(&cfull[cst], cph)) {
             fail(p.status, abort_flag);
             ok = false;
             break;
           }
           fence_after();
-          const uint64_t ad = sdesc_sw128(sA + stage * Q_A_BYTES);
+          const uint64_t ad = sdesc_sw128(sA + ast * Q_A_BYTES);
           const uint64_t bd = sdesc_sw128(sB + cst * Q_B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          commit(&empty[stage]);
+          commit(&aempty[ast]);
           commit(&cempty[cst]);
-          last_stage = stage;
-          last_ph = ph;
-          if (++stage == Q_RSTAGES) { stage = 0; ph ^= 1; }
+          last_ast = ast;
+          last_aph = aph;
+          if (++ast == Q_ASTAGES) { ast = 0; aph ^= 1; }
           if (++cst == Q_CSTAGES) { cst = 0; cph ^= 1; }
         }
         if (!ok) break;
         commit(&tfull[acc]);
         acc ^= 1;
-        if (acc == 0) aph ^= 1;
+        if (acc == 0) tph ^= 1;
       }
-      if (*abort_flag && last_stage >= 0)  // the MMAs issued so far finish before TMEM is freed
-        (void)mbar_wait(&empty[last_stage], last_ph);
+      if (*abort_flag && last_ast >= 0)  // the MMAs issued so far finish before TMEM is freed
+        (void)mbar_wait(&aempty[last_ast], last_aph);
     }
   } else if (warp < 6) {
     const int q = warp & 3;  // TMEM lane quarter this warp may read
@@ -686,21 +720,24 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     // codes, columns 8w .. 8w + 7 of the k-block) becomes 16-byte chunk w of the row's 128 bytes,
     // stored at chunk position w ^ (row % 8) (the 128-byte swizzle).
     const int row = (warp - 6) * 32 + lane;
-    int stage = 0, cst = 0;
-    uint32_t ph = 0, cph = 0;
+    int qst = 0, cst = 0;
+    uint32_t qph = 0, cph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], ph)) ||
+        if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qst], qph)) ||
             !__all_sync(0xffffffffu, mbar_wait(&cempty[cst], cph ^ 1))) {
           fail(p.status, abort_flag);
           ok = false;
           break;
         }
-        const uint4 *src = reinterpret_cast<const uint4 *>(sQ + stage * Q_C_BYTES + row * 32);
+        const uint8_t *raw = sR + qst * Q_R_BYTES;
+        const uint4 *src = reinterpret_cast<const uint4 *>(raw + row * 32);
         const uint4 q0 = src[0], q1 = src[1];
-        const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sS + stage * Q_S_BYTES + row * 4);
+        const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(raw + Q_C_BYTES + row * 4);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[qst]);  // the raw stage is in registers now
         const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
         uint8_t *dst = sB + cst * Q_B_BYTES + row * 128;
 #pragma unroll
@@ -716,11 +753,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
         }
         fence_proxy_async_smem();  // the tensor cores read these stores through the async proxy
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&cfull[cst]);
-          mbar_arrive(&empty[stage]);
-        }
-        if (++stage == Q_RSTAGES) { stage = 0; ph ^= 1; }
+        if (lane == 0) mbar_arrive(&cfull[cst]);
+        if (++qst == Q_QSTAGES) { qst = 0; qph ^= 1; }
         if (++cst == Q_CSTAGES) { cst = 0; cph ^= 1; }
       }
       if (!ok) break;
