@@ -37,6 +37,38 @@ __device__ __forceinline__ __half2 nvfp4_pair_f16(uint32_t byte, __half2 scale2)
   const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(byte & 0xFFu), __NV_E2M1);
   return __hmul2(*reinterpret_cast<const __half2 *>(&r), scale2);
 }
+// Four bytes of FP4 E2M1 code pairs (byte k = columns 2k, 2k + 1; low nibble first) to four
+// f16x2, each times its scale pair (exact, as nvfp4_pair_f16): the word is split into its bytes
+// by one mov, so no shifts per pair.
+__device__ __forceinline__ void nvfp4_word_f16(uint32_t w, __half2 scale2, uint32_t (&o)[4]) {
+  uint32_t h0, h1, h2, h3;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(w));
+  const uint32_t hs[4] = {h0, h1, h2, h3};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&hs[k]), scale2);
+    o[k] = *reinterpret_cast<const uint32_t *>(&v);
+  }
+}
+// Two FP8 E4M3 scales (the low two bytes of `codes`) to f16 (exact), each duplicated into a pair.
+__device__ __forceinline__ void e4m3_scales_f16x2(uint32_t codes, __half2 &s0, __half2 &s1) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+      : "=r"(h)
+      : "r"(codes));
+  const __half2 p = *reinterpret_cast<const __half2 *>(&h);
+  s0 = __low2half2(p);
+  s1 = __high2half2(p);
+}
 __device__ __forceinline__ __half2 e4m3_scale_f16x2(uint32_t code) {
   const __half_raw r = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)(code & 0xFFu), __NV_E4M3);
   const __half h = *reinterpret_cast<const __half *>(&r);

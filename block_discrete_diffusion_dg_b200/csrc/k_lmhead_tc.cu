@@ -720,6 +720,9 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     // codes, columns 8w .. 8w + 7 of the k-block) becomes 16-byte chunk w of the row's 128 bytes,
     // stored at chunk position w ^ (row % 8) (the 128-byte swizzle).
     const int row = (warp - 6) * 32 + lane;
+    uint32_t chunk_off[8];  // byte offset of 16-byte chunk c of this row in a tile (swizzled)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) chunk_off[c] = (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
     int qst = 0, cst = 0;
     uint32_t qph = 0, cph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
@@ -739,17 +742,15 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&qempty[qst]);  // the raw stage is in registers now
         const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        uint8_t *dst = sB + cst * Q_B_BYTES + row * 128;
+        __half2 sc[4];  // scale j covers words 2j and 2j + 1
+        e4m3_scales_f16x2(sc4, sc[0], sc[1]);
+        e4m3_scales_f16x2(sc4 >> 16, sc[2], sc[3]);
+        uint8_t *tile = sB + cst * Q_B_BYTES;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const __half2 sc = e4m3_scale_f16x2(sc4 >> (8 * (c >> 1)));
           uint32_t o[4];
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const __half2 v = nvfp4_pair_f16(w[c] >> (8 * b), sc);
-            o[b] = *reinterpret_cast<const uint32_t *>(&v);
-          }
-          *reinterpret_cast<uint4 *>(dst + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          nvfp4_word_f16(w[c], sc[c >> 1], o);
+          *reinterpret_cast<uint4 *>(tile + chunk_off[c]) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();  // the tensor cores read these stores through the async proxy
         __syncwarp();

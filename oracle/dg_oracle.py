@@ -77,8 +77,11 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 
 
 def round_f16(x: np.ndarray) -> np.ndarray:
-    """Round fp64 values to the nearest IEEE binary16 value (ties to even), returned as fp64."""
-    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+    """Round fp64 values to the nearest IEEE binary16 value (ties to even), returned as fp64.
+
+    Values that round past the largest finite binary16 (65504) become +-inf."""
+    with np.errstate(over="ignore"):
+        return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
 
 
 def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:

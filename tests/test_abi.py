@@ -21,7 +21,8 @@ def built():
 
 
 def _header_functions():
-    src = open(os.path.join(ROOT, "include", "dg.h")).read()
+    with open(os.path.join(ROOT, "include", "dg.h")) as fh:
+        src = fh.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(dg_[a-z_0-9]+)\s*\(", src)))
 
