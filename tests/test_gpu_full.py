@@ -2,6 +2,8 @@
 top-8, vocabulary 262144, canvas 256, prompt K/V 4096) in the launch configuration the
 benchmark times: the all-MASK canvas and the half-committed canvas.
 
+The same two states run with the tied embedding / LM head in NVFP4 (workload layer_nvfp4).
+
 The oracle runs the whole step in fp64 (its LM head over every masked row), so every row's
 entropy and argmax is compared; logits (2e-2 max-abs) are compared on every row through the
 debug logits.  Rows whose oracle router decision is a near tie (gap between the 8th and 9th
@@ -47,8 +49,28 @@ def _entropy_of(lg: np.ndarray) -> np.ndarray:
     return -(p * np.log(np.where(p > 0, p, 1.0))).sum(1)
 
 
+@pytest.fixture(scope="module")
+def wl_nvfp4():
+    return Workload(synth.get_config("layer_nvfp4"), gen_device="cuda")
+
+
 @pytest.mark.parametrize("kind", ["all_mask", "half"])
 def test_layer_step_full_size(wl, oracle_inputs, kind):
+    _full_step(wl, oracle_inputs, kind)
+
+
+@pytest.mark.parametrize("kind", ["all_mask", "half"])
+def test_layer_nvfp4_step_full_size(wl_nvfp4, kind):
+    """The same step with the tied embedding / LM head in NVFP4: the embedding rows decoded in
+    the prologue, fp16 normalised rows, the expanded-weight LM head, every row's entropy and
+    argmax against the oracle's exact NVFP4 decode."""
+    wl = wl_nvfp4
+    oi = (wl.oracle(), decode_cache(wl.cfg, wl.kv["k"]), decode_cache(wl.cfg, wl.kv["v"]),
+          synth.to_numpy(wl.kv["cache_len"]))
+    _full_step(wl, oi, kind)
+
+
+def _full_step(wl, oracle_inputs, kind):
     cfg = wl.cfg
     om, kc, vc, cl = oracle_inputs
     st_np = np_state(synth.make_canvas_state(cfg, kind))
