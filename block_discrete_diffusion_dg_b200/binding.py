@@ -83,6 +83,8 @@ _SIGS = {
                             _VP, _VP]),
     "dg_canvas_step": (_I32, [_PCFG, _PMODEL, _I32, _VP, _VP, _VP, _VP, _VP, _I32, ctypes.c_double,
                               _VP, _VP, _VP, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "dg_generate": (_I32, [_PCFG, _PMODEL, _I32, _VP, _VP, _VP, _VP, _VP, _I32, ctypes.c_double,
+                           _VP, _VP, _VP, _I32, _I32, _VP, _SZ, _VP, _VP]),
 }
 
 
@@ -280,6 +282,16 @@ def dg_canvas_step(cfg, model: Model, batch, tokens, masked, n_masked, done, ste
                                 _p(entropy_out), _p(argmax_out), _p(logits_dbg), _p(expert_load),
                                 _p(forced_topk), w, wb, _p(dev_status), _stream(stream)),
            "dg_canvas_step")
+
+
+def dg_generate(cfg, model: Model, batch, tokens, masked, n_masked, done, step, max_steps, gamma,
+                k_cache, v_cache, cache_len, cache_cap, append, ws, dev_status=None, stream=None):
+    w, wb = _ws(ws)
+    _check(lib().dg_generate(ctypes.byref(cfg), ctypes.byref(model.struct), batch, _p(tokens),
+                             _p(masked), _p(n_masked), _p(done), _p(step), max_steps, float(gamma),
+                             _p(k_cache), _p(v_cache), _p(cache_len), cache_cap, int(append), w, wb,
+                             _p(dev_status), _stream(stream)),
+           "dg_generate")
 
 
 def exported_symbols() -> Sequence[str]:

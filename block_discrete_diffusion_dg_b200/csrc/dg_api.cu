@@ -5,6 +5,8 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <string>
 #include <vector>
 
 #include "dg_common.cuh"
@@ -39,6 +41,11 @@ void note_launch(cudaStream_t s, const char *name) {
   }
 }
 
+bool &pdl_allowed() {
+  static thread_local bool on = true;
+  return on;
+}
+
 int check_launch(const char *what) {
   const cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) return DG_OK;
@@ -61,7 +68,7 @@ inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
   B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_WDQ, B_LIVE, B_ROWS, B_NROWS, B_SLOT, B_FIN, B_LOGITS, B_PART,
-  B_ENT, B_AM, B_ATTN, B_HP, B_COUNT
+  B_ENT, B_AM, B_ATTN, B_HP, B_GEN, B_COUNT
 };
 
 struct Layout {
@@ -135,6 +142,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_ENT] = T * 4;
   sz[B_AM] = T * 4;
   { const int op = o_parts(c, (int)T); sz[B_HP] = op > 1 ? T * d * 4 * op : 0; }
+  sz[B_GEN] = 16;  // dg_generate's loop counter
   sz[B_ATTN] = attention_ws_bytes(c.act_dtype, batch, n, c.n_q_heads, c.n_kv_heads, c.head_dim,
                                   cap);
   size_t o = 0;
@@ -420,6 +428,57 @@ int check_ws(const dg_config *c, int batch, int n, int cap, const void *ws, size
   if (((uintptr_t)ws) & 255) return DG_ERR_INVALID_ARG;
   if (ws_bytes < L->total) return DG_ERR_WORKSPACE;
   return DG_OK;
+}
+
+}  // namespace
+}  // namespace dg
+
+namespace dg {
+namespace {
+
+// Condition of dg_generate's device loop (one thread, after the step's EB kernel): run the body
+// again while some canvas is not done, no device error has been recorded, and fewer than `cap`
+// iterations have run (the cap ends the loop even if an error keeps a canvas from finishing).
+__global__ void gen_cond_kernel(cudaGraphConditionalHandle h, const int32_t *done, int batch,
+                                int32_t *iter, int cap, const int32_t *st) {
+  int running = 0;
+  for (int b = 0; b < batch; ++b) running |= (done[b] == 0);
+  const int it = *iter + 1;
+  *iter = it;
+  const bool ok = st == nullptr || *st == DG_OK;
+  cudaGraphSetConditional(h, (running && ok && it < cap) ? 1u : 0u);
+}
+
+// A stream of this thread for capturing graph bodies (one per device).
+cudaStream_t capture_stream() {
+  static thread_local cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!streams[dev]) cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+  return streams[dev];
+}
+
+// Records a failed CUDA call (dg_last_cuda_error) and returns DG_ERR_CUDA.
+int cuda_fail(const char *what, cudaError_t e) {
+  (void)cudaGetLastError();
+  snprintf(g_err, sizeof(g_err), "%s: %s", what, cudaGetErrorString(e));
+  return DG_ERR_CUDA;
+}
+
+// Instantiated device-loop graphs, keyed by every argument that is baked into them.
+struct GenCache {
+  std::mutex mu;
+  std::vector<std::pair<std::string, cudaGraphExec_t>> entries;  // most recent last
+};
+GenCache &gen_cache() {
+  static GenCache c;
+  return c;
+}
+constexpr size_t GEN_CACHE_MAX = 8;
+
+template <typename T> void key_add(std::string &k, const T &v) {
+  k.append(reinterpret_cast<const char *>(&v), sizeof(T));
 }
 
 }  // namespace
@@ -720,6 +779,128 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                     s));
   return launch_eb_select(batch, C, ent, am, quant_gamma(gamma), max_steps, tokens, masked,
                           nullptr, n_masked, done, step, dev_status, s);
+}
+
+int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
+                uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step, int max_steps,
+                double gamma, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
+                int append, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
+    return DG_ERR_INVALID_ARG;
+  if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
+  if (cache_cap < 0 || (cache_cap > 0 && (!k_cache || !v_cache))) return DG_ERR_INVALID_ARG;
+  if (append && (cache_cap <= 0 || cfg->canvas > cache_cap)) return DG_ERR_INVALID_ARG;
+  if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
+  for (int l = 0; l < cfg->n_layers; ++l)
+    if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
+  if (!lm_weights_ok(*cfg, lm_weights(*cfg, model))) return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, batch, cfg->canvas, cache_cap, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  int32_t *iter = w.at<int32_t>(B_GEN);
+  const cudaStream_t s = (cudaStream_t)stream;
+
+  std::string key;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  key_add(key, dev);
+  key_add(key, *cfg);
+  key_add(key, model->emb);
+  key_add(key, model->emb_scale);
+  key_add(key, model->emb_scale_global);
+  for (int l = 0; l < cfg->n_layers; ++l) key_add(key, model->layers[l]);
+  const void *ptrs[] = {tokens, masked, n_masked, done, step, k_cache, v_cache, cache_len, ws,
+                        dev_status};
+  key.append(reinterpret_cast<const char *>(ptrs), sizeof(ptrs));
+  key_add(key, batch);
+  key_add(key, max_steps);
+  key_add(key, gamma);
+  key_add(key, cache_cap);
+  key_add(key, ws_bytes);
+
+  cudaGraphExec_t exec = nullptr;
+  {
+    GenCache &gc = gen_cache();
+    std::lock_guard<std::mutex> lock(gc.mu);
+    for (auto &e : gc.entries)
+      if (e.first == key) exec = e.second;
+  }
+  if (!exec) {
+    // parent graph: reset the loop counter, then a while node whose body is one captured step
+    // and the condition kernel.  Programmatic edges are tried first; without them if the body
+    // does not take them.
+    int rc = DG_ERR_CUDA;
+    for (int attempt = 0; attempt < 2 && rc != DG_OK; ++attempt) {
+      cudaGraph_t g = nullptr;
+      cudaError_t e = cudaGraphCreate(&g, 0);
+      if (e != cudaSuccess) return cuda_fail("cudaGraphCreate", e);
+      cudaMemsetParams mp{};
+      mp.dst = iter;
+      mp.value = 0;
+      mp.elementSize = 4;
+      mp.width = 1;
+      mp.height = 1;
+      cudaGraphNode_t reset = nullptr, loop = nullptr;
+      cudaGraphConditionalHandle h{};
+      cudaGraphNodeParams cp{};
+      e = cudaGraphAddMemsetNode(&reset, g, nullptr, 0, &mp);
+      if (e == cudaSuccess) e = cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault);
+      if (e == cudaSuccess) {
+        cp.type = cudaGraphNodeTypeConditional;
+        cp.conditional.handle = h;
+        cp.conditional.type = cudaGraphCondTypeWhile;
+        cp.conditional.size = 1;
+        e = cudaGraphAddNode(&loop, g, &reset, 1, &cp);
+      }
+      cudaStream_t cs = capture_stream();
+      if (e == cudaSuccess && !cs) e = cudaErrorInvalidDevice;
+      if (e == cudaSuccess)
+        e = cudaStreamBeginCaptureToGraph(cs, cp.conditional.phGraph_out[0], nullptr, nullptr, 0,
+                                          cudaStreamCaptureModeThreadLocal);
+      if (e != cudaSuccess) {
+        cudaGraphDestroy(g);
+        return cuda_fail("dg_generate graph", e);
+      }
+      pdl_allowed() = attempt == 0;
+      int src = dg_canvas_step(cfg, model, batch, tokens, masked, n_masked, done, step, max_steps,
+                               gamma, k_cache, v_cache, cache_len, cache_cap, nullptr, nullptr,
+                               nullptr, nullptr, nullptr, ws, ws_bytes, dev_status, cs);
+      if (src == DG_OK) {
+        gen_cond_kernel<<<1, 1, 0, cs>>>(h, done, batch, iter, max_steps + 1, dev_status);
+        src = check_launch("gen_cond");
+      }
+      pdl_allowed() = true;
+      cudaGraph_t body = nullptr;
+      e = cudaStreamEndCapture(cs, &body);
+      if (src == DG_OK && e == cudaSuccess) e = cudaGraphInstantiate(&exec, g, 0);
+      cudaGraphDestroy(g);
+      if (src != DG_OK && src != DG_ERR_CUDA) {
+        (void)cudaGetLastError();
+        return src;  // the step refused its arguments (checked above, so not expected)
+      }
+      if (src == DG_OK && e == cudaSuccess) {
+        rc = DG_OK;
+      } else {  // a launch or the graph was refused: once more without programmatic edges
+        exec = nullptr;
+        rc = src != DG_OK ? DG_ERR_CUDA : cuda_fail("dg_generate graph", e);
+        (void)cudaGetLastError();
+      }
+    }
+    if (rc != DG_OK) return rc;
+    GenCache &gc = gen_cache();
+    std::lock_guard<std::mutex> lock(gc.mu);
+    if (gc.entries.size() >= GEN_CACHE_MAX) {
+      cudaGraphExecDestroy(gc.entries.front().second);  // freed when its launches complete
+      gc.entries.erase(gc.entries.begin());
+    }
+    gc.entries.emplace_back(key, exec);
+  }
+  const cudaError_t e = cudaGraphLaunch(exec, s);
+  if (e != cudaSuccess) return cuda_fail("dg_generate launch", e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!append) return DG_OK;
+  return dg_kv_append(cfg, model, batch, tokens, cfg->canvas, k_cache, v_cache, cache_len,
+                      cache_cap, nullptr, ws, ws_bytes, dev_status, stream);
 }
 
 }  // extern "C"

@@ -187,6 +187,9 @@ namespace dg {
 // timing event on `s` before the launch, labelled `name`).
 void note_launch(cudaStream_t s, const char *name);
 int check_launch(const char *what);      // DG_OK or DG_ERR_CUDA (records the message)
+// Whether launches of this thread carry programmatic stream serialisation (on by default; off
+// while a step is captured into a graph body that may not take programmatic edges).
+bool &pdl_allowed();
 
 
 // Launches `k` with programmatic stream serialisation allowed (see pdl_wait); errors surface
@@ -203,7 +206,7 @@ inline void launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cuda
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_allowed() ? 1 : 0;
   (void)cudaLaunchKernelEx(&cfg, k, static_cast<P>(args)...);
 }
 
@@ -223,8 +226,9 @@ inline void launch_pdl_cluster(void (*k)(P...), dim3 grid, dim3 block, size_t sm
   at[1].val.clusterDim.x = cluster_x;
   at[1].val.clusterDim.y = 1;
   at[1].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 2;
+  const bool pdl = pdl_allowed();
+  cfg.attrs = pdl ? at : at + 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   (void)cudaLaunchKernelEx(&cfg, k, static_cast<P>(args)...);
 }
 }  // namespace dg

@@ -271,6 +271,27 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                    const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
                    void *stream);
 
+/* Device-resident generation: dg_canvas_step repeated on the device until every canvas is done
+ * ("DiffusionGemma Technical Report", explanatory visual: a canvas is refined over a number of
+ * steps until confident and stable; Figure 4 stage 3: the finished canvas goes back through the
+ * causal encoder), with no host round trip per step, then, if `append` is non-zero, dg_kv_append
+ * of the canvases' final tokens (n_tokens = canvas; their cache_len grows by canvas).
+ * The steps run as one CUDA graph: a while node whose body is one step and a one-thread kernel
+ * that keeps the loop going while some done[b] is 0, *dev_status (if non-NULL) is DG_OK and fewer
+ * than max_steps + 1 iterations have run.  Every canvas finishes within max_steps steps (D7), so
+ * the bound only ends a loop that a device error (DG_ERR_NUMERIC, DG_ERR_TIMEOUT) has stalled;
+ * the error is then in *dev_status.  Canvases already done are skipped, as in dg_canvas_step.
+ * Arguments, layouts and errors as dg_canvas_step and dg_kv_append (k_cache and v_cache are
+ * written only by the append; with append, cache_cap >= canvas).  The instantiated graph is
+ * cached inside the library per argument set (device, config, weight pointers, state, cache and
+ * scratch pointers, sizes, max_steps, gamma; at most 8, least recent dropped), so repeated calls
+ * with the same buffers launch one graph.  Not capturable into another graph; profiling
+ * (dg_profile_begin) must be off while a new argument set is first used. */
+int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
+                uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step, int max_steps,
+                double gamma, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
+                int append, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
 /* ---- fixed-scratch entry point ---------------------------------------------------------- */
 
 /* dg_logits_entropy for callers that cannot provide device scratch memory.  The pages have no

@@ -382,6 +382,42 @@ def test_step_parity_reduced(name, batch):
     assert total_tie < 0.3 * 3 * cfg.canvas * batch
 
 
+def test_device_generate_equals_host_loop():
+    """dg_generate against the host loop of dg_canvas_step on the same bf16 workload (batch 2,
+    the second canvas already done): the same kernels in the same order, so the final states and
+    the appended caches are identical; a max_steps cap of 3 ends both loops at the third step."""
+    cfg = synth.reduced("layer", batch=2, n_canvases=1, gamma=0.5)
+    for max_steps in (cfg.max_steps, 3):
+        wl = Workload(cfg, gen_device="cpu", state_kind="all_mask")
+        st0 = np_state(wl.state)
+        st0["done"][1] = 1
+        kv_h = {k: v.clone() for k, v in wl.kv.items()}
+        kv_d = {k: v.clone() for k, v in wl.kv.items()}
+        h = torch_state(st0)
+        n = 0
+        while not bool(h["done"].all()):
+            B.dg_canvas_step(wl.dgcfg, wl.dgmodel, 2, h["tokens"], h["masked"], h["n_masked"],
+                             h["done"], h["step"], max_steps, cfg.gamma, kv_h["k"], kv_h["v"],
+                             kv_h["cache_len"], wl.cap, None, None, None, wl.ws, wl.status)
+            n += 1
+            assert n <= max_steps
+        B.dg_kv_append(wl.dgcfg, wl.dgmodel, 2, h["tokens"], cfg.canvas, kv_h["k"], kv_h["v"],
+                       kv_h["cache_len"], wl.cap, wl.ws, wl.status)
+        d = torch_state(st0)
+        B.dg_generate(wl.dgcfg, wl.dgmodel, 2, d["tokens"], d["masked"], d["n_masked"], d["done"],
+                      d["step"], max_steps, cfg.gamma, kv_d["k"], kv_d["v"], kv_d["cache_len"],
+                      wl.cap, 1, wl.ws, wl.status)
+        torch.cuda.synchronize()
+        wl.check_status()
+        for k in h:
+            assert torch.equal(h[k], d[k]), k
+        for k in ("k", "v", "cache_len"):
+            assert torch.equal(kv_h[k], kv_d[k]), k
+        assert int(d["step"][0].item()) == n and int(d["step"][1].item()) == 0
+        if max_steps == 3:
+            assert n == 3
+
+
 @pytest.mark.parametrize("emb", ["", "nvfp4"])
 def test_kv_append_parity_two_layers(emb):
     cfg = synth.reduced("stack30", n_layers=2, prompt_len=64, n_canvases=2, emb=emb)

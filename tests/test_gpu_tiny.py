@@ -109,6 +109,37 @@ def test_tiny_generate_and_append(wl):
     np.testing.assert_allclose(v_dev.cpu().numpy(), vc, atol=1e-5)
 
 
+def test_tiny_device_generate_matches_oracle(wl):
+    """dg_generate (the step loop as one graph with a device-side while condition, then the
+    append) over two canvases against the oracle's generation: tokens, step counts, cache."""
+    cfg = wl.cfg
+    kv0 = {k: v.clone() for k, v in wl.kv.items()}
+    model = wl.oracle()
+    kc = decode_cache(cfg, kv0["k"])
+    vc = decode_cache(cfg, kv0["v"])
+    cl = synth.to_numpy(kv0["cache_len"])
+    o_tok, o_steps, o_len = O.generate(cfg, model, kc, vc, cl, cfg.n_canvases, cfg.gamma,
+                                       cfg.max_steps)
+    k_dev, v_dev, len_dev = kv0["k"], kv0["v"], kv0["cache_len"]
+    ws = B.alloc_workspace(wl.dgcfg, cfg.batch, cfg.canvas, wl.cap)
+    st = torch_state(np_state(synth.make_canvas_state(cfg, "all_mask")))
+    for c in range(cfg.n_canvases):
+        fresh = torch_state(np_state(synth.make_canvas_state(cfg, "all_mask")))
+        for k in st:          # the same state buffers every canvas: the second call reuses the graph
+            st[k].copy_(fresh[k])
+        B.dg_generate(wl.dgcfg, wl.dgmodel, 1, st["tokens"], st["masked"], st["n_masked"],
+                      st["done"], st["step"], cfg.max_steps, cfg.gamma, k_dev, v_dev, len_dev,
+                      wl.cap, 1, ws, wl.status)
+        torch.cuda.synchronize()
+        wl.check_status()
+        assert int(st["done"].item()) == 1
+        assert int(st["step"].item()) == o_steps[0, c]
+        assert (st["tokens"].cpu().numpy()[0] == o_tok[0, c]).all()
+    assert int(len_dev.item()) == o_len[0]
+    np.testing.assert_allclose(k_dev.cpu().numpy(), kc, atol=1e-5)
+    np.testing.assert_allclose(v_dev.cpu().numpy(), vc, atol=1e-5)
+
+
 def _eb_case(C, rng, gamma, force, nan=False):
     H = rng.choice(np.array([0.0, -0.0, -1e-7, 0.05, 0.1, 0.1, 0.25, 0.3, 1.0, 6.0], np.float32), C)
     H = np.where(rng.uniform(size=C) < 0.5, rng.uniform(0, 2, C).astype(np.float32), H).astype(np.float32)
