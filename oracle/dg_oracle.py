@@ -234,6 +234,22 @@ def router_topk(y: np.ndarray, w_r: np.ndarray, top_k: int):
     return idx.astype(np.int32), gp / gp.sum(axis=1, keepdims=True), z
 
 
+def with_shared_experts(idx: np.ndarray, gates: np.ndarray, n_experts: int, n_shared: int):
+    """Append the always-on shared experts to every token's routed slots.
+
+    The model card lists the MoE as 8 active experts of 128 "+1 shared": a shared expert takes
+    every token regardless of the router.  Reading taken: shared expert s is stored as expert
+    n_experts + s, enters with gate 1 (it is not router-weighted), and its slot follows the
+    routed ones (slot order k, k + 1, ...).
+    """
+    if n_shared <= 0:
+        return idx, gates
+    T = idx.shape[0]
+    ids = np.broadcast_to(np.arange(n_experts, n_experts + n_shared, dtype=np.int32), (T, n_shared))
+    return (np.concatenate([idx, ids], axis=1),
+            np.concatenate([gates, np.ones((T, n_shared))], axis=1))
+
+
 def router_margin(z: np.ndarray, top_k: int) -> np.ndarray:
     """Per token: gap between the k-th and (k+1)-th largest router logit (inf if k = E)."""
     E = z.shape[1]
@@ -426,6 +442,7 @@ def layer_rest(cfg, model: OracleModel, l: int, x, q, k, v, kc, vc, causal: bool
     if info is not None:
         info.setdefault("router_margin", []).append(router_margin(z, cfg.top_k))
         info.setdefault("router_idx", []).append(idx)
+    idx, gates = with_shared_experts(idx, gates, cfg.n_experts, getattr(cfg, "n_shared", 0))
     return moe_ffn(y, idx, gates, lambda e: model.expert(l, e), h, act)
 
 

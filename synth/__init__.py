@@ -62,6 +62,7 @@ class Cfg:
     state: str = "all_mask"  # initial canvas state: "all_mask" or "half"
     prefill_ids: bool = False  # prompt given as token ids (prefilled by the append path)
     emb: str = ""            # tied embedding / LM head storage: "" = the activation type, or "nvfp4"
+    n_shared: int = 0        # always-on shared experts, stored after the routed ones
 
     @property
     def mask_id(self) -> int:
@@ -192,11 +193,12 @@ def make_model(cfg: Cfg, device="cpu", seed: Optional[int] = None) -> dict:
         rkind = "f32" if cfg.w == "f32" else "bf16"
         lay["w_router"], _ = _store_weight(_normal(g, (cfg.n_experts, d), cfg.router_std, device), rkind)
         gus, gss, dws, dss = [], [], [], []
-        for _e in range(cfg.n_experts):
+        n_all = cfg.n_experts + cfg.n_shared   # shared experts are drawn after the routed ones
+        for _e in range(n_all):
             w, s = _store_weight(_normal(g, (2 * cfg.d_ff, d), std, device), cfg.w)
             gus.append(w)
             gss.append(s)
-        for _e in range(cfg.n_experts):
+        for _e in range(n_all):
             w, s = _store_weight(_normal(g, (d, cfg.d_ff), std, device), cfg.w)
             dws.append(w)
             dss.append(s)

@@ -311,6 +311,32 @@ def test_moe_single_expert_is_plain_gated_ffn():
             assert abs(got[t, c] - want) < 1e-12
 
 
+def test_shared_expert_adds_a_plain_gated_ffn():
+    """Routed experts with zero weights plus one shared expert: the MoE output is the residual
+    plus the shared expert's gated FFN with gate 1, whatever the router chose (torch computes
+    the FFN: gelu with the tanh approximation, float64 matmuls)."""
+    T, d, F, E, k = 7, 16, 12, 4, 2
+    y = rng.standard_normal((T, d))
+    res = rng.standard_normal((T, d))
+    w_gu = rng.standard_normal((2 * F, d)) * 0.3
+    w_d = rng.standard_normal((d, F)) * 0.3
+    zero = (np.zeros((2 * F, d)), np.zeros((d, F)))
+    idx = rng.integers(0, E, (T, k)).astype(np.int32)
+    gates = rng.uniform(0.1, 1.0, (T, k))
+    idx2, gates2 = O.with_shared_experts(idx, gates, E, 1)
+    assert idx2.shape == (T, k + 1) and (idx2[:, k] == E).all() and (gates2[:, k] == 1.0).all()
+    assert np.array_equal(idx2[:, :k], idx) and np.array_equal(gates2[:, :k], gates)
+    out = O.moe_ffn(y, idx2, gates2, lambda e: (w_gu, w_d) if e == E else zero, res, "f32")
+    yt = torch.from_numpy(y)
+    u = yt @ torch.from_numpy(w_gu).T
+    a = torch.nn.functional.gelu(u[:, :F], approximate="tanh") * u[:, F:]
+    want = torch.from_numpy(res) + a @ torch.from_numpy(w_d).T
+    np.testing.assert_allclose(out, want.numpy(), rtol=1e-12, atol=1e-12)
+    # no shared experts: unchanged routing
+    i0, g0 = O.with_shared_experts(idx, gates, E, 0)
+    assert i0 is idx and g0 is gates
+
+
 def test_moe_token_permutation_equivariance():
     T, d, F, E = 8, 10, 6, 5
     y = rng.standard_normal((T, d))
