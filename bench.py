@@ -431,7 +431,8 @@ def run_dg(args, world, rank, local):
     init = [{k: v.to(dev) for k, v in synth.make_canvas_state(cfg, s_).items()} for s_ in states]
     ns = len(init)
     st = {k: v.clone() for k, v in init[0].items()}
-    load = torch.zeros((cfg.n_layers, cfg.n_experts), dtype=torch.int32, device=dev)
+    load = torch.zeros((cfg.n_layers, cfg.n_experts + cfg.n_shared), dtype=torch.int32,
+                       device=dev)
 
     def one_step(i, stream=None, expert_load=None):
         src = init[i % ns]

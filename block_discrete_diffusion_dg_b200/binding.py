@@ -38,7 +38,7 @@ class DgConfig(ctypes.Structure):
                 ("vocab", ctypes.c_int32), ("canvas", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("rope_theta", ctypes.c_double), ("rms_eps", ctypes.c_double),
                 ("act_dtype", ctypes.c_int32), ("w_dtype", ctypes.c_int32),
-                ("emb_dtype", ctypes.c_int32)]
+                ("emb_dtype", ctypes.c_int32), ("n_shared", ctypes.c_int32)]
 
 
 class DgLayerWeights(ctypes.Structure):
@@ -131,7 +131,8 @@ def make_config(c) -> DgConfig:
     emb = DG_NVFP4 if getattr(c, "emb", "") == "nvfp4" else act
     return DgConfig(c.d_model, c.n_q_heads, c.n_kv_heads, c.head_dim, c.n_experts, c.top_k, c.d_ff,
                     c.vocab, c.canvas, c.n_layers, float(c.rope_theta), float(c.rms_eps), act,
-                    {"f32": DG_F32, "bf16": DG_BF16, "e4m3": DG_E4M3}[c.w], emb)
+                    {"f32": DG_F32, "bf16": DG_BF16, "e4m3": DG_E4M3}[c.w], emb,
+                    int(getattr(c, "n_shared", 0)))
 
 
 def make_layer(lay: dict) -> DgLayerWeights:

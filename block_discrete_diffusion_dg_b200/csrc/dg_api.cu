@@ -96,11 +96,12 @@ int router_parts(const dg_config &c, int T) {
 
 Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   const size_t T = (size_t)batch * n, a = esz(c.act_dtype);
-  const size_t d = c.d_model, hd = c.head_dim, k = c.top_k, F = c.d_ff;
+  // routing slots and experts include the shared experts
+  const size_t d = c.d_model, hd = c.head_dim, k = c.top_k + c.n_shared, F = c.d_ff;
   const size_t qkvw = (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * hd;
   const size_t TK = T * k;
   Layout L;
-  L.max_tiles = (int)((TK + min_tile_m() - 1) / min_tile_m()) + c.n_experts;
+  L.max_tiles = (int)((TK + min_tile_m() - 1) / min_tile_m()) + c.n_experts + c.n_shared;
   size_t sz[B_COUNT];
   const size_t T128 = (T + 127) / 128 * 128;  // tensor-core A operands read whole 128-row tiles
   sz[B_X] = T * d * 4;  // residual stream: fp32
@@ -116,7 +117,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_Z] = T * (size_t)c.n_experts * 4 * router_parts(c, (int)T);
   sz[B_IDX] = TK * 4;
   sz[B_W] = TK * 4;
-  sz[B_OFF] = (size_t)(c.n_experts + 1) * 4;
+  sz[B_OFF] = (size_t)(c.n_experts + c.n_shared + 1) * 4;
   sz[B_PERM] = TK * 4;
   sz[B_INV] = TK * 4;
   sz[B_TILES] = (size_t)L.max_tiles * sizeof(GroupTile);
@@ -128,7 +129,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   // e4m3 weights on the tensor-core path: bf16 copies of one layer's matrices (the expert
   // matrices are the largest; QKV and the output projection reuse the front of the region)
   sz[B_WDQ] = c.w_dtype == DG_E4M3
-                  ? ((size_t)c.n_experts * 3 * F * d +
+                  ? ((size_t)(c.n_experts + c.n_shared) * 3 * F * d +
                      (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * hd * d) * 2
                   : 0;
   sz[B_LIVE] = T;
@@ -167,6 +168,8 @@ bool cfg_ok(const dg_config *c) {
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return false;
   if (c->n_experts <= 0 || c->n_experts > 256 || c->top_k <= 0 || c->top_k > c->n_experts ||
       c->top_k > 32)
+    return false;
+  if (c->n_shared < 0 || c->n_experts + c->n_shared > 256 || c->top_k + c->n_shared > 32)
     return false;
   if (c->d_ff <= 0 || c->d_ff % 8 || c->vocab < 2 || c->canvas <= 0 || c->canvas > 1024)
     return false;
@@ -308,16 +311,17 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
                         ws.at<int32_t>(B_IDX), ws.at<float>(B_W), ws.at<int32_t>(B_OFF),
                         ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV),
                         tc ? experts_tc_tile_tokens() : SIMT_TILE_M, ws.at<GroupTile>(B_TILES),
-                        ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s, forced, rp));
+                        ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s, forced, rp,
+                        c.n_shared));
     *tiles_ready = true;
     return DG_OK;
   }
   if (forced) return DG_ERR_UNSUPPORTED;  // forced routing needs the tensor-core router
   DG_TRY(launch_router(c.act_dtype, router_type(&c), T, d, c.n_experts, c.top_k,
                        ws.at<void>(B_Y), w.w_router, token_live, ws.at<int32_t>(B_IDX),
-                       ws.at<float>(B_W), s));
-  return launch_permute(T, c.top_k, c.n_experts, ws.at<int32_t>(B_IDX), ws.at<int32_t>(B_OFF),
-                        ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV), s);
+                       ws.at<float>(B_W), s, c.n_shared));
+  return launch_permute(T, c.top_k + c.n_shared, c.n_experts + c.n_shared, ws.at<int32_t>(B_IDX),
+                        ws.at<int32_t>(B_OFF), ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV), s);
 }
 
 // The expert FFN, then combine + residual into `out`; the combine also writes RMSNorm(out) to
@@ -328,7 +332,8 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
                 const void *residual, void *out, cudaStream_t s, bool tiles_ready = false,
                 int32_t *load_out = nullptr, void *a_out = nullptr,
                 const int32_t *slot = nullptr, void *f_out = nullptr) {
-  const int d = c.d_model, F = c.d_ff, E = c.n_experts, k = c.top_k;
+  // every slot, the shared experts' included (experts n_experts .. n_experts + n_shared - 1)
+  const int d = c.d_model, F = c.d_ff, E = c.n_experts + c.n_shared, k = c.top_k + c.n_shared;
   const int TK = T * k;
   const bool tc = experts_tc(c);
   if (!tiles_ready)
@@ -597,13 +602,13 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
     DG_TRY(launch_gemm_tc_dense(w.at<void>(B_Y), n_tokens, w_router, E, d, w.at<float>(B_Z), nullptr,
                                 E, "router_logits_tc", nullptr, s));
     DG_TRY(launch_router_topk(n_tokens, E, cfg->top_k, w.at<float>(B_Z), token_live, topk_idx,
-                              topk_w, s));
+                              topk_w, s, nullptr, 1, cfg->n_shared));
   } else {
     DG_TRY(launch_router(cfg->act_dtype, router_type(cfg), n_tokens, d, E, cfg->top_k, y,
-                         w_router, token_live, topk_idx, topk_w, s));
+                         w_router, token_live, topk_idx, topk_w, s, cfg->n_shared));
   }
-  return launch_permute(n_tokens, cfg->top_k, cfg->n_experts, topk_idx, expert_off, perm,
-                        inv_perm, s);
+  return launch_permute(n_tokens, cfg->top_k + cfg->n_shared, cfg->n_experts + cfg->n_shared,
+                        topk_idx, expert_off, perm, inv_perm, s);
 }
 
 int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t *topk_idx,
@@ -760,7 +765,7 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                             w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
                             w.at<void>(B_VN), 0, done, w.at<void>(B_O), w.at<void>(B_ATTN),
                             dev_status, s));
-    int32_t *load_l = expert_load ? expert_load + (size_t)l * c.n_experts : nullptr;
+    int32_t *load_l = expert_load ? expert_load + (size_t)l * (c.n_experts + c.n_shared) : nullptr;
     bool tiles_ready = false;
     DG_TRY(attn_out_and_route(c, lw, w, T, live, load_l, &tiles_ready, s,
                               forced_topk ? forced_topk + (size_t)l * T * c.top_k : nullptr));

@@ -91,21 +91,23 @@ int launch_attention_tc(int batch, int n, int Hq, int Hkv, int hd, const void *q
                         void *out, void *ws, int32_t *st, cudaStream_t s);
 
 // ---- MoE (k_moe.cu) ---------------------------------------------------------------------------
+// n_shared: shared experts E .. E + n_shared - 1 appended to every live token's slots (gate 1);
+// the outputs are then [T][k + n_shared].
 int launch_router(int act, int wr_type, int T, int d, int E, int k, const void *y,
                   const void *w_router, const uint8_t *token_live, int32_t *topk_idx,
-                  float *topk_w, cudaStream_t s);
+                  float *topk_w, cudaStream_t s, int n_shared = 0);
 // Top-k + gates from fp32 router logits z [T][E] (E <= 256, k <= 32), one warp per token.
 int launch_router_topk(int T, int E, int k, const float *z, const uint8_t *token_live,
                        int32_t *topk_idx, float *topk_w, cudaStream_t s,
                        const int32_t *forced = nullptr,
-                       int n_parts = 1);
+                       int n_parts = 1, int n_shared = 0);
 // Top-k + gates (router_topk, many blocks), then the stable permutation and the tile list in one
 // block (permute_tiles).
 int launch_route(int T, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
                  cudaStream_t s, const int32_t *forced = nullptr,
-                 int n_parts = 1);
+                 int n_parts = 1, int n_shared = 0);
 // Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
 int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s);

@@ -17,7 +17,7 @@ namespace {
 constexpr int ROUTER_TPB = 4;  // tokens per router block
 
 template <typename T, typename WT>
-__global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__ y,
+__global__ void router_kernel(int T_, int d, int E, int k, int S, const T *__restrict__ y,
                               const WT *__restrict__ wr, const uint8_t *__restrict__ token_live,
                               int32_t *topk_idx, float *topk_w) {
   pdl_wait();
@@ -73,12 +73,17 @@ __global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__
       const float p = expf(bv - zsel0);
       denom += p;
       if (lane == 0) {
-        topk_idx[(size_t)t * k + j] = live ? bi : -1;
-        topk_w[(size_t)t * k + j] = p;  // normalised below
+        topk_idx[(size_t)t * (k + S) + j] = live ? bi : -1;
+        topk_w[(size_t)t * (k + S) + j] = p;  // normalised below
       }
     }
     __syncwarp();
-    if (lane < k) topk_w[(size_t)t * k + lane] = live ? topk_w[(size_t)t * k + lane] / denom : 0.f;
+    if (lane < k)
+      topk_w[(size_t)t * (k + S) + lane] = live ? topk_w[(size_t)t * (k + S) + lane] / denom : 0.f;
+    if (lane < S) {  // shared experts: every live token, gate 1, after the routed slots
+      topk_idx[(size_t)t * (k + S) + k + lane] = live ? E + lane : -1;
+      topk_w[(size_t)t * (k + S) + k + lane] = live ? 1.f : 0.f;
+    }
   }
 }
 
@@ -88,8 +93,8 @@ __global__ void router_kernel(int T_, int d, int E, int k, const T *__restrict__
 // the k largest logits; the gates are still the softmax over the selected logits.
 // z may hold n_parts fp32 partial sums [n_parts][T][E] (split-K router logits), added in order.
 
-__global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict__ z, int n_parts,
-                                   const uint8_t *__restrict__ token_live,
+__global__ void router_topk_kernel(int T_, int E, int k, int S, const float *__restrict__ z,
+                                   int n_parts, const uint8_t *__restrict__ token_live,
                                    const int32_t *__restrict__ forced, int32_t *topk_idx,
                                    float *topk_w) {
   pdl_wait();
@@ -114,8 +119,12 @@ __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
     if (lane < k) {
-      topk_idx[(size_t)t * k + lane] = (live && ok) ? e : -1;
-      topk_w[(size_t)t * k + lane] = (live && ok) ? p / denom : 0.f;
+      topk_idx[(size_t)t * (k + S) + lane] = (live && ok) ? e : -1;
+      topk_w[(size_t)t * (k + S) + lane] = (live && ok) ? p / denom : 0.f;
+    }
+    if (lane < S) {  // shared experts: every live token, gate 1, after the routed slots
+      topk_idx[(size_t)t * (k + S) + k + lane] = live ? E + lane : -1;
+      topk_w[(size_t)t * (k + S) + k + lane] = live ? 1.f : 0.f;
     }
     return;
   }
@@ -153,8 +162,12 @@ __global__ void router_topk_kernel(int T_, int E, int k, const float *__restrict
     if (lane == j) { mine = p; my_idx = bi; }
   }
   if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = live ? my_idx : -1;
-    topk_w[(size_t)t * k + lane] = live ? mine / denom : 0.f;
+    topk_idx[(size_t)t * (k + S) + lane] = live ? my_idx : -1;
+    topk_w[(size_t)t * (k + S) + lane] = live ? mine / denom : 0.f;
+  }
+  if (lane < S) {  // shared experts: every live token, gate 1, after the routed slots
+    topk_idx[(size_t)t * (k + S) + k + lane] = live ? E + lane : -1;
+    topk_w[(size_t)t * (k + S) + k + lane] = live ? 1.f : 0.f;
   }
 }
 
@@ -652,8 +665,9 @@ int launch_combine_norm(int act, int T_, int d, int k, double eps, const int32_t
 
 int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void *y,
                   const void *w_router, const uint8_t *token_live, int32_t *topk_idx,
-                  float *topk_w, cudaStream_t s) {
+                  float *topk_w, cudaStream_t s, int n_shared) {
   if (T_ <= 0) return DG_OK;
+  if (n_shared < 0 || k + n_shared > 32) return DG_ERR_UNSUPPORTED;
   const int threads = E < 32 ? 32 : (E > 256 ? 256 : ((E + 31) / 32) * 32);
   const size_t smem = sizeof(float) * ROUTER_TPB * (size_t)(d + E);
   const int grid = (T_ + ROUTER_TPB - 1) / ROUTER_TPB;
@@ -661,13 +675,13 @@ int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void 
     auto kf = router_kernel<float, float>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     note_launch(s, "router");
-    launch_pdl(kf, grid, threads, smem, s, T_, d, E, k, (const float *)y, (const float *)w_router,
+    launch_pdl(kf, grid, threads, smem, s, T_, d, E, k, n_shared, (const float *)y, (const float *)w_router,
                                    token_live, topk_idx, topk_w);
   } else if (act == DG_BF16 && wr_type == DG_BF16) {
     auto kb = router_kernel<bf16, bf16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     note_launch(s, "router");
-    launch_pdl(kb, grid, threads, smem, s, T_, d, E, k, (const bf16 *)y, (const bf16 *)w_router,
+    launch_pdl(kb, grid, threads, smem, s, T_, d, E, k, n_shared, (const bf16 *)y, (const bf16 *)w_router,
                                    token_live, topk_idx, topk_w);
   } else {
     return DG_ERR_UNSUPPORTED;
@@ -677,29 +691,31 @@ int launch_router(int act, int wr_type, int T_, int d, int E, int k, const void 
 
 int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *token_live,
                        int32_t *topk_idx, float *topk_w, cudaStream_t s, const int32_t *forced,
-                       int n_parts) {
+                       int n_parts, int n_shared) {
   if (T_ <= 0) return DG_OK;
-  if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
+  if (E > 256 || n_shared < 0 || k + n_shared > 32) return DG_ERR_UNSUPPORTED;
   note_launch(s, "router_topk");
-  launch_pdl(router_topk_kernel, (T_ + 7) / 8, 256, 0, s, T_, E, k, z, n_parts, token_live, forced,
-                                                  topk_idx, topk_w);
+  launch_pdl(router_topk_kernel, (T_ + 7) / 8, 256, 0, s, T_, E, k, n_shared, z, n_parts,
+             token_live, forced, topk_idx, topk_w);
   return check_launch("router_topk");
 }
 
 int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
-                 cudaStream_t s, const int32_t *forced, int n_parts) {
+                 cudaStream_t s, const int32_t *forced, int n_parts, int n_shared) {
   if (T_ <= 0) return DG_OK;
-  if (E > 256 || k > 32) return DG_ERR_UNSUPPORTED;
-  const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced, n_parts);
+  const int ka = k + n_shared, Ea = E + n_shared;  // slots and experts with the shared ones
+  if (Ea > 256 || n_shared < 0 || ka > 32) return DG_ERR_UNSUPPORTED;
+  const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced, n_parts,
+                                    n_shared);
   if (rc != DG_OK) return rc;
   note_launch(s, "permute_tiles");
-  if (T_ * k <= 2048)
-    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, T_ * k, E, topk_idx, expert_off, perm,
+  if (T_ * ka <= 2048)
+    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
                inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
   else
-    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, T_ * k, E, topk_idx, expert_off, perm,
+    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
                inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
   return check_launch("permute_tiles");
 }

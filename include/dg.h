@@ -80,14 +80,17 @@ typedef struct dg_config {
   int32_t w_dtype;   /* DG_F32 (with act F32), DG_BF16 or DG_E4M3 (with act BF16) */
   int32_t emb_dtype; /* the tied embedding / LM head: act_dtype, or DG_NVFP4 (with act BF16,
                         d_model a multiple of 256, at most 4096) */
+  int32_t n_shared;  /* always-on shared experts S >= 0 (the model card's MoE "+1 shared"):
+                        experts E .. E + S - 1 of the expert arrays take every live token with
+                        gate 1, in the slots after its k routed ones; E + S <= 256, k + S <= 32 */
 } dg_config;
 
 /* One layer's weights (device pointers).  Every matrix is [out][in], `in` contiguous.
  *   w_qkv     [(Hq + 2 Hkv) hd][d]   rows: q heads, then k heads, then v heads
  *   w_o       [d][Hq hd]
  *   w_router  [E][d]                 BF16 (F32 when w_dtype is F32), never E4M3
- *   w_gate_up [E][2F][d]             rows [0,F) gate, [F,2F) up
- *   w_down    [E][d][F]
+ *   w_gate_up [E + S][2F][d]         rows [0,F) gate, [F,2F) up (S = n_shared: the shared
+ *   w_down    [E + S][d][F]          experts after the E routed ones)
  * s_* : fp32 per-output-channel scales, required for E4M3 and ignored otherwise. */
 typedef struct dg_layer_weights {
   const void *w_qkv;     const float *s_qkv;
@@ -163,9 +166,10 @@ int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
  * z = y W_r^T (fp32), p = softmax(z) over all E, the k largest p (lower expert index first on
  * equal values), renormalised to sum 1.  Then assignments (t, j) are grouped by expert,
  * stable in (t, j) order:
- *   y [T][d]; topk_idx int32 [T][k]; topk_w fp32 [T][k]; expert_off int32 [E + 1]
- *   (exclusive prefix of per-expert counts); perm int32 [T k]: perm[p] = t k + j of the
- *   assignment at permuted position p; inv_perm int32 [T k]: the inverse.
+ *   y [T][d]; topk_idx int32 [T][k + S]; topk_w fp32 [T][k + S] (S = n_shared: slots
+ *   k .. k + S - 1 hold the shared experts E .. E + S - 1 with weight 1); expert_off int32
+ *   [E + S + 1] (exclusive prefix of per-expert counts); perm int32 [T (k + S)]: perm[p] =
+ *   t (k + S) + j of the assignment at permuted position p; inv_perm: the inverse.
  *   token_live: device uint8 [T] or NULL; a token with token_live[t] == 0 gets no experts
  *   (topk_idx = -1, weight 0) and no assignments. */
 int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *w_router,
@@ -176,7 +180,8 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
 /* Expert FFN with combine and residual (same passages).  For assignment (t, j) with expert e:
  *   [g; u] = y_t W_gu,e^T ; a = gelu_tanh(g) * u (stored in the activation type) ;
  *   Y = a W_d,e^T (fp32) ;
- *   out_t = residual_t + sum_j topk_w[t][j] Y_(t,j), summed in fp32 in slot order j = 0..k-1.
+ *   out_t = residual_t + sum_j topk_w[t][j] Y_(t,j), summed in fp32 in slot order
+ *   j = 0 .. k + S - 1 (the shared experts' slots last, weight 1).
  * Routing arrays as produced by dg_moe_route.  y [T][d] in the activation type; residual and
  * out [T][d] fp32 (out may not alias y; it may alias residual). */
 int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t *topk_idx,
@@ -256,7 +261,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
  * entropy_out fp32 [B][C], argmax_out int32 [B][C] (or NULL): written at the positions that
  * were masked when the step began.  logits_dbg (or NULL): fp32 [B C][V], row b C + i written for
  * each such position (debug and parity only; costs a full logits write).  expert_load (or
- * NULL): int32 [n_layers][E], the number of (token, slot) assignments each expert received in
+ * NULL): int32 [n_layers][E + S], the number of (token, slot) assignments each expert received in
  * each layer this step (for load monitoring and byte accounting).  forced_topk (or NULL):
  * int32 [n_layers][B C][k] expert ids that replace each layer's router top-k choice (the gates
  * are still the softmax of this step's router logits over the given experts).  It lets a caller

@@ -114,24 +114,35 @@ def _rms_rows(T, d, gen, scale=1.0):
     return y.float().to(torch.bfloat16)
 
 
-def test_router_parity_and_permutation(cfg, gen):
+@pytest.mark.parametrize("S", [0, 1])
+def test_router_parity_and_permutation(cfg, gen, S):
+    """Router top-k and the stable permutation; with S = 1 a shared expert (id E, gate 1) fills
+    the last slot of every live token and takes part in the grouping."""
+    cfg = dataclasses.replace(cfg, n_shared=S)
     T, d, E, k = 300, cfg.d_model, cfg.n_experts, cfg.top_k
     y = _rms_rows(T, d, gen)
     wr = (torch.randn((E, d), generator=gen) * 0.02).to(torch.bfloat16)
     live = (torch.rand(T, generator=gen) < 0.9).to(torch.uint8)
     dgc = B.make_config(cfg)
-    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
-    gw = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
-    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
-    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    ka = k + S
+    idx = torch.empty((T, ka), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, ka), dtype=torch.float32, device="cuda")
+    off = torch.empty(E + S + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * ka, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * ka, dtype=torch.int32, device="cuda")
     B.dg_moe_route(dgc, T, y.cuda(), wr.cuda(), live.cuda(), idx, gw, off, perm, inv,
                    B.alloc_workspace(dgc, 1, T, 0))
     torch.cuda.synchronize()
     idx, gw, off, perm, inv = (t.cpu().numpy() for t in (idx, gw, off, perm, inv))
+    lv = live.numpy().astype(bool)
+    if S:
+        assert (idx[lv, k] == E).all() and (gw[lv, k] == 1.0).all()
+        assert (idx[~lv, k] == -1).all() and (gw[~lv, k] == 0).all()
+        full_idx, idx, gw = idx, idx[:, :k], gw[:, :k]
+    else:
+        full_idx = idx
     o_idx, o_g, z = O.router_topk(dec(y), dec(wr), k)
     margin = O.router_margin(z, k)
-    lv = live.numpy().astype(bool)
     assert (idx[~lv] == -1).all() and (gw[~lv] == 0).all()
     # the order within the top-k is by probability, so every adjacent pair is a decision too
     zs = -np.sort(-z, axis=1)
@@ -142,9 +153,9 @@ def test_router_parity_and_permutation(cfg, gen):
     np.testing.assert_allclose(gw[safe], o_g[safe], rtol=2e-5, atol=1e-6)
     np.testing.assert_allclose(gw[lv].sum(1), 1.0, rtol=1e-5)
     # permutation: stable grouping of the live assignments by expert
-    flat = idx.reshape(-1)
+    flat = full_idx.reshape(-1)
     valid = np.nonzero(flat >= 0)[0]
-    counts = np.bincount(flat[valid], minlength=E)
+    counts = np.bincount(flat[valid], minlength=E + S)
     assert (off == np.concatenate([[0], np.cumsum(counts)])).all()
     want = valid[np.argsort(flat[valid], kind="stable")]
     assert (perm[:len(valid)] == want).all()
@@ -362,12 +373,15 @@ def _step_compare(wl, st_np, check_eb=True):
     return new_np, n_tie
 
 
-@pytest.mark.parametrize("name,batch", [("layer", 1), ("batch32", 2), ("layer_nvfp4", 1)])
+@pytest.mark.parametrize("name,batch", [("layer", 1), ("batch32", 2), ("layer_nvfp4", 1),
+                                        ("layer+shared", 2)])
 def test_step_parity_reduced(name, batch):
     # the NVFP4 case draws its router with std 1/sqrt(d) (as the batch-32 workload does): with
     # 0.02 its all-MASK rows put 68 of 192 router decisions within the near-tie margin, which
     # leaves too few rows to compare (39 for the bf16 layer, 28 with this router)
     over = {"router_std": 1.0 / 16.0} if name == "layer_nvfp4" else {}
+    if name == "layer+shared":  # one always-on shared expert next to the 16 routed ones
+        name, over = "layer", {"n_shared": 1}
     cfg = synth.reduced(name, batch=batch, **over)
     wl = Workload(cfg, gen_device="cpu", state_kind="all_mask")
     st = np_state(wl.state)
@@ -426,7 +440,9 @@ def test_kv_append_parity_two_layers(emb):
     # prefill 64 random prompt ids first, then append one canvas of 64
     wl.kv["cache_len"].zero_()
     toks1 = wl.kv["prompt_ids"][:, :64].contiguous()
-    toks2 = torch.randint(0, cfg.vocab, (1, cfg.canvas), dtype=torch.int32).cuda()
+    tg = torch.Generator()
+    tg.manual_seed(7)   # the appended canvas's tokens: seeded, not the process-wide generator
+    toks2 = torch.randint(0, cfg.vocab, (1, cfg.canvas), dtype=torch.int32, generator=tg).cuda()
     for toks in (toks1, toks2):
         B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, toks, toks.shape[1], kc, vc, wl.kv["cache_len"],
                        wl.cap, wl.ws, wl.status)
