@@ -77,6 +77,65 @@ def test_host_side_argument_rejection_launches_nothing():
     assert L.dg_launch_count() == n0
 
 
+def test_new_config_fields_and_entry_points_reject_on_the_host():
+    """NVFP4 LM head, shared experts and dg_generate: invalid configurations and arguments are
+    refused before any launch (no GPU needed)."""
+    L = B.lib()
+    n0 = L.dg_launch_count()
+    # NVFP4 needs bf16 activations and d_model a multiple of 256 (at most 4096)
+    ok = B.make_config(synth.reduced("layer_nvfp4"))
+    assert B.dg_workspace_size(ok, 1, 64, 256) > 0
+    bad = B.make_config(synth.reduced("layer_nvfp4"))
+    bad.d_model = 320
+    assert B.dg_workspace_size(bad, 1, 64, 256) == 0
+    bad = B.make_config(synth.get_config("layer_nvfp4"))
+    bad.d_model = 8192
+    assert B.dg_workspace_size(bad, 1, 64, 256) == 0
+    bad = B.make_config(synth.get_config("tiny"))
+    bad.emb_dtype = B.DG_NVFP4
+    assert B.dg_workspace_size(bad, 1, 16, 64) == 0
+    # the bf16 LM-head entry point refuses an NVFP4 config; the NVFP4 one a bf16 config and a
+    # non-positive tensor scale
+    assert L.dg_logits_entropy(ctypes.byref(ok), 4, None, 8, None, 8, 8, 8, None, 256, 1 << 30,
+                               None, None) == B.DG_ERR_INVALID_ARG
+    bf = B.make_config(synth.reduced("layer"))
+    assert L.dg_logits_entropy_nvfp4(ctypes.byref(bf), 4, None, 8, None, 16, 16, 1.0, 8, 8, None,
+                                     256, 1 << 30, None, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_logits_entropy_nvfp4(ctypes.byref(ok), 4, None, 8, None, 16, 16, 0.0, 8, 8, None,
+                                     256, 1 << 30, None, None) == B.DG_ERR_INVALID_ARG
+    # shared experts: n_shared >= 0, E + S <= 256, k + S <= 32; the scratch grows with them
+    sh = B.make_config(synth.reduced("layer", n_shared=1))
+    base = B.make_config(synth.reduced("layer"))
+    assert B.dg_workspace_size(sh, 1, 64, 256) > B.dg_workspace_size(base, 1, 64, 256)
+    for field, val in (("n_shared", -1), ("n_shared", 241)):
+        bad = B.make_config(synth.reduced("layer"))
+        setattr(bad, field, val)
+        assert B.dg_workspace_size(bad, 1, 64, 256) == 0
+    bad = B.make_config(synth.reduced("layer"))
+    bad.top_k, bad.n_shared = 16, 17
+    assert B.dg_workspace_size(bad, 1, 64, 256) == 0
+    # dg_generate: no model, zero max_steps, negative gamma, append without a cache (a model
+    # struct of placeholder pointers passes the null checks; nothing is dereferenced on the host)
+    cfg = B.make_config(synth.get_config("tiny"))
+    lw = (B.DgLayerWeights * 1)(B.DgLayerWeights(8, None, 8, None, 8, 8, None, 8, None))
+    model = B.DgModel(ctypes.cast(lw, ctypes.POINTER(B.DgLayerWeights)), 8, None, 1.0)
+    # tokens, masked, n_masked, done, step, max_steps, gamma, k, v, cache_len, cache_cap,
+    # append, ws, ws_bytes, dev_status, stream
+    args = [8, 8, 8, 8, 8, 16, 0.1, 8, 8, 8, 64, 0, 256, 1 << 30, None, None]
+    assert L.dg_generate(ctypes.byref(cfg), None, 1, *args) == B.DG_ERR_INVALID_ARG
+    for i, v in ((5, 0), (6, -1.0), (6, math.nan)):
+        a2 = list(args)
+        a2[i] = v
+        assert L.dg_generate(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
+    a2 = list(args)
+    a2[10], a2[11] = 0, 1          # append with no cache
+    assert L.dg_generate(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
+    a2 = list(args)
+    a2[12] = 257                   # misaligned scratch
+    assert L.dg_generate(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
+    assert L.dg_launch_count() == n0
+
+
 def test_binding_refuses_host_tensors():
     import torch
     with pytest.raises(ValueError):
