@@ -191,6 +191,34 @@ def test_stack_prefill_denoise_append_two_layers():
     assert good, stat
 
 
+def test_prefill_one_call_of_1024_tokens_two_layers():
+    """A long prompt prefilled by one dg_kv_append of 1024 tokens (four canvases' worth): causal
+    attention over the whole chunk, the expert GEMMs beyond the 256-token split-K path and the
+    2048-assignment permutation; caches against the oracle's append of the same ids (full width,
+    2 layers, the oracle's expert choices handed to the device as in the other stack tests)."""
+    n = 1024
+    cfg = synth.get_config("stack30", n_layers=2, prompt_len=n, n_canvases=1)
+    wl = Workload(cfg, gen_device="cuda")
+    om = wl.oracle()
+    ids = wl.kv["prompt_ids"][:, :n].contiguous()
+    ws = B.alloc_workspace(wl.dgcfg, 1, n, wl.cap)
+    k_dev, v_dev, len_dev = wl.kv["k"], wl.kv["v"], wl.kv["cache_len"]
+    ok = np.zeros(decode_cache(cfg, k_dev).shape)
+    ov = np.zeros_like(ok)
+    info = {}
+    ln = O.kv_append(cfg, om, ids.cpu().numpy(), ok, ov, np.zeros(1, np.int32), info)
+    forced = torch.from_numpy(np.stack([r.reshape(-1, cfg.top_k) for r in info["router_idx"]])).cuda()
+    B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, ids, n, k_dev, v_dev, len_dev, wl.cap, ws, wl.status,
+                   forced_topk=forced)
+    torch.cuda.synchronize()
+    wl.check_status()
+    assert int(len_dev.item()) == ln[0] == n
+    for name, dev, orc in (("k", k_dev, ok), ("v", v_dev, ov)):
+        g = decode_cache(cfg, dev)[:, :, :, :n, :]
+        good, stat = kv_close(g, orc[:, :, :, :n, :], cfg.n_layers)
+        assert good, (name, stat)
+
+
 def test_stack30_generate_invariants():
     """The full 30-layer workload: prefill, 4 canvases of at most 32 steps, appends."""
     cfg = synth.get_config("stack30")
