@@ -395,6 +395,38 @@ def _golden_eb():
     return cases
 
 
+
+def test_eb_fixed_point_quantisers_exact_rational():
+    """Q(H) = nearest integer to H 2^32 (ties to even) and Q(gamma) = floor(gamma 2^32), checked
+    with exact rational arithmetic on the binary values (fractions.Fraction)."""
+    from fractions import Fraction
+    g = np.random.default_rng(11)
+    hs = np.concatenate([g.uniform(0, 20, 500), [0.0, 2.0 ** -33, 3 * 2.0 ** -33, 12.5,
+                                                 np.float32(0.1), np.float32(math.log(262144))]])
+    for h in hs.astype(np.float32):
+        exact = Fraction(float(h)) * 2 ** 32
+        fl = exact.numerator // exact.denominator
+        rem = exact - fl
+        want = fl + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1) else 0)
+        assert O.eb_quantize(float(h)) == want
+    # ties: 2^-33 is exactly half a unit (rounds to even 0), 3 * 2^-33 is 1.5 units (rounds to 2)
+    assert O.eb_quantize(2.0 ** -33) == 0 and O.eb_quantize(3 * 2.0 ** -33) == 2
+    for gm in list(g.uniform(0, 50, 200)) + [0.0, 1.0, 0.1, 1e-12]:
+        exact = Fraction(float(gm)) * 2 ** 32
+        assert O.eb_quantize_bound(gm) == exact.numerator // exact.denominator
+    assert O.eb_quantize_bound(math.inf) == np.iinfo(np.int64).max
+
+
+def test_router_margin_brute_force():
+    g = np.random.default_rng(12)
+    z = g.standard_normal((40, 9))
+    for k in (1, 3, 8):
+        m = O.router_margin(z, k)
+        for t in range(z.shape[0]):
+            srt = sorted(z[t], reverse=True)
+            assert m[t] == srt[k - 1] - srt[k]
+    assert np.isinf(O.router_margin(z, 9)).all()
+
 @pytest.mark.parametrize("case", _golden_eb())
 def test_eb_hand_worked(case):
     gamma, H, masked, want = case
