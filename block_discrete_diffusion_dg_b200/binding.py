@@ -249,6 +249,8 @@ def dg_logits_entropy_static(cfg, n_rows, n_rows_dev, h, row_idx, w_lm, entropy,
 
 def dg_logits_entropy_nvfp4(cfg, n_rows, n_rows_dev, h, row_idx, w_codes, w_scale, w_scale_global,
                             entropy, argmax, logits_dbg, ws, dev_status=None, stream=None):
+    """dg_logits_entropy with the LM head in NVFP4: uint8 codes [d/64][Vp][32], uint8 E4M3
+    scales [d/64][Vp][4] and the fp32 tensor scale (cfg.emb_dtype must be DG_NVFP4)."""
     w, wb = _ws(ws)
     _check(lib().dg_logits_entropy_nvfp4(ctypes.byref(cfg), n_rows, _p(n_rows_dev), _p(h),
                                          _p(row_idx), _p(w_codes), _p(w_scale),
@@ -287,6 +289,8 @@ def dg_canvas_step(cfg, model: Model, batch, tokens, masked, n_masked, done, ste
 
 def dg_generate(cfg, model: Model, batch, tokens, masked, n_masked, done, step, max_steps, gamma,
                 k_cache, v_cache, cache_len, cache_cap, append, ws, dev_status=None, stream=None):
+    """The step loop on the device until every canvas is done (one CUDA graph with a
+    conditional while node, cached per argument set), then the append if `append`."""
     w, wb = _ws(ws)
     _check(lib().dg_generate(ctypes.byref(cfg), ctypes.byref(model.struct), batch, _p(tokens),
                              _p(masked), _p(n_masked), _p(done), _p(step), max_steps, float(gamma),
