@@ -30,7 +30,7 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-__all__ = ["Cfg", "CONFIGS", "get_config", "make_model", "make_prompt_kv",
+__all__ = ["Cfg", "WORKLOADS", "get_config", "make_model", "make_prompt_kv",
            "make_canvas_state", "to_numpy", "reduced"]
 
 
@@ -77,7 +77,7 @@ class Cfg:
         return self.prompt_len + self.n_canvases * self.canvas
 
 
-CONFIGS: Dict[str, Cfg] = {
+WORKLOADS: Dict[str, Cfg] = {
     "tiny": Cfg("tiny", 64, 2, 1, 32, 8, 2, 128, 512, 16, 1, "f32", "f32", 1, 32,
                 0.1, 16, 2, 0),
     "layer": Cfg("layer", 2048, 16, 8, 128, 128, 8, 768, 262144, 256, 1, "bf16", "bf16",
@@ -102,7 +102,7 @@ NVFP4_ROW_PAD = 256
 
 
 def get_config(name: str, **overrides) -> Cfg:
-    return dataclasses.replace(CONFIGS[name], **overrides)
+    return dataclasses.replace(WORKLOADS[name], **overrides)
 
 
 def reduced(name: str, **overrides) -> Cfg:
@@ -111,7 +111,7 @@ def reduced(name: str, **overrides) -> Cfg:
     Keeps head_dim, head counts, top_k and the storage types (so the same kernel
     code paths run) but shrinks the dims the oracle pays for.
     """
-    base = CONFIGS[name]
+    base = WORKLOADS[name]
     small = dict(d_model=256, n_experts=16, d_ff=128, vocab=4096, canvas=64,
                  prompt_len=192, name=base.name + "-reduced")
     small.update(overrides)
