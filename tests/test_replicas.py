@@ -82,3 +82,20 @@ def test_reference_arm_under_torchrun_two_ranks(tmp_path):
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 2
     assert d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+
+
+def test_step_byte_accounting_by_weight_format():
+    """The step roofline's bytes: the LM head is V d bytes x 2 in bf16 and V d x 9/16 in NVFP4
+    (half a byte per code plus one E4M3 scale per 16); experts count only those touched, shared
+    experts included through the routing counts."""
+    import bench
+    import synth
+    lay = synth.get_config("layer")
+    q4 = synth.get_config("layer_nvfp4")
+    a, b = bench.step_bytes(lay, 28.0), bench.step_bytes(q4, 28.0)
+    V, d = lay.vocab, lay.d_model
+    assert a["lm_head"] == V * d * 2 and b["lm_head"] == V * d * 9 / 16
+    assert a["experts"] == b["experts"] == 28.0 * 3 * lay.d_ff * d * 2
+    assert a["total"] - b["total"] == (V * d * 2 - V * d * 9 / 16) + lay.canvas * d * (2 - 9 / 16)
+    f = bench.step_flops(lay, 256.0)
+    assert f["lm_head"] == 2 * 256 * d * V
