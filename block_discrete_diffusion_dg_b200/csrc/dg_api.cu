@@ -161,6 +161,9 @@ struct Ws {
   template <typename P> P *at(Buf b) const { return reinterpret_cast<P *>(base + L->off[b]); }
 };
 
+}  // namespace
+
+// Shape and dtype checks shared by every entry point (declared in dg_kernels.h).
 bool cfg_ok(const dg_config *c) {
   if (!c) return false;
   if (c->d_model <= 0 || c->d_model % 8 || c->n_q_heads <= 0 || c->n_kv_heads <= 0) return false;
@@ -180,6 +183,8 @@ bool cfg_ok(const dg_config *c) {
   if (c->emb_dtype == DG_NVFP4) return c->d_model % 256 == 0 && c->d_model <= 4096;
   return c->emb_dtype == DG_BF16;
 }
+
+namespace {
 
 // The tied embedding / LM head as the calls take it.
 struct LmWeights {

@@ -187,6 +187,8 @@ namespace dg {
 // timing event on `s` before the launch, labelled `name`).
 void note_launch(cudaStream_t s, const char *name);
 int check_launch(const char *what);      // DG_OK or DG_ERR_CUDA (records the message)
+// Shape and dtype checks of a dg_config that every entry point runs before any launch.
+bool cfg_ok(const dg_config *c);
 // Whether launches of this thread carry programmatic stream serialisation (on by default; off
 // while a step is captured into a graph body that may not take programmatic edges).
 bool &pdl_allowed();

@@ -34,7 +34,10 @@
  *     the expert FFN) is fp32 for every activation type; the tensors that feed a matrix product
  *     or the attention (normalised rows, q, k, v, attention output, expert activations) are in
  *     the activation type.
- *   - Functions are stateless and may be called from several host threads on different streams.
+ *   - Calls keep no state between them and may be made from several host threads on different
+ *     streams, with two exceptions, documented at their declarations: dg_generate keeps the
+ *     CUDA graphs it instantiates (a bounded cache), and dg_logits_entropy_static keeps its
+ *     scratch in one fixed device array shared by all its calls.
  */
 #ifndef DG_H
 #define DG_H
@@ -154,7 +157,11 @@ const char *dg_profile_name(int i);
  *   q      [B][n_tokens][Hq][hd]        k_cache, v_cache [B][Hkv][cache_cap][hd] (one layer)
  *   k_new, v_new [B][Hkv][n_tokens][hd] out [B][n_tokens][Hq][hd]
  *   cache_len: device int32[B], each <= cache_cap.  done: device int32[B] or NULL; canvases
- *   with done[b] != 0 are skipped (their `out` rows are left as they were). */
+ *   with done[b] != 0 are skipped (their `out` rows are left as they were).
+ * Range: with bf16 activations the tensor-core kernels (head_dim 64 and 128) convert V to fp16
+ *   for the P V product; every bf16 value of magnitude below 65520 is exact there, larger ones
+ *   become +-inf and make the affected outputs non-finite.  Keep |v| < 65520 (K and q have no
+ *   such limit). */
 int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
                    const void *k_cache, const void *v_cache, const int32_t *cache_len,
                    int cache_cap, const void *k_new, const void *v_new, int causal,
@@ -309,8 +316,13 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
  *   Limits: bf16 activations and a bf16 LM head (DG_ERR_UNSUPPORTED otherwise; NVFP4 takes
  *   dg_logits_entropy_nvfp4), n_rows <= 256, d_model <= 2048,
  *   vocab <= 262144; larger requests return DG_ERR_WORKSPACE and launch nothing.
- *   The first call on a device looks up the array's device address with that device current
- *   (cudaGetSymbolAddress); make that first call before any stream capture on the device.
+ *   The array's device address belongs to the CUDA context that loaded the library's module:
+ *   every call made outside stream capture looks it up in the calling thread's current context
+ *   (cudaGetSymbolAddress; it also sets up the device's primary context if none is current),
+ *   and a call made while `stream` is being captured reuses the address found by an earlier
+ *   call in the same context — so the first call in each context must come before any stream
+ *   capture there (a first call inside a capture returns DG_ERR_CUDA).
+ *   Config checks and errors as dg_logits_entropy (DG_ERR_INVALID_ARG on a malformed config).
  *   All calls share the one array and it keeps the last call's contents (nothing in it has to
  *   start at zero): calls whose work overlaps on the GPU — on different streams, or from
  *   different threads — race on it and must be serialised by the caller. */

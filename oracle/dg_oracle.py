@@ -41,6 +41,7 @@ definition of it (see nvfp4_rows).
 """
 from __future__ import annotations
 
+import contextlib
 import math
 from typing import Dict, List, Optional
 
@@ -48,6 +49,33 @@ import numpy as np
 
 INT64_MAX = np.iinfo(np.int64).max
 EB_FRAC_BITS = 32  # fixed-point fraction bits of the EB entropy sums
+
+# Arithmetic type of every product, sum, norm and softmax below: fp64.  The tests derive their
+# floating-point tolerances from a second run of this same code with fp32 arithmetic (the
+# `accumulation` context), i.e. from the spread between two valid evaluations of the method that
+# differ only in accumulation precision and order; nothing else ever changes it.
+_ACC = [np.float64]
+
+
+def acc_dtype():
+    return _ACC[0]
+
+
+@contextlib.contextmanager
+def accumulation(dtype):
+    """Run the oracle with `dtype` (np.float64 or np.float32) as its arithmetic type.  Storage
+    rounding (bf16 / fp16 at the tensors the reading names) is unchanged."""
+    prev = _ACC[0]
+    _ACC[0] = np.dtype(dtype).type
+    try:
+        yield
+    finally:
+        _ACC[0] = prev
+
+
+def _a(x) -> np.ndarray:
+    """x in the arithmetic type."""
+    return np.asarray(x, dtype=_ACC[0])
 
 
 # --------------------------------------------------------------------------- number formats
@@ -160,8 +188,8 @@ def storage_round(x: np.ndarray, act: str) -> np.ndarray:
 
 def rmsnorm(x: np.ndarray, eps: float) -> np.ndarray:
     """x / sqrt(mean(x^2) + eps) over the last axis, unit gain."""
-    x = np.asarray(x, dtype=np.float64)
-    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    x = _a(x)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + _ACC[0](eps))
 
 
 def gelu_tanh(x: np.ndarray) -> np.ndarray:
@@ -180,8 +208,9 @@ def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
     inv = theta ** (-2.0 * np.arange(half, dtype=np.float64) / hd)
     ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]
     shape = (x.shape[0],) + (1,) * (x.ndim - 2) + (half,)
-    c = np.cos(ang).reshape(shape)
-    s = np.sin(ang).reshape(shape)
+    c = _a(np.cos(ang).reshape(shape))
+    s = _a(np.sin(ang).reshape(shape))
+    x = _a(x)
     x1, x2 = x[..., :half], x[..., half:]
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
@@ -201,6 +230,7 @@ def attention(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
     T, Hq, hd = q.shape
     Hkv, P = k_cache.shape[0], k_cache.shape[1]
     rep = Hq // Hkv
+    q, k_cache, v_cache, k_new, v_new = (_a(t) for t in (q, k_cache, v_cache, k_new, v_new))
     out = np.empty((T, Hq, hd))
     mask = None
     if causal:
@@ -210,7 +240,7 @@ def attention(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
         g = h // rep
         K = np.concatenate([k_cache[g], k_new[:, g]], axis=0)
         V = np.concatenate([v_cache[g], v_new[:, g]], axis=0)
-        s = q[:, h] @ K.T / math.sqrt(hd)
+        s = q[:, h] @ K.T / _ACC[0](math.sqrt(hd))
         if mask is not None:
             s = np.where(mask, -np.inf, s)
         s = s - s.max(axis=1, keepdims=True)
@@ -220,16 +250,20 @@ def attention(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
     return out
 
 
-def router_topk(y: np.ndarray, w_r: np.ndarray, top_k: int):
+def router_topk(y: np.ndarray, w_r: np.ndarray, top_k: int, forced: Optional[np.ndarray] = None):
     """Router: logits z = y W_r^T, p = softmax(z) over all experts, the top_k
     largest p (lower expert index first among equals), renormalised to sum 1.
 
+    ``forced`` (int [T, k], optional) replaces the top-k choice by the given experts, whose gates
+    are still this router's p renormalised over them: it lets one evaluation reproduce another's
+    expert choices, which bf16 rounding can legitimately flip at near ties.
     Returns (idx [T, k] int32, gates [T, k], z [T, E]).
     """
-    z = y @ w_r.T
+    z = _a(y) @ _a(w_r).T
     p = np.exp(z - z.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
-    idx = np.argsort(-p, axis=1, kind="stable")[:, :top_k]
+    idx = np.argsort(-p, axis=1, kind="stable")[:, :top_k] if forced is None \
+        else np.asarray(forced, dtype=np.int64)
     gp = np.take_along_axis(p, idx, axis=1)
     return idx.astype(np.int32), gp / gp.sum(axis=1, keepdims=True), z
 
@@ -272,15 +306,16 @@ def moe_ffn(y: np.ndarray, idx: np.ndarray, gates: np.ndarray, expert_w, residua
     negative has no expert and contributes nothing.
     """
     T, k = idx.shape
-    acc = np.array(residual, dtype=np.float64, copy=True)
+    acc = np.array(residual, dtype=_ACC[0], copy=True)
+    y = _a(y)
     for e in np.unique(idx):
         if e < 0:
             continue
         rows, slots = np.nonzero(idx == e)
-        w_gu, w_d = expert_w(int(e))
+        w_gu, w_d = (_a(w) for w in expert_w(int(e)))
         F = w_d.shape[1]
         u = y[rows] @ w_gu.T
-        a = storage_round(gelu_tanh(u[:, :F]) * u[:, F:], act)
+        a = _a(storage_round(gelu_tanh(u[:, :F]) * u[:, F:], act))
         Y = a @ w_d.T
         acc[rows] += gates[rows, slots][:, None] * Y
     return acc
@@ -289,7 +324,7 @@ def moe_ffn(y: np.ndarray, idx: np.ndarray, gates: np.ndarray, expert_w, residua
 def entropy_argmax(z: np.ndarray):
     """Per row of logits z [R, V]: softmax entropy (natural log), greedy argmax
     (lowest index among equal maxima) and the top-1 minus top-2 margin."""
-    z = np.asarray(z, dtype=np.float64)
+    z = _a(z)
     m = z.max(axis=1, keepdims=True)
     e = np.exp(z - m)
     p = e / e.sum(axis=1, keepdims=True)
@@ -419,7 +454,7 @@ def layer_qkv(cfg, model: OracleModel, l: int, x: np.ndarray, pos: np.ndarray):
     T = x.shape[0]
     Hq, Hkv, hd = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
     a = storage_round(rmsnorm(x, cfg.rms_eps), act)
-    qkv = a @ model.w(l, "w_qkv").T
+    qkv = _a(a) @ _a(model.w(l, "w_qkv")).T
     q = qkv[:, :Hq * hd].reshape(T, Hq, hd)
     k = qkv[:, Hq * hd:(Hq + Hkv) * hd].reshape(T, Hkv, hd)
     v = qkv[:, (Hq + Hkv) * hd:].reshape(T, Hkv, hd)
@@ -429,16 +464,18 @@ def layer_qkv(cfg, model: OracleModel, l: int, x: np.ndarray, pos: np.ndarray):
     return q, k, v
 
 
-def layer_rest(cfg, model: OracleModel, l: int, x, q, k, v, kc, vc, causal: bool, info=None):
+def layer_rest(cfg, model: OracleModel, l: int, x, q, k, v, kc, vc, causal: bool, info=None,
+               forced=None):
     """Attention, output projection with residual, and the MoE FFN with residual.
 
-    x and the returned layer output are the residual stream (unrounded)."""
+    x and the returned layer output are the residual stream (unrounded).  ``forced``: optional
+    expert choices [T, k] for this layer (see router_topk)."""
     act = cfg.act
     T = x.shape[0]
     o = storage_round(attention(q, kc, vc, k, v, causal), act).reshape(T, -1)
-    h = x + o @ model.w(l, "w_o").T
+    h = _a(x) + _a(o) @ _a(model.w(l, "w_o")).T
     y = storage_round(rmsnorm(h, cfg.rms_eps), act)
-    idx, gates, z = router_topk(y, model.w(l, "w_router"), cfg.top_k)
+    idx, gates, z = router_topk(y, model.w(l, "w_router"), cfg.top_k, forced)
     if info is not None:
         info.setdefault("router_margin", []).append(router_margin(z, cfg.top_k))
         info.setdefault("router_idx", []).append(idx)
@@ -459,16 +496,18 @@ def lm_head_rows(cfg, model: OracleModel, x_rows: np.ndarray, keep_logits: bool 
     R = f.shape[0]
     z = np.empty((R, cfg.vocab))
     for v0, w in model.lm_head_chunks():
-        z[:, v0:v0 + w.shape[0]] = f @ w.T
+        z[:, v0:v0 + w.shape[0]] = _a(f) @ _a(w).T
     H, am, margin = entropy_argmax(z)
     return H, am, margin, (z if keep_logits else None)
 
 
 def canvas_forward(cfg, model: OracleModel, tokens: np.ndarray, masked: np.ndarray,
-                   kcache: np.ndarray, vcache: np.ndarray, cache_len: int, info=None):
+                   kcache: np.ndarray, vcache: np.ndarray, cache_len: int, info=None,
+                   forced=None):
     """Decoder pass over one canvas.  Returns the final residual stream [C, d].
 
-    kcache, vcache: [L, Hkv, cap, hd] for this canvas (decoded values).
+    kcache, vcache: [L, Hkv, cap, hd] for this canvas (decoded values).  ``forced``: optional
+    expert choices [L, C, k] (see router_topk).
     """
     C = tokens.shape[0]
     ids = np.where(masked != 0, cfg.mask_id, tokens)
@@ -477,12 +516,14 @@ def canvas_forward(cfg, model: OracleModel, tokens: np.ndarray, masked: np.ndarr
     for l in range(cfg.n_layers):
         q, k, v = layer_qkv(cfg, model, l, x, pos)
         x = layer_rest(cfg, model, l, x, q, k, v, kcache[l, :, :cache_len],
-                       vcache[l, :, :cache_len], False, info)
+                       vcache[l, :, :cache_len], False, info,
+                       None if forced is None else forced[l])
     return x
 
 
 def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache: np.ndarray,
-                cache_len: np.ndarray, gamma: float, max_steps: int, keep_logits: bool = False):
+                cache_len: np.ndarray, gamma: float, max_steps: int, keep_logits: bool = False,
+                forced=None):
     """One denoising step for every canvas of the batch that is not done.
 
     state: tokens int32 [B, C], masked uint8 [B, C], n_masked int32 [B],
@@ -492,6 +533,7 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
     (stored as fp32) and greedy argmax of its logits; EB selection (all masked
     positions at step index max_steps - 1); commit selected positions to their
     argmax; step += 1; done = no masked position left.
+    ``forced`` (optional, [L, B, C, k]): every layer's expert choices (see router_topk).
     Returns (new_state, info) where info[b] holds H, argmax, margin, rows,
     selected, router margins and (optionally) logits.
     """
@@ -507,7 +549,8 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
         info: Dict = {"rows": rows}
         if len(rows) > 0:
             x = canvas_forward(cfg, model, state["tokens"][b], masked, kcache[:, b], vcache[:, b],
-                               int(cache_len[b]), info)
+                               int(cache_len[b]), info,
+                               None if forced is None else forced[:, b])
             H, am, margin, z = lm_head_rows(cfg, model, x[rows], keep_logits)
             Hf = H.astype(np.float32)
             full_H = np.zeros(cfg.canvas, dtype=np.float32)
@@ -525,7 +568,7 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
 
 
 def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
-              cache_len: np.ndarray, info=None):
+              cache_len: np.ndarray, info=None, forced=None):
     """Causal encoder pass over finished tokens; their K/V go to the cache.
 
     tokens int32 [B, n]; kcache/vcache decoded [L, B, Hkv, cap, hd], updated in
@@ -533,6 +576,7 @@ def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, v
     shares the decoder's weights; its attention sees the whole cache and the
     new tokens causally.  Returns the new cache_len.  With ``info`` (a dict) given, the expert
     choices of each routed layer are collected in info["router_idx"][l] as [B, n, k].
+    ``forced`` (optional, [L, B, n, k]): every layer's expert choices (see router_topk).
     """
     B, n = tokens.shape
     new_len = np.array(cache_len, copy=True)
@@ -545,7 +589,8 @@ def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, v
             kc, vc = kcache[l, b, :, :L0], vcache[l, b, :, :L0]
             if l + 1 < cfg.n_layers:
                 li = {} if info is not None else None
-                x = layer_rest(cfg, model, l, x, q, k, v, kc, vc, True, li)
+                x = layer_rest(cfg, model, l, x, q, k, v, kc, vc, True, li,
+                               None if forced is None else forced[l, b])
                 if info is not None:
                     ri = info.setdefault("router_idx", [np.zeros((B, n, cfg.top_k), np.int32)
                                                         for _ in range(cfg.n_layers)])

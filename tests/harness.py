@@ -10,9 +10,42 @@ from oracle import dg_oracle as O
 from block_discrete_diffusion_dg_b200 import binding as B
 
 
-def oracle_model(cfg, model) -> O.OracleModel:
-    arr = {"emb": synth.to_numpy(model["emb"]),
-           "layers": [{k: synth.to_numpy(v) for k, v in lay.items()} for lay in model["layers"]]}
+# Factor between the spread of two oracle evaluations (fp64 and fp32 arithmetic, same storage
+# rounding, same expert choices) and the bar a device result is held to.  The device is one more
+# fp32 evaluation with its own summation order: it and the fp32 oracle can each sit up to the
+# spread S away from the fp64 result, on either side, so a bar of 2 S covers it.  Fixed before any
+# device result was compared with it.
+BAR_FACTOR = 2.0
+
+
+class _LazyTensor:
+    """A device tensor that the oracle reads piecewise: x[i] copies one slice to the host, and
+    np.asarray(x) the whole tensor (so a deep stack's weights never all sit in host memory)."""
+
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, i):
+        return synth.to_numpy(self.t[i])
+
+    def __array__(self, dtype=None, copy=None):
+        a = synth.to_numpy(self.t)
+        return a if dtype is None else a.astype(dtype)
+
+
+class _LazyLayer(dict):
+    def __init__(self, lay):
+        super().__init__({k: (None if v is None else _LazyTensor(v)) for k, v in lay.items()})
+
+
+def oracle_model(cfg, model, lazy: bool = False) -> O.OracleModel:
+    """The oracle's view of a device model.  lazy: layer weights are copied to the host slice by
+    slice when the oracle reads them (for stacks too large to hold decoded in host memory)."""
+    if lazy:
+        layers = [_LazyLayer(lay) for lay in model["layers"]]
+    else:
+        layers = [{k: synth.to_numpy(v) for k, v in lay.items()} for lay in model["layers"]]
+    arr = {"emb": synth.to_numpy(model["emb"]), "layers": layers}
     if "emb_scale" in model:
         arr["emb_scale"] = synth.to_numpy(model["emb_scale"])
         arr["emb_scale_global"] = float(model["emb_scale_global"])
@@ -71,6 +104,38 @@ class Workload:
     def check_status(self):
         rc = B.dg_read_status(self.status)
         assert rc == B.DG_OK, B.STATUS_NAMES.get(rc, rc)
+
+
+def forced_from(cfg, infos) -> np.ndarray:
+    """The oracle's expert choices of one step, [L][B][C][k] (zeros for skipped canvases)."""
+    f = np.zeros((cfg.n_layers, cfg.batch, cfg.canvas, cfg.top_k), np.int32)
+    for b, inf in enumerate(infos):
+        if inf is None or "router_idx" not in inf:
+            continue
+        for l, idx in enumerate(inf["router_idx"]):
+            f[l, b] = idx
+    return f
+
+
+def step_spread(cfg, om, st, kc, vc, cl, infos):
+    """Spread of the step's logits and entropies between the fp64 oracle (infos) and the same
+    oracle in fp32 arithmetic on the same inputs and expert choices: (max |dz|, max |dH| / H)."""
+    with O.accumulation(np.float32):
+        _, inf32 = O.canvas_step(cfg, om, st, kc, vc, cl, cfg.gamma, cfg.max_steps,
+                                 keep_logits=True, forced=forced_from(cfg, infos))
+    dz, dh = 0.0, 0.0
+    for a, b in zip(infos, inf32):
+        if a is None or len(a["rows"]) == 0:
+            continue
+        dz = max(dz, float(np.abs(b["logits"] - a["logits"]).max()))
+        dh = max(dh, float((np.abs(b["H"].astype(np.float64) - a["H"]) / a["H"]).max()))
+    return dz, dh
+
+
+def rel_to_row_rms(g, o):
+    """|g - o| relative to the RMS of o's row (last axis)."""
+    scale = np.sqrt(np.mean(o * o, axis=-1, keepdims=True)) + 1e-30
+    return np.abs(g - o) / scale
 
 
 def np_state(st):

@@ -3,21 +3,26 @@
 * long context: the one-layer model with 131072 prompt K/V tokens, half-committed canvas; the
   oracle runs the whole step (fp64 attention over 131328 keys).
 * batch of 32: 32 canvases x 256 through the one-layer model with e4m3 expert/attention weights
-  (one fp32 scale per output channel), 1024 prompt tokens each; the oracle runs two sampled
-  canvases (the others are marked done on its side; canvases are independent).
-* 30-layer stack: a full-width step of a 4-layer stack on synthetic prompt K/V against the oracle;
-  prefill -> denoise -> append against the oracle at full width and 2 layers; and the 30-layer
-  generate loop of the workload (prompt 2048 prefilled in 256-token chunks, 4 canvases, at most 32
-  steps each) checked by its invariants.
-  Through several layers two valid bf16 computations route a growing share of tokens to
-  different experts (a near tie flips, and that token's later state, hence its later choices,
-  differ by O(1): about 10% of the tokens by the 4th layer).  The multi-layer comparisons
-  therefore hand the device the oracle's expert choices (forced_topk; the gates are still the
-  device's own) and then hold every row to the float bars, the logit bar widened with depth
-  (logit_tol) by the measured growth of bf16 rounding noise.
-Bars as in test_gpu_full: logits 2e-2 max-abs and entropies 1e-3 relative on rows without a
-router near tie, argmax bit-exact against the device's own logits, EB bit-exact on the oracle's
-entropies."""
+  (one fp32 scale per output channel), 1024 prompt tokens each; the oracle runs eight canvases,
+  the first and the last among them (the others are marked done on its side; canvases are
+  independent), and every canvas is checked to have taken its one step.
+* stacks: a full-width step of a 4-layer stack and of the full 30-layer stack on synthetic prompt
+  K/V, and the 30-layer append of a canvas, against the oracle; prefill -> denoise -> append
+  against the oracle at full width and 2 layers; and the 30-layer generate loop of the workload
+  (prompt 2048 prefilled in 256-token chunks, 4 canvases, at most 32 steps each) checked by its
+  invariants.
+
+Bars.  One layer: the stated bf16 bars, logits 2e-2 max-abs and entropies 1e-3 relative, on
+every masked row, in a step that takes the oracle's expert choices (forced_topk; the gates are
+still the device's own); and in a free-running step on every row without a router near tie
+(where a bf16 router input can legitimately pick the other expert), whose count is reported and
+held small.  Several layers: two valid evaluations of the method already differ by more than
+2e-2 after a few layers (a bf16 rounding flip of one element of q moves every score of its row,
+and the flips compound with depth), so the bar there is derived from the oracle alone:
+BAR_FACTOR times the spread between the fp64 oracle and the same oracle in fp32 arithmetic on the
+same inputs and expert choices, and never below the one-layer bar.  K/V caches after layer 0 are
+held the same way (element error relative to its row's RMS).  Argmax is bit-exact against the
+device's own logits, EB bit-exact on the oracle's entropies."""
 import numpy as np
 import pytest
 import torch
@@ -25,55 +30,29 @@ import torch
 import synth
 from oracle import dg_oracle as O
 from block_discrete_diffusion_dg_b200 import binding as B
-from harness import Workload, np_state, torch_state, decode_cache
+from harness import (BAR_FACTOR, Workload, decode_cache, forced_from, np_state, oracle_model,
+                     rel_to_row_rms, step_spread, torch_state)
 
 pytestmark = pytest.mark.gpu
 
 LOGIT_TOL = 2e-2
 ENT_RTOL = 1e-3
 ROUTER_TIE = 1e-2
+NEAR_TIE_MAX = 0.2      # at most this share of a canvas's rows may be router near ties
 
 
-def logit_tol(n_layers: int) -> float:
-    """The 2e-2 bf16 bar for one layer, widened for a stack by the growth of bf16 rounding noise
-    with depth.  Measured at full width with shared routing (all-MASK canvas, 67M logits), the
-    device-vs-oracle logit error has std 0.0025 / 0.0036 / 0.0043, 99.99th percentile
-    0.010 / 0.014 / 0.017 and maximum 0.015-0.017 / 0.021-0.022 / 0.025-0.034 at 1 / 2 / 4
-    layers (the maximum is a tail statistic that varies with the canvas state).  The bar is
-    2e-2 (1 + log2(L) / 2): 0.02 / 0.03 / 0.04, keeping >15% headroom over every observed
-    maximum."""
-    return LOGIT_TOL * (1.0 + np.log2(max(n_layers, 1)) / 2.0)
+def _device_forced(cfg, infos):
+    """The oracle's expert choices as the device's forced-routing table [n_layers][B C][k]."""
+    f = forced_from(cfg, infos).reshape(cfg.n_layers, cfg.batch * cfg.canvas, cfg.top_k)
+    return torch.from_numpy(np.ascontiguousarray(f)).cuda()
 
 
-def kv_close(g, o, n_layers):
-    """K/V rows after layer 0 carry the same depth noise: each element within 2^-4 of its
-    row's RMS, the median error within 2^-9 of it.  Measured after a 2-layer prefill and append
-    (4M elements per tensor), the error relative to the row RMS has 99.9th percentile 0.018,
-    99.999th 0.021 and a maximum of 0.021-0.034 that varies with the tokens; 2^-4 keeps ~1.8x
-    headroom over that maximum."""
-    scale = np.sqrt(np.mean(o * o, axis=-1, keepdims=True)) + 1e-30
-    rel = np.abs(g - o) / scale
-    return rel.max() <= 2.0 ** -4 and np.median(rel) <= 2.0 ** -9, (rel.max(), np.median(rel))
-
-
-def _forced(cfg, infos):
-    """The oracle's expert choices of a step as the device's forced-routing table
-    [n_layers][B C][k] (canvases the oracle skipped: zeros; the device skips them too)."""
-    f = np.zeros((cfg.n_layers, cfg.batch * cfg.canvas, cfg.top_k), np.int32)
-    for b, inf in enumerate(infos):
-        if inf is None or "router_idx" not in inf:
-            continue
-        for l, idx in enumerate(inf["router_idx"]):
-            f[l, b * cfg.canvas:(b + 1) * cfg.canvas] = idx
-    return torch.from_numpy(f).cuda()
-
-
-def _check_step(wl, st_np, canvases=None, min_ok=0.6, force=False):
-    """One device step against the oracle on the canvases listed (default: all).  With force,
-    the device takes the oracle's expert choices (deep stacks: see test module docstring) and
-    every row is held to the float bars."""
+def _check_step(wl, st_np, canvases=None, derive=False):
+    """One device step against the oracle on the canvases listed (default: all): a free-running
+    step (one layer only; rows without a router near tie) and a step with the oracle's expert
+    choices (every row).  derive: multi-layer bars from the oracle's fp64/fp32 spread."""
     cfg = wl.cfg
-    om = wl.oracle() if not hasattr(wl, "_om") else wl._om
+    om = getattr(wl, "_om", None) or wl.oracle()
     wl._om = om
     kc, vc = decode_cache(cfg, wl.kv["k"]), decode_cache(cfg, wl.kv["v"])
     cl = synth.to_numpy(wl.kv["cache_len"])
@@ -84,25 +63,49 @@ def _check_step(wl, st_np, canvases=None, min_ok=0.6, force=False):
         o_st["done"][skip] = 1
     new_np, infos = O.canvas_step(cfg, om, o_st, kc, vc, cl, cfg.gamma, cfg.max_steps,
                                   keep_logits=True)
-    g_st, ent, am, lg = wl.step(torch_state(st_np), logits=True,
-                                forced=_forced(cfg, infos) if force else None)
-    wl.check_status()
-    ent, am = ent.cpu().numpy(), am.cpu().numpy()
-    n_rows = 0
+    lbar, ebar = LOGIT_TOL, ENT_RTOL
+    if derive:
+        dz, dh = step_spread(cfg, om, o_st, kc, vc, cl, infos)
+        lbar, ebar = max(LOGIT_TOL, BAR_FACTOR * dz), max(ENT_RTOL, BAR_FACTOR * dh)
+        print(f"\n{cfg.n_layers} layers: oracle fp64/fp32 spread logits {dz:.4f} entropy {dh:.2e}"
+              f" -> bars {lbar:.4f} / {ebar:.2e}")
+    runs = [("forced", _device_forced(cfg, infos))]
+    if cfg.n_layers == 1:
+        runs.insert(0, ("free", None))
+    g_st = None
+    for mode, forced in runs:
+        g_st, ent, am, lg = wl.step(torch_state(st_np), logits=True, forced=forced)
+        wl.check_status()
+        ent, am = ent.cpu().numpy(), am.cpu().numpy()
+        n_rows, worst = 0, 0.0
+        for b, inf in enumerate(infos):
+            if inf is None:
+                continue
+            rows = inf["rows"]
+            lgb = lg[b * cfg.canvas:(b + 1) * cfg.canvas].cpu().numpy()[rows]
+            assert (am[b, rows] == np.argmax(lgb, axis=1)).all()
+            if mode == "free":
+                rmarg = np.min(np.stack(inf["router_margin"]), axis=0)[rows]
+                ok = rmarg > ROUTER_TIE
+                print(f"canvas {b}: {int((~ok).sum())} of {len(rows)} rows are router near ties")
+                assert (~ok).sum() <= NEAR_TIE_MAX * len(rows)
+            else:
+                ok = np.ones(len(rows), bool)
+            err = np.abs(lgb[ok] - inf["logits"][ok]).max()
+            worst = max(worst, float(err))
+            assert err <= lbar, (mode, b, err, lbar)
+            np.testing.assert_allclose(ent[b, rows][ok], inf["H"][ok], rtol=ebar)
+            safe = ok & (inf["margin"] > 2 * lbar)
+            assert (am[b, rows][safe] == inf["argmax"][safe]).all()
+            n_rows += len(rows)
+        print(f"{mode}: max logit error {worst:.4f} (bar {lbar:.4f}) over {n_rows} rows")
+        if canvases is None:
+            assert n_rows > 0
+    # EB on the oracle's entropies, each canvas alone
     for b, inf in enumerate(infos):
         if inf is None:
             continue
         rows = inf["rows"]
-        lgb = lg[b * cfg.canvas:(b + 1) * cfg.canvas].cpu().numpy()[rows]
-        assert (am[b, rows] == np.argmax(lgb, axis=1)).all()
-        rmarg = np.min(np.stack(inf["router_margin"]), axis=0)[rows]
-        ok = np.ones(len(rows), bool) if force else rmarg > ROUTER_TIE
-        assert ok.sum() >= min_ok * len(rows), ok.sum()
-        assert np.abs(lgb[ok] - inf["logits"][ok]).max() <= logit_tol(cfg.n_layers)
-        np.testing.assert_allclose(ent[b, rows][ok], inf["H"][ok], rtol=ENT_RTOL)
-        safe = ok & (inf["margin"] > 2 * LOGIT_TOL)
-        assert (am[b, rows][safe] == inf["argmax"][safe]).all()
-        # EB on the oracle's entropies, this canvas alone
         e_in = np.zeros((1, cfg.canvas), np.float32)
         a_in = np.zeros((1, cfg.canvas), np.int32)
         e_in[0, rows] = inf["H"]
@@ -113,11 +116,38 @@ def _check_step(wl, st_np, canvases=None, min_ok=0.6, force=False):
                        one["n_masked"], one["done"], one["step"])
         for k in ("tokens", "masked", "n_masked", "done", "step"):
             assert (one[k].cpu().numpy()[0] == new_np[k][b]).all(), k
-        n_rows += len(rows)
-    # canvases the device skipped are unchanged
-    if canvases is None:
-        assert n_rows > 0
     return g_st
+
+
+def _append_check(wl, om, toks, ok, ov, ln, n, ws=None):
+    """Append `toks` [1, n] on the device (with the oracle's expert choices) and in the oracle
+    (fp64, and fp32 with the same choices); every new K/V element of every layer within
+    max(2^-7, BAR_FACTOR x the oracle's fp64/fp32 spread), relative to its row's RMS (2^-7: about
+    two bf16 ulps of a typical element, the floor for a single rounding flip)."""
+    cfg = wl.cfg
+    o32k, o32v = ok.copy(), ov.copy()
+    info = {}
+    ln2 = O.kv_append(cfg, om, toks.cpu().numpy(), ok, ov, ln, info)
+    forced_np = np.stack([r for r in info["router_idx"]]) if "router_idx" in info else \
+        np.zeros((cfg.n_layers, 1, n, cfg.top_k), np.int32)        # [L][B][n][k]
+    with O.accumulation(np.float32):
+        O.kv_append(cfg, om, toks.cpu().numpy(), o32k, o32v, ln, None, forced=forced_np)
+    forced = torch.from_numpy(np.ascontiguousarray(forced_np.reshape(cfg.n_layers, -1, cfg.top_k))).cuda()
+    B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, toks, n, wl.kv["k"], wl.kv["v"], wl.kv["cache_len"],
+                   wl.cap, wl.ws if ws is None else ws, wl.status, forced_topk=forced)
+    torch.cuda.synchronize()
+    wl.check_status()
+    assert int(wl.kv["cache_len"].item()) == ln2[0]
+    sl = slice(int(ln[0]), int(ln2[0]))
+    for name, dev, o64, o32 in (("k", wl.kv["k"], ok, o32k), ("v", wl.kv["v"], ov, o32v)):
+        g = decode_cache(cfg, dev)[:, :, :, sl, :]
+        ref = o64[:, :, :, sl, :]
+        rel_d = float(rel_to_row_rms(g, ref).max())
+        rel_o = float(rel_to_row_rms(o32[:, :, :, sl, :], ref).max())
+        bar = max(2.0 ** -7, BAR_FACTOR * rel_o)
+        print(f"\n{name}: device {rel_d:.4f} vs oracle spread {rel_o:.4f} -> bar {bar:.4f}")
+        assert rel_d <= bar, (name, rel_d, bar)
+    return ln2
 
 
 def test_longctx_step_full_size():
@@ -130,7 +160,7 @@ def test_batch32_fp8_step_sampled_canvases():
     cfg = synth.get_config("batch32")
     wl = Workload(cfg, gen_device="cuda")
     st = np_state(synth.make_canvas_state(cfg, "all_mask"))
-    g_st = _check_step(wl, st, canvases=(0, 17))
+    g_st = _check_step(wl, st, canvases=(0, 5, 10, 15, 17, 22, 27, 31))
     # every canvas advanced by one step and committed exactly one token (entropies ~ ln V >> gamma)
     assert (g_st["step"].cpu().numpy() == 1).all()
     assert (g_st["n_masked"].cpu().numpy() == cfg.canvas - 1).all()
@@ -139,7 +169,24 @@ def test_batch32_fp8_step_sampled_canvases():
 def test_stack_step_full_width_four_layers():
     cfg = synth.get_config("stack30", n_layers=4, prefill_ids=False, prompt_len=1024)
     wl = Workload(cfg, gen_device="cuda")
-    _check_step(wl, np_state(synth.make_canvas_state(cfg, "half")), force=True)
+    _check_step(wl, np_state(synth.make_canvas_state(cfg, "half")), derive=True)
+
+
+@pytest.mark.slow
+def test_stack30_step_and_append_vs_oracle():
+    """The full 30-layer stack at full width: one denoising step of a half-committed canvas over a
+    2048-token synthetic prompt cache, then the causal append of a committed canvas, both against
+    the oracle with its expert choices handed to the device and bars derived from the oracle's
+    fp64/fp32 spread.  The oracle reads the device's weights layer by layer."""
+    cfg = synth.get_config("stack30", prefill_ids=False)
+    wl = Workload(cfg, gen_device="cuda")
+    wl._om = oracle_model(cfg, wl.model, lazy=True)
+    _check_step(wl, np_state(synth.make_canvas_state(cfg, "half")), derive=True)
+    ok, ov = decode_cache(cfg, wl.kv["k"]), decode_cache(cfg, wl.kv["v"])
+    ln = synth.to_numpy(wl.kv["cache_len"]).copy()
+    g = torch.Generator(device="cpu").manual_seed(30)
+    toks = torch.randint(0, cfg.vocab, (1, cfg.canvas), generator=g, dtype=torch.int32).cuda()
+    _append_check(wl, wl._om, toks, ok, ov, ln, cfg.canvas)
 
 
 def test_stack_prefill_denoise_append_two_layers():
@@ -148,47 +195,27 @@ def test_stack_prefill_denoise_append_two_layers():
     cfg = synth.get_config("stack30", n_layers=2, prompt_len=512, n_canvases=1)
     wl = Workload(cfg, gen_device="cuda")
     om = wl.oracle()
+    wl._om = om
     ids = wl.kv["prompt_ids"]
-    k_dev, v_dev, len_dev = wl.kv["k"], wl.kv["v"], wl.kv["cache_len"]
-    ok = np.zeros(decode_cache(cfg, k_dev).shape)
+    ok = np.zeros(decode_cache(cfg, wl.kv["k"]).shape)
     ov = np.zeros_like(ok)
     ln = np.zeros(1, np.int32)
     for c0 in range(0, cfg.prompt_len, 256):
-        chunk = ids[:, c0:c0 + 256].contiguous()
-        info = {}
-        ln = O.kv_append(cfg, om, chunk.cpu().numpy(), ok, ov, ln, info)
-        forced = torch.from_numpy(np.stack([r.reshape(-1, cfg.top_k) for r in info["router_idx"]])).cuda()
-        B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, chunk, 256, k_dev, v_dev, len_dev, wl.cap, wl.ws,
-                       wl.status, forced_topk=forced)
-    torch.cuda.synchronize()
-    wl.check_status()
-    assert int(len_dev.item()) == ln[0] == cfg.prompt_len
-    gk = decode_cache(cfg, k_dev)[:, :, :, :cfg.prompt_len, :]   # [L][B][Hkv][rows][hd]
-    good, stat = kv_close(gk, ok[:, :, :, :cfg.prompt_len, :], cfg.n_layers)
-    assert good, stat
+        ln = _append_check(wl, om, ids[:, c0:c0 + 256].contiguous(), ok, ov, ln, 256)
+    assert int(wl.kv["cache_len"].item()) == ln[0] == cfg.prompt_len
     # two denoising steps from the oracle's state on the oracle-prefilled cache
     wl.kv["k"] = torch.from_numpy(ok).to(torch.bfloat16).cuda()
     wl.kv["v"] = torch.from_numpy(ov).to(torch.bfloat16).cuda()
     wl.kv["cache_len"] = torch.from_numpy(ln).cuda()
     st = np_state(synth.make_canvas_state(cfg, "all_mask"))
     for _ in range(2):
-        _check_step(wl, st, force=True)
+        _check_step(wl, st, derive=True)
         kc, vc = decode_cache(cfg, wl.kv["k"]), decode_cache(cfg, wl.kv["v"])
         st, _ = O.canvas_step(cfg, om, st, kc, vc, ln, cfg.gamma, cfg.max_steps)
     # append a committed canvas
     toks = torch.randint(0, cfg.vocab, (1, cfg.canvas), dtype=torch.int32).cuda()
-    info = {}
-    ln2 = O.kv_append(cfg, om, toks.cpu().numpy(), ok, ov, ln, info)
-    forced = torch.from_numpy(np.stack([r.reshape(-1, cfg.top_k) for r in info["router_idx"]])).cuda()
-    B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, toks, cfg.canvas, wl.kv["k"], wl.kv["v"],
-                   wl.kv["cache_len"], wl.cap, wl.ws, wl.status, forced_topk=forced)
-    torch.cuda.synchronize()
-    wl.check_status()
-    assert int(wl.kv["cache_len"].item()) == ln2[0]
-    gk = decode_cache(cfg, wl.kv["k"])[:, :, :, ln[0]:ln2[0], :]
-    assert gk.shape[3] == cfg.canvas
-    good, stat = kv_close(gk, ok[:, :, :, ln[0]:ln2[0], :], cfg.n_layers)
-    assert good, stat
+    ln2 = _append_check(wl, om, toks, ok, ov, ln, cfg.canvas)
+    assert ln2[0] == ln[0] + cfg.canvas
 
 
 def test_prefill_one_call_of_1024_tokens_two_layers():
@@ -202,21 +229,10 @@ def test_prefill_one_call_of_1024_tokens_two_layers():
     om = wl.oracle()
     ids = wl.kv["prompt_ids"][:, :n].contiguous()
     ws = B.alloc_workspace(wl.dgcfg, 1, n, wl.cap)
-    k_dev, v_dev, len_dev = wl.kv["k"], wl.kv["v"], wl.kv["cache_len"]
-    ok = np.zeros(decode_cache(cfg, k_dev).shape)
+    ok = np.zeros(decode_cache(cfg, wl.kv["k"]).shape)
     ov = np.zeros_like(ok)
-    info = {}
-    ln = O.kv_append(cfg, om, ids.cpu().numpy(), ok, ov, np.zeros(1, np.int32), info)
-    forced = torch.from_numpy(np.stack([r.reshape(-1, cfg.top_k) for r in info["router_idx"]])).cuda()
-    B.dg_kv_append(wl.dgcfg, wl.dgmodel, 1, ids, n, k_dev, v_dev, len_dev, wl.cap, ws, wl.status,
-                   forced_topk=forced)
-    torch.cuda.synchronize()
-    wl.check_status()
-    assert int(len_dev.item()) == ln[0] == n
-    for name, dev, orc in (("k", k_dev, ok), ("v", v_dev, ov)):
-        g = decode_cache(cfg, dev)[:, :, :, :n, :]
-        good, stat = kv_close(g, orc[:, :, :, :n, :], cfg.n_layers)
-        assert good, (name, stat)
+    ln = _append_check(wl, om, ids, ok, ov, np.zeros(1, np.int32), n, ws=ws)
+    assert ln[0] == n
 
 
 def test_stack30_generate_invariants():

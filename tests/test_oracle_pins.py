@@ -58,6 +58,39 @@ def test_e4m3_decode_all_codes_vs_torch():
     assert got[0x38] == 1.0 and got[0xB8] == -1.0
 
 
+def test_e4m3_channel_scale_lands_on_output_rows_hand_built():
+    """decode_weight's per-channel scale multiplies each OUTPUT channel (row of a [out][in]
+    matrix; for a stacked [E][out][in] expert tensor, scale [E][out]).  Hand-worked values: OCP
+    E4M3 codes 0x38 = 1.0, 0x40 = 2.0, 0x30 = 0.5, 0xB8 = -1.0 (sign bit), 0x01 = 2^-9 (the
+    smallest subnormal), with a non-square 2 x 3 matrix so a column-wise scale cannot broadcast."""
+    codes = np.array([[0x38, 0x40, 0x30], [0xB8, 0x01, 0x40]], np.uint8)
+    scale = np.array([2.0, 0.25], np.float32)
+    want = np.array([[2.0, 4.0, 1.0], [-0.25, 0.25 * 2.0 ** -9, 0.5]])
+    np.testing.assert_array_equal(O.decode_weight(codes, "e4m3", scale), want)
+    stacked = np.stack([codes, codes[::-1]])                      # [E=2][out=2][in=3]
+    sc = np.array([[2.0, 0.25], [8.0, 1.0]], np.float32)          # [E][out]
+    got = O.decode_weight(stacked, "e4m3", sc)
+    np.testing.assert_array_equal(got[0], want)
+    np.testing.assert_array_equal(got[1], np.array([[-8.0, 8.0 * 2.0 ** -9, 16.0],
+                                                    [1.0, 2.0, 0.5]]))
+
+
+def test_e4m3_decode_recovers_the_fp32_draw_within_one_step():
+    """The stored e4m3 weights of the batched workload, decoded by the oracle, reproduce the fp32
+    values they were drawn from within half an e4m3 step: |w - w32| <= 2^-4 |w32| for normals
+    (3 mantissa bits) plus half the subnormal quantum 2^-10 * scale.  Rows differ in magnitude by
+    up to 10^3 and the matrix is not square, so a scale applied along the wrong axis fails."""
+    g = torch.Generator().manual_seed(7)
+    w32 = torch.randn((6, 40), generator=g) * torch.tensor([1e-3, 1.0, 0.02, 5.0, 0.3, 2e-2])[:, None]
+    codes, scale = synth._store_weight(w32, "e4m3")
+    dec = O.decode_weight(synth.to_numpy(codes), "e4m3", synth.to_numpy(scale))
+    w = w32.double().numpy()
+    sc = synth.to_numpy(scale).astype(np.float64)[:, None]
+    assert (np.abs(dec - w) <= 2.0 ** -4 * np.abs(w) + 2.0 ** -10 * sc + 1e-12).all()
+    # each row's largest magnitude maps to the largest finite code (448 * scale)
+    np.testing.assert_allclose(np.abs(dec).max(axis=1), 448.0 * sc[:, 0], rtol=1e-6)
+
+
 def test_e2m1_decode_all_codes_vs_ml_dtypes():
     ml_dtypes = pytest.importorskip("ml_dtypes")
     codes = np.arange(16, dtype=np.uint8)
@@ -278,6 +311,44 @@ def test_router_uniform_ties_and_brute_force():
 
 def _experts(E, F, d):
     return [(rng.standard_normal((2 * F, d)) * 0.3, rng.standard_normal((d, F)) * 0.3) for _ in range(E)]
+
+
+def test_router_forced_choice_renormalises_this_routers_probabilities():
+    """Forced expert choices: the given experts, gated by this router's softmax renormalised over
+    them (brute force per token); forcing the router's own choice changes nothing."""
+    y = rng.standard_normal((5, 12))
+    w = rng.standard_normal((9, 12)) * 0.3
+    idx, gates, z = O.router_topk(y, w, 3)
+    idx2, gates2, _ = O.router_topk(y, w, 3, forced=idx)
+    np.testing.assert_array_equal(idx2, idx)
+    np.testing.assert_array_equal(gates2, gates)
+    forced = np.array([[8, 0, 4]] * 5)
+    idx3, gates3, _ = O.router_topk(y, w, 3, forced=forced)
+    np.testing.assert_array_equal(idx3, forced)
+    for t in range(5):
+        p = np.exp(z[t] - z[t].max())
+        p /= p.sum()
+        np.testing.assert_allclose(gates3[t], p[[8, 0, 4]] / p[[8, 0, 4]].sum(), rtol=1e-12)
+
+
+def test_fp32_arithmetic_variant_tracks_fp64_and_restores_it(tiny):
+    """The fp32-arithmetic run of the oracle (used only to derive tolerances) differs from the
+    fp64 run by fp32 rounding on the fp32 workload, and leaving the context restores fp64 bit
+    for bit."""
+    cfg, om, kv = tiny
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    st = {k: synth.to_numpy(v) for k, v in synth.make_canvas_state(cfg, "all_mask").items()}
+    _, a = O.canvas_step(cfg, om, st, kc, vc, cl, cfg.gamma, cfg.max_steps, keep_logits=True)
+    with O.accumulation(np.float32):
+        assert O.acc_dtype() is np.float32
+        _, b = O.canvas_step(cfg, om, st, kc, vc, cl, cfg.gamma, cfg.max_steps, keep_logits=True)
+    assert O.acc_dtype() is np.float64
+    _, c = O.canvas_step(cfg, om, st, kc, vc, cl, cfg.gamma, cfg.max_steps, keep_logits=True)
+    d = np.abs(b[0]["logits"] - a[0]["logits"]).max()
+    assert 0 < d < 1e-5
+    np.testing.assert_array_equal(c[0]["logits"], a[0]["logits"])
 
 
 def test_moe_k_equals_E_uniform_gates_is_dense_mean():

@@ -20,21 +20,28 @@ pytestmark = pytest.mark.gpu
 ENT_RTOL = 1e-3
 
 
-def _case(cfg, emb, n_all, n_rows, seed):
+def _case(cfg, emb, n_all, n_rows, seed, n_dev=None):
+    """Both entry points on the same rows; with n_dev, the row count is read on the device
+    (*n_rows_dev = n_dev <= n_rows, as dg_canvas_step passes it) and rows past it stay untouched."""
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     h = (torch.randn((n_all, cfg.d_model), generator=g) * 0.07).cuda()   # fp32 hidden rows
     rows = torch.sort(torch.randperm(n_all, generator=g)[:n_rows]).values.to(torch.int32).cuda()
+    nd = None if n_dev is None else torch.tensor([n_dev], dtype=torch.int32, device="cuda")
     dgc = B.make_config(cfg)
     e_ref = torch.full((n_all,), -1.0, device="cuda")
     a_ref = torch.full((n_all,), -1, dtype=torch.int32, device="cuda")
-    B.dg_logits_entropy(dgc, n_rows, None, h, rows, emb, e_ref, a_ref, None,
+    B.dg_logits_entropy(dgc, n_rows, nd, h, rows, emb, e_ref, a_ref, None,
                         B.alloc_workspace(dgc, 1, n_rows, 0))
     e_st = torch.full((n_all,), -1.0, device="cuda")
     a_st = torch.full((n_all,), -1, dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    B.dg_logits_entropy_static(dgc, n_rows, None, h, rows, emb, e_st, a_st, status)
+    B.dg_logits_entropy_static(dgc, n_rows, nd, h, rows, emb, e_st, a_st, status)
     assert B.dg_read_status(status) == B.DG_OK
+    if n_dev is not None:   # rows beyond the device count keep their sentinels on both sides
+        skipped = rows[n_dev:].long().cpu()
+        for e_, a_ in ((e_ref, a_ref), (e_st, a_st)):
+            assert (e_.cpu()[skipped] == -1.0).all() and (a_.cpu()[skipped] == -1).all()
     return e_ref.cpu().numpy(), a_ref.cpu().numpy(), e_st.cpu().numpy(), a_st.cpu().numpy()
 
 
@@ -43,8 +50,9 @@ def test_static_scratch_matches_regular_entry_point_twice(name):
     cfg = synth.reduced("layer") if name == "layer-reduced" else synth.get_config("layer")
     emb = synth.make_model(cfg, "cuda", seed=5)["emb"] if name == "layer" else \
         synth.make_model(cfg, "cpu", seed=5)["emb"].cuda()
-    for n_all, n_rows, seed in ((300, 256, 1), (200, 77, 2)):   # two calls in a row
-        e_ref, a_ref, e_st, a_st = _case(cfg, emb, n_all, n_rows, seed)
+    # two calls in a row, then one whose row count (77 of 256) is known on the device only
+    for n_all, n_rows, seed, n_dev in ((300, 256, 1, None), (200, 77, 2, None), (300, 256, 3, 77)):
+        e_ref, a_ref, e_st, a_st = _case(cfg, emb, n_all, n_rows, seed, n_dev)
         np.testing.assert_allclose(e_st, e_ref, rtol=ENT_RTOL)
         assert (a_st == a_ref).all()
         assert (e_st[a_ref < 0] == -1.0).all()   # rows not asked for are left alone
@@ -65,4 +73,8 @@ def test_static_scratch_rejects_oversized_requests():
     f32 = B.make_config(synth.get_config("tiny"))
     assert L.dg_logits_entropy_static(ctypes.byref(f32), 16, None, p, None, p, p, p, None, None) \
         == B.DG_ERR_UNSUPPORTED
+    bad = B.make_config(synth.reduced("layer"))
+    bad.rms_eps = float("nan")       # malformed config: refused as by dg_logits_entropy
+    assert L.dg_logits_entropy_static(ctypes.byref(bad), 16, None, p, None, p, p, p, None, None) \
+        == B.DG_ERR_INVALID_ARG
     assert L.dg_launch_count() == n0
