@@ -396,6 +396,135 @@ def eb_select(H: np.ndarray, masked: np.ndarray, gamma: float, force_all: bool) 
     return sel
 
 
+# --------------------------------------------------------------------------- sampler variants
+#
+# The pages describe a canvas that starts from random noise and is refined over the steps
+# ("DiffusionGemma Technical Report": explanatory visual "Inference: block-wise diffusion decoding",
+# "What they did", Figure 3 with uniform noise at t = 1.0), a model that corrects its own mistakes
+# while denoising, before the output is final (ainewsonline.de article), a sampler whose
+# temperature is annealed over the step budget N (report, Figure 9: a larger N anneals more
+# mildly; Figure 10: tau_t = 1 when annealing is off), and weights that still run in standard
+# autoregressive mode, leaving room for hybrid diffusion-AR decoding (report, "What they did"
+# and "Limits and open work").  None of them is given as a formula; the readings taken are:
+#
+# * temperature: linear in the step index, tau_s = tau_start + (tau_end - tau_start) s / (N - 1)
+#   (fp64), N = max_steps.  tau > 0: the token is drawn from softmax(z / tau) and the entropy the
+#   EB rule ranks is that distribution's.  tau <= 0: greedy argmax with the entropy at tau = 1
+#   (the method without sampling).
+# * drawing from softmax(z / tau): the Gumbel-max rule, argmax_v (z_v / tau + G_v) with G_v
+#   standard Gumbel, G = -ln(-ln U).  The fp32 value 1 / tau multiplies the logits.
+# * randomness: one counter-based generator, Philox4x32-10 (Salmon, Moraes, Dror and Shaw,
+#   "Parallel random numbers: as easy as 1, 2, 3", SC 2011), keyed by the 64-bit seed (low word
+#   first).  The counter names the draw: (v >> 2, a1, a2, (tag << 24) | b) for vocabulary entry v
+#   (word v & 3 of the output) of stream (tag, b, a1, a2).  U = ((w >> 9) + 1/2) 2^-23, exact in
+#   fp32 and strictly inside (0, 1).
+# * uniform-noise canvas: position i of canvas b holds (w0 * V) >> 32 for the first output word
+#   w0 of counter (i, 0, 0, (TAG_NOISE << 24) | b); every position starts not final.
+# * revisable drafts (noise canvas): a position that is not final is embedded by its current
+#   draft token (not MASK); each step the EB rule makes the lowest-entropy prefix final as
+#   before, and every other non-final position takes the step's prediction as its new draft.
+#   Final positions never change.
+# * autoregressive mode: the same weights as the causal encoder; the new tokens of a sequence
+#   are appended to its cache as by the append, the LAST layer runs in full as well, and the
+#   final RMSNorm + LM head of the last new row predict the next token (the standard next-token
+#   reading of a causal decoder).  Hybrid decoding is a sequence that alternates canvases and
+#   autoregressive tokens on one cache.
+
+PHILOX_M0, PHILOX_M1 = 0xD2511F53, 0xCD9E8D57   # round multipliers
+PHILOX_W0, PHILOX_W1 = 0x9E3779B9, 0xBB67AE85   # key increments (Weyl sequence)
+_M32 = 0xFFFFFFFF
+TAG_DENOISE, TAG_NOISE, TAG_AR = 1, 2, 3          # counter word 3 = (tag << 24) | canvas
+
+
+def philox4x32_10(c0, c1, c2, c3, k0: int, k1: int):
+    """Philox4x32 with 10 rounds on 32-bit counter words (numpy arrays or ints, broadcast) and
+    the 2-word key.  A round maps (c0, c1, c2, c3) with key (k0, k1) to
+        (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)),
+    hi / lo the upper / lower 32 bits of the 64-bit product; the key grows by (W0, W1) before
+    every round after the first.  Returns the four output words as uint64 arrays (< 2^32)."""
+    c = [np.asarray(x, dtype=np.uint64) & np.uint64(_M32) for x in (c0, c1, c2, c3)]
+    c = np.broadcast_arrays(*c)
+    c = [np.array(x, dtype=np.uint64) for x in c]
+    ka, kb = int(k0) & _M32, int(k1) & _M32
+    m0, m1, m32 = np.uint64(PHILOX_M0), np.uint64(PHILOX_M1), np.uint64(_M32)
+    for r in range(10):
+        if r:
+            ka, kb = (ka + PHILOX_W0) & _M32, (kb + PHILOX_W1) & _M32
+        p0 = c[0] * m0            # < 2^64: exact in uint64
+        p1 = c[2] * m1
+        c = [(p1 >> np.uint64(32)) ^ c[1] ^ np.uint64(ka), p1 & m32,
+             (p0 >> np.uint64(32)) ^ c[3] ^ np.uint64(kb), p0 & m32]
+    return c
+
+
+def seed_key(seed: int):
+    """The generator's key: the 64-bit seed as (low word, high word)."""
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    return seed & _M32, seed >> 32
+
+
+def stream_words(seed: int, tag: int, b: int, a1: int, a2: int, n: int) -> np.ndarray:
+    """The 32-bit words w_0 .. w_{n-1} of stream (tag, b, a1, a2): w_v is word v & 3 of the
+    generator at counter (v >> 2, a1, a2, (tag << 24) | b)."""
+    v = np.arange(n, dtype=np.uint64)
+    k0, k1 = seed_key(seed)
+    words = philox4x32_10(v >> np.uint64(2), a1, a2, (int(tag) << 24) | int(b), k0, k1)
+    return np.choose((v & np.uint64(3)).astype(np.int64), words)
+
+
+def uniform_open(words: np.ndarray) -> np.ndarray:
+    """U = ((w >> 9) + 1/2) 2^-23 in (0, 1), fp64 (exact)."""
+    return ((np.asarray(words, dtype=np.uint64) >> np.uint64(9)).astype(np.float64) + 0.5) \
+        * 2.0 ** -23
+
+
+def gumbel(words: np.ndarray) -> np.ndarray:
+    """Standard Gumbel draws G = -ln(-ln U) (fp64)."""
+    return -np.log(-np.log(uniform_open(words)))
+
+
+def temperature(step: int, max_steps: int, tau_start: float, tau_end: float) -> float:
+    """tau_s, linear from tau_start at step 0 to tau_end at step max_steps - 1 (fp64)."""
+    frac = min(int(step), max_steps - 1) / max(max_steps - 1, 1)
+    return tau_start + (tau_end - tau_start) * frac
+
+
+def inv_temperature(tau: float) -> np.float32:
+    """The fp32 multiplier 1 / tau applied to the logits."""
+    return np.float32(1.0 / tau)
+
+
+def sample_row(z: np.ndarray, tau: float, g: Optional[np.ndarray]):
+    """One row of logits z [V] at temperature tau with Gumbel draws g [V].
+    Returns (entropy, token, key margin): tau <= 0 is greedy (entropy at tau = 1, margin the
+    top-1 minus top-2 logit); otherwise the entropy of softmax(z / tau), the token
+    argmax(z / tau + g) (first index among equal keys) and the margin between its two largest
+    keys."""
+    z = np.asarray(z, dtype=np.float64)[None, :]
+    if not tau > 0.0:
+        H, am, margin = entropy_argmax(z)
+        return float(H[0]), int(am[0]), float(margin[0])
+    zs = z * float(inv_temperature(tau))
+    H, _, _ = entropy_argmax(zs)
+    keys = zs[0] + g
+    tok = int(np.argmax(keys))
+    part = -np.partition(-keys, 1)
+    return float(H[0]), tok, float(part[0] - part[1])
+
+
+def noise_canvas(seed: int, batch: int, canvas: int, vocab: int) -> dict:
+    """Uniform-noise canvases: tokens [B, C] with every position not final."""
+    toks = np.zeros((batch, canvas), dtype=np.int32)
+    k0, k1 = seed_key(seed)
+    i = np.arange(canvas, dtype=np.uint64)
+    for b in range(batch):
+        w0 = philox4x32_10(i, 0, 0, (TAG_NOISE << 24) | b, k0, k1)[0]
+        toks[b] = ((w0 * np.uint64(vocab)) >> np.uint64(32)).astype(np.int32)
+    return {"tokens": toks, "masked": np.ones((batch, canvas), dtype=np.uint8),
+            "n_masked": np.full(batch, canvas, dtype=np.int32),
+            "done": np.zeros(batch, dtype=np.int32), "step": np.zeros(batch, dtype=np.int32)}
+
+
 # --------------------------------------------------------------------------- the model
 
 class OracleModel:
@@ -503,14 +632,15 @@ def lm_head_rows(cfg, model: OracleModel, x_rows: np.ndarray, keep_logits: bool 
 
 def canvas_forward(cfg, model: OracleModel, tokens: np.ndarray, masked: np.ndarray,
                    kcache: np.ndarray, vcache: np.ndarray, cache_len: int, info=None,
-                   forced=None):
+                   forced=None, drafts: bool = False):
     """Decoder pass over one canvas.  Returns the final residual stream [C, d].
 
     kcache, vcache: [L, Hkv, cap, hd] for this canvas (decoded values).  ``forced``: optional
-    expert choices [L, C, k] (see router_topk).
+    expert choices [L, C, k] (see router_topk).  ``drafts``: positions that are not final are
+    embedded by their draft token (the noise canvas) instead of MASK.
     """
     C = tokens.shape[0]
-    ids = np.where(masked != 0, cfg.mask_id, tokens)
+    ids = tokens if drafts else np.where(masked != 0, cfg.mask_id, tokens)
     x = model.emb_rows(ids)
     pos = cache_len + np.arange(C)
     for l in range(cfg.n_layers):
@@ -523,7 +653,7 @@ def canvas_forward(cfg, model: OracleModel, tokens: np.ndarray, masked: np.ndarr
 
 def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache: np.ndarray,
                 cache_len: np.ndarray, gamma: float, max_steps: int, keep_logits: bool = False,
-                forced=None):
+                forced=None, sampler: Optional[dict] = None):
     """One denoising step for every canvas of the batch that is not done.
 
     state: tokens int32 [B, C], masked uint8 [B, C], n_masked int32 [B],
@@ -534,8 +664,12 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
     positions at step index max_steps - 1); commit selected positions to their
     argmax; step += 1; done = no masked position left.
     ``forced`` (optional, [L, B, C, k]): every layer's expert choices (see router_topk).
-    Returns (new_state, info) where info[b] holds H, argmax, margin, rows,
-    selected, router margins and (optionally) logits.
+    ``sampler`` (optional): {"tau_start", "tau_end", "seed", "revise"} — the temperature-annealed
+    Gumbel-max draw of each masked position's token (tau_s of the canvas's step), the EB rule on
+    the entropies at tau_s, and with "revise" the noise-canvas drafts (see the sampler-variant
+    readings above).  Without it: greedy argmax, entropy at tau = 1, absorbing MASK positions.
+    Returns (new_state, info) where info[b] holds H, argmax (the chosen tokens), margin, rows,
+    selected, tau, router margins and (optionally) logits.
     """
     new = {k: np.array(v, copy=True) for k, v in state.items()}
     infos: List[Optional[Dict]] = []
@@ -548,15 +682,28 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
         rows = np.nonzero(masked)[0]
         info: Dict = {"rows": rows}
         if len(rows) > 0:
+            revise = bool(sampler and sampler.get("revise"))
             x = canvas_forward(cfg, model, state["tokens"][b], masked, kcache[:, b], vcache[:, b],
                                int(cache_len[b]), info,
-                               None if forced is None else forced[:, b])
-            H, am, margin, z = lm_head_rows(cfg, model, x[rows], keep_logits)
+                               None if forced is None else forced[:, b], drafts=revise)
+            H, am, margin, z = lm_head_rows(cfg, model, x[rows], keep_logits or sampler is not None)
+            if sampler is not None:
+                tau = temperature(int(state["step"][b]), max_steps, sampler["tau_start"],
+                                  sampler["tau_end"])
+                info["tau"] = tau
+                for j, i in enumerate(rows):
+                    g = None if not tau > 0.0 else gumbel(stream_words(
+                        sampler["seed"], TAG_DENOISE, b, int(i), int(state["step"][b]), cfg.vocab))
+                    H[j], am[j], margin[j] = sample_row(z[j], tau, g)
+                if not keep_logits:
+                    z = None
             Hf = H.astype(np.float32)
             full_H = np.zeros(cfg.canvas, dtype=np.float32)
             full_H[rows] = Hf
             force = state["step"][b] >= max_steps - 1
             sel = eb_select(full_H, masked, gamma, force)
+            if sampler is not None and sampler.get("revise"):   # drafts take the predictions
+                new["tokens"][b, rows] = am
             new["tokens"][b, sel] = am[np.searchsorted(rows, np.nonzero(sel)[0])]
             new["masked"][b, sel] = 0
             info.update(H=Hf, argmax=am, margin=margin, logits=z, selected=sel)
@@ -568,7 +715,7 @@ def canvas_step(cfg, model: OracleModel, state: dict, kcache: np.ndarray, vcache
 
 
 def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
-              cache_len: np.ndarray, info=None, forced=None):
+              cache_len: np.ndarray, info=None, forced=None, last_rows: Optional[list] = None):
     """Causal encoder pass over finished tokens; their K/V go to the cache.
 
     tokens int32 [B, n]; kcache/vcache decoded [L, B, Hkv, cap, hd], updated in
@@ -577,6 +724,9 @@ def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, v
     new tokens causally.  Returns the new cache_len.  With ``info`` (a dict) given, the expert
     choices of each routed layer are collected in info["router_idx"][l] as [B, n, k].
     ``forced`` (optional, [L, B, n, k]): every layer's expert choices (see router_topk).
+    ``last_rows`` (a list, optional): the last layer also runs its attention and expert FFN,
+    and the final residual row of each sequence's last new token is appended to the list (the
+    autoregressive mode's LM-head input).
     """
     B, n = tokens.shape
     new_len = np.array(cache_len, copy=True)
@@ -587,7 +737,7 @@ def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, v
         for l in range(cfg.n_layers):
             q, k, v = layer_qkv(cfg, model, l, x, pos)
             kc, vc = kcache[l, b, :, :L0], vcache[l, b, :, :L0]
-            if l + 1 < cfg.n_layers:
+            if l + 1 < cfg.n_layers or last_rows is not None:
                 li = {} if info is not None else None
                 x = layer_rest(cfg, model, l, x, q, k, v, kc, vc, True, li,
                                None if forced is None else forced[l, b])
@@ -598,7 +748,29 @@ def kv_append(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, v
             kcache[l, b, :, L0:L0 + n] = k.transpose(1, 0, 2)
             vcache[l, b, :, L0:L0 + n] = v.transpose(1, 0, 2)
         new_len[b] = L0 + n
+        if last_rows is not None:
+            last_rows.append(x[n - 1])
     return new_len
+
+
+def ar_step(cfg, model: OracleModel, tokens: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
+            cache_len: np.ndarray, tau: float = 0.0, seed: int = 0, info=None, forced=None):
+    """Autoregressive mode: append tokens [B, n] (the causal encoder; K/V into the cache, updated
+    in place), run the last layer in full, and predict each sequence's next token from the final
+    RMSNorm + LM head of its last new row.  tau > 0 draws it from softmax(z / tau) with the
+    Gumbel stream (TAG_AR, b, p, 0), p = the position of the predicted token (cache_len + n).
+    Returns (next tokens int32 [B], entropies fp32 [B], key margins [B], new cache_len, logits
+    [B, V])."""
+    B, n = tokens.shape
+    last: list = []
+    new_len = kv_append(cfg, model, tokens, kcache, vcache, cache_len, info, forced, last)
+    H, am, margin, z = lm_head_rows(cfg, model, np.stack(last), keep_logits=True)
+    for b in range(B):
+        g = None
+        if tau > 0.0:
+            g = gumbel(stream_words(seed, TAG_AR, b, int(cache_len[b]) + n, 0, cfg.vocab))
+        H[b], am[b], margin[b] = sample_row(z[b], tau, g)
+    return am.astype(np.int32), H.astype(np.float32), margin, new_len, z
 
 
 def generate(cfg, model: OracleModel, kcache, vcache, cache_len, n_canvases: int, gamma: float,
