@@ -54,9 +54,22 @@ class DgModel(ctypes.Structure):
                 ("emb_scale", ctypes.c_void_p), ("emb_scale_global", ctypes.c_float)]
 
 
+class DgSampler(ctypes.Structure):
+    """dg_sampler: temperature schedule (tau_start at step 0 .. tau_end at the last step of the
+    budget; <= 0 greedy), the generator's 64-bit seed, and revisable drafts (noise canvas)."""
+    _fields_ = [("tau_start", ctypes.c_double), ("tau_end", ctypes.c_double),
+                ("seed", ctypes.c_uint64), ("revise", ctypes.c_int32)]
+
+
+def make_sampler(tau_start=0.0, tau_end=None, seed=0, revise=False) -> DgSampler:
+    return DgSampler(float(tau_start), float(tau_start if tau_end is None else tau_end),
+                     int(seed) & 0xFFFFFFFFFFFFFFFF, 1 if revise else 0)
+
+
 _lib: Optional[ctypes.CDLL] = None
 _VP, _I32, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _PCFG, _PMODEL, _PLW = ctypes.POINTER(DgConfig), ctypes.POINTER(DgModel), ctypes.POINTER(DgLayerWeights)
+_PSMP = ctypes.POINTER(DgSampler)
 
 _SIGS = {
     "dg_workspace_size": (_SZ, [_PCFG, _I32, _I32, _I32]),
@@ -78,13 +91,20 @@ _SIGS = {
     "dg_logits_entropy_nvfp4": (_I32, [_PCFG, _I32, _VP, _VP, _VP, _VP, _VP, ctypes.c_float, _VP,
                                        _VP, _VP, _VP, _SZ, _VP, _VP]),
     "dg_eb_select": (_I32, [_I32, _I32, _VP, _VP, ctypes.c_double, _I32, _VP, _VP, _VP, _VP, _VP,
-                            _VP, _VP, _VP]),
+                            _VP, _I32, _VP, _VP]),
     "dg_kv_append": (_I32, [_PCFG, _PMODEL, _I32, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _SZ,
                             _VP, _VP]),
     "dg_canvas_step": (_I32, [_PCFG, _PMODEL, _I32, _VP, _VP, _VP, _VP, _VP, _I32, ctypes.c_double,
                               _VP, _VP, _VP, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "dg_generate": (_I32, [_PCFG, _PMODEL, _I32, _VP, _VP, _VP, _VP, _VP, _I32, ctypes.c_double,
-                           _VP, _VP, _VP, _I32, _I32, _VP, _SZ, _VP, _VP]),
+                           _PSMP, _VP, _VP, _VP, _I32, _I32, _VP, _SZ, _VP, _VP]),
+    "dg_canvas_step_sampler": (_I32, [_PCFG, _PMODEL, _I32, _VP, _VP, _VP, _VP, _VP, _I32,
+                                      ctypes.c_double, _PSMP, _VP, _VP, _VP, _I32, _VP, _VP, _VP,
+                                      _VP, _VP, _SZ, _VP, _VP]),
+    "dg_debug_wait_probe": (_I32, [ctypes.c_longlong, _I32, _VP, _VP]),
+    "dg_noise_canvas": (_I32, [_I32, _I32, _I32, ctypes.c_uint64, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "dg_ar_step": (_I32, [_PCFG, _PMODEL, _I32, _VP, _I32, _VP, _VP, _VP, _I32, _PSMP, _VP, _VP,
+                          _VP, _VP, _VP, _SZ, _VP, _VP]),
 }
 
 
@@ -260,10 +280,10 @@ def dg_logits_entropy_nvfp4(cfg, n_rows, n_rows_dev, h, row_idx, w_codes, w_scal
 
 
 def dg_eb_select(batch, canvas, entropy, argmax, gamma, max_steps, tokens, masked, selected,
-                 n_masked, done, step, dev_status=None, stream=None):
+                 n_masked, done, step, dev_status=None, stream=None, revise=False):
     _check(lib().dg_eb_select(batch, canvas, _p(entropy), _p(argmax), float(gamma), max_steps,
                               _p(tokens), _p(masked), _p(selected), _p(n_masked), _p(done), _p(step),
-                              _p(dev_status), _stream(stream)), "dg_eb_select")
+                              1 if revise else 0, _p(dev_status), _stream(stream)), "dg_eb_select")
 
 
 def dg_kv_append(cfg, model: Model, batch, tokens, n_tokens, k_cache, v_cache, cache_len, cache_cap,
@@ -288,15 +308,58 @@ def dg_canvas_step(cfg, model: Model, batch, tokens, masked, n_masked, done, ste
 
 
 def dg_generate(cfg, model: Model, batch, tokens, masked, n_masked, done, step, max_steps, gamma,
-                k_cache, v_cache, cache_len, cache_cap, append, ws, dev_status=None, stream=None):
+                k_cache, v_cache, cache_len, cache_cap, append, ws, dev_status=None, stream=None,
+                sampler: Optional[DgSampler] = None):
     """The step loop on the device until every canvas is done (one CUDA graph with a
     conditional while node, cached per argument set), then the append if `append`."""
     w, wb = _ws(ws)
     _check(lib().dg_generate(ctypes.byref(cfg), ctypes.byref(model.struct), batch, _p(tokens),
                              _p(masked), _p(n_masked), _p(done), _p(step), max_steps, float(gamma),
+                             None if sampler is None else ctypes.byref(sampler),
                              _p(k_cache), _p(v_cache), _p(cache_len), cache_cap, int(append), w, wb,
                              _p(dev_status), _stream(stream)),
            "dg_generate")
+
+
+def dg_canvas_step_sampler(cfg, model: Model, batch, tokens, masked, n_masked, done, step,
+                           max_steps, gamma, sampler: DgSampler, k_cache, v_cache, cache_len,
+                           cache_cap, entropy_out, argmax_out, logits_dbg, ws, dev_status=None,
+                           stream=None, forced_topk=None):
+    """dg_canvas_step with a sampler variant (temperature-annealed draws, revisable drafts)."""
+    w, wb = _ws(ws)
+    _check(lib().dg_canvas_step_sampler(ctypes.byref(cfg), ctypes.byref(model.struct), batch,
+                                        _p(tokens), _p(masked), _p(n_masked), _p(done), _p(step),
+                                        max_steps, float(gamma), ctypes.byref(sampler),
+                                        _p(k_cache), _p(v_cache), _p(cache_len), cache_cap,
+                                        _p(entropy_out), _p(argmax_out), _p(logits_dbg),
+                                        _p(forced_topk), w, wb, _p(dev_status), _stream(stream)),
+           "dg_canvas_step_sampler")
+
+
+def dg_noise_canvas(batch, canvas, vocab, seed, tokens, masked, n_masked, done, step, stream=None):
+    """Uniform-noise canvases (every position a revisable draft)."""
+    _check(lib().dg_noise_canvas(batch, canvas, vocab, int(seed) & 0xFFFFFFFFFFFFFFFF, _p(tokens),
+                                 _p(masked), _p(n_masked), _p(done), _p(step), _stream(stream)),
+           "dg_noise_canvas")
+
+
+def dg_ar_step(cfg, model: Model, batch, tokens, n_tokens, k_cache, v_cache, cache_len, cache_cap,
+               next_token, entropy, logits_dbg, ws, dev_status=None, stream=None,
+               sampler: Optional[DgSampler] = None, forced_topk=None):
+    """Autoregressive mode: append the tokens, predict each sequence's next token."""
+    w, wb = _ws(ws)
+    _check(lib().dg_ar_step(ctypes.byref(cfg), ctypes.byref(model.struct), batch, _p(tokens),
+                            n_tokens, _p(k_cache), _p(v_cache), _p(cache_len), cache_cap,
+                            None if sampler is None else ctypes.byref(sampler), _p(next_token),
+                            _p(entropy), _p(logits_dbg), _p(forced_topk), w, wb, _p(dev_status),
+                            _stream(stream)),
+           "dg_ar_step")
+
+
+def dg_debug_wait_probe(limit_cycles, arrive, dev_status, stream=None):
+    """Run the bounded device wait alone (see dg.h); expiry records DG_ERR_TIMEOUT."""
+    _check(lib().dg_debug_wait_probe(int(limit_cycles), 1 if arrive else 0, _p(dev_status),
+                                     _stream(stream)), "dg_debug_wait_probe")
 
 
 def exported_symbols() -> Sequence[str]:

@@ -395,7 +395,7 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
 int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_rows_dev,
                const void *h, const int32_t *row_idx, const LmWeights &lw, float *entropy,
                int32_t *argmax, float *logits_out, int scatter_logits, int32_t *st,
-               cudaStream_t s) {
+               cudaStream_t s, const SampleSpec *smp = nullptr) {
   const void *w_lm = lw.w;
   if (h)  // an NVFP4 LM head multiplies fp16 rows
     DG_TRY(launch_rmsnorm(c.act_dtype, h, row_idx, n_rows_dev, max_rows, c.d_model, c.rms_eps,
@@ -404,11 +404,11 @@ int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_
     return launch_lmhead_q4(ws.at<void>(B_FIN), max_rows, n_rows_dev,
                             static_cast<const uint8_t *>(lw.w), lw.scale, lw.g, c.vocab,
                             c.d_model, row_idx, entropy, argmax, logits_out,
-                            scatter_logits ? row_idx : nullptr, ws.at<void>(B_PART), st, s);
+                            scatter_logits ? row_idx : nullptr, ws.at<void>(B_PART), st, s, smp);
   if (lmhead_tc_supported(c.act_dtype, c.d_model))
     return launch_lmhead_tc(ws.at<void>(B_FIN), max_rows, n_rows_dev, w_lm, c.vocab, c.d_model,
                             row_idx, entropy, argmax, logits_out,
-                            scatter_logits ? row_idx : nullptr, ws.at<void>(B_PART), st, s);
+                            scatter_logits ? row_idx : nullptr, ws.at<void>(B_PART), st, s, smp);
   float *logits = (logits_out && !scatter_logits) ? logits_out : ws.at<float>(B_LOGITS);
   GemmDesc g{};
   g.act = c.act_dtype; g.w = c.act_dtype;
@@ -418,7 +418,7 @@ int lm_entropy(const dg_config &c, const Ws &ws, int max_rows, const int32_t *n_
   g.name = "lm_head_logits";
   DG_TRY(launch_gemm_simt(g, EPI_F32, logits, c.vocab, nullptr, s));
   DG_TRY(launch_entropy_rows(logits, c.vocab, max_rows, n_rows_dev, row_idx, entropy, argmax, st,
-                             s));
+                             s, smp));
   if (logits_out && scatter_logits)
     DG_TRY(launch_scatter_rows(logits, c.vocab, max_rows, n_rows_dev, row_idx, logits_out, s));
   return DG_OK;
@@ -429,6 +429,25 @@ long long quant_gamma(double gamma) {
   const double v = std::floor(gamma * 4294967296.0);
   if (v >= 9.2233720368547758e18) return INT64_MAX;
   return (long long)v;
+}
+
+bool sampler_ok(const dg_sampler *smp) {
+  return !smp || (std::isfinite(smp->tau_start) && std::isfinite(smp->tau_end));
+}
+
+// The LM head's draw for canvas rows: greedy unless the schedule has a positive temperature.
+SampleSpec canvas_spec(const dg_sampler *smp, const int32_t *step, int canvas, int max_steps) {
+  SampleSpec sp{};
+  if (!smp || !(smp->tau_start > 0.0 || smp->tau_end > 0.0)) return sp;
+  sp.mode = SAMPLE_CANVAS;
+  sp.step = step;
+  sp.canvas = canvas;
+  sp.max_steps = max_steps;
+  sp.tau0 = smp->tau_start;
+  sp.tau1 = smp->tau_end;
+  sp.key0 = (uint32_t)(smp->seed & 0xFFFFFFFFu);
+  sp.key1 = (uint32_t)(smp->seed >> 32);
+  return sp;
 }
 
 int check_ws(const dg_config *c, int batch, int n, int cap, const void *ws, size_t ws_bytes,
@@ -570,6 +589,11 @@ const char *dg_profile_name(int i) {
   return g_prof.name[i];
 }
 
+int dg_debug_wait_probe(long long limit_cycles, int arrive, int32_t *dev_status, void *stream) {
+  if (limit_cycles < 1 || limit_cycles > 4000000000LL || !dev_status) return DG_ERR_INVALID_ARG;
+  return launch_wait_probe(limit_cycles, arrive ? 1 : 0, dev_status, (cudaStream_t)stream);
+}
+
 int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
                    const void *k_cache, const void *v_cache, const int32_t *cache_len,
                    int cache_cap, const void *k_new, const void *v_new, int causal,
@@ -664,7 +688,7 @@ int dg_logits_entropy_nvfp4(const dg_config *cfg, int n_rows, const int32_t *n_r
 
 int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
                  double gamma, int max_steps, int32_t *tokens, uint8_t *masked,
-                 uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
+                 uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step, int revise,
                  int32_t *dev_status, void *stream) {
   if (batch <= 0 || canvas <= 0 || canvas > 1024 || max_steps <= 0) return DG_ERR_INVALID_ARG;
   if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
@@ -672,7 +696,7 @@ int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *arg
     return DG_ERR_INVALID_ARG;
   return launch_eb_select(batch, canvas, entropy, argmax, quant_gamma(gamma), max_steps, tokens,
                           masked, selected, n_masked, done, step, dev_status,
-                          (cudaStream_t)stream);
+                          (cudaStream_t)stream, revise ? 1 : 0);
 }
 
 int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
@@ -725,15 +749,91 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
   return launch_add_cache_len(batch, n_tokens, cache_cap, cache_len, s);
 }
 
-int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
-                   uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
-                   int max_steps, double gamma, const void *k_cache, const void *v_cache,
-                   const int32_t *cache_len, int cache_cap, float *entropy_out,
-                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load,
-                   const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
-                   void *stream) {
+int dg_ar_step(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
+               int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
+               const dg_sampler *smp, int32_t *next_token, float *entropy, float *logits_dbg,
+               const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+               void *stream) {
+  if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || n_tokens <= 0)
+    return DG_ERR_INVALID_ARG;
+  if (!tokens || !k_cache || !v_cache || !cache_len || cache_cap <= 0 || !next_token)
+    return DG_ERR_INVALID_ARG;
+  if (!sampler_ok(smp)) return DG_ERR_INVALID_ARG;
+  if (n_tokens > cache_cap) return DG_ERR_CAPACITY;
+  for (int l = 0; l < cfg->n_layers; ++l)
+    if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
+  const LmWeights emb = lm_weights(*cfg, model);
+  if (!lm_weights_ok(*cfg, emb)) return DG_ERR_INVALID_ARG;
+  Layout L;
+  DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
+  Ws w{(char *)ws, &L};
+  const dg_config &c = *cfg;
+  const cudaStream_t s = (cudaStream_t)stream;
+  const int T = batch * n_tokens, d = c.d_model;
+  const size_t layer_elems = (size_t)batch * c.n_kv_heads * cache_cap * c.head_dim;
+  const size_t ae = esz(c.act_dtype);
+  int32_t *slot = w.at<int32_t>(B_SLOT);
+  DG_TRY(launch_prologue(c.act_dtype, tokens, nullptr, model->emb, T, d, c.vocab, c.rms_eps,
+                         w.at<void>(B_X), w.at<void>(B_A), dev_status, batch, n_tokens, c.head_dim,
+                         c.rope_theta, cache_len, w.at<float>(B_CS), nullptr, nullptr, nullptr,
+                         nullptr, nullptr, s, emb.scale, emb.g));
+  DG_TRY(launch_last_row_slots(batch, n_tokens, slot, s));
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights &lw = model->layers[l];
+    char *kc = (char *)k_cache + l * layer_elems * ae;
+    char *vc = (char *)v_cache + l * layer_elems * ae;
+    DG_TRY(qkv_proj(c, lw, w, T, s));
+    DG_TRY(launch_qkv_split(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                            w.at<float>(B_QKV), qkv_parts(c, T), w.at<float>(B_CS), w.at<void>(B_Q),
+                            w.at<void>(B_KN), w.at<void>(B_VN), kc, vc, cache_len, cache_cap,
+                            dev_status, s));
+    DG_TRY(launch_attention(c.act_dtype, batch, n_tokens, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                            w.at<void>(B_Q), kc, vc, cache_len, cache_cap, w.at<void>(B_KN),
+                            w.at<void>(B_VN), 1, nullptr, w.at<void>(B_O),
+                            w.at<void>(B_ATTN), dev_status, s));
+    bool tiles_ready = false;
+    DG_TRY(attn_out_and_route(c, lw, w, T, nullptr, nullptr, &tiles_ready, s,
+                              forced_topk ? forced_topk + (size_t)l * T * c.top_k : nullptr));
+    // the last layer's combine writes the final-norm row of each sequence's last token
+    const bool last = l + 1 == c.n_layers;
+    DG_TRY(moe_experts(c, lw, w, T, w.at<void>(B_Y), w.at<int32_t>(B_IDX), w.at<float>(B_W),
+                       w.at<int32_t>(B_OFF), w.at<int32_t>(B_PERM), w.at<int32_t>(B_INV),
+                       w.at<void>(B_H), w.at<void>(B_X), s, tiles_ready, nullptr,
+                       last ? nullptr : w.at<void>(B_A), last ? slot : nullptr,
+                       last ? w.at<void>(B_FIN) : nullptr));
+  }
+  SampleSpec sp{};
+  if (smp && smp->tau_start > 0.0) {
+    sp.mode = SAMPLE_AR;
+    sp.pos = cache_len;
+    sp.pos_add = n_tokens;
+    sp.tau0 = smp->tau_start;
+    sp.key0 = (uint32_t)(smp->seed & 0xFFFFFFFFu);
+    sp.key1 = (uint32_t)(smp->seed >> 32);
+  }
+  DG_TRY(lm_entropy(c, w, batch, nullptr, nullptr, nullptr, emb,
+                    entropy ? entropy : w.at<float>(B_ENT), next_token, logits_dbg, 0, dev_status,
+                    s, &sp));
+  return launch_add_cache_len(batch, n_tokens, cache_cap, cache_len, s);
+}
+
+}  // extern "C"
+
+namespace dg {
+namespace {
+
+// One denoising step (dg_canvas_step), with the sampler variant `smp` (null: greedy argmax,
+// entropy at tau = 1, masked positions embedded as MASK).
+int canvas_step_impl(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
+                     uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
+                     int max_steps, double gamma, const void *k_cache, const void *v_cache,
+                     const int32_t *cache_len, int cache_cap, float *entropy_out,
+                     int32_t *argmax_out, float *logits_dbg, int32_t *expert_load,
+                     const int32_t *forced_topk, const dg_sampler *smp, void *ws,
+                     size_t ws_bytes, int32_t *dev_status, void *stream) {
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
     return DG_ERR_INVALID_ARG;
+  if (!sampler_ok(smp)) return DG_ERR_INVALID_ARG;
   if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
   if (cache_cap < 0 || (cache_cap > 0 && (!k_cache || !v_cache))) return DG_ERR_INVALID_ARG;
   if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
@@ -753,10 +853,11 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
   int32_t *rows = w.at<int32_t>(B_ROWS), *n_rows = w.at<int32_t>(B_NROWS);
 
   int32_t *slot = w.at<int32_t>(B_SLOT);
+  const int revise = smp && smp->revise ? 1 : 0;
   DG_TRY(launch_prologue(c.act_dtype, tokens, masked, model->emb, T, d, c.vocab, c.rms_eps,
                          w.at<void>(B_X), w.at<void>(B_A), dev_status, batch, C, c.head_dim,
                          c.rope_theta, cache_len, w.at<float>(B_CS), done, rows, n_rows, slot, live,
-                         s, emb.scale, emb.g));
+                         s, emb.scale, emb.g, revise));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights &lw = model->layers[l];
     const char *kc = (const char *)k_cache + l * layer_elems * ae;
@@ -785,22 +886,66 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
   }
   float *ent = entropy_out ? entropy_out : w.at<float>(B_ENT);
   int32_t *am = argmax_out ? argmax_out : w.at<int32_t>(B_AM);
+  const SampleSpec sp = canvas_spec(smp, step, C, max_steps);
   DG_TRY(lm_entropy(c, w, T, n_rows, nullptr, rows, emb, ent, am, logits_dbg, 1, dev_status,
-                    s));
+                    s, &sp));
   return launch_eb_select(batch, C, ent, am, quant_gamma(gamma), max_steps, tokens, masked,
-                          nullptr, n_masked, done, step, dev_status, s);
+                          nullptr, n_masked, done, step, dev_status, s, revise);
+}
+
+}  // namespace
+}  // namespace dg
+
+extern "C" {
+
+int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
+                   uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
+                   int max_steps, double gamma, const void *k_cache, const void *v_cache,
+                   const int32_t *cache_len, int cache_cap, float *entropy_out,
+                   int32_t *argmax_out, float *logits_dbg, int32_t *expert_load,
+                   const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+                   void *stream) {
+  return canvas_step_impl(cfg, model, batch, tokens, masked, n_masked, done, step, max_steps,
+                          gamma, k_cache, v_cache, cache_len, cache_cap, entropy_out, argmax_out,
+                          logits_dbg, expert_load, forced_topk, nullptr, ws, ws_bytes, dev_status,
+                          stream);
+}
+
+int dg_canvas_step_sampler(const dg_config *cfg, const dg_model *model, int batch,
+                           int32_t *tokens, uint8_t *masked, int32_t *n_masked, int32_t *done,
+                           int32_t *step, int max_steps, double gamma, const dg_sampler *smp,
+                           const void *k_cache, const void *v_cache, const int32_t *cache_len,
+                           int cache_cap, float *entropy_out, int32_t *argmax_out,
+                           float *logits_dbg, const int32_t *forced_topk, void *ws,
+                           size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!smp) return DG_ERR_INVALID_ARG;
+  return canvas_step_impl(cfg, model, batch, tokens, masked, n_masked, done, step, max_steps,
+                          gamma, k_cache, v_cache, cache_len, cache_cap, entropy_out, argmax_out,
+                          logits_dbg, nullptr, forced_topk, smp, ws, ws_bytes, dev_status,
+                          stream);
+}
+
+int dg_noise_canvas(int batch, int canvas, int vocab, uint64_t seed, int32_t *tokens,
+                    uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
+                    void *stream) {
+  if (batch <= 0 || canvas <= 0 || canvas > 1024 || vocab < 1) return DG_ERR_INVALID_ARG;
+  if (!tokens || !masked || !n_masked || !done || !step) return DG_ERR_INVALID_ARG;
+  return launch_noise_canvas(batch, canvas, vocab, (uint32_t)(seed & 0xFFFFFFFFu),
+                             (uint32_t)(seed >> 32), tokens, masked, n_masked, done, step,
+                             (cudaStream_t)stream);
 }
 
 int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
                 uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step, int max_steps,
-                double gamma, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
-                int append, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+                double gamma, const dg_sampler *smp, void *k_cache, void *v_cache,
+                int32_t *cache_len, int cache_cap, int append, void *ws, size_t ws_bytes,
+                int32_t *dev_status, void *stream) {
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
   if (cache_cap < 0 || (cache_cap > 0 && (!k_cache || !v_cache))) return DG_ERR_INVALID_ARG;
   if (append && (cache_cap <= 0 || cfg->canvas > cache_cap)) return DG_ERR_INVALID_ARG;
-  if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
+  if (!(gamma >= 0.0) || !sampler_ok(smp)) return DG_ERR_INVALID_ARG;
   for (int l = 0; l < cfg->n_layers; ++l)
     if (!lw_ok(cfg, &model->layers[l])) return DG_ERR_INVALID_ARG;
   if (!lm_weights_ok(*cfg, lm_weights(*cfg, model))) return DG_ERR_INVALID_ARG;
@@ -825,6 +970,12 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
   key_add(key, batch);
   key_add(key, max_steps);
   key_add(key, gamma);
+  const dg_sampler no_smp{0.0, 0.0, 0, 0};
+  key_add(key, smp ? smp->tau_start : no_smp.tau_start);
+  key_add(key, smp ? smp->tau_end : no_smp.tau_end);
+  key_add(key, smp ? smp->seed : no_smp.seed);
+  key_add(key, smp ? smp->revise : no_smp.revise);
+  key_add(key, smp != nullptr);
   key_add(key, cache_cap);
   key_add(key, ws_bytes);
 
@@ -872,9 +1023,10 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
         return cuda_fail("dg_generate graph", e);
       }
       pdl_allowed() = attempt == 0;
-      int src = dg_canvas_step(cfg, model, batch, tokens, masked, n_masked, done, step, max_steps,
-                               gamma, k_cache, v_cache, cache_len, cache_cap, nullptr, nullptr,
-                               nullptr, nullptr, nullptr, ws, ws_bytes, dev_status, cs);
+      int src = canvas_step_impl(cfg, model, batch, tokens, masked, n_masked, done, step,
+                                 max_steps, gamma, k_cache, v_cache, cache_len, cache_cap, nullptr,
+                                 nullptr, nullptr, nullptr, nullptr, smp, ws, ws_bytes, dev_status,
+                                 cs);
       if (src == DG_OK) {
         gen_cond_kernel<<<1, 1, 0, cs>>>(h, done, batch, iter, max_steps + 1, dev_status);
         src = check_launch("gen_cond");

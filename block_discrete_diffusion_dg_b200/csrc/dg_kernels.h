@@ -19,12 +19,13 @@ int launch_embed_norm(int act, const int32_t *tokens, const uint8_t *masked, con
                       int32_t *st, cudaStream_t s);
 // Embedding + pre-norm of `rows` rows, the RoPE table, and (row_idx non-null) the compaction of
 // the rows needing logits (row_idx, *n_rows, slot [rows]: index in row_idx or -1, token_live).
+// drafts: masked rows are embedded by their token (a revisable draft) instead of MASK.
 int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const void *emb, int rows,
                     int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
                     int n, int hd, double theta, const int32_t *cache_len, float *cs,
                     const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
                     uint8_t *token_live, cudaStream_t s, const uint8_t *emb_scale = nullptr,
-                    float emb_g = 1.0f);
+                    float emb_g = 1.0f, int drafts = 0);
 // Rows of an NVFP4 matrix of `rows` rows as stored (padded to a multiple of 256).
 inline int nvfp4_rows_pad(int rows) { return (rows + 255) / 256 * 256; }
 // e4m3 codes [n] -> bf16 [n] (n % 16 == 0), exact.
@@ -136,12 +137,40 @@ int launch_combine(int act, int T, int d, int k, const int32_t *topk_idx, const 
                    const int32_t *inv_perm, const void *Y, const void *res, void *out,
                    cudaStream_t s);
 
+// ---- sampler variants (sampler.cuh) -----------------------------------------------------------
+// How the LM-head kernels turn logits into a token: greedy (argmax, entropy at tau = 1), or the
+// Gumbel-max draw at a per-row temperature (entropy of softmax(z / tau)) for canvas rows (source
+// row b * canvas + i; tau annealed with step[b]) or autoregressive rows (source row b; tau0).
+enum { SAMPLE_GREEDY = 0, SAMPLE_CANVAS = 1, SAMPLE_AR = 2 };
+enum { SAMPLE_TAG_DENOISE = 1, SAMPLE_TAG_NOISE = 2, SAMPLE_TAG_AR = 3 };
+struct SampleSpec {
+  int mode;              // SAMPLE_*
+  const int32_t *step;   // SAMPLE_CANVAS: per-canvas step counters (device)
+  const int32_t *pos;    // SAMPLE_AR: per-sequence cache length before the append (device)
+  int canvas, pos_add, max_steps;
+  double tau0, tau1;     // temperature at step 0 and at step max_steps - 1
+  uint32_t key0, key1;   // generator key: the seed's low and high words
+};
+
+// Uniform-noise canvases: tokens[b][i] = (w0 * vocab) >> 32 for the first word w0 of stream
+// (TAG_NOISE, b, i, 0); masked = 1, n_masked = canvas, done = 0, step = 0.
+int launch_noise_canvas(int batch, int canvas, int vocab, uint32_t key0, uint32_t key1,
+                        int32_t *tokens, uint8_t *masked, int32_t *n_masked, int32_t *done,
+                        int32_t *step, cudaStream_t s);
+// slot[t] = b for the last of the n tokens of sequence b (t = b n + n - 1), -1 otherwise.
+int launch_last_row_slots(int batch, int n, int32_t *slot, cudaStream_t s);
+
+// Bounded-wait probe (k_debug.cu): one CTA holds TMEM and waits at most limit_cycles on an
+// mbarrier phase that completes only if `arrive`; on expiry DG_ERR_TIMEOUT goes to *st.
+int launch_wait_probe(long long limit_cycles, int arrive, int32_t *st, cudaStream_t s);
+
 // ---- entropy / argmax (k_entropy.cu) -----------------------------------------------------------
 // From materialised fp32 logits [rows][V]: per row r < *n_rows: H and argmax stored at
 // out index row_idx ? row_idx[r] : r.
+// smp (or null: greedy): the draw of each row's token (source row = row_idx ? row_idx[r] : r).
 int launch_entropy_rows(const float *logits, int V, int max_rows, const int32_t *n_rows,
                         const int32_t *row_idx, float *entropy, int32_t *argmax, int32_t *st,
-                        cudaStream_t s);
+                        cudaStream_t s, const SampleSpec *smp = nullptr);
 
 // ---- LM head on tensor cores with fused entropy (k_lmhead_tc.cu) ----------------------------
 // F: normalised rows [roundup(max_rows, 128)][K] bf16 (rows >= *n_rows_dev ignored); w_lm [V][K].
@@ -154,12 +183,14 @@ bool lmhead_tc_supported(int act, int d);
 int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, const uint8_t *codes,
                      const uint8_t *scales, float gscale, int V, int K, const int32_t *row_idx,
                      float *entropy, int32_t *argmax, float *logits, const int32_t *logits_rows,
-                     void *ws, int32_t *st, cudaStream_t s);
+                     void *ws, int32_t *st, cudaStream_t s, const SampleSpec *smp = nullptr);
 size_t lmhead_tc_ws_bytes(int max_rows, int V);
+// smp (or null: greedy): each row's token drawn as SampleSpec says (source row as the outputs);
+// the debug logits stay the raw z.
 int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,
                      int V, int K, const int32_t *row_idx, float *entropy, int32_t *argmax,
                      float *logits, const int32_t *logits_rows, void *ws, int32_t *st,
-                     cudaStream_t s);
+                     cudaStream_t s, const SampleSpec *smp = nullptr);
 
 // ---- tensor-core GEMMs (k_gemm_tc.cu) -----------------------------------------------------------
 bool gemm_tc_supported(int act, int w, int K);
@@ -183,9 +214,10 @@ int launch_gemm_tc_experts(int gate_up, const void *W, int E, int w_rows, int F,
 int experts_tc_tile_tokens();
 
 // ---- EB select (k_eb.cu) -------------------------------------------------------------------
+// revise: masked positions that are not committed take argmax as their new draft token.
 int launch_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
                      long long q_gamma, int max_steps, int32_t *tokens, uint8_t *masked,
                      uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
-                     int32_t *st, cudaStream_t s);
+                     int32_t *st, cudaStream_t s, int revise = 0);
 
 }  // namespace dg

@@ -32,6 +32,16 @@ struct EntState {
       u = fmaf(e, z - m, u);
     }
   }
+  // Sampler variants: the softmax state takes the scaled logit v, the argmax the key (v plus a
+  // Gumbel draw); indices of one state arrive in increasing order.
+  __device__ __forceinline__ void add_keyed(float v, float key, int i) {
+    const float av0 = av;
+    const int am0 = am;
+    add(v, i);
+    av = av0;
+    am = am0;
+    if (key > av) { av = key; am = i; }
+  }
   __device__ __forceinline__ void merge(const EntState &o) {
     if (o.av > av || (o.av == av && o.am < am)) { av = o.av; am = o.am; }
     if (o.s <= 0.f) return;

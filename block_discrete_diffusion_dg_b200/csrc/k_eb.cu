@@ -26,7 +26,8 @@ __global__ void __launch_bounds__(1024) eb_kernel(int C, const float *__restrict
                                                   const int32_t *__restrict__ am, long long qg,
                                                   int max_steps, int32_t *tokens, uint8_t *masked,
                                                   uint8_t *selected, int32_t *n_masked,
-                                                  int32_t *done, int32_t *step, int32_t *st) {
+                                                  int32_t *done, int32_t *step, int32_t *st,
+                                                  int revise) {
   pdl_wait();
   pdl_trigger();
   __shared__ unsigned long long keys[1024];
@@ -74,6 +75,8 @@ __global__ void __launch_bounds__(1024) eb_kernel(int C, const float *__restrict
         tokens[base + tid] = am[base + tid];
         masked[base + tid] = 0;
         atomicAdd(&n_commit, 1);
+      } else if (revise) {
+        tokens[base + tid] = am[base + tid];  // the draft takes this step's prediction
       }
     }
     if (selected) selected[base + tid] = commit ? 1 : 0;
@@ -92,13 +95,13 @@ __global__ void __launch_bounds__(1024) eb_kernel(int C, const float *__restrict
 int launch_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
                      long long q_gamma, int max_steps, int32_t *tokens, uint8_t *masked,
                      uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
-                     int32_t *st, cudaStream_t s) {
+                     int32_t *st, cudaStream_t s, int revise) {
   if (batch <= 0) return DG_OK;
   int N = 32;
   while (N < canvas) N <<= 1;
   note_launch(s, "eb_select");
   launch_pdl(eb_kernel, batch, N, 0, s, canvas, entropy, argmax, q_gamma, max_steps, tokens, masked,
-                                selected, n_masked, done, step, st);
+                                selected, n_masked, done, step, st, revise);
   return check_launch("eb_select");
 }
 

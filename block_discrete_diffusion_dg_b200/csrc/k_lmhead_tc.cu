@@ -18,9 +18,14 @@
 // working on the same vocabulary tile run together and share it through L2.
 // Every wait is bounded (tc::WAIT_LIMIT_CYCLES); on expiry the kernel records DG_ERR_TIMEOUT,
 // drains what it issued, frees TMEM and returns.
+// Sampler variants (SAMPLE = true instantiations): each row's logits are multiplied by its 1/tau
+// and its token is the argmax of z/tau + Gumbel noise drawn from the row's counter stream (the
+// report's annealed-temperature sampler, Figures 9 and 10; see sampler.cuh); the entropy is that
+// of softmax(z/tau).  A greedy row (tau <= 0) in such a launch keeps tau = 1 and no noise.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 #include "entropy_state.cuh"
+#include "sampler.cuh"
 #include "tc_common.cuh"
 #include "tc_host.h"
 
@@ -50,6 +55,9 @@ struct Params {
   const uint8_t *q_codes, *q_scales;
   int rows_pad;
   float gscale;
+  // sampler variants: the draw of each row's token (source row = row_src ? row_src[r] : r)
+  SampleSpec smp;
+  const int32_t *row_src;
 };
 
 __device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
@@ -65,15 +73,24 @@ __device__ __forceinline__ void fail(int32_t *st, volatile int *abort_flag) {
 // unrolled loop made every column its own dependent block, and the epilogue took ~14 us per
 // 256-column tile instead of ~5).  A ragged chunk (the end of the vocabulary) tests each column.
 // SCALED: the logits are the accumulator values times gs (the NVFP4 tensor scale).
-template <bool SCALED = false>
+// SAMPLE: the logits are further multiplied by the row's 1/tau (rd), the softmax state is that of
+// the scaled logits, and av / am track the maximum of the keys z/tau + G (G = 0 for a greedy row)
+// instead of the logits.
+template <bool SCALED = false, bool SAMPLE = false>
 __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, int col0, float &m,
-                                          float &s, float &u, float &av, int &am, float gs = 1.f) {
+                                          float &s, float &u, float &av, int &am, float gs = 1.f,
+                                          const RowDraw *rd = nullptr, uint32_t k0 = 0u,
+                                          uint32_t k1 = 0u) {
   float cm, cs, cu;
   float mn;
+  const float mul = SAMPLE ? rd->inv_tau : 1.f;
   if (nvalid == 32) {
     float v[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
+    for (int j = 0; j < 32; ++j) {
+      v[j] = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
+      if (SAMPLE) v[j] *= mul;
+    }
     float t[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
@@ -82,7 +99,7 @@ __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, i
 #pragma unroll
       for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
     cm = t[0];
-    if (cm > av) {
+    if (!SAMPLE && cm > av) {
       uint32_t bits = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) bits |= (v[j] == cm) ? (1u << j) : 0u;
@@ -100,26 +117,77 @@ __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, i
     }
     cs = (ps[0] + ps[1]) + (ps[2] + ps[3]);
     cu = (pu[0] + pu[1]) + (pu[2] + pu[3]);
+    if (SAMPLE) {  // keys = scaled logits + Gumbel draws; first maximum
+      if (rd->on) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 g = gumbel4(*rd, (uint32_t)(col0 >> 2) + q, k0, k1);
+          v[4 * q] += g.x;
+          v[4 * q + 1] += g.y;
+          v[4 * q + 2] += g.z;
+          v[4 * q + 3] += g.w;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+      const float ck = t[0];
+      if (ck > av) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) bits |= (v[j] == ck) ? (1u << j) : 0u;
+        av = ck;
+        am = col0 + __ffs(bits) - 1;
+      }
+    }
   } else {
     cm = -INFINITY;
     int ci = 0;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const float v = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
+      float v = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
+      if (SAMPLE) v *= mul;
       if (j < nvalid && v > cm) { cm = v; ci = j; }
     }
-    if (cm > av) { av = cm; am = col0 + ci; }
+    if (!SAMPLE && cm > av) { av = cm; am = col0 + ci; }
     mn = fmaxf(m, cm);
     cs = 0.f;
     cu = 0.f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       if (j < nvalid) {
-        const float d = (SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j])) - mn;
+        float v = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
+        if (SAMPLE) v *= mul;
+        const float d = v - mn;
         const float e = __expf(d);
         cs += e;
         cu = fmaf(e, d, cu);
       }
+    }
+    if (SAMPLE) {
+      float ck = -INFINITY;
+      int ck_i = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (4 * q < nvalid) {
+          const float4 g = rd->on ? gumbel4(*rd, (uint32_t)(col0 >> 2) + q, k0, k1)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * q + e;
+            if (j < nvalid) {
+              float v = SCALED ? __uint_as_float(r[j]) * gs : __uint_as_float(r[j]);
+              v = v * mul + gg[e];
+              if (v > ck) { ck = v; ck_i = j; }
+            }
+          }
+        }
+      }
+      if (ck > av) { av = ck; am = col0 + ck_i; }
     }
   }
   if (s > 0.f) {
@@ -132,6 +200,7 @@ __device__ __forceinline__ void ent_chunk(const uint32_t (&r)[32], int nvalid, i
   m = mn;
 }
 
+template <bool SAMPLE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, Params p) {
@@ -254,6 +323,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       fence_after();
       const int row = mt * BM + q * 32 + lane;
       const bool row_ok = row < n_rows;
+      RowDraw rd{1.f, 0, 0u, 0u, 0u};
+      if (SAMPLE && row_ok) rd = row_draw(p.smp, p.row_src ? p.row_src[row] : row);
       float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
       int am = 0x7fffffff;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
@@ -268,7 +339,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tbase + c * 32, r);
         tmem_ld_wait(r);
         const int nvalid = min(32, p.V - col0);
-        ent_chunk(r, nvalid, col0, m, s, uu, av, am);
+        ent_chunk<false, SAMPLE>(r, nvalid, col0, m, s, uu, av, am, 1.f, &rd, p.smp.key0,
+                                 p.smp.key1);
         if (lrow) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -316,6 +388,7 @@ constexpr int PB_BYTES = (BN / 2) * BK * 2;  // this CTA's 128 of the unit's 256
 constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * (PA_BYTES + PB_BYTES) + 256;
 static_assert(P_SMEM_BYTES <= 232448, "more shared memory than one CTA may have");
 
+template <bool SAMPLE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     lmhead_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, Params p) {
@@ -442,6 +515,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       fence_after();
       const int row = mp * 2 * BM + (int)rank * BM + q * 32 + lane;
       const bool row_ok = row < n_rows;
+      RowDraw rd{1.f, 0, 0u, 0u, 0u};
+      if (SAMPLE && row_ok) rd = row_draw(p.smp, p.row_src ? p.row_src[row] : row);
       float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
       int am = 0x7fffffff;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
@@ -456,7 +531,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tbase + c * 32, r);
         tmem_ld_wait(r);
         const int nvalid = min(32, p.V - col0);
-        ent_chunk(r, nvalid, col0, m, s, uu, av, am);
+        ent_chunk<false, SAMPLE>(r, nvalid, col0, m, s, uu, av, am, 1.f, &rd, p.smp.key0,
+                                 p.smp.key1);
         if (lrow) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -522,6 +598,7 @@ constexpr size_t Q_SMEM = 1024 + (size_t)Q_CSTAGES * Q_B_BYTES + (size_t)Q_ASTAG
 static_assert(Q_SMEM <= 232448, "more shared memory than one CTA may have");
 static_assert(Q_CONV_WARPS * 32 == BN, "one converter thread per vocabulary row of a tile");
 
+template <bool SAMPLE>
 __global__ void __launch_bounds__(Q_THREADS, 1)
     lmhead_q4_kernel(const __grid_constant__ CUtensorMap tmA, Params p) {
   pdl_wait();
@@ -684,6 +761,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
       fence_after();
       const int row = mt * BM + q * 32 + lane;
       const bool row_ok = row < n_rows;
+      RowDraw rd{1.f, 0, 0u, 0u, 0u};
+      if (SAMPLE && row_ok) rd = row_draw(p.smp, p.row_src ? p.row_src[row] : row);
       float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
       int am = 0x7fffffff;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
@@ -698,7 +777,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
         tmem_ld32(tbase + c * 32, r);
         tmem_ld_wait(r);
         const int nvalid = min(32, p.V - col0);
-        ent_chunk<true>(r, nvalid, col0, m, s, uu, av, am, p.gscale);
+        ent_chunk<true, SAMPLE>(r, nvalid, col0, m, s, uu, av, am, p.gscale, &rd, p.smp.key0,
+                                p.smp.key1);
         if (lrow) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -824,7 +904,7 @@ __global__ void __launch_bounds__(256) lm_combine_kernel(const float4 *__restric
 int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, const uint8_t *codes,
                      const uint8_t *scales, float gscale, int V, int K, const int32_t *row_idx,
                      float *entropy, int32_t *argmax, float *logits, const int32_t *logits_rows,
-                     void *ws, int32_t *st, cudaStream_t s) {
+                     void *ws, int32_t *st, cudaStream_t s, const SampleSpec *smp) {
   if (max_rows <= 0) return DG_OK;
   if (K % 256 != 0 || ((uintptr_t)codes & 15) || ((uintptr_t)scales & 15)) return DG_ERR_UNSUPPORTED;
   const int n_vtiles = (V + BN - 1) / BN;
@@ -849,11 +929,17 @@ int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, con
   p.q_scales = scales;
   p.rows_pad = nvfp4_rows_pad(V + 1);
   p.gscale = gscale;
-  cudaFuncSetAttribute(lmhead_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Q_SMEM);
+  const bool sample = smp && smp->mode != SAMPLE_GREEDY;
+  if (sample) {
+    p.smp = *smp;
+    p.row_src = row_idx;
+  }
+  auto kq = sample ? lmhead_q4_kernel<true> : lmhead_q4_kernel<false>;
+  cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Q_SMEM);
   const int units_all = ((max_rows + BM - 1) / BM) * n_vtiles;
   const int grid = units_all < num_sms() ? units_all : num_sms();
   note_launch(s, "lm_head_q4");
-  launch_pdl(lmhead_q4_kernel, grid, Q_THREADS, Q_SMEM, s, tmA, p);
+  launch_pdl(kq, grid, Q_THREADS, Q_SMEM, s, tmA, p);
   rc = check_launch("lm_head_q4");
   if (rc != DG_OK) return rc;
   note_launch(s, "lm_combine");
@@ -872,7 +958,7 @@ bool lmhead_tc_supported(int act, int d) { return act == DG_BF16 && d % BK == 0 
 int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,
                      int V, int K, const int32_t *row_idx, float *entropy, int32_t *argmax,
                      float *logits, const int32_t *logits_rows, void *ws, int32_t *st,
-                     cudaStream_t s) {
+                     cudaStream_t s, const SampleSpec *smp) {
   if (max_rows <= 0) return DG_OK;
   const int n_vtiles = (V + BN - 1) / BN;
   CUtensorMap tmA, tmB;
@@ -884,7 +970,7 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
   rc = make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_lm, (uint64_t)K, (uint64_t)V,
                     (uint64_t)K * 2, BK, BN);
   if (rc != DG_OK) return rc;
-  Params p;
+  Params p{};
   p.n_rows_dev = n_rows_dev;
   p.max_rows = max_rows;
   p.V = V;
@@ -896,6 +982,13 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
   p.logits = logits;
   p.logits_rows = logits_rows;
   p.status = st;
+  const bool sample = smp && smp->mode != SAMPLE_GREEDY;
+  if (sample) {
+    p.smp = *smp;
+    p.row_src = row_idx;
+  }
+  auto k1 = sample ? lmhead_tc_kernel<true> : lmhead_tc_kernel<false>;
+  auto k2 = sample ? lmhead_tc2_kernel<true> : lmhead_tc2_kernel<false>;
   // The number of rows is known on the device only.  Up to 128 rows the single-CTA kernel runs;
   // beyond, CTA pairs with the 2-SM MMA (each SM streams half of every weight tile).  When both
   // are possible both are launched and the one that does not apply returns at once.
@@ -905,25 +998,22 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
     rc = make_tmap_2d(&tmB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_lm, (uint64_t)K, (uint64_t)V,
                       (uint64_t)K * 2, BK, BN / 2);  // each CTA loads 128 of the 256 rows
     if (rc != DG_OK) return rc;
-    cudaFuncSetAttribute(lmhead_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)P_SMEM_BYTES);
+    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
     const int pairs_max = ((max_rows + 2 * BM - 1) / (2 * BM)) * n_vtiles;
     const int pairs = pairs_max < num_sms() / 2 ? pairs_max : num_sms() / 2;
     note_launch(s, "lm_head_tc2");
-    launch_pdl_cluster(lmhead_tc2_kernel, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, tmA, tmB2,
-                       p);
+    launch_pdl_cluster(k2, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, tmA, tmB2, p);
     rc = check_launch("lm_head_tc2");
     if (rc != DG_OK) return rc;
   }
-  cudaFuncSetAttribute(lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)SMEM_BYTES);
+  cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   {
     const int units_max = n_vtiles;  // one row tile: the single-CTA kernel's only case here
     const int units_all = ((max_rows + BM - 1) / BM) * n_vtiles;
     const int um = p.only_one_tile ? units_max : units_all;
     const int grid = um < num_sms() ? um : num_sms();
     note_launch(s, "lm_head_tc");
-    launch_pdl(lmhead_tc_kernel, grid, NUM_THREADS, SMEM_BYTES, s, tmA, tmB, p);
+    launch_pdl(k1, grid, NUM_THREADS, SMEM_BYTES, s, tmA, tmB, p);
   }
   rc = check_launch("lm_head_tc");
   if (rc != DG_OK) return rc;

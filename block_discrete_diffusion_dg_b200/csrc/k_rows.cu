@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(256) prologue_kernel(
     int n, int hd, double theta, const int32_t *__restrict__ cache_len, float *cs, int batch,
     int canvas, const int32_t *__restrict__ done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
     uint8_t *token_live, const uint8_t *__restrict__ emb_q, const uint8_t *__restrict__ emb_s,
-    float emb_g, int emb_rows_pad) {
+    float emb_g, int emb_rows_pad, int drafts) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red[8];
@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(256) prologue_kernel(
   const int bid = blockIdx.x;
   if (bid < rows) {  // embedding + pre-norm
     const int row = bid;
-    int id = (masked && masked[row]) ? vocab : tokens[row];
+    // a masked row is embedded as MASK, or by its revisable draft token (noise canvas)
+    int id = (masked && masked[row] && !drafts) ? vocab : tokens[row];
     if (id < 0 || id > vocab) {
       if (threadIdx.x == 0) set_status(st, DG_ERR_INVALID_ARG);
       id = vocab;
@@ -366,7 +367,8 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
                     int d, int vocab, double eps, void *x_out, void *a_out, int32_t *st, int batch,
                     int n, int hd, double theta, const int32_t *cache_len, float *cs,
                     const int32_t *done, int32_t *row_idx, int32_t *n_rows, int32_t *slot,
-                    uint8_t *token_live, cudaStream_t s, const uint8_t *emb_scale, float emb_g) {
+                    uint8_t *token_live, cudaStream_t s, const uint8_t *emb_scale, float emb_g,
+                    int drafts) {
   if (rows <= 0) return DG_OK;
   const uint8_t *emb_q = emb_scale ? static_cast<const uint8_t *>(emb) : nullptr;
   const int rows_pad = nvfp4_rows_pad(vocab + 1);
@@ -377,11 +379,11 @@ int launch_prologue(int act, const int32_t *tokens, const uint8_t *masked, const
   if (act == DG_F32)
     launch_pdl(prologue_kernel<float>, grid, 256, 0, s, tokens, masked, (const float *)emb, rows, d, vocab, (float)eps, (float *)x_out,
         (float *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
-        n_rows, slot, token_live, emb_q, emb_scale, emb_g, rows_pad);
+        n_rows, slot, token_live, emb_q, emb_scale, emb_g, rows_pad, drafts);
   else
     launch_pdl(prologue_kernel<bf16>, grid, 256, 0, s, tokens, masked, (const bf16 *)emb, rows, d, vocab, (float)eps, (float *)x_out,
         (bf16 *)a_out, st, rope_blocks, n, hd, theta, cache_len, cs, batch, n, done, row_idx,
-        n_rows, slot, token_live, emb_q, emb_scale, emb_g, rows_pad);
+        n_rows, slot, token_live, emb_q, emb_scale, emb_g, rows_pad, drafts);
   return check_launch("prologue");
 }
 

@@ -45,14 +45,18 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase of parity `parity` to complete; false after WAIT_LIMIT_CYCLES.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Waits for the phase of parity `parity` to complete; false after `limit` SM clock cycles.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try(bar, parity)) {
-    if (clock64() - t0 > WAIT_LIMIT_CYCLES) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+// Waits for the phase of parity `parity` to complete; false after WAIT_LIMIT_CYCLES.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, WAIT_LIMIT_CYCLES);
 }
 
 // ---- TMA ----------------------------------------------------------------------------------------

@@ -115,6 +115,29 @@ typedef struct dg_model {
   float emb_scale_global;
 } dg_model;
 
+/* Sampler variants ("DiffusionGemma Technical Report": explanatory visual and Figure 3, a canvas
+ * that starts as uniform noise; Figure 9, a temperature annealed over the step budget N, milder
+ * for a larger N; Figure 10, tau_t = 1 with annealing off; ainewsonline.de article: the model
+ * corrects its own mistakes while denoising, before the output is final).  The pages give no
+ * formulas; the library's readings:
+ *   tau_s = tau_start + (tau_end - tau_start) * min(s, N - 1) / max(N - 1, 1)  (fp64; s = the
+ *           canvas's step index, N = max_steps).  tau_s > 0: each masked position's token is
+ *           drawn from softmax(z / tau_s) as argmax_v (z_v * (1/tau_s) + G_v), G = -ln(-ln U)
+ *           (Gumbel-max; 1/tau_s rounded to fp32), and the EB rule ranks the entropies of
+ *           softmax(z / tau_s).  tau_s <= 0: greedy argmax, entropy at tau = 1.
+ *   U = ((w >> 9) + 1/2) * 2^-23, w a word of Philox4x32-10 (Salmon et al., SC 2011) keyed by
+ *           (seed low word, seed high word) at counter (v >> 2, i, s, (1 << 24) | b), word v & 3,
+ *           for vocabulary entry v of position i of canvas b at step s.
+ *   revise: positions that are not final (masked = 1) hold revisable draft tokens: they are
+ *           embedded by their token instead of MASK, and every such position the EB rule does not
+ *           commit takes this step's drawn token as its new draft (committed positions are final,
+ *           as before).  Used with dg_noise_canvas. */
+typedef struct dg_sampler {
+  double tau_start, tau_end; /* temperature at step 0 and at step max_steps - 1 (finite) */
+  uint64_t seed;             /* generator key */
+  int32_t revise;            /* 1: revisable drafts (noise canvas); 0: absorbing MASK positions */
+} dg_sampler;
+
 /* ---- sizes and status ------------------------------------------------------------------ */
 
 /* Bytes of scratch the calls below need for `batch` canvases of `n_tokens` tokens each and a
@@ -145,6 +168,16 @@ int dg_profile_begin(int max_records);
 int dg_profile_mark(void *stream);
 int dg_profile_end(float *ms, int max_out, int *n_out);
 const char *dg_profile_name(int i);
+
+/* Diagnostic of the bounded device-side wait (not a step of the method).  Every wait inside the
+ * library's tensor-core kernels gives up after about 2 s (4e9 SM cycles): the kernel then records
+ * DG_ERR_TIMEOUT in *dev_status, waits (again bounded) for what it has issued, frees its tensor
+ * memory and returns, so a stalled kernel never hangs the device.  This probe runs that wait
+ * primitive alone: one CTA allocates tensor memory and waits at most limit_cycles (1 .. 4e9) on
+ * an mbarrier phase that completes only if `arrive` != 0 (the probe arrives on it itself); no
+ * copy or MMA is issued.  On expiry *dev_status gets DG_ERR_TIMEOUT (first error wins); either
+ * way the tensor memory is freed and the context stays usable. */
+int dg_debug_wait_probe(long long limit_cycles, int arrive, int32_t *dev_status, void *stream);
 
 /* ---- the hot-path operations ------------------------------------------------------------ */
 
@@ -236,11 +269,13 @@ int dg_logits_entropy_nvfp4(const dg_config *cfg, int n_rows, const int32_t *n_r
  * n_masked[b] -= k, step[b] += 1, done[b] = (n_masked[b] == 0).
  *   entropy fp32 [B][C] and argmax int32 [B][C] are read at masked positions only;
  *   tokens int32, masked uint8, selected uint8 (or NULL) [B][C]; n_masked, done, step int32 [B].
+ * revise != 0 (the noise canvas's revisable drafts, see dg_sampler): every masked position that
+ * is not committed also takes tokens[b][i] = argmax[b][i] and stays masked.
  * canvas <= 1024, gamma >= 0.  A non-finite entropy at a masked position sets DG_ERR_NUMERIC
  * and leaves that canvas unchanged. */
 int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *argmax,
                  double gamma, int max_steps, int32_t *tokens, uint8_t *masked,
-                 uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
+                 uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step, int revise,
                  int32_t *dev_status, void *stream);
 
 /* Encode & append ("DiffusionGemma Technical Report", Figure 4, stage 3; model card,
@@ -256,6 +291,27 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
                  int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
                  const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
                  void *stream);
+
+/* Autoregressive mode ("DiffusionGemma Technical Report", What they did: the fine-tuned weights
+ * still run as a standard autoregressive model, leaving room for hybrid diffusion-AR decoding;
+ * "Limits and open work": routing requests between diffusion and AR decoding).  Reading: the
+ * causal encoder is the AR model.  For each sequence b, tokens[b][0 .. n_tokens) (device int32,
+ * ids in [0, V)) are appended to the cache exactly as by dg_kv_append, the last layer also runs
+ * its attention and expert FFN, and the final RMSNorm + LM head of the last new row give the
+ * next token: next_token[b] = argmax z (greedy), or with smp->tau_start > 0 a draw from
+ * softmax(z / tau_start) by the Gumbel-max rule of dg_sampler on the stream of counter
+ * (v >> 2, p, 0, (3 << 24) | b), p = cache_len[b] + n_tokens (the predicted token's position;
+ * tau_end and revise are not used).  entropy[b] (or NULL): the entropy of that distribution.
+ * logits_dbg (or NULL): fp32 [B][V] raw logits.  forced_topk (or NULL): int32
+ * [n_layers][B n_tokens][k] expert ids (see dg_canvas_step).  Then cache_len[b] += n_tokens.
+ * The next token is not appended: pass it as the next call's token.  A diffusion canvas and AR
+ * tokens may follow one another on the same cache (hybrid decoding).  Workspace as
+ * dg_workspace_size(cfg, batch, n_tokens, cache_cap).  Errors as dg_kv_append. */
+int dg_ar_step(const dg_config *cfg, const dg_model *model, int batch, const int32_t *tokens,
+               int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
+               const dg_sampler *smp, int32_t *next_token, float *entropy, float *logits_dbg,
+               const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
+               void *stream);
 
 /* One denoising step of every live canvas ("DiffusionGemma Technical Report", Figure 4,
  * stage 2 and the explanatory visual): embed the canvas (masked positions as MASK = V), run
@@ -283,6 +339,27 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                    const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
                    void *stream);
 
+/* dg_canvas_step with a sampler variant (dg_sampler, non-NULL): the temperature-annealed
+ * Gumbel-max draw of each masked position's token (tau_s of its canvas's step; argmax_out then
+ * holds the drawn tokens and entropy_out the entropies at tau_s), and with smp->revise the
+ * revisable drafts of a noise canvas.  logits_dbg stays the raw z.  Other arguments, outputs and
+ * errors as dg_canvas_step (no expert_load).  DG_ERR_INVALID_ARG for a non-finite temperature. */
+int dg_canvas_step_sampler(const dg_config *cfg, const dg_model *model, int batch,
+                           int32_t *tokens, uint8_t *masked, int32_t *n_masked, int32_t *done,
+                           int32_t *step, int max_steps, double gamma, const dg_sampler *smp,
+                           const void *k_cache, const void *v_cache, const int32_t *cache_len,
+                           int cache_cap, float *entropy_out, int32_t *argmax_out,
+                           float *logits_dbg, const int32_t *forced_topk, void *ws,
+                           size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* Uniform-noise canvases (see dg_sampler): tokens[b][i] = (w0 * vocab) >> 32 for the first word
+ * w0 of Philox4x32-10 at counter (i, 0, 0, (2 << 24) | b) keyed by the seed; masked = 1 (every
+ * position a revisable draft), n_masked[b] = canvas, done[b] = 0, step[b] = 0.  Device arrays as
+ * in dg_eb_select; canvas <= 1024. */
+int dg_noise_canvas(int batch, int canvas, int vocab, uint64_t seed, int32_t *tokens,
+                    uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
+                    void *stream);
+
 /* Device-resident generation: dg_canvas_step repeated on the device until every canvas is done
  * ("DiffusionGemma Technical Report", explanatory visual: a canvas is refined over a number of
  * steps until confident and stable; Figure 4 stage 3: the finished canvas goes back through the
@@ -296,13 +373,15 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
  * Arguments, layouts and errors as dg_canvas_step and dg_kv_append (k_cache and v_cache are
  * written only by the append; with append, cache_cap >= canvas).  The instantiated graph is
  * cached inside the library per argument set (device, config, weight pointers, state, cache and
- * scratch pointers, sizes, max_steps, gamma; at most 8, least recent dropped), so repeated calls
- * with the same buffers launch one graph.  Not capturable into another graph; profiling
- * (dg_profile_begin) must be off while a new argument set is first used. */
+ * scratch pointers, sizes, max_steps, gamma, sampler values; at most 8, least recent dropped), so
+ * repeated calls with the same buffers launch one graph.  Not capturable into another graph;
+ * profiling (dg_profile_begin) must be off while a new argument set is first used.
+ * smp (or NULL: greedy): the sampler variant of every step, as dg_canvas_step_sampler. */
 int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t *tokens,
                 uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step, int max_steps,
-                double gamma, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
-                int append, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+                double gamma, const dg_sampler *smp, void *k_cache, void *v_cache,
+                int32_t *cache_len, int cache_cap, int append, void *ws, size_t ws_bytes,
+                int32_t *dev_status, void *stream);
 
 /* ---- fixed-scratch entry point ---------------------------------------------------------- */
 

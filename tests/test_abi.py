@@ -60,12 +60,12 @@ def test_host_side_argument_rejection_launches_nothing():
     n0 = L.dg_launch_count()
     cfg = B.make_config(synth.get_config("tiny"))
     # batch 0, canvas > 1024, negative gamma, NaN gamma, null state: all rejected before launch
-    assert L.dg_eb_select(0, 16, None, None, 1.0, 16, None, None, None, None, None, None, None, None) \
+    assert L.dg_eb_select(0, 16, None, None, 1.0, 16, None, None, None, None, None, None, 0, None, None) \
         == B.DG_ERR_INVALID_ARG
-    assert L.dg_eb_select(1, 2048, 8, 8, 1.0, 16, 8, 8, None, 8, 8, 8, None, None) == B.DG_ERR_INVALID_ARG
-    assert L.dg_eb_select(1, 16, 8, 8, -1.0, 16, 8, 8, None, 8, 8, 8, None, None) == B.DG_ERR_INVALID_ARG
-    assert L.dg_eb_select(1, 16, 8, 8, math.nan, 16, 8, 8, None, 8, 8, 8, None, None) == B.DG_ERR_INVALID_ARG
-    assert L.dg_eb_select(1, 16, 8, 8, 1.0, 16, None, 8, None, 8, 8, 8, None, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_eb_select(1, 2048, 8, 8, 1.0, 16, 8, 8, None, 8, 8, 8, 0, None, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_eb_select(1, 16, 8, 8, -1.0, 16, 8, 8, None, 8, 8, 8, 0, None, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_eb_select(1, 16, 8, 8, math.nan, 16, 8, 8, None, 8, 8, 8, 0, None, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_eb_select(1, 16, 8, 8, 1.0, 16, None, 8, None, 8, 8, 8, 0, None, None) == B.DG_ERR_INVALID_ARG
     # workspace too small / misaligned
     assert L.dg_moe_route(ctypes.byref(cfg), 16, 8, 8, None, 8, 8, 8, 8, 8, 256, 16, None, None) \
         == B.DG_ERR_WORKSPACE
@@ -119,20 +119,57 @@ def test_new_config_fields_and_entry_points_reject_on_the_host():
     cfg = B.make_config(synth.get_config("tiny"))
     lw = (B.DgLayerWeights * 1)(B.DgLayerWeights(8, None, 8, None, 8, 8, None, 8, None))
     model = B.DgModel(ctypes.cast(lw, ctypes.POINTER(B.DgLayerWeights)), 8, None, 1.0)
-    # tokens, masked, n_masked, done, step, max_steps, gamma, k, v, cache_len, cache_cap,
-    # append, ws, ws_bytes, dev_status, stream
-    args = [8, 8, 8, 8, 8, 16, 0.1, 8, 8, 8, 64, 0, 256, 1 << 30, None, None]
+    # tokens, masked, n_masked, done, step, max_steps, gamma, sampler, k, v, cache_len,
+    # cache_cap, append, ws, ws_bytes, dev_status, stream
+    args = [8, 8, 8, 8, 8, 16, 0.1, None, 8, 8, 8, 64, 0, 256, 1 << 30, None, None]
     assert L.dg_generate(ctypes.byref(cfg), None, 1, *args) == B.DG_ERR_INVALID_ARG
-    for i, v in ((5, 0), (6, -1.0), (6, math.nan)):
+    bad_smp = B.make_sampler(math.nan)
+    for i, v in ((5, 0), (6, -1.0), (6, math.nan), (7, ctypes.byref(bad_smp))):
         a2 = list(args)
         a2[i] = v
         assert L.dg_generate(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
     a2 = list(args)
-    a2[10], a2[11] = 0, 1          # append with no cache
+    a2[11], a2[12] = 0, 1          # append with no cache
     assert L.dg_generate(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
     a2 = list(args)
-    a2[12] = 257                   # misaligned scratch
+    a2[13] = 257                   # misaligned scratch
     assert L.dg_generate(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
+    assert L.dg_launch_count() == n0
+
+
+def test_sampler_entry_points_reject_on_the_host():
+    """dg_noise_canvas, dg_canvas_step_sampler and dg_ar_step refuse bad arguments before any
+    launch: empty or oversized canvases, a missing or non-finite sampler, missing outputs."""
+    L = B.lib()
+    n0 = L.dg_launch_count()
+    assert L.dg_noise_canvas(0, 16, 512, 1, 8, 8, 8, 8, 8, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_noise_canvas(1, 2048, 512, 1, 8, 8, 8, 8, 8, None) == B.DG_ERR_INVALID_ARG
+    assert L.dg_noise_canvas(1, 16, 512, 1, None, 8, 8, 8, 8, None) == B.DG_ERR_INVALID_ARG
+    cfg = B.make_config(synth.get_config("tiny"))
+    lw = (B.DgLayerWeights * 1)(B.DgLayerWeights(8, None, 8, None, 8, 8, None, 8, None))
+    model = B.DgModel(ctypes.cast(lw, ctypes.POINTER(B.DgLayerWeights)), 8, None, 1.0)
+    good, nan_smp = B.make_sampler(1.0, 0.5, 3), B.make_sampler(1.0, math.inf, 3)
+    # tokens, masked, n_masked, done, step, max_steps, gamma, sampler, k, v, cache_len, cap,
+    # entropy, argmax, logits, forced, ws, ws_bytes, dev_status, stream
+    args = [8, 8, 8, 8, 8, 16, 0.1, ctypes.byref(good), 8, 8, 8, 64, None, None, None, None, 257,
+            1 << 30, None, None]
+    assert L.dg_canvas_step_sampler(ctypes.byref(cfg), ctypes.byref(model), 1, *args) \
+        == B.DG_ERR_INVALID_ARG                     # misaligned scratch
+    for i, v in ((7, None), (7, ctypes.byref(nan_smp))):
+        a2 = list(args)
+        a2[i], a2[16] = v, 256
+        assert L.dg_canvas_step_sampler(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) \
+            == B.DG_ERR_INVALID_ARG
+    # tokens, n_tokens, k, v, cache_len, cap, sampler, next, entropy, logits, forced, ws, ws_bytes,
+    # dev_status, stream
+    ar = [8, 1, 8, 8, 8, 64, None, 8, None, None, None, 256, 1 << 30, None, None]
+    for i, v in ((7, None), (1, 0), (6, ctypes.byref(nan_smp))):
+        a2 = list(ar)
+        a2[i] = v
+        assert L.dg_ar_step(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_INVALID_ARG
+    a2 = list(ar)
+    a2[1] = 65                      # more tokens than the cache holds
+    assert L.dg_ar_step(ctypes.byref(cfg), ctypes.byref(model), 1, *a2) == B.DG_ERR_CAPACITY
     assert L.dg_launch_count() == n0
 
 
