@@ -32,6 +32,11 @@ import torch  # noqa: E402
 
 METRIC = "canvas denoise steps/s and output tok/s at batch 1; % of step roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures (the ~8 TB/s HBM3e of the DGX part and the dense bf16 tensor peak), for a
+# second roofline fraction beside the one against the measured peaks
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+# the other workloads measured in the same process as the headline one (single GPU only)
+EXTRA_WORKLOADS = ("longctx", "batch32", "layer_nvfp4", "stack30")
 
 
 def load_peaks():
@@ -285,7 +290,29 @@ def workload_desc(cfg) -> str:
             f"{cfg.prompt_len}, gamma {cfg.gamma}, batch {cfg.batch}; canvas states: {states}")
 
 
-def run_generate(args, world, rank):
+def run_extras(args, world, rank, local) -> dict:
+    """The other workloads, one after another in this process (each freed before the next):
+    steps/s, ms per step, the step roofline and the dominant kernel's roofline, clocks."""
+    out = {}
+    sub = argparse.Namespace(**vars(args))
+    sub.steps = args.extra_steps
+    for name in EXTRA_WORKLOADS:
+        torch.cuda.empty_cache()
+        try:
+            if name == "stack30":
+                sub.workload = name
+                r = run_generate(sub, world, rank, full=False)
+            else:
+                r = run_dg(sub, world, rank, local, workload=name, full=False)
+            out[name] = r
+        except Exception as e:  # a workload that cannot run here is reported, not fatal
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_generate(args, world, rank, full=True):
     """Block-autoregressive generation of the 30-layer workload: the prompt (2048 ids) is
     prefilled through the append in 256-token chunks (not timed), then n_canvases canvases are
     denoised from all-MASK until done and appended.  Timed both ways: dg_generate (the step loop
@@ -312,6 +339,15 @@ def run_generate(args, world, rank):
 
     init = {k: v.to(dev) for k, v in synth.make_canvas_state(cfg, "all_mask").items()}
     st = {k: v.clone() for k, v in init.items()}
+    # the experts a representative step routes tokens to (the first step of the first canvas,
+    # all MASK, cache = the prefilled prompt): the byte count of the step roofline
+    load = torch.zeros((cfg.n_layers, cfg.n_experts + cfg.n_shared), dtype=torch.int32, device=dev)
+    B.dg_canvas_step(dgcfg, dgm, cfg.batch, st["tokens"], st["masked"], st["n_masked"], st["done"],
+                     st["step"], cfg.max_steps, cfg.gamma, kv["k"], kv["v"], kv["cache_len"], cap,
+                     None, None, None, ws, status, stream, expert_load=load)
+    touched = float((load > 0).sum().item())
+    for k in st:
+        st[k].copy_(init[k])
 
     def generate_host():
         # the host reads each step's done flag
@@ -345,7 +381,8 @@ def run_generate(args, world, rank):
             counts.append(st["step"].max())
         return int(torch.stack(counts).sum().item())
 
-    modes = [("device", generate_device), ("host", generate_host)]
+    modes = [("device", generate_device), ("host", generate_host)] if full else \
+        [("device", generate_device)]
     try:
         generate_device()
         torch.cuda.synchronize()
@@ -383,6 +420,12 @@ def run_generate(args, world, rank):
     loops = {name: {"steps": v[0], "ms_per_step": round(v[1] / v[0], 4)} for name, v in timed.items()}
     toks = cfg.n_canvases * cfg.canvas * cfg.batch
     peaks, peak_src = load_peaks()
+    step_roof = step_roofline(step_bytes(cfg, touched), step_flops(cfg, cfg.batch * cfg.canvas),
+                              ms / steps, peaks, peak_src)
+    step_roof["experts_touched"] = touched
+    step_roof["note"] = ("bytes and FLOPs of the first all-MASK step over the prefilled prompt "
+                         "(its routed experts, all 30 layers, the LM head over 256 rows) against "
+                         "the loop's mean time per step, which also carries the appends")
     line = {"metric": METRIC, "value": round(rate, 3), "unit": "steps/s",
             "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": round(ms / steps, 4), "clocks": clk,
@@ -397,29 +440,49 @@ def run_generate(args, world, rank):
             "loops": loops,
             "output_tok_s": round(world * toks / (ms / 1e3), 2),
             "gpu_launches": int(launches) if modes[0][0] == "host" else
-            int(timed["host"][2] + steps),
+            (int(timed["host"][2] + steps) if "host" in timed else None),
             "gpu_launches_note": ("counted launches of the host loop" if modes[0][0] == "host" else
                                   "the device loop replays, per step, the kernels the host loop "
                                   "launches for the same steps (counted there), plus one "
                                   "condition kernel per step"),
+            "step_roofline": step_roof,
             "impl": "dg", "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    if not full:   # launches are counted on the host loop, which this short form skips
+        line.pop("gpu_launches_note", None)
+    return line
 
 
-# DRAM traffic per launch of the dominant kernel from one ncu capture of the same kernel build
-# (profiles/tc_kernels_canvas_step_layer.md); set to None when the kernel changes.
-# DRAM bytes (read + write) per LM-head launch from one ncu capture of this workload: the mean of
-# the all-MASK (1075.327 MB + 8.534 MB) and half-committed (1076.766 MB + 5.687 MB) launches.
-NCU_TRAFFIC = {"lm_head_tc": {"bytes": (1075327000 + 8534016 + 1076766000 + 5686528) // 2,
-                              "source": "profiles/tc_kernels_canvas_step_layer.md"}}
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from one ncu capture, as
+    recorded in profiles/ncu_traffic.json together with the SHA-256 (first 16 hex digits) of the
+    kernel's source file at the time of the capture.  None when there is no record or the source
+    has changed since (the counters then describe another build)."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+    except (OSError, ValueError):
+        return None
+    r = rec.get(kernel, {}).get(workload)
+    if not r:
+        return None
+    src = os.path.join(ROOT, "block_discrete_diffusion_dg_b200", "csrc", r["source_file"])
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if sha != r["source_sha16"]:
+        return None
+    return {"bytes": int(r["bytes_per_launch"]), "source": "profiles/ncu_traffic.json",
+            "captured": r.get("command", "")}
 
 
-def run_dg(args, world, rank, local):
+def run_dg(args, world, rank, local, workload=None, full=True):
+    """One workload's step, replayed from CUDA graphs; returns the JSON line (a dict).  full: also
+    the end-to-end leg through the C ABI with host buffers and the CPU baseline."""
     import synth
     from block_discrete_diffusion_dg_b200 import binding as B
     B.lib()
-    cfg = synth.get_config(args.workload)
+    cfg = synth.get_config(workload or args.workload)
     dev = torch.device("cuda", torch.cuda.current_device())
     model = synth.make_model(cfg, dev)
     kv = synth.make_prompt_kv(cfg, dev)
@@ -579,26 +642,26 @@ def run_dg(args, world, rank, local):
         if dom_bytes:
             ach = dom_bytes / dur / 1e9
             peak = peaks["hbm_gbs"]
-            tr = NCU_TRAFFIC.get(dom) if cfg.name == "layer" else None
+            tr = ncu_traffic(dom, cfg.name)
             roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
                     "unit": "GB/s", "frac": round(ach / peak, 4),
                     "traffic": tr["bytes"] if tr else None,
                     "algorithmic_bytes_per_launch": int(dom_bytes),
                     "peak_source": f"{peak_src} (burst copy, of measured)",
-                    "traffic_source": tr["source"] if tr else None}
+                    "traffic_source": tr["source"] if tr else
+                    "none: no ncu capture of this kernel source on this workload"}
     if roof:
         roof["timing"] = f"CUDA events before each launch, {kp}-step profile pass ({prof_mode})"
-    t_bytes = sb["total"] / (peaks["hbm_gbs"] * 1e9)
-    t_flops = sf["total"] / (peaks["bf16_tflops_sustained"] * 1e12)
-    step_roof = {"bound": "hbm" if t_bytes >= t_flops else "tensor",
-                 "roofline_us": round(1e6 * max(t_bytes, t_flops), 1),
-                 "measured_us": round(1e3 * ms_step, 1),
-                 "frac": round(1e6 * max(t_bytes, t_flops) / (1e3 * ms_step), 4),
-                 "algorithmic_bytes": int(sb["total"]),
-                 "algorithmic_flops": sf["total"],
-                 "experts_touched_per_state": touched,
-                 "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, "
-                          f"{peaks['bf16_tflops_sustained']} TF/s sustained (of measured)"}
+    step_roof = step_roofline(sb, sf, ms_step, peaks, peak_src)
+    step_roof["experts_touched_per_state"] = touched
+    if not full:
+        return {"metric": METRIC, "value": round(steps_s, 3), "unit": "steps/s",
+                "ms_per_step": round(ms_step, 4), "output_tok_s": round(steps_s * float(np.mean(committed)), 2),
+                "config": {"workload": workload_desc(cfg), "batch": cfg.batch,
+                           "cuda_graph": bool(graphs), "steps": args.steps},
+                "step_roofline": step_roof, "roofline": roof, "clocks": clk,
+                "gpu_launches": int(launches), "launches_per_step": int(per_step_launches),
+                "kernels_top3": dict(list(breakdown.items())[:3])}
 
     # ---- end to end through the C ABI with host buffers ----
     pin = [{k: v.cpu().pin_memory() for k, v in s_.items()} for s_ in init]
@@ -656,8 +719,27 @@ def run_dg(args, world, rank, local):
             "step_roofline": step_roof, "roofline": roof, "kernels": breakdown,
             "gpu_launches": int(launches), "launches_per_step": int(per_step_launches),
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clk, "impl": "dg"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    return line
+
+
+def step_roofline(sb: dict, sf: dict, ms_step: float, peaks: dict, peak_src: str) -> dict:
+    """max(bytes / HBM peak, FLOPs / tensor peak) for one step against its measured time, with
+    the measured peaks (the fraction the target is judged on) and, beside it, the nominal ones."""
+    t_bytes = sb["total"] / (peaks["hbm_gbs"] * 1e9)
+    t_flops = sf["total"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    n_bytes = sb["total"] / (NOMINAL["hbm_gbs"] * 1e9)
+    n_flops = sf["total"] / (NOMINAL["bf16_tflops"] * 1e12)
+    return {"bound": "hbm" if t_bytes >= t_flops else "tensor",
+            "roofline_us": round(1e6 * max(t_bytes, t_flops), 1),
+            "measured_us": round(1e3 * ms_step, 1),
+            "frac": round(1e6 * max(t_bytes, t_flops) / (1e3 * ms_step), 4),
+            "frac_nominal": round(1e6 * max(n_bytes, n_flops) / (1e3 * ms_step), 4),
+            "algorithmic_bytes": int(sb["total"]),
+            "algorithmic_flops": sf["total"],
+            "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, "
+                     f"{peaks['bf16_tflops_sustained']} TF/s sustained (frac, of measured); "
+                     f"nominal {NOMINAL['hbm_gbs']} GB/s, {NOMINAL['bf16_tflops']} TF/s "
+                     f"(frac_nominal)"}
 
 
 def main():
@@ -670,6 +752,10 @@ def main():
     ap.add_argument("--ref-frac", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct launches")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="measure the headline workload only (no 'workloads' object)")
+    ap.add_argument("--extra-steps", type=int, default=20,
+                    help="timed steps of each extra workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -677,10 +763,15 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
-        elif args.workload == "stack30":
-            run_generate(args, world, rank)
         else:
-            run_dg(args, world, rank, local)
+            if args.workload == "stack30":
+                line = run_generate(args, world, rank)
+            else:
+                line = run_dg(args, world, rank, local)
+            if world == 1 and args.workload == "layer" and not args.no_extra:
+                line["workloads"] = run_extras(args, world, rank, local)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
     finally:
         if world > 1 and args.impl == "dg":
             torch.distributed.destroy_process_group()

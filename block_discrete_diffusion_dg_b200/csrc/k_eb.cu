@@ -10,11 +10,14 @@
 // Bit-exactness: keys are (fp32 bits of max(H, 0), position) — order-preserving for H >= 0 and
 // lower position first on ties, so all keys are distinct; sums run in int64 fixed point with 32
 // fraction bits (Q(H) = nearest integer to H * 2^32, exact in fp64), so the prefix test is exact
-// and independent of summation order.  The sum over the ranks before r in sorted order is the
-// sum of Q over the keys smaller than the rank-r key, which each thread forms directly by one pass
-// over the keys in shared memory (every thread reads the same key at a time: a broadcast), so no
-// sort is needed.  At step index >= max_steps - 1 every masked position is committed (the canvas
-// always finishes within max_steps).
+// and independent of summation order.
+//
+// The block sorts the keys (bitonic network: compare-exchange partners closer than a warp by
+// shuffles, farther ones through shared memory), so thread r holds the rank-r key; an exclusive
+// block scan of Q over the ranks gives each rank its prefix sum, and the committing ranks write
+// their positions.  At step index >= max_steps - 1 every masked position is committed (the canvas
+// always finishes within max_steps).  With `revise` (the noise canvas's revisable drafts) every
+// masked position that does not commit takes argmax as its new draft token.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -22,66 +25,89 @@ namespace dg {
 
 namespace {
 
-__global__ void __launch_bounds__(1024) eb_kernel(int C, const float *__restrict__ H,
-                                                  const int32_t *__restrict__ am, long long qg,
-                                                  int max_steps, int32_t *tokens, uint8_t *masked,
-                                                  uint8_t *selected, int32_t *n_masked,
-                                                  int32_t *done, int32_t *step, int32_t *st,
-                                                  int revise) {
+template <int N>
+__global__ void __launch_bounds__(N) eb_kernel(int C, const float *__restrict__ H,
+                                               const int32_t *__restrict__ am, long long qg,
+                                               int max_steps, int32_t *tokens, uint8_t *masked,
+                                               uint8_t *selected, int32_t *n_masked,
+                                               int32_t *done, int32_t *step, int32_t *st,
+                                               int revise) {
   pdl_wait();
   pdl_trigger();
-  __shared__ unsigned long long keys[1024];
-  __shared__ long long qv[1024];
-  __shared__ int bad, n_valid, n_commit;
-  const int b = blockIdx.x, tid = threadIdx.x;
-  if (done[b]) return;
-  if (tid == 0) { bad = 0; n_valid = 0; n_commit = 0; }
-  __syncthreads();
+  __shared__ unsigned long long sk[N];
+  __shared__ long long wsum[N / 32];
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (done[b]) return;  // uniform in the block
   const size_t base = (size_t)b * C;
-  unsigned long long key = ~0ull;
-  long long q = 0;
   const bool mine = tid < C && masked[base + tid];
+  unsigned long long key = ~0ull;  // positions that are not candidates sort last
+  bool bad = false;
   if (mine) {
     float h = H[base + tid];
-    if (!isfinite(h)) atomicOr(&bad, 1);
+    bad = !isfinite(h);
     h = (h > 0.f) ? h : 0.f;  // negative rounding residue and -0 count as +0
     key = ((unsigned long long)__float_as_uint(h) << 32) | (unsigned)tid;
-    q = __double2ll_rn((double)h * 4294967296.0);
-    atomicAdd(&n_valid, 1);
   }
-  if (tid < C) {
-    keys[tid] = key;
-    qv[tid] = q;
-  }
-  __syncthreads();
-  if (bad) {
+  if (__syncthreads_or(bad)) {
     if (tid == 0) set_status(st, DG_ERR_NUMERIC);
     return;
   }
-  if (tid < C) {
-    bool commit = false;
-    if (mine) {
-      int rank = 0;
-      long long excl = 0;  // sum of Q over the smaller keys = the exclusive prefix in sorted order
-      for (int j = 0; j < C; ++j) {
-        const unsigned long long kj = keys[j];
-        if (kj < key) {
-          ++rank;
-          excl += qv[j];
-        }
+  const int n_valid = __syncthreads_count(mine);
+  // bitonic sort, ascending over the block
+#pragma unroll 1
+  for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll 1
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      unsigned long long other;
+      if (j >= 32) {
+        sk[tid] = key;
+        __syncthreads();
+        other = sk[tid ^ j];
+        __syncthreads();
+      } else {
+        other = __shfl_xor_sync(0xffffffffu, key, j);
       }
-      commit = step[b] >= max_steps - 1 || rank == 0 || excl <= qg;
-      if (commit) {
-        tokens[base + tid] = am[base + tid];
-        masked[base + tid] = 0;
-        atomicAdd(&n_commit, 1);
-      } else if (revise) {
-        tokens[base + tid] = am[base + tid];  // the draft takes this step's prediction
-      }
+      const bool keep_min = ((tid & k) == 0) == ((tid & j) == 0);
+      key = keep_min ? (key < other ? key : other) : (key < other ? other : key);
     }
-    if (selected) selected[base + tid] = commit ? 1 : 0;
+  }
+  // rank tid's fixed-point entropy and the exclusive prefix sum over the ranks before it
+  long long q = 0;
+  if (tid < n_valid) q = __double2ll_rn((double)__uint_as_float((uint32_t)(key >> 32)) * 4294967296.0);
+  long long incl = q;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    long long t = lane < N / 32 ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += v;
+    }
+    __syncwarp();
+    if (lane < N / 32) wsum[lane] = t;  // inclusive warp totals
   }
   __syncthreads();
+  const long long excl = incl - q + (warp > 0 ? wsum[warp - 1] : 0);
+  const bool commit = tid < n_valid && (step[b] >= max_steps - 1 || tid == 0 || excl <= qg);
+  if (selected && tid < C) selected[base + tid] = 0;
+  __syncthreads();  // the clears land before the committed positions are marked
+  if (tid < n_valid) {
+    const int pos = (int)(key & 0xffffffffu);
+    if (commit) {
+      tokens[base + pos] = am[base + pos];
+      masked[base + pos] = 0;
+      if (selected) selected[base + pos] = 1;
+    } else if (revise) {
+      tokens[base + pos] = am[base + pos];  // the draft takes this step's prediction
+    }
+  }
+  const int n_commit = __syncthreads_count(commit);
   if (tid == 0) {
     const int left = n_valid - n_commit;
     n_masked[b] = left;
@@ -97,11 +123,16 @@ int launch_eb_select(int batch, int canvas, const float *entropy, const int32_t 
                      uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step,
                      int32_t *st, cudaStream_t s, int revise) {
   if (batch <= 0) return DG_OK;
+  if (canvas > 1024) return DG_ERR_UNSUPPORTED;
   int N = 32;
   while (N < canvas) N <<= 1;
+  void (*k)(int, const float *, const int32_t *, long long, int, int32_t *, uint8_t *, uint8_t *,
+            int32_t *, int32_t *, int32_t *, int32_t *, int) =
+      N == 32 ? eb_kernel<32> : N == 64 ? eb_kernel<64> : N == 128 ? eb_kernel<128>
+      : N == 256 ? eb_kernel<256> : N == 512 ? eb_kernel<512> : eb_kernel<1024>;
   note_launch(s, "eb_select");
-  launch_pdl(eb_kernel, batch, N, 0, s, canvas, entropy, argmax, q_gamma, max_steps, tokens, masked,
-                                selected, n_masked, done, step, st, revise);
+  launch_pdl(k, batch, N, 0, s, canvas, entropy, argmax, q_gamma, max_steps, tokens, masked,
+             selected, n_masked, done, step, st, revise);
   return check_launch("eb_select");
 }
 

@@ -38,7 +38,11 @@ pytestmark = pytest.mark.gpu
 LOGIT_TOL = 2e-2
 ENT_RTOL = 1e-3
 ROUTER_TIE = 1e-2
-NEAR_TIE_MAX = 0.2      # at most this share of a canvas's rows may be router near ties
+# At most this share of a canvas's rows may be router near ties in the free-running check (the
+# forced-routing check covers every row).  With E = 128 router logits ~N(0, s^2), s ~ 1, the gap
+# between the 8th and 9th largest is roughly exponential with mean 1 / (E phi(x_8)) ~ 0.06 s, so a
+# 1e-2 margin catches ~15-25% of the rows; the cap keeps the free-running comparison substantive.
+NEAR_TIE_MAX = 0.3
 
 
 def _device_forced(cfg, infos):

@@ -10,7 +10,7 @@ Each state runs twice on the device: once with the oracle's expert choices hande
 (forced_topk; the gates are still the device's own), where EVERY masked row is held to the bars,
 and once free-running, where rows whose oracle router decision is a near tie (gap between the 8th
 and 9th expert logit below 1e-2, where bf16 rounding of the router input can legitimately swap
-the expert) are left out of the float checks, counted, and held to at most a fifth of the rows.
+the expert) are left out of the float checks, counted, and held to at most 30% of the rows.
 EB selections are checked bit-exact with the oracle's fp32 entropies fed to the device sampler."""
 import numpy as np
 import pytest
@@ -26,7 +26,11 @@ pytestmark = pytest.mark.gpu
 LOGIT_TOL = 2e-2
 ENT_RTOL = 1e-3
 ROUTER_TIE = 1e-2
-NEAR_TIE_MAX = 0.2      # at most this share of the rows may be router near ties
+# At most this share of a canvas's rows may be router near ties in the free-running check (the
+# forced-routing check covers every row).  With E = 128 router logits ~N(0, s^2), s ~ 1, the gap
+# between the 8th and 9th largest is roughly exponential with mean 1 / (E phi(x_8)) ~ 0.06 s, so a
+# 1e-2 margin catches ~15-25% of the rows; the cap keeps the free-running comparison substantive.
+NEAR_TIE_MAX = 0.3
 
 
 @pytest.fixture(scope="module")
