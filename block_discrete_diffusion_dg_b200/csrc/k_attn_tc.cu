@@ -389,7 +389,8 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).  P_X is written
 // over S_X as two fp16 parts, P = P_hi + P_lo (hi pairs in columns [0,64), lo pairs in [64,128)),
 // and O_X += P_hi V + P_lo V, so P reaches the product with ~22 significant bits; S_X of the next
-// key tile is issued only once P_X V of this one has completed.  The tensor cores run PV_A(i), S_A(i+1), PV_B(i), S_B(i+1):
+// key tile is issued right behind P_X V of this one (in-order MMA execution keeps the read of P
+// ahead of the overwrite).  The tensor cores run PV_A(i), S_A(i+1), PV_B(i), S_B(i+1):
 // while one softmax warpgroup works on its tile, the MMAs of the other proceed.
 // Warp roles (384 threads):
 //   warp 0     TMA: both Q tiles once, then K and V tiles of 128 keys (3- and 2-stage rings);
@@ -592,9 +593,12 @@ __global__ void __launch_bounds__(T5_THR, 1)
         fence_after();
         issue_pv(0, i);
         const bool more = i + 1 < N;
-        if (more) {  // S_A(i+1) overwrites P_A(i): wait for PV_A(i) to complete
-          if (!mbar_wait(&k_full[(i + 1) % T5_KS], ((i + 1) / T5_KS) & 1) ||
-              !mbar_wait(&pv_done[0], ph)) {
+        // S_x(i+1) is written over P_x(i), which PV_x(i) reads.  It is issued right behind it:
+        // MMAs issued by one thread execute in issue order (tcgen05.mma -> tcgen05.mma is a
+        // pipelined pair), so PV_x(i) has read P_x(i) before S_x(i+1) writes those columns, and the
+        // tensor pipe does not drain between the two.
+        if (more) {
+          if (!mbar_wait(&k_full[(i + 1) % T5_KS], ((i + 1) / T5_KS) & 1)) {
             ok = false;
             break;
           }
@@ -606,8 +610,6 @@ __global__ void __launch_bounds__(T5_THR, 1)
         issue_pv(1, i);
         commit(&v_empty[vs]);
         if (more) {
-          if (!mbar_wait(&pv_done[1], ph)) { ok = false; break; }
-          fence_after();
           issue_s(1, i + 1);
           commit(&k_empty[(i + 1) % T5_KS]);
         }
