@@ -109,6 +109,11 @@ int launch_route(int T, int E, int k, const float *z, const uint8_t *token_live,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
                  cudaStream_t s, const int32_t *forced = nullptr,
                  int n_parts = 1, int n_shared = 0);
+// The stable permutation and the tile list in one block (the second half of launch_route).
+int launch_permute_tiles(int T, int E, int k, const int32_t *topk_idx, int32_t *expert_off,
+                         int32_t *perm, int32_t *inv_perm, int tile_m, GroupTile *tiles,
+                         int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s,
+                         int n_shared = 0);
 // Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
 int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s);
@@ -185,6 +190,7 @@ int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, con
                      float *entropy, int32_t *argmax, float *logits, const int32_t *logits_rows,
                      void *ws, int32_t *st, cudaStream_t s, const SampleSpec *smp = nullptr);
 size_t lmhead_tc_ws_bytes(int max_rows, int V);
+size_t lmhead_q4_ws_bytes(int max_rows, int V);   // the NVFP4 LM head's partials
 // smp (or null: greedy): each row's token drawn as SampleSpec says (source row as the outputs);
 // the debug logits stay the raw z.
 int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,

@@ -339,6 +339,41 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
   // the (m, l) of up to eight splits and their O slices are loaded together, then combined in
   // split order
   const size_t sstride = (size_t)B * Hq * n, r0 = ((size_t)b * Hq + h) * n + i;
+  if (splits <= 16) {  // one round of loads: every split's (m, l) and O slice at once
+    float2 ml[16];
+    float4 v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < splits) {
+        const size_t r = j * sstride + r0;
+        ml[j] = part_ml[r];
+        if (lane * 4 < HD) v[j] = reinterpret_cast<const float4 *>(part_o + r * HD)[lane];
+      }
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < splits) m = fmaxf(m, ml[j].x);
+    const float base = m == -INFINITY ? 0.f : m;
+    float l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= splits) continue;
+      const float c = exp2f(ml[j].x - base);
+      l += ml[j].y * c;
+      if (lane * 4 < HD) {
+        acc.x += v[j].x * c; acc.y += v[j].y * c; acc.z += v[j].z * c; acc.w += v[j].w * c;
+      }
+    }
+    const float il = l > 0.f ? 1.f / l : 0.f;
+    if (lane * 4 < HD) {
+      bf16 *o = out + (((size_t)b * n + i) * Hq + h) * HD + lane * 4;
+      *reinterpret_cast<__nv_bfloat162 *>(o) = __floats2bfloat162_rn(acc.x * il, acc.y * il);
+      *reinterpret_cast<__nv_bfloat162 *>(o + 2) = __floats2bfloat162_rn(acc.z * il, acc.w * il);
+    }
+    return;
+  }
   float m = -INFINITY;
   for (int s0 = 0; s0 < splits; s0 += 8) {
     float mv[8];

@@ -12,8 +12,10 @@
 // fraction bits (Q(H) = nearest integer to H * 2^32, exact in fp64), so the prefix test is exact
 // and independent of summation order.
 //
-// The block sorts the keys (bitonic network: compare-exchange partners closer than a warp by
-// shuffles, farther ones through shared memory), so thread r holds the rank-r key; an exclusive
+// When the smallest entropy alone exceeds gamma exactly one position commits (rank 1 would need
+// Q(H_(0)) <= Q(gamma), and later prefixes only grow), so a block minimum of the keys decides it.
+// Otherwise the block sorts the keys (bitonic network: compare-exchange partners closer than a
+// warp by shuffles, farther ones through shared memory), so thread r holds the rank-r key; an exclusive
 // block scan of Q over the ranks gives each rank its prefix sum, and the committing ranks write
 // their positions.  At step index >= max_steps - 1 every masked position is committed (the canvas
 // always finishes within max_steps).  With `revise` (the noise canvas's revisable drafts) every
@@ -37,13 +39,17 @@ __global__ void __launch_bounds__(N) eb_kernel(int C, const float *__restrict__ 
   __shared__ unsigned long long sk[N];
   __shared__ long long wsum[N / 32];
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (done[b]) return;  // uniform in the block
   const size_t base = (size_t)b * C;
+  // every input of this canvas is loaded at once (one round trip), then the done flag decides
+  const int is_done = done[b], stp = step[b];
   const bool mine = tid < C && masked[base + tid];
+  const float h_in = tid < C ? H[base + tid] : 0.f;
+  const int32_t am_in = tid < C ? am[base + tid] : 0;
+  if (is_done) return;  // uniform in the block
   unsigned long long key = ~0ull;  // positions that are not candidates sort last
   bool bad = false;
   if (mine) {
-    float h = H[base + tid];
+    float h = h_in;
     bad = !isfinite(h);
     h = (h > 0.f) ? h : 0.f;  // negative rounding residue and -0 count as +0
     key = ((unsigned long long)__float_as_uint(h) << 32) | (unsigned)tid;
@@ -53,6 +59,42 @@ __global__ void __launch_bounds__(N) eb_kernel(int C, const float *__restrict__ 
     return;
   }
   const int n_valid = __syncthreads_count(mine);
+  const bool force = stp >= max_steps - 1;
+  // Rank 1 commits iff Q(H_(0)) <= Q(gamma), and the prefix sums only grow, so when the smallest
+  // entropy alone exceeds the bound exactly one position (the smallest key) commits: a block
+  // minimum replaces the sort.
+  unsigned long long kmin = key;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long v = __shfl_xor_sync(0xffffffffu, kmin, o);
+    kmin = v < kmin ? v : kmin;
+  }
+  if (lane == 0) sk[warp] = kmin;
+  __syncthreads();
+  kmin = sk[0];
+  for (int w = 1; w < N / 32; ++w) kmin = sk[w] < kmin ? sk[w] : kmin;
+  const long long q_min =
+      n_valid > 0 ? __double2ll_rn((double)__uint_as_float((uint32_t)(kmin >> 32)) * 4294967296.0)
+                  : 0;
+  if (!force && n_valid > 0 && q_min > qg) {
+    if (tid < C) {
+      const bool commit = key == kmin;  // keys are distinct: the one smallest candidate
+      if (commit) {
+        tokens[base + tid] = am_in;
+        masked[base + tid] = 0;
+      } else if (revise && mine) {
+        tokens[base + tid] = am_in;  // the draft takes this step's prediction
+      }
+      if (selected) selected[base + tid] = commit ? 1 : 0;
+    }
+    if (tid == 0) {
+      n_masked[b] = n_valid - 1;
+      step[b] = stp + 1;
+      done[b] = (n_valid - 1 == 0);
+    }
+    return;
+  }
+  __syncthreads();  // sk is reused by the sort
   // bitonic sort, ascending over the block
 #pragma unroll 1
   for (int k = 2; k <= N; k <<= 1) {
@@ -94,7 +136,7 @@ __global__ void __launch_bounds__(N) eb_kernel(int C, const float *__restrict__ 
   }
   __syncthreads();
   const long long excl = incl - q + (warp > 0 ? wsum[warp - 1] : 0);
-  const bool commit = tid < n_valid && (step[b] >= max_steps - 1 || tid == 0 || excl <= qg);
+  const bool commit = tid < n_valid && (force || tid == 0 || excl <= qg);
   if (selected && tid < C) selected[base + tid] = 0;
   __syncthreads();  // the clears land before the committed positions are marked
   if (tid < n_valid) {
@@ -111,7 +153,7 @@ __global__ void __launch_bounds__(N) eb_kernel(int C, const float *__restrict__ 
   if (tid == 0) {
     const int left = n_valid - n_commit;
     n_masked[b] = left;
-    step[b] = step[b] + 1;
+    step[b] = stp + 1;
     done[b] = (left == 0);
   }
 }

@@ -87,12 +87,76 @@ __global__ void router_kernel(int T_, int d, int E, int k, int S, const T *__res
   }
 }
 
-// Top-k and gates from router logits z [T][E] (fp32), one warp per token: the k largest logits
-// (lower expert index first on equal values), gates = softmax over the selected logits.
-// With `forced` non-null the k experts of token t are forced[t][0..k-1] (in that order) instead of
-// the k largest logits; the gates are still the softmax over the selected logits.
-// z may hold n_parts fp32 partial sums [n_parts][T][E] (split-K router logits), added in order.
+// Top-k and gates of one token by one warp, from its router logits held as zv[i] = z[lane + 32 i]
+// (-inf past E): the k largest logits (lower expert index first on equal values), gates = softmax
+// over the selected logits.  With `forced_row` non-null the k experts are forced_row[0..k-1] (in
+// that order) instead; the gates are still the softmax over the selected logits.  Writes slots
+// [0, k) and the S shared-expert slots after them (gate 1); a token that is not live gets -1 / 0.
+__device__ __forceinline__ void route_warp(const float (&zv)[8], int E, int k, int S, bool live,
+                                           const int32_t *__restrict__ forced_row,
+                                           int32_t *idx_row, float *w_row) {
+  const int lane = threadIdx.x & 31;
+  if (forced_row) {
+    const int e = lane < k ? forced_row[lane] : -1;
+    const bool ok = e >= 0 && e < E;
+    float mine_z = -INFINITY;
+    const int src_lane = ok ? (e & 31) : 0, src_i = ok ? (e >> 5) : 0;
+    // every lane fetches the logit its forced expert's owner holds (one shuffle per register)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float v = __shfl_sync(0xffffffffu, zv[i], src_lane);
+      if (i == src_i) mine_z = v;
+    }
+    const float ze = ok ? mine_z : -INFINITY;
+    const float z0 = __shfl_sync(0xffffffffu, ze, 0);
+    const float p = (lane < k && ok) ? expf(ze - z0) : 0.f;
+    float denom = p;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+    if (lane < k) {
+      idx_row[lane] = (live && ok) ? e : -1;
+      w_row[lane] = (live && ok) ? p / denom : 0.f;
+    }
+  } else {
+    unsigned taken = 0u;
+    float z0 = 0.f, denom = 0.f, mine = 0.f;
+    int my_idx = -1;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !(taken & (1u << i)) && (zv[i] > bv || (zv[i] == bv && e < bi))) {
+          bv = zv[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (j == 0) z0 = bv;
+      const float p = expf(bv - z0);
+      denom += p;
+      if (lane == j) { mine = p; my_idx = bi; }
+    }
+    if (lane < k) {
+      idx_row[lane] = live ? my_idx : -1;
+      w_row[lane] = live ? mine / denom : 0.f;
+    }
+  }
+  if (lane < S) {  // shared experts: every live token, gate 1, after the routed slots
+    idx_row[k + lane] = live ? E + lane : -1;
+    w_row[k + lane] = live ? 1.f : 0.f;
+  }
+}
 
+// Top-k and gates from router logits z [T][E] (fp32), one warp per token (route_warp).
+// z may hold n_parts fp32 partial sums [n_parts][T][E] (split-K router logits), added in order.
 __global__ void router_topk_kernel(int T_, int E, int k, int S, const float *__restrict__ z,
                                    int n_parts, const uint8_t *__restrict__ token_live,
                                    const int32_t *__restrict__ forced, int32_t *topk_idx,
@@ -103,72 +167,15 @@ __global__ void router_topk_kernel(int T_, int E, int k, int S, const float *__r
   const int lane = threadIdx.x & 31;
   if (t >= T_) return;
   const bool live = token_live == nullptr || token_live[t] != 0;
-  const float *zr = z + (size_t)t * E;
-  const size_t zs = (size_t)T_ * E;
-  if (forced) {
-    const int e = lane < k ? forced[(size_t)t * k + lane] : -1;
-    const bool ok = e >= 0 && e < E;
-    float ze = -INFINITY;
-    if (ok) {
-      ze = zr[e];
-      for (int s = 1; s < n_parts; ++s) ze += zr[s * zs + e];
-    }
-    const float z0 = __shfl_sync(0xffffffffu, ze, 0);
-    const float p = (lane < k && ok) ? expf(ze - z0) : 0.f;
-    float denom = p;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
-    if (lane < k) {
-      topk_idx[(size_t)t * (k + S) + lane] = (live && ok) ? e : -1;
-      topk_w[(size_t)t * (k + S) + lane] = (live && ok) ? p / denom : 0.f;
-    }
-    if (lane < S) {  // shared experts: every live token, gate 1, after the routed slots
-      topk_idx[(size_t)t * (k + S) + k + lane] = live ? E + lane : -1;
-      topk_w[(size_t)t * (k + S) + k + lane] = live ? 1.f : 0.f;
-    }
-    return;
-  }
   float zv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) zv[i] = 0.f;
-  sum_parts8(zr, n_parts, zs, lane, 32, E, zv);
+  sum_parts8(z + (size_t)t * E, n_parts, (size_t)T_ * E, lane, 32, E, zv);
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     if (lane + 32 * i >= E) zv[i] = -INFINITY;
-  unsigned taken = 0u;
-  float z0 = 0.f, denom = 0.f, mine = 0.f;
-  int my_idx = -1;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken & (1u << i)) && (zv[i] > bv || (zv[i] == bv && e < bi))) {
-        bv = zv[i];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (j == 0) z0 = bv;
-    const float p = expf(bv - z0);
-    denom += p;
-    if (lane == j) { mine = p; my_idx = bi; }
-  }
-  if (lane < k) {
-    topk_idx[(size_t)t * (k + S) + lane] = live ? my_idx : -1;
-    topk_w[(size_t)t * (k + S) + lane] = live ? mine / denom : 0.f;
-  }
-  if (lane < S) {  // shared experts: every live token, gate 1, after the routed slots
-    topk_idx[(size_t)t * (k + S) + k + lane] = live ? E + lane : -1;
-    topk_w[(size_t)t * (k + S) + k + lane] = live ? 1.f : 0.f;
-  }
+  route_warp(zv, E, k, S, live, forced ? forced + (size_t)t * k : nullptr,
+             topk_idx + (size_t)t * (k + S), topk_w + (size_t)t * (k + S));
 }
 
 // Permutation and tile list in one block of 1024 threads (T k <= 65536, E <= 256): from the top-k
@@ -700,6 +707,23 @@ int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *toke
   return check_launch("router_topk");
 }
 
+int launch_permute_tiles(int T_, int E, int k, const int32_t *topk_idx, int32_t *expert_off,
+                         int32_t *perm, int32_t *inv_perm, int tile_m, GroupTile *tiles,
+                         int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s,
+                         int n_shared) {
+  if (T_ <= 0) return DG_OK;
+  const int ka = k + n_shared, Ea = E + n_shared;
+  if (Ea > 256 || n_shared < 0 || ka > 32) return DG_ERR_UNSUPPORTED;
+  note_launch(s, "permute_tiles");
+  if (T_ * ka <= 2048)
+    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
+               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
+  else
+    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
+               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
+  return check_launch("permute_tiles");
+}
+
 int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
@@ -710,14 +734,8 @@ int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live
   const int rc = launch_router_topk(T_, E, k, z, token_live, topk_idx, topk_w, s, forced, n_parts,
                                     n_shared);
   if (rc != DG_OK) return rc;
-  note_launch(s, "permute_tiles");
-  if (T_ * ka <= 2048)
-    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
-               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
-  else
-    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
-               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
-  return check_launch("permute_tiles");
+  return launch_permute_tiles(T_, E, k, topk_idx, expert_off, perm, inv_perm, tile_m, tiles,
+                              n_tiles, max_tiles, load_out, s, n_shared);
 }
 
 int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
