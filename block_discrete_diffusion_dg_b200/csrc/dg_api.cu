@@ -139,9 +139,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   const bool tc_lm = lmhead_tc_supported(c.act_dtype, c.d_model);
   sz[B_FIN] = T128 * d * a;
   sz[B_LOGITS] = tc_lm ? 0 : T * (size_t)c.vocab * 4;
-  sz[B_PART] = tc_lm ? (c.emb_dtype == DG_NVFP4 ? lmhead_q4_ws_bytes((int)T, c.vocab)
-                                               : lmhead_tc_ws_bytes((int)T, c.vocab))
-                    : 0;
+  sz[B_PART] = tc_lm ? lmhead_tc_ws_bytes((int)T, c.vocab) : 0;
   sz[B_ENT] = T * 4;
   sz[B_AM] = T * 4;
   { const int op = o_parts(c, (int)T); sz[B_HP] = op > 1 ? T * d * 4 * op : 0; }

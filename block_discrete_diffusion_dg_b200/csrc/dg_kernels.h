@@ -190,7 +190,6 @@ int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, con
                      float *entropy, int32_t *argmax, float *logits, const int32_t *logits_rows,
                      void *ws, int32_t *st, cudaStream_t s, const SampleSpec *smp = nullptr);
 size_t lmhead_tc_ws_bytes(int max_rows, int V);
-size_t lmhead_q4_ws_bytes(int max_rows, int V);   // the NVFP4 LM head's partials
 // smp (or null: greedy): each row's token drawn as SampleSpec says (source row as the outputs);
 // the debug logits stay the raw z.
 int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, const void *w_lm,

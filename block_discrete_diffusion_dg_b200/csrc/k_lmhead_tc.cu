@@ -562,49 +562,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// The LM head with NVFP4 weights, one CTA per SM.  A unit is (a pair of 128-row tiles, 128
-// vocabulary rows): the weight tile of a k-block is expanded ONCE and multiplied against both row
-// tiles, so at 256 rows the expansion work is that of 128 rows (units with one row tile when the
-// row count is at most 128).  The weight tile of a k-block arrives as 4 KB of FP4 codes and 512 B
-// of E4M3 block scales (two 1-D bulk copies from the k-block-major layout); converter warps
-// expand it in shared memory into the fp16 tile the MMA reads, in the 128-byte-swizzled K-major
-// layout TMA would have written: one hardware e2m1x2 -> f16x2 conversion and one f16x2 multiply
-// by the block scale per pair of weights (e2m1 * e4m3 is exact in fp16).  The MMA is kind::f16
-// with fp16 operands, so the normalised rows come in fp16 too; the tensor scale is applied to the
-// fp32 logits in the epilogue.  (A bf16 tile would need two more conversions per pair, and those
-// run at a quarter of the FP32 rate.)
-// Three rings: codes and scales (6 stages of two k-blocks), the normalised rows of both row
-// tiles (3 stages of one k-block, 2 x 16 KB, L2-resident) and the expanded tiles (2 stages of two
-// k-blocks, 32 KB) between converters and MMA.  A converter handoff covers two k-blocks of the
-// 128-row tile, so each one carries as much expansion work as a 256-row k-block would.
+// The LM head with NVFP4 weights, one CTA per SM, for any number of rows (units (row tile,
+// vocabulary tile), the row tile varying fastest).  The weight tile of a k-block arrives as 8 KB
+// of FP4 codes and 1 KB of E4M3 block scales (two 1-D bulk copies from the k-block-major
+// layout); converter warps expand it in shared memory into the fp16 tile the MMA reads, in the
+// 128-byte-swizzled K-major layout TMA would have written: one hardware e2m1x2 -> f16x2
+// conversion and one f16x2 multiply by the block scale per pair of weights (e2m1 * e4m3 is exact
+// in fp16).  The MMA is kind::f16 with fp16 operands, so the normalised rows come in fp16 too;
+// the tensor scale is applied to the fp32 logits in the epilogue.  (A bf16 tile would need two
+// more conversions per pair, and those run at a quarter of the FP32 rate.)
+// Three rings.  A k-block carries only 9 KB of weight bytes from DRAM, so the codes and scales
+// get a ring of their own (8 stages, 72 KB in flight per SM), filled by one producer warp; the
+// normalised rows (L2-resident) get a 5-stage TMA ring filled by another (5 rows stages and 8
+// weight stages measured ~3% faster than 3 and 12); the expanded tiles a 2-stage ring between
+// converters and MMA.
+// With one ring for all three, a stage's 9 KB could not be refilled before its MMA completed,
+// and four stages kept ~36 KB in flight: the loop ran at DRAM latency / 4 per k-block.
 //   warp 0      producer of the codes and scales ring;
-//   warp 1      TMEM owner and MMA issuer (M 128, N 128, K 16; one accumulator per row tile,
-//               two sets of them, so the epilogue of a unit overlaps the MMAs of the next);
-//   warps 2-5   entropy epilogue (as lmhead_tc_kernel, logits times the tensor scale), both
-//               row tiles of a unit;
-//   warps 6-13  converters: thread i expands vocabulary row i % 128 of k-block i / 128 of the
-//               stage, then fences its stores for the tensor cores' (async) proxy;
+//   warp 1      TMEM owner and MMA issuer (M 128, N 256, K 16), two 256-column accumulators;
+//   warps 2-5   entropy epilogue (as lmhead_tc_kernel, logits times the tensor scale);
+//   warps 6-13  converters: thread i expands vocabulary row i of the tile, then fences its stores
+//               for the tensor cores' (async) proxy;
 //   warp 14     producer of the normalised-rows ring (TMA).
 // Every wait is bounded.
-constexpr int Q_BN = 128;                // vocabulary rows per unit
-constexpr int Q_QSTAGES = 6, Q_ASTAGES = 3, Q_CSTAGES = 2, Q_CONV_WARPS = 8;
-constexpr int Q_KPS = 2;                 // k-blocks per codes / expanded stage
-constexpr int Q_A_TILE = BM * BK * 2;    // 16 KB normalised rows (fp16) of one row tile
-constexpr int Q_A_BYTES = 2 * Q_A_TILE;  // both row tiles of a unit
-constexpr int Q_C_BYTES = Q_BN * BK / 2;   // 4 KB FP4 codes of one k-block
-constexpr int Q_S_BYTES = Q_BN * BK / 16;  // 512 B E4M3 scales of one k-block
-constexpr int Q_KR_BYTES = Q_C_BYTES + Q_S_BYTES;
-constexpr int Q_R_BYTES = Q_KPS * Q_KR_BYTES;  // one codes stage
-constexpr int Q_KB_BYTES = Q_BN * BK * 2;      // 16 KB expanded fp16 tile of one k-block
-constexpr int Q_B_BYTES = Q_KPS * Q_KB_BYTES;  // one expanded stage
+constexpr int Q_QSTAGES = 8, Q_ASTAGES = 5, Q_CSTAGES = 2, Q_CONV_WARPS = 8;
+constexpr int Q_A_BYTES = BM * BK * 2;   // 16 KB normalised rows (fp16)
+constexpr int Q_C_BYTES = BN * BK / 2;   // 8 KB FP4 codes
+constexpr int Q_S_BYTES = BN * BK / 16;  // 1 KB E4M3 scales
+constexpr int Q_R_BYTES = Q_C_BYTES + Q_S_BYTES;
+constexpr int Q_B_BYTES = BN * BK * 2;   // 32 KB expanded fp16 tile
 constexpr int Q_THREADS = 32 * (6 + Q_CONV_WARPS + 1);
 constexpr int Q_APROD_WARP = 6 + Q_CONV_WARPS;
-constexpr uint32_t Q_TMEM_COLS = 4 * Q_BN;  // 2 sets x 2 row tiles x 128 columns
 constexpr size_t Q_SMEM = 1024 + (size_t)Q_CSTAGES * Q_B_BYTES + (size_t)Q_ASTAGES * Q_A_BYTES +
                           (size_t)Q_QSTAGES * Q_R_BYTES + 512;
 static_assert(Q_SMEM <= 232448, "more shared memory than one CTA may have");
-static_assert(Q_CONV_WARPS * 32 == Q_KPS * Q_BN, "one converter thread per row and k-block");
-static_assert(Q_KR_BYTES % 16 == 0 && Q_C_BYTES % 16 == 0, "bulk copies move 16-byte multiples");
+static_assert(Q_CONV_WARPS * 32 == BN, "one converter thread per vocabulary row of a tile");
 
 template <bool SAMPLE>
 __global__ void __launch_bounds__(Q_THREADS, 1)
@@ -613,9 +605,9 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sB = smem;                               // [Q_CSTAGES][2][16 KB], 1024-aligned
-  uint8_t *sA = sB + Q_CSTAGES * Q_B_BYTES;         // [Q_ASTAGES][2][16 KB], 1024-aligned
-  uint8_t *sR = sA + Q_ASTAGES * Q_A_BYTES;         // [Q_QSTAGES][2][4 KB codes + 512 B scales]
+  uint8_t *sB = smem;                               // [Q_CSTAGES][32 KB], 1024-aligned
+  uint8_t *sA = sB + Q_CSTAGES * Q_B_BYTES;         // [Q_ASTAGES][16 KB], 1024-aligned
+  uint8_t *sR = sA + Q_ASTAGES * Q_A_BYTES;         // [Q_QSTAGES][8 KB codes + 1 KB scales]
   uint64_t *qfull = reinterpret_cast<uint64_t *>(sR + Q_QSTAGES * Q_R_BYTES);
   uint64_t *qempty = qfull + Q_QSTAGES;
   uint64_t *afull = qempty + Q_QSTAGES;
@@ -631,12 +623,9 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   int n_rows = p.max_rows;
   if (p.n_rows_dev) n_rows = min(*p.n_rows_dev, p.max_rows);
   const int m_tiles = (n_rows + BM - 1) / BM;
-  const int m_pairs = (m_tiles + 1) / 2;
-  const int units = m_pairs * p.n_vtiles;
+  const int units = m_tiles * p.n_vtiles;
   if ((int)blockIdx.x >= units) return;  // uniform across the block
-  const int kblocks = p.K / BK;  // a multiple of Q_KPS (K % 256 == 0)
-  // row tiles of the pair of unit u (1 or 2)
-  auto pair_tiles = [&](int mp) { return min(2, m_tiles - 2 * mp); };
+  const int kblocks = p.K / BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Q_QSTAGES; ++s) {
@@ -660,7 +649,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   }
   if (warp == Q_APROD_WARP && lane == 0) tma_prefetch_desc(&tmA);
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Q_TMEM_COLS);
+    tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   fence_before();
@@ -677,16 +666,14 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
 #pragma unroll
       for (int s = 0; s < Q_QSTAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        const int nt = u / m_pairs;
-        for (int kk = 0; kk < kblocks / Q_KPS; ++kk) {
+        const int nt = u / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&qempty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
           mbar_expect_tx(&qfull[stage], Q_R_BYTES);
-          for (int kh = 0; kh < Q_KPS; ++kh) {
-            const size_t slab = (size_t)(kk * Q_KPS + kh) * p.rows_pad + (size_t)nt * Q_BN;
-            uint8_t *dst = sR + stage * Q_R_BYTES + kh * Q_KR_BYTES;
-            bulk_load(dst, p.q_codes + slab * (BK / 2), Q_C_BYTES, &qfull[stage]);
-            bulk_load(dst + Q_C_BYTES, p.q_scales + slab * (BK / 16), Q_S_BYTES, &qfull[stage]);
-          }
+          const size_t slab = (size_t)kb * p.rows_pad + (size_t)nt * BN;
+          uint8_t *dst = sR + stage * Q_R_BYTES;
+          bulk_load(dst, p.q_codes + slab * (BK / 2), Q_C_BYTES, &qfull[stage]);
+          bulk_load(dst + Q_C_BYTES, p.q_scales + slab * (BK / 16), Q_S_BYTES, &qfull[stage]);
           armed[stage] = 1;
           armed_ph[stage] = ph;
           if (++stage == Q_QSTAGES) { stage = 0; ph ^= 1; }
@@ -698,7 +685,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
       }
     }
   } else if (warp == Q_APROD_WARP) {
-    if (lane == 0) {  // normalised rows of the unit's row tiles
+    if (lane == 0) {  // normalised rows
       int stage = 0;
       uint32_t ph = 0;
       int armed[Q_ASTAGES];
@@ -706,13 +693,11 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
 #pragma unroll
       for (int s = 0; s < Q_ASTAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        const int mp = u % m_pairs, nmt = pair_tiles(mp);
+        const int mt = u % m_tiles;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&aempty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
-          mbar_expect_tx(&afull[stage], (uint32_t)(nmt * Q_A_TILE));
-          for (int mt = 0; mt < nmt; ++mt)
-            tma_load_2d(sA + stage * Q_A_BYTES + mt * Q_A_TILE, &tmA, &afull[stage], kb * BK,
-                        (2 * mp + mt) * BM);
+          mbar_expect_tx(&afull[stage], Q_A_BYTES);
+          tma_load_2d(sA + stage * Q_A_BYTES, &tmA, &afull[stage], kb * BK, mt * BM);
           armed[stage] = 1;
           armed_ph[stage] = ph;
           if (++stage == Q_ASTAGES) { stage = 0; ph ^= 1; }
@@ -725,45 +710,33 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16(BM, Q_BN);
+      const uint32_t idesc = idesc_f16(BM, BN);
       int ast = 0, cst = 0, acc = 0;
       uint32_t aph = 0, cph = 0, tph = 0;
       int last_ast = -1;
       uint32_t last_aph = 0;
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        const int nmt = pair_tiles(u % m_pairs);
         if (!mbar_wait(&tempty[acc], tph ^ 1)) { fail(p.status, abort_flag); break; }
         fence_after();
+        const uint32_t d = tmem + acc * BN;
         bool ok = true;
-        for (int kk = 0; kk < kblocks / Q_KPS && ok; ++kk) {
-          if (!mbar_wait(&cfull[cst], cph)) {
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&afull[ast], aph) || !mbar_wait(&cfull[cst], cph)) {
             fail(p.status, abort_flag);
             ok = false;
             break;
           }
-          for (int kh = 0; kh < Q_KPS; ++kh) {
-            const int kb = kk * Q_KPS + kh;
-            if (!mbar_wait(&afull[ast], aph)) {
-              fail(p.status, abort_flag);
-              ok = false;
-              break;
-            }
-            fence_after();
-            const uint64_t bd = sdesc_sw128(sB + cst * Q_B_BYTES + kh * Q_KB_BYTES);
-            for (int mt = 0; mt < nmt; ++mt) {
-              const uint32_t d = tmem + (uint32_t)(acc * 2 + mt) * Q_BN;
-              const uint64_t ad = sdesc_sw128(sA + ast * Q_A_BYTES + mt * Q_A_TILE);
+          fence_after();
+          const uint64_t ad = sdesc_sw128(sA + ast * Q_A_BYTES);
+          const uint64_t bd = sdesc_sw128(sB + cst * Q_B_BYTES);
 #pragma unroll
-              for (int k = 0; k < BK / 16; ++k)
-                mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-            }
-            commit(&aempty[ast]);
-            last_ast = ast;
-            last_aph = aph;
-            if (++ast == Q_ASTAGES) { ast = 0; aph ^= 1; }
-          }
-          if (!ok) break;
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          commit(&aempty[ast]);
           commit(&cempty[cst]);
+          last_ast = ast;
+          last_aph = aph;
+          if (++ast == Q_ASTAGES) { ast = 0; aph ^= 1; }
           if (++cst == Q_CSTAGES) { cst = 0; cph ^= 1; }
         }
         if (!ok) break;
@@ -780,75 +753,70 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     uint32_t aph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
-      const int mp = u % m_pairs, nt = u / m_pairs, nmt = pair_tiles(mp);
+      const int mt = u % m_tiles, nt = u / m_tiles;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph))) {
         fail(p.status, abort_flag);
         break;
       }
       fence_after();
-      for (int mt = 0; mt < nmt; ++mt) {
-        const int row = (2 * mp + mt) * BM + q * 32 + lane;
-        const bool row_ok = row < n_rows;
-        RowDraw rd{1.f, 0, 0u, 0u, 0u};
-        if (SAMPLE && row_ok) rd = row_draw(p.smp, p.row_src ? p.row_src[row] : row);
-        float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
-        int am = 0x7fffffff;
-        const uint32_t tbase =
-            tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 2 + mt) * Q_BN;
-        float *lrow = nullptr;
-        if (p.logits && row_ok)
-          lrow = p.logits + (size_t)(p.logits_rows ? p.logits_rows[row] : row) * p.V;
+      const int row = mt * BM + q * 32 + lane;
+      const bool row_ok = row < n_rows;
+      RowDraw rd{1.f, 0, 0u, 0u, 0u};
+      if (SAMPLE && row_ok) rd = row_draw(p.smp, p.row_src ? p.row_src[row] : row);
+      float m = -INFINITY, s = 0.f, uu = 0.f, av = -INFINITY;
+      int am = 0x7fffffff;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float *lrow = nullptr;
+      if (p.logits && row_ok)
+        lrow = p.logits + (size_t)(p.logits_rows ? p.logits_rows[row] : row) * p.V;
 #pragma unroll 1
-        for (int c = 0; c < Q_BN / 32; ++c) {
-          const int col0 = nt * Q_BN + c * 32;
-          if (col0 >= p.V) break;  // uniform in the warp
-          uint32_t r[32];
-          tmem_ld32(tbase + c * 32, r);
-          tmem_ld_wait(r);
-          const int nvalid = min(32, p.V - col0);
-          ent_chunk<true, SAMPLE>(r, nvalid, col0, m, s, uu, av, am, p.gscale, &rd, p.smp.key0,
-                                  p.smp.key1);
-          if (lrow) {
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nt * BN + c * 32;
+        if (col0 >= p.V) break;  // uniform in the warp
+        uint32_t r[32];
+        tmem_ld32(tbase + c * 32, r);
+        tmem_ld_wait(r);
+        const int nvalid = min(32, p.V - col0);
+        ent_chunk<true, SAMPLE>(r, nvalid, col0, m, s, uu, av, am, p.gscale, &rd, p.smp.key0,
+                                p.smp.key1);
+        if (lrow) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) lrow[col0 + j] = __uint_as_float(r[j]) * p.gscale;
-          }
-        }
-        if (row_ok) {
-          const size_t o = (size_t)row * p.n_vtiles + nt;
-          p.part[o] = make_float4(m, s, uu, av);
-          p.part_am[o] = am;
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid) lrow[col0 + j] = __uint_as_float(r[j]) * p.gscale;
         }
       }
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (row_ok) {
+        const size_t o = (size_t)row * p.n_vtiles + nt;
+        p.part[o] = make_float4(m, s, uu, av);
+        p.part_am[o] = am;
+      }
       acc ^= 1;
       if (acc == 0) aph ^= 1;
     }
   } else {
-    // converter: thread i of warps 6-13 owns vocabulary row i % 128 of k-block i / 128 of each
-    // stage.  Codes word w (8 codes, columns 8w .. 8w + 7 of the k-block) becomes 16-byte chunk w
-    // of the row's 128 bytes, stored at chunk position w ^ (row % 8) (the 128-byte swizzle).
-    const int cid = (warp - 6) * 32 + lane;
-    const int row = cid % Q_BN, kh = cid / Q_BN;
-    uint32_t chunk_off[8];  // byte offset of 16-byte chunk c of this row in its tile (swizzled)
+    // converter: thread i of warps 6-13 owns vocabulary row i of the tile.  Codes word w (8
+    // codes, columns 8w .. 8w + 7 of the k-block) becomes 16-byte chunk w of the row's 128 bytes,
+    // stored at chunk position w ^ (row % 8) (the 128-byte swizzle).
+    const int row = (warp - 6) * 32 + lane;
+    uint32_t chunk_off[8];  // byte offset of 16-byte chunk c of this row in a tile (swizzled)
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      chunk_off[c] = (uint32_t)(kh * Q_KB_BYTES + row * 128 + ((c ^ (row & 7)) << 4));
+    for (int c = 0; c < 8; ++c) chunk_off[c] = (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
     int qst = 0, cst = 0;
     uint32_t qph = 0, cph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
       bool ok = true;
-      for (int kk = 0; kk < kblocks / Q_KPS; ++kk) {
+      for (int kb = 0; kb < kblocks; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qst], qph)) ||
             !__all_sync(0xffffffffu, mbar_wait(&cempty[cst], cph ^ 1))) {
           fail(p.status, abort_flag);
           ok = false;
           break;
         }
-        const uint8_t *raw = sR + qst * Q_R_BYTES + kh * Q_KR_BYTES;
+        const uint8_t *raw = sR + qst * Q_R_BYTES;
         const uint4 *src = reinterpret_cast<const uint4 *>(raw + row * 32);
         const uint4 q0 = src[0], q1 = src[1];
         const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(raw + Q_C_BYTES + row * 4);
@@ -877,7 +845,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     fence_after();
-    tmem_dealloc(tmem, Q_TMEM_COLS);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -939,7 +907,7 @@ int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, con
                      void *ws, int32_t *st, cudaStream_t s, const SampleSpec *smp) {
   if (max_rows <= 0) return DG_OK;
   if (K % 256 != 0 || ((uintptr_t)codes & 15) || ((uintptr_t)scales & 15)) return DG_ERR_UNSUPPORTED;
-  const int n_vtiles = (V + Q_BN - 1) / Q_BN;
+  const int n_vtiles = (V + BN - 1) / BN;
   CUtensorMap tmA;
   const int rows_alloc = (max_rows + BM - 1) / BM * BM;
   int rc = make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, F, (uint64_t)K,
@@ -968,7 +936,7 @@ int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, con
   }
   auto kq = sample ? lmhead_q4_kernel<true> : lmhead_q4_kernel<false>;
   cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Q_SMEM);
-  const int units_all = ((max_rows + 2 * BM - 1) / (2 * BM)) * n_vtiles;
+  const int units_all = ((max_rows + BM - 1) / BM) * n_vtiles;
   const int grid = units_all < num_sms() ? units_all : num_sms();
   note_launch(s, "lm_head_q4");
   launch_pdl(kq, grid, Q_THREADS, Q_SMEM, s, tmA, p);
@@ -982,11 +950,6 @@ int launch_lmhead_q4(const void *F, int max_rows, const int32_t *n_rows_dev, con
 
 size_t lmhead_tc_ws_bytes(int max_rows, int V) {
   const size_t nvt = (size_t)(V + BN - 1) / BN;
-  return (size_t)max_rows * nvt * (sizeof(float4) + sizeof(int32_t)) + 256;
-}
-
-size_t lmhead_q4_ws_bytes(int max_rows, int V) {
-  const size_t nvt = (size_t)(V + Q_BN - 1) / Q_BN;
   return (size_t)max_rows * nvt * (sizeof(float4) + sizeof(int32_t)) + 256;
 }
 
