@@ -503,10 +503,10 @@ int launch_gemm_tc_split(const void *W, int N, const void *X, int T, int T_alloc
 // Token tile of the expert GEMMs and the depth of their shared-memory ring (weights stream through
 // STAGES x 16 KB; the routed tokens take BN_MAX x 128 bytes per stage).
 #ifndef DG_MOE_BN
-#define DG_MOE_BN 64
+#define DG_MOE_BN 128
 #endif
 #ifndef DG_MOE_STAGES
-#define DG_MOE_STAGES 4
+#define DG_MOE_STAGES 3
 #endif
 #ifndef DG_MOE_CTAS_PER_SM
 #define DG_MOE_CTAS_PER_SM 2
