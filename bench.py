@@ -661,7 +661,7 @@ def run_dg(args, world, rank, local, workload=None, full=True):
                            "cuda_graph": bool(graphs), "steps": args.steps},
                 "step_roofline": step_roof, "roofline": roof, "clocks": clk,
                 "gpu_launches": int(launches), "launches_per_step": int(per_step_launches),
-                "kernels_top3": dict(list(breakdown.items())[:3])}
+                "kernels_top": dict(list(breakdown.items())[:8])}
 
     # ---- end to end through the C ABI with host buffers ----
     pin = [{k: v.cpu().pin_memory() for k, v in s_.items()} for s_ in init]

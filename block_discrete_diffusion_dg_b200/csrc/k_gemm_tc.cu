@@ -416,12 +416,14 @@ bool gemm_tc_supported(int act, int w, int K) {
 }
 
 // Dense: out[M][N] = A[M][K] * W[N][K]^T (+ res[M][N]), fp32 output.  At batch 1 these are
-// latency-bound weight streams (M = 256 tokens), so the channel tiles are narrow (32, or 16 for
-// N <= 256) to spread each weight matrix over enough CTAs.
+// latency-bound weight streams (M = 256 tokens), so the channel tiles are narrow (64, or 16 for
+// N <= 256) to spread each weight matrix over enough CTAs.  With many token rows (M >= 1024, e.g.
+// 32 canvases) the product is compute-bound instead: 128 x 256 tiles, so each activation tile is
+// read N / 256 times rather than N / 64 and every MMA is the full 256 columns wide.
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
                          const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s,
                          const float *scale) {
-  const int BN = N <= 256 ? 16 : 64;
+  const int BN = N <= 256 ? 16 : (M >= 1024 ? 256 : 64);
   const int M_alloc = (M + BM - 1) / BM * BM;  // A has room for whole tiles (caller's layout)
   CUtensorMap ta, tb;
   int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M_alloc, (uint64_t)K * 2, BK,
@@ -443,6 +445,7 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
   p.status = st;
   const int units = p.m_tiles * ((N + BN - 1) / BN);
   if (BN == 16) return launch<16, 10, 16>(ta, tb, p, units, name, s);
+  if (BN == 256) return launch<256, 4, 256>(ta, tb, p, units, name, s);
   return launch<64, 8, 64>(ta, tb, p, units, name, s);
 }
 

@@ -31,114 +31,63 @@ __global__ void rope_table_kernel(int n, int hd, double theta, const int32_t *__
   }
 }
 
-// qkv holds n_parts fp32 partial sums [n_parts][B n][width] (split-K projection), added here in
-// slice order; the summed row is staged in shared memory.
+// RoPE and head split after the QKV projection.  qkv holds n_parts fp32 partial sums
+// [n_parts][B n][width] (split-K projection), added here in slice order.  One thread per 8
+// outputs, several rows per block, no shared memory.  For a q or k head, item h covers columns 4h .. 4h + 3 of the head's first half and their rotate-half
+// partners 4h + hd/2 .. 4h + hd/2 + 3; for a v head, columns 8h .. 8h + 7.  Each thread sums its
+// two float4 of the split-K partials (slice order), rotates, and stores.
 template <typename T>
-__global__ void qkv_split_kernel(int n, int Hq, int Hkv, int hd, const float *__restrict__ qkv,
-                                 int n_parts, size_t part_stride, const float *__restrict__ cs,
-                                 T *q, T *k_new, T *v_new, T *k_cache, T *v_cache,
-                                 const int32_t *__restrict__ cache_len, int cap, int32_t *st) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ float qkv_row[];
-  const int row = blockIdx.x;  // b*n + i
-  const int b = row / n, i = row % n;
-  const int half = hd / 2;
-  const int width = (Hq + 2 * Hkv) * hd;
-  for (int e0 = threadIdx.x; e0 < width; e0 += 8 * blockDim.x) {
-    float acc[8];
-    sum_parts8(qkv + (size_t)row * width, n_parts, part_stride, e0, blockDim.x, width, acc);
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (e0 + j * (int)blockDim.x < width) qkv_row[e0 + j * blockDim.x] = acc[j];
-  }
-  __syncthreads();
-  const float *src = qkv_row;
-  const float *c = cs + (size_t)row * hd;
-  int crow = -1;
-  if (k_cache) {
-    const int r = cache_len[b] + i;
-    if (cache_len[b] + n > cap) {
-      if (threadIdx.x == 0) set_status(st, DG_ERR_CAPACITY);
-    } else {
-      crow = r;
-    }
-  }
-  for (int e = threadIdx.x; e < width; e += blockDim.x) {
-    const int head = e / hd, dd = e % hd;
-    float v = src[e];
-    if (head < Hq + Hkv) {  // rotate q and k
-      const int j = dd % half;
-      const float co = c[2 * j], si = c[2 * j + 1];
-      const float x1 = src[head * hd + j], x2 = src[head * hd + j + half];
-      v = (dd < half) ? (x1 * co - x2 * si) : (x2 * co + x1 * si);
-    }
-    const T tv = from_f<T>(v);
-    if (head < Hq) {
-      q[(size_t)row * Hq * hd + e] = tv;
-    } else {
-      const bool is_k = head < Hq + Hkv;
-      const int g = is_k ? head - Hq : head - Hq - Hkv;
-      T *dst = is_k ? k_new : v_new;
-      dst[(((size_t)b * Hkv + g) * n + i) * hd + dd] = tv;
-      if (crow >= 0) {
-        T *cd = is_k ? k_cache : v_cache;
-        cd[(((size_t)b * Hkv + g) * cap + crow) * hd + dd] = tv;
-      }
-    }
-  }
-}
-
-// qkv_split_kernel with one float4 per thread (blockDim = width / 4 <= 1024): the summed row is
-// staged in shared memory, then each thread rotates and stores its four consecutive values.
-template <typename T>
-__global__ void __launch_bounds__(1024) qkv_split4_kernel(
-    int n, int Hq, int Hkv, int hd, const float4 *__restrict__ qkv, int n_parts,
+__global__ void __launch_bounds__(256) qkv_rope_kernel(
+    int rows, int n, int Hq, int Hkv, int hd, const float4 *__restrict__ qkv, int n_parts,
     size_t part_stride4, const float *__restrict__ cs, T *q, T *k_new, T *v_new, T *k_cache,
     T *v_cache, const int32_t *__restrict__ cache_len, int cap, int32_t *st) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ float4 qkv_row4[];
-  const int row = blockIdx.x;  // b*n + i
+  const int per_head = hd / 8, items = (Hq + 2 * Hkv) * per_head;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)rows * items) return;
+  const int row = (int)(gid / items), it = (int)(gid % items);
   const int b = row / n, i = row % n;
-  const int half = hd / 2;
-  const int width4 = (Hq + 2 * Hkv) * hd / 4;
-  const int t = threadIdx.x;
-  qkv_row4[t] = sum_parts4(qkv + (size_t)row * width4 + t, n_parts, part_stride4);
+  const int half = hd / 2, head = it / per_head, h8 = it % per_head;
+  const bool rotate = head < Hq + Hkv;
+  const int c0 = rotate ? 4 * h8 : 8 * h8, c1 = rotate ? half + 4 * h8 : 8 * h8 + 4;
+  const float4 *src = qkv + (size_t)row * ((Hq + 2 * Hkv) * hd / 4) + head * (hd / 4);
+  const float4 a = sum_parts4(src + c0 / 4, n_parts, part_stride4);
+  const float4 p = sum_parts4(src + c1 / 4, n_parts, part_stride4);
+  float o0[4] = {a.x, a.y, a.z, a.w}, o1[4] = {p.x, p.y, p.z, p.w};
+  if (rotate) {
+    const float *c = cs + (size_t)row * hd;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = c0 + u;
+      const float co = c[2 * j], si = c[2 * j + 1];
+      const float x1 = o0[u], x2 = o1[u];
+      o0[u] = x1 * co - x2 * si;
+      o1[u] = x2 * co + x1 * si;
+    }
+  }
   int crow = -1;
-  if (k_cache) {
+  if (k_cache && head >= Hq) {
     if (cache_len[b] + n > cap) {
-      if (t == 0) set_status(st, DG_ERR_CAPACITY);
+      if (i == 0 && it == Hq * per_head) set_status(st, DG_ERR_CAPACITY);
     } else {
       crow = cache_len[b] + i;
     }
   }
-  __syncthreads();
-  const float *src = reinterpret_cast<const float *>(qkv_row4);
-  const float *c = cs + (size_t)row * hd;
-  const int e0 = 4 * t, head = e0 / hd, dd0 = e0 % hd;
-  float v[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int dd = dd0 + u;
-    v[u] = src[e0 + u];
-    if (head < Hq + Hkv) {  // rotate q and k
-      const int j = dd % half;
-      const float co = c[2 * j], si = c[2 * j + 1];
-      const float x1 = src[head * hd + j], x2 = src[head * hd + j + half];
-      v[u] = (dd < half) ? (x1 * co - x2 * si) : (x2 * co + x1 * si);
-    }
-  }
   if (head < Hq) {
-    store4<T>(q + (size_t)row * Hq * hd + e0, v[0], v[1], v[2], v[3]);
+    T *dst = q + (size_t)row * Hq * hd + head * hd;
+    store4<T>(dst + c0, o0[0], o0[1], o0[2], o0[3]);
+    store4<T>(dst + c1, o1[0], o1[1], o1[2], o1[3]);
   } else {
     const bool is_k = head < Hq + Hkv;
     const int g = is_k ? head - Hq : head - Hq - Hkv;
-    T *dst = is_k ? k_new : v_new;
-    store4<T>(dst + (((size_t)b * Hkv + g) * n + i) * hd + dd0, v[0], v[1], v[2], v[3]);
+    T *dst = (is_k ? k_new : v_new) + (((size_t)b * Hkv + g) * n + i) * hd;
+    store4<T>(dst + c0, o0[0], o0[1], o0[2], o0[3]);
+    store4<T>(dst + c1, o1[0], o1[1], o1[2], o1[3]);
     if (crow >= 0) {
-      T *cd = is_k ? k_cache : v_cache;
-      store4<T>(cd + (((size_t)b * Hkv + g) * cap + crow) * hd + dd0, v[0], v[1], v[2], v[3]);
+      T *cd = (is_k ? k_cache : v_cache) + (((size_t)b * Hkv + g) * cap + crow) * hd;
+      store4<T>(cd + c0, o0[0], o0[1], o0[2], o0[3]);
+      store4<T>(cd + c1, o1[0], o1[1], o1[2], o1[3]);
     }
   }
 }
@@ -163,33 +112,23 @@ int launch_qkv_split(int act, int batch, int n, int Hq, int Hkv, int hd, const f
                      int n_parts, const float *cs, void *q, void *k_new, void *v_new,
                      void *k_cache, void *v_cache, const int32_t *cache_len, int cap, int32_t *st,
                      cudaStream_t s) {
-  note_launch(s, "qkv_split");
   const int width = (Hq + 2 * Hkv) * hd;
-  const size_t smem = (size_t)width * sizeof(float);
   const size_t stride = (size_t)batch * n * width;
-  if (smem > 48 * 1024) return DG_ERR_UNSUPPORTED;
-  if (width % 4 == 0 && width / 4 <= 1024 && width / 4 >= 32 && hd % 4 == 0) {
+  if (hd % 8 == 0) {
+    note_launch(s, "qkv_split");
+    const long long work = (long long)batch * n * (width / 8);
+    const int grid = (int)((work + 255) / 256);
     if (act == DG_F32)
-      launch_pdl(qkv_split4_kernel<float>, batch * n, width / 4, smem, s, n, Hq, Hkv, hd,
+      launch_pdl(qkv_rope_kernel<float>, grid, 256, 0, s, batch * n, n, Hq, Hkv, hd,
                  (const float4 *)qkv, n_parts, stride / 4, cs, (float *)q, (float *)k_new,
                  (float *)v_new, (float *)k_cache, (float *)v_cache, cache_len, cap, st);
     else
-      launch_pdl(qkv_split4_kernel<bf16>, batch * n, width / 4, smem, s, n, Hq, Hkv, hd,
+      launch_pdl(qkv_rope_kernel<bf16>, grid, 256, 0, s, batch * n, n, Hq, Hkv, hd,
                  (const float4 *)qkv, n_parts, stride / 4, cs, (bf16 *)q, (bf16 *)k_new,
                  (bf16 *)v_new, (bf16 *)k_cache, (bf16 *)v_cache, cache_len, cap, st);
     return check_launch("qkv_split");
   }
-  if (act == DG_F32)
-    launch_pdl(qkv_split_kernel<float>, batch * n, 256, smem, s, n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
-                                                         (float *)q, (float *)k_new,
-                                                         (float *)v_new, (float *)k_cache,
-                                                         (float *)v_cache, cache_len, cap, st);
-  else
-    launch_pdl(qkv_split_kernel<bf16>, batch * n, 256, smem, s, n, Hq, Hkv, hd, qkv, n_parts, stride, cs,
-                                                        (bf16 *)q, (bf16 *)k_new, (bf16 *)v_new,
-                                                        (bf16 *)k_cache, (bf16 *)v_cache,
-                                                        cache_len, cap, st);
-  return check_launch("qkv_split");
+  return DG_ERR_UNSUPPORTED;  // head_dim is 32, 64 or 128 (cfg_ok)
 }
 
 int launch_add_cache_len(int batch, int n, int cap, int32_t *cache_len, cudaStream_t s) {
