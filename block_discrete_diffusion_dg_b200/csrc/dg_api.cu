@@ -68,7 +68,7 @@ inline size_t esz(int dt) { return dt == DG_F32 ? 4 : (dt == DG_BF16 ? 2 : 1); }
 enum Buf {
   B_X, B_A, B_QKV, B_CS, B_Q, B_KN, B_VN, B_O, B_H, B_Y, B_IDX, B_W, B_OFF, B_PERM, B_INV,
   B_TILES, B_NTILES, B_U, B_ACT, B_YE, B_XP, B_Z, B_WDQ, B_LIVE, B_ROWS, B_NROWS, B_SLOT, B_FIN, B_LOGITS, B_PART,
-  B_ENT, B_AM, B_ATTN, B_HP, B_GEN, B_COUNT
+  B_ENT, B_AM, B_ATTN, B_HP, B_GEN, B_PCNT, B_COUNT
 };
 
 struct Layout {
@@ -144,6 +144,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
   sz[B_AM] = T * 4;
   { const int op = o_parts(c, (int)T); sz[B_HP] = op > 1 ? T * d * 4 * op : 0; }
   sz[B_GEN] = 16;  // dg_generate's loop counter
+  sz[B_PCNT] = permute_scratch_bytes((int)TK, c.n_experts + c.n_shared);
   sz[B_ATTN] = attention_ws_bytes(c.act_dtype, batch, n, c.n_q_heads, c.n_kv_heads, c.head_dim,
                                   cap);
   size_t o = 0;
@@ -317,7 +318,7 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
                         ws.at<int32_t>(B_PERM), ws.at<int32_t>(B_INV),
                         tc ? experts_tc_tile_tokens() : SIMT_TILE_M, ws.at<GroupTile>(B_TILES),
                         ws.at<int32_t>(B_NTILES), ws.L->max_tiles, load_out, s, forced, rp,
-                        c.n_shared));
+                        c.n_shared, ws.at<int32_t>(B_PCNT)));
     *tiles_ready = true;
     return DG_OK;
   }

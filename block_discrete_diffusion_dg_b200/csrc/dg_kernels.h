@@ -108,12 +108,15 @@ int launch_route(int T, int E, int k, const float *z, const uint8_t *token_live,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
                  cudaStream_t s, const int32_t *forced = nullptr,
-                 int n_parts = 1, int n_shared = 0);
+                 int n_parts = 1, int n_shared = 0, int32_t *scratch = nullptr);
 // The stable permutation and the tile list in one block (the second half of launch_route).
 int launch_permute_tiles(int T, int E, int k, const int32_t *topk_idx, int32_t *expert_off,
                          int32_t *perm, int32_t *inv_perm, int tile_m, GroupTile *tiles,
                          int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s,
-                         int n_shared = 0);
+                         int n_shared = 0, int32_t *scratch = nullptr);
+// Scratch the permutation needs beyond 2048 assignments (per-block counts); with scratch null
+// there, one block does it all (slower).
+size_t permute_scratch_bytes(int n_assign, int E);
 // Builds expert_off [E+1] and perm/inv_perm [T k] (stable in flat order t k + j).
 int launch_permute(int T, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
                    int32_t *perm, int32_t *inv_perm, cudaStream_t s);

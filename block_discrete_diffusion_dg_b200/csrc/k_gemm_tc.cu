@@ -423,7 +423,7 @@ bool gemm_tc_supported(int act, int w, int K) {
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,
                          const float *res, int ldo, const char *name, int32_t *st, cudaStream_t s,
                          const float *scale) {
-  const int BN = N <= 256 ? 16 : (M >= 1024 ? 256 : 64);
+  const int BN = M >= 1024 ? (N <= 128 ? 128 : 256) : (N <= 256 ? 16 : 64);
   const int M_alloc = (M + BM - 1) / BM * BM;  // A has room for whole tiles (caller's layout)
   CUtensorMap ta, tb;
   int rc = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M_alloc, (uint64_t)K * 2, BK,
@@ -446,6 +446,7 @@ int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, floa
   const int units = p.m_tiles * ((N + BN - 1) / BN);
   if (BN == 16) return launch<16, 10, 16>(ta, tb, p, units, name, s);
   if (BN == 256) return launch<256, 4, 256>(ta, tb, p, units, name, s);
+  if (BN == 128) return launch<128, 6, 128>(ta, tb, p, units, name, s);
   return launch<64, 8, 64>(ta, tb, p, units, name, s);
 }
 

@@ -254,6 +254,131 @@ __global__ void __launch_bounds__(1024) permute_tiles_kernel(int n_assign, int E
   }
 }
 
+// The permutation and tile list for many assignments (more than 2048), in three launches over
+// blocks of 2048 consecutive assignments, with the same outputs as permute_tiles_kernel:
+//   perm_count: per block, the number of its assignments routed to each expert -> bcnt[blk][e];
+//   perm_offsets (one block): expert offsets (exclusive scan of the totals), expert_off, counts,
+//     the tile list, and each block's first position within each expert -> bcnt[blk][e];
+//   perm_scatter: per block, the rank of each assignment among the same-expert ones of its block
+//     (warp match + per-(expert, warp) counts, first half of a warp before the second, as in
+//     permute_tiles_small_kernel) plus its block's first position.
+// Assignments a0 = 64 w + lane and a1 = a0 + 32 of warp w, in increasing index order, so the
+// grouping is stable in assignment order.
+constexpr int PERM_CHUNK = 2048;
+
+__global__ void __launch_bounds__(1024) perm_count_kernel(int n_assign, int E,
+                                                          const int32_t *__restrict__ topk_idx,
+                                                          int32_t *bcnt) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int cnt[256];
+  const int tid = threadIdx.x, blk = blockIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int j = tid; j < PERM_CHUNK; j += blockDim.x) {
+    const int a = blk * PERM_CHUNK + j;
+    if (a < n_assign) {
+      const int e = topk_idx[a];
+      if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) bcnt[(size_t)blk * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(1024) perm_offsets_kernel(int n_blocks, int E, int32_t *bcnt,
+                                                            int32_t *expert_off, int tile_m,
+                                                            GroupTile *tiles, int32_t *n_tiles,
+                                                            int max_tiles, int32_t *load_out) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int tot[256], off[257], toff[257];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int t = 0;
+    for (int b = 0; b < n_blocks; ++b) t += bcnt[(size_t)b * E + e];
+    tot[e] = t;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, tacc = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e] = acc;
+      toff[e] = tacc;
+      acc += tot[e];
+      tacc += (tot[e] + tile_m - 1) / tile_m;
+    }
+    off[E] = acc;
+    toff[E] = tacc;
+    *n_tiles = min(tacc, max_tiles);
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) expert_off[e] = off[e];
+  for (int e = tid; e < E; e += blockDim.x) {
+    if (load_out) load_out[e] = tot[e];
+    int run = off[e];
+    for (int b = 0; b < n_blocks; ++b) {  // block b's first position within expert e
+      const int c = bcnt[(size_t)b * E + e];
+      bcnt[(size_t)b * E + e] = run;
+      run += c;
+    }
+    const int nt = toff[e + 1] - toff[e];
+    for (int i = 0; i < nt; ++i) {
+      const int slot = toff[e] + i;
+      if (slot < max_tiles) tiles[slot] = GroupTile{e, i * tile_m};
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024) perm_scatter_kernel(int n_assign, int E,
+                                                            const int32_t *__restrict__ topk_idx,
+                                                            const int32_t *__restrict__ bbase,
+                                                            int32_t *perm, int32_t *inv_perm) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int hist[256 * 32];  // [expert][warp] counts, then exclusive prefixes over the warps
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, blk = blockIdx.x;
+  for (int i = tid; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int a0 = blk * PERM_CHUNK + w * 64 + lane, a1 = a0 + 32;
+  int e0 = a0 < n_assign ? topk_idx[a0] : -1;
+  int e1 = a1 < n_assign ? topk_idx[a1] : -1;
+  if (e0 >= E) e0 = -1;
+  if (e1 >= E) e1 = -1;
+  const unsigned lt = (1u << lane) - 1u;
+  const unsigned m0 = __match_any_sync(0xffffffffu, e0), m1 = __match_any_sync(0xffffffffu, e1);
+  const int r0 = __popc(m0 & lt), r1 = __popc(m1 & lt);
+  if (e0 >= 0 && r0 == 0) hist[e0 * 32 + w] = __popc(m0);
+  __syncwarp();
+  const int base1 = e1 >= 0 ? hist[e1 * 32 + w] : 0;  // e1's count in the warp's first half
+  __syncwarp();
+  if (e1 >= 0 && r1 == 0) hist[e1 * 32 + w] = base1 + __popc(m1);
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {  // exclusive prefix over the warps, per expert
+    int run = 0;
+    for (int ww = 0; ww < 32; ++ww) {
+      const int c = hist[e * 32 + ww];
+      hist[e * 32 + ww] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (e0 >= 0) {
+    const int pos = bbase[(size_t)blk * E + e0] + hist[e0 * 32 + w] + r0;
+    perm[pos] = a0;
+    inv_perm[a0] = pos;
+  } else if (a0 < n_assign) {
+    inv_perm[a0] = -1;
+  }
+  if (e1 >= 0) {
+    const int pos = bbase[(size_t)blk * E + e1] + hist[e1 * 32 + w] + base1 + r1;
+    perm[pos] = a1;
+    inv_perm[a1] = pos;
+  } else if (a1 < n_assign) {
+    inv_perm[a1] = -1;
+  }
+}
+
 // permute_tiles_kernel for at most 2048 assignments in one pass (one block of 1024 threads, two
 // assignments per thread: a0 = 64 w + lane and a1 = a0 + 32 for warp w).  Counting sort: the rank
 // of an assignment among the same-expert ones of its warp half comes from __match_any_sync, the
@@ -707,27 +832,51 @@ int launch_router_topk(int T_, int E, int k, const float *z, const uint8_t *toke
   return check_launch("router_topk");
 }
 
+size_t permute_scratch_bytes(int n_assign, int E) {
+  return (size_t)((n_assign + PERM_CHUNK - 1) / PERM_CHUNK) * E * sizeof(int32_t);
+}
+
 int launch_permute_tiles(int T_, int E, int k, const int32_t *topk_idx, int32_t *expert_off,
                          int32_t *perm, int32_t *inv_perm, int tile_m, GroupTile *tiles,
                          int32_t *n_tiles, int max_tiles, int32_t *load_out, cudaStream_t s,
-                         int n_shared) {
+                         int n_shared, int32_t *scratch) {
   if (T_ <= 0) return DG_OK;
   const int ka = k + n_shared, Ea = E + n_shared;
   if (Ea > 256 || n_shared < 0 || ka > 32) return DG_ERR_UNSUPPORTED;
-  note_launch(s, "permute_tiles");
-  if (T_ * ka <= 2048)
-    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
+  const int n_assign = T_ * ka;
+  if (n_assign <= PERM_CHUNK) {
+    note_launch(s, "permute_tiles");
+    launch_pdl(permute_tiles_small_kernel, 1, 1024, 0, s, n_assign, Ea, topk_idx, expert_off,
+               perm, inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
+    return check_launch("permute_tiles");
+  }
+  if (!scratch) {
+    note_launch(s, "permute_tiles");
+    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, n_assign, Ea, topk_idx, expert_off, perm,
                inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
-  else
-    launch_pdl(permute_tiles_kernel, 1, 1024, 0, s, T_ * ka, Ea, topk_idx, expert_off, perm,
-               inv_perm, tile_m, tiles, n_tiles, max_tiles, load_out);
-  return check_launch("permute_tiles");
+    return check_launch("permute_tiles");
+  }
+  const int nb = (n_assign + PERM_CHUNK - 1) / PERM_CHUNK;
+  note_launch(s, "perm_count");
+  launch_pdl(perm_count_kernel, nb, 1024, 0, s, n_assign, Ea, topk_idx, scratch);
+  int rc = check_launch("perm_count");
+  if (rc != DG_OK) return rc;
+  note_launch(s, "perm_offsets");
+  launch_pdl(perm_offsets_kernel, 1, 1024, 0, s, nb, Ea, scratch, expert_off, tile_m, tiles,
+             n_tiles, max_tiles, load_out);
+  rc = check_launch("perm_offsets");
+  if (rc != DG_OK) return rc;
+  note_launch(s, "perm_scatter");
+  launch_pdl(perm_scatter_kernel, nb, 1024, 0, s, n_assign, Ea, topk_idx, scratch, perm,
+             inv_perm);
+  return check_launch("perm_scatter");
 }
 
 int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live, int32_t *topk_idx,
                  float *topk_w, int32_t *expert_off, int32_t *perm, int32_t *inv_perm, int tile_m,
                  GroupTile *tiles, int32_t *n_tiles, int max_tiles, int32_t *load_out,
-                 cudaStream_t s, const int32_t *forced, int n_parts, int n_shared) {
+                 cudaStream_t s, const int32_t *forced, int n_parts, int n_shared,
+                 int32_t *scratch) {
   if (T_ <= 0) return DG_OK;
   const int ka = k + n_shared, Ea = E + n_shared;  // slots and experts with the shared ones
   if (Ea > 256 || n_shared < 0 || ka > 32) return DG_ERR_UNSUPPORTED;
@@ -735,7 +884,7 @@ int launch_route(int T_, int E, int k, const float *z, const uint8_t *token_live
                                     n_shared);
   if (rc != DG_OK) return rc;
   return launch_permute_tiles(T_, E, k, topk_idx, expert_off, perm, inv_perm, tile_m, tiles,
-                              n_tiles, max_tiles, load_out, s, n_shared);
+                              n_tiles, max_tiles, load_out, s, n_shared, scratch);
 }
 
 int launch_permute(int T_, int k, int E, const int32_t *topk_idx, int32_t *expert_off,
