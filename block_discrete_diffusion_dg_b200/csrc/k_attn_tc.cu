@@ -13,8 +13,11 @@
 // Precision: S = Q K^T takes the stored bf16 q and k exactly (fp32 accumulation).  The second
 // product takes V in fp16 (every bf16 value of V is exact in fp16 for |v| < 65504; below fp16's
 // normal range the absolute error stays < 3e-8) and P:
-//   tcgen05 kernel: P = P_hi + P_lo, two fp16 parts (~22 significant bits), so P adds no
-//                   rounding visible at bf16 storage of the output;
+//   tcgen05 kernel: P = P_hi + P_lo, two fp16 parts (~22 significant bits).  The output is an
+//                   average over many keys with cancelling signs, so a relative error e in each p
+//                   reaches O at about e * sqrt(effective keys) of O's own size: with one fp16
+//                   part (e ~ 2^-12) about a tenth of the outputs land on the other side of a bf16
+//                   rounding boundary, which shows in the logits downstream;
 //   mma.sync kernel: P in fp16 (11 significant bits).
 // The mma.sync kernel: 8 warps x 16 rows; K/V tiles of 64 keys double-buffered with cp.async
 // (zero-filled past the end) in XOR-swizzled shared memory read by ldmatrix; each thread converts
@@ -80,6 +83,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   const __half2 v = __floats2half2_rn(lo, hi);
@@ -433,21 +442,42 @@ __global__ void attn_merge_kernel(int splits, int B, int Hq, int n, const float 
 //   warps 2-3  convert each landed V tile from bf16 to fp16 in place and zero the rows past the
 //              last valid key (so masked keys contribute exactly 0 * 0);
 //   warps 4-7  softmax of tile A, warps 8-11 of tile B: one query row per thread (= TMEM lane);
-//              read S, mask, running max in the log2 domain, P = 2^(t - m) written back to TMEM
-//              as fp16 hi and lo pairs, row sum in fp32.
+//              the row of S read in one round of TMEM loads, mask, running max in the log2
+//              domain, P = 2^(t - m) written back to TMEM as fp16 hi and lo pairs, row sum in
+//              fp32 (scale-and-shift, sum and split in packed fp32x2 arithmetic).
 // The running maximum is applied lazily: O is rescaled (read, scaled, written back in TMEM) only
-// when a row's maximum grows by more than 2^8, so between rescales P can reach 256 (exact in
+// when a row's maximum grows by more than 2^8, so between rescales P can reach 256 (well inside
 // fp16's range; the final O / l is unchanged because O and l always share the same base).
 // Control flow of the softmax warps is warp-uniform (votes on every exit and on the rescale
 // decision): TMEM loads and stores are .sync.aligned and need all 32 lanes.
 // Every wait is bounded; on expiry the kernel records DG_ERR_TIMEOUT, lets issued copies and
 // MMAs finish, frees TMEM and returns.
+#ifndef DG_ATTN_REGS_LO
+#define DG_ATTN_REGS_LO 104
+#endif
+#ifndef DG_ATTN_REGS_HI
+#define DG_ATTN_REGS_HI 200
+#endif
 constexpr int T5_HD = 128, T5_KT = 128, T5_KS = 3, T5_VS = 2, T5_THR = 384;
 constexpr int T5_HALF = 128 * 128;       // one box: 128 rows x 64 bf16 (128-byte rows) = 16 KB
 constexpr int T5_TILE = 2 * T5_HALF;     // 128 rows x 128 head dims = 32 KB
 constexpr uint32_t T5_COL_S = 0, T5_COL_O = 256, T5_TMEM_COLS = 512;
 constexpr float T5_RESCALE = 8.f;        // log2 of the largest P between rescales
 constexpr size_t T5_SMEM = 1024 + (size_t)T5_TILE * (2 + T5_KS + T5_VS) + 512;
+// registers per thread at launch, and after the split for the copy / MMA / converter warpgroup
+// (LO) and the two softmax warpgroups (HI)
+constexpr int T5_REGS = 168, T5_REGS_LO = DG_ATTN_REGS_LO, T5_REGS_HI = DG_ATTN_REGS_HI;
+static_assert(128 * T5_REGS_LO + 256 * T5_REGS_HI <= T5_THR * T5_REGS, "register split");
+static_assert(T5_THR * T5_REGS <= 65536, "launch registers");
+
+template <int R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
 constexpr unsigned FULL = 0xffffffffu;
 
 struct T5Args {
@@ -543,7 +573,12 @@ __global__ void __launch_bounds__(T5_THR, 1)
     valid = min(T5_KT, (cache ? len : a.n) - j0);
   };
 
+  // Register split: the copy / MMA / converter warpgroup hands registers to the two softmax
+  // warpgroups, which hold a whole row of S.  Launch: 384 threads x T5_REGS; after the split:
+  // 128 x T5_REGS_LO + 256 x T5_REGS_HI, no more than the launch holds (the host checks the
+  // kernel's register count before the first launch).
   if (warp == 0) {
+    setmaxnreg_dec<T5_REGS_LO>();
     if (lane == 0) {
       uint32_t armed_k = 0, armed_v = 0;  // tiles whose copies were issued
       bool ok = true;
@@ -580,31 +615,38 @@ __global__ void __launch_bounds__(T5_THR, 1)
         (void)mbar_wait(&v_full[i % T5_VS], (i / T5_VS) & 1);
     }
   } else if (warp == 1) {
+    setmaxnreg_dec<T5_REGS_LO>();
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(ROWS, T5_KT);
       const uint32_t id_p = idesc_f16_bmn(ROWS, T5_HD);
       bool ok = mbar_wait(q_full, 0);
       fence_after();
+      // Descriptors of the operand buffers, computed once: a descriptor's start-address field is
+      // the shared-memory byte address / 16 (all of shared memory fits its 14 bits), so an offset
+      // of b bytes is added as b / 16.  Issuing an MMA then costs an add and the instruction;
+      // building both descriptors per MMA cost more issue time than an N = 128 MMA takes.
+      const uint64_t dq = sdesc_sw128(sQ), dk = sdesc_sw128(sK);
+      const uint64_t dv = sdesc_sw128_mn(sV, T5_HALF);
       auto issue_s = [&](int x, int i) {   // S_x(i) = Q_x K_i^T into S_x
-        const int ks = i % T5_KS;
+        const uint64_t ab = dq + (uint64_t)((x * T5_TILE) >> 4);
+        const uint64_t bb = dk + (uint64_t)(((i % T5_KS) * T5_TILE) >> 4);
         const uint32_t d = tmem + T5_COL_S + (uint32_t)x * 128;
 #pragma unroll
         for (int kk = 0; kk < T5_HD / 16; ++kk) {
-          const int hf = kk >> 2, k4 = kk & 3;
-          const uint64_t ad = sdesc_sw128(sQ + x * T5_TILE + hf * T5_HALF) + 2 * k4;
-          const uint64_t bd = sdesc_sw128(sK + ks * T5_TILE + hf * T5_HALF) + 2 * k4;
-          mma_bf16(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * T5_HALF) >> 4) + 2 * (kk & 3);
+          mma_bf16(d, ab + off, bb + off, id_s, kk > 0 ? 1u : 0u);
         }
         commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int i) {  // O_x += P_x V_i
-        const int vs = i % T5_VS;
+        const uint64_t bb = dv + (uint64_t)(((i % T5_VS) * T5_TILE) >> 4);
         const uint32_t pa = tmem + T5_COL_S + (uint32_t)x * 128;
         const uint32_t d = tmem + T5_COL_O + (uint32_t)x * 128;
+        const uint32_t acc0 = i != 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < T5_KT / 16; ++kk) {  // P = P_hi + P_lo, both against the same V
-          const uint64_t bd = sdesc_sw128_mn(sV + vs * T5_TILE + kk * 16 * 128, T5_HALF);
-          mma_f16_ts(d, pa + kk * 8, bd, id_p, (i | kk) != 0 ? 1u : 0u);
+          const uint64_t bd = bb + (uint64_t)((kk * 16 * 128) >> 4);
+          mma_f16_ts(d, pa + kk * 8, bd, id_p, kk != 0 ? 1u : acc0);
           mma_f16_ts(d, pa + 64 + kk * 8, bd, id_p, 1u);
         }
         commit(&pv_done[x]);
@@ -654,6 +696,7 @@ __global__ void __launch_bounds__(T5_THR, 1)
       (void)mbar_wait(mma_fin, 0);
     }
   } else if (warp < 4) {
+    setmaxnreg_dec<T5_REGS_LO>();
     const int ct = threadIdx.x - 64;  // 0..63
     for (int i = 0; i < N; ++i) {
       if (__any_sync(FULL, *abort_flag != 0)) break;
@@ -667,7 +710,7 @@ __global__ void __launch_bounds__(T5_THR, 1)
       tile_src(i, cache, row, j0, valid);
       uint8_t *base = sV + vs * T5_TILE;
       // 16-byte chunk c sits in key row (c mod 1024) / 8 of its half (the swizzle only permutes
-      // chunks within a row), so the conversion is in place and per chunk
+      // chunks within a row), so the work is in place and per chunk
 #pragma unroll 4
       for (int c = ct; c < T5_TILE / 16; c += 64) {
         uint4 *pc = reinterpret_cast<uint4 *>(base + c * 16);
@@ -679,9 +722,10 @@ __global__ void __launch_bounds__(T5_THR, 1)
       if (lane == 0) mbar_arrive(&v_ready[vs]);
     }
   } else {
-    const int x = (warp - 4) >> 2;          // query tile (A or B) of this warpgroup
-    const int q4 = warp & 3;                // TMEM lane quarter of this warp
-    const int r = q4 * 32 + lane;           // query row of the tile
+    setmaxnreg_inc<T5_REGS_HI>();
+    const int x = (warp - 4) >> 2;            // query tile (A or B) of this warpgroup
+    const int q4 = warp & 3;                  // TMEM lane quarter of this warp
+    const int r = q4 * 32 + lane;             // query row of the tile
     const int hl = r / qpc, pos = i0 + x * qpc + r % qpc, h = g * rep + hl;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
     const uint32_t cS = T5_COL_S + (uint32_t)x * 128, cO = T5_COL_O + (uint32_t)x * 128;
@@ -701,40 +745,29 @@ __global__ void __launch_bounds__(T5_THR, 1)
       tile_src(i, cache, row, j0, valid);
       int lim = valid;
       if (a.causal && !cache) lim = min(lim, pos - j0 + 1);
-      const bool partial = __any_sync(FULL, lim < T5_KT);   // a partial or causal tile: mask
-      auto mask = [&](uint32_t (&v)[32], int c) {
-        if (partial) {
+      // the row of S in registers: two 64-column TMEM loads (few tcgen05 instructions, since
+      // they share the SM's tensor-memory instruction path with the MMAs of the other tile)
+      uint32_t sa[64], sb[64];
+      tmem_ld64(tmem + lrow + cS, sa);
+      tmem_ld64(tmem + lrow + cS + 64, sb);
+      tmem_ld_wait64(sa);
+      tmem_ld_wait64(sb);
+      if (__any_sync(FULL, lim < T5_KT)) {   // a partial or causal tile: mask
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j >= lim) v[j] = __float_as_uint(-INFINITY);
+        for (int j = 0; j < 64; ++j) {
+          if (j >= lim) sa[j] = __float_as_uint(-INFINITY);
+          if (64 + j >= lim) sb[j] = __float_as_uint(-INFINITY);
         }
-      };
-      float m8[8];
-      auto fold_max = [&](const uint32_t (&v)[32], bool first) {
+      }
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      auto fold_max = [&](const uint32_t (&v)[64]) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          m8[j & 7] = (first && j < 8) ? __uint_as_float(v[j]) : fmaxf(m8[j & 7], __uint_as_float(v[j]));
+        for (int j = 0; j < 64; j += 2)
+          m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
       };
-      // S chunks (32 columns each) 1 and 3 for the maximum, then 0 and 2, kept in registers
-      uint32_t sa[32], sb[32];
-      tmem_ld32(tmem + lrow + cS + 32, sa);
-      tmem_ld32(tmem + lrow + cS + 96, sb);
-      tmem_ld_wait(sa);
-      tmem_ld_wait(sb);
-      mask(sa, 1);
-      mask(sb, 3);
-      fold_max(sa, true);
-      fold_max(sb, false);
-      tmem_ld32(tmem + lrow + cS + 0, sa);
-      tmem_ld32(tmem + lrow + cS + 64, sb);
-      tmem_ld_wait(sa);
-      tmem_ld_wait(sb);
-      mask(sa, 0);
-      mask(sb, 2);
-      fold_max(sa, false);
-      fold_max(sb, false);
-      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+      fold_max(sa);
+      fold_max(sb);
+      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       const float m_new = fmaxf(m_use, mt);
       // a row whose maximum grew by more than 2^8 needs O rescaled; the whole warp then rescales
       // (factor 1 where nothing changed; a row with nothing accumulated yet only takes m_new)
@@ -763,38 +796,31 @@ __global__ void __launch_bounds__(T5_THR, 1)
         m_use = m_new;  // nothing accumulated yet (O is exactly 0 or not yet written)
       }
       const float nb = m_use == -INFINITY ? 0.f : -m_use;
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      // P of the 32 keys of S chunk c, split into two fp16 parts (P = hi + lo to ~22 bits):
-      // hi pairs go to columns [16c, 16c + 16) of S, lo pairs to [64 + 16c, 64 + 16c + 16).
-      // Chunk c's columns are overwritten by the P of chunks 2c and 2c + 1 (hi) and of chunks
-      // 2c - 4 and 2c - 3 (lo), so the order below reads every chunk before it is covered.
-      auto emit = [&](const uint32_t (&v)[32], int c) {
-        uint32_t ph[16], pl[16];
+      const float2 sl2v = make_float2(sl2, sl2), nbv = make_float2(nb, nb);
+      float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // P of 64 keys (half hf of the row), split into two fp16 parts (P = hi + lo to ~22 bits):
+      // hi pairs go to columns [32 hf, 32 hf + 32) of S, lo pairs to [64 + 32 hf, 96 + 32 hf).
+      // Every S value of the row is in registers by then, so the order of the writes is free.
+      auto emit = [&](const uint32_t (&v)[64], int hf) {
+        uint32_t ph[32], pl[32];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(v[j]), sl2, nb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), sl2, nb));
-          s4[(j >> 1) & 3] += p0 + p1;
-          const __half2 hi = __floats2half2_rn(p0, p1);
-          const float2 hf = __half22float2(hi);
-          const __half2 lo = __floats2half2_rn(p0 - hf.x, p1 - hf.y);
+        for (int j = 0; j < 64; j += 2) {
+          const float2 t = __ffma2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                      sl2v, nbv);
+          const float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+          s2[(j >> 1) & 1] = __fadd2_rn(s2[(j >> 1) & 1], p);
+          const __half2 hi = __floats2half2_rn(p.x, p.y);
+          const float2 d = __ffma2_rn(__half22float2(hi), make_float2(-1.f, -1.f), p);  // p - hi
+          const __half2 lo = __floats2half2_rn(d.x, d.y);
           ph[j >> 1] = *reinterpret_cast<const uint32_t *>(&hi);
           pl[j >> 1] = *reinterpret_cast<const uint32_t *>(&lo);
         }
-        tmem_st16(tmem + lrow + cS + c * 16, ph);
-        tmem_st16(tmem + lrow + cS + 64 + c * 16, pl);
+        tmem_st32(tmem + lrow + cS + hf * 32, ph);
+        tmem_st32(tmem + lrow + cS + 64 + hf * 32, pl);
       };
-      emit(sa, 0);                            // writes over S chunks 0 (held) and 2 (held in sb)
-      tmem_ld32(tmem + lrow + cS + 32, sa);   // S chunk 1 again (untouched so far)
-      tmem_ld_wait(sa);
-      mask(sa, 1);
-      emit(sa, 1);                            // over S chunks 0 and 2 (both consumed or held)
-      tmem_ld32(tmem + lrow + cS + 96, sa);   // S chunk 3 again (untouched so far)
-      tmem_ld_wait(sa);
-      mask(sa, 3);
-      emit(sb, 2);                            // over S chunks 1 (consumed) and 3 (held in sa)
-      emit(sa, 3);
-      l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      emit(sa, 0);
+      emit(sb, 1);
+      l += (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
       tmem_st_wait();
       fence_before();
       __syncwarp();
@@ -956,6 +982,13 @@ int launch_tc5(int batch, int n, int Hq, int Hkv, const void *q, const void *k_c
     tvc = tvn;
   }
   if (rc != DG_OK) return rc;
+  // the in-kernel register split needs the launch to hold T5_REGS registers per thread; a build
+  // that allocated fewer would leave setmaxnreg.inc waiting, so it is refused here
+  static const int regs = [] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, attn_tc5_kernel) == cudaSuccess ? fa.numRegs : -1;
+  }();
+  if (regs < T5_REGS) return DG_ERR_UNSUPPORTED;
   dim3 grid((n + 2 * qpc - 1) / (2 * qpc), Hkv, batch * a.splits);
   note_launch(s, "attn_tc");
   cudaFuncSetAttribute(attn_tc5_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T5_SMEM);

@@ -222,6 +222,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ph = 0, aph = 0;
       int last_stage = -1;
       uint32_t last_ph = 0;
+      // stage descriptors = base descriptor + byte offset / 16 (the start-address field holds the
+      // shared-memory address / 16), so the issue loop does not rebuild them per k-block
+      const uint64_t dA = sdesc_sw128(sA), dB = sdesc_sw128(sB);
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
         const Unit x = decode<BN_MAX>(p, u);
         const uint32_t idesc = idesc_bf16(BM, x.n_mma);
@@ -234,8 +237,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = kb0; kb < kb0 + kpb; ++kb) {
           if (!mbar_wait(&full[stage], ph)) { fail(p.status, abort_flag); ok = false; break; }
           fence_after();
-          const uint64_t ad = sdesc_sw128(sA + stage * C::A_BYTES);
-          const uint64_t bd = sdesc_sw128(sB + stage * C::B_BYTES);
+          const uint64_t ad = dA + (uint64_t)((stage * C::A_BYTES) >> 4);
+          const uint64_t bd = dB + (uint64_t)((stage * C::B_BYTES) >> 4);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
