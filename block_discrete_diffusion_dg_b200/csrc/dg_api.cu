@@ -252,7 +252,8 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
     const int parts = qkv_parts(c, T);
     if (parts > 1)
       return launch_gemm_tc_split(wq, g.N, ws.at<void>(B_A), T, (T + 127) / 128 * 128, c.d_model,
-                                  parts, ws.at<float>(B_QKV), "gemm_qkv_tc", nullptr, s, g.bscale);
+                                  parts, ws.at<float>(B_QKV), "gemm_qkv_tc", nullptr, s, g.bscale,
+                                  wq == w.w_qkv);
     return launch_gemm_tc_dense(ws.at<void>(B_A), T, wq, g.N, c.d_model, ws.at<float>(B_QKV),
                                 nullptr, g.N, "gemm_qkv_tc", nullptr, s, g.bscale);
   }
@@ -287,7 +288,7 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
     const void *wo = tc_weight(c, ws, w.w_o, (size_t)d * hq, 0, s, &rc);
     if (rc != DG_OK) return rc;
     DG_TRY(launch_gemm_tc_split(wo, d, ws.at<void>(B_O), T, T128, hq, op, ws.at<float>(B_HP),
-                                "gemm_o_resid_tc", nullptr, s, g.bscale));
+                                "gemm_o_resid_tc", nullptr, s, g.bscale, wo == w.w_o));
     DG_TRY(launch_resid_norm(c.act_dtype, ws.at<float>(B_HP), op, ws.at<float>(B_X), T, d,
                              c.rms_eps, ws.at<float>(B_H), ws.at<void>(B_Y), s));
   } else {
@@ -307,7 +308,8 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
     const int rp = router_parts(c, T);
     if (rp > 1)
       DG_TRY(launch_gemm_tc_split(w.w_router, c.n_experts, ws.at<void>(B_Y), T, T128, d, rp,
-                                  ws.at<float>(B_Z), "router_logits_tc", nullptr, s, nullptr));
+                                  ws.at<float>(B_Z), "router_logits_tc", nullptr, s, nullptr,
+                                  true));
     else
       DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_Y), T, w.w_router, c.n_experts, d,
                                   ws.at<float>(B_Z), nullptr, c.n_experts, "router_logits_tc",

@@ -203,11 +203,13 @@ int launch_lmhead_tc(const void *F, int max_rows, const int32_t *n_rows_dev, con
 // ---- tensor-core GEMMs (k_gemm_tc.cu) -----------------------------------------------------------
 bool gemm_tc_supported(int act, int w, int K);
 // Swap-AB split-K projection for at most 256 tokens: part[s][t][n] (fp32) over K slices s.
+// w_static: W is a model weight that no kernel of the stream writes (not a dequantised scratch
+// copy), so the kernel may fetch it before waiting on the preceding kernel.
 bool split_supported(int act, int w, int T, int N, int K);
 int split_k_slices(int N, int K, int max_slices = 16);
 int launch_gemm_tc_split(const void *W, int N, const void *X, int T, int T_alloc, int K,
                          int k_split, float *part, const char *name, int32_t *st, cudaStream_t s,
-                         const float *scale);
+                         const float *scale, bool w_static);
 // out[M][N] = A[M][K] W[N][K]^T (+ res[M][N]) in fp32; A has room for roundup(M, 128) rows.
 // scale (or null): per output channel (W row), multiplies the fp32 accumulator.
 int launch_gemm_tc_dense(const void *A, int M, const void *W, int N, int K, float *out,

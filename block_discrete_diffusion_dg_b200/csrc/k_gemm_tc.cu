@@ -54,6 +54,8 @@ struct Params {
   const float *scale;  // per output channel (dense: [N]; experts: [E][w_rows]) or null
   int smem_epi;        // split with one unit per CTA: stage the tile in the (then idle) pipeline
                        // buffers and write it with one TMA store through tmC
+  int a_static;        // split: A is a weight no kernel of the stream writes, so its first stages
+                       // are fetched before the wait on the preceding kernel
   int32_t *status;
 };
 
@@ -133,7 +135,11 @@ template <int BN_MAX, int STAGES, int B_BOX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, Params p) {
-  pdl_wait();
+  // Programmatic dependent launch: with a static A the weight stream starts before the wait on the
+  // preceding kernel (whose output only B and the stores depend on); every role that reads that
+  // output or writes this kernel's output waits first.
+  const bool early = p.kind == K_SPLIT && p.a_static;
+  if (!early) pdl_wait();
   pdl_trigger();
   using C = Cfg<BN_MAX, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -187,6 +193,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t armed_ph[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) { armed[s] = 0; armed_ph[s] = 0; }
+      // early: the A boxes of the first unit's first k-blocks go out before the dependency wait
+      // (the ring is empty, so stages 0 .. pre-1 in phase 0 are free); the loop below then adds
+      // only their B boxes, which the same full barrier counts
+      int pre = 0;
+      if (early) {
+        const Unit x = decode<BN_MAX>(p, blockIdx.x);
+        const int nb = (x.n_mma + B_BOX - 1) / B_BOX;
+        const int kpb = kblocks / p.k_split, kb0 = x.col0 * kpb;
+        pre = kpb < STAGES ? kpb : STAGES;
+        for (int j = 0; j < pre; ++j) {
+          mbar_expect_tx(&full[j], C::A_BYTES + (uint32_t)nb * B_BOX * BK * 2);
+          tma_load_2d(sA + j * C::A_BYTES, &tmA, &full[j], (kb0 + j) * BK, x.a_row0);
+          armed[j] = 1;
+        }
+        pdl_wait();
+      }
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
         const Unit x = decode<BN_MAX>(p, u);
         const int nb = (x.n_mma + B_BOX - 1) / B_BOX;
@@ -195,11 +217,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int kb0 = p.kind == K_SPLIT ? x.col0 * kpb : 0;
         for (int kb = kb0; kb < kb0 + kpb; ++kb) {
           if (!mbar_wait(&empty[stage], ph ^ 1)) { fail(p.status, abort_flag); break; }
-          mbar_expect_tx(&full[stage], bytes);
           uint8_t *a = sA + stage * C::A_BYTES;
-          if (x.a_row1 < 0) {
+          if (u == (int)blockIdx.x && kb - kb0 < pre) {
+            // A already in flight, bytes already expected
+          } else if (x.a_row1 < 0) {
+            mbar_expect_tx(&full[stage], bytes);
             tma_load_2d(a, &tmA, &full[stage], kb * BK, x.a_row0);
           } else {
+            mbar_expect_tx(&full[stage], bytes);
             tma_load_2d(a, &tmA, &full[stage], kb * BK, x.a_row0);
             tma_load_2d(a + 64 * BK * 2, &tmA, &full[stage], kb * BK, x.a_row1);
           }
@@ -255,6 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (*abort_flag && last_stage >= 0) (void)mbar_wait(&empty[last_stage], last_ph);
     }
   } else {
+    if (early) pdl_wait();  // before the first read of the tiles or store of this kernel's output
     const int q = warp & 3;
     int acc = 0;
     uint32_t aph = 0;
@@ -472,7 +498,7 @@ bool split_supported(int act, int w, int T, int N, int K) {
 
 int launch_gemm_tc_split(const void *W, int N, const void *X, int T, int T_alloc, int K,
                          int k_split, float *part, const char *name, int32_t *st, cudaStream_t s,
-                         const float *scale) {
+                         const float *scale, bool w_static) {
   if (T <= 0 || T > 256 || N % BM || K % (BK * k_split)) return DG_ERR_UNSUPPORTED;
   const int bn = T <= 128 ? 128 : 256;
   CUtensorMap ta, tb;
@@ -492,6 +518,7 @@ int launch_gemm_tc_split(const void *W, int N, const void *X, int T, int T_alloc
   p.ldo = N;
   p.scale = scale;
   p.status = st;
+  p.a_static = w_static ? 1 : 0;
   const int units = p.m_tiles * k_split;
   // one unit per CTA: the epilogue stages the tile in shared memory and stores it with TMA
   CUtensorMap tc_out;
