@@ -621,11 +621,15 @@ def run_dg(args, world, rank, local, workload=None, full=True):
     roof = None
     if dom == "attn_tc":  # long contexts: the attention is a tensor-bound contraction
         ach = sf["attention"] / cfg.n_layers / dur / 1e12
+        tr = ncu_traffic(dom, cfg.name)
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 1),
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "traffic": None,
+                "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
+                "traffic": tr["bytes"] if tr else None,
                 "algorithmic_flops_per_launch": sf["attention"] / cfg.n_layers,
-                "peak_source": f"{peak_src} (cuBLAS bf16, sustained, of measured)"}
+                "peak_source": f"{peak_src} (cuBLAS bf16, sustained, of measured)",
+                "traffic_source": tr["source"] if tr else
+                "none: no ncu capture of this kernel source on this workload"}
     elif dom in ("lm_head_tc", "lm_head_q4") and \
             sf["lm_head"] / (peaks["bf16_tflops_sustained"] * 1e12) > \
             lm_bytes / (peaks["hbm_gbs"] * 1e9):
