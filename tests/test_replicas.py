@@ -99,3 +99,24 @@ def test_step_byte_accounting_by_weight_format():
     assert a["total"] - b["total"] == (V * d * 2 - V * d * 9 / 16) + lay.canvas * d * (2 - 9 / 16)
     f = bench.step_flops(lay, 256.0)
     assert f["lm_head"] == 2 * 256 * d * V
+
+
+def test_traffic_records_match_their_kernel_sources():
+    """Every DRAM-traffic record under profiles/ names the kernel source it was captured from;
+    the benchmark reports it only while that source is unchanged, and drops it otherwise."""
+    import hashlib
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+    assert rec
+    for kernel, by_wl in rec.items():
+        for wl, r in by_wl.items():
+            assert r["bytes_per_launch"] >= r["algorithmic_bytes_per_launch"] > 0
+            assert "--clock-control none" in r["command"]
+            src = os.path.join(ROOT, "block_discrete_diffusion_dg_b200", "csrc", r["source_file"])
+            sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+            got = bench.ncu_traffic(kernel, wl)
+            if sha == r["source_sha16"]:
+                assert got and got["bytes"] == r["bytes_per_launch"]
+            else:
+                assert got is None
+    assert bench.ncu_traffic("no_such_kernel", "layer") is None
