@@ -162,8 +162,10 @@ def test_router_parity_and_permutation(cfg, gen, S):
     assert (inv[want] == np.arange(len(valid))).all() and (inv[flat < 0] == -1).all()
 
 
-def _routing(T, E, k, gen, live_frac=1.0):
-    idx = np.stack([torch.randperm(E, generator=gen).numpy()[:k] for _ in range(T)]).astype(np.int32)
+def _routing(T, E, k, gen, live_frac=1.0, pool=None):
+    # pool: route every token among the first `pool` experts only (few, heavily loaded experts)
+    P = E if pool is None else pool
+    idx = np.stack([torch.randperm(P, generator=gen).numpy()[:k] for _ in range(T)]).astype(np.int32)
     w = torch.rand((T, k), generator=gen).double().numpy() + 0.05
     w = (w / w.sum(1, keepdims=True)).astype(np.float32)
     flat = idx.reshape(-1)
@@ -173,15 +175,21 @@ def _routing(T, E, k, gen, live_frac=1.0):
     return idx, w, off, perm, inv
 
 
-@pytest.mark.parametrize("wtype", ["bf16", "e4m3"])
-def test_moe_ffn_parity(cfg, gen, wtype):
-    c = synth.reduced("layer" if wtype == "bf16" else "batch32", batch=1)
-    T, d, E, k = 300, c.d_model, c.n_experts, c.top_k
+# "spread" routes 300 tokens over all experts of the reduced model.  At the full width (d 2048,
+# F 768: 32 and 12 k-blocks per weight tile) "skewed" sends 300 tokens to k + 1 of 16 experts
+# (two full 128-token tiles and a ragged one per expert, so units outnumber the CTAs) and "few"
+# has 3 tokens (one-token tiles: the smallest MMA width and mostly idle CTAs).
+@pytest.mark.parametrize("wtype,routing", [("bf16", "spread"), ("e4m3", "spread"),
+                                           ("bf16", "skewed"), ("bf16", "few")])
+def test_moe_ffn_parity(cfg, gen, wtype, routing):
+    wide = {} if routing == "spread" else dict(d_model=2048, d_ff=768)
+    c = synth.reduced("layer" if wtype == "bf16" else "batch32", batch=1, **wide)
+    T, d, E, k = (3 if routing == "few" else 300), c.d_model, c.n_experts, c.top_k
     model = synth.make_model(c, "cpu", seed=11)
     lay = {kk: (v.cuda() if v is not None else None) for kk, v in model["layers"][0].items()}
     y = _rms_rows(T, d, gen)
     res = torch.randn((T, d), generator=gen) * 0.05   # residual stream: fp32
-    idx, w, off, perm, inv = _routing(T, E, k, gen)
+    idx, w, off, perm, inv = _routing(T, E, k, gen, pool=(k + 1 if routing == "skewed" else None))
     dgc = B.make_config(c)
     out = torch.empty((T, d), dtype=torch.float32, device="cuda")
     d_ = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
@@ -197,12 +205,12 @@ def test_moe_ffn_parity(cfg, gen, wtype):
     # <= 2^-7 |a|, so |g - o| <= 2^-7 sum_j w_j sum_f |a_jf| |W_d[c, f]| (+ fp32 accumulation).
     yv = dec(y)
     bound = np.zeros_like(o)
-    for t in range(T):
-        for j in range(k):
-            wgu, wd = om.expert(0, int(idx[t, j]))
-            u = yv[t] @ wgu.T
-            a = O.round_bf16(O.gelu_tanh(u[:c.d_ff]) * u[c.d_ff:])
-            bound[t] += w[t, j] * (np.abs(a) @ np.abs(wd).T)
+    for e in np.unique(idx):  # the tokens of one expert at a time (same sum, grouped)
+        ts, js = np.nonzero(idx == e)
+        wgu, wd = om.expert(0, int(e))
+        u = yv[ts] @ wgu.T
+        a = O.round_bf16(O.gelu_tanh(u[:, :c.d_ff]) * u[:, c.d_ff:])
+        np.add.at(bound, ts, w[ts, js, None] * (np.abs(a) @ np.abs(wd).T))
     err = np.abs(g - o)
     assert (err <= 2.0 ** -7 * bound + 1e-5).all(), float((err / (bound + 1e-9)).max())
     assert np.median(err) < 1e-5
