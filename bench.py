@@ -149,38 +149,34 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ oracle sample
 
-def oracle_sample_step(cfg, om, state_np, kc, vc, cache_len, frac_den: int = 16):
-    """One bounded sample of the oracle's step; returns the extrapolated step time in seconds.
+def oracle_step_time(cfg, om, state_np, kc, vc, cache_len) -> float:
+    """Host seconds of one step of the oracle as it stands (``canvas_step``, fp64 numpy).
 
-    Runs the oracle's attention part (pre-norm, QKV, RoPE, attention, output projection, norm,
-    router) over the whole canvas, the expert FFN of the experts e < E/frac_den only, and the LM
-    head + entropy over a vocabulary slice of V/frac_den rows for every masked position.  The
-    expert and LM-head times are scaled by frac_den (each expert and each vocabulary row costs
-    the same), the rest is counted once.
+    With one canvas (every headline workload) this is the whole step, timed as it runs.  With a
+    batch of canvases only the first runs (the others are marked done, so the oracle skips them)
+    and the time is multiplied by the batch: the canvases are independent and cost the same.
     """
     from oracle import dg_oracle as O
+    st = {k: np.array(v, copy=True) for k, v in state_np.items()}
+    st["done"][1:] = 1
     t0 = time.perf_counter()
-    C = cfg.canvas
-    ids = np.where(state_np["masked"][0] != 0, cfg.mask_id, state_np["tokens"][0])
-    x = om.emb_rows(ids)
-    pos = int(cache_len[0]) + np.arange(C)
-    q, k, v = O.layer_qkv(cfg, om, 0, x, pos)
-    o = O.storage_round(O.attention(q, kc[0, 0, :, :cache_len[0]], vc[0, 0, :, :cache_len[0]], k, v,
-                                    False), cfg.act).reshape(C, -1)
-    h = O.storage_round(x + o @ om.w(0, "w_o").T, cfg.act)
-    y = O.storage_round(O.rmsnorm(h, cfg.rms_eps), cfg.act)
-    idx, gates, _ = O.router_topk(y, om.w(0, "w_router"), cfg.top_k)
-    t1 = time.perf_counter()
-    keep = idx < max(1, cfg.n_experts // frac_den)
-    O.moe_ffn(y, np.where(keep, idx, -1), gates, lambda e: om.expert(0, e), h, cfg.act)
-    t2 = time.perf_counter()
-    rows = np.nonzero(state_np["masked"][0])[0]
-    f = O.storage_round(O.rmsnorm(h[rows], cfg.rms_eps), cfg.act)
-    vs = cfg.vocab // frac_den
-    _, w = next(om.lm_head_chunks(vs))      # vocabulary rows [0, vs), decoded
-    O.entropy_argmax(f @ w.T)
-    t3 = time.perf_counter()
-    return (t1 - t0) + frac_den * ((t2 - t1) + (t3 - t2))
+    O.canvas_step(cfg, om, st, kc, vc, cache_len, cfg.gamma, cfg.max_steps)
+    return (time.perf_counter() - t0) * cfg.batch
+
+
+def oracle_sample_desc(cfg, steps: int) -> str:
+    one = (f"{steps} whole oracle canvas step(s), the all-MASK and half-committed canvas states "
+           f"alternating, timed as they ran")
+    if cfg.batch > 1:
+        one += f"; one canvas of the {cfg.batch} runs and its time is multiplied by {cfg.batch}"
+    return one
+
+
+def headline_config(cfg, world: int) -> dict:
+    """The ``config`` object of a canvas-step line; both arms print the same one."""
+    return {"workload": workload_desc(cfg), "batch": cfg.batch, "canvas": cfg.canvas,
+            "prompt_kv": cfg.prompt_len, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (>2 GB of weights per step); no flush"}
 
 
 def cpu_threads() -> int:
@@ -264,19 +260,17 @@ def run_reference(args, world, rank):
     states = [{k: synth.to_numpy(v) for k, v in synth.make_canvas_state(cfg, s).items()}
               for s in ("all_mask", "half")]
     for i in range(args.warmup):
-        oracle_sample_step(cfg, om, states[i % 2], kc, vc, cl, args.ref_frac)
-    times = [oracle_sample_step(cfg, om, states[i % 2], kc, vc, cl, args.ref_frac)
-             for i in range(args.steps)]
+        oracle_step_time(cfg, om, states[i % 2], kc, vc, cl)
+    times = [oracle_step_time(cfg, om, states[i % 2], kc, vc, cl) for i in range(args.steps)]
     t = float(np.sum(times))
     v = args.steps / t
-    sample = (f"per step: attention part over the whole canvas, experts e < E/{args.ref_frac} and "
-              f"an LM-head vocab slice of V/{args.ref_frac}, both scaled by {args.ref_frac}")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": workload_desc(cfg), "batch": cfg.batch},
+            "data": "synthetic (seeded random-init weights, N(0,1) prompt K/V)",
+            "config": headline_config(cfg, world),
             "cpu_baseline": {"kind": "oracle", "value": v, "unit": "steps/s", "cores": cpu_threads(),
-                             "sample": sample},
+                             "sample": oracle_sample_desc(cfg, args.steps)},
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -702,23 +696,17 @@ def run_dg(args, world, rank, local, workload=None, full=True):
         kc = O.decode_act(synth.to_numpy(kv["k"]), cfg.act)
         vc = O.decode_act(synth.to_numpy(kv["v"]), cfg.act)
         cl = synth.to_numpy(kv["cache_len"])
-        ts = [oracle_sample_step(cfg, om, {k: synth.to_numpy(v) for k, v in init[i].items()},
-                                 kc, vc, cl, args.ref_frac) for i in range(ns)]
-        tstep = float(np.mean(ts)) * cfg.batch      # the sample runs one canvas
-        cpu = {"value": 1.0 / tstep, "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"one all-MASK and one half-committed step; attention part over the whole "
-                         f"canvas, experts e < E/{args.ref_frac} and an LM-head vocab slice of "
-                         f"V/{args.ref_frac}, both scaled by {args.ref_frac}"}
+        ts = [oracle_step_time(cfg, om, {k: synth.to_numpy(v) for k, v in init[i].items()},
+                               kc, vc, cl) for i in range(ns)]
+        cpu = {"value": ns / float(np.sum(ts)), "unit": "steps/s", "cores": cpu_threads(),
+               "kind": "oracle", "sample": oracle_sample_desc(cfg, ns)}
 
     tok_s = steps_s * float(np.mean(committed))     # tokens committed over all canvases
     line = {"metric": METRIC, "value": round(steps_s, 3), "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random-init weights, N(0,1) prompt K/V)",
-            "config": {"workload": workload_desc(cfg), "batch": cfg.batch, "canvas": cfg.canvas,
-                       "prompt_kv": cfg.prompt_len, "parallelism": f"replicas x{world}",
-                       "cuda_graph": bool(graphs),
-                       "l2": "inputs larger than L2 (>2 GB of weights per step); no flush"},
+            "config": headline_config(cfg, world), "cuda_graph": bool(graphs),
             "output_tok_s": round(tok_s, 2), "tokens_committed_per_step": committed,
             "step_roofline": step_roof, "roofline": roof, "kernels": breakdown,
             "gpu_launches": int(launches), "launches_per_step": int(per_step_launches),
@@ -753,7 +741,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--workload", default="layer")
-    ap.add_argument("--ref-frac", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct launches")
     ap.add_argument("--no-extra", action="store_true",

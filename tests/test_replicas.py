@@ -9,6 +9,7 @@ import json
 import os
 import socket
 import subprocess
+import time
 import sys
 
 import pytest
@@ -73,8 +74,10 @@ def test_reference_arm_under_torchrun_two_ranks(tmp_path):
            os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
            "--gpus", "2", "--steps", "2", "--warmup", "3"]
     env = dict(os.environ, OMP_NUM_THREADS="1")
+    t0 = time.perf_counter()
     r = subprocess.run(cmd, cwd=str(tmp_path), env=env, capture_output=True, text=True,
                        timeout=300)
+    wall = time.perf_counter() - t0
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1                   # rank 0 only
@@ -82,6 +85,13 @@ def test_reference_arm_under_torchrun_two_ranks(tmp_path):
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 2
     assert d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    # whole oracle steps, timed as they ran: the timed steps fit inside the run's wall clock, and
+    # the line carries the same config object as the CUDA arm's
+    import bench
+    import synth
+    assert d["ms_per_step"] * d["steps"] / 1e3 < wall
+    assert "whole oracle canvas step" in d["cpu_baseline"]["sample"]
+    assert d["config"] == bench.headline_config(synth.get_config("tiny"), 2)
 
 
 def test_step_byte_accounting_by_weight_format():
