@@ -159,6 +159,7 @@ Layout make_layout(const dg_config &c, int batch, int n, int cap) {
 struct Ws {
   char *base;
   const Layout *L;
+  int32_t *st;  // the caller's device status word (may be null): bounded-wait timeouts land here
   template <typename P> P *at(Buf b) const { return reinterpret_cast<P *>(base + L->off[b]); }
 };
 
@@ -252,10 +253,10 @@ int qkv_proj(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int T,
     const int parts = qkv_parts(c, T);
     if (parts > 1)
       return launch_gemm_tc_split(wq, g.N, ws.at<void>(B_A), T, (T + 127) / 128 * 128, c.d_model,
-                                  parts, ws.at<float>(B_QKV), "gemm_qkv_tc", nullptr, s, g.bscale,
+                                  parts, ws.at<float>(B_QKV), "gemm_qkv_tc", ws.st, s, g.bscale,
                                   wq == w.w_qkv);
     return launch_gemm_tc_dense(ws.at<void>(B_A), T, wq, g.N, c.d_model, ws.at<float>(B_QKV),
-                                nullptr, g.N, "gemm_qkv_tc", nullptr, s, g.bscale);
+                                nullptr, g.N, "gemm_qkv_tc", ws.st, s, g.bscale);
   }
   return launch_gemm_simt(g, EPI_F32, ws.at<void>(B_QKV), g.N, nullptr, s);
 }
@@ -288,7 +289,7 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
     const void *wo = tc_weight(c, ws, w.w_o, (size_t)d * hq, 0, s, &rc);
     if (rc != DG_OK) return rc;
     DG_TRY(launch_gemm_tc_split(wo, d, ws.at<void>(B_O), T, T128, hq, op, ws.at<float>(B_HP),
-                                "gemm_o_resid_tc", nullptr, s, g.bscale, wo == w.w_o));
+                                "gemm_o_resid_tc", ws.st, s, g.bscale, wo == w.w_o));
     DG_TRY(launch_resid_norm(c.act_dtype, ws.at<float>(B_HP), op, ws.at<float>(B_X), T, d,
                              c.rms_eps, ws.at<float>(B_H), ws.at<void>(B_Y), s));
   } else {
@@ -297,7 +298,7 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
       const void *wo = tc_weight(c, ws, w.w_o, (size_t)d * hq, 0, s, &rc);
       if (rc != DG_OK) return rc;
       DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_O), T, wo, d, hq, ws.at<float>(B_H),
-                                  ws.at<float>(B_X), d, "gemm_o_resid_tc", nullptr, s, g.bscale));
+                                  ws.at<float>(B_X), d, "gemm_o_resid_tc", ws.st, s, g.bscale));
     } else
       DG_TRY(launch_gemm_simt(g, EPI_RESID, ws.at<void>(B_H), d, ws.at<void>(B_X), s));
     DG_TRY(launch_rmsnorm(c.act_dtype, ws.at<void>(B_H), nullptr, nullptr, T, d, c.rms_eps,
@@ -308,12 +309,12 @@ int attn_out_and_route(const dg_config &c, const dg_layer_weights &w, const Ws &
     const int rp = router_parts(c, T);
     if (rp > 1)
       DG_TRY(launch_gemm_tc_split(w.w_router, c.n_experts, ws.at<void>(B_Y), T, T128, d, rp,
-                                  ws.at<float>(B_Z), "router_logits_tc", nullptr, s, nullptr,
+                                  ws.at<float>(B_Z), "router_logits_tc", ws.st, s, nullptr,
                                   true));
     else
       DG_TRY(launch_gemm_tc_dense(ws.at<void>(B_Y), T, w.w_router, c.n_experts, d,
                                   ws.at<float>(B_Z), nullptr, c.n_experts, "router_logits_tc",
-                                  nullptr, s));
+                                  ws.st, s));
     const bool tc = experts_tc(c);
     DG_TRY(launch_route(T, c.n_experts, c.top_k, ws.at<float>(B_Z), token_live,
                         ws.at<int32_t>(B_IDX), ws.at<float>(B_W), ws.at<int32_t>(B_OFF),
@@ -360,11 +361,11 @@ int moe_experts(const dg_config &c, const dg_layer_weights &w, const Ws &ws, int
     DG_TRY(launch_gemm_tc_experts(1, wgu, E, 2 * F, F, ws.at<void>(B_XP), TK, d,
                                   ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
                                   ws.L->max_tiles, expert_off, ws.at<void>(B_ACT), F,
-                                  "moe_gate_up_tc", nullptr, s, e4 ? w.s_gate_up : nullptr));
+                                  "moe_gate_up_tc", ws.st, s, e4 ? w.s_gate_up : nullptr));
     DG_TRY(launch_gemm_tc_experts(0, wdn, E, d, F, ws.at<void>(B_ACT), TK, F,
                                   ws.at<GroupTile>(B_TILES), ws.at<int32_t>(B_NTILES),
                                   ws.L->max_tiles, expert_off, ws.at<void>(B_YE), d,
-                                  "moe_down_tc", nullptr, s, e4 ? w.s_down : nullptr));
+                                  "moe_down_tc", ws.st, s, e4 ? w.s_down : nullptr));
   } else {
     GemmDesc g1{};
     g1.act = c.act_dtype; g1.w = c.w_dtype;
@@ -617,14 +618,13 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
                  const uint8_t *token_live, int32_t *topk_idx, float *topk_w,
                  int32_t *expert_off, int32_t *perm, int32_t *inv_perm, void *ws,
                  size_t ws_bytes, int32_t *dev_status, void *stream) {
-  (void)dev_status;
   if (!cfg_ok(cfg) || n_tokens <= 0) return DG_ERR_INVALID_ARG;
   if (!y || !w_router || !topk_idx || !topk_w || !expert_off || !perm || !inv_perm)
     return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, 1, n_tokens, 0, ws, ws_bytes, &L));
   const cudaStream_t s = (cudaStream_t)stream;
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   const int d = cfg->d_model, E = cfg->n_experts;
   if (gemm_tc_supported(cfg->act_dtype, router_type(cfg), d) && E % 16 == 0) {
     // the tensor-core router reads whole 128-row tiles: stage y into the padded scratch rows
@@ -632,7 +632,7 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
                                           cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return check_launch("dg_moe_route copy");
     DG_TRY(launch_gemm_tc_dense(w.at<void>(B_Y), n_tokens, w_router, E, d, w.at<float>(B_Z), nullptr,
-                                E, "router_logits_tc", nullptr, s));
+                                E, "router_logits_tc", w.st, s));
     DG_TRY(launch_router_topk(n_tokens, E, cfg->top_k, w.at<float>(B_Z), token_live, topk_idx,
                               topk_w, s, nullptr, 1, cfg->n_shared));
   } else {
@@ -647,14 +647,13 @@ int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t 
                const float *topk_w, const int32_t *expert_off, const int32_t *perm,
                const int32_t *inv_perm, const dg_layer_weights *lw, const void *residual,
                void *out, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
-  (void)dev_status;
   if (!cfg_ok(cfg) || n_tokens <= 0 || !lw_ok(cfg, lw)) return DG_ERR_INVALID_ARG;
   if (!y || !topk_idx || !topk_w || !expert_off || !perm || !inv_perm || !residual || !out)
     return DG_ERR_INVALID_ARG;
   if (out == y) return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, 1, n_tokens, 0, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   return moe_experts(*cfg, *lw, w, n_tokens, y, topk_idx, topk_w, expert_off, perm, inv_perm,
                      residual, out, (cudaStream_t)stream);
 }
@@ -668,7 +667,7 @@ int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_de
     return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, 1, n_rows, 0, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   return lm_entropy(*cfg, w, n_rows, n_rows_dev, h, row_idx, LmWeights{w_lm, nullptr, 1.0f},
                     entropy, argmax, logits_dbg, 0, dev_status, (cudaStream_t)stream);
 }
@@ -684,7 +683,7 @@ int dg_logits_entropy_nvfp4(const dg_config *cfg, int n_rows, const int32_t *n_r
   if (!lm_weights_ok(*cfg, lw)) return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, 1, n_rows, 0, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   return lm_entropy(*cfg, w, n_rows, n_rows_dev, h, row_idx, lw, entropy, argmax, logits_dbg, 0,
                     dev_status, (cudaStream_t)stream);
 }
@@ -716,7 +715,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
   if (!lm_weights_ok(*cfg, emb)) return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   const dg_config &c = *cfg;
   const cudaStream_t s = (cudaStream_t)stream;
   const int T = batch * n_tokens, d = c.d_model;
@@ -769,7 +768,7 @@ int dg_ar_step(const dg_config *cfg, const dg_model *model, int batch, const int
   if (!lm_weights_ok(*cfg, emb)) return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, batch, n_tokens, cache_cap, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   const dg_config &c = *cfg;
   const cudaStream_t s = (cudaStream_t)stream;
   const int T = batch * n_tokens, d = c.d_model;
@@ -848,7 +847,7 @@ int canvas_step_impl(const dg_config *cfg, const dg_model *model, int batch, int
   const int C = c.canvas, T = batch * C, d = c.d_model;
   Layout L;
   DG_TRY(check_ws(cfg, batch, C, cache_cap, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   const cudaStream_t s = (cudaStream_t)stream;
   const size_t layer_elems = (size_t)batch * c.n_kv_heads * cache_cap * c.head_dim;
   const size_t ae = esz(c.act_dtype);
@@ -954,7 +953,7 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
   if (!lm_weights_ok(*cfg, lm_weights(*cfg, model))) return DG_ERR_INVALID_ARG;
   Layout L;
   DG_TRY(check_ws(cfg, batch, cfg->canvas, cache_cap, ws, ws_bytes, &L));
-  Ws w{(char *)ws, &L};
+  Ws w{(char *)ws, &L, dev_status};
   int32_t *iter = w.at<int32_t>(B_GEN);
   const cudaStream_t s = (cudaStream_t)stream;
 
