@@ -981,12 +981,16 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
   key_add(key, cache_cap);
   key_add(key, ws_bytes);
 
+  // A cached graph is launched under the cache lock, so another thread cannot evict (destroy) it
+  // between the lookup and the launch; a destroyed graph that is already launched finishes.
   cudaGraphExec_t exec = nullptr;
+  cudaError_t launched = cudaErrorUnknown;
   {
     GenCache &gc = gen_cache();
     std::lock_guard<std::mutex> lock(gc.mu);
     for (auto &e : gc.entries)
       if (e.first == key) exec = e.second;
+    if (exec) launched = cudaGraphLaunch(exec, s);
   }
   if (!exec) {
     // parent graph: reset the loop counter, then a while node whose body is one captured step
@@ -1058,9 +1062,9 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
       gc.entries.erase(gc.entries.begin());
     }
     gc.entries.emplace_back(key, exec);
+    launched = cudaGraphLaunch(exec, s);
   }
-  const cudaError_t e = cudaGraphLaunch(exec, s);
-  if (e != cudaSuccess) return cuda_fail("dg_generate launch", e);
+  if (launched != cudaSuccess) return cuda_fail("dg_generate launch", launched);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (!append) return DG_OK;
   return dg_kv_append(cfg, model, batch, tokens, cfg->canvas, k_cache, v_cache, cache_len,
