@@ -9,10 +9,33 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
 namespace dg {
+
+// NVTX range over one entry point's host work (its checks and launches); a profiler projects it
+// onto the kernels it launched, so a timeline groups them under the call (and the layer) that
+// issued them.  Without an attached tool the calls return at once.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  // a range named `name` carrying an integer payload (the layer index)
+  NvtxRange(const char *name, int payload) {
+    nvtxEventAttributes_t a{};
+    a.version = NVTX_VERSION;
+    a.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    a.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    a.message.ascii = name;
+    a.payloadType = NVTX_PAYLOAD_TYPE_INT32;
+    a.payload.iValue = payload;
+    nvtxRangePushEx(&a);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 static std::atomic<unsigned long long> g_launches{0};
 static thread_local char g_err[256] = "no error";
@@ -603,6 +626,7 @@ int dg_canvas_attn(const dg_config *cfg, int batch, int n_tokens, const void *q,
                    int cache_cap, const void *k_new, const void *v_new, int causal,
                    const int32_t *done, void *out, void *ws, size_t ws_bytes,
                    int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_canvas_attn");
   if (!cfg_ok(cfg) || batch <= 0 || n_tokens <= 0 || cache_cap < 0) return DG_ERR_INVALID_ARG;
   if (!q || !cache_len || !k_new || !v_new || !out) return DG_ERR_INVALID_ARG;
   if (cache_cap > 0 && (!k_cache || !v_cache)) return DG_ERR_INVALID_ARG;
@@ -618,6 +642,7 @@ int dg_moe_route(const dg_config *cfg, int n_tokens, const void *y, const void *
                  const uint8_t *token_live, int32_t *topk_idx, float *topk_w,
                  int32_t *expert_off, int32_t *perm, int32_t *inv_perm, void *ws,
                  size_t ws_bytes, int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_moe_route");
   if (!cfg_ok(cfg) || n_tokens <= 0) return DG_ERR_INVALID_ARG;
   if (!y || !w_router || !topk_idx || !topk_w || !expert_off || !perm || !inv_perm)
     return DG_ERR_INVALID_ARG;
@@ -647,6 +672,7 @@ int dg_moe_ffn(const dg_config *cfg, int n_tokens, const void *y, const int32_t 
                const float *topk_w, const int32_t *expert_off, const int32_t *perm,
                const int32_t *inv_perm, const dg_layer_weights *lw, const void *residual,
                void *out, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_moe_ffn");
   if (!cfg_ok(cfg) || n_tokens <= 0 || !lw_ok(cfg, lw)) return DG_ERR_INVALID_ARG;
   if (!y || !topk_idx || !topk_w || !expert_off || !perm || !inv_perm || !residual || !out)
     return DG_ERR_INVALID_ARG;
@@ -662,6 +688,7 @@ int dg_logits_entropy(const dg_config *cfg, int n_rows, const int32_t *n_rows_de
                       const void *h, const int32_t *row_idx, const void *w_lm, float *entropy,
                       int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
                       int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_logits_entropy");
   if (!cfg_ok(cfg) || cfg->emb_dtype == DG_NVFP4 || n_rows <= 0 || !h || !w_lm || !entropy ||
       !argmax)
     return DG_ERR_INVALID_ARG;
@@ -677,6 +704,7 @@ int dg_logits_entropy_nvfp4(const dg_config *cfg, int n_rows, const int32_t *n_r
                             const uint8_t *w_scale, float w_scale_global, float *entropy,
                             int32_t *argmax, float *logits_dbg, void *ws, size_t ws_bytes,
                             int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_logits_entropy_nvfp4");
   if (!cfg_ok(cfg) || cfg->emb_dtype != DG_NVFP4 || n_rows <= 0 || !h || !entropy || !argmax)
     return DG_ERR_INVALID_ARG;
   const LmWeights lw{w_codes, w_scale, w_scale_global};
@@ -692,6 +720,7 @@ int dg_eb_select(int batch, int canvas, const float *entropy, const int32_t *arg
                  double gamma, int max_steps, int32_t *tokens, uint8_t *masked,
                  uint8_t *selected, int32_t *n_masked, int32_t *done, int32_t *step, int revise,
                  int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_eb_select");
   if (batch <= 0 || canvas <= 0 || canvas > 1024 || max_steps <= 0) return DG_ERR_INVALID_ARG;
   if (!(gamma >= 0.0)) return DG_ERR_INVALID_ARG;
   if (!entropy || !argmax || !tokens || !masked || !n_masked || !done || !step)
@@ -705,6 +734,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
                  int n_tokens, void *k_cache, void *v_cache, int32_t *cache_len, int cache_cap,
                  const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
                  void *stream) {
+  const NvtxRange nvtx_range("dg_kv_append");
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || n_tokens <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !k_cache || !v_cache || !cache_len || cache_cap <= 0) return DG_ERR_INVALID_ARG;
@@ -726,6 +756,7 @@ int dg_kv_append(const dg_config *cfg, const dg_model *model, int batch, const i
                          c.rope_theta, cache_len, w.at<float>(B_CS), nullptr, nullptr, nullptr,
                          nullptr, nullptr, s, emb.scale, emb.g));
   for (int l = 0; l < c.n_layers; ++l) {
+    const NvtxRange layer_range("layer", l);
     const dg_layer_weights &lw = model->layers[l];
     char *kc = (char *)k_cache + l * layer_elems * ae;
     char *vc = (char *)v_cache + l * layer_elems * ae;
@@ -756,6 +787,7 @@ int dg_ar_step(const dg_config *cfg, const dg_model *model, int batch, const int
                const dg_sampler *smp, int32_t *next_token, float *entropy, float *logits_dbg,
                const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
                void *stream) {
+  const NvtxRange nvtx_range("dg_ar_step");
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || n_tokens <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !k_cache || !v_cache || !cache_len || cache_cap <= 0 || !next_token)
@@ -781,6 +813,7 @@ int dg_ar_step(const dg_config *cfg, const dg_model *model, int batch, const int
                          nullptr, nullptr, s, emb.scale, emb.g));
   DG_TRY(launch_last_row_slots(batch, n_tokens, slot, s));
   for (int l = 0; l < c.n_layers; ++l) {
+    const NvtxRange layer_range("layer", l);
     const dg_layer_weights &lw = model->layers[l];
     char *kc = (char *)k_cache + l * layer_elems * ae;
     char *vc = (char *)v_cache + l * layer_elems * ae;
@@ -861,6 +894,7 @@ int canvas_step_impl(const dg_config *cfg, const dg_model *model, int batch, int
                          c.rope_theta, cache_len, w.at<float>(B_CS), done, rows, n_rows, slot, live,
                          s, emb.scale, emb.g, revise));
   for (int l = 0; l < c.n_layers; ++l) {
+    const NvtxRange layer_range("layer", l);
     const dg_layer_weights &lw = model->layers[l];
     const char *kc = (const char *)k_cache + l * layer_elems * ae;
     const char *vc = (const char *)v_cache + l * layer_elems * ae;
@@ -907,6 +941,7 @@ int dg_canvas_step(const dg_config *cfg, const dg_model *model, int batch, int32
                    int32_t *argmax_out, float *logits_dbg, int32_t *expert_load,
                    const int32_t *forced_topk, void *ws, size_t ws_bytes, int32_t *dev_status,
                    void *stream) {
+  const NvtxRange nvtx_range("dg_canvas_step");
   return canvas_step_impl(cfg, model, batch, tokens, masked, n_masked, done, step, max_steps,
                           gamma, k_cache, v_cache, cache_len, cache_cap, entropy_out, argmax_out,
                           logits_dbg, expert_load, forced_topk, nullptr, ws, ws_bytes, dev_status,
@@ -920,6 +955,7 @@ int dg_canvas_step_sampler(const dg_config *cfg, const dg_model *model, int batc
                            int cache_cap, float *entropy_out, int32_t *argmax_out,
                            float *logits_dbg, const int32_t *forced_topk, void *ws,
                            size_t ws_bytes, int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_canvas_step_sampler");
   if (!smp) return DG_ERR_INVALID_ARG;
   return canvas_step_impl(cfg, model, batch, tokens, masked, n_masked, done, step, max_steps,
                           gamma, k_cache, v_cache, cache_len, cache_cap, entropy_out, argmax_out,
@@ -930,6 +966,7 @@ int dg_canvas_step_sampler(const dg_config *cfg, const dg_model *model, int batc
 int dg_noise_canvas(int batch, int canvas, int vocab, uint64_t seed, int32_t *tokens,
                     uint8_t *masked, int32_t *n_masked, int32_t *done, int32_t *step,
                     void *stream) {
+  const NvtxRange nvtx_range("dg_noise_canvas");
   if (batch <= 0 || canvas <= 0 || canvas > 1024 || vocab < 1) return DG_ERR_INVALID_ARG;
   if (!tokens || !masked || !n_masked || !done || !step) return DG_ERR_INVALID_ARG;
   return launch_noise_canvas(batch, canvas, vocab, (uint32_t)(seed & 0xFFFFFFFFu),
@@ -942,6 +979,7 @@ int dg_generate(const dg_config *cfg, const dg_model *model, int batch, int32_t 
                 double gamma, const dg_sampler *smp, void *k_cache, void *v_cache,
                 int32_t *cache_len, int cache_cap, int append, void *ws, size_t ws_bytes,
                 int32_t *dev_status, void *stream) {
+  const NvtxRange nvtx_range("dg_generate");
   if (!cfg_ok(cfg) || !model || !model->layers || !model->emb || batch <= 0 || max_steps <= 0)
     return DG_ERR_INVALID_ARG;
   if (!tokens || !masked || !n_masked || !done || !step || !cache_len) return DG_ERR_INVALID_ARG;
