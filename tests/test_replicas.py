@@ -130,3 +130,20 @@ def test_traffic_records_match_their_kernel_sources():
             else:
                 assert got is None
     assert bench.ncu_traffic("no_such_kernel", "layer") is None
+
+
+def test_step_roofline_bound_and_fractions():
+    """The step roofline is max(bytes / HBM peak, FLOPs / tensor peak) against the measured step
+    time, reported as a fraction of the measured peaks and, beside it, of the nominal ones."""
+    import bench
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1500.0}
+    # 3 GB at 6 TB/s = 500 us; 300 GFLOP at 1.5 PF/s = 200 us: HBM-bound, 500 us of 1000 us
+    r = bench.step_roofline({"total": 3e9}, {"total": 3e11}, 1.0, peaks, "measured")
+    assert r["bound"] == "hbm" and r["roofline_us"] == pytest.approx(500.0)
+    assert r["frac"] == pytest.approx(0.5)
+    assert r["frac_nominal"] == pytest.approx(3e9 / (bench.NOMINAL["hbm_gbs"] * 1e9) / 1e-3,
+                                              rel=1e-3)
+    # 1.2 PFLOP-s of work: tensor-bound (800 us) over a 1 GB stream (167 us)
+    r = bench.step_roofline({"total": 1e9}, {"total": 1.2e12}, 1.0, peaks, "measured")
+    assert r["bound"] == "tensor" and r["roofline_us"] == pytest.approx(800.0)
+    assert r["frac"] == pytest.approx(0.8)
