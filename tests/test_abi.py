@@ -177,3 +177,29 @@ def test_binding_refuses_host_tensors():
     import torch
     with pytest.raises(ValueError):
         B._p(torch.zeros(4))
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    """include/dg.h compiles as strict C99 and a C program linked against libdg.so calls it: the
+    boundary needs no C++ or Python.  Without a GPU the calls only exercise the host-side checks."""
+    src = tmp_path / "use_dg.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "dg.h"
+int main(void) {
+  dg_config c = {0};                                       /* all zero: not a valid model */
+  const size_t ws = dg_workspace_size(&c, 1, 256, 0);
+  const int rc = dg_eb_select(0, 0, NULL, NULL, 0.0, 0, NULL, NULL, NULL, NULL, NULL, NULL, 0,
+                              NULL, NULL);
+  const int rs = dg_logits_entropy_static(NULL, 1, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL);
+  printf("%zu %d %d\n", ws, rc, rs);
+  return (ws == 0 && rc == DG_ERR_INVALID_ARG && rs == DG_ERR_INVALID_ARG) ? 0 : 1;
+}
+''')
+    exe = tmp_path / "use_dg"
+    pkg = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    B.LIB_PATH, "-Wl,-rpath," + pkg], check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.stdout, r.stderr)
