@@ -278,6 +278,25 @@ def m_sample_row_multiplies_by_tau(orig):
     return lambda z, tau, g: orig(z, 1.0 / tau if tau > 0.0 else tau, g)
 
 
+# ----------------------------------------------------------------- the step and the append
+
+def m_append_sees_later_tokens(orig):
+    return lambda cfg, model, l, x, q, k, v, kc, vc, causal, *a, **kw: orig(
+        cfg, model, l, x, q, k, v, kc, vc, False, *a, **kw)
+
+
+def m_append_positions_from_zero(orig):
+    def f(cfg, model, l, x, pos):
+        p = np.asarray(pos)
+        return orig(cfg, model, l, x, p - p[0])
+    return f
+
+
+def m_step_cap_one_late(orig):
+    return lambda cfg, model, state, kc, vc, cl, gamma, max_steps, *a, **kw: orig(
+        cfg, model, state, kc, vc, cl, gamma, max_steps + 1, *a, **kw)
+
+
 # ----------------------------------------------------------------- the cases
 
 _TINY = []
@@ -363,6 +382,12 @@ MUTANTS = [
     ("temperature over N, not N - 1", "temperature", m_temperature_over_n, SAMPLER),
     ("logits times tau", "sample_row", m_sample_row_multiplies_by_tau,
      SAMPLER + [(S.test_gumbel_max_draw_follows_softmax_at_temperature, ())]),
+    ("append attends to later tokens", "layer_rest", m_append_sees_later_tokens,
+     [(P.test_append_is_a_causal_encoder_two_layers, ())]),
+    ("positions ignore the cache length", "layer_qkv", m_append_positions_from_zero,
+     [(P.test_tiny_kv_append_single_layer_is_direct_projection, (_tiny_once,))]),
+    ("step cap one step late", "canvas_step", m_step_cap_one_late,
+     [(P.test_tiny_infinite_bound_and_step_cap, (_tiny_once,))]),
 ]
 
 

@@ -697,3 +697,32 @@ def test_moe_negative_expert_slot_contributes_nothing():
     only0 = O.moe_ffn(y, idx[:, :1], g[:, :1], lambda e: ws[e], res, "f32")
     np.testing.assert_allclose(part, only0, atol=1e-13)
     assert not np.allclose(part, full)
+
+
+def test_append_is_a_causal_encoder_two_layers():
+    """The append is a causal encoder ("DiffusionGemma Technical Report", Figure 4, stage 3):
+    appending the first n tokens of a sequence writes exactly the K/V rows that appending the
+    whole sequence writes for them, in every layer, because no row sees a later token; and a row
+    of the second layer does depend on the earlier tokens."""
+    cfg = synth.get_config("tiny", n_layers=2)
+    m = synth.make_model(cfg, "cpu")
+    om = O.OracleModel(cfg, {"emb": synth.to_numpy(m["emb"]),
+                             "layers": [{k: synth.to_numpy(v) for k, v in lay.items()}
+                                        for lay in m["layers"]]})
+    kv = synth.make_prompt_kv(cfg, "cpu")
+    kc0 = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc0 = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    toks = rng.integers(0, cfg.vocab, (1, 12)).astype(np.int32)
+    ka, va = kc0.copy(), vc0.copy()
+    O.kv_append(cfg, om, toks, ka, va, cl)
+    kb, vb = kc0.copy(), vc0.copy()
+    O.kv_append(cfg, om, toks[:, :5], kb, vb, cl)
+    r0, r1 = int(cl[0]), int(cl[0]) + 5
+    np.testing.assert_allclose(kb[..., r0:r1, :], ka[..., r0:r1, :], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(vb[..., r0:r1, :], va[..., r0:r1, :], rtol=0, atol=1e-12)
+    t2 = toks.copy()
+    t2[0, 0] = (t2[0, 0] + 1) % cfg.vocab
+    kc2, vc2 = kc0.copy(), vc0.copy()
+    O.kv_append(cfg, om, t2, kc2, vc2, cl)
+    assert np.abs(kc2[1, ..., r0 + 7, :] - ka[1, ..., r0 + 7, :]).max() > 1e-6
