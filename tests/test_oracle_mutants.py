@@ -297,6 +297,19 @@ def m_step_cap_one_late(orig):
         cfg, model, state, kc, vc, cl, gamma, max_steps + 1, *a, **kw)
 
 
+def m_commit_indexes_argmax_by_position(orig):
+    # the committed token read from the argmax list at the canvas position, not at the row index
+    def f(cfg, model, state, kc, vc, cl, gamma, max_steps, *a, **kw):
+        new, infos = orig(cfg, model, state, kc, vc, cl, gamma, max_steps, *a, **kw)
+        for b, info in enumerate(infos):
+            if info and "selected" in info:
+                pos = np.nonzero(info["selected"])[0]
+                am = info["argmax"]
+                new["tokens"][b, pos] = am[np.minimum(pos, len(am) - 1)]
+        return new, infos
+    return f
+
+
 # ----------------------------------------------------------------- the cases
 
 _TINY = []
@@ -388,6 +401,9 @@ MUTANTS = [
      [(P.test_tiny_kv_append_single_layer_is_direct_projection, (_tiny_once,))]),
     ("step cap one step late", "canvas_step", m_step_cap_one_late,
      [(P.test_tiny_infinite_bound_and_step_cap, (_tiny_once,))]),
+    ("commit reads the argmax at the position", "canvas_step",
+     m_commit_indexes_argmax_by_position,
+     [(P.test_tiny_commit_writes_each_rows_own_argmax, (_tiny_once,))]),
 ]
 
 

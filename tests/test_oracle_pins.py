@@ -726,3 +726,30 @@ def test_append_is_a_causal_encoder_two_layers():
     kc2, vc2 = kc0.copy(), vc0.copy()
     O.kv_append(cfg, om, t2, kc2, vc2, cl)
     assert np.abs(kc2[1, ..., r0 + 7, :] - ka[1, ..., r0 + 7, :]).max() > 1e-6
+
+
+def test_tiny_commit_writes_each_rows_own_argmax(tiny):
+    """On a canvas whose open rows are not its first positions, every position the step commits
+    receives the argmax of its own row's logits (computed here from the returned logits), and the
+    final positions keep their tokens.  The open positions carry distinct draft tokens (the
+    revisable-draft canvas, greedy), so their rows, and their argmaxes, differ."""
+    cfg, model, kv = tiny
+    kc = synth.to_numpy(kv["k"]).astype(np.float64)
+    vc = synth.to_numpy(kv["v"]).astype(np.float64)
+    cl = synth.to_numpy(kv["cache_len"])
+    st = _state(cfg)
+    g = np.random.default_rng(5)
+    st["tokens"][0] = g.integers(0, cfg.vocab, cfg.canvas)
+    done_pos = g.permutation(cfg.canvas)[: cfg.canvas // 2]
+    st["masked"][0, done_pos] = 0
+    st["n_masked"][0] = int(st["masked"][0].sum())
+    greedy_drafts = {"tau_start": 0.0, "tau_end": 0.0, "seed": 0, "revise": True}
+    st2, info = O.canvas_step(cfg, model, st, kc, vc, cl, 1e9, cfg.max_steps, keep_logits=True,
+                              sampler=greedy_drafts)
+    rows = info[0]["rows"]
+    assert (rows == np.nonzero(st["masked"][0])[0]).all()
+    own = np.argmax(info[0]["logits"], axis=1)
+    assert len(set(own.tolist())) > 1                       # the check below can tell rows apart
+    assert st2["masked"][0].sum() == 0                       # an unbounded gamma commits them all
+    np.testing.assert_array_equal(st2["tokens"][0, rows], own)
+    np.testing.assert_array_equal(st2["tokens"][0, done_pos], st["tokens"][0, done_pos])
