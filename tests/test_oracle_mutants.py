@@ -274,6 +274,14 @@ def m_temperature_over_n(orig):
     return f
 
 
+def m_gumbel_subtracted(orig):
+    return lambda z, tau, g: orig(z, tau, None if g is None else -np.asarray(g))
+
+
+def m_gumbel_sign(orig):
+    return lambda words: np.log(-np.log(O.uniform_open(words)))
+
+
 def m_sample_row_multiplies_by_tau(orig):
     return lambda z, tau, g: orig(z, 1.0 / tau if tau > 0.0 else tau, g)
 
@@ -395,6 +403,9 @@ MUTANTS = [
     ("temperature over N, not N - 1", "temperature", m_temperature_over_n, SAMPLER),
     ("logits times tau", "sample_row", m_sample_row_multiplies_by_tau,
      SAMPLER + [(S.test_gumbel_max_draw_follows_softmax_at_temperature, ())]),
+    ("Gumbel noise subtracted", "sample_row", m_gumbel_subtracted,
+     [(S.test_gumbel_max_draw_follows_softmax_at_temperature, ())]),
+    ("Gumbel transform sign flipped", "gumbel", m_gumbel_sign, SAMPLER),
     ("append attends to later tokens", "layer_rest", m_append_sees_later_tokens,
      [(P.test_append_is_a_causal_encoder_two_layers, ())]),
     ("positions ignore the cache length", "layer_qkv", m_append_positions_from_zero,
